@@ -1,0 +1,351 @@
+"""Plain, slow CPU oracle of one GPT-2 training step, in float64.
+
+TEST INFRASTRUCTURE ONLY. Only the test suite, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import this module. It shares no code
+with the CUDA path (the only common module is the seeded input generator,
+which holds none of the model's arithmetic).
+
+Every function writes out the plain definition the pages give, with a numpy
+matmul / exp / sum as the only library steps: attention materialises the whole
+T x T score matrix, the loss takes an explicit log-softmax over every
+vocabulary column, and the backward pass is derived by hand from the forward.
+
+Sources (page title, section):
+  * "GPT-2 from Scratch": "The config", "Embeddings: tokens and positions",
+    "CausalSelfAttention" (fused qkv, heads, causal mask, scaled dot-product,
+    output projection), "The MLP and GPT-2's GELU", "The Block: pre-LN and
+    residuals", "Forward: logits, and loss when targets are given",
+    "Weight tying", "AdamW, and weight decay on matrices only",
+    "Gradient clipping", "How to scale up" (gradient accumulation).
+  * "Let's reproduce GPT-2 (124M)" synopsis: "Matching GPT-3's optimization
+    hyperparameters" (betas, eps, clip 1.0, decay on 2-D tensors only) and
+    "Gradient accumulation, and the bug in getting it right".
+  * "Pretraining and fine-tuning nanoGPT-124M from scratch", "Supervised
+    fine-tuning" (targets of -1 are skipped by the loss).
+
+Readings where the pages are silent or the extraction lost the formula:
+  * GELU: the formula image is missing from "The MLP and GPT-2's GELU"; the
+    page names the tanh approximation of Hendrycks & Gimpel and PyTorch's
+    nn.GELU(approximate="tanh"), so gelu(u) = 0.5 u (1 + tanh(sqrt(2/pi)(u + 0.044715 u^3))).
+  * LayerNorm: biased variance, eps = 1e-5 inside the square root (PyTorch's
+    default, "Debugging checklist" item 6).
+  * Padded vocabulary columns take part in the softmax (no masking).
+  * Loss with ignore_index: mean over the targets != -1 of that call; if every
+    target is -1 the loss and all gradients are 0.
+  * Clip: coef = min(1, max_norm / (norm + 1e-6)); the reported norm is pre-clip.
+  * AdamW: decoupled decay scaled by lr, bias correction on both moments,
+    eps added after the square root, step counter starting at 1.
+
+Pins (tests/test_oracle_pins.py): finite differences, a torch float64
+autograd model plus torch's own cross_entropy / clip_grad_norm_ / AdamW,
+closed forms (initial loss, CE of equal logits, AdamW step 1, clip), the
+causal invariant, the T = 1 attention case, GELU identities, LN moments,
+the parameter count of "Counting parameters: 124,439,808", accumulation
+equivalence and single-batch overfitting. Parity pinned for every function.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+
+LN_EPS = 1e-5
+ADAM_BETA1 = 0.9
+ADAM_BETA2 = 0.95
+ADAM_EPS = 1e-8
+WEIGHT_DECAY = 0.1
+GRAD_CLIP = 1.0
+GELU_C = math.sqrt(2.0 / math.pi)
+
+
+@dataclass(frozen=True)
+class Shape:
+    n_layer: int
+    n_head: int
+    n_embd: int
+    vocab_size: int
+    block_size: int
+
+
+# ----------------------------------------------------------------------------
+# Parameters: "GPT-2 from Scratch", "The full model" / "Weight tying".
+# wte is the lm_head weight (one tensor, listed once).
+# ----------------------------------------------------------------------------
+def layout(s: Shape):
+    C, V = s.n_embd, s.vocab_size
+    names = [("wte", (V, C)), ("wpe", (s.block_size, C))]
+    for l in range(s.n_layer):
+        names += [
+            (f"h.{l}.ln_1.weight", (C,)), (f"h.{l}.ln_1.bias", (C,)),
+            (f"h.{l}.attn.c_attn.weight", (3 * C, C)), (f"h.{l}.attn.c_attn.bias", (3 * C,)),
+            (f"h.{l}.attn.c_proj.weight", (C, C)), (f"h.{l}.attn.c_proj.bias", (C,)),
+            (f"h.{l}.ln_2.weight", (C,)), (f"h.{l}.ln_2.bias", (C,)),
+            (f"h.{l}.mlp.c_fc.weight", (4 * C, C)), (f"h.{l}.mlp.c_fc.bias", (4 * C,)),
+            (f"h.{l}.mlp.c_proj.weight", (C, 4 * C)), (f"h.{l}.mlp.c_proj.bias", (C,)),
+        ]
+    names += [("ln_f.weight", (C,)), ("ln_f.bias", (C,))]
+    return names
+
+
+def unflatten(s: Shape, flat) -> dict:
+    out, off = {}, 0
+    for name, shp in layout(s):
+        n = int(np.prod(shp))
+        out[name] = np.asarray(flat[off:off + n], dtype=np.float64).reshape(shp).copy()
+        off += n
+    assert off == len(flat), (off, len(flat))
+    return out
+
+
+def flatten(s: Shape, d: dict) -> np.ndarray:
+    return np.concatenate([np.asarray(d[name], dtype=np.float64).reshape(-1) for name, _ in layout(s)])
+
+
+def decays(s: Shape) -> dict:
+    """Weight decay applies to tensors with dim >= 2: the matrices and the two
+    embeddings ("AdamW, and weight decay on matrices only")."""
+    return {name: (WEIGHT_DECAY if len(shp) >= 2 else 0.0) for name, shp in layout(s)}
+
+
+# ----------------------------------------------------------------------------
+# Building blocks, forward and hand-derived backward.
+# ----------------------------------------------------------------------------
+def layer_norm(x, w, b):
+    """nn.LayerNorm over the last axis: (x - mean) / sqrt(biased var + eps) * w + b."""
+    mu = x.mean(axis=-1, keepdims=True)
+    xc = x - mu
+    var = (xc * xc).mean(axis=-1, keepdims=True)
+    rstd = 1.0 / np.sqrt(var + LN_EPS)
+    xhat = xc * rstd
+    return xhat * w + b, (xhat, rstd)
+
+
+def layer_norm_backward(dy, saved, w):
+    """Gradient of layer_norm with respect to x, w and b (rows are independent)."""
+    xhat, rstd = saved
+    dxhat = dy * w
+    dw = (dy * xhat).reshape(-1, dy.shape[-1]).sum(axis=0)
+    db = dy.reshape(-1, dy.shape[-1]).sum(axis=0)
+    dx = rstd * (dxhat - dxhat.mean(axis=-1, keepdims=True)
+                 - xhat * (dxhat * xhat).mean(axis=-1, keepdims=True))
+    return dx, dw, db
+
+
+def gelu_tanh(u):
+    """GPT-2's GELU, tanh approximation ("The MLP and GPT-2's GELU")."""
+    return 0.5 * u * (1.0 + np.tanh(GELU_C * (u + 0.044715 * u ** 3)))
+
+
+def gelu_tanh_grad(u):
+    t = np.tanh(GELU_C * (u + 0.044715 * u ** 3))
+    return 0.5 * (1.0 + t) + 0.5 * u * (1.0 - t * t) * GELU_C * (1.0 + 3.0 * 0.044715 * u * u)
+
+
+def linear(x, w, b=None):
+    """nn.Linear with the (out, in) weight layout: x @ w.T + b."""
+    y = x @ w.T
+    return y if b is None else y + b
+
+
+def causal_attention(q, k, v):
+    """softmax(q k^T / sqrt(hd)) with -inf above the diagonal, then @ v.
+
+    q, k, v: (B, H, T, hd). Returns y (B, H, T, hd) and the probabilities P
+    (B, H, T, T) ("CausalSelfAttention", "Scaled dot-product and the output
+    projection" and "The causal mask as a registered buffer").
+    """
+    T, hd = q.shape[-2], q.shape[-1]
+    att = (q @ np.swapaxes(k, -1, -2)) / math.sqrt(hd)
+    future = np.triu(np.ones((T, T), dtype=bool), k=1)
+    att = np.where(future, -np.inf, att)
+    att = att - att.max(axis=-1, keepdims=True)
+    p = np.exp(att)
+    p = p / p.sum(axis=-1, keepdims=True)
+    return p @ v, p
+
+
+def causal_attention_backward(dy, q, k, v, p):
+    hd = q.shape[-1]
+    dv = np.swapaxes(p, -1, -2) @ dy
+    dp = dy @ np.swapaxes(v, -1, -2)
+    ds = p * (dp - (dp * p).sum(axis=-1, keepdims=True))   # softmax Jacobian, rowwise
+    dq = (ds @ k) / math.sqrt(hd)
+    dk = (np.swapaxes(ds, -1, -2) @ q) / math.sqrt(hd)
+    return dq, dk, dv
+
+
+def cross_entropy(logits, targets):
+    """F.cross_entropy(..., ignore_index=-1): mean of lse(row) - row[target] over
+    the rows whose target is not -1. Returns (loss, dlogits) where dlogits is the
+    gradient of that mean (softmax - onehot) / n_valid, zero on ignored rows."""
+    rows = logits.reshape(-1, logits.shape[-1])
+    t = targets.reshape(-1)
+    valid = t != -1
+    n_valid = int(valid.sum())
+    m = rows.max(axis=-1, keepdims=True)
+    e = np.exp(rows - m)
+    s = e.sum(axis=-1, keepdims=True)
+    lse = (m + np.log(s))[:, 0]
+    d = e / s
+    if n_valid == 0:
+        return 0.0, np.zeros_like(rows).reshape(logits.shape)
+    tv = np.where(valid, t, 0)
+    picked = rows[np.arange(rows.shape[0]), tv]
+    loss = float(((lse - picked) * valid).sum() / n_valid)
+    d[np.arange(rows.shape[0]), tv] -= 1.0
+    d *= (valid[:, None] / n_valid)
+    return loss, d.reshape(logits.shape)
+
+
+# ----------------------------------------------------------------------------
+# The model ("The full model", "The Block: pre-LN and residuals").
+# ----------------------------------------------------------------------------
+def forward(s: Shape, P: dict, idx, targets=None):
+    """Returns (loss or None, logits (B,T,V), cache). idx, targets: (B, T) ints."""
+    idx = np.asarray(idx)
+    B, T = idx.shape
+    assert T <= s.block_size
+    C, H = s.n_embd, s.n_head
+    hd = C // H
+    cache = {"idx": idx, "layers": []}
+    x = P["wte"][idx] + P["wpe"][np.arange(T)][None, :, :]          # (B,T,C)
+    for l in range(s.n_layer):
+        pre = f"h.{l}."
+        c = {}
+        a, c["ln1"] = layer_norm(x, P[pre + "ln_1.weight"], P[pre + "ln_1.bias"])
+        qkv = linear(a, P[pre + "attn.c_attn.weight"], P[pre + "attn.c_attn.bias"])
+        q, k, v = qkv[..., :C], qkv[..., C:2 * C], qkv[..., 2 * C:]
+        heads = lambda z: z.reshape(B, T, H, hd).transpose(0, 2, 1, 3)  # noqa: E731
+        q, k, v = heads(q), heads(k), heads(v)
+        y, p = causal_attention(q, k, v)
+        y = y.transpose(0, 2, 1, 3).reshape(B, T, C)
+        x = x + linear(y, P[pre + "attn.c_proj.weight"], P[pre + "attn.c_proj.bias"])
+        m, c["ln2"] = layer_norm(x, P[pre + "ln_2.weight"], P[pre + "ln_2.bias"])
+        u = linear(m, P[pre + "mlp.c_fc.weight"], P[pre + "mlp.c_fc.bias"])
+        g = gelu_tanh(u)
+        x = x + linear(g, P[pre + "mlp.c_proj.weight"], P[pre + "mlp.c_proj.bias"])
+        c.update(a=a, q=q, k=k, v=v, p=p, y=y, m=m, u=u, g=g)
+        cache["layers"].append(c)
+    f, cache["lnf"] = layer_norm(x, P["ln_f.weight"], P["ln_f.bias"])
+    cache["f"] = f
+    logits = linear(f, P["wte"])                                      # tied lm_head
+    loss = None
+    if targets is not None:
+        loss, dlogits = cross_entropy(logits, np.asarray(targets))
+        cache["dlogits"] = dlogits
+    return loss, logits, cache
+
+
+def backward(s: Shape, P: dict, cache, loss_scale: float = 1.0) -> dict:
+    """Exact gradient of loss_scale * loss with respect to every parameter."""
+    idx = cache["idx"]
+    B, T = idx.shape
+    C, H = s.n_embd, s.n_head
+    hd = C // H
+    G = {name: np.zeros(shp) for name, shp in layout(s)}
+    dlogits = cache["dlogits"] * loss_scale                           # (B,T,V)
+    f = cache["f"]
+    # lm_head (tied): logits = f @ wte.T
+    G["wte"] += dlogits.reshape(-1, dlogits.shape[-1]).T @ f.reshape(-1, C)
+    df = dlogits @ P["wte"]
+    dx, G["ln_f.weight"], G["ln_f.bias"] = layer_norm_backward(df, cache["lnf"], P["ln_f.weight"])
+    for l in reversed(range(s.n_layer)):
+        pre = f"h.{l}."
+        c = cache["layers"][l]
+        # x_out = x_mid + c_proj(gelu(c_fc(ln_2(x_mid))))
+        dproj = dx
+        G[pre + "mlp.c_proj.weight"] += dproj.reshape(-1, C).T @ c["g"].reshape(-1, 4 * C)
+        G[pre + "mlp.c_proj.bias"] += dproj.reshape(-1, C).sum(axis=0)
+        dg = dproj @ P[pre + "mlp.c_proj.weight"]
+        du = dg * gelu_tanh_grad(c["u"])
+        G[pre + "mlp.c_fc.weight"] += du.reshape(-1, 4 * C).T @ c["m"].reshape(-1, C)
+        G[pre + "mlp.c_fc.bias"] += du.reshape(-1, 4 * C).sum(axis=0)
+        dm = du @ P[pre + "mlp.c_fc.weight"]
+        dln, dw, db = layer_norm_backward(dm, c["ln2"], P[pre + "ln_2.weight"])
+        G[pre + "ln_2.weight"] += dw
+        G[pre + "ln_2.bias"] += db
+        dx = dx + dln
+        # x_mid = x_in + c_proj(attn(ln_1(x_in)))
+        G[pre + "attn.c_proj.weight"] += dx.reshape(-1, C).T @ c["y"].reshape(-1, C)
+        G[pre + "attn.c_proj.bias"] += dx.reshape(-1, C).sum(axis=0)
+        dy = (dx @ P[pre + "attn.c_proj.weight"]).reshape(B, T, H, hd).transpose(0, 2, 1, 3)
+        dq, dk, dv = causal_attention_backward(dy, c["q"], c["k"], c["v"], c["p"])
+        merge = lambda z: z.transpose(0, 2, 1, 3).reshape(B, T, C)  # noqa: E731
+        dqkv = np.concatenate([merge(dq), merge(dk), merge(dv)], axis=-1)
+        G[pre + "attn.c_attn.weight"] += dqkv.reshape(-1, 3 * C).T @ c["a"].reshape(-1, C)
+        G[pre + "attn.c_attn.bias"] += dqkv.reshape(-1, 3 * C).sum(axis=0)
+        da = dqkv @ P[pre + "attn.c_attn.weight"]
+        dln, dw, db = layer_norm_backward(da, c["ln1"], P[pre + "ln_1.weight"])
+        G[pre + "ln_1.weight"] += dw
+        G[pre + "ln_1.bias"] += db
+        dx = dx + dln
+    # x0 = wte[idx] + wpe[arange(T)]: scatter-add into the same tied wte gradient
+    np.add.at(G["wte"], idx.reshape(-1), dx.reshape(-1, C))
+    G["wpe"][:T] += dx.sum(axis=0)
+    return G
+
+
+# ----------------------------------------------------------------------------
+# Update: "Gradient clipping" and "AdamW, and weight decay on matrices only".
+# ----------------------------------------------------------------------------
+def grad_norm(G: dict) -> float:
+    """Global L2 norm over every unique parameter tensor (the tied wte once)."""
+    return math.sqrt(sum(float((g * g).sum()) for g in G.values()))
+
+
+def clip_coefficient(norm: float, max_norm: float = GRAD_CLIP) -> float:
+    return min(1.0, max_norm / (norm + 1e-6))
+
+
+def adamw_update(s: Shape, P: dict, G: dict, M: dict, V: dict, t: int, lr: float,
+                 max_norm: float = GRAD_CLIP):
+    """One clipped AdamW step. t is the 1-based step counter after increment.
+
+    Returns the pre-clip global norm. P, M, V are updated in place."""
+    norm = grad_norm(G)
+    coef = clip_coefficient(norm, max_norm)
+    bc1 = 1.0 - ADAM_BETA1 ** t
+    bc2 = 1.0 - ADAM_BETA2 ** t
+    wd = decays(s)
+    for name in P:
+        g = G[name] * coef
+        M[name] = ADAM_BETA1 * M[name] + (1.0 - ADAM_BETA1) * g
+        V[name] = ADAM_BETA2 * V[name] + (1.0 - ADAM_BETA2) * g * g
+        mhat = M[name] / bc1
+        vhat = V[name] / bc2
+        P[name] = P[name] * (1.0 - lr * wd[name]) - lr * mhat / (np.sqrt(vhat) + ADAM_EPS)
+    return norm
+
+
+def zeros_like(s: Shape) -> dict:
+    return {name: np.zeros(shp) for name, shp in layout(s)}
+
+
+def train_step(s: Shape, P: dict, M: dict, V: dict, t: int, idx, targets, lr: float,
+               max_norm: float = GRAD_CLIP):
+    """zero_grad, forward, loss, backward, clip, AdamW ("The loop").
+
+    Returns (loss, pre-clip norm, grads). P, M, V updated in place; t is the
+    step number after increment (1 for the first step)."""
+    loss, _, cache = forward(s, P, idx, targets)
+    G = backward(s, P, cache)
+    norm = adamw_update(s, P, G, M, V, t, lr, max_norm)
+    return loss, norm, G
+
+
+def accumulate_grads(s: Shape, P: dict, batches, n_micro=None):
+    """Gradient accumulation: each micro-batch's mean loss divided by the number
+    of micro-batches before its gradient is added ("How to scale up";
+    "Gradient accumulation, and the bug in getting it right"). Returns
+    (mean of the micro losses, summed grads)."""
+    n = n_micro or len(batches)
+    G = zeros_like(s)
+    total = 0.0
+    for idx, tgt in batches:
+        loss, _, cache = forward(s, P, idx, tgt)
+        g = backward(s, P, cache, loss_scale=1.0 / n)
+        for k in G:
+            G[k] += g[k]
+        total += loss
+    return total / n, G

@@ -1,0 +1,457 @@
+"""Pins of the CPU oracle to facts other than itself (no GPU needed).
+
+Each test checks the oracle against something the pages or the mathematics
+fix: printed values (tests/golden/pages_values.json), closed forms, invariants,
+finite differences, and independent library routines (torch's nn.LayerNorm,
+scaled_dot_product_attention, nn.GELU(approximate="tanh"), F.cross_entropy,
+clip_grad_norm_ and torch.optim.AdamW, with gradients from autograd).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import gpt2_oracle as O
+from decoder_only_transformer_sm_b200 import synthetic as S
+
+GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "pages_values.json")))
+
+TINY = O.Shape(n_layer=2, n_head=4, n_embd=128, vocab_size=1024, block_size=64)
+MICRO = O.Shape(n_layer=2, n_head=2, n_embd=16, vocab_size=64, block_size=8)
+
+
+def _syn(s: O.Shape):
+    return S.ModelShape(s.n_layer, s.n_head, s.n_embd, s.vocab_size, s.block_size)
+
+
+def _params(s, seed=0, kind="init"):
+    flat = S.init_params(_syn(s), seed) if kind == "init" else S.random_params(_syn(s), seed)
+    return O.unflatten(s, flat.astype(np.float64))
+
+
+# ----------------------------------------------------------------------------
+# Shapes and parameter count ("Counting parameters: 124,439,808").
+# ----------------------------------------------------------------------------
+def test_param_count_matches_pages():
+    s = O.Shape(12, 12, 768, 50257, 1024)
+    n = sum(int(np.prod(shp)) for _, shp in O.layout(s))
+    assert n == GOLDEN["param_count_124M_tied"]["value"]
+    # untied lm_head would add exactly V*C
+    assert 50257 * 768 == GOLDEN["tie_delta"]["value"]
+    # the mask buffers (one T_max x T_max per layer) are not parameters
+    assert 12 * 1024 * 1024 == GOLDEN["mask_buffer_delta"]["value"]
+    assert 12 * 768 ** 2 == GOLDEN["per_block_weights_124M"]["value"]
+
+
+def test_layout_agrees_with_generator_layout():
+    for s in (TINY, O.Shape(12, 12, 768, 50304, 1024)):
+        a = [(n, tuple(shp)) for n, shp in O.layout(s)]
+        b = [(n, tuple(shp)) for n, shp, _ in S.param_layout(_syn(s))]
+        assert a == b
+
+
+def test_debug_shapes():
+    g = GOLDEN["debug_shapes"]
+    s = O.Shape(1, 12, 768, 50257, 1024)   # one block is enough for the shapes
+    rng = np.random.default_rng(0)
+    P = {name: rng.normal(0, 0.02, shp) for name, shp in O.layout(s)}
+    idx = rng.integers(0, 50257, (2, 5))
+    _, logits, cache = O.forward(s, P, idx)
+    assert list(logits.shape) == g["logits"]
+    assert list(cache["f"].shape) == g["residual"]
+    assert list(cache["layers"][0]["p"].shape) == g["scores"]
+
+
+def test_resid_init_std():
+    assert round(0.02 / math.sqrt(2 * 12), 4) == GOLDEN["resid_init_std_12_layers"]["value"]
+    flat = S.init_params(_syn(O.Shape(12, 12, 768, 50304, 1024)), seed=3)
+    P = O.unflatten(O.Shape(12, 12, 768, 50304, 1024), flat)
+    w = P["h.5.mlp.c_proj.weight"]
+    assert abs(w.std() - 0.02 / math.sqrt(24)) < 2e-5
+    assert abs(P["h.5.mlp.c_fc.weight"].std() - 0.02) < 5e-5
+    assert np.all(P["h.5.ln_1.weight"] == 1) and np.all(P["h.5.attn.c_attn.bias"] == 0)
+
+
+# ----------------------------------------------------------------------------
+# Initial loss ~ ln V ("Debugging checklist" item 2).
+# E[loss] ~ ln V + Var(logit)/2 with Var(logit) = 0.02^2 * C for unit-variance LN rows.
+# ----------------------------------------------------------------------------
+def test_initial_loss_tiny():
+    P = _params(TINY, seed=0)
+    idx, tgt = S.uniform_tokens(4, 64, 1024, seed=1000)
+    loss, _, _ = O.forward(TINY, P, idx, tgt)
+    closed = math.log(1024) + 0.5 * 0.02 ** 2 * 128
+    assert abs(loss - closed) < 0.05, (loss, closed)
+
+
+@pytest.mark.slow
+def test_initial_loss_124M_padded():
+    s = O.Shape(12, 12, 768, 50304, 1024)
+    P = O.unflatten(s, S.init_params(_syn(s), seed=0))
+    idx, tgt = S.zipf_tokens(1, 256, 50257, seed=1001)
+    loss, _, _ = O.forward(s, P, idx, tgt)
+    assert abs(loss - GOLDEN["init_loss_V50304"]["value"]) < 0.2
+    assert abs(loss - (math.log(50304) + 0.5 * 0.02 ** 2 * 768)) < 0.1
+
+
+# ----------------------------------------------------------------------------
+# Attention ("Debugging checklist" item 3; causal mask section).
+# ----------------------------------------------------------------------------
+def test_attention_rows_and_future():
+    rng = np.random.default_rng(1)
+    q, k, v = (rng.normal(size=(2, 3, 17, 8)) for _ in range(3))
+    y, p = O.causal_attention(q, k, v)
+    assert np.allclose(p.sum(-1), 1.0, atol=1e-12)
+    assert np.all(p[..., np.triu_indices(17, 1)[0], np.triu_indices(17, 1)[1]] == 0.0)
+    # brute force, one (b, h, i) at a time
+    for (b, h, i) in [(0, 0, 0), (1, 2, 16), (0, 1, 7)]:
+        s = np.array([q[b, h, i] @ k[b, h, j] / math.sqrt(8) for j in range(i + 1)])
+        w = np.exp(s - s.max()); w /= w.sum()
+        assert np.allclose(y[b, h, i], (w[:, None] * v[b, h, :i + 1]).sum(0), atol=1e-12)
+
+
+def test_attention_T1_is_v():
+    rng = np.random.default_rng(2)
+    q, k, v = (rng.normal(size=(2, 3, 1, 8)) for _ in range(3))
+    y, _ = O.causal_attention(q, k, v)
+    assert np.array_equal(y, v)
+
+
+def test_causal_invariance():
+    P = _params(TINY, seed=4, kind="random")
+    idx, _ = S.uniform_tokens(2, 40, 1024, seed=5)
+    _, la, _ = O.forward(TINY, P, idx)
+    idx2 = idx.copy()
+    t = 17
+    idx2[:, t + 1:] = (idx2[:, t + 1:] + 123) % 1024
+    _, lb, _ = O.forward(TINY, P, idx2)
+    assert np.array_equal(la[:, :t + 1], lb[:, :t + 1])
+    assert not np.allclose(la[:, t + 1:], lb[:, t + 1:])
+
+
+def test_position_zero_indexing():
+    """Row t uses wpe[t] (positions start at 0): changing wpe[7] moves only position 7.
+
+    The perturbation is random, since a constant shift of a row is removed by LayerNorm."""
+    P = _params(TINY, seed=6, kind="random")
+    idx, _ = S.uniform_tokens(1, 8, 1024, seed=7)
+    _, la, _ = O.forward(TINY, P, idx)
+    P["wpe"][7] += np.random.default_rng(0).normal(size=128)   # last used position
+    _, lb, _ = O.forward(TINY, P, idx)
+    assert np.array_equal(la[:, :7], lb[:, :7]) and not np.allclose(la[:, 7], lb[:, 7])
+
+
+# ----------------------------------------------------------------------------
+# GELU ("The MLP and GPT-2's GELU").
+# ----------------------------------------------------------------------------
+def test_gelu_identities():
+    x = np.linspace(-12, 12, 200001)
+    assert O.gelu_tanh(np.array([0.0]))[0] == 0.0
+    assert np.max(np.abs(O.gelu_tanh(x) - O.gelu_tanh(-x) - x)) < 1e-13
+    erf_gelu = 0.5 * x * (1 + np.vectorize(math.erf)(x / math.sqrt(2)))
+    d = np.max(np.abs(O.gelu_tanh(x) - erf_gelu))
+    assert d < GOLDEN["gelu_tanh_vs_erf_bound"]["value"] and d > 1e-5
+    h = 1e-6
+    fd = (O.gelu_tanh(x + h) - O.gelu_tanh(x - h)) / (2 * h)
+    assert np.max(np.abs(fd - O.gelu_tanh_grad(x))) < 1e-8
+    # torch's own tanh-GELU as a library routine
+    torch = pytest.importorskip("torch")
+    t = torch.nn.functional.gelu(torch.from_numpy(x), approximate="tanh").numpy()
+    assert np.max(np.abs(t - O.gelu_tanh(x))) < 1e-14
+
+
+# ----------------------------------------------------------------------------
+# LayerNorm moments (biased variance, eps inside the sqrt).
+# ----------------------------------------------------------------------------
+def test_layernorm_moments():
+    rng = np.random.default_rng(8)
+    x = rng.normal(3.0, 0.01, size=(5, 64))
+    y, _ = O.layer_norm(x, np.ones(64), np.zeros(64))
+    var = x.var(axis=-1)
+    assert np.allclose(y.mean(-1), 0.0, atol=1e-12)
+    assert np.allclose((y * y).mean(-1), var / (var + O.LN_EPS), rtol=1e-12)
+    b = rng.normal(size=64)
+    y2, _ = O.layer_norm(x, np.ones(64), b)
+    assert np.allclose(y2.mean(-1), b.mean(), atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# Cross-entropy with ignore_index = -1.
+# ----------------------------------------------------------------------------
+def test_cross_entropy_closed_forms():
+    V = 37
+    logits = np.full((2, 3, V), 0.7)
+    tg = np.array([[1, -1, 5], [36, 0, -1]])
+    loss, d = O.cross_entropy(logits, tg)
+    assert abs(loss - math.log(V)) < 1e-14
+    nv = 4
+    expect = np.full((2, 3, V), 1.0 / V / nv)
+    expect[1 - 1 + 0, 1] = 0; expect[1, 2] = 0
+    for (b, t) in [(0, 0), (0, 2), (1, 0), (1, 1)]:
+        expect[b, t, tg[b, t]] -= 1.0 / nv
+    assert np.allclose(d, expect, atol=1e-15)
+    # all ignored
+    loss0, d0 = O.cross_entropy(logits, np.full((2, 3), -1))
+    assert loss0 == 0.0 and not d0.any()
+
+
+def test_cross_entropy_vs_torch():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(9)
+    logits = rng.normal(size=(50, 77)) * 3
+    tg = rng.integers(-1, 77, size=50)
+    loss, d = O.cross_entropy(logits, tg)
+    lt = torch.tensor(logits, requires_grad=True)
+    ref = torch.nn.functional.cross_entropy(lt, torch.tensor(tg), ignore_index=-1)
+    ref.backward()
+    assert abs(loss - ref.item()) < 1e-13
+    assert np.max(np.abs(d - lt.grad.numpy())) < 1e-15
+
+
+# ----------------------------------------------------------------------------
+# Finite differences of the whole loss (double precision).
+# ----------------------------------------------------------------------------
+def _fd_check(s, P, idx, tgt, coords_per_tensor, rng, h=1e-5):
+    loss, _, cache = O.forward(s, P, idx, tgt)
+    G = O.backward(s, P, cache)
+    for name, shp in O.layout(s):
+        n = int(np.prod(shp))
+        picks = np.arange(n) if coords_per_tensor is None or n <= coords_per_tensor \
+            else rng.choice(n, coords_per_tensor, replace=False)
+        flatp = P[name].reshape(-1)
+        g = G[name].reshape(-1)
+        for i in picks:
+            old = flatp[i]
+            flatp[i] = old + h
+            lp, _, _ = O.forward(s, P, idx, tgt)
+            flatp[i] = old - h
+            lm, _, _ = O.forward(s, P, idx, tgt)
+            flatp[i] = old
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - g[i]) <= 1e-5 * abs(g[i]) + 2e-9, (name, i, fd, g[i])
+
+
+def test_finite_differences_micro_every_coordinate():
+    s = MICRO
+    P = _params(s, seed=10, kind="random")
+    for k in P:                                   # larger weights: stronger nonlinearity
+        if k.endswith(".weight") and P[k].ndim == 2 or k in ("wte", "wpe"):
+            P[k] *= 10.0
+    idx, tgt = S.uniform_tokens(2, 8, 64, seed=11)
+    tgt[0, :3] = -1
+    _fd_check(s, P, idx, tgt, None, np.random.default_rng(0))
+
+
+def test_finite_differences_tiny_sampled():
+    P = _params(TINY, seed=12, kind="random")
+    idx, tgt = S.uniform_tokens(2, 24, 1024, seed=13)
+    tgt[1, :10] = -1
+    _fd_check(TINY, P, idx, tgt, 6, np.random.default_rng(1))
+
+
+# ----------------------------------------------------------------------------
+# Independent model from torch library layers, autograd and torch's optimiser.
+# ----------------------------------------------------------------------------
+def _torch_model_step(s, flat, idx, tgt, lr, steps, max_norm=1.0):
+    torch = pytest.importorskip("torch")
+    F = torch.nn.functional
+    names = [n for n, _ in O.layout(s)]
+    shapes = dict(O.layout(s))
+    P = {}
+    off = 0
+    for n in names:
+        k = int(np.prod(shapes[n]))
+        P[n] = torch.tensor(flat[off:off + k].reshape(shapes[n]), dtype=torch.float64, requires_grad=True)
+        off += k
+    C, H = s.n_embd, s.n_head
+
+    def model(idx_t, tgt_t):
+        B, T = idx_t.shape
+        x = F.embedding(idx_t, P["wte"]) + F.embedding(torch.arange(T), P["wpe"])
+        for l in range(s.n_layer):
+            p = f"h.{l}."
+            a = F.layer_norm(x, (C,), P[p + "ln_1.weight"], P[p + "ln_1.bias"], eps=1e-5)
+            q, k, v = F.linear(a, P[p + "attn.c_attn.weight"], P[p + "attn.c_attn.bias"]).split(C, dim=2)
+            q, k, v = (z.view(B, T, H, C // H).transpose(1, 2) for z in (q, k, v))
+            y = F.scaled_dot_product_attention(q, k, v, is_causal=True)
+            y = y.transpose(1, 2).contiguous().view(B, T, C)
+            x = x + F.linear(y, P[p + "attn.c_proj.weight"], P[p + "attn.c_proj.bias"])
+            m = F.layer_norm(x, (C,), P[p + "ln_2.weight"], P[p + "ln_2.bias"], eps=1e-5)
+            u = F.gelu(F.linear(m, P[p + "mlp.c_fc.weight"], P[p + "mlp.c_fc.bias"]), approximate="tanh")
+            x = x + F.linear(u, P[p + "mlp.c_proj.weight"], P[p + "mlp.c_proj.bias"])
+        f = F.layer_norm(x, (C,), P["ln_f.weight"], P["ln_f.bias"], eps=1e-5)
+        logits = F.linear(f, P["wte"])
+        return F.cross_entropy(logits.view(-1, logits.size(-1)), tgt_t.view(-1), ignore_index=-1)
+
+    decay = [P[n] for n in names if P[n].dim() >= 2]
+    nodecay = [P[n] for n in names if P[n].dim() < 2]
+    opt = torch.optim.AdamW([{"params": decay, "weight_decay": 0.1},
+                             {"params": nodecay, "weight_decay": 0.0}],
+                            lr=lr, betas=(0.9, 0.95), eps=1e-8, foreach=False)
+    out = []
+    for _ in range(steps):
+        opt.zero_grad(set_to_none=True)
+        loss = model(torch.tensor(idx, dtype=torch.long), torch.tensor(tgt, dtype=torch.long))
+        loss.backward()
+        grads = {n: P[n].grad.detach().clone().numpy() for n in names}
+        norm = torch.nn.utils.clip_grad_norm_(list(P.values()), max_norm)
+        opt.step()
+        out.append((loss.item(), float(norm), grads))
+    params = {n: P[n].detach().numpy().copy() for n in names}
+    return out, params
+
+
+@pytest.mark.parametrize("max_norm", [1.0, 0.01])
+def test_oracle_matches_torch_library_model(max_norm):
+    s = TINY
+    flat = S.random_params(S.ModelShape(2, 4, 128, 1024, 64), seed=14).astype(np.float64)
+    idx, tgt = S.uniform_tokens(3, 33, 1024, seed=15)
+    tgt[2, :9] = -1
+    ref, ref_params = _torch_model_step(s, flat, idx, tgt, lr=6e-4, steps=2, max_norm=max_norm)
+    P = O.unflatten(s, flat)
+    M, V = O.zeros_like(s), O.zeros_like(s)
+    for t in (1, 2):
+        loss, norm, G = O.train_step(s, P, M, V, t, idx, tgt, lr=6e-4, max_norm=max_norm)
+        rl, rn, rg = ref[t - 1]
+        assert abs(loss - rl) < 1e-12
+        assert abs(norm - rn) < 1e-12
+        for n in G:
+            assert np.max(np.abs(G[n] - rg[n])) < 1e-12 * max(1.0, np.max(np.abs(rg[n]))), n
+    for n in P:
+        assert np.max(np.abs(P[n] - ref_params[n])) < 1e-12, n
+
+
+# ----------------------------------------------------------------------------
+# Update closed forms ("Gradient clipping"; AdamW step 1).
+# ----------------------------------------------------------------------------
+def test_adamw_step1_closed_form_and_clip():
+    s = MICRO
+    rng = np.random.default_rng(16)
+    P = _params(s, seed=17, kind="random")
+    P0 = {k: v.copy() for k, v in P.items()}
+    G = {k: rng.normal(size=v.shape) for k, v in P.items()}
+    M, V = O.zeros_like(s), O.zeros_like(s)
+    lr = 1e-3
+    norm = O.adamw_update(s, P, G, M, V, 1, lr)
+    true_norm = math.sqrt(sum((g * g).sum() for g in G.values()))
+    assert abs(norm - true_norm) < 1e-12
+    c = 1.0 / (true_norm + 1e-6)
+    assert c < 1
+    # post-clip norm = norm / (norm + 1e-6)
+    post = math.sqrt(sum(((c * g) ** 2).sum() for g in G.values()))
+    assert abs(post - true_norm / (true_norm + 1e-6)) < 1e-12
+    for name, shp in O.layout(s):
+        wd = 0.1 if len(shp) == 2 else 0.0
+        cg = c * G[name]
+        assert np.allclose(M[name], 0.1 * cg, rtol=1e-14, atol=0)
+        assert np.allclose(V[name], 0.05 * cg * cg, rtol=1e-14, atol=0)
+        expect = P0[name] * (1 - lr * wd) - lr * cg / (np.abs(cg) + 1e-8)
+        assert np.allclose(P[name], expect, rtol=1e-12, atol=1e-16), name
+
+
+def test_no_clip_below_threshold():
+    s = MICRO
+    P = _params(s, seed=18, kind="random")
+    G = {k: np.full(v.shape, 1e-4) for k, v in P.items()}
+    M, V = O.zeros_like(s), O.zeros_like(s)
+    O.adamw_update(s, P, G, M, V, 1, 1e-3)
+    assert np.allclose(M["wte"], 0.1 * 1e-4, rtol=1e-14)
+
+
+def test_decay_groups():
+    d = O.decays(TINY)
+    assert d["wte"] == 0.1 and d["wpe"] == 0.1 and d["h.0.attn.c_attn.weight"] == 0.1
+    assert d["h.1.mlp.c_proj.bias"] == 0.0 and d["h.0.ln_1.weight"] == 0.0 and d["ln_f.bias"] == 0.0
+
+
+# ----------------------------------------------------------------------------
+# Gradient accumulation ("Gradient accumulation, and the bug in getting it right").
+# ----------------------------------------------------------------------------
+def test_accumulation_equals_big_batch():
+    s = TINY
+    P = _params(s, seed=19, kind="random")
+    idx, tgt = S.uniform_tokens(4, 20, 1024, seed=20)
+    loss_big, _, cache = O.forward(s, P, idx, tgt)
+    G_big = O.backward(s, P, cache)
+    loss_acc, G_acc = O.accumulate_grads(s, P, [(idx[i:i + 1], tgt[i:i + 1]) for i in range(4)])
+    assert abs(loss_big - loss_acc) < 1e-12
+    for n in G_big:
+        assert np.max(np.abs(G_big[n] - G_acc[n])) < 1e-13, n
+
+
+# ----------------------------------------------------------------------------
+# Weight tying: one wte row feeds both the input and its logit column.
+# ----------------------------------------------------------------------------
+def test_tying_changes_input_and_output():
+    s = TINY
+    P = _params(s, seed=21, kind="random")
+    idx = np.array([[5, 6, 7]])
+    _, la, _ = O.forward(s, P, idx)
+    rng = np.random.default_rng(0)           # random vectors: LayerNorm removes constant shifts
+    P["wte"][900] += rng.normal(size=128)    # a token that is not in the input
+    _, lb, _ = O.forward(s, P, idx)
+    d = np.abs(la - lb)[0]
+    assert d[:, 900].min() > 0 and np.array_equal(np.delete(d, 900, axis=1), np.zeros((3, 1023)))
+    P["wte"][6] += rng.normal(size=128)   # the token at position 1: positions >= 1 move everywhere,
+    _, lc, _ = O.forward(s, P, idx)     # position 0 only in its output column 6
+    d0 = np.abs(lb[0, 0] - lc[0, 0])
+    assert d0[6] > 0 and np.array_equal(np.delete(d0, 6), np.zeros(1023))
+    assert np.abs(lb[0, 1:] - lc[0, 1:]).min() > 0
+
+
+# ----------------------------------------------------------------------------
+# Overfitting one batch ("Debugging checklist" item 4).
+# ----------------------------------------------------------------------------
+@pytest.mark.slow
+def test_overfit_single_batch():
+    s = O.Shape(n_layer=2, n_head=4, n_embd=64, vocab_size=128, block_size=16)
+    P = O.unflatten(s, S.init_params(S.ModelShape(2, 4, 64, 128, 16), seed=22))
+    M, V = O.zeros_like(s), O.zeros_like(s)
+    idx, tgt = S.uniform_tokens(2, 16, 128, seed=23)
+    first = None
+    for t in range(1, 201):
+        loss, _, _ = O.train_step(s, P, M, V, t, idx, tgt, lr=3e-3)
+        first = first if first is not None else loss
+    assert first > 4.5 and loss < 0.1, (first, loss)
+
+
+# ----------------------------------------------------------------------------
+# The pins are sensitive: a planted mistake in the oracle's backward fails them.
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("mutation", ["ln_drop_term", "gelu_grad_const", "attn_rowsum", "tie_scatter"])
+def test_planted_mistakes_are_caught(monkeypatch, mutation):
+    if mutation == "ln_drop_term":
+        def bad(dy, saved, w):
+            xhat, rstd = saved
+            dxhat = dy * w
+            dx = rstd * (dxhat - dxhat.mean(axis=-1, keepdims=True))
+            return dx, (dy * xhat).reshape(-1, dy.shape[-1]).sum(0), dy.reshape(-1, dy.shape[-1]).sum(0)
+        monkeypatch.setattr(O, "layer_norm_backward", bad)
+    elif mutation == "gelu_grad_const":
+        good = O.gelu_tanh_grad
+        monkeypatch.setattr(O, "gelu_tanh_grad", lambda u: good(u) * 1.01)
+    elif mutation == "attn_rowsum":
+        def bad(dy, q, k, v, p):
+            hd = q.shape[-1]
+            dv = np.swapaxes(p, -1, -2) @ dy
+            ds = p * (dy @ np.swapaxes(v, -1, -2))
+            return (ds @ k) / math.sqrt(hd), (np.swapaxes(ds, -1, -2) @ q) / math.sqrt(hd), dv
+        monkeypatch.setattr(O, "causal_attention_backward", bad)
+    elif mutation == "tie_scatter":
+        good_backward = O.backward
+
+        def bad_backward(s, P, cache, loss_scale=1.0):
+            G = good_backward(s, P, cache, loss_scale)
+            G["wte"][cache["idx"].reshape(-1)] *= 0.5      # lose part of the embedding scatter
+            return G
+        monkeypatch.setattr(O, "backward", bad_backward)
+    s = MICRO
+    P = _params(s, seed=30, kind="random")
+    for k in P:
+        if P[k].ndim == 2:
+            P[k] *= 10.0
+    idx, tgt = S.uniform_tokens(2, 8, 64, seed=31)
+    with pytest.raises(AssertionError):
+        _fd_check(s, P, idx, tgt, 8, np.random.default_rng(2))
