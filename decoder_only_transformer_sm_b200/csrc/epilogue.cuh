@@ -1,0 +1,108 @@
+// GEMM epilogue application, shared by the SIMT and the tensor-core GEMMs.
+#pragma once
+
+#include "kernels.cuh"
+
+namespace gpt2 {
+
+// Scalar epilogue for columns [col, col + n) of one row (n <= N_MAX).
+template <typename T>
+__device__ __forceinline__ void epilogue_scalar(const Epilogue& ep, long long row, int col, int n,
+                                                const float* acc) {
+    const long long base = row * ep.ldo + col;
+    for (int j = 0; j < n; ++j) {
+        const float a = acc[j];
+        switch (ep.kind) {
+        case EPI_STORE: reinterpret_cast<T*>(ep.out)[base + j] = from_f<T>(a); break;
+        case EPI_BIAS: reinterpret_cast<T*>(ep.out)[base + j] = from_f<T>(a + ep.bias[col + j]); break;
+        case EPI_BIAS_GELU: {
+            T u = from_f<T>(a + ep.bias[col + j]);   // stored pre-activation
+            reinterpret_cast<T*>(ep.out2)[base + j] = u;
+            reinterpret_cast<T*>(ep.out)[base + j] = from_f<T>(gelu_tanh(to_f(u)));
+            break;
+        }
+        case EPI_BIAS_RESID:
+            reinterpret_cast<float*>(ep.out)[base + j] = ep.resid[base + j] + (a + ep.bias[col + j]);
+            break;
+        case EPI_DGELU: {
+            const T u = reinterpret_cast<const T*>(ep.aux)[base + j];
+            reinterpret_cast<T*>(ep.out)[base + j] = from_f<T>(a * gelu_tanh_grad(to_f(u)));
+            break;
+        }
+        case EPI_ACCUM_F32: {
+            float* o = reinterpret_cast<float*>(ep.out) + base + j;
+            *o = (ep.beta != 0.f ? ep.beta * *o : 0.f) + a;
+            break;
+        }
+        default: break;
+        }
+    }
+}
+
+// Four consecutive columns, all in range, 4-element aligned.
+template <typename T>
+__device__ __forceinline__ void epilogue_vec4(const Epilogue& ep, long long base, int col, const float* acc) {
+    float v[4], b[4];
+    switch (ep.kind) {
+    case EPI_STORE:
+        store4(reinterpret_cast<T*>(ep.out) + base, acc);
+        break;
+    case EPI_BIAS:
+        load4(ep.bias + col, b);
+        for (int j = 0; j < 4; ++j) v[j] = acc[j] + b[j];
+        store4(reinterpret_cast<T*>(ep.out) + base, v);
+        break;
+    case EPI_BIAS_GELU: {
+        load4(ep.bias + col, b);
+        for (int j = 0; j < 4; ++j) v[j] = to_f(from_f<T>(acc[j] + b[j]));   // value as stored
+        store4(reinterpret_cast<T*>(ep.out2) + base, v);
+        for (int j = 0; j < 4; ++j) v[j] = gelu_tanh(v[j]);
+        store4(reinterpret_cast<T*>(ep.out) + base, v);
+        break;
+    }
+    case EPI_BIAS_RESID: {
+        float r[4];
+        load4(ep.bias + col, b);
+        load4(ep.resid + base, r);
+        for (int j = 0; j < 4; ++j) v[j] = r[j] + (acc[j] + b[j]);
+        store4(reinterpret_cast<float*>(ep.out) + base, v);
+        break;
+    }
+    case EPI_DGELU: {
+        float u[4];
+        load4(reinterpret_cast<const T*>(ep.aux) + base, u);
+        for (int j = 0; j < 4; ++j) v[j] = acc[j] * gelu_tanh_grad(u[j]);
+        store4(reinterpret_cast<T*>(ep.out) + base, v);
+        break;
+    }
+    case EPI_ACCUM_F32: {
+        float* o = reinterpret_cast<float*>(ep.out) + base;
+        if (ep.beta != 0.f) {
+            float old[4];
+            load4(o, old);
+            for (int j = 0; j < 4; ++j) v[j] = ep.beta * old[j] + acc[j];
+        } else {
+            for (int j = 0; j < 4; ++j) v[j] = acc[j];
+        }
+        store4(o, v);
+        break;
+    }
+    default: break;
+    }
+}
+
+// Apply the epilogue to N_RUN consecutive columns [col, col + N_RUN) of one row.
+// Columns at or beyond n_cols are skipped.
+template <typename T, int N_RUN>
+__device__ __forceinline__ void epilogue_run(const Epilogue& ep, long long row, int col, int n_cols,
+                                             const float* acc) {
+    const long long base = row * ep.ldo + col;
+    if (col + N_RUN <= n_cols && (base & 3) == 0 && (col & 3) == 0) {
+#pragma unroll
+        for (int j = 0; j < N_RUN; j += 4) epilogue_vec4<T>(ep, base + j, col + j, acc + j);
+    } else {
+        epilogue_scalar<T>(ep, row, col, min(N_RUN, n_cols - col), acc);
+    }
+}
+
+}  // namespace gpt2

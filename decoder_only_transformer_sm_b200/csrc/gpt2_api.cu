@@ -1,0 +1,727 @@
+// Runtime and C ABI of the GPT-2 training step: owns every buffer of one model
+// and enqueues the kernels of forward, loss, backward, clip and AdamW on the
+// handle's stream.
+//
+// Step structure ("GPT-2 from Scratch": "The full model", "The Block: pre-LN and
+// residuals", "The loop", "Gradient clipping", "AdamW, and weight decay on
+// matrices only"; "Let's reproduce GPT-2 (124M)", "Gradient accumulation, and
+// the bug in getting it right"):
+//   x0 = wte[idx] + wpe[t]
+//   per block: x += c_proj(attn(ln_1(x)));  x += mlp_c_proj(gelu(c_fc(ln_2(x))))
+//   logits = ln_f(x) wte^T;  loss = mean CE over targets != -1
+//   backward in reverse; grads accumulate (scaled by loss_scale per micro-batch)
+//   norm = ||g||_2;  g *= min(1, clip / (norm + 1e-6));  AdamW.
+#include "gpt2.h"
+#include "kernels.cuh"
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+using namespace gpt2;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const std::string& msg) {
+    g_last_error = msg;
+    return code;
+}
+
+#define CK(call)                                                                                   \
+    do {                                                                                           \
+        cudaError_t e_ = (call);                                                                   \
+        if (e_ != cudaSuccess) {                                                                   \
+            return fail(GPT2_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_));        \
+        }                                                                                          \
+    } while (0)
+
+struct TensorRec {
+    std::string name;
+    int ndim;
+    long long shape[2];
+    long long offset;
+    int decay;
+};
+
+struct DevScalars {
+    double loss_accum;   // accumulated scaled training loss
+    double fwd_loss;     // loss of the last forward-only call
+    double sumsq;        // global gradient sum of squares
+    int n_valid;         // targets != -1 in the current micro-batch
+    unsigned status;     // STATUS_* bits
+};
+
+struct LayerOff {   // offsets of one block's tensors in the flat vector
+    long long ln1w, ln1b, wqkv, bqkv, wproj, bproj, ln2w, ln2b, wfc, bfc, wfcp, bfcp;
+};
+
+}  // namespace
+
+namespace gpt2 {
+int set_error(int code, const char* msg) { return fail(code, msg); }
+}  // namespace gpt2
+
+struct gpt2_handle {
+    gpt2_config cfg;
+    cudaStream_t stream = nullptr;
+    int device = 0, num_sms = 148;
+    bool bf16_mode = false;
+    int C = 0, L = 0, H = 0, hd = 0, V = 0, maxBT = 0;
+
+    std::vector<TensorRec> tensors;
+    std::vector<LayerOff> lo;
+    long long off_wte = 0, off_wpe = 0, off_lnfw = 0, off_lnfb = 0;
+    long long n_params = 0;
+
+    float* params = nullptr;
+    float* grads = nullptr;
+    float* mom1 = nullptr;
+    float* mom2 = nullptr;
+    bf16* shadow = nullptr;
+    AdamChunk* d_chunks = nullptr;
+    int n_chunks = 0;
+
+    // activations (element type = act type of the mode)
+    char* act_pool = nullptr;
+    std::vector<float*> resid;          // 2L+1 of (BT, C) fp32
+    std::vector<float*> ln_mean, ln_rstd;  // 2L+1 of (BT)
+    std::vector<void*> ln1, ln2, qkv, att, fch, fcg;  // per layer
+    std::vector<float*> lse;            // per layer (B, H, T)
+    void* lnf = nullptr;
+    void* logits = nullptr;
+    float* dres = nullptr;
+    void* dres_act = nullptr;
+    void* dtmp = nullptr;
+    void* dO = nullptr;
+    void* dqkv = nullptr;
+    void* du = nullptr;
+    float* dpre = nullptr;
+    int* d_tokens = nullptr;
+
+    DevScalars* d_sc = nullptr;
+    DevScalars* h_sc = nullptr;   // pinned
+
+    long long step_t = 0;
+    long long launches = 0;
+    bool use_tc_gemm = true;
+    std::string host_error;   // set by enqueue helpers that cannot report a status
+
+    Ctx ctx() {
+        Ctx c;
+        c.stream = stream;
+        c.status = &d_sc->status;
+        c.launches = &launches;
+        c.num_sms = num_sms;
+        return c;
+    }
+};
+
+namespace {
+
+// ---------------------------------------------------------------- validation
+int validate_config(const gpt2_config* c) {
+    if (!c) return fail(GPT2_ERR_INVALID_ARG, "cfg is NULL");
+    if (c->n_layer < 1 || c->n_head < 1 || c->n_embd < 1 || c->vocab_size < 1 || c->block_size < 1 ||
+        c->max_B < 1 || c->max_T < 1)
+        return fail(GPT2_ERR_INVALID_ARG, "all sizes must be >= 1");
+    if (c->n_embd % c->n_head != 0) return fail(GPT2_ERR_INVALID_ARG, "n_embd must be a multiple of n_head");
+    const int hd = c->n_embd / c->n_head;
+    if (hd != 32 && hd != 64) return fail(GPT2_ERR_INVALID_ARG, "head width n_embd/n_head must be 32 or 64");
+    if (c->n_embd % 64 != 0) return fail(GPT2_ERR_INVALID_ARG, "n_embd must be a multiple of 64");
+    if (c->n_embd > 2048) return fail(GPT2_ERR_INVALID_ARG, "n_embd must be <= 2048");
+    if (c->vocab_size % 8 != 0) return fail(GPT2_ERR_INVALID_ARG, "vocab_size must be a multiple of 8 (pad it)");
+    if (c->max_T > c->block_size) return fail(GPT2_ERR_INVALID_ARG, "max_T must be <= block_size");
+    if (c->precision != GPT2_PRECISION_FP32 && c->precision != GPT2_PRECISION_BF16)
+        return fail(GPT2_ERR_INVALID_ARG, "precision must be GPT2_PRECISION_FP32 or GPT2_PRECISION_BF16");
+    if (c->flags != 0) return fail(GPT2_ERR_INVALID_ARG, "flags must be 0");
+    if ((long long)c->max_B * c->max_T > (1LL << 30)) return fail(GPT2_ERR_INVALID_ARG, "max_B*max_T too large");
+    return GPT2_OK;
+}
+
+int check_bt(const gpt2_handle* h, int B, int T) {
+    if (B < 1 || T < 1) return fail(GPT2_ERR_INVALID_ARG, "B and T must be >= 1");
+    if (B > h->cfg.max_B) return fail(GPT2_ERR_INVALID_ARG, "B exceeds max_B");
+    if (T > h->cfg.max_T) return fail(GPT2_ERR_INVALID_ARG, "T exceeds max_T");
+    if (T > h->cfg.block_size) return fail(GPT2_ERR_INVALID_ARG, "T exceeds block_size");
+    if ((long long)B * T > h->maxBT) return fail(GPT2_ERR_INVALID_ARG, "B*T exceeds max_B*max_T");
+    return GPT2_OK;
+}
+
+void build_layout(gpt2_handle* h) {
+    const long long C = h->C, V = h->V;
+    long long off = 0;
+    auto add = [&](const std::string& name, long long r, long long c) {
+        TensorRec t;
+        t.name = name;
+        t.ndim = c ? 2 : 1;
+        t.shape[0] = r;
+        t.shape[1] = c;
+        t.offset = off;
+        t.decay = c ? 1 : 0;
+        h->tensors.push_back(t);
+        long long o = off;
+        off += c ? r * c : r;
+        return o;
+    };
+    h->off_wte = add("wte", V, C);
+    h->off_wpe = add("wpe", h->cfg.block_size, C);
+    for (int l = 0; l < h->L; ++l) {
+        std::string p = "h." + std::to_string(l) + ".";
+        LayerOff o;
+        o.ln1w = add(p + "ln_1.weight", C, 0);
+        o.ln1b = add(p + "ln_1.bias", C, 0);
+        o.wqkv = add(p + "attn.c_attn.weight", 3 * C, C);
+        o.bqkv = add(p + "attn.c_attn.bias", 3 * C, 0);
+        o.wproj = add(p + "attn.c_proj.weight", C, C);
+        o.bproj = add(p + "attn.c_proj.bias", C, 0);
+        o.ln2w = add(p + "ln_2.weight", C, 0);
+        o.ln2b = add(p + "ln_2.bias", C, 0);
+        o.wfc = add(p + "mlp.c_fc.weight", 4 * C, C);
+        o.bfc = add(p + "mlp.c_fc.bias", 4 * C, 0);
+        o.wfcp = add(p + "mlp.c_proj.weight", C, 4 * C);
+        o.bfcp = add(p + "mlp.c_proj.bias", C, 0);
+        h->lo.push_back(o);
+    }
+    h->off_lnfw = add("ln_f.weight", C, 0);
+    h->off_lnfb = add("ln_f.bias", C, 0);
+    h->n_params = off;
+}
+
+std::vector<AdamChunk> build_chunks(const gpt2_handle* h) {
+    std::vector<AdamChunk> out;
+    const long long CH = 1 << 16;
+    for (const auto& t : h->tensors) {
+        const long long n = t.ndim == 2 ? t.shape[0] * t.shape[1] : t.shape[0];
+        for (long long s = 0; s < n; s += CH) {
+            AdamChunk c;
+            c.start = t.offset + s;
+            c.count = (int)std::min(CH, n - s);
+            c.decay = t.decay;
+            out.push_back(c);
+        }
+    }
+    return out;
+}
+
+size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
+
+int init_weights(gpt2_handle* h) {
+    Ctx c = h->ctx();
+    const float resid_std = 0.02f / sqrtf(2.0f * h->L);
+    for (size_t i = 0; i < h->tensors.size(); ++i) {
+        const TensorRec& t = h->tensors[i];
+        const long long n = t.ndim == 2 ? t.shape[0] * t.shape[1] : t.shape[0];
+        float* p = h->params + t.offset;
+        const bool is_ln = t.name.find("ln_") != std::string::npos;
+        const bool is_weight = t.name.size() >= 6 && t.name.compare(t.name.size() - 6, 6, "weight") == 0;
+        if (t.ndim == 2) {
+            const bool resid_proj = t.name.size() >= 13 && t.name.compare(t.name.size() - 13, 13, "c_proj.weight") == 0;
+            launch_fill_normal(c, p, n, resid_proj ? resid_std : 0.02f, h->cfg.seed, (unsigned long long)i);
+        } else if (is_ln && is_weight) {
+            launch_fill_const(c, p, n, 1.0f);
+        } else {
+            CK(cudaMemsetAsync(p, 0, n * sizeof(float), h->stream));
+        }
+    }
+    CK(cudaGetLastError());
+    return GPT2_OK;
+}
+
+int refresh_shadow(gpt2_handle* h) {
+    if (!h->bf16_mode) return GPT2_OK;
+    Ctx c = h->ctx();
+    launch_to_bf16(c, h->params, h->shadow, h->n_params);
+    CK(cudaGetLastError());
+    return GPT2_OK;
+}
+
+// ------------------------------------------------------------ GEMM dispatch
+template <typename A>
+void gemm(gpt2_handle* h, GemmLayout layout, const void* a, const void* b, int M, int N, int K, const Epilogue& ep);
+
+template <>
+void gemm<float>(gpt2_handle* h, GemmLayout layout, const void* a, const void* b, int M, int N, int K,
+                 const Epilogue& ep) {
+    launch_gemm_simt<float>(h->ctx(), layout, (const float*)a, (const float*)b, M, N, K, ep);
+}
+
+template <>
+void gemm<bf16>(gpt2_handle* h, GemmLayout layout, const void* a, const void* b, int M, int N, int K,
+                const Epilogue& ep) {
+    if (h->use_tc_gemm && gemm_tc_supported(layout, M, N, K)) {
+        if (!launch_gemm_tc(h->ctx(), layout, (const bf16*)a, (const bf16*)b, M, N, K, ep))
+            h->host_error = "tensor-map encoding failed for a tensor-core GEMM";
+    } else {
+        launch_gemm_simt<bf16>(h->ctx(), layout, (const bf16*)a, (const bf16*)b, M, N, K, ep);
+    }
+}
+
+Epilogue epi(int kind, void* out, long long ldo) {
+    Epilogue e;
+    e.kind = kind;
+    e.out = out;
+    e.ldo = ldo;
+    return e;
+}
+
+// Weight operand pointer: fp32 master (fp32 mode) or its bf16 copy (bf16 mode).
+template <typename A> const A* wop(gpt2_handle* h, long long off);
+template <> const float* wop<float>(gpt2_handle* h, long long off) { return h->params + off; }
+template <> const bf16* wop<bf16>(gpt2_handle* h, long long off) { return h->shadow + off; }
+
+// ------------------------------------------------------------------ forward
+template <typename A>
+void forward_impl(gpt2_handle* h, const int* idx, const int* targets, int B, int T, A* logits_out,
+                  double* loss_slot, float loss_scale, bool write_grad) {
+    Ctx c = h->ctx();
+    const int BT = B * T, C = h->C, V = h->V, L = h->L;
+    float* P = h->params;
+    launch_embed_ln<A>(c, idx, P + h->off_wte, P + h->off_wpe, BT, T, C, V, P + h->lo[0].ln1w, P + h->lo[0].ln1b,
+                       h->resid[0], (A*)h->ln1[0], h->ln_mean[0], h->ln_rstd[0]);
+    for (int l = 0; l < L; ++l) {
+        const LayerOff& o = h->lo[l];
+        Epilogue e = epi(EPI_BIAS, h->qkv[l], 3 * C);
+        e.bias = P + o.bqkv;
+        gemm<A>(h, GEMM_NT, h->ln1[l], wop<A>(h, o.wqkv), BT, 3 * C, C, e);
+        launch_attention_fwd_simt<A>(c, (const A*)h->qkv[l], (A*)h->att[l], h->lse[l], B, T, h->H, h->hd);
+        e = epi(EPI_BIAS_RESID, h->resid[2 * l + 1], C);
+        e.bias = P + o.bproj;
+        e.resid = h->resid[2 * l];
+        gemm<A>(h, GEMM_NT, h->att[l], wop<A>(h, o.wproj), BT, C, C, e);
+        launch_layernorm_fwd<A>(c, h->resid[2 * l + 1], P + o.ln2w, P + o.ln2b, (A*)h->ln2[l], h->ln_mean[2 * l + 1],
+                                h->ln_rstd[2 * l + 1], BT, C);
+        e = epi(EPI_BIAS_GELU, h->fcg[l], 4 * C);
+        e.out2 = h->fch[l];
+        e.bias = P + o.bfc;
+        gemm<A>(h, GEMM_NT, h->ln2[l], wop<A>(h, o.wfc), BT, 4 * C, C, e);
+        e = epi(EPI_BIAS_RESID, h->resid[2 * l + 2], C);
+        e.bias = P + o.bfcp;
+        e.resid = h->resid[2 * l + 1];
+        gemm<A>(h, GEMM_NT, h->fcg[l], wop<A>(h, o.wfcp), BT, C, 4 * C, e);
+        if (l + 1 < L)
+            launch_layernorm_fwd<A>(c, h->resid[2 * l + 2], P + h->lo[l + 1].ln1w, P + h->lo[l + 1].ln1b,
+                                    (A*)h->ln1[l + 1], h->ln_mean[2 * l + 2], h->ln_rstd[2 * l + 2], BT, C);
+    }
+    launch_layernorm_fwd<A>(c, h->resid[2 * L], P + h->off_lnfw, P + h->off_lnfb, (A*)h->lnf, h->ln_mean[2 * L],
+                            h->ln_rstd[2 * L], BT, C);
+    A* lg = logits_out ? logits_out : (A*)h->logits;
+    gemm<A>(h, GEMM_NT, h->lnf, wop<A>(h, h->off_wte), BT, V, C, epi(EPI_STORE, lg, V));
+    if (targets) {
+        launch_count_targets(c, targets, BT, V, &h->d_sc->n_valid);
+        launch_classifier<A>(c, lg, targets, BT, V, &h->d_sc->n_valid, loss_scale, loss_slot, write_grad ? 1 : 0);
+    }
+}
+
+// ----------------------------------------------------------------- backward
+template <typename A>
+void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
+    Ctx c = h->ctx();
+    const int BT = B * T, C = h->C, V = h->V, L = h->L;
+    float* P = h->params;
+    float* G = h->grads;
+    // lm_head (tied): dlnf = dlogits wte ; dwte += dlogits^T lnf
+    gemm<A>(h, GEMM_NN, h->logits, wop<A>(h, h->off_wte), BT, C, V, epi(EPI_STORE, h->dtmp, C));
+    Epilogue acc = epi(EPI_ACCUM_F32, G + h->off_wte, C);
+    acc.beta = 1.f;
+    gemm<A>(h, GEMM_TN, h->logits, h->lnf, V, C, BT, acc);
+    launch_layernorm_bwd<A>(c, (const A*)h->dtmp, h->resid[2 * L], h->ln_mean[2 * L], h->ln_rstd[2 * L],
+                            P + h->off_lnfw, nullptr, h->dres, (A*)h->dres_act, G + h->off_lnfw, G + h->off_lnfb,
+                            G + h->lo[L - 1].bfcp, BT, C);
+    for (int l = L - 1; l >= 0; --l) {
+        const LayerOff& o = h->lo[l];
+        // mlp.c_proj: dW += dY^T g ; du = (dY W) * gelu'(u)
+        acc = epi(EPI_ACCUM_F32, G + o.wfcp, 4 * C);
+        acc.beta = 1.f;
+        gemm<A>(h, GEMM_TN, h->dres_act, h->fcg[l], C, 4 * C, BT, acc);
+        Epilogue e = epi(EPI_DGELU, h->du, 4 * C);
+        e.aux = h->fch[l];
+        gemm<A>(h, GEMM_NN, h->dres_act, wop<A>(h, o.wfcp), BT, 4 * C, C, e);
+        launch_colsum<A>(c, (const A*)h->du, BT, 4 * C, G + o.bfc);
+        // mlp.c_fc: dW += du^T ln2 ; dln2 = du W
+        acc = epi(EPI_ACCUM_F32, G + o.wfc, C);
+        acc.beta = 1.f;
+        gemm<A>(h, GEMM_TN, h->du, h->ln2[l], 4 * C, C, BT, acc);
+        gemm<A>(h, GEMM_NN, h->du, wop<A>(h, o.wfc), BT, C, 4 * C, epi(EPI_STORE, h->dtmp, C));
+        // ln_2 backward + residual; colsum of the result is the attn.c_proj bias gradient
+        launch_layernorm_bwd<A>(c, (const A*)h->dtmp, h->resid[2 * l + 1], h->ln_mean[2 * l + 1],
+                                h->ln_rstd[2 * l + 1], P + o.ln2w, h->dres, h->dres, (A*)h->dres_act, G + o.ln2w,
+                                G + o.ln2b, G + o.bproj, BT, C);
+        // attn.c_proj
+        acc = epi(EPI_ACCUM_F32, G + o.wproj, C);
+        acc.beta = 1.f;
+        gemm<A>(h, GEMM_TN, h->dres_act, h->att[l], C, C, BT, acc);
+        gemm<A>(h, GEMM_NN, h->dres_act, wop<A>(h, o.wproj), BT, C, C, epi(EPI_STORE, h->dO, C));
+        // attention
+        launch_attention_bwd_simt<A>(c, (const A*)h->qkv[l], (const A*)h->att[l], (const A*)h->dO, h->lse[l],
+                                     h->dpre, (A*)h->dqkv, B, T, h->H, h->hd);
+        launch_colsum<A>(c, (const A*)h->dqkv, BT, 3 * C, G + o.bqkv);
+        // attn.c_attn
+        acc = epi(EPI_ACCUM_F32, G + o.wqkv, C);
+        acc.beta = 1.f;
+        gemm<A>(h, GEMM_TN, h->dqkv, h->ln1[l], 3 * C, C, BT, acc);
+        gemm<A>(h, GEMM_NN, h->dqkv, wop<A>(h, o.wqkv), BT, C, 3 * C, epi(EPI_STORE, h->dtmp, C));
+        // ln_1 backward + residual; colsum is the previous block's mlp.c_proj bias gradient
+        launch_layernorm_bwd<A>(c, (const A*)h->dtmp, h->resid[2 * l], h->ln_mean[2 * l], h->ln_rstd[2 * l],
+                                P + o.ln1w, h->dres, h->dres, (A*)h->dres_act, G + o.ln1w, G + o.ln1b,
+                                l > 0 ? G + h->lo[l - 1].bfcp : nullptr, BT, C);
+    }
+    launch_embed_bwd(c, idx, h->dres, B, T, C, V, G + h->off_wte, G + h->off_wpe);
+}
+
+int read_scalars(gpt2_handle* h) {
+    CK(cudaMemcpyAsync(h->h_sc, h->d_sc, sizeof(DevScalars), cudaMemcpyDeviceToHost, h->stream));
+    CK(cudaStreamSynchronize(h->stream));
+    CK(cudaGetLastError());
+    return GPT2_OK;
+}
+
+int status_error(gpt2_handle* h) {
+    const unsigned s = h->h_sc->status;
+    if (s & STATUS_TIMEOUT) return fail(GPT2_ERR_TIMEOUT, "a bounded wait inside a kernel gave up");
+    if (s & STATUS_BAD_TOKEN) return fail(GPT2_ERR_BAD_TOKEN, "token id or target out of range");
+    return GPT2_OK;
+}
+
+int pending_error(gpt2_handle* h) {
+    if (h->host_error.empty()) return GPT2_OK;
+    std::string m = h->host_error;
+    h->host_error.clear();
+    return fail(GPT2_ERR_CUDA, m);
+}
+
+int accumulate_impl(gpt2_handle* h, const int* idx, const int* targets, int B, int T, float loss_scale) {
+    if (h->bf16_mode) {
+        forward_impl<bf16>(h, idx, targets, B, T, nullptr, &h->d_sc->loss_accum, loss_scale, true);
+        backward_impl<bf16>(h, idx, B, T);
+    } else {
+        forward_impl<float>(h, idx, targets, B, T, nullptr, &h->d_sc->loss_accum, loss_scale, true);
+        backward_impl<float>(h, idx, B, T);
+    }
+    CK(cudaGetLastError());
+    return pending_error(h);
+}
+
+int zero_grad_impl(gpt2_handle* h) {
+    CK(cudaMemsetAsync(h->grads, 0, h->n_params * sizeof(float), h->stream));
+    CK(cudaMemsetAsync(&h->d_sc->loss_accum, 0, sizeof(double), h->stream));
+    return GPT2_OK;
+}
+
+int update_impl(gpt2_handle* h, float lr, float* loss_host, float* norm_host) {
+    Ctx c = h->ctx();
+    CK(cudaMemsetAsync(&h->d_sc->sumsq, 0, sizeof(double), h->stream));
+    launch_sumsq(c, h->grads, h->n_params, &h->d_sc->sumsq);
+    const long long t = h->step_t + 1;
+    const double bc1 = 1.0 - pow(0.9, (double)t), bc2 = 1.0 - pow(0.95, (double)t);
+    const float clip = h->cfg.grad_clip > 0.f ? h->cfg.grad_clip : 1.0f;
+    launch_adamw(c, h->d_chunks, h->n_chunks, h->params, h->grads, h->mom1, h->mom2,
+                 h->bf16_mode ? h->shadow : nullptr, &h->d_sc->sumsq, &h->d_sc->loss_accum, lr, clip, (float)bc1,
+                 (float)bc2, 0.1f);
+    CK(cudaGetLastError());
+    int rc = read_scalars(h);
+    if (rc) return rc;
+    const double loss = h->h_sc->loss_accum, ss = h->h_sc->sumsq;
+    if (loss_host) *loss_host = (float)loss;
+    if (norm_host) *norm_host = (float)sqrt(ss);
+    rc = status_error(h);
+    if (rc) return rc;
+    if (!std::isfinite(loss) || !std::isfinite(ss))
+        return fail(GPT2_ERR_NONFINITE, "loss or gradient norm is not finite; update skipped");
+    h->step_t = t;
+    return GPT2_OK;
+}
+
+}  // namespace
+
+// =============================================================== C ABI
+extern "C" {
+
+const char* gpt2_last_error(void) { return g_last_error.c_str(); }
+
+int gpt2_create(const gpt2_config* cfg, void* stream, gpt2_handle** out) {
+    g_last_error.clear();
+    if (!out) return fail(GPT2_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    int rc = validate_config(cfg);
+    if (rc) return rc;
+    int dev = 0;
+    CK(cudaGetDevice(&dev));
+    cudaDeviceProp prop;
+    CK(cudaGetDeviceProperties(&prop, dev));
+    if (prop.major != 10)
+        return fail(GPT2_ERR_UNSUPPORTED_ARCH, std::string("device is sm_") + std::to_string(prop.major) +
+                                                   std::to_string(prop.minor) + ", this library is built for sm_100a");
+    gpt2_handle* h = new gpt2_handle();
+    h->cfg = *cfg;
+    h->stream = (cudaStream_t)stream;
+    h->device = dev;
+    h->num_sms = prop.multiProcessorCount;
+    h->bf16_mode = cfg->precision == GPT2_PRECISION_BF16;
+    h->C = cfg->n_embd;
+    h->L = cfg->n_layer;
+    h->H = cfg->n_head;
+    h->hd = cfg->n_embd / cfg->n_head;
+    h->V = cfg->vocab_size;
+    h->maxBT = cfg->max_B * cfg->max_T;
+    if (const char* e = getenv("GPT2_B200_SIMT_GEMM")) h->use_tc_gemm = (e[0] == '0');
+    build_layout(h);
+
+    auto cleanup_fail = [&](int code, const std::string& msg) {
+        gpt2_destroy(h);
+        return fail(code, msg);
+    };
+    auto dmalloc = [&](void** p, size_t bytes) -> bool {
+        if (cudaMalloc(p, bytes) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        return true;
+    };
+    const size_t np = (size_t)h->n_params;
+    if (!dmalloc((void**)&h->params, np * 4) || !dmalloc((void**)&h->grads, np * 4) ||
+        !dmalloc((void**)&h->mom1, np * 4) || !dmalloc((void**)&h->mom2, np * 4) ||
+        (h->bf16_mode && !dmalloc((void**)&h->shadow, np * 2)))
+        return cleanup_fail(GPT2_ERR_OOM, "cudaMalloc of parameter state failed");
+    std::vector<AdamChunk> chunks = build_chunks(h);
+    h->n_chunks = (int)chunks.size();
+    if (!dmalloc((void**)&h->d_chunks, chunks.size() * sizeof(AdamChunk)))
+        return cleanup_fail(GPT2_ERR_OOM, "cudaMalloc of chunk table failed");
+    if (cudaMemcpy(h->d_chunks, chunks.data(), chunks.size() * sizeof(AdamChunk), cudaMemcpyHostToDevice) !=
+        cudaSuccess)
+        return cleanup_fail(GPT2_ERR_CUDA, "chunk table upload failed");
+
+    // activation pool
+    const size_t es = h->bf16_mode ? 2 : 4;
+    const size_t BT = (size_t)h->maxBT, C = h->C, L = h->L, V = h->V;
+    const size_t BHT = (size_t)cfg->max_B * h->H * cfg->max_T;
+    std::vector<std::pair<void**, size_t>> plan;
+    h->resid.assign(2 * L + 1, nullptr);
+    h->ln_mean.assign(2 * L + 1, nullptr);
+    h->ln_rstd.assign(2 * L + 1, nullptr);
+    h->ln1.assign(L, nullptr); h->ln2.assign(L, nullptr); h->qkv.assign(L, nullptr);
+    h->att.assign(L, nullptr); h->fch.assign(L, nullptr); h->fcg.assign(L, nullptr);
+    h->lse.assign(L, nullptr);
+    for (size_t i = 0; i < 2 * L + 1; ++i) {
+        plan.push_back({(void**)&h->resid[i], BT * C * 4});
+        plan.push_back({(void**)&h->ln_mean[i], BT * 4});
+        plan.push_back({(void**)&h->ln_rstd[i], BT * 4});
+    }
+    for (size_t l = 0; l < L; ++l) {
+        plan.push_back({&h->ln1[l], BT * C * es});
+        plan.push_back({&h->ln2[l], BT * C * es});
+        plan.push_back({&h->qkv[l], BT * 3 * C * es});
+        plan.push_back({&h->att[l], BT * C * es});
+        plan.push_back({&h->fch[l], BT * 4 * C * es});
+        plan.push_back({&h->fcg[l], BT * 4 * C * es});
+        plan.push_back({(void**)&h->lse[l], BHT * 4});
+    }
+    plan.push_back({&h->lnf, BT * C * es});
+    plan.push_back({&h->logits, BT * V * es});
+    plan.push_back({(void**)&h->dres, BT * C * 4});
+    plan.push_back({&h->dres_act, BT * C * es});
+    plan.push_back({&h->dtmp, BT * C * es});
+    plan.push_back({&h->dO, BT * C * es});
+    plan.push_back({&h->dqkv, BT * 3 * C * es});
+    plan.push_back({&h->du, BT * 4 * C * es});
+    plan.push_back({(void**)&h->dpre, BHT * 4});
+    plan.push_back({(void**)&h->d_tokens, 2 * BT * 4});
+    size_t total = 0;
+    for (auto& p : plan) total += align_up(p.second);
+    if (!dmalloc((void**)&h->act_pool, total)) return cleanup_fail(GPT2_ERR_OOM, "cudaMalloc of activations failed");
+    size_t off = 0;
+    for (auto& p : plan) {
+        *p.first = h->act_pool + off;
+        off += align_up(p.second);
+    }
+    if (!dmalloc((void**)&h->d_sc, sizeof(DevScalars))) return cleanup_fail(GPT2_ERR_OOM, "cudaMalloc failed");
+    if (cudaMallocHost((void**)&h->h_sc, sizeof(DevScalars)) != cudaSuccess)
+        return cleanup_fail(GPT2_ERR_OOM, "cudaMallocHost failed");
+    if (cudaMemsetAsync(h->d_sc, 0, sizeof(DevScalars), h->stream) != cudaSuccess ||
+        cudaMemsetAsync(h->mom1, 0, np * 4, h->stream) != cudaSuccess ||
+        cudaMemsetAsync(h->mom2, 0, np * 4, h->stream) != cudaSuccess ||
+        cudaMemsetAsync(h->grads, 0, np * 4, h->stream) != cudaSuccess)
+        return cleanup_fail(GPT2_ERR_CUDA, "initial memset failed");
+    h->launches = 0;
+    rc = init_weights(h);
+    if (!rc) rc = refresh_shadow(h);
+    if (!rc && cudaStreamSynchronize(h->stream) != cudaSuccess) rc = fail(GPT2_ERR_CUDA, "init sync failed");
+    if (rc) {
+        std::string msg = g_last_error;
+        return cleanup_fail(rc, msg);
+    }
+    *out = h;
+    return GPT2_OK;
+}
+
+void gpt2_destroy(gpt2_handle* h) {
+    if (!h) return;
+    cudaStreamSynchronize(h->stream);
+    cudaFree(h->params);
+    cudaFree(h->grads);
+    cudaFree(h->mom1);
+    cudaFree(h->mom2);
+    cudaFree(h->shadow);
+    cudaFree(h->d_chunks);
+    cudaFree(h->act_pool);
+    cudaFree(h->d_sc);
+    if (h->h_sc) cudaFreeHost(h->h_sc);
+    delete h;
+}
+
+int gpt2_set_stream(gpt2_handle* h, void* stream) {
+    if (!h) return fail(GPT2_ERR_INVALID_ARG, "handle is NULL");
+    h->stream = (cudaStream_t)stream;
+    return GPT2_OK;
+}
+
+int gpt2_num_params(const gpt2_handle* h, int64_t* n) {
+    if (!h || !n) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    *n = h->n_params;
+    return GPT2_OK;
+}
+
+int gpt2_param_layout(const gpt2_handle* h, gpt2_tensor_info* out, int capacity, int* count) {
+    if (!h || !count) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    *count = (int)h->tensors.size();
+    if (!out) return GPT2_OK;
+    if (capacity < *count) return fail(GPT2_ERR_INVALID_ARG, "capacity smaller than the tensor count");
+    for (size_t i = 0; i < h->tensors.size(); ++i) {
+        const TensorRec& t = h->tensors[i];
+        gpt2_tensor_info& o = out[i];
+        memset(&o, 0, sizeof(o));
+        strncpy(o.name, t.name.c_str(), sizeof(o.name) - 1);
+        o.ndim = t.ndim;
+        o.shape[0] = t.shape[0];
+        o.shape[1] = t.ndim == 2 ? t.shape[1] : 0;
+        o.offset = t.offset;
+        o.decay = t.decay;
+    }
+    return GPT2_OK;
+}
+
+static int copy_flat(gpt2_handle* h, void* dst, const void* src, size_t bytes, bool to_device_buf, int on_device) {
+    cudaMemcpyKind k = on_device ? cudaMemcpyDeviceToDevice
+                                 : (to_device_buf ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToHost);
+    CK(cudaMemcpyAsync(dst, src, bytes, k, h->stream));
+    CK(cudaStreamSynchronize(h->stream));
+    return GPT2_OK;
+}
+
+int gpt2_set_params(gpt2_handle* h, const float* flat, int on_device) {
+    if (!h || !flat) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    int rc = copy_flat(h, h->params, flat, h->n_params * 4, true, on_device);
+    if (rc) return rc;
+    h->launches = 0;
+    rc = refresh_shadow(h);
+    if (rc) return rc;
+    CK(cudaStreamSynchronize(h->stream));
+    return GPT2_OK;
+}
+
+int gpt2_get_params(gpt2_handle* h, float* flat, int on_device) {
+    if (!h || !flat) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    return copy_flat(h, flat, h->params, h->n_params * 4, false, on_device);
+}
+
+int gpt2_get_grads(gpt2_handle* h, float* flat, int on_device) {
+    if (!h || !flat) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    return copy_flat(h, flat, h->grads, h->n_params * 4, false, on_device);
+}
+
+int gpt2_get_opt_state(gpt2_handle* h, float* m, float* v, int64_t* step, int on_device) {
+    if (!h) return fail(GPT2_ERR_INVALID_ARG, "NULL handle");
+    int rc = GPT2_OK;
+    if (m) rc = copy_flat(h, m, h->mom1, h->n_params * 4, false, on_device);
+    if (!rc && v) rc = copy_flat(h, v, h->mom2, h->n_params * 4, false, on_device);
+    if (step) *step = h->step_t;
+    return rc;
+}
+
+int gpt2_set_opt_state(gpt2_handle* h, const float* m, const float* v, int64_t step, int on_device) {
+    if (!h || !m || !v || step < 0) return fail(GPT2_ERR_INVALID_ARG, "bad argument");
+    int rc = copy_flat(h, h->mom1, m, h->n_params * 4, true, on_device);
+    if (!rc) rc = copy_flat(h, h->mom2, v, h->n_params * 4, true, on_device);
+    if (!rc) h->step_t = step;
+    return rc;
+}
+
+int gpt2_forward(gpt2_handle* h, const int32_t* idx, const int32_t* targets, int B, int T, void* logits_dev,
+                 float* loss_host) {
+    if (!h || !idx) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    int rc = check_bt(h, B, T);
+    if (rc) return rc;
+    h->launches = 0;
+    CK(cudaMemsetAsync(&h->d_sc->fwd_loss, 0, sizeof(double), h->stream));
+    if (h->bf16_mode)
+        forward_impl<bf16>(h, idx, targets, B, T, (bf16*)logits_dev, &h->d_sc->fwd_loss, 1.f, false);
+    else
+        forward_impl<float>(h, idx, targets, B, T, (float*)logits_dev, &h->d_sc->fwd_loss, 1.f, false);
+    CK(cudaGetLastError());
+    rc = pending_error(h);
+    if (rc) return rc;
+    if (loss_host || targets) {
+        rc = read_scalars(h);
+        if (rc) return rc;
+        if (loss_host) *loss_host = (float)h->h_sc->fwd_loss;
+        return status_error(h);
+    }
+    return GPT2_OK;
+}
+
+int gpt2_zero_grad(gpt2_handle* h) {
+    if (!h) return fail(GPT2_ERR_INVALID_ARG, "NULL handle");
+    return zero_grad_impl(h);
+}
+
+int gpt2_accumulate(gpt2_handle* h, const int32_t* idx, const int32_t* targets, int B, int T, float loss_scale) {
+    if (!h || !idx || !targets) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    int rc = check_bt(h, B, T);
+    if (rc) return rc;
+    h->launches = 0;
+    return accumulate_impl(h, idx, targets, B, T, loss_scale);
+}
+
+int gpt2_update(gpt2_handle* h, float lr, float* loss_host, float* grad_norm_host) {
+    if (!h) return fail(GPT2_ERR_INVALID_ARG, "NULL handle");
+    h->launches = 0;
+    return update_impl(h, lr, loss_host, grad_norm_host);
+}
+
+int gpt2_step(gpt2_handle* h, const int32_t* idx, const int32_t* targets, int B, int T, float lr, float* loss_host,
+              float* grad_norm_host) {
+    if (!h || !idx || !targets) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    int rc = check_bt(h, B, T);
+    if (rc) return rc;
+    h->launches = 0;
+    rc = zero_grad_impl(h);
+    if (!rc) rc = accumulate_impl(h, idx, targets, B, T, 1.f);
+    if (!rc) rc = update_impl(h, lr, loss_host, grad_norm_host);
+    return rc;
+}
+
+int gpt2_step_host(gpt2_handle* h, const int32_t* idx_host, const int32_t* targets_host, int B, int T, float lr,
+                   float* loss_host, float* grad_norm_host) {
+    if (!h || !idx_host || !targets_host) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    int rc = check_bt(h, B, T);
+    if (rc) return rc;
+    const size_t n = (size_t)B * T;
+    CK(cudaMemcpyAsync(h->d_tokens, idx_host, n * 4, cudaMemcpyHostToDevice, h->stream));
+    CK(cudaMemcpyAsync(h->d_tokens + n, targets_host, n * 4, cudaMemcpyHostToDevice, h->stream));
+    h->launches = 0;
+    rc = zero_grad_impl(h);
+    if (!rc) rc = accumulate_impl(h, h->d_tokens, h->d_tokens + n, B, T, 1.f);
+    if (!rc) rc = update_impl(h, lr, loss_host, grad_norm_host);
+    return rc;
+}
+
+int gpt2_last_launch_count(const gpt2_handle* h, int64_t* n) {
+    if (!h || !n) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    *n = h->launches;
+    return GPT2_OK;
+}
+
+}  // extern "C"

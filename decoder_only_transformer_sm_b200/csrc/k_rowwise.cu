@@ -1,0 +1,407 @@
+// Memory-bound row-wise kernels: embedding (+ first LayerNorm), LayerNorm
+// forward/backward fused with the residual-gradient add and bias-gradient
+// column sums, the cross-entropy classifier, column sums and the embedding
+// backward scatter-add.
+//
+// Source definitions ("GPT-2 from Scratch"): "Embeddings: tokens and
+// positions" (x = wte[idx] + wpe[t], positions from 0); "The Block: pre-LN and
+// residuals" (nn.LayerNorm, eps 1e-5, biased variance); "Forward: logits, and
+// loss when targets are given" (F.cross_entropy with ignore_index=-1);
+// "Weight tying" (the embedding gradient lands in the same wte gradient as the
+// lm_head weight gradient).
+#include "kernels.cuh"
+
+namespace gpt2 {
+
+namespace {
+
+constexpr float LN_EPS = 1e-5f;
+
+// A row of C floats spread over one warp: lane l holds float4 chunks
+// l, l + 32, ..., i.e. columns 4*(l + 32 i) .. +3, for i < NV.
+template <int NV>
+struct RowFrag {
+    float v[NV][4];
+};
+
+template <typename T, int NV, bool EMBED>
+__global__ void __launch_bounds__(256) ln_fwd_kernel(const int* __restrict__ idx, const float* __restrict__ wte,
+                                                      const float* __restrict__ wpe, int Tn, int V,
+                                                      const float* __restrict__ x_in, const float* __restrict__ w,
+                                                      const float* __restrict__ b, float* __restrict__ x_out,
+                                                      T* __restrict__ y, float* __restrict__ mean,
+                                                      float* __restrict__ rstd, int rows, int C, unsigned* status) {
+    const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    float v[NV][4];
+    const float* src;
+    const float* src2 = nullptr;
+    if (EMBED) {
+        int tok = idx[row];
+        if (tok < 0 || tok >= V) {
+            if (lane == 0) atomicOr(status, STATUS_BAD_TOKEN);
+            tok = tok < 0 ? 0 : V - 1;
+        }
+        src = wte + (long long)tok * C;
+        src2 = wpe + (long long)(row % Tn) * C;
+    } else {
+        src = x_in + (long long)row * C;
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c = (lane + 32 * i) * 4;
+        if (c < C) {
+            load4(src + c, v[i]);
+            if (EMBED) {
+                float p[4];
+                load4(src2 + c, p);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) v[i][j] += p[j];
+                store4(x_out + (long long)row * C + c, v[i]);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) s += v[i][j];
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[i][j] = 0.f;
+        }
+    }
+    const float mu = warp_sum(s) / C;
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c = (lane + 32 * i) * 4;
+        if (c < C) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) { float d = v[i][j] - mu; ss += d * d; }
+        }
+    }
+    const float rs = rsqrtf(warp_sum(ss) / C + LN_EPS);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c = (lane + 32 * i) * 4;
+        if (c < C) {
+            float ww[4], bb[4], o[4];
+            load4(w + c, ww);
+            load4(b + c, bb);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o[j] = (v[i][j] - mu) * rs * ww[j] + bb[j];
+            store4(y + (long long)row * C + c, o);
+        }
+    }
+    if (lane == 0) { mean[row] = mu; rstd[row] = rs; }
+}
+
+template <typename T, int NV>
+__global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, const float* __restrict__ x,
+                                                      const float* __restrict__ mean, const float* __restrict__ rstd,
+                                                      const float* __restrict__ w, const float* dres_in,
+                                                      float* dres_out, T* __restrict__ dres_act,
+                                                      float* __restrict__ dw, float* __restrict__ db,
+                                                      float* __restrict__ dbias_next, int rows, int C) {
+    extern __shared__ float red[];   // [3][C]
+    for (int i = threadIdx.x; i < 3 * C; i += blockDim.x) red[i] = 0.f;
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int warps_total = (gridDim.x * blockDim.x) >> 5;
+    float adw[NV][4], adb[NV][4], adn[NV][4];
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) adw[i][j] = adb[i][j] = adn[i][j] = 0.f;
+
+    for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < rows; row += warps_total) {
+        const float mu = mean[row], rs = rstd[row];
+        float g[NV][4], xh[NV][4], dxh[NV][4];
+        float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int c = (lane + 32 * i) * 4;
+            if (c < C) {
+                float xx[4], ww[4];
+                load4(dy + (long long)row * C + c, g[i]);
+                load4(x + (long long)row * C + c, xx);
+                load4(w + c, ww);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    xh[i][j] = (xx[j] - mu) * rs;
+                    dxh[i][j] = g[i][j] * ww[j];
+                    s1 += dxh[i][j];
+                    s2 += dxh[i][j] * xh[i][j];
+                }
+            }
+        }
+        s1 = warp_sum(s1) / C;
+        s2 = warp_sum(s2) / C;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int c = (lane + 32 * i) * 4;
+            if (c < C) {
+                float o[4], r[4] = {0.f, 0.f, 0.f, 0.f};
+                if (dres_in) load4(dres_in + (long long)row * C + c, r);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    o[j] = rs * (dxh[i][j] - s1 - xh[i][j] * s2) + r[j];
+                    adw[i][j] += g[i][j] * xh[i][j];
+                    adb[i][j] += g[i][j];
+                    adn[i][j] += o[j];
+                }
+                store4(dres_out + (long long)row * C + c, o);
+                if (dres_act) store4(dres_act + (long long)row * C + c, o);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c = (lane + 32 * i) * 4;
+        if (c < C) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                atomicAdd(&red[c + j], adw[i][j]);
+                atomicAdd(&red[C + c + j], adb[i][j]);
+                atomicAdd(&red[2 * C + c + j], adn[i][j]);
+            }
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < C; i += blockDim.x) {
+        atomicAdd(&dw[i], red[i]);
+        atomicAdd(&db[i], red[C + i]);
+        if (dbias_next) atomicAdd(&dbias_next[i], red[2 * C + i]);
+    }
+}
+
+__global__ void count_targets_kernel(const int* __restrict__ t, int n, int V, int* n_valid, unsigned* status) {
+    __shared__ int cnt[32];
+    int c = 0;
+    bool bad = false;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int v = t[i];
+        c += (v != -1);
+        bad |= (v < -1 || v >= V);
+    }
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, STATUS_BAD_TOKEN);
+    if ((threadIdx.x & 31) == 0) cnt[threadIdx.x >> 5] = c;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        int v = (threadIdx.x < (blockDim.x >> 5)) ? cnt[threadIdx.x] : 0;
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (threadIdx.x == 0) *n_valid = v;
+    }
+}
+
+// One block per row. Pass 1: running max and sum of exp (online softmax) over
+// all V columns; pass 2 (write_grad): dlogits = (softmax - onehot) * scale / n_valid,
+// written in place; rows whose target is -1 get zeros.
+template <typename T>
+__global__ void __launch_bounds__(512) classifier_kernel(T* logits, const int* __restrict__ targets, int V,
+                                                          const int* __restrict__ n_valid, float scale,
+                                                          double* loss_accum, int write_grad) {
+    const long long row = blockIdx.x;
+    T* lr = logits + row * V;
+    int tgt = targets[row];
+    const bool valid = (tgt >= 0 && tgt < V);
+    float lt = 0.f;
+    if (threadIdx.x == 0 && valid) lt = to_f(lr[tgt]);
+    float m = -INFINITY, s = 0.f;
+    for (int c = threadIdx.x * 4; c < V; c += blockDim.x * 4) {
+        float v[4];
+        load4(lr + c, v);
+        float mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+        if (mx > m) { s *= expf(m - mx); m = mx; }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) s += expf(v[j] - m);
+    }
+    // block reduction of (m, s)
+    __shared__ float sm[32], ssum[32];
+    __shared__ float s_lse;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+        float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+        float mm = fmaxf(m, m2);
+        s = (m == -INFINITY ? 0.f : s * expf(m - mm)) + (m2 == -INFINITY ? 0.f : s2 * expf(m2 - mm));
+        m = mm;
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    if (lane == 0) { sm[warp] = m; ssum[warp] = s; }
+    __syncthreads();
+    if (warp == 0) {
+        m = lane < nw ? sm[lane] : -INFINITY;
+        s = lane < nw ? ssum[lane] : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+            float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+            float mm = fmaxf(m, m2);
+            s = (m == -INFINITY ? 0.f : s * expf(m - mm)) + (m2 == -INFINITY ? 0.f : s2 * expf(m2 - mm));
+            m = mm;
+        }
+        if (lane == 0) s_lse = m + logf(s);
+    }
+    __syncthreads();
+    const float lse = s_lse;
+    const int nv = *n_valid;
+    if (threadIdx.x == 0 && valid && nv > 0)
+        atomicAdd(loss_accum, (double)scale * (double)(lse - lt) / (double)nv);
+    if (!write_grad) return;
+    const float gs = (valid && nv > 0) ? scale / (float)nv : 0.f;
+    for (int c = threadIdx.x * 4; c < V; c += blockDim.x * 4) {
+        float v[4];
+        load4(lr + c, v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = (expf(v[j] - lse) - (c + j == tgt ? 1.f : 0.f)) * gs;
+        store4(lr + c, v);
+    }
+}
+
+template <typename T>
+__global__ void colsum_kernel(const T* __restrict__ in, int rows, int cols, int rows_per_block, float* out) {
+    // blockDim = (32, 8): threadIdx.x picks a column, threadIdx.y strides rows
+    __shared__ float part[8][33];
+    const int col = blockIdx.x * 32 + threadIdx.x;
+    const int r0 = blockIdx.y * rows_per_block;
+    const int r1 = min(rows, r0 + rows_per_block);
+    float s = 0.f;
+    if (col < cols)
+        for (int r = r0 + threadIdx.y; r < r1; r += 8) s += to_f(in[(long long)r * cols + col]);
+    part[threadIdx.y][threadIdx.x] = s;
+    __syncthreads();
+    if (threadIdx.y == 0 && col < cols) {
+        float t = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) t += part[i][threadIdx.x];
+        atomicAdd(&out[col], t);
+    }
+}
+
+__global__ void embed_bwd_wte_kernel(const int* __restrict__ idx, const float* __restrict__ dx, int rows, int C,
+                                     int V, float* dwte) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // float4 index
+    const long long per_row = C / 4;
+    if (i >= (long long)rows * per_row) return;
+    const long long row = i / per_row;
+    const int c = (int)(i % per_row) * 4;
+    int tok = idx[row];
+    tok = tok < 0 ? 0 : (tok >= V ? V - 1 : tok);
+    float v[4];
+    load4(dx + row * C + c, v);
+    float* d = dwte + (long long)tok * C + c;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) atomicAdd(d + j, v[j]);
+}
+
+__global__ void embed_bwd_wpe_kernel(const float* __restrict__ dx, int B, int Tn, int C, float* dwpe) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (long long)Tn * C) return;
+    float s = 0.f;
+    for (int b = 0; b < B; ++b) s += dx[(long long)b * Tn * C + i];
+    dwpe[i] += s;
+}
+
+template <typename T, bool EMBED>
+void ln_fwd_dispatch(const Ctx& ctx, const int* idx, const float* wte, const float* wpe, int Tn, int V,
+                     const float* x_in, const float* w, const float* b, float* x_out, T* y, float* mean,
+                     float* rstd, int rows, int C) {
+    const int threads = 256;
+    const int blocks = ceil_div(rows, threads / 32);
+    const int nv = ceil_div(C, 128);
+#define LNF_CASE(N)                                                                                 \
+    case N:                                                                                         \
+        ln_fwd_kernel<T, N, EMBED><<<blocks, threads, 0, ctx.stream>>>(idx, wte, wpe, Tn, V, x_in, w, b, \
+                                                                       x_out, y, mean, rstd, rows, C,  \
+                                                                       ctx.status);                  \
+        break;
+    switch (nv) {
+        LNF_CASE(1) LNF_CASE(2) LNF_CASE(3) LNF_CASE(4) LNF_CASE(5) LNF_CASE(6) LNF_CASE(7)
+        LNF_CASE(8) LNF_CASE(9) LNF_CASE(10) LNF_CASE(11) LNF_CASE(12) LNF_CASE(13) LNF_CASE(14)
+        LNF_CASE(15) LNF_CASE(16)
+        default: break;
+    }
+#undef LNF_CASE
+    ++*ctx.launches;
+}
+
+}  // namespace
+
+template <typename T>
+void launch_embed_ln(const Ctx& ctx, const int* idx, const float* wte, const float* wpe, int rows, int Tn, int C,
+                     int V, const float* w, const float* b, float* x, T* y, float* mean, float* rstd) {
+    ln_fwd_dispatch<T, true>(ctx, idx, wte, wpe, Tn, V, nullptr, w, b, x, y, mean, rstd, rows, C);
+}
+
+template <typename T>
+void launch_layernorm_fwd(const Ctx& ctx, const float* x, const float* w, const float* b, T* y, float* mean,
+                          float* rstd, int rows, int C) {
+    ln_fwd_dispatch<T, false>(ctx, nullptr, nullptr, nullptr, 1, 1, x, w, b, nullptr, y, mean, rstd, rows, C);
+}
+
+template <typename T>
+void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const float* mean, const float* rstd,
+                          const float* w, const float* dres_in, float* dres_out, T* dres_act, float* dw,
+                          float* db, float* dbias_next, int rows, int C) {
+    const int threads = 256;
+    const int blocks = min(ceil_div(rows, threads / 32), ctx.num_sms * 4);
+    const size_t smem = 3 * C * sizeof(float);
+    const int nv = ceil_div(C, 128);
+#define LNB_CASE(N)                                                                                      \
+    case N:                                                                                              \
+        ln_bwd_kernel<T, N><<<blocks, threads, smem, ctx.stream>>>(dy, x, mean, rstd, w, dres_in, dres_out, \
+                                                                   dres_act, dw, db, dbias_next, rows, C); \
+        break;
+    switch (nv) {
+        LNB_CASE(1) LNB_CASE(2) LNB_CASE(3) LNB_CASE(4) LNB_CASE(5) LNB_CASE(6) LNB_CASE(7)
+        LNB_CASE(8) LNB_CASE(9) LNB_CASE(10) LNB_CASE(11) LNB_CASE(12) LNB_CASE(13) LNB_CASE(14)
+        LNB_CASE(15) LNB_CASE(16)
+        default: break;
+    }
+#undef LNB_CASE
+    ++*ctx.launches;
+}
+
+void launch_count_targets(const Ctx& ctx, const int* targets, int n, int V, int* n_valid) {
+    count_targets_kernel<<<1, 1024, 0, ctx.stream>>>(targets, n, V, n_valid, ctx.status);
+    ++*ctx.launches;
+}
+
+template <typename T>
+void launch_classifier(const Ctx& ctx, T* logits, const int* targets, int rows, int V, const int* n_valid,
+                       float scale, double* loss_accum, int write_grad) {
+    classifier_kernel<T><<<rows, 512, 0, ctx.stream>>>(logits, targets, V, n_valid, scale, loss_accum, write_grad);
+    ++*ctx.launches;
+}
+
+template <typename T>
+void launch_colsum(const Ctx& ctx, const T* in, int rows, int cols, float* out) {
+    const int rpb = 256;
+    dim3 grid(ceil_div(cols, 32), ceil_div(rows, rpb));
+    colsum_kernel<T><<<grid, dim3(32, 8), 0, ctx.stream>>>(in, rows, cols, rpb, out);
+    ++*ctx.launches;
+}
+
+void launch_embed_bwd(const Ctx& ctx, const int* idx, const float* dx, int B, int Tn, int C, int V, float* dwte,
+                      float* dwpe) {
+    const long long n4 = (long long)B * Tn * (C / 4);
+    embed_bwd_wte_kernel<<<(unsigned)ceil_div_ll(n4, 256), 256, 0, ctx.stream>>>(idx, dx, B * Tn, C, V, dwte);
+    embed_bwd_wpe_kernel<<<(unsigned)ceil_div_ll((long long)Tn * C, 256), 256, 0, ctx.stream>>>(dx, B, Tn, C, dwpe);
+    *ctx.launches += 2;
+}
+
+#define INST(T)                                                                                                 \
+    template void launch_embed_ln<T>(const Ctx&, const int*, const float*, const float*, int, int, int, int,   \
+                                     const float*, const float*, float*, T*, float*, float*);                  \
+    template void launch_layernorm_fwd<T>(const Ctx&, const float*, const float*, const float*, T*, float*,    \
+                                          float*, int, int);                                                   \
+    template void launch_layernorm_bwd<T>(const Ctx&, const T*, const float*, const float*, const float*,      \
+                                          const float*, const float*, float*, T*, float*, float*, float*, int, \
+                                          int);                                                                \
+    template void launch_classifier<T>(const Ctx&, T*, const int*, int, int, const int*, float, double*, int); \
+    template void launch_colsum<T>(const Ctx&, const T*, int, int, float*);
+INST(float)
+INST(bf16)
+#undef INST
+
+}  // namespace gpt2

@@ -1,0 +1,54 @@
+// Kernel-level C ABI (gpt2_kernels.h): single operations on caller-owned
+// device buffers.
+#include <string>
+
+#include "gpt2_kernels.h"
+#include "kernels.cuh"
+
+using namespace gpt2;
+
+namespace gpt2 {
+int set_error(int code, const char* msg);   // defined in gpt2_api.cu
+}
+
+extern "C" int gpt2k_matmul_bf16(int layout, const void* A, const void* B, int M, int N, int K, int epilogue,
+                                 void* out, int64_t ldo, void* out2, const float* bias, const float* resid,
+                                 const void* aux, float beta, int engine, uint32_t* status_dev, void* stream) {
+    if (layout < GPT2K_NT || layout > GPT2K_TN) return set_error(GPT2_ERR_INVALID_ARG, "unknown layout");
+    if (epilogue < GPT2K_EPI_STORE || epilogue > GPT2K_EPI_ACCUM_F32)
+        return set_error(GPT2_ERR_INVALID_ARG, "unknown epilogue");
+    if (M < 1 || N < 1 || K < 1 || ldo < N) return set_error(GPT2_ERR_INVALID_ARG, "bad sizes");
+    if (!A || !B || !out || !status_dev) return set_error(GPT2_ERR_INVALID_ARG, "NULL operand");
+    const bool needs_bias = epilogue == GPT2K_EPI_BIAS || epilogue == GPT2K_EPI_BIAS_GELU ||
+                            epilogue == GPT2K_EPI_BIAS_RESID;
+    if ((needs_bias && !bias) || (epilogue == GPT2K_EPI_BIAS_GELU && !out2) ||
+        (epilogue == GPT2K_EPI_BIAS_RESID && !resid) || (epilogue == GPT2K_EPI_DGELU && !aux))
+        return set_error(GPT2_ERR_INVALID_ARG, "epilogue operand missing");
+    long long launches = 0;
+    Ctx c;
+    c.stream = (cudaStream_t)stream;
+    c.status = status_dev;
+    c.launches = &launches;
+    c.num_sms = 148;
+    Epilogue e;
+    e.kind = epilogue;
+    e.out = out;
+    e.ldo = ldo;
+    e.out2 = out2;
+    e.bias = bias;
+    e.resid = resid;
+    e.aux = aux;
+    e.beta = beta;
+    const GemmLayout L = (GemmLayout)layout;
+    if (engine == 1) {
+        if (!gemm_tc_supported(L, M, N, K))
+            return set_error(GPT2_ERR_INVALID_ARG, "shape not supported by the tensor-core GEMM");
+        if (!launch_gemm_tc(c, L, (const bf16*)A, (const bf16*)B, M, N, K, e))
+            return set_error(GPT2_ERR_CUDA, "tensor-map encoding failed");
+    } else {
+        launch_gemm_simt<bf16>(c, L, (const bf16*)A, (const bf16*)B, M, N, K, e);
+    }
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return set_error(GPT2_ERR_CUDA, cudaGetErrorString(err));
+    return GPT2_OK;
+}

@@ -1,0 +1,118 @@
+// Launchers of every kernel of the training step (internal C++ interface).
+// Each launcher enqueues on ctx.stream and counts its launches in *ctx.launches.
+#pragma once
+
+#include "common.cuh"
+
+namespace gpt2 {
+
+struct Ctx {
+    cudaStream_t stream;
+    unsigned* status;      // device status word (STATUS_* bits)
+    long long* launches;   // host counter of kernel launches
+    int num_sms;
+};
+
+// ----------------------------------------------------------------------------
+// GEMM epilogues. The contraction produces fp32 acc(row, col); the epilogue
+// turns it into the stored result.
+// ----------------------------------------------------------------------------
+enum EpiKind {
+    EPI_STORE = 0,       // out[act]  = acc
+    EPI_BIAS = 1,        // out[act]  = acc + bias[col]
+    EPI_BIAS_GELU = 2,   // out2[act] = u = acc + bias[col];  out[act] = gelu(u)
+    EPI_BIAS_RESID = 3,  // out[f32]  = resid[f32] + acc + bias[col]
+    EPI_DGELU = 4,       // out[act]  = acc * gelu'(aux[act])
+    EPI_ACCUM_F32 = 5,   // out[f32]  = beta * out + acc
+};
+
+struct Epilogue {
+    int kind = EPI_STORE;
+    void* out = nullptr;
+    long long ldo = 0;
+    void* out2 = nullptr;          // EPI_BIAS_GELU pre-activation output (ld = ldo)
+    const float* bias = nullptr;
+    const float* resid = nullptr;  // EPI_BIAS_RESID input (ld = ldo)
+    const void* aux = nullptr;     // EPI_DGELU pre-activation input (ld = ldo)
+    float beta = 0.f;
+};
+
+// Operand layouts of C[M,N] = sum_k A(m,k) B(n,k):
+//   GEMM_NT: A row-major [M,K], B row-major [N,K]   (forward: y = x W^T)
+//   GEMM_NN: A row-major [M,K], B row-major [K,N]   (dgrad:  dx = dy W)
+//   GEMM_TN: A row-major [K,M], B row-major [K,N]   (wgrad:  dW = dy^T x)
+enum GemmLayout { GEMM_NT = 0, GEMM_NN = 1, GEMM_TN = 2 };
+
+// SIMT fp32-accumulating GEMM (any layout, any size). T = float or bf16 operands.
+template <typename T>
+void launch_gemm_simt(const Ctx& ctx, GemmLayout layout, const T* A, const T* B, int M, int N, int K,
+                      const Epilogue& ep);
+
+// Tensor-core GEMM (tcgen05 + TMEM + TMA), bf16 operands, fp32 accumulation.
+// gemm_tc_supported: shape/layout constraints (16-byte row strides).
+// launch_gemm_tc returns false if a tensor map could not be encoded (nothing
+// is launched; the runtime reports it as an error).
+bool gemm_tc_supported(GemmLayout layout, int M, int N, int K);
+bool launch_gemm_tc(const Ctx& ctx, GemmLayout layout, const bf16* A, const bf16* B, int M, int N, int K,
+                    const Epilogue& ep);
+
+// ----------------------------------------------------------------------------
+// Row-wise kernels.
+// ----------------------------------------------------------------------------
+// x[r] = wte[idx[r]] + wpe[r % T]; then y = LN(x) with (w, b); mean/rstd saved.
+template <typename T>
+void launch_embed_ln(const Ctx& ctx, const int* idx, const float* wte, const float* wpe, int rows, int Tn, int C,
+                     int V, const float* w, const float* b, float* x, T* y, float* mean, float* rstd);
+template <typename T>
+void launch_layernorm_fwd(const Ctx& ctx, const float* x, const float* w, const float* b, T* y, float* mean,
+                          float* rstd, int rows, int C);
+// dx = LN'(x)^T dy (+ dres_in); writes dres_out (fp32) and dres_act (operand copy);
+// accumulates dw += sum dy*xhat, db += sum dy and, if dbias_next != null,
+// dbias_next += sum_rows dres_out.
+template <typename T>
+void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const float* mean, const float* rstd,
+                          const float* w, const float* dres_in, float* dres_out, T* dres_act, float* dw,
+                          float* db, float* dbias_next, int rows, int C);
+
+// Count targets != -1 (and flag out-of-range targets) into *n_valid.
+void launch_count_targets(const Ctx& ctx, const int* targets, int n, int V, int* n_valid);
+// Cross-entropy over each row of logits (in place -> dlogits * scale / n_valid);
+// loss_accum (double) += scale * sum(lse - logit[target]) / n_valid.
+template <typename T>
+void launch_classifier(const Ctx& ctx, T* logits, const int* targets, int rows, int V, const int* n_valid,
+                       float scale, double* loss_accum, int write_grad);
+// Column sums: out[c] += sum_r in[r, c].
+template <typename T>
+void launch_colsum(const Ctx& ctx, const T* in, int rows, int cols, float* out);
+// dwte[idx[r]] += dx[r]; dwpe[t] += sum_b dx[b, t].
+void launch_embed_bwd(const Ctx& ctx, const int* idx, const float* dx, int B, int Tn, int C, int V, float* dwte,
+                      float* dwpe);
+
+// ----------------------------------------------------------------------------
+// Attention (causal, per (b, h); q/k/v are column blocks of the qkv rows).
+// ----------------------------------------------------------------------------
+template <typename T>
+void launch_attention_fwd_simt(const Ctx& ctx, const T* qkv, T* out, float* lse, int B, int Tn, int H, int hd);
+template <typename T>
+void launch_attention_bwd_simt(const Ctx& ctx, const T* qkv, const T* out, const T* dout, const float* lse,
+                               float* dpre /* (B,H,T) scratch */, T* dqkv, int B, int Tn, int H, int hd);
+
+// ----------------------------------------------------------------------------
+// Optimiser and parameter utilities.
+// ----------------------------------------------------------------------------
+struct AdamChunk {        // a run of elements inside one tensor
+    long long start;
+    int count;
+    int decay;
+};
+void launch_sumsq(const Ctx& ctx, const float* g, long long n, double* out);
+void launch_adamw(const Ctx& ctx, const AdamChunk* chunks, int n_chunks, float* p, const float* g, float* m,
+                  float* v, bf16* shadow, const double* sumsq, const double* loss_accum, float lr, float clip,
+                  float bc1, float bc2, float wd);
+void launch_to_bf16(const Ctx& ctx, const float* in, bf16* out, long long n);
+// Normal(0, std) fill from a counter-based generator (Philox4x32-10) keyed by seed.
+void launch_fill_normal(const Ctx& ctx, float* p, long long n, float std, unsigned long long seed,
+                        unsigned long long stream_id);
+void launch_fill_const(const Ctx& ctx, float* p, long long n, float value);
+
+}  // namespace gpt2

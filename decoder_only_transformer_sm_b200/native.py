@@ -1,0 +1,240 @@
+"""ctypes binding of libgpt2_b200.so (include/gpt2.h): argument marshalling only.
+
+Every step of the training step runs in the library's CUDA kernels; this module
+only converts Python/torch/numpy arguments into the C ABI's pointers and sizes.
+If the library is missing the calls raise: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgpt2_b200.so")
+
+GPT2_OK = 0
+ERRORS = {
+    -1: "INVALID_ARG", -2: "OOM", -3: "CUDA", -4: "UNSUPPORTED_ARCH",
+    -5: "NONFINITE", -6: "BAD_TOKEN", -7: "TIMEOUT",
+}
+PRECISION = {"fp32": 0, "bf16": 1}
+
+
+class Gpt2Error(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"GPT2_ERR_{ERRORS.get(code, code)} ({code}): {msg}")
+        self.code = code
+
+
+class Config(ctypes.Structure):
+    _fields_ = [
+        ("n_layer", ctypes.c_int32), ("n_head", ctypes.c_int32), ("n_embd", ctypes.c_int32),
+        ("vocab_size", ctypes.c_int32), ("block_size", ctypes.c_int32),
+        ("max_B", ctypes.c_int32), ("max_T", ctypes.c_int32), ("precision", ctypes.c_int32),
+        ("seed", ctypes.c_uint64), ("grad_clip", ctypes.c_float), ("flags", ctypes.c_uint32),
+    ]
+
+
+class TensorInfo(ctypes.Structure):
+    _fields_ = [
+        ("name", ctypes.c_char * 48), ("ndim", ctypes.c_int32), ("shape", ctypes.c_int64 * 2),
+        ("offset", ctypes.c_int64), ("decay", ctypes.c_int32),
+    ]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library once; raise if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} not found: build it with `python -m decoder_only_transformer_sm_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    sig = {
+        "gpt2_last_error": (ctypes.c_char_p, []),
+        "gpt2_create": (I, [ctypes.POINTER(Config), P, ctypes.POINTER(P)]),
+        "gpt2_destroy": (None, [P]),
+        "gpt2_set_stream": (I, [P, P]),
+        "gpt2_num_params": (I, [P, ctypes.POINTER(ctypes.c_int64)]),
+        "gpt2_param_layout": (I, [P, P, I, ctypes.POINTER(I)]),
+        "gpt2_set_params": (I, [P, P, I]),
+        "gpt2_get_params": (I, [P, P, I]),
+        "gpt2_get_grads": (I, [P, P, I]),
+        "gpt2_get_opt_state": (I, [P, P, P, ctypes.POINTER(ctypes.c_int64), I]),
+        "gpt2_set_opt_state": (I, [P, P, P, ctypes.c_int64, I]),
+        "gpt2_forward": (I, [P, P, P, I, I, P, ctypes.POINTER(F)]),
+        "gpt2_zero_grad": (I, [P]),
+        "gpt2_accumulate": (I, [P, P, P, I, I, F]),
+        "gpt2_update": (I, [P, F, ctypes.POINTER(F), ctypes.POINTER(F)]),
+        "gpt2_step": (I, [P, P, P, I, I, F, ctypes.POINTER(F), ctypes.POINTER(F)]),
+        "gpt2_step_host": (I, [P, P, P, I, I, F, ctypes.POINTER(F), ctypes.POINTER(F)]),
+        "gpt2_last_launch_count": (I, [P, ctypes.POINTER(ctypes.c_int64)]),
+        "gpt2k_matmul_bf16": (I, [I, P, P, I, I, I, I, P, ctypes.c_int64, P, P, P, P, F, I, P, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(rc: int):
+    if rc != GPT2_OK:
+        raise Gpt2Error(rc, load_library().gpt2_last_error().decode())
+
+
+def _ptr(x) -> int | None:
+    """Raw address of a torch tensor or numpy array (None passes NULL)."""
+    if x is None:
+        return None
+    if isinstance(x, np.ndarray):
+        assert x.flags["C_CONTIGUOUS"]
+        return x.ctypes.data
+    assert x.is_contiguous()
+    return x.data_ptr()
+
+
+class GPT2:
+    """One model on the current CUDA device, created through gpt2_create."""
+
+    def __init__(self, n_layer: int, n_head: int, n_embd: int, vocab_size: int, block_size: int,
+                 max_B: int, max_T: int, precision: str = "bf16", seed: int = 0, grad_clip: float = 1.0,
+                 stream=None):
+        lib = load_library()
+        self._lib = lib
+        cfg = Config(n_layer, n_head, n_embd, vocab_size, block_size, max_B, max_T,
+                     PRECISION[precision], seed, grad_clip, 0)
+        h = ctypes.c_void_p()
+        _check(lib.gpt2_create(ctypes.byref(cfg), stream, ctypes.byref(h)))
+        self._h = h
+        self.cfg = cfg
+        self.precision = precision
+        n = ctypes.c_int64()
+        _check(lib.gpt2_num_params(h, ctypes.byref(n)))
+        self.n_params = n.value
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.gpt2_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def set_stream(self, stream_ptr):
+        _check(self._lib.gpt2_set_stream(self._h, stream_ptr))
+
+    def layout(self):
+        cnt = ctypes.c_int()
+        _check(self._lib.gpt2_param_layout(self._h, None, 0, ctypes.byref(cnt)))
+        arr = (TensorInfo * cnt.value)()
+        _check(self._lib.gpt2_param_layout(self._h, arr, cnt.value, ctypes.byref(cnt)))
+        out = []
+        for t in arr:
+            shape = tuple(int(t.shape[i]) for i in range(t.ndim))
+            out.append((t.name.decode(), shape, int(t.offset), bool(t.decay)))
+        return out
+
+    # ---- flat state (host numpy float32 or device torch float32) ----
+    def set_params(self, flat):
+        on_dev = 0 if isinstance(flat, np.ndarray) else 1
+        if on_dev == 0:
+            flat = np.ascontiguousarray(flat, dtype=np.float32)
+        assert flat.size == self.n_params if on_dev == 0 else flat.numel() == self.n_params
+        _check(self._lib.gpt2_set_params(self._h, _ptr(flat), on_dev))
+
+    def get_params(self) -> np.ndarray:
+        out = np.empty(self.n_params, np.float32)
+        _check(self._lib.gpt2_get_params(self._h, _ptr(out), 0))
+        return out
+
+    def get_grads(self) -> np.ndarray:
+        out = np.empty(self.n_params, np.float32)
+        _check(self._lib.gpt2_get_grads(self._h, _ptr(out), 0))
+        return out
+
+    def get_opt_state(self):
+        m = np.empty(self.n_params, np.float32)
+        v = np.empty(self.n_params, np.float32)
+        t = ctypes.c_int64()
+        _check(self._lib.gpt2_get_opt_state(self._h, _ptr(m), _ptr(v), ctypes.byref(t), 0))
+        return m, v, t.value
+
+    def set_opt_state(self, m, v, step: int):
+        m = np.ascontiguousarray(m, np.float32)
+        v = np.ascontiguousarray(v, np.float32)
+        _check(self._lib.gpt2_set_opt_state(self._h, _ptr(m), _ptr(v), step, 0))
+
+    # ---- compute (device int32 token tensors) ----
+    def forward(self, idx, targets=None, logits=None):
+        B, T = idx.shape
+        loss = ctypes.c_float()
+        _check(self._lib.gpt2_forward(self._h, _ptr(idx), _ptr(targets), B, T, _ptr(logits),
+                                      ctypes.byref(loss) if targets is not None else None))
+        return loss.value if targets is not None else None
+
+    def zero_grad(self):
+        _check(self._lib.gpt2_zero_grad(self._h))
+
+    def accumulate(self, idx, targets, loss_scale: float):
+        B, T = idx.shape
+        _check(self._lib.gpt2_accumulate(self._h, _ptr(idx), _ptr(targets), B, T, loss_scale))
+
+    def update(self, lr: float):
+        loss, norm = ctypes.c_float(), ctypes.c_float()
+        _check(self._lib.gpt2_update(self._h, lr, ctypes.byref(loss), ctypes.byref(norm)))
+        return loss.value, norm.value
+
+    def step(self, idx, targets, lr: float):
+        B, T = idx.shape
+        loss, norm = ctypes.c_float(), ctypes.c_float()
+        _check(self._lib.gpt2_step(self._h, _ptr(idx), _ptr(targets), B, T, lr,
+                                   ctypes.byref(loss), ctypes.byref(norm)))
+        return loss.value, norm.value
+
+    def step_host(self, idx, targets, lr: float):
+        """idx/targets: host int32 arrays or pinned CPU torch tensors."""
+        B, T = idx.shape
+        loss, norm = ctypes.c_float(), ctypes.c_float()
+        _check(self._lib.gpt2_step_host(self._h, _ptr(idx), _ptr(targets), B, T, lr,
+                                        ctypes.byref(loss), ctypes.byref(norm)))
+        return loss.value, norm.value
+
+    def last_launch_count(self) -> int:
+        n = ctypes.c_int64()
+        _check(self._lib.gpt2_last_launch_count(self._h, ctypes.byref(n)))
+        return n.value
+
+
+# ---------------------------------------------------------------------------
+# Kernel-level entry points (include/gpt2_kernels.h).
+# ---------------------------------------------------------------------------
+LAYOUT = {"NT": 0, "NN": 1, "TN": 2}
+EPILOGUE = {"store": 0, "bias": 1, "bias_gelu": 2, "bias_resid": 3, "dgelu": 4, "accum_f32": 5}
+
+
+def matmul_bf16(layout: str, A, B, M: int, N: int, K: int, epilogue: str, out, ldo: int | None = None,
+                out2=None, bias=None, resid=None, aux=None, beta: float = 0.0, engine: str = "tc",
+                status=None, stream=None):
+    """gpt2k_matmul_bf16 on torch device tensors; returns the device status tensor."""
+    import torch
+    lib = load_library()
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=out.device)
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    rc = lib.gpt2k_matmul_bf16(LAYOUT[layout], _ptr(A), _ptr(B), M, N, K, EPILOGUE[epilogue], _ptr(out),
+                               ldo if ldo is not None else N, _ptr(out2), _ptr(bias), _ptr(resid), _ptr(aux),
+                               beta, 1 if engine == "tc" else 0, _ptr(status), stream)
+    _check(rc)
+    return status

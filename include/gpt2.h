@@ -1,0 +1,179 @@
+/*
+ * gpt2.h -- C ABI of the B200 GPT-2 training-step library (libgpt2_b200.so).
+ *
+ * One handle owns one GPT-2 model on one CUDA device: fp32 master weights,
+ * fp32 gradients, fp32 AdamW moments, a bf16 copy of the weights (bf16 mode),
+ * every saved activation and all workspace. All memory is allocated in
+ * gpt2_create and released in gpt2_destroy; no other call allocates.
+ *
+ * What a step computes (page title, section of the source pages):
+ *   forward      "GPT-2 from Scratch": "Embeddings: tokens and positions",
+ *                "CausalSelfAttention", "The MLP and GPT-2's GELU",
+ *                "The Block: pre-LN and residuals", "The full model"
+ *                (tied lm_head: "Weight tying").
+ *   loss         "Forward: logits, and loss when targets are given":
+ *                mean cross-entropy over the targets that are not -1
+ *                ("Pretraining and fine-tuning nanoGPT-124M from scratch",
+ *                "Supervised fine-tuning": -1 targets are skipped).
+ *   backward     the exact gradient of that loss.
+ *   update       "Gradient clipping" (global L2 norm, clip at grad_clip) and
+ *                "AdamW, and weight decay on matrices only" (betas 0.9/0.95,
+ *                eps 1e-8, decay 0.1 on 2-D tensors only, lr-scaled decoupled
+ *                decay, bias correction of both moments).
+ *   accumulation "How to scale up" and "Let's reproduce GPT-2 (124M)",
+ *                "Gradient accumulation, and the bug in getting it right":
+ *                each micro-batch's mean loss is multiplied by loss_scale
+ *                (1/n_micro) before its gradient is added.
+ *
+ * Conventions
+ *   * Every function returns GPT2_OK (0) or a negative GPT2_ERR_* code;
+ *     gpt2_last_error() gives a message for the calling thread's last error.
+ *   * Pointers named *_dev are CUDA device pointers owned by the caller,
+ *     read or written in order on the handle's stream. Pointers named *_host
+ *     are host memory (pinned or pageable) owned by the caller.
+ *   * Token ids and targets are int32, row-major (B, T). A target of -1 is
+ *     ignored by the loss. Ids must lie in [0, vocab_size); targets in
+ *     {-1} U [0, vocab_size). An out-of-range id is clamped on the device and
+ *     reported as GPT2_ERR_BAD_TOKEN by the next synchronising call.
+ *   * One handle is used from one thread at a time; handles are independent.
+ */
+#ifndef GPT2_B200_H
+#define GPT2_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define GPT2_OK                    0
+#define GPT2_ERR_INVALID_ARG      -1  /* bad size, null pointer, T > block_size, ... */
+#define GPT2_ERR_OOM              -2  /* cudaMalloc failed in gpt2_create            */
+#define GPT2_ERR_CUDA             -3  /* a CUDA runtime call or kernel launch failed  */
+#define GPT2_ERR_UNSUPPORTED_ARCH -4  /* the current device is not sm_100             */
+#define GPT2_ERR_NONFINITE        -5  /* loss or gradient norm not finite; the update
+                                         was skipped (parameters, moments and the step
+                                         counter are unchanged)                         */
+#define GPT2_ERR_BAD_TOKEN        -6  /* an id or target outside its range was seen   */
+#define GPT2_ERR_TIMEOUT          -7  /* a bounded wait inside a kernel gave up        */
+
+/* Arithmetic modes. */
+#define GPT2_PRECISION_FP32 0  /* fp32 everywhere, fp32 FMA matmuls (no TF32)        */
+#define GPT2_PRECISION_BF16 1  /* bf16 matmul/attention operands, fp32 accumulation,
+                                  fp32 residual stream, LayerNorm, softmax, loss,
+                                  gradients, master weights and AdamW state          */
+
+typedef struct gpt2_config {
+    int32_t n_layer;     /* number of blocks                                         */
+    int32_t n_head;      /* heads; head width n_embd / n_head must be 32 or 64        */
+    int32_t n_embd;      /* residual width C; a multiple of 64                        */
+    int32_t vocab_size;  /* rows of wte = columns of the logits (padded, e.g. 50304)  */
+    int32_t block_size;  /* rows of wpe = largest T                                   */
+    int32_t max_B;       /* largest batch passed to forward/accumulate/step           */
+    int32_t max_T;       /* largest sequence length (<= block_size)                   */
+    int32_t precision;   /* GPT2_PRECISION_FP32 or GPT2_PRECISION_BF16                */
+    uint64_t seed;       /* seed of the on-device initialisation                      */
+    float grad_clip;     /* clip threshold of the global gradient norm; <= 0 means 1.0 */
+    uint32_t flags;      /* reserved, must be 0                                       */
+} gpt2_config;
+
+typedef struct gpt2_tensor_info {
+    char name[48];       /* e.g. "wte", "h.3.attn.c_attn.weight", "ln_f.bias"         */
+    int32_t ndim;        /* 1 or 2                                                    */
+    int64_t shape[2];    /* (out, in) for Linear weights, (rows, C) for embeddings    */
+    int64_t offset;      /* element offset in the flat parameter vector               */
+    int32_t decay;       /* 1 if AdamW applies weight decay to this tensor (ndim 2)    */
+} gpt2_tensor_info;
+
+typedef struct gpt2_handle gpt2_handle;
+
+/* Message of the calling thread's last error ("" if none). Never NULL. */
+const char* gpt2_last_error(void);
+
+/* Create a model on the current CUDA device.
+ * cfg     : sizes and mode (see gpt2_config). Copied; the caller keeps ownership.
+ * stream  : cudaStream_t every later call is ordered on (NULL = legacy default).
+ * out     : receives the handle.
+ * Weights are initialised on the device ("GPT-2 from Scratch", "Initialization:
+ * 0.02, and the residual scaling"): N(0, 0.02) for wte, wpe and the Linear
+ * weights, N(0, 0.02/sqrt(2 n_layer)) for both c_proj weights, zero biases,
+ * LayerNorm weight 1, bias 0. AdamW moments and the step counter start at 0.
+ * Errors: INVALID_ARG (sizes), UNSUPPORTED_ARCH, OOM, CUDA. */
+int gpt2_create(const gpt2_config* cfg, void* stream, gpt2_handle** out);
+
+/* Release every resource of the handle (synchronises its stream). NULL is a no-op. */
+void gpt2_destroy(gpt2_handle* h);
+
+/* Change the stream later calls are ordered on. */
+int gpt2_set_stream(gpt2_handle* h, void* stream);
+
+/* Number of parameters with the tied wte/lm_head counted once
+ * ("Counting parameters: 124,439,808" at vocab 50257, 12 layers, width 768). */
+int gpt2_num_params(const gpt2_handle* h, int64_t* n);
+
+/* Ordered parameter list of the flat vector used by the get/set calls:
+ * wte, wpe, h.{l}.{ln_1.weight, ln_1.bias, attn.c_attn.weight, attn.c_attn.bias,
+ * attn.c_proj.weight, attn.c_proj.bias, ln_2.weight, ln_2.bias, mlp.c_fc.weight,
+ * mlp.c_fc.bias, mlp.c_proj.weight, mlp.c_proj.bias}, ln_f.weight, ln_f.bias.
+ * out may be NULL to query *count; otherwise it must hold capacity entries. */
+int gpt2_param_layout(const gpt2_handle* h, gpt2_tensor_info* out, int capacity, int* count);
+
+/* Copy the flat fp32 master parameters in or out (n_params floats).
+ * on_device != 0: flat is a device pointer; else host memory. set also refreshes
+ * the bf16 weight copy. Synchronous. */
+int gpt2_set_params(gpt2_handle* h, const float* flat, int on_device);
+int gpt2_get_params(gpt2_handle* h, float* flat, int on_device);
+/* Accumulated fp32 gradients (after the last accumulate/step, before clipping). */
+int gpt2_get_grads(gpt2_handle* h, float* flat, int on_device);
+/* AdamW state: first and second moments (n_params floats each) and the step count. */
+int gpt2_get_opt_state(gpt2_handle* h, float* m, float* v, int64_t* step, int on_device);
+int gpt2_set_opt_state(gpt2_handle* h, const float* m, const float* v, int64_t step, int on_device);
+
+/* Forward pass only (no gradients, no parameter change).
+ * idx_dev      : (B, T) int32 token ids on the device.
+ * targets_dev  : (B, T) int32 or NULL. With targets, *loss_host receives the mean
+ *                cross-entropy over targets != -1 (0 if all are -1).
+ * logits_dev   : NULL or a device buffer for (B, T, vocab_size) logits: fp32 in
+ *                fp32 mode, bf16 in bf16 mode.
+ * loss_host    : NULL or a host float. If non-NULL the call synchronises.
+ * Errors: INVALID_ARG (B > max_B, T > max_T, T > block_size, B or T < 1). */
+int gpt2_forward(gpt2_handle* h, const int32_t* idx_dev, const int32_t* targets_dev,
+                 int B, int T, void* logits_dev, float* loss_host);
+
+/* Set every gradient to zero and clear the accumulated loss. Asynchronous. */
+int gpt2_zero_grad(gpt2_handle* h);
+
+/* Forward + loss + backward of one micro-batch; adds loss_scale x d(loss) to the
+ * gradients and loss_scale x loss to the accumulated loss. Asynchronous (no
+ * synchronisation, no host readback). targets_dev must not be NULL. */
+int gpt2_accumulate(gpt2_handle* h, const int32_t* idx_dev, const int32_t* targets_dev,
+                    int B, int T, float loss_scale);
+
+/* Clip + AdamW on the accumulated gradients, step counter += 1.
+ * loss_host / grad_norm_host (nullable host floats) receive the accumulated loss
+ * and the pre-clip global gradient norm. Synchronises once at the end.
+ * Returns NONFINITE (and leaves parameters, moments, step unchanged) if the
+ * norm or the accumulated loss is not finite. */
+int gpt2_update(gpt2_handle* h, float lr, float* loss_host, float* grad_norm_host);
+
+/* One full training step: zero_grad, accumulate(loss_scale = 1), update.
+ * Device-resident inputs. */
+int gpt2_step(gpt2_handle* h, const int32_t* idx_dev, const int32_t* targets_dev,
+              int B, int T, float lr, float* loss_host, float* grad_norm_host);
+
+/* The same step taking HOST token buffers: the ids and targets are copied to the
+ * device on the handle's stream inside the call (pinned memory gives an
+ * asynchronous copy), then the step runs and the two scalars are read back. */
+int gpt2_step_host(gpt2_handle* h, const int32_t* idx_host, const int32_t* targets_host,
+                   int B, int T, float lr, float* loss_host, float* grad_norm_host);
+
+/* Number of kernel launches the last forward/accumulate/update/step issued. */
+int gpt2_last_launch_count(const gpt2_handle* h, int64_t* n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPT2_B200_H */

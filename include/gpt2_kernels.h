@@ -1,0 +1,64 @@
+/*
+ * gpt2_kernels.h -- kernel-level C ABI of libgpt2_b200.so.
+ *
+ * Single operations of the training step, exposed for unit tests and for
+ * callers that assemble their own step. All pointers are CUDA device pointers
+ * owned by the caller; every call enqueues on `stream` (a cudaStream_t, NULL =
+ * legacy default stream) and returns without synchronising. `status_dev`
+ * points to one caller-owned device uint32 that kernels OR error bits into
+ * (bit 0: out-of-range token, bit 1: a bounded in-kernel wait gave up).
+ * Return codes are the GPT2_* codes of gpt2.h; gpt2_last_error() explains them.
+ */
+#ifndef GPT2_B200_KERNELS_H
+#define GPT2_B200_KERNELS_H
+
+#include <stdint.h>
+
+#include "gpt2.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Operand layouts of C[M,N] = sum_k A(m,k) B(n,k) (row-major storage):
+ *   GPT2K_NT: A [M,K], B [N,K]  -- forward of nn.Linear, y = x W^T
+ *   GPT2K_NN: A [M,K], B [K,N]  -- input gradient, dx = dy W
+ *   GPT2K_TN: A [K,M], B [K,N]  -- weight gradient, dW = dy^T x            */
+#define GPT2K_NT 0
+#define GPT2K_NN 1
+#define GPT2K_TN 2
+
+/* Epilogues ("GPT-2 from Scratch": nn.Linear bias, "The MLP and GPT-2's GELU",
+ * "The Block: pre-LN and residuals"):
+ *   GPT2K_EPI_STORE      out = acc                                (bf16)
+ *   GPT2K_EPI_BIAS       out = acc + bias[n]                      (bf16)
+ *   GPT2K_EPI_BIAS_GELU  out2 = u = acc + bias[n]; out = gelu_tanh(u) (bf16)
+ *   GPT2K_EPI_BIAS_RESID out = resid + acc + bias[n]              (fp32)
+ *   GPT2K_EPI_DGELU      out = acc * gelu_tanh'(aux)              (bf16)
+ *   GPT2K_EPI_ACCUM_F32  out = beta * out + acc                   (fp32)      */
+#define GPT2K_EPI_STORE 0
+#define GPT2K_EPI_BIAS 1
+#define GPT2K_EPI_BIAS_GELU 2
+#define GPT2K_EPI_BIAS_RESID 3
+#define GPT2K_EPI_DGELU 4
+#define GPT2K_EPI_ACCUM_F32 5
+
+/* bf16 GEMM with fp32 accumulation and a fused epilogue.
+ * A, B        : bf16 operands in the given layout.
+ * out, ldo    : result matrix [M, N] with row stride ldo (elements).
+ * out2        : pre-activation output of GPT2K_EPI_BIAS_GELU (same ldo), else NULL.
+ * bias        : fp32 [N] for the BIAS* epilogues, else NULL.
+ * resid       : fp32 [M, N] (stride ldo) for GPT2K_EPI_BIAS_RESID, else NULL.
+ * aux         : bf16 [M, N] (stride ldo) pre-activation for GPT2K_EPI_DGELU, else NULL.
+ * engine      : 1 = tcgen05 tensor cores (TMA + TMEM), 0 = SIMT fp32-FMA kernel.
+ * Errors: INVALID_ARG (sizes < 1, unknown layout/epilogue, a required pointer
+ * NULL, or engine 1 with K, N (or M for TN) not a multiple of 8). */
+int gpt2k_matmul_bf16(int layout, const void* A, const void* B, int M, int N, int K, int epilogue, void* out,
+                      int64_t ldo, void* out2, const float* bias, const float* resid, const void* aux, float beta,
+                      int engine, uint32_t* status_dev, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPT2_B200_KERNELS_H */

@@ -1,0 +1,76 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+function include/*.h declares, and rejects bad configurations before touching
+the device."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+from decoder_only_transformer_sm_b200 import native
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(gpt2\w*)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = native.load_library()
+    decl = _declared_functions()
+    assert len(decl) >= 18, decl
+    out = subprocess.run(["nm", "-D", "--defined-only", native.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(\w+)$", out, flags=re.M))
+    missing = [d for d in decl if d not in exported]
+    assert not missing, missing
+    for d in decl:
+        getattr(lib, d)
+
+
+def test_library_has_no_runtime_dependency_on_libcuda():
+    out = subprocess.run(["ldd", native.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out and "libcudart.so" not in out
+
+
+def _create(**kw):
+    lib = native.load_library()
+    base = dict(n_layer=2, n_head=4, n_embd=128, vocab_size=1024, block_size=64, max_B=4, max_T=64,
+                precision=0, seed=0, grad_clip=1.0, flags=0)
+    base.update(kw)
+    cfg = native.Config(*[base[f] for f, _ in native.Config._fields_])
+    h = ctypes.c_void_p()
+    rc = lib.gpt2_create(ctypes.byref(cfg), None, ctypes.byref(h))
+    return rc, lib.gpt2_last_error().decode(), h
+
+
+@pytest.mark.parametrize("kw,msg", [
+    (dict(n_head=3), "multiple of n_head"),
+    (dict(n_embd=192, n_head=2), "32 or 64"),
+    (dict(n_embd=96, n_head=3), "multiple of 64"),
+    (dict(vocab_size=50257), "multiple of 8"),
+    (dict(max_T=65), "block_size"),
+    (dict(precision=7), "precision"),
+    (dict(n_layer=0), ">= 1"),
+    (dict(flags=1), "flags"),
+])
+def test_invalid_configs_rejected_on_host(kw, msg):
+    rc, err, h = _create(**kw)
+    assert rc == -1 and msg in err and not h.value
+
+
+def test_null_arguments():
+    lib = native.load_library()
+    assert lib.gpt2_create(None, None, None) == -1
+    h = ctypes.c_void_p()
+    assert lib.gpt2_create(None, None, ctypes.byref(h)) == -1
+    lib.gpt2_destroy(None)   # no-op
+    n = ctypes.c_int64()
+    assert lib.gpt2_num_params(None, ctypes.byref(n)) == -1
