@@ -1,0 +1,366 @@
+#!/usr/bin/env python
+"""Throughput of the GPT-2 training step on B200 (tokens/s and MFU).
+
+Workload: GPT-2 124M (12 layers, 12 heads, width 768, vocabulary padded to
+50304, block 1024), one full bf16 training step at B=16, T=1024: forward,
+cross-entropy (ignore_index=-1), backward, global-norm clip at 1.0 and AdamW
+(0.9, 0.95, wd 0.1 on 2-D tensors), fp32 master weights and moments. Tokens
+are synthetic: Zipf(1.1) over the 50257 real GPT-2 ids, targets the same rows
+shifted by one (the pages' FineWeb-Edu / Shakespeare corpora are not
+available). Weights: the pages' random init (std 0.02, residual projections
+0.02/sqrt(24)).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs one process per GPU (torchrun). Each rank trains its own replica on
+its own batches (no data-path collective; weak scaling); the step time is the
+max over ranks. `--impl reference` times the CPU oracle (float64 numpy) on a
+bounded sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(n_layer=12, n_head=12, n_embd=768, vocab_size=50304, vocab_real=50257, block_size=1024,
+                B=16, T=1024)
+LR = 6e-4
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def n_params_padded(w) -> int:
+    C, L, V, Tm = w["n_embd"], w["n_layer"], w["vocab_size"], w["block_size"]
+    per_block = 2 * C + (3 * C * C + 3 * C) + (C * C + C) + 2 * C + (4 * C * C + 4 * C) + (4 * C * C + C)
+    return V * C + Tm * C + L * per_block + 2 * C
+
+
+def flops_per_token(w) -> float:
+    """6N + 12 L C T (N with the tied wte counted once, padded vocabulary)."""
+    return 6.0 * n_params_padded(w) + 12.0 * w["n_layer"] * w["n_embd"] * w["T"]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                     hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+                except ValueError:
+                    continue
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        pmax = max(r["power"] for r in rows)
+        loaded = [r for r in rows if r["power"] >= 0.5 * pmax] or rows
+        reasons = []
+        for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                          ("pcap", "sw_power_cap")):
+            if any(r[key].lower().startswith("active") for r in loaded):
+                reasons.append(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": reasons, "samples": len(loaded), "power_w_max": pmax}
+
+
+# ----------------------------------------------------------------------------
+# reference arm: the CPU oracle, as it stands
+# ----------------------------------------------------------------------------
+def oracle_step_time(T_sample: int, warm: int, steps: int):
+    import numpy as np
+    from threadpoolctl import threadpool_info
+    from oracle import gpt2_oracle as O
+    from decoder_only_transformer_sm_b200 import synthetic as S
+    w = WORKLOAD
+    s = O.Shape(w["n_layer"], w["n_head"], w["n_embd"], w["vocab_size"], w["block_size"])
+    P = O.unflatten(s, S.init_params(S.GPT2_124M, seed=0))
+    M, V = O.zeros_like(s), O.zeros_like(s)
+    idx, tgt = S.zipf_tokens(1, T_sample, w["vocab_real"], seed=1001)
+    for i in range(warm):
+        wi, wt = S.zipf_tokens(1, 16, w["vocab_real"], seed=7 + i)
+        O.forward(s, P, wi, wt)
+    times = []
+    t = 0
+    for _ in range(steps):
+        t += 1
+        t0 = time.perf_counter()
+        O.train_step(s, P, M, V, t, idx, tgt, lr=LR)
+        times.append(time.perf_counter() - t0)
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    del np
+    return times, threads
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    T_sample = 512
+    times, threads = oracle_step_time(T_sample, args.warmup, args.steps)
+    sec = sum(times) / len(times)
+    value = T_sample / sec
+    sample = (f"one float64 oracle step (forward, loss, backward, clip, AdamW on all 124.5M parameters) "
+              f"on B=1 x T={T_sample} Zipf tokens per timed step; warm-up steps are forward passes on 16 tokens")
+    line = {
+        "metric": "training tokens/sec (GPT-2 124M, B=16, T=1024, bf16 step)",
+        "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * sec, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic Zipf(1.1) tokens", "impl": "reference",
+        "config": {"workload": "gpt2-124m train step, oracle sample B=1 T=%d" % T_sample, "B": 1, "T": T_sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+def kernel_source_sha(name: str) -> str:
+    p = os.path.join(ROOT, "decoder_only_transformer_sm_b200", "csrc", name)
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16] if os.path.exists(p) else ""
+
+
+SITE_SOURCES = [("gemm", "k_gemm_tc.cu"), ("attention", "k_attention_simt.cu"), ("layernorm", "k_rowwise.cu"),
+                ("classifier", "k_rowwise.cu"), ("adamw", "k_optim.cu"), ("grad norm", "k_optim.cu"),
+                ("embed", "k_rowwise.cu"), ("bias colsum", "k_rowwise.cu")]
+
+
+def source_of(site: str) -> str:
+    for prefix, f in SITE_SOURCES:
+        if prefix in site:
+            return f
+    return ""
+
+
+def traffic_for(site: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(site)
+    if not e or e.get("kernel_source_sha") != kernel_source_sha(source_of(site)):
+        return None
+    return e.get("bytes_per_launch")
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from decoder_only_transformer_sm_b200 import native, synthetic as S
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    w = WORKLOAD
+    B, T = w["B"], w["T"]
+    stream = torch.cuda.current_stream()
+    m = native.GPT2(w["n_layer"], w["n_head"], w["n_embd"], w["vocab_size"], w["block_size"], B, T,
+                    precision="bf16", seed=1234 + rank, stream=stream.cuda_stream)
+    nb = 2
+    host = [S.zipf_tokens(B, T, w["vocab_real"], seed=1001 + 97 * rank + i) for i in range(nb)]
+    pin = [(torch.from_numpy(i).pin_memory(), torch.from_numpy(t).pin_memory()) for i, t in host]
+    dev = [(i.cuda(), t.cuda()) for i, t in pin]
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for k in range(args.warmup):
+        m.step(*dev[k % nb], LR)
+    torch.cuda.synchronize()
+
+    # ---- timed region: device-resident inputs ----
+    losses = []
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches = 0
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for k in range(args.steps):
+            loss, norm = m.step(*dev[k % nb], LR)
+            launches += m.last_launch_count()
+            losses.append(loss)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    clocks = clk.summary()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+
+    # ---- end to end: host (pinned) token buffers through gpt2_step_host ----
+    barrier()
+    torch.cuda.synchronize()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for k in range(args.steps):
+        m.step_host(pin[k % nb][0], pin[k % nb][1], LR)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = max_over_ranks(e2.elapsed_time(e3) / args.steps)
+
+    # ---- per-launch-site device times (CUDA events on the launching stream) ----
+    m.profile(True)
+    for k in range(args.steps):
+        m.step(*dev[k % nb], LR)
+    stats = m.profile_read()
+    m.profile(False)
+    m.close()
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    tokens = B * T * world
+    value = tokens / (ms / 1000.0)
+    fpt = flops_per_token(w)
+    total_ms = sum(s["total_ms"] for s in stats) / args.steps
+    sites = sorted(stats, key=lambda s: -s["total_ms"])
+    dom = sites[0]
+    per_launch_ms = dom["total_ms"] / dom["launches"]
+    if dom["name"].startswith("gemm") or dom["name"].startswith("attention"):
+        bound, unit = "tensor", "TFLOP/s"
+        achieved = dom["flops"] / dom["launches"] / (per_launch_ms / 1e3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+        peak_note = f"bf16_tflops_sustained of {peak_src} (kernel timed inside a long step)"
+    else:
+        bound, unit = "hbm", "GB/s"
+        achieved = dom["bytes"] / dom["launches"] / (per_launch_ms / 1e3) / 1e9
+        peak = peaks.get("hbm_gbs")
+        peak_note = f"hbm_gbs of {peak_src}"
+    breakdown = []
+    for s in sites[:12]:
+        t = s["total_ms"] / args.steps
+        row = {"site": s["name"], "ms_per_step": round(t, 4), "share": round(t / total_ms, 4),
+               "launches_per_step": s["launches"] // args.steps}
+        if s["flops"] > 0:
+            row["tflops"] = round(s["flops"] / (s["total_ms"] / 1e3) / 1e12, 1)
+        if s["bytes"] > 0:
+            row["gbs"] = round(s["bytes"] / (s["total_ms"] / 1e3) / 1e9, 1)
+        breakdown.append(row)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        times, threads = oracle_step_time(1024, 0, 1)
+        cpu = {"value": 1024 / times[0], "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": "one float64 oracle step (forward, loss, backward, clip, AdamW on all 124.5M "
+                         "parameters) on B=1 x T=1024 Zipf tokens, timed on this host"}
+    line = {
+        "metric": "training tokens/sec (GPT-2 124M, B=16, T=1024, bf16 step)",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic Zipf(1.1) tokens, random-init weights",
+        "config": {"workload": "gpt2-124m train step (fwd+CE+bwd+clip+AdamW), B=16 T=1024 V=50304 bf16",
+                   "B": B, "T": T, "tokens_per_step_per_gpu": B * T,
+                   "parallelism": "replicas" if world > 1 else "single-gpu",
+                   "l2": "working set (6+ GB of activations per step) larger than the 126 MB L2; no flush"},
+        "mfu": {"flops_per_token": fpt, "vs_nominal_2250": value * fpt / world / (NOMINAL_BF16_TFLOPS * 1e12),
+                "vs_measured_sustained": value * fpt / world / (peaks.get("bf16_tflops_sustained", 1400.0) * 1e12),
+                "peak_source": peak_src},
+        "roofline": {"kernel": dom["name"], "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak if peak else None, "traffic": traffic_for(dom["name"]),
+                     "per_launch_ms": per_launch_ms, "peak_note": peak_note},
+        "kernels": breakdown,
+        "cpu_baseline": cpu,
+        "e2e": {"value": tokens / (ms_e2e / 1000.0), "unit": "tokens/s",
+                "h2d_bytes_per_step": 2 * B * T * 4, "d2h_bytes_per_step": 40},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "loss_first_last": [losses[0], losses[-1]],
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

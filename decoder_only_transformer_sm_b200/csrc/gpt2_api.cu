@@ -18,6 +18,7 @@
 #include <cstdio>
 #include <cstring>
 #include <string>
+#include <unordered_map>
 #include <vector>
 
 using namespace gpt2;
@@ -53,6 +54,12 @@ struct DevScalars {
     double sumsq;        // global gradient sum of squares
     int n_valid;         // targets != -1 in the current micro-batch
     unsigned status;     // STATUS_* bits
+};
+
+struct ProfSite {
+    std::string name;
+    long long launches = 0;
+    double ms = 0, flops = 0, bytes = 0;
 };
 
 struct LayerOff {   // offsets of one block's tensors in the flat vector
@@ -109,6 +116,13 @@ struct gpt2_handle {
     long long launches = 0;
     bool use_tc_gemm = true;
     std::string host_error;   // set by enqueue helpers that cannot report a status
+
+    bool profiling = false;
+    std::vector<ProfSite> psites;
+    std::unordered_map<std::string, int> pidx;
+    std::vector<cudaEvent_t> pev;
+    size_t pev_used = 0;
+    std::vector<std::pair<int, size_t>> ppending;
 
     Ctx ctx() {
         Ctx c;
@@ -239,25 +253,96 @@ int refresh_shadow(gpt2_handle* h) {
     return GPT2_OK;
 }
 
+// ----------------------------------------------------------- profiling
+// With profiling on, every launch site is bracketed by two CUDA events on the
+// handle's stream; the elapsed times are summed per site when the stream is
+// next synchronised. flops/bytes are the algorithmic work of one launch.
+int prof_site(gpt2_handle* h, const std::string& name) {
+    auto it = h->pidx.find(name);
+    if (it != h->pidx.end()) return it->second;
+    ProfSite ps;
+    ps.name = name;
+    h->psites.push_back(ps);
+    h->pidx[name] = (int)h->psites.size() - 1;
+    return (int)h->psites.size() - 1;
+}
+
+template <class F>
+void prof(gpt2_handle* h, const char* name, int M, int N, int K, double flops, double bytes, F&& launch) {
+    if (!h->profiling || h->pev_used + 2 > h->pev.size()) {
+        launch();
+        return;
+    }
+    std::string nm(name);
+    if (M > 0) nm += " " + std::to_string(M) + "x" + std::to_string(N) + "x" + std::to_string(K);
+    const int site = prof_site(h, nm);
+    ProfSite& ps = h->psites[site];
+    ps.flops += flops;
+    ps.bytes += bytes;
+    ps.launches += 1;
+    const size_t e = h->pev_used;
+    cudaEventRecord(h->pev[e], h->stream);
+    launch();
+    cudaEventRecord(h->pev[e + 1], h->stream);
+    h->pev_used += 2;
+    h->ppending.push_back({site, e});
+}
+
+void prof_collect(gpt2_handle* h) {
+    for (auto& pr : h->ppending) {
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, h->pev[pr.second], h->pev[pr.second + 1]) == cudaSuccess)
+            h->psites[pr.first].ms += ms;
+    }
+    cudaGetLastError();
+    h->ppending.clear();
+    h->pev_used = 0;
+}
+
+#define PROF(name, M, N, K, flops, bytes, ...) prof(h, name, M, N, K, flops, bytes, [&]() { __VA_ARGS__; })
+
 // ------------------------------------------------------------ GEMM dispatch
 template <typename A>
-void gemm(gpt2_handle* h, GemmLayout layout, const void* a, const void* b, int M, int N, int K, const Epilogue& ep);
+void gemm_raw(gpt2_handle* h, GemmLayout layout, const void* a, const void* b, int M, int N, int K,
+              const Epilogue& ep);
 
 template <>
-void gemm<float>(gpt2_handle* h, GemmLayout layout, const void* a, const void* b, int M, int N, int K,
-                 const Epilogue& ep) {
+void gemm_raw<float>(gpt2_handle* h, GemmLayout layout, const void* a, const void* b, int M, int N, int K,
+                     const Epilogue& ep) {
     launch_gemm_simt<float>(h->ctx(), layout, (const float*)a, (const float*)b, M, N, K, ep);
 }
 
 template <>
-void gemm<bf16>(gpt2_handle* h, GemmLayout layout, const void* a, const void* b, int M, int N, int K,
-                const Epilogue& ep) {
+void gemm_raw<bf16>(gpt2_handle* h, GemmLayout layout, const void* a, const void* b, int M, int N, int K,
+                    const Epilogue& ep) {
     if (h->use_tc_gemm && gemm_tc_supported(layout, M, N, K)) {
         if (!launch_gemm_tc(h->ctx(), layout, (const bf16*)a, (const bf16*)b, M, N, K, ep))
             h->host_error = "tensor-map encoding failed for a tensor-core GEMM";
     } else {
         launch_gemm_simt<bf16>(h->ctx(), layout, (const bf16*)a, (const bf16*)b, M, N, K, ep);
     }
+}
+
+// Algorithmic bytes of one GEMM: operands once, the output once (read too for
+// read-modify-write epilogues).
+double gemm_bytes(int M, int N, int K, size_t es, const Epilogue& ep) {
+    double b = ((double)M * K + (double)N * K) * es;
+    const double mn = (double)M * N;
+    switch (ep.kind) {
+    case EPI_BIAS_GELU: b += 2 * mn * es; break;
+    case EPI_BIAS_RESID: b += 2 * mn * 4; break;
+    case EPI_DGELU: b += 2 * mn * es; break;
+    case EPI_ACCUM_F32: b += (ep.beta != 0.f ? 2 : 1) * mn * 4; break;
+    default: b += mn * es; break;
+    }
+    return b;
+}
+
+template <typename A>
+void gemm(gpt2_handle* h, const char* site, GemmLayout layout, const void* a, const void* b, int M, int N, int K,
+          const Epilogue& ep) {
+    PROF(site, M, N, K, 2.0 * M * N * K, gemm_bytes(M, N, K, sizeof(A), ep),
+         gemm_raw<A>(h, layout, a, b, M, N, K, ep));
 }
 
 Epilogue epi(int kind, void* out, long long ldo) {
@@ -278,41 +363,50 @@ template <typename A>
 void forward_impl(gpt2_handle* h, const int* idx, const int* targets, int B, int T, A* logits_out,
                   double* loss_slot, float loss_scale, bool write_grad) {
     Ctx c = h->ctx();
-    const int BT = B * T, C = h->C, V = h->V, L = h->L;
+    const int BT = B * T, C = h->C, V = h->V, L = h->L, H = h->H, hd = h->hd;
+    const double es = sizeof(A);
+    const double ln_fwd_bytes = (double)BT * C * (4 + es) + 8.0 * BT;
+    const double att_fwd_flops = 2.0 * B * H * (double)T * (T + 1) * hd;   // causal QK^T and PV
     float* P = h->params;
-    launch_embed_ln<A>(c, idx, P + h->off_wte, P + h->off_wpe, BT, T, C, V, P + h->lo[0].ln1w, P + h->lo[0].ln1b,
-                       h->resid[0], (A*)h->ln1[0], h->ln_mean[0], h->ln_rstd[0]);
+    PROF("embed+ln_1", 0, 0, 0, 0.0, (double)BT * C * (4 + 4 + 4 + es),
+         launch_embed_ln<A>(c, idx, P + h->off_wte, P + h->off_wpe, BT, T, C, V, P + h->lo[0].ln1w,
+                            P + h->lo[0].ln1b, h->resid[0], (A*)h->ln1[0], h->ln_mean[0], h->ln_rstd[0]));
     for (int l = 0; l < L; ++l) {
         const LayerOff& o = h->lo[l];
         Epilogue e = epi(EPI_BIAS, h->qkv[l], 3 * C);
         e.bias = P + o.bqkv;
-        gemm<A>(h, GEMM_NT, h->ln1[l], wop<A>(h, o.wqkv), BT, 3 * C, C, e);
-        launch_attention_fwd_simt<A>(c, (const A*)h->qkv[l], (A*)h->att[l], h->lse[l], B, T, h->H, h->hd);
+        gemm<A>(h, "gemm fwd c_attn", GEMM_NT, h->ln1[l], wop<A>(h, o.wqkv), BT, 3 * C, C, e);
+        PROF("attention fwd", 0, 0, 0, att_fwd_flops, (double)BT * C * es * 4,
+             launch_attention_fwd_simt<A>(c, (const A*)h->qkv[l], (A*)h->att[l], h->lse[l], B, T, H, hd));
         e = epi(EPI_BIAS_RESID, h->resid[2 * l + 1], C);
         e.bias = P + o.bproj;
         e.resid = h->resid[2 * l];
-        gemm<A>(h, GEMM_NT, h->att[l], wop<A>(h, o.wproj), BT, C, C, e);
-        launch_layernorm_fwd<A>(c, h->resid[2 * l + 1], P + o.ln2w, P + o.ln2b, (A*)h->ln2[l], h->ln_mean[2 * l + 1],
-                                h->ln_rstd[2 * l + 1], BT, C);
+        gemm<A>(h, "gemm fwd attn.c_proj", GEMM_NT, h->att[l], wop<A>(h, o.wproj), BT, C, C, e);
+        PROF("layernorm fwd", 0, 0, 0, 0.0, ln_fwd_bytes,
+             launch_layernorm_fwd<A>(c, h->resid[2 * l + 1], P + o.ln2w, P + o.ln2b, (A*)h->ln2[l],
+                                     h->ln_mean[2 * l + 1], h->ln_rstd[2 * l + 1], BT, C));
         e = epi(EPI_BIAS_GELU, h->fcg[l], 4 * C);
         e.out2 = h->fch[l];
         e.bias = P + o.bfc;
-        gemm<A>(h, GEMM_NT, h->ln2[l], wop<A>(h, o.wfc), BT, 4 * C, C, e);
+        gemm<A>(h, "gemm fwd c_fc+gelu", GEMM_NT, h->ln2[l], wop<A>(h, o.wfc), BT, 4 * C, C, e);
         e = epi(EPI_BIAS_RESID, h->resid[2 * l + 2], C);
         e.bias = P + o.bfcp;
         e.resid = h->resid[2 * l + 1];
-        gemm<A>(h, GEMM_NT, h->fcg[l], wop<A>(h, o.wfcp), BT, C, 4 * C, e);
-        if (l + 1 < L)
-            launch_layernorm_fwd<A>(c, h->resid[2 * l + 2], P + h->lo[l + 1].ln1w, P + h->lo[l + 1].ln1b,
-                                    (A*)h->ln1[l + 1], h->ln_mean[2 * l + 2], h->ln_rstd[2 * l + 2], BT, C);
+        gemm<A>(h, "gemm fwd mlp.c_proj", GEMM_NT, h->fcg[l], wop<A>(h, o.wfcp), BT, C, 4 * C, e);
+        const bool last = (l + 1 == L);
+        PROF("layernorm fwd", 0, 0, 0, 0.0, ln_fwd_bytes,
+             launch_layernorm_fwd<A>(c, h->resid[2 * l + 2], last ? P + h->off_lnfw : P + h->lo[l + 1].ln1w,
+                                     last ? P + h->off_lnfb : P + h->lo[l + 1].ln1b,
+                                     last ? (A*)h->lnf : (A*)h->ln1[l + 1], h->ln_mean[2 * l + 2],
+                                     h->ln_rstd[2 * l + 2], BT, C));
     }
-    launch_layernorm_fwd<A>(c, h->resid[2 * L], P + h->off_lnfw, P + h->off_lnfb, (A*)h->lnf, h->ln_mean[2 * L],
-                            h->ln_rstd[2 * L], BT, C);
     A* lg = logits_out ? logits_out : (A*)h->logits;
-    gemm<A>(h, GEMM_NT, h->lnf, wop<A>(h, h->off_wte), BT, V, C, epi(EPI_STORE, lg, V));
+    gemm<A>(h, "gemm fwd lm_head", GEMM_NT, h->lnf, wop<A>(h, h->off_wte), BT, V, C, epi(EPI_STORE, lg, V));
     if (targets) {
-        launch_count_targets(c, targets, BT, V, &h->d_sc->n_valid);
-        launch_classifier<A>(c, lg, targets, BT, V, &h->d_sc->n_valid, loss_scale, loss_slot, write_grad ? 1 : 0);
+        PROF("count targets", 0, 0, 0, 0.0, 4.0 * BT, launch_count_targets(c, targets, BT, V, &h->d_sc->n_valid));
+        PROF("classifier", 0, 0, 0, 0.0, (double)BT * V * es * (write_grad ? 2 : 1),
+             launch_classifier<A>(c, lg, targets, BT, V, &h->d_sc->n_valid, loss_scale, loss_slot,
+                                  write_grad ? 1 : 0));
     }
 }
 
@@ -320,56 +414,69 @@ void forward_impl(gpt2_handle* h, const int* idx, const int* targets, int B, int
 template <typename A>
 void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
     Ctx c = h->ctx();
-    const int BT = B * T, C = h->C, V = h->V, L = h->L;
+    const int BT = B * T, C = h->C, V = h->V, L = h->L, H = h->H, hd = h->hd;
+    const double es = sizeof(A);
+    const double ln_bwd_bytes = (double)BT * C * (es + 4 + 4 + 4 + es);
+    const double att_bwd_flops = 5.0 * B * H * (double)T * (T + 1) * hd;   // S recompute, dV, dP, dQ, dK
     float* P = h->params;
     float* G = h->grads;
     // lm_head (tied): dlnf = dlogits wte ; dwte += dlogits^T lnf
-    gemm<A>(h, GEMM_NN, h->logits, wop<A>(h, h->off_wte), BT, C, V, epi(EPI_STORE, h->dtmp, C));
+    gemm<A>(h, "gemm dgrad lm_head", GEMM_NN, h->logits, wop<A>(h, h->off_wte), BT, C, V,
+            epi(EPI_STORE, h->dtmp, C));
     Epilogue acc = epi(EPI_ACCUM_F32, G + h->off_wte, C);
     acc.beta = 1.f;
-    gemm<A>(h, GEMM_TN, h->logits, h->lnf, V, C, BT, acc);
-    launch_layernorm_bwd<A>(c, (const A*)h->dtmp, h->resid[2 * L], h->ln_mean[2 * L], h->ln_rstd[2 * L],
-                            P + h->off_lnfw, nullptr, h->dres, (A*)h->dres_act, G + h->off_lnfw, G + h->off_lnfb,
-                            G + h->lo[L - 1].bfcp, BT, C);
+    gemm<A>(h, "gemm wgrad lm_head", GEMM_TN, h->logits, h->lnf, V, C, BT, acc);
+    PROF("layernorm bwd", 0, 0, 0, 0.0, ln_bwd_bytes - 4.0 * BT * C,
+         launch_layernorm_bwd<A>(c, (const A*)h->dtmp, h->resid[2 * L], h->ln_mean[2 * L], h->ln_rstd[2 * L],
+                                 P + h->off_lnfw, nullptr, h->dres, (A*)h->dres_act, G + h->off_lnfw,
+                                 G + h->off_lnfb, G + h->lo[L - 1].bfcp, BT, C));
     for (int l = L - 1; l >= 0; --l) {
         const LayerOff& o = h->lo[l];
         // mlp.c_proj: dW += dY^T g ; du = (dY W) * gelu'(u)
         acc = epi(EPI_ACCUM_F32, G + o.wfcp, 4 * C);
         acc.beta = 1.f;
-        gemm<A>(h, GEMM_TN, h->dres_act, h->fcg[l], C, 4 * C, BT, acc);
+        gemm<A>(h, "gemm wgrad mlp.c_proj", GEMM_TN, h->dres_act, h->fcg[l], C, 4 * C, BT, acc);
         Epilogue e = epi(EPI_DGELU, h->du, 4 * C);
         e.aux = h->fch[l];
-        gemm<A>(h, GEMM_NN, h->dres_act, wop<A>(h, o.wfcp), BT, 4 * C, C, e);
-        launch_colsum<A>(c, (const A*)h->du, BT, 4 * C, G + o.bfc);
+        gemm<A>(h, "gemm dgrad mlp.c_proj+dgelu", GEMM_NN, h->dres_act, wop<A>(h, o.wfcp), BT, 4 * C, C, e);
+        PROF("bias colsum", 0, 0, 0, 0.0, (double)BT * 4 * C * es,
+             launch_colsum<A>(c, (const A*)h->du, BT, 4 * C, G + o.bfc));
         // mlp.c_fc: dW += du^T ln2 ; dln2 = du W
         acc = epi(EPI_ACCUM_F32, G + o.wfc, C);
         acc.beta = 1.f;
-        gemm<A>(h, GEMM_TN, h->du, h->ln2[l], 4 * C, C, BT, acc);
-        gemm<A>(h, GEMM_NN, h->du, wop<A>(h, o.wfc), BT, C, 4 * C, epi(EPI_STORE, h->dtmp, C));
+        gemm<A>(h, "gemm wgrad c_fc", GEMM_TN, h->du, h->ln2[l], 4 * C, C, BT, acc);
+        gemm<A>(h, "gemm dgrad c_fc", GEMM_NN, h->du, wop<A>(h, o.wfc), BT, C, 4 * C, epi(EPI_STORE, h->dtmp, C));
         // ln_2 backward + residual; colsum of the result is the attn.c_proj bias gradient
-        launch_layernorm_bwd<A>(c, (const A*)h->dtmp, h->resid[2 * l + 1], h->ln_mean[2 * l + 1],
-                                h->ln_rstd[2 * l + 1], P + o.ln2w, h->dres, h->dres, (A*)h->dres_act, G + o.ln2w,
-                                G + o.ln2b, G + o.bproj, BT, C);
+        PROF("layernorm bwd", 0, 0, 0, 0.0, ln_bwd_bytes,
+             launch_layernorm_bwd<A>(c, (const A*)h->dtmp, h->resid[2 * l + 1], h->ln_mean[2 * l + 1],
+                                     h->ln_rstd[2 * l + 1], P + o.ln2w, h->dres, h->dres, (A*)h->dres_act,
+                                     G + o.ln2w, G + o.ln2b, G + o.bproj, BT, C));
         // attn.c_proj
         acc = epi(EPI_ACCUM_F32, G + o.wproj, C);
         acc.beta = 1.f;
-        gemm<A>(h, GEMM_TN, h->dres_act, h->att[l], C, C, BT, acc);
-        gemm<A>(h, GEMM_NN, h->dres_act, wop<A>(h, o.wproj), BT, C, C, epi(EPI_STORE, h->dO, C));
+        gemm<A>(h, "gemm wgrad attn.c_proj", GEMM_TN, h->dres_act, h->att[l], C, C, BT, acc);
+        gemm<A>(h, "gemm dgrad attn.c_proj", GEMM_NN, h->dres_act, wop<A>(h, o.wproj), BT, C, C,
+                epi(EPI_STORE, h->dO, C));
         // attention
-        launch_attention_bwd_simt<A>(c, (const A*)h->qkv[l], (const A*)h->att[l], (const A*)h->dO, h->lse[l],
-                                     h->dpre, (A*)h->dqkv, B, T, h->H, h->hd);
-        launch_colsum<A>(c, (const A*)h->dqkv, BT, 3 * C, G + o.bqkv);
+        PROF("attention bwd", 0, 0, 0, att_bwd_flops, (double)BT * C * es * 8,
+             launch_attention_bwd_simt<A>(c, (const A*)h->qkv[l], (const A*)h->att[l], (const A*)h->dO, h->lse[l],
+                                          h->dpre, (A*)h->dqkv, B, T, H, hd));
+        PROF("bias colsum", 0, 0, 0, 0.0, (double)BT * 3 * C * es,
+             launch_colsum<A>(c, (const A*)h->dqkv, BT, 3 * C, G + o.bqkv));
         // attn.c_attn
         acc = epi(EPI_ACCUM_F32, G + o.wqkv, C);
         acc.beta = 1.f;
-        gemm<A>(h, GEMM_TN, h->dqkv, h->ln1[l], 3 * C, C, BT, acc);
-        gemm<A>(h, GEMM_NN, h->dqkv, wop<A>(h, o.wqkv), BT, C, 3 * C, epi(EPI_STORE, h->dtmp, C));
+        gemm<A>(h, "gemm wgrad c_attn", GEMM_TN, h->dqkv, h->ln1[l], 3 * C, C, BT, acc);
+        gemm<A>(h, "gemm dgrad c_attn", GEMM_NN, h->dqkv, wop<A>(h, o.wqkv), BT, C, 3 * C,
+                epi(EPI_STORE, h->dtmp, C));
         // ln_1 backward + residual; colsum is the previous block's mlp.c_proj bias gradient
-        launch_layernorm_bwd<A>(c, (const A*)h->dtmp, h->resid[2 * l], h->ln_mean[2 * l], h->ln_rstd[2 * l],
-                                P + o.ln1w, h->dres, h->dres, (A*)h->dres_act, G + o.ln1w, G + o.ln1b,
-                                l > 0 ? G + h->lo[l - 1].bfcp : nullptr, BT, C);
+        PROF("layernorm bwd", 0, 0, 0, 0.0, ln_bwd_bytes,
+             launch_layernorm_bwd<A>(c, (const A*)h->dtmp, h->resid[2 * l], h->ln_mean[2 * l], h->ln_rstd[2 * l],
+                                     P + o.ln1w, h->dres, h->dres, (A*)h->dres_act, G + o.ln1w, G + o.ln1b,
+                                     l > 0 ? G + h->lo[l - 1].bfcp : nullptr, BT, C));
     }
-    launch_embed_bwd(c, idx, h->dres, B, T, C, V, G + h->off_wte, G + h->off_wpe);
+    PROF("embedding bwd", 0, 0, 0, 0.0, (double)BT * C * 12 + (double)T * C * 8,
+         launch_embed_bwd(c, idx, h->dres, B, T, C, V, G + h->off_wte, G + h->off_wpe));
 }
 
 int read_scalars(gpt2_handle* h) {
@@ -414,16 +521,18 @@ int zero_grad_impl(gpt2_handle* h) {
 int update_impl(gpt2_handle* h, float lr, float* loss_host, float* norm_host) {
     Ctx c = h->ctx();
     CK(cudaMemsetAsync(&h->d_sc->sumsq, 0, sizeof(double), h->stream));
-    launch_sumsq(c, h->grads, h->n_params, &h->d_sc->sumsq);
+    PROF("grad norm", 0, 0, 0, 0.0, 4.0 * h->n_params, launch_sumsq(c, h->grads, h->n_params, &h->d_sc->sumsq));
     const long long t = h->step_t + 1;
     const double bc1 = 1.0 - pow(0.9, (double)t), bc2 = 1.0 - pow(0.95, (double)t);
     const float clip = h->cfg.grad_clip > 0.f ? h->cfg.grad_clip : 1.0f;
-    launch_adamw(c, h->d_chunks, h->n_chunks, h->params, h->grads, h->mom1, h->mom2,
-                 h->bf16_mode ? h->shadow : nullptr, &h->d_sc->sumsq, &h->d_sc->loss_accum, lr, clip, (float)bc1,
-                 (float)bc2, 0.1f);
+    PROF("adamw+clip", 0, 0, 0, 0.0, (28.0 + (h->bf16_mode ? 2.0 : 0.0)) * h->n_params,
+         launch_adamw(c, h->d_chunks, h->n_chunks, h->params, h->grads, h->mom1, h->mom2,
+                      h->bf16_mode ? h->shadow : nullptr, &h->d_sc->sumsq, &h->d_sc->loss_accum, lr, clip,
+                      (float)bc1, (float)bc2, 0.1f));
     CK(cudaGetLastError());
     int rc = read_scalars(h);
     if (rc) return rc;
+    if (h->profiling) prof_collect(h);
     const double loss = h->h_sc->loss_accum, ss = h->h_sc->sumsq;
     if (loss_host) *loss_host = (float)loss;
     if (norm_host) *norm_host = (float)sqrt(ss);
@@ -569,6 +678,7 @@ void gpt2_destroy(gpt2_handle* h) {
     cudaFree(h->act_pool);
     cudaFree(h->d_sc);
     if (h->h_sc) cudaFreeHost(h->h_sc);
+    for (cudaEvent_t e : h->pev) cudaEventDestroy(e);
     delete h;
 }
 
@@ -716,6 +826,39 @@ int gpt2_step_host(gpt2_handle* h, const int32_t* idx_host, const int32_t* targe
     if (!rc) rc = accumulate_impl(h, h->d_tokens, h->d_tokens + n, B, T, 1.f);
     if (!rc) rc = update_impl(h, lr, loss_host, grad_norm_host);
     return rc;
+}
+
+int gpt2_profile(gpt2_handle* h, int enable) {
+    if (!h) return fail(GPT2_ERR_INVALID_ARG, "NULL handle");
+    CK(cudaStreamSynchronize(h->stream));
+    h->ppending.clear();
+    h->pev_used = 0;
+    h->psites.clear();
+    h->pidx.clear();
+    h->profiling = enable != 0;
+    if (h->profiling && h->pev.empty()) {
+        h->pev.resize(8192);
+        for (auto& e : h->pev) CK(cudaEventCreate(&e));
+    }
+    return GPT2_OK;
+}
+
+int gpt2_profile_read(gpt2_handle* h, gpt2_kernel_stat* out, int capacity, int* count) {
+    if (!h || !count) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    CK(cudaStreamSynchronize(h->stream));
+    prof_collect(h);
+    *count = (int)h->psites.size();
+    if (!out) return GPT2_OK;
+    if (capacity < *count) return fail(GPT2_ERR_INVALID_ARG, "capacity smaller than the site count");
+    for (size_t i = 0; i < h->psites.size(); ++i) {
+        memset(&out[i], 0, sizeof(out[i]));
+        strncpy(out[i].name, h->psites[i].name.c_str(), sizeof(out[i].name) - 1);
+        out[i].launches = h->psites[i].launches;
+        out[i].total_ms = h->psites[i].ms;
+        out[i].flops = h->psites[i].flops;
+        out[i].bytes = h->psites[i].bytes;
+    }
+    return GPT2_OK;
 }
 
 int gpt2_last_launch_count(const gpt2_handle* h, int64_t* n) {

@@ -37,6 +37,13 @@ class Config(ctypes.Structure):
     ]
 
 
+class KernelStat(ctypes.Structure):
+    _fields_ = [
+        ("name", ctypes.c_char * 96), ("launches", ctypes.c_int64), ("total_ms", ctypes.c_double),
+        ("flops", ctypes.c_double), ("bytes", ctypes.c_double),
+    ]
+
+
 class TensorInfo(ctypes.Structure):
     _fields_ = [
         ("name", ctypes.c_char * 48), ("ndim", ctypes.c_int32), ("shape", ctypes.c_int64 * 2),
@@ -75,6 +82,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gpt2_step": (I, [P, P, P, I, I, F, ctypes.POINTER(F), ctypes.POINTER(F)]),
         "gpt2_step_host": (I, [P, P, P, I, I, F, ctypes.POINTER(F), ctypes.POINTER(F)]),
         "gpt2_last_launch_count": (I, [P, ctypes.POINTER(ctypes.c_int64)]),
+        "gpt2_profile": (I, [P, I]),
+        "gpt2_profile_read": (I, [P, P, I, ctypes.POINTER(I)]),
         "gpt2k_matmul_bf16": (I, [I, P, P, I, I, I, I, P, ctypes.c_int64, P, P, P, P, F, I, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -209,6 +218,18 @@ class GPT2:
         _check(self._lib.gpt2_step_host(self._h, _ptr(idx), _ptr(targets), B, T, lr,
                                         ctypes.byref(loss), ctypes.byref(norm)))
         return loss.value, norm.value
+
+    def profile(self, enable: bool = True):
+        _check(self._lib.gpt2_profile(self._h, 1 if enable else 0))
+
+    def profile_read(self):
+        """List of dicts: name, launches, total_ms, flops, bytes (per launch site)."""
+        cnt = ctypes.c_int()
+        _check(self._lib.gpt2_profile_read(self._h, None, 0, ctypes.byref(cnt)))
+        arr = (KernelStat * max(cnt.value, 1))()
+        _check(self._lib.gpt2_profile_read(self._h, arr, cnt.value, ctypes.byref(cnt)))
+        return [dict(name=a.name.decode(), launches=int(a.launches), total_ms=float(a.total_ms),
+                     flops=float(a.flops), bytes=float(a.bytes)) for a in arr[:cnt.value]]
 
     def last_launch_count(self) -> int:
         n = ctypes.c_int64()

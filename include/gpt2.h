@@ -172,6 +172,22 @@ int gpt2_step_host(gpt2_handle* h, const int32_t* idx_host, const int32_t* targe
 /* Number of kernel launches the last forward/accumulate/update/step issued. */
 int gpt2_last_launch_count(const gpt2_handle* h, int64_t* n);
 
+/* Per-launch-site timing. With profiling enabled, every kernel launch site is
+ * bracketed by two CUDA events on the handle's stream (device time, no host
+ * synchronisation added); gpt2_profile_read synchronises and returns, per site,
+ * the launch count, summed device milliseconds and the summed algorithmic
+ * FLOPs and HBM bytes. gpt2_profile(h, 1) clears the statistics. */
+typedef struct gpt2_kernel_stat {
+    char name[96];       /* site, e.g. "gemm fwd lm_head 16384x50304x768", "classifier" */
+    int64_t launches;
+    double total_ms;
+    double flops;        /* algorithmic floating-point operations, all launches        */
+    double bytes;        /* algorithmic HBM bytes (each operand once), all launches    */
+} gpt2_kernel_stat;
+
+int gpt2_profile(gpt2_handle* h, int enable);
+int gpt2_profile_read(gpt2_handle* h, gpt2_kernel_stat* out, int capacity, int* count);
+
 #ifdef __cplusplus
 }
 #endif
