@@ -52,3 +52,58 @@ extern "C" int gpt2k_matmul_bf16(int layout, const void* A, const void* B, int M
     if (err != cudaSuccess) return set_error(GPT2_ERR_CUDA, cudaGetErrorString(err));
     return GPT2_OK;
 }
+
+namespace {
+int check_attention_args(int dtype, int B, int T, int H, int hd, int engine, const void* a, const void* b,
+                         const void* c, const uint32_t* status) {
+    if (dtype != GPT2K_F32 && dtype != GPT2K_BF16) return set_error(GPT2_ERR_INVALID_ARG, "unknown dtype");
+    if (B < 1 || T < 1 || H < 1) return set_error(GPT2_ERR_INVALID_ARG, "B, T, H must be >= 1");
+    if (hd != 32 && hd != 64) return set_error(GPT2_ERR_INVALID_ARG, "head width must be 32 or 64");
+    if (engine != 0) return set_error(GPT2_ERR_INVALID_ARG, "unknown attention engine");
+    if (!a || !b || !c || !status) return set_error(GPT2_ERR_INVALID_ARG, "NULL operand");
+    return GPT2_OK;
+}
+
+Ctx kctx(void* stream, uint32_t* status, long long* launches) {
+    Ctx c;
+    c.stream = (cudaStream_t)stream;
+    c.status = status;
+    c.launches = launches;
+    c.num_sms = 148;
+    return c;
+}
+}  // namespace
+
+extern "C" int gpt2k_attention_fwd(int dtype, const void* qkv, void* out, float* lse, int B, int T, int H, int hd,
+                                   int engine, uint32_t* status_dev, void* stream) {
+    int rc = check_attention_args(dtype, B, T, H, hd, engine, qkv, out, lse, status_dev);
+    if (rc) return rc;
+    long long launches = 0;
+    Ctx c = kctx(stream, status_dev, &launches);
+    if (dtype == GPT2K_F32)
+        launch_attention_fwd_simt<float>(c, (const float*)qkv, (float*)out, lse, B, T, H, hd);
+    else
+        launch_attention_fwd_simt<bf16>(c, (const bf16*)qkv, (bf16*)out, lse, B, T, H, hd);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return set_error(GPT2_ERR_CUDA, cudaGetErrorString(err));
+    return GPT2_OK;
+}
+
+extern "C" int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, const void* dout, const float* lse,
+                                   void* dqkv, int B, int T, int H, int hd, float* workspace_dev, int engine,
+                                   uint32_t* status_dev, void* stream) {
+    int rc = check_attention_args(dtype, B, T, H, hd, engine, qkv, out, dout, status_dev);
+    if (rc) return rc;
+    if (!lse || !dqkv || !workspace_dev) return set_error(GPT2_ERR_INVALID_ARG, "NULL operand");
+    long long launches = 0;
+    Ctx c = kctx(stream, status_dev, &launches);
+    if (dtype == GPT2K_F32)
+        launch_attention_bwd_simt<float>(c, (const float*)qkv, (const float*)out, (const float*)dout, lse,
+                                         workspace_dev, (float*)dqkv, B, T, H, hd);
+    else
+        launch_attention_bwd_simt<bf16>(c, (const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse,
+                                        workspace_dev, (bf16*)dqkv, B, T, H, hd);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return set_error(GPT2_ERR_CUDA, cudaGetErrorString(err));
+    return GPT2_OK;
+}

@@ -85,6 +85,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gpt2_profile": (I, [P, I]),
         "gpt2_profile_read": (I, [P, P, I, ctypes.POINTER(I)]),
         "gpt2k_matmul_bf16": (I, [I, P, P, I, I, I, I, P, ctypes.c_int64, P, P, P, P, F, I, P, P]),
+        "gpt2k_attention_fwd": (I, [I, P, P, P, I, I, I, I, I, P, P]),
+        "gpt2k_attention_bwd": (I, [I, P, P, P, P, P, I, I, I, I, P, I, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -259,3 +261,36 @@ def matmul_bf16(layout: str, A, B, M: int, N: int, K: int, epilogue: str, out, l
                                beta, 1 if engine == "tc" else 0, _ptr(status), stream)
     _check(rc)
     return status
+
+
+def _dtype_code(t) -> int:
+    import torch
+    return {torch.float32: 0, torch.bfloat16: 1}[t.dtype]
+
+
+def _stream_and_status(ref, status, stream):
+    import torch
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=ref.device)
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    return status, stream
+
+
+def attention_fwd(qkv, out, lse, B: int, T: int, H: int, hd: int, engine: int = 0, status=None, stream=None):
+    """gpt2k_attention_fwd on torch device tensors; returns the status tensor."""
+    status, stream = _stream_and_status(qkv, status, stream)
+    _check(load_library().gpt2k_attention_fwd(_dtype_code(qkv), _ptr(qkv), _ptr(out), _ptr(lse), B, T, H, hd,
+                                              engine, _ptr(status), stream))
+    return status
+
+
+def attention_bwd(qkv, out, dout, lse, dqkv, B: int, T: int, H: int, hd: int, workspace, engine: int = 0,
+                  status=None, stream=None):
+    """gpt2k_attention_bwd on torch device tensors (workspace: B*H*T float32)."""
+    status, stream = _stream_and_status(qkv, status, stream)
+    _check(load_library().gpt2k_attention_bwd(_dtype_code(qkv), _ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse),
+                                              _ptr(dqkv), B, T, H, hd, _ptr(workspace), engine, _ptr(status),
+                                              stream))
+    return status
+

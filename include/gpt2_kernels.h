@@ -57,6 +57,31 @@ int gpt2k_matmul_bf16(int layout, const void* A, const void* B, int M, int N, in
                       int64_t ldo, void* out2, const float* bias, const float* resid, const void* aux, float beta,
                       int engine, uint32_t* status_dev, void* stream);
 
+/* Element types of activation operands. */
+#define GPT2K_F32 0
+#define GPT2K_BF16 1
+
+/* Causal multi-head self-attention forward ("GPT-2 from Scratch",
+ * "CausalSelfAttention": softmax(q k^T / sqrt(hd)) with future positions masked,
+ * times v; "Let's reproduce GPT-2 (124M)", "FlashAttention and vocabulary
+ * padding": online softmax, no T x T matrix in memory).
+ * qkv  : (B, T, 3C) rows [q | k | v], C = H * hd; head h owns columns
+ *        [h*hd, (h+1)*hd) of each C-wide block.
+ * out  : (B, T, C), heads concatenated in head order.
+ * lse  : (B, H, T) fp32 log-sum-exp of each softmax row (for the backward).
+ * dtype: GPT2K_F32 or GPT2K_BF16 (qkv, out); arithmetic is fp32.
+ * engine: 0 = SIMT kernel. hd must be 32 or 64; T >= 1. */
+int gpt2k_attention_fwd(int dtype, const void* qkv, void* out, float* lse, int B, int T, int H, int hd,
+                        int engine, uint32_t* status_dev, void* stream);
+
+/* Backward of gpt2k_attention_fwd: dqkv (B, T, 3C) = [dq | dk | dv] from qkv,
+ * out, dout (B, T, C) and lse.
+ * workspace_dev: caller-owned scratch of B*H*T floats (D = rowsum(dout * out)).
+ * engine: 0 = SIMT kernel. */
+int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, const void* dout, const float* lse,
+                        void* dqkv, int B, int T, int H, int hd, float* workspace_dev, int engine,
+                        uint32_t* status_dev, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

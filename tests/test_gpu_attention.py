@@ -1,0 +1,68 @@
+"""Attention kernels through gpt2k_attention_fwd/bwd against the oracle's
+causal_attention / causal_attention_backward (float64, materialised T x T).
+
+Tolerances (max|gpu - ref| / max|ref| per tensor): fp32 1e-4; bf16 operands
+2e-2 (outputs and gradients are stored in bf16, 2^-8 relative)."""
+import numpy as np
+import pytest
+
+from oracle import gpt2_oracle as O
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+CASES = [(2, 64, 4, 32), (3, 37, 2, 64), (1, 1, 3, 64), (2, 200, 12, 64), (1, 1024, 2, 64)]
+
+
+def _heads(x, B, T, H, hd):
+    return x.reshape(B, T, H, hd).transpose(0, 2, 1, 3)
+
+
+def _merge(x, B, T, H, hd):
+    return x.transpose(0, 2, 1, 3).reshape(B, T, H * hd)
+
+
+def _rel(a, b):
+    return float(np.max(np.abs(a - b)) / max(np.max(np.abs(b)), 1e-30))
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("case", CASES)
+def test_attention_fwd_bwd_vs_oracle(dtype, case):
+    from decoder_only_transformer_sm_b200 import native
+    B, T, H, hd = case
+    C = H * hd
+    tdt = torch.float32 if dtype == "fp32" else torch.bfloat16
+    g = torch.Generator().manual_seed(B * 1000 + T * 10 + H)
+    qkv = torch.randn((B, T, 3 * C), generator=g).to(tdt).cuda()
+    dout = torch.randn((B, T, C), generator=g).to(tdt).cuda()
+    out = torch.empty((B, T, C), dtype=tdt, device="cuda")
+    lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
+    dqkv = torch.empty_like(qkv)
+    ws = torch.empty((B * H * T,), dtype=torch.float32, device="cuda")
+    st = native.attention_fwd(qkv, out, lse, B, T, H, hd)
+    native.attention_bwd(qkv, out, dout, lse, dqkv, B, T, H, hd, ws, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    x = qkv.float().cpu().numpy().astype(np.float64)
+    q, k, v = (_heads(x[..., i * C:(i + 1) * C], B, T, H, hd) for i in range(3))
+    y, p = O.causal_attention(q, k, v)
+    tol = 1e-4 if dtype == "fp32" else 2e-2
+    assert _rel(out.float().cpu().numpy(), _merge(y, B, T, H, hd)) < tol
+    ref_lse = np.log(np.sum(np.exp((q @ k.transpose(0, 1, 3, 2)) / np.sqrt(hd)
+                                   + np.triu(np.full((T, T), -np.inf), 1)), axis=-1))
+    assert np.max(np.abs(lse.cpu().numpy() - ref_lse)) < (1e-4 if dtype == "fp32" else 2e-2)
+    # backward against the oracle, fed the kernel's own (rounded) output gradient
+    do = _heads(dout.float().cpu().numpy().astype(np.float64), B, T, H, hd)
+    dq, dk, dv = O.causal_attention_backward(do, q, k, v, p)
+    got = dqkv.float().cpu().numpy()
+    for i, ref in enumerate((dq, dk, dv)):
+        assert _rel(got[..., i * C:(i + 1) * C], _merge(ref, B, T, H, hd)) < tol, i
+
+
+def test_attention_rejects_bad_head_width():
+    from decoder_only_transformer_sm_b200 import native
+    x = torch.zeros((1, 4, 3 * 48), device="cuda")
+    with pytest.raises(native.Gpt2Error):
+        native.attention_fwd(x, torch.zeros((1, 4, 48), device="cuda"), torch.zeros((1, 1, 4), device="cuda"),
+                             1, 4, 1, 48)
