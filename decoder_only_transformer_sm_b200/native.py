@@ -294,3 +294,18 @@ def attention_bwd(qkv, out, dout, lse, dqkv, B: int, T: int, H: int, hd: int, wo
                                               stream))
     return status
 
+
+def attention_bwd_noalloc(qkv, out, dout, lse, dqkv, B: int, T: int, H: int, hd: int, engine: int = 0,
+                          status=None, stream=None):
+    """gpt2k_attention_bwd_noalloc: the attention backward with the library's own
+    fixed scratch (B*H*T <= 262144), for callers that cannot allocate device memory."""
+    lib = load_library()
+    fn = lib.gpt2k_attention_bwd_noalloc
+    if fn.argtypes is None:
+        P, I = ctypes.c_void_p, ctypes.c_int
+        fn.restype = I
+        fn.argtypes = [I, P, P, P, P, P, I, I, I, I, I, P, P]
+    status, stream = _stream_and_status(qkv, status, stream)
+    _check(fn(_dtype_code(qkv), _ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dqkv), B, T, H, hd, engine,
+              _ptr(status), stream))
+    return status

@@ -82,6 +82,23 @@ int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, const void*
                         void* dqkv, int B, int T, int H, int hd, float* workspace_dev, int engine,
                         uint32_t* status_dev, void* stream);
 
+/* gpt2k_attention_bwd without a workspace argument, for callers that cannot
+ * allocate device memory (a framework whose caching allocator owns the GPU's
+ * memory, or a latency-critical loop where cudaMalloc's implicit device
+ * synchronisation is not allowed). The source pages have no counterpart: this
+ * is an interface variant, the arithmetic is that of gpt2k_attention_bwd.
+ * Scratch: a fixed 1 MiB device array inside the library (held by every GPU
+ * that loads the library until exit), so B*H*T must be <= 262144; larger
+ * sizes return GPT2_ERR_INVALID_ARG. The call allocates nothing. Its first
+ * call on a device, with that device current, looks up the array's device
+ * address (cudaGetSymbolAddress) and caches it; make that first call before
+ * any stream capture. Every call shares the array: calls that overlap on the
+ * GPU race, and must not be issued. Other arguments and errors as
+ * gpt2k_attention_bwd. */
+int gpt2k_attention_bwd_noalloc(int dtype, const void* qkv, const void* out, const void* dout, const float* lse,
+                                void* dqkv, int B, int T, int H, int hd, int engine, uint32_t* status_dev,
+                                void* stream);
+
 #ifdef __cplusplus
 }
 #endif
