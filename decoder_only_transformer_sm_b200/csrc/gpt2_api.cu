@@ -115,6 +115,7 @@ struct gpt2_handle {
     long long step_t = 0;
     long long launches = 0;
     bool use_tc_gemm = true;
+    bool use_tc_attention = true;
     std::string host_error;   // set by enqueue helpers that cannot report a status
 
     bool profiling = false;
@@ -345,6 +346,34 @@ void gemm(gpt2_handle* h, const char* site, GemmLayout layout, const void* a, co
          gemm_raw<A>(h, layout, a, b, M, N, K, ep));
 }
 
+// Attention dispatch: tensor-core kernels in bf16 mode, SIMT fp32 kernels in fp32 mode.
+template <typename A>
+void attn_fwd(gpt2_handle* h, const A* qkv, A* out, float* lse, int B, int T);
+template <>
+void attn_fwd<float>(gpt2_handle* h, const float* qkv, float* out, float* lse, int B, int T) {
+    launch_attention_fwd_simt<float>(h->ctx(), qkv, out, lse, B, T, h->H, h->hd);
+}
+template <>
+void attn_fwd<bf16>(gpt2_handle* h, const bf16* qkv, bf16* out, float* lse, int B, int T) {
+    if (h->use_tc_attention) launch_attention_fwd_mma(h->ctx(), qkv, out, lse, B, T, h->H, h->hd);
+    else launch_attention_fwd_simt<bf16>(h->ctx(), qkv, out, lse, B, T, h->H, h->hd);
+}
+template <typename A>
+void attn_bwd(gpt2_handle* h, const A* qkv, const A* out, const A* dout, const float* lse, A* dqkv, int B, int T);
+template <>
+void attn_bwd<float>(gpt2_handle* h, const float* qkv, const float* out, const float* dout, const float* lse,
+                     float* dqkv, int B, int T) {
+    launch_attention_bwd_simt<float>(h->ctx(), qkv, out, dout, lse, h->dpre, dqkv, B, T, h->H, h->hd);
+}
+template <>
+void attn_bwd<bf16>(gpt2_handle* h, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
+                    bf16* dqkv, int B, int T) {
+    if (h->use_tc_attention)
+        launch_attention_bwd_mma(h->ctx(), qkv, out, dout, lse, h->dpre, dqkv, B, T, h->H, h->hd);
+    else
+        launch_attention_bwd_simt<bf16>(h->ctx(), qkv, out, dout, lse, h->dpre, dqkv, B, T, h->H, h->hd);
+}
+
 Epilogue epi(int kind, void* out, long long ldo) {
     Epilogue e;
     e.kind = kind;
@@ -377,7 +406,7 @@ void forward_impl(gpt2_handle* h, const int* idx, const int* targets, int B, int
         e.bias = P + o.bqkv;
         gemm<A>(h, "gemm fwd c_attn", GEMM_NT, h->ln1[l], wop<A>(h, o.wqkv), BT, 3 * C, C, e);
         PROF("attention fwd", 0, 0, 0, att_fwd_flops, (double)BT * C * es * 4,
-             launch_attention_fwd_simt<A>(c, (const A*)h->qkv[l], (A*)h->att[l], h->lse[l], B, T, H, hd));
+             attn_fwd<A>(h, (const A*)h->qkv[l], (A*)h->att[l], h->lse[l], B, T));
         e = epi(EPI_BIAS_RESID, h->resid[2 * l + 1], C);
         e.bias = P + o.bproj;
         e.resid = h->resid[2 * l];
@@ -459,8 +488,8 @@ void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
                 epi(EPI_STORE, h->dO, C));
         // attention
         PROF("attention bwd", 0, 0, 0, att_bwd_flops, (double)BT * C * es * 8,
-             launch_attention_bwd_simt<A>(c, (const A*)h->qkv[l], (const A*)h->att[l], (const A*)h->dO, h->lse[l],
-                                          h->dpre, (A*)h->dqkv, B, T, H, hd));
+             attn_bwd<A>(h, (const A*)h->qkv[l], (const A*)h->att[l], (const A*)h->dO, h->lse[l], (A*)h->dqkv, B,
+                         T));
         PROF("bias colsum", 0, 0, 0, 0.0, (double)BT * 3 * C * es,
              launch_colsum<A>(c, (const A*)h->dqkv, BT, 3 * C, G + o.bqkv));
         // attn.c_attn
@@ -577,6 +606,7 @@ int gpt2_create(const gpt2_config* cfg, void* stream, gpt2_handle** out) {
     h->V = cfg->vocab_size;
     h->maxBT = cfg->max_B * cfg->max_T;
     if (const char* e = getenv("GPT2_B200_SIMT_GEMM")) h->use_tc_gemm = (e[0] == '0');
+    if (const char* e = getenv("GPT2_B200_SIMT_ATTENTION")) h->use_tc_attention = (e[0] == '0');
     build_layout(h);
 
     auto cleanup_fail = [&](int code, const std::string& msg) {

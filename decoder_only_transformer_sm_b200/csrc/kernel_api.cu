@@ -59,7 +59,9 @@ int check_attention_args(int dtype, int B, int T, int H, int hd, int engine, con
     if (dtype != GPT2K_F32 && dtype != GPT2K_BF16) return set_error(GPT2_ERR_INVALID_ARG, "unknown dtype");
     if (B < 1 || T < 1 || H < 1) return set_error(GPT2_ERR_INVALID_ARG, "B, T, H must be >= 1");
     if (hd != 32 && hd != 64) return set_error(GPT2_ERR_INVALID_ARG, "head width must be 32 or 64");
-    if (engine != 0) return set_error(GPT2_ERR_INVALID_ARG, "unknown attention engine");
+    if (engine != 0 && engine != 1) return set_error(GPT2_ERR_INVALID_ARG, "unknown attention engine");
+    if (engine == 1 && dtype != GPT2K_BF16)
+        return set_error(GPT2_ERR_INVALID_ARG, "the tensor-core attention engine takes bf16 operands");
     if (!a || !b || !c || !status) return set_error(GPT2_ERR_INVALID_ARG, "NULL operand");
     return GPT2_OK;
 }
@@ -80,7 +82,9 @@ extern "C" int gpt2k_attention_fwd(int dtype, const void* qkv, void* out, float*
     if (rc) return rc;
     long long launches = 0;
     Ctx c = kctx(stream, status_dev, &launches);
-    if (dtype == GPT2K_F32)
+    if (engine == 1)
+        launch_attention_fwd_mma(c, (const bf16*)qkv, (bf16*)out, lse, B, T, H, hd);
+    else if (dtype == GPT2K_F32)
         launch_attention_fwd_simt<float>(c, (const float*)qkv, (float*)out, lse, B, T, H, hd);
     else
         launch_attention_fwd_simt<bf16>(c, (const bf16*)qkv, (bf16*)out, lse, B, T, H, hd);
@@ -97,7 +101,10 @@ extern "C" int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, 
     if (!lse || !dqkv || !workspace_dev) return set_error(GPT2_ERR_INVALID_ARG, "NULL operand");
     long long launches = 0;
     Ctx c = kctx(stream, status_dev, &launches);
-    if (dtype == GPT2K_F32)
+    if (engine == 1)
+        launch_attention_bwd_mma(c, (const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, workspace_dev,
+                                 (bf16*)dqkv, B, T, H, hd);
+    else if (dtype == GPT2K_F32)
         launch_attention_bwd_simt<float>(c, (const float*)qkv, (const float*)out, (const float*)dout, lse,
                                          workspace_dev, (float*)dqkv, B, T, H, hd);
     else

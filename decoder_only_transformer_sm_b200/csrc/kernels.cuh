@@ -97,6 +97,12 @@ template <typename T>
 void launch_attention_bwd_simt(const Ctx& ctx, const T* qkv, const T* out, const T* dout, const float* lse,
                                float* dpre /* (B,H,T) scratch */, T* dqkv, int B, int Tn, int H, int hd);
 
+// Tensor-core flash attention (mma.sync m16n8k16, bf16 operands, fp32 softmax).
+void launch_attention_fwd_mma(const Ctx& ctx, const bf16* qkv, bf16* out, float* lse, int B, int Tn, int H,
+                              int hd);
+void launch_attention_bwd_mma(const Ctx& ctx, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
+                              float* dpre, bf16* dqkv, int B, int Tn, int H, int hd);
+
 // ----------------------------------------------------------------------------
 // Optimiser and parameter utilities.
 // ----------------------------------------------------------------------------

@@ -70,14 +70,16 @@ int gpt2k_matmul_bf16(int layout, const void* A, const void* B, int M, int N, in
  * out  : (B, T, C), heads concatenated in head order.
  * lse  : (B, H, T) fp32 log-sum-exp of each softmax row (for the backward).
  * dtype: GPT2K_F32 or GPT2K_BF16 (qkv, out); arithmetic is fp32.
- * engine: 0 = SIMT kernel. hd must be 32 or 64; T >= 1. */
+ * engine: 0 = SIMT kernel (fp32 arithmetic throughout); 1 = tensor-core flash
+ *         kernel (bf16 only: mma.sync bf16 products, fp32 accumulation and
+ *         softmax). hd must be 32 or 64; T >= 1. */
 int gpt2k_attention_fwd(int dtype, const void* qkv, void* out, float* lse, int B, int T, int H, int hd,
                         int engine, uint32_t* status_dev, void* stream);
 
 /* Backward of gpt2k_attention_fwd: dqkv (B, T, 3C) = [dq | dk | dv] from qkv,
  * out, dout (B, T, C) and lse.
  * workspace_dev: caller-owned scratch of B*H*T floats (D = rowsum(dout * out)).
- * engine: 0 = SIMT kernel. */
+ * engine: 0 = SIMT kernel; 1 = tensor-core kernels (bf16 only). */
 int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, const void* dout, const float* lse,
                         void* dqkv, int B, int T, int H, int hd, float* workspace_dev, int engine,
                         uint32_t* status_dev, void* stream);

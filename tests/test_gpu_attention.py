@@ -23,12 +23,13 @@ def _merge(x, B, T, H, hd):
 
 
 def _rel(a, b):
-    return float(np.max(np.abs(a - b)) / max(np.max(np.abs(b)), 1e-30))
+    # floor 1e-3 (inputs are O(1)): at T = 1 the exact dQ is identically zero
+    return float(np.max(np.abs(a - b)) / max(np.max(np.abs(b)), 1e-3))
 
 
-@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("dtype,engine", [("fp32", 0), ("bf16", 0), ("bf16", 1)])
 @pytest.mark.parametrize("case", CASES)
-def test_attention_fwd_bwd_vs_oracle(dtype, case):
+def test_attention_fwd_bwd_vs_oracle(dtype, engine, case):
     from decoder_only_transformer_sm_b200 import native
     B, T, H, hd = case
     C = H * hd
@@ -40,8 +41,8 @@ def test_attention_fwd_bwd_vs_oracle(dtype, case):
     lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
     dqkv = torch.empty_like(qkv)
     ws = torch.empty((B * H * T,), dtype=torch.float32, device="cuda")
-    st = native.attention_fwd(qkv, out, lse, B, T, H, hd)
-    native.attention_bwd(qkv, out, dout, lse, dqkv, B, T, H, hd, ws, status=st)
+    st = native.attention_fwd(qkv, out, lse, B, T, H, hd, engine=engine)
+    native.attention_bwd(qkv, out, dout, lse, dqkv, B, T, H, hd, ws, engine=engine, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     x = qkv.float().cpu().numpy().astype(np.float64)
