@@ -78,6 +78,36 @@ __device__ __forceinline__ float gelu_tanh_grad(float u) {
     return 0.5f * (1.0f + t) + 0.5f * u * (1.0f - t * t) * c * (1.0f + 3.0f * 0.044715f * u * u);
 }
 
+// The same GELU through the logistic identity 0.5 (1 + tanh z) = 1 / (1 + e^(-2z)):
+// gelu(u) = u * s with s = sigmoid(2z), z = sqrt(2/pi) (u + 0.044715 u^3), and
+// gelu'(u) = s + 2 u s (1 - s) sqrt(2/pi) (1 + 3 * 0.044715 u^2) since
+// 1 - tanh(z)^2 = 4 s (1 - s). One exponential and one reciprocal, no
+// cancellation in either tail. Used where the result is stored in bf16.
+__device__ __forceinline__ float rcp_approx(float x) {   // hardware reciprocal (rcp.approx), 1/inf = 0
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float gelu_sigmoid_s(float u) {
+    const float c = 0.7978845608028654f;
+    const float z = c * fmaf(0.044715f * u, u * u, u);
+    return rcp_approx(1.0f + __expf(-2.0f * z));
+}
+__device__ __forceinline__ float gelu_fast(float u) { return u * gelu_sigmoid_s(u); }
+__device__ __forceinline__ float gelu_fast_grad(float u) {
+    const float c = 0.7978845608028654f;
+    const float s = gelu_sigmoid_s(u);
+    return fmaf(2.0f * u * s * (1.0f - s) * c, fmaf(3.0f * 0.044715f * u, u, 1.0f), s);
+}
+// GELU and its derivative for an output element type: exact tanh form for fp32
+// results, the logistic form for bf16 results.
+template <typename T> __device__ __forceinline__ float gelu_for(float u);
+template <> __device__ __forceinline__ float gelu_for<float>(float u) { return gelu_tanh(u); }
+template <> __device__ __forceinline__ float gelu_for<bf16>(float u) { return gelu_fast(u); }
+template <typename T> __device__ __forceinline__ float gelu_grad_for(float u);
+template <> __device__ __forceinline__ float gelu_grad_for<float>(float u) { return gelu_tanh_grad(u); }
+template <> __device__ __forceinline__ float gelu_grad_for<bf16>(float u) { return gelu_fast_grad(u); }
+
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ long long ceil_div_ll(long long a, long long b) { return (a + b - 1) / b; }
 

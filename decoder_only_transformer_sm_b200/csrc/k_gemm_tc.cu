@@ -1,20 +1,26 @@
-// Tensor-core GEMM for sm_100a: TMA loads into a multi-stage shared-memory
-// ring, tcgen05.mma (kind::f16, bf16 operands) issued by one thread into an
-// fp32 accumulator in tensor memory, and an epilogue that reads the
-// accumulator with tcgen05.ld and applies the fused bias / GELU / residual /
-// dGELU / fp32-accumulate step while storing.
+// Persistent tensor-core GEMM for sm_100a.
+//
+// One CTA per SM walks a static list of work units (output tile x K split).
+// Warp 0 streams A/B k-blocks with TMA into a 4-stage shared-memory ring that
+// runs continuously across units; warp 1 issues tcgen05.mma (kind::f16, bf16
+// operands, M=128, N=256, K=16) from one thread into one of two fp32
+// accumulators in tensor memory (2 x 256 columns = all 512); warps 2..9 read
+// the other accumulator with tcgen05.ld and run the fused epilogue while the
+// next unit's MMAs proceed, then hand the accumulator back. Each epilogue warp
+// turns its rows around in a private swizzled shared-memory buffer so that
+// results and epilogue inputs move through global memory as whole 128-byte rows.
 //
 // All three operand layouts of the training step run on the same kernel:
 //   NT (forward, y = x W^T):   A K-major,  B K-major
 //   NN (dgrad,   dx = dy W):   A K-major,  B N-major
 //   TN (wgrad,   dW = dy^T x): A M-major,  B N-major
 // MN-major operands are loaded as 64-element-wide boxes (one 128-byte swizzle
-// row per k) and described to the MMA as MN-major; no operand is transposed
-// in memory.
-//
-// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and
-// MMA issuer, warps 2..5 = epilogue (TMEM lane quarter = warp % 4).
+// row per k) and described to the MMA as MN-major; no operand is transposed in
+// memory. Skinny weight-gradient shapes are split along K; their partial sums
+// are added to the fp32 gradient with atomics.
 #include <cudaTypedefs.h>
+
+#include <cstring>
 
 #include "epilogue.cuh"
 #include "tc_ptx.cuh"
@@ -23,46 +29,182 @@ namespace gpt2 {
 
 namespace {
 
-constexpr int BM = 128, BN = 128, BK = 64, STAGES = 3;   // 2 CTAs per SM
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
-constexpr int B_BYTES = BN * BK * 2;   // 16 KB
+constexpr int B_BYTES = BN * BK * 2;   // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int THREADS = 192;
-constexpr int MN_BOX_BYTES = 64 * BK * 2;   // one 64-wide MN-major box: 8 KB
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;   // 320
+constexpr int MN_BOX_BYTES = 64 * BK * 2;       // one 64-wide MN-major box: 8 KB
+constexpr int TMEM_COLS = 2 * BN;               // two accumulators
+constexpr int EBUF = 4096;                      // per epilogue warp: 32 rows x 128 bytes
+constexpr int EPI_BYTES = EPI_WARPS * EBUF;
 
 struct Ctl {
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
-    uint64_t accum;
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t drain;
     uint32_t tmem_base;
     uint32_t abort;
 };
 
-constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + sizeof(Ctl);
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + EPI_BYTES + 1024 + sizeof(Ctl);
 
-template <int A_MN, int B_MN>
-__global__ void __launch_bounds__(THREADS, 2)
+// Byte offset of 16-byte segment c (0..7) of row r (0..31) in a warp's chunk
+// buffer of 128-byte rows; the XOR keeps both access patterns (a lane per
+// row, and eight lanes per row) free of bank conflicts.
+__device__ __forceinline__ uint32_t swz(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
+
+struct Units {
+    int tiles_m, tiles_n, splits, kb_total, kb_per_split;
+    __device__ __forceinline__ int count() const { return tiles_m * tiles_n * splits; }
+    // unit -> (m block, n block, first and end k-block); n fastest, then m, then split
+    __device__ __forceinline__ void decode(int u, int& mb, int& nb, int& kb0, int& kb1) const {
+        nb = u % tiles_n;
+        mb = (u / tiles_n) % tiles_m;
+        const int s = u / (tiles_n * tiles_m);
+        kb0 = s * kb_per_split;
+        kb1 = min(kb_total, kb0 + kb_per_split);
+    }
+};
+
+// One chunk of the epilogue for the calling warp: rows row0 .. row0+31 (lane =
+// row of acc) by CW columns from col0, CW = 64 for bf16 results and 32 for fp32
+// results, i.e. 128 bytes per row. Results (and the residual / GELU' inputs,
+// which have the same shape as the result) pass through the warp's
+// shared-memory buffer, so global memory is read and written in whole 128-byte
+// rows, four rows per instruction; each lane updates its row's 16-byte
+// segments in place in the buffer.
+template <int KIND>
+__device__ __forceinline__ void epilogue_chunk(const Epilogue& ep, float* acc, int row0, int col0, int M, int N,
+                                               uint8_t* buf) {
+    constexpr bool F32 = (KIND == EPI_BIAS_RESID || KIND == EPI_ACCUM_F32);
+    constexpr int EPS = F32 ? 4 : 8;           // elements per 16-byte segment
+    constexpr int ES = F32 ? 4 : 2;            // element size
+    constexpr int kind = KIND;
+    const int lane = threadIdx.x & 31;
+    const int lrow = lane >> 3, lseg = lane & 7;   // copy pattern: 8 lanes per row, 4 rows per step
+    constexpr bool has_in = (kind == EPI_BIAS_RESID || kind == EPI_DGELU);
+    constexpr bool has_bias = (kind == EPI_BIAS || kind == EPI_BIAS_GELU || kind == EPI_BIAS_RESID);
+    if (has_in) {
+        const char* src = kind == EPI_BIAS_RESID ? reinterpret_cast<const char*>(ep.resid)
+                                                 : reinterpret_cast<const char*>(ep.aux);
+#pragma unroll
+        for (int st = 0; st < 8; ++st) {
+            const int r = st * 4 + lrow;
+            const int c = col0 + lseg * EPS;
+            uint4 q = make_uint4(0, 0, 0, 0);
+            if (row0 + r < M && c < N) q = *reinterpret_cast<const uint4*>(src + ((long long)(row0 + r) * ep.ldo + c) * ES);
+            *reinterpret_cast<uint4*>(buf + swz(r, lseg)) = q;
+        }
+        __syncwarp();
+    }
+    constexpr int npass = kind == EPI_BIAS_GELU ? 2 : 1;   // GELU: u (out2), then gelu(u) (out)
+#pragma unroll
+    for (int pass = 0; pass < npass; ++pass) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            float* x = acc + c * EPS;
+            float in[EPS], b[EPS];
+            if (has_in) {
+                if (F32) {
+                    const float4 q = *reinterpret_cast<const float4*>(buf + swz(lane, c));
+                    in[0] = q.x; in[1] = q.y; in[2] = q.z; in[3] = q.w;
+                } else {
+                    load8(reinterpret_cast<const bf16*>(buf + swz(lane, c)), in);
+                }
+            }
+            if (has_bias && pass == 0) {
+#pragma unroll
+                for (int g = 0; g < EPS / 4; ++g) {
+                    float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (col0 + c * EPS + 4 * g < N) q = *reinterpret_cast<const float4*>(ep.bias + col0 + c * EPS + 4 * g);
+                    b[4 * g] = q.x; b[4 * g + 1] = q.y; b[4 * g + 2] = q.z; b[4 * g + 3] = q.w;
+                }
+            }
+            float v[EPS];
+#pragma unroll
+            for (int j = 0; j < EPS; ++j) {
+                switch (kind) {
+                case EPI_BIAS: v[j] = x[j] + b[j]; break;
+                case EPI_BIAS_GELU:
+                    if (pass == 0) {
+                        x[j] = __bfloat162float(__float2bfloat16_rn(x[j] + b[j]));   // u as stored
+                        v[j] = x[j];
+                    } else {
+                        v[j] = gelu_fast(x[j]);
+                    }
+                    break;
+                case EPI_BIAS_RESID: v[j] = in[j] + (x[j] + b[j]); break;
+                case EPI_DGELU: v[j] = x[j] * gelu_fast_grad(in[j]); break;
+                default: v[j] = x[j]; break;
+                }
+            }
+            if (F32) {
+                *reinterpret_cast<float4*>(buf + swz(lane, c)) = make_float4(v[0], v[1], v[2], v[3]);
+            } else {
+                store8(reinterpret_cast<bf16*>(buf + swz(lane, c)), v);
+            }
+        }
+        __syncwarp();
+        // whole rows out to global memory
+        char* dst = reinterpret_cast<char*>((kind == EPI_BIAS_GELU && pass == 0) ? ep.out2 : ep.out);
+#pragma unroll
+        for (int st = 0; st < 8; ++st) {
+            const int r = st * 4 + lrow;
+            const int c = col0 + lseg * EPS;
+            if (row0 + r < M && c < N) {
+                const uint4 q = *reinterpret_cast<const uint4*>(buf + swz(r, lseg));
+                char* gp = dst + ((long long)(row0 + r) * ep.ldo + c) * ES;
+                if (F32 && kind == EPI_ACCUM_F32) {
+                    float4 a = *reinterpret_cast<const float4*>(&q);
+                    if (ep.split_atomic) {
+                        atomicAdd(reinterpret_cast<float4*>(gp), a);
+                    } else {
+                        if (ep.beta != 0.f) {
+                            const float4 o = *reinterpret_cast<const float4*>(gp);
+                            a.x += ep.beta * o.x; a.y += ep.beta * o.y; a.z += ep.beta * o.z; a.w += ep.beta * o.w;
+                        }
+                        *reinterpret_cast<float4*>(gp) = a;
+                    }
+                } else {
+                    *reinterpret_cast<uint4*>(gp) = q;
+                }
+            }
+        }
+        __syncwarp();
+    }
+}
+
+template <int A_MN, int B_MN, int KIND>
+__global__ void __launch_bounds__(THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
-                   int K, Epilogue ep, unsigned* status) {
+                   Units units, Epilogue ep, unsigned* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
+    uint8_t* epi_smem = smem + STAGES * STAGE_BYTES;
+    Ctl* ctl = reinterpret_cast<Ctl*>(epi_smem + EPI_BYTES);
     volatile uint32_t* abort = &ctl->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
-    const int num_kb = (K + BK - 1) / BK;
+    const int n_units = units.count();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             tc::mbar_init(&ctl->full[s], 1);
             tc::mbar_init(&ctl->empty[s], 1);
         }
-        tc::mbar_init(&ctl->accum, 1);
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(&ctl->acc_full[b], 1);
+            tc::mbar_init(&ctl->acc_empty[b], EPI_WARPS);
+        }
+        tc::mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
         tc::fence_barrier_init();
     }
     if (warp == 1) {
-        tc::tmem_alloc(&ctl->tmem_base, BN);
+        tc::tmem_alloc(&ctl->tmem_base, TMEM_COLS);
         tc::tmem_relinquish();
     }
     tc::fence_before_sync();
@@ -70,74 +212,120 @@ __global__ void __launch_bounds__(THREADS, 2)
     tc::fence_after_sync();
     const uint32_t tmem = ctl->tmem_base;
 
-    if (warp == 0 && lane == 0) {
-        // ---------------------------------------------------------- producer
-        tc::tma_prefetch_desc(&tmA);
-        tc::tma_prefetch_desc(&tmB);
-        for (int kb = 0; kb < num_kb; ++kb) {
-            const int s = kb % STAGES;
-            const uint32_t ph = (kb / STAGES) & 1;
-            if (!tc::mbar_wait(&ctl->empty[s], ph ^ 1, abort, status)) break;
-            tc::mbar_expect_tx(&ctl->full[s], STAGE_BYTES);
-            uint8_t* sa = smem + s * STAGE_BYTES;
-            uint8_t* sb = sa + A_BYTES;
-            const int k0 = kb * BK;
-            if (A_MN) {
-                tc::tma_load_2d(sa, &tmA, m0, k0, &ctl->full[s]);
-                tc::tma_load_2d(sa + MN_BOX_BYTES, &tmA, m0 + 64, k0, &ctl->full[s]);
-            } else {
-                tc::tma_load_2d(sa, &tmA, k0, m0, &ctl->full[s]);
-            }
-            if (B_MN) {
-                tc::tma_load_2d(sb, &tmB, n0, k0, &ctl->full[s]);
-                tc::tma_load_2d(sb + MN_BOX_BYTES, &tmB, n0 + 64, k0, &ctl->full[s]);
-            } else {
-                tc::tma_load_2d(sb, &tmB, k0, n0, &ctl->full[s]);
-            }
-        }
-    } else if (warp == 1 && lane == 0) {
-        // --------------------------------------------------------- MMA issue
-        constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN, A_MN, B_MN);
-        for (int kb = 0; kb < num_kb; ++kb) {
-            const int s = kb % STAGES;
-            const uint32_t ph = (kb / STAGES) & 1;
-            if (!tc::mbar_wait(&ctl->full[s], ph, abort, status)) break;
-            tc::fence_after_sync();
-            const uint32_t a_base = tc::smem_u32(smem + s * STAGE_BYTES);
-            const uint32_t b_base = a_base + A_BYTES;
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------------ producer
+            tc::tma_prefetch_desc(&tmA);
+            tc::tma_prefetch_desc(&tmB);
+            uint32_t it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+                int mb, nb, kb0, kb1;
+                units.decode(u, mb, nb, kb0, kb1);
+                const int m0 = mb * BM, n0 = nb * BN;
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!tc::mbar_wait(&ctl->empty[s], ph ^ 1, abort, status)) { ok = false; break; }
+                    tc::mbar_expect_tx(&ctl->full[s], STAGE_BYTES);
+                    uint8_t* sa = smem + s * STAGE_BYTES;
+                    uint8_t* sb = sa + A_BYTES;
+                    const int k0 = kb * BK;
+                    if (A_MN) {
+                        tc::tma_load_2d(sa, &tmA, m0, k0, &ctl->full[s]);
+                        tc::tma_load_2d(sa + MN_BOX_BYTES, &tmA, m0 + 64, k0, &ctl->full[s]);
+                    } else {
+                        tc::tma_load_2d(sa, &tmA, k0, m0, &ctl->full[s]);
+                    }
+                    if (B_MN) {
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-                // K-major: +32 bytes per 16-element k step inside the swizzle row;
-                // MN-major: +16 rows of 128 bytes.
-                const uint64_t da = A_MN ? tc::smem_desc_sw128(a_base + kk * 2048, MN_BOX_BYTES, 1024)
-                                         : tc::smem_desc_sw128(a_base + kk * 32, 16, 1024);
-                const uint64_t db = B_MN ? tc::smem_desc_sw128(b_base + kk * 2048, MN_BOX_BYTES, 1024)
-                                         : tc::smem_desc_sw128(b_base + kk * 32, 16, 1024);
-                tc::mma_bf16(tmem, da, db, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        for (int c = 0; c < BN / 64; ++c)
+                            tc::tma_load_2d(sb + c * MN_BOX_BYTES, &tmB, n0 + 64 * c, k0, &ctl->full[s]);
+                    } else {
+                        tc::tma_load_2d(sb, &tmB, k0, n0, &ctl->full[s]);
+                    }
+                }
             }
-            tc::mma_commit(&ctl->empty[s]);   // stage free once these MMAs finish
         }
-        tc::mma_commit(&ctl->accum);          // accumulator complete (also after an abort)
-    } else if (warp >= 2) {
-        // ---------------------------------------------------------- epilogue
-        uint32_t ok = 0;
-        if (lane == 0) ok = tc::mbar_wait(&ctl->accum, 0, abort, status) ? 1u : 0u;
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (ok) {
-            tc::fence_after_sync();
-            const int quarter = warp & 3;
-            const int row = m0 + quarter * 32 + lane;
-#pragma unroll 1
-            for (int c = 0; c < BN; c += 32) {
-                float acc[32];
-                tc::tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, acc);
-                if (row < M && n0 + c < N) epilogue_run<bf16, 32>(ep, row, n0 + c, N, acc);
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ----------------------------------------------------- MMA issue
+            constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN, A_MN, B_MN);
+            uint32_t it = 0, acc_it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++acc_it) {
+                int mb, nb, kb0, kb1;
+                units.decode(u, mb, nb, kb0, kb1);
+                const uint32_t ab = acc_it & 1, aph = (acc_it >> 1) & 1;
+                if (!tc::mbar_wait(&ctl->acc_empty[ab], aph ^ 1, abort, status)) break;
+                tc::fence_after_sync();
+                const uint32_t d_tmem = tmem + ab * BN;
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!tc::mbar_wait(&ctl->full[s], ph, abort, status)) { ok = false; break; }
+                    tc::fence_after_sync();
+                    const uint32_t a_base = tc::smem_u32(smem + s * STAGE_BYTES);
+                    const uint32_t b_base = a_base + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        // K-major: +32 bytes per 16-element k step inside the swizzle row;
+                        // MN-major: +16 rows of 128 bytes.
+                        const uint64_t da = A_MN ? tc::smem_desc_sw128(a_base + kk * 2048, MN_BOX_BYTES, 1024)
+                                                 : tc::smem_desc_sw128(a_base + kk * 32, 16, 1024);
+                        const uint64_t db = B_MN ? tc::smem_desc_sw128(b_base + kk * 2048, MN_BOX_BYTES, 1024)
+                                                 : tc::smem_desc_sw128(b_base + kk * 32, 16, 1024);
+                        tc::mma_bf16(d_tmem, da, db, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc::mma_commit(&ctl->empty[s]);   // stage free once these MMAs finish
+                }
+                tc::mma_commit(&ctl->acc_full[ab]);    // accumulator ready for the epilogue
             }
+            // every MMA issued by this thread has completed once `drain` fires; this
+            // wait ignores an abort (it must not free TMEM under running MMAs) but is
+            // still bounded in time
+            volatile uint32_t no_abort = 0;
+            tc::mma_commit(&ctl->drain);
+            tc::mbar_wait(&ctl->drain, 0, &no_abort, status);
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue
+        const int ew = warp - 2;                 // 0..7
+        const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
+        const int col_half = ew >> 2;            // columns [half*BN/2, half*BN/2 + BN/2)
+        uint8_t* buf = epi_smem + ew * EBUF;
+        constexpr bool f32_out = (KIND == EPI_BIAS_RESID || KIND == EPI_ACCUM_F32);
+        uint32_t acc_it = 0;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++acc_it) {
+            int mb, nb, kb0, kb1;
+            units.decode(u, mb, nb, kb0, kb1);
+            const uint32_t ab = acc_it & 1, aph = (acc_it >> 1) & 1;
+            uint32_t ok = 0;
+            if (lane == 0) ok = tc::mbar_wait(&ctl->acc_full[ab], aph, abort, status) ? 1u : 0u;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc::fence_after_sync();
+            const int row0 = mb * BM + quarter * 32;
+            const int cbase = col_half * (BN / 2);
+            const uint32_t taddr = tmem + ab * BN + cbase + ((uint32_t)(quarter * 32) << 16);
+            constexpr int CW = f32_out ? 32 : 64;   // columns per chunk (128 bytes of results per row)
+#pragma unroll 1
+            for (int c = 0; c < BN / 2; c += CW) {
+                const int col0 = nb * BN + cbase + c;
+                if (col0 >= N) break;
+                float acc[CW];
+                tc::tmem_ld_32x32b_x32(taddr + (uint32_t)c, acc);
+                if (CW == 64) tc::tmem_ld_32x32b_x32(taddr + (uint32_t)c + 32, acc + 32);
+                if (row0 < M) epilogue_chunk<KIND>(ep, acc, row0, col0, M, N, buf);
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&ctl->acc_empty[ab]);
         }
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 1) tc::tmem_dealloc(tmem, BN);
+    if (warp == 1) tc::tmem_dealloc(tmem, TMEM_COLS);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -152,31 +340,85 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// Row-major bf16 matrix [rows][cols]; box = box_cols (inner, 64 = 128 B) x box_rows.
-bool make_map(CUtensorMap* m, const bf16* ptr, long long rows, long long cols, int box_cols, int box_rows) {
+// Row-major matrix [rows][cols] with row stride ld (elements); box = box_cols
+// (inner) x box_rows.
+bool make_map_t(CUtensorMap* m, const void* ptr, bool f32, long long rows, long long cols, long long ld,
+                int box_cols, int box_rows, CUtensorMapSwizzle sw) {
     auto fn = encode_fn();
     if (!fn) return false;
+    const int es = f32 ? 4 : 2;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * es};
     cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<bf16*>(ptr), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                    const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-template <int A_MN, int B_MN>
-void launch_variant(const Ctx& ctx, const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
-                    const Epilogue& ep) {
+// Operand map: bf16 [rows][cols], 128-byte swizzle, 64-element inner box.
+bool make_map(CUtensorMap* m, const bf16* ptr, long long rows, long long cols, int box_cols, int box_rows) {
+    return make_map_t(m, ptr, false, rows, cols, cols, box_cols, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+int g_num_sms = 0;
+
+template <int A_MN, int B_MN, int KIND>
+void launch_kernel(dim3 grid, cudaStream_t stream, const CUtensorMap& ta, const CUtensorMap& tb, int M, int N,
+                   const Units& u, const Epilogue& ep, unsigned* status) {
     static bool configured = false;
     if (!configured) {
-        cudaFuncSetAttribute(gemm_tc_kernel<A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(gemm_tc_kernel<A_MN, B_MN, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES);
         configured = true;
     }
-    dim3 grid(ceil_div(N, BN), ceil_div(M, BM));
-    gemm_tc_kernel<A_MN, B_MN><<<grid, THREADS, SMEM_BYTES, ctx.stream>>>(ta, tb, M, N, K, ep, ctx.status);
+    gemm_tc_kernel<A_MN, B_MN, KIND><<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, M, N, u, ep, status);
+}
+
+template <int A_MN, int B_MN>
+bool launch_variant(const Ctx& ctx, const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
+                    Epilogue ep) {
+    if (g_num_sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (g_num_sms <= 0) g_num_sms = 148;
+    }
+    Units u;
+    u.tiles_m = ceil_div(M, BM);
+    u.tiles_n = ceil_div(N, BN);
+    u.kb_total = ceil_div(K, BK);
+    u.splits = 1;
+    const int tiles = u.tiles_m * u.tiles_n;
+    // Split K when the output has too few tiles to fill the GPU and the epilogue
+    // accumulates into fp32 (partials are then added with atomics).
+    if (ep.kind == EPI_ACCUM_F32 && ep.beta == 1.f && tiles < g_num_sms) {
+        int s = (2 * g_num_sms + tiles / 2) / tiles;
+        s = min(s, max(1, u.kb_total / 8));
+        u.splits = max(1, s);
+    }
+    u.kb_per_split = ceil_div(u.kb_total, u.splits);
+    u.splits = ceil_div(u.kb_total, u.kb_per_split);
+    if (u.splits > 1) ep.split_atomic = 1;
+    const int n_units = tiles * u.splits;
+    const dim3 grid(min(n_units, g_num_sms));
+    switch (ep.kind) {
+    case EPI_STORE: launch_kernel<A_MN, B_MN, EPI_STORE>(grid, ctx.stream, ta, tb, M, N, u, ep, ctx.status); break;
+    case EPI_BIAS: launch_kernel<A_MN, B_MN, EPI_BIAS>(grid, ctx.stream, ta, tb, M, N, u, ep, ctx.status); break;
+    case EPI_BIAS_GELU:
+        launch_kernel<A_MN, B_MN, EPI_BIAS_GELU>(grid, ctx.stream, ta, tb, M, N, u, ep, ctx.status);
+        break;
+    case EPI_BIAS_RESID:
+        launch_kernel<A_MN, B_MN, EPI_BIAS_RESID>(grid, ctx.stream, ta, tb, M, N, u, ep, ctx.status);
+        break;
+    case EPI_DGELU: launch_kernel<A_MN, B_MN, EPI_DGELU>(grid, ctx.stream, ta, tb, M, N, u, ep, ctx.status); break;
+    case EPI_ACCUM_F32:
+        launch_kernel<A_MN, B_MN, EPI_ACCUM_F32>(grid, ctx.stream, ta, tb, M, N, u, ep, ctx.status);
+        break;
+    default: return false;
+    }
+    return true;
 }
 
 }  // namespace
@@ -195,15 +437,15 @@ bool launch_gemm_tc(const Ctx& ctx, GemmLayout layout, const bf16* A, const bf16
     switch (layout) {
     case GEMM_NT:   // A [M][K], B [N][K]
         ok = make_map(&ta, A, M, K, 64, BM) && make_map(&tb, B, N, K, 64, BN);
-        if (ok) launch_variant<0, 0>(ctx, ta, tb, M, N, K, ep);
+        if (ok) ok = launch_variant<0, 0>(ctx, ta, tb, M, N, K, ep);
         break;
     case GEMM_NN:   // A [M][K], B [K][N]
         ok = make_map(&ta, A, M, K, 64, BM) && make_map(&tb, B, K, N, 64, BK);
-        if (ok) launch_variant<0, 1>(ctx, ta, tb, M, N, K, ep);
+        if (ok) ok = launch_variant<0, 1>(ctx, ta, tb, M, N, K, ep);
         break;
     default:        // GEMM_TN: A [K][M], B [K][N]
         ok = make_map(&ta, A, K, M, 64, BK) && make_map(&tb, B, K, N, 64, BK);
-        if (ok) launch_variant<1, 1>(ctx, ta, tb, M, N, K, ep);
+        if (ok) ok = launch_variant<1, 1>(ctx, ta, tb, M, N, K, ep);
         break;
     }
     if (ok) ++*ctx.launches;

@@ -43,6 +43,9 @@ extern "C" int gpt2k_matmul_bf16(int layout, const void* A, const void* B, int M
     if (engine == 1) {
         if (!gemm_tc_supported(L, M, N, K))
             return set_error(GPT2_ERR_INVALID_ARG, "shape not supported by the tensor-core GEMM");
+        if (ldo % 8 != 0) return set_error(GPT2_ERR_INVALID_ARG, "the tensor-core GEMM needs ldo % 8 == 0");
+        if (epilogue == GPT2K_EPI_ACCUM_F32 && beta != 0.f && beta != 1.f)
+            return set_error(GPT2_ERR_INVALID_ARG, "the tensor-core GEMM accumulates with beta 0 or 1");
         if (!launch_gemm_tc(c, L, (const bf16*)A, (const bf16*)B, M, N, K, e))
             return set_error(GPT2_ERR_CUDA, "tensor-map encoding failed");
     } else {

@@ -35,6 +35,7 @@ struct Epilogue {
     const float* resid = nullptr;  // EPI_BIAS_RESID input (ld = ldo)
     const void* aux = nullptr;     // EPI_DGELU pre-activation input (ld = ldo)
     float beta = 0.f;
+    int split_atomic = 0;          // EPI_ACCUM_F32 partial sums of a K split: atomicAdd into out
 };
 
 // Operand layouts of C[M,N] = sum_k A(m,k) B(n,k):

@@ -52,7 +52,8 @@ extern "C" {
  * aux         : bf16 [M, N] (stride ldo) pre-activation for GPT2K_EPI_DGELU, else NULL.
  * engine      : 1 = tcgen05 tensor cores (TMA + TMEM), 0 = SIMT fp32-FMA kernel.
  * Errors: INVALID_ARG (sizes < 1, unknown layout/epilogue, a required pointer
- * NULL, or engine 1 with K, N (or M for TN) not a multiple of 8). */
+ * NULL, or engine 1 with K, N, ldo (or M for TN) not a multiple of 8, or
+ * GPT2K_EPI_ACCUM_F32 with beta other than 0 or 1). */
 int gpt2k_matmul_bf16(int layout, const void* A, const void* B, int M, int N, int K, int epilogue, void* out,
                       int64_t ldo, void* out2, const float* bias, const float* resid, const void* aux, float beta,
                       int engine, uint32_t* status_dev, void* stream);
