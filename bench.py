@@ -305,7 +305,7 @@ def run_ours(args):
         peak = peaks.get("hbm_gbs")
         peak_note = f"hbm_gbs of {peak_src}"
     breakdown = []
-    for s in sites[:12]:
+    for s in sites:
         t = s["total_ms"] / args.steps
         row = {"site": s["name"], "ms_per_step": round(t, 4), "share": round(t / total_ms, 4),
                "launches_per_step": s["launches"] // args.steps}

@@ -14,6 +14,7 @@
 #include "gpt2.h"
 #include "kernels.cuh"
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -107,6 +108,7 @@ struct gpt2_handle {
     void* dqkv = nullptr;
     void* du = nullptr;
     float* dpre = nullptr;
+    float* red_scratch = nullptr;   // per-block partial column sums (LayerNorm bwd, bias grads)
     int* d_tokens = nullptr;
 
     DevScalars* d_sc = nullptr;
@@ -458,7 +460,7 @@ void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
     PROF("layernorm bwd", 0, 0, 0, 0.0, ln_bwd_bytes - 4.0 * BT * C,
          launch_layernorm_bwd<A>(c, (const A*)h->dtmp, h->resid[2 * L], h->ln_mean[2 * L], h->ln_rstd[2 * L],
                                  P + h->off_lnfw, nullptr, h->dres, (A*)h->dres_act, G + h->off_lnfw,
-                                 G + h->off_lnfb, G + h->lo[L - 1].bfcp, BT, C));
+                                 G + h->off_lnfb, G + h->lo[L - 1].bfcp, BT, C, h->red_scratch));
     for (int l = L - 1; l >= 0; --l) {
         const LayerOff& o = h->lo[l];
         // mlp.c_proj: dW += dY^T g ; du = (dY W) * gelu'(u)
@@ -469,7 +471,7 @@ void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
         e.aux = h->fch[l];
         gemm<A>(h, "gemm dgrad mlp.c_proj+dgelu", GEMM_NN, h->dres_act, wop<A>(h, o.wfcp), BT, 4 * C, C, e);
         PROF("bias colsum", 0, 0, 0, 0.0, (double)BT * 4 * C * es,
-             launch_colsum<A>(c, (const A*)h->du, BT, 4 * C, G + o.bfc));
+             launch_colsum<A>(c, (const A*)h->du, BT, 4 * C, G + o.bfc, h->red_scratch));
         // mlp.c_fc: dW += du^T ln2 ; dln2 = du W
         acc = epi(EPI_ACCUM_F32, G + o.wfc, C);
         acc.beta = 1.f;
@@ -479,7 +481,7 @@ void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
         PROF("layernorm bwd", 0, 0, 0, 0.0, ln_bwd_bytes,
              launch_layernorm_bwd<A>(c, (const A*)h->dtmp, h->resid[2 * l + 1], h->ln_mean[2 * l + 1],
                                      h->ln_rstd[2 * l + 1], P + o.ln2w, h->dres, h->dres, (A*)h->dres_act,
-                                     G + o.ln2w, G + o.ln2b, G + o.bproj, BT, C));
+                                     G + o.ln2w, G + o.ln2b, G + o.bproj, BT, C, h->red_scratch));
         // attn.c_proj
         acc = epi(EPI_ACCUM_F32, G + o.wproj, C);
         acc.beta = 1.f;
@@ -491,7 +493,7 @@ void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
              attn_bwd<A>(h, (const A*)h->qkv[l], (const A*)h->att[l], (const A*)h->dO, h->lse[l], (A*)h->dqkv, B,
                          T));
         PROF("bias colsum", 0, 0, 0, 0.0, (double)BT * 3 * C * es,
-             launch_colsum<A>(c, (const A*)h->dqkv, BT, 3 * C, G + o.bqkv));
+             launch_colsum<A>(c, (const A*)h->dqkv, BT, 3 * C, G + o.bqkv, h->red_scratch));
         // attn.c_attn
         acc = epi(EPI_ACCUM_F32, G + o.wqkv, C);
         acc.beta = 1.f;
@@ -502,7 +504,7 @@ void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
         PROF("layernorm bwd", 0, 0, 0, 0.0, ln_bwd_bytes,
              launch_layernorm_bwd<A>(c, (const A*)h->dtmp, h->resid[2 * l], h->ln_mean[2 * l], h->ln_rstd[2 * l],
                                      P + o.ln1w, h->dres, h->dres, (A*)h->dres_act, G + o.ln1w, G + o.ln1b,
-                                     l > 0 ? G + h->lo[l - 1].bfcp : nullptr, BT, C));
+                                     l > 0 ? G + h->lo[l - 1].bfcp : nullptr, BT, C, h->red_scratch));
     }
     PROF("embedding bwd", 0, 0, 0, 0.0, (double)BT * C * 12 + (double)T * C * 8,
          launch_embed_bwd(c, idx, h->dres, B, T, C, V, G + h->off_wte, G + h->off_wpe));
@@ -667,6 +669,11 @@ int gpt2_create(const gpt2_config* cfg, void* stream, gpt2_handle** out) {
     plan.push_back({&h->dqkv, BT * 3 * C * es});
     plan.push_back({&h->du, BT * 4 * C * es});
     plan.push_back({(void**)&h->dpre, BHT * 4});
+    {
+        const size_t ln_part = (size_t)ln_bwd_blocks(h->num_sms) * 3 * C;
+        const size_t cs_part = (size_t)colsum_row_blocks((int)BT) * 4 * C;
+        plan.push_back({(void**)&h->red_scratch, std::max(ln_part, cs_part) * 4});
+    }
     plan.push_back({(void**)&h->d_tokens, 2 * BT * 4});
     size_t total = 0;
     for (auto& p : plan) total += align_up(p.second);

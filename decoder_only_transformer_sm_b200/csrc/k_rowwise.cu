@@ -17,6 +17,7 @@ namespace {
 
 constexpr float LN_EPS = 1e-5f;
 
+
 // A row of C floats spread over one warp: lane l holds float4 chunks
 // l, l + 32, ..., i.e. columns 4*(l + 32 i) .. +3, for i < NV.
 template <int NV>
@@ -99,9 +100,8 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, c
                                                       const float* __restrict__ mean, const float* __restrict__ rstd,
                                                       const float* __restrict__ w, const float* dres_in,
                                                       float* dres_out, T* __restrict__ dres_act,
-                                                      float* __restrict__ dw, float* __restrict__ db,
-                                                      float* __restrict__ dbias_next, int rows, int C) {
-    extern __shared__ float red[];   // [3][C]
+                                                      float* __restrict__ partial, int rows, int C) {
+    extern __shared__ float red[];   // [3][C]: sum dy*xhat, sum dy, sum dres_out over this block's rows
     for (int i = threadIdx.x; i < 3 * C; i += blockDim.x) red[i] = 0.f;
     __syncthreads();
     const int lane = threadIdx.x & 31;
@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, c
 
     for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < rows; row += warps_total) {
         const float mu = mean[row], rs = rstd[row];
-        float g[NV][4], xh[NV][4], dxh[NV][4];
+        float g[NV][4], xh[NV][4], rin[NV][4];
         float s1 = 0.f, s2 = 0.f;
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
@@ -123,13 +123,15 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, c
                 float xx[4], ww[4];
                 load4(dy + (long long)row * C + c, g[i]);
                 load4(x + (long long)row * C + c, xx);
+                if (dres_in) load4(dres_in + (long long)row * C + c, rin[i]);
+                else rin[i][0] = rin[i][1] = rin[i][2] = rin[i][3] = 0.f;
                 load4(w + c, ww);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     xh[i][j] = (xx[j] - mu) * rs;
-                    dxh[i][j] = g[i][j] * ww[j];
-                    s1 += dxh[i][j];
-                    s2 += dxh[i][j] * xh[i][j];
+                    const float d = g[i][j] * ww[j];
+                    s1 += d;
+                    s2 += d * xh[i][j];
                 }
             }
         }
@@ -139,11 +141,11 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, c
         for (int i = 0; i < NV; ++i) {
             const int c = (lane + 32 * i) * 4;
             if (c < C) {
-                float o[4], r[4] = {0.f, 0.f, 0.f, 0.f};
-                if (dres_in) load4(dres_in + (long long)row * C + c, r);
+                float ww[4], o[4];
+                load4(w + c, ww);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    o[j] = rs * (dxh[i][j] - s1 - xh[i][j] * s2) + r[j];
+                    o[j] = rs * (g[i][j] * ww[j] - s1 - xh[i][j] * s2) + rin[i][j];
                     adw[i][j] += g[i][j] * xh[i][j];
                     adb[i][j] += g[i][j];
                     adn[i][j] += o[j];
@@ -166,10 +168,40 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, c
         }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < C; i += blockDim.x) {
-        atomicAdd(&dw[i], red[i]);
-        atomicAdd(&db[i], red[C + i]);
-        if (dbias_next) atomicAdd(&dbias_next[i], red[2 * C + i]);
+    float* part = partial + (long long)blockIdx.x * 3 * C;
+    for (int i = threadIdx.x; i < 3 * C; i += blockDim.x) part[i] = red[i];
+}
+
+// out_k[j] += sum over nblk partial rows of partial[b][k * n + j], k < n_out;
+// a null out_k is skipped. Block = 32 columns x 8 row groups: each thread sums
+// every 8th partial row of its column (coalesced across the warp), then the 8
+// group sums are added in a fixed order (deterministic).
+__global__ void __launch_bounds__(256) colred_finalize_kernel(const float* __restrict__ partial, int nblk, int n,
+                                                              int n_out, float* out0, float* out1, float* out2) {
+    __shared__ float part[8][33];
+    const int i = blockIdx.x * 32 + threadIdx.x;
+    const int stride = n * n_out;
+    float s = 0.f;
+    if (i < stride) {
+        int b = threadIdx.y;
+        for (; b + 24 < nblk; b += 32) {   // four independent loads in flight
+            const float a0 = partial[(long long)b * stride + i];
+            const float a1 = partial[(long long)(b + 8) * stride + i];
+            const float a2 = partial[(long long)(b + 16) * stride + i];
+            const float a3 = partial[(long long)(b + 24) * stride + i];
+            s += (a0 + a1) + (a2 + a3);
+        }
+        for (; b < nblk; b += 8) s += partial[(long long)b * stride + i];
+    }
+    part[threadIdx.y][threadIdx.x] = s;
+    __syncthreads();
+    if (threadIdx.y == 0 && i < stride) {
+        float t = 0.f;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) t += part[g][threadIdx.x];
+        const int k = i / n, j = i % n;
+        float* out = k == 0 ? out0 : (k == 1 ? out1 : out2);
+        if (out) out[j] += t;
     }
 }
 
@@ -193,9 +225,38 @@ __global__ void count_targets_kernel(const int* __restrict__ t, int n, int V, in
     }
 }
 
+// Eight consecutive elements (16 bytes of bf16, 32 of fp32).
+__device__ __forceinline__ void load8v(const float* p, float* v) { load4(p, v); load4(p + 4, v + 4); }
+__device__ __forceinline__ void load8v(const bf16* p, float* v) {
+    const uint4 q = *reinterpret_cast<const uint4*>(p);
+    const unsigned u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[j]));
+        v[2 * j] = f.x;
+        v[2 * j + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void store8v(float* p, const float* v) { store4(p, v); store4(p + 4, v + 4); }
+__device__ __forceinline__ void store8v(bf16* p, const float* v) {
+    uint4 q;
+    __nv_bfloat162 t[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) t[j] = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+    q.x = *reinterpret_cast<unsigned*>(&t[0]);
+    q.y = *reinterpret_cast<unsigned*>(&t[1]);
+    q.z = *reinterpret_cast<unsigned*>(&t[2]);
+    q.w = *reinterpret_cast<unsigned*>(&t[3]);
+    *reinterpret_cast<uint4*>(p) = q;
+}
+// exp for the softmax: CUDA's expf for fp32 logits, its fast __expf for bf16 logits.
+template <typename T> __device__ __forceinline__ float sm_exp(float x);
+template <> __device__ __forceinline__ float sm_exp<float>(float x) { return expf(x); }
+template <> __device__ __forceinline__ float sm_exp<bf16>(float x) { return __expf(x); }
+
 // One block per row. Pass 1: running max and sum of exp (online softmax) over
 // all V columns; pass 2 (write_grad): dlogits = (softmax - onehot) * scale / n_valid,
-// written in place; rows whose target is -1 get zeros.
+// written in place; rows whose target is -1 get zeros. V is a multiple of 8.
 template <typename T>
 __global__ void __launch_bounds__(512) classifier_kernel(T* logits, const int* __restrict__ targets, int V,
                                                           const int* __restrict__ n_valid, float scale,
@@ -207,13 +268,15 @@ __global__ void __launch_bounds__(512) classifier_kernel(T* logits, const int* _
     float lt = 0.f;
     if (threadIdx.x == 0 && valid) lt = to_f(lr[tgt]);
     float m = -INFINITY, s = 0.f;
-    for (int c = threadIdx.x * 4; c < V; c += blockDim.x * 4) {
-        float v[4];
-        load4(lr + c, v);
-        float mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
-        if (mx > m) { s *= expf(m - mx); m = mx; }
+    for (int c = threadIdx.x * 8; c < V; c += blockDim.x * 8) {
+        float v[8];
+        load8v(lr + c, v);
+        float mx = v[0];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) s += expf(v[j] - m);
+        for (int j = 1; j < 8; ++j) mx = fmaxf(mx, v[j]);
+        if (mx > m) { s *= sm_exp<T>(m - mx); m = mx; }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s += sm_exp<T>(v[j] - m);
     }
     // block reduction of (m, s)
     __shared__ float sm[32], ssum[32];
@@ -249,33 +312,48 @@ __global__ void __launch_bounds__(512) classifier_kernel(T* logits, const int* _
         atomicAdd(loss_accum, (double)scale * (double)(lse - lt) / (double)nv);
     if (!write_grad) return;
     const float gs = (valid && nv > 0) ? scale / (float)nv : 0.f;
-    for (int c = threadIdx.x * 4; c < V; c += blockDim.x * 4) {
-        float v[4];
-        load4(lr + c, v);
+    for (int c = threadIdx.x * 8; c < V; c += blockDim.x * 8) {
+        float v[8];
+        load8v(lr + c, v);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] = (expf(v[j] - lse) - (c + j == tgt ? 1.f : 0.f)) * gs;
-        store4(lr + c, v);
+        for (int j = 0; j < 8; ++j) v[j] = (sm_exp<T>(v[j] - lse) - (c + j == tgt ? 1.f : 0.f)) * gs;
+        store8v(lr + c, v);
     }
 }
 
+// Partial column sums of in[rows][cols] over blocks of rows: each thread owns 8
+// consecutive columns and walks the block's rows with 16-byte loads.
 template <typename T>
-__global__ void colsum_kernel(const T* __restrict__ in, int rows, int cols, int rows_per_block, float* out) {
-    // blockDim = (32, 8): threadIdx.x picks a column, threadIdx.y strides rows
-    __shared__ float part[8][33];
-    const int col = blockIdx.x * 32 + threadIdx.x;
+__global__ void colsum_partial_kernel(const T* __restrict__ in, int rows, int cols, int rows_per_block,
+                                      float* __restrict__ partial) {
+    const int col = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+    if (col >= cols) return;
     const int r0 = blockIdx.y * rows_per_block;
     const int r1 = min(rows, r0 + rows_per_block);
-    float s = 0.f;
-    if (col < cols)
-        for (int r = r0 + threadIdx.y; r < r1; r += 8) s += to_f(in[(long long)r * cols + col]);
-    part[threadIdx.y][threadIdx.x] = s;
-    __syncthreads();
-    if (threadIdx.y == 0 && col < cols) {
-        float t = 0.f;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int r = r0;
+    for (; r + 4 <= r1; r += 4) {   // four rows of loads in flight
+        float v[4][8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) t += part[i][threadIdx.x];
-        atomicAdd(&out[col], t);
+        for (int k = 0; k < 4; ++k) {
+            load4(in + (long long)(r + k) * cols + col, v[k]);
+            load4(in + (long long)(r + k) * cols + col + 4, v[k] + 4);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] += v[k][j];
     }
+    for (; r < r1; ++r) {
+        float v[8];
+        load4(in + (long long)r * cols + col, v);
+        load4(in + (long long)r * cols + col + 4, v + 4);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] += v[j];
+    }
+    float* p = partial + (long long)blockIdx.y * cols + col;
+    store4(p, acc);
+    store4(p + 4, acc + 4);
 }
 
 __global__ void embed_bwd_wte_kernel(const int* __restrict__ idx, const float* __restrict__ dx, int rows, int C,
@@ -342,15 +420,15 @@ void launch_layernorm_fwd(const Ctx& ctx, const float* x, const float* w, const 
 template <typename T>
 void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const float* mean, const float* rstd,
                           const float* w, const float* dres_in, float* dres_out, T* dres_act, float* dw,
-                          float* db, float* dbias_next, int rows, int C) {
+                          float* db, float* dbias_next, int rows, int C, float* scratch) {
     const int threads = 256;
-    const int blocks = min(ceil_div(rows, threads / 32), ctx.num_sms * 4);
+    const int blocks = min(ceil_div(rows, threads / 32), ln_bwd_blocks(ctx.num_sms));
     const size_t smem = 3 * C * sizeof(float);
     const int nv = ceil_div(C, 128);
 #define LNB_CASE(N)                                                                                      \
     case N:                                                                                              \
         ln_bwd_kernel<T, N><<<blocks, threads, smem, ctx.stream>>>(dy, x, mean, rstd, w, dres_in, dres_out, \
-                                                                   dres_act, dw, db, dbias_next, rows, C); \
+                                                                   dres_act, scratch, rows, C);            \
         break;
     switch (nv) {
         LNB_CASE(1) LNB_CASE(2) LNB_CASE(3) LNB_CASE(4) LNB_CASE(5) LNB_CASE(6) LNB_CASE(7)
@@ -359,7 +437,9 @@ void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const flo
         default: break;
     }
 #undef LNB_CASE
-    ++*ctx.launches;
+    colred_finalize_kernel<<<ceil_div(3 * C, 32), dim3(32, 8), 0, ctx.stream>>>(scratch, blocks, C, 3, dw, db,
+                                                                                 dbias_next);
+    *ctx.launches += 2;
 }
 
 void launch_count_targets(const Ctx& ctx, const int* targets, int n, int V, int* n_valid) {
@@ -375,11 +455,14 @@ void launch_classifier(const Ctx& ctx, T* logits, const int* targets, int rows, 
 }
 
 template <typename T>
-void launch_colsum(const Ctx& ctx, const T* in, int rows, int cols, float* out) {
-    const int rpb = 256;
-    dim3 grid(ceil_div(cols, 32), ceil_div(rows, rpb));
-    colsum_kernel<T><<<grid, dim3(32, 8), 0, ctx.stream>>>(in, rows, cols, rpb, out);
-    ++*ctx.launches;
+void launch_colsum(const Ctx& ctx, const T* in, int rows, int cols, float* out, float* scratch) {
+    const int nblk = colsum_row_blocks(rows);
+    const int rpb = ceil_div(rows, nblk);
+    dim3 grid(ceil_div(cols, 8 * 128), nblk);
+    colsum_partial_kernel<T><<<grid, 128, 0, ctx.stream>>>(in, rows, cols, rpb, scratch);
+    colred_finalize_kernel<<<ceil_div(cols, 32), dim3(32, 8), 0, ctx.stream>>>(scratch, nblk, cols, 1, out,
+                                                                               nullptr, nullptr);
+    *ctx.launches += 2;
 }
 
 void launch_embed_bwd(const Ctx& ctx, const int* idx, const float* dx, int B, int Tn, int C, int V, float* dwte,
@@ -397,9 +480,9 @@ void launch_embed_bwd(const Ctx& ctx, const int* idx, const float* dx, int B, in
                                           float*, int, int);                                                   \
     template void launch_layernorm_bwd<T>(const Ctx&, const T*, const float*, const float*, const float*,      \
                                           const float*, const float*, float*, T*, float*, float*, float*, int, \
-                                          int);                                                                \
+                                          int, float*);                                                        \
     template void launch_classifier<T>(const Ctx&, T*, const int*, int, int, const int*, float, double*, int); \
-    template void launch_colsum<T>(const Ctx&, const T*, int, int, float*);
+    template void launch_colsum<T>(const Ctx&, const T*, int, int, float*, float*);
 INST(float)
 INST(bf16)
 #undef INST

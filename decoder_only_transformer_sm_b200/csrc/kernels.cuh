@@ -69,11 +69,13 @@ void launch_layernorm_fwd(const Ctx& ctx, const float* x, const float* w, const 
                           float* rstd, int rows, int C);
 // dx = LN'(x)^T dy (+ dres_in); writes dres_out (fp32) and dres_act (operand copy);
 // accumulates dw += sum dy*xhat, db += sum dy and, if dbias_next != null,
-// dbias_next += sum_rows dres_out.
+// dbias_next += sum_rows dres_out. Column sums go through per-block partials in
+// scratch (ln_bwd_blocks(num_sms) x 3C floats) and a fixed-order finalize.
+inline int ln_bwd_blocks(int num_sms) { return 2 * num_sms; }
 template <typename T>
 void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const float* mean, const float* rstd,
                           const float* w, const float* dres_in, float* dres_out, T* dres_act, float* dw,
-                          float* db, float* dbias_next, int rows, int C);
+                          float* db, float* dbias_next, int rows, int C, float* scratch);
 
 // Count targets != -1 (and flag out-of-range targets) into *n_valid.
 void launch_count_targets(const Ctx& ctx, const int* targets, int n, int V, int* n_valid);
@@ -82,9 +84,11 @@ void launch_count_targets(const Ctx& ctx, const int* targets, int n, int V, int*
 template <typename T>
 void launch_classifier(const Ctx& ctx, T* logits, const int* targets, int rows, int V, const int* n_valid,
                        float scale, double* loss_accum, int write_grad);
-// Column sums: out[c] += sum_r in[r, c].
+// Column sums: out[c] += sum_r in[r, c], through colsum_row_blocks(rows) x cols
+// partials in scratch and a fixed-order finalize. cols is a multiple of 8.
+inline int colsum_row_blocks(int rows) { return (rows + 127) / 128; }
 template <typename T>
-void launch_colsum(const Ctx& ctx, const T* in, int rows, int cols, float* out);
+void launch_colsum(const Ctx& ctx, const T* in, int rows, int cols, float* out, float* scratch);
 // dwte[idx[r]] += dx[r]; dwpe[t] += sum_b dx[b, t].
 void launch_embed_bwd(const Ctx& ctx, const int* idx, const float* dx, int B, int Tn, int C, int V, float* dwte,
                       float* dwpe);
