@@ -218,7 +218,7 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
     w = WORKLOAD
-    B, T = w["B"], w["T"]
+    B, T = args.batch, w["T"]
     stream = torch.cuda.current_stream()
     m = native.GPT2(w["n_layer"], w["n_head"], w["n_embd"], w["vocab_size"], w["block_size"], B, T,
                     precision="bf16", seed=1234 + rank, stream=stream.cuda_stream)
@@ -353,6 +353,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=WORKLOAD["B"],
+                    help="sequences per step (default 16, the benchmark workload); smaller values are for "
+                         "small-footprint profiler captures and do not produce the benchmark number")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -118,6 +118,7 @@ struct gpt2_handle {
     long long launches = 0;
     bool use_tc_gemm = true;
     bool use_tc_attention = true;
+    bool use_tcgen05_attention = false;   // tcgen05 forward (slower than the mma.sync kernel so far)
     std::string host_error;   // set by enqueue helpers that cannot report a status
 
     bool profiling = false;
@@ -357,8 +358,14 @@ void attn_fwd<float>(gpt2_handle* h, const float* qkv, float* out, float* lse, i
 }
 template <>
 void attn_fwd<bf16>(gpt2_handle* h, const bf16* qkv, bf16* out, float* lse, int B, int T) {
-    if (h->use_tc_attention) launch_attention_fwd_mma(h->ctx(), qkv, out, lse, B, T, h->H, h->hd);
-    else launch_attention_fwd_simt<bf16>(h->ctx(), qkv, out, lse, B, T, h->H, h->hd);
+    if (!h->use_tc_attention) {
+        launch_attention_fwd_simt<bf16>(h->ctx(), qkv, out, lse, B, T, h->H, h->hd);
+    } else if (h->use_tcgen05_attention && attention_tc_supported(h->hd)) {
+        if (!launch_attention_fwd_tc(h->ctx(), qkv, out, lse, B, T, h->H))
+            h->host_error = "tensor-map encoding failed for the attention forward";
+    } else {
+        launch_attention_fwd_mma(h->ctx(), qkv, out, lse, B, T, h->H, h->hd);
+    }
 }
 template <typename A>
 void attn_bwd(gpt2_handle* h, const A* qkv, const A* out, const A* dout, const float* lse, A* dqkv, int B, int T);
@@ -609,6 +616,7 @@ int gpt2_create(const gpt2_config* cfg, void* stream, gpt2_handle** out) {
     h->maxBT = cfg->max_B * cfg->max_T;
     if (const char* e = getenv("GPT2_B200_SIMT_GEMM")) h->use_tc_gemm = (e[0] == '0');
     if (const char* e = getenv("GPT2_B200_SIMT_ATTENTION")) h->use_tc_attention = (e[0] == '0');
+    if (const char* e = getenv("GPT2_B200_TCGEN05_ATTENTION")) h->use_tcgen05_attention = (e[0] == '1');
     build_layout(h);
 
     auto cleanup_fail = [&](int code, const std::string& msg) {

@@ -101,20 +101,16 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, c
                                                       const float* __restrict__ w, const float* dres_in,
                                                       float* dres_out, T* __restrict__ dres_act,
                                                       float* __restrict__ partial, int rows, int C) {
-    extern __shared__ float red[];   // [3][C]: sum dy*xhat, sum dy, sum dres_out over this block's rows
+    // [3][C]: sum dy*xhat, sum dy, sum dres_out over this block's rows, added
+    // per row with shared-memory atomics (keeps registers low: several blocks per SM)
+    extern __shared__ float red[];
     for (int i = threadIdx.x; i < 3 * C; i += blockDim.x) red[i] = 0.f;
     __syncthreads();
     const int lane = threadIdx.x & 31;
     const int warps_total = (gridDim.x * blockDim.x) >> 5;
-    float adw[NV][4], adb[NV][4], adn[NV][4];
-#pragma unroll
-    for (int i = 0; i < NV; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) adw[i][j] = adb[i][j] = adn[i][j] = 0.f;
-
     for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < rows; row += warps_total) {
         const float mu = mean[row], rs = rstd[row];
-        float g[NV][4], xh[NV][4], rin[NV][4];
+        float g[NV][4], xh[NV][4];
         float s1 = 0.f, s2 = 0.f;
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
@@ -123,8 +119,6 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, c
                 float xx[4], ww[4];
                 load4(dy + (long long)row * C + c, g[i]);
                 load4(x + (long long)row * C + c, xx);
-                if (dres_in) load4(dres_in + (long long)row * C + c, rin[i]);
-                else rin[i][0] = rin[i][1] = rin[i][2] = rin[i][3] = 0.f;
                 load4(w + c, ww);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -141,29 +135,18 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, c
         for (int i = 0; i < NV; ++i) {
             const int c = (lane + 32 * i) * 4;
             if (c < C) {
-                float ww[4], o[4];
+                float ww[4], o[4], r[4] = {0.f, 0.f, 0.f, 0.f};
                 load4(w + c, ww);
+                if (dres_in) load4(dres_in + (long long)row * C + c, r);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    o[j] = rs * (g[i][j] * ww[j] - s1 - xh[i][j] * s2) + rin[i][j];
-                    adw[i][j] += g[i][j] * xh[i][j];
-                    adb[i][j] += g[i][j];
-                    adn[i][j] += o[j];
+                    o[j] = rs * (g[i][j] * ww[j] - s1 - xh[i][j] * s2) + r[j];
+                    atomicAdd(&red[c + j], g[i][j] * xh[i][j]);
+                    atomicAdd(&red[C + c + j], g[i][j]);
+                    atomicAdd(&red[2 * C + c + j], o[j]);
                 }
                 store4(dres_out + (long long)row * C + c, o);
                 if (dres_act) store4(dres_act + (long long)row * C + c, o);
-            }
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        const int c = (lane + 32 * i) * 4;
-        if (c < C) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                atomicAdd(&red[c + j], adw[i][j]);
-                atomicAdd(&red[C + c + j], adb[i][j]);
-                atomicAdd(&red[2 * C + c + j], adn[i][j]);
             }
         }
     }
@@ -173,32 +156,23 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, c
 }
 
 // out_k[j] += sum over nblk partial rows of partial[b][k * n + j], k < n_out;
-// a null out_k is skipped. Block = 32 columns x 8 row groups: each thread sums
-// every 8th partial row of its column (coalesced across the warp), then the 8
-// group sums are added in a fixed order (deterministic).
-__global__ void __launch_bounds__(256) colred_finalize_kernel(const float* __restrict__ partial, int nblk, int n,
-                                                              int n_out, float* out0, float* out1, float* out2) {
-    __shared__ float part[8][33];
+// a null out_k is skipped. Block = 32 columns x 32 row groups: each thread sums
+// every 32nd partial row of its column (coalesced across the warp), then the
+// 32 group sums are added in a fixed order (deterministic).
+__global__ void __launch_bounds__(1024) colred_finalize_kernel(const float* __restrict__ partial, int nblk, int n,
+                                                               int n_out, float* out0, float* out1, float* out2) {
+    __shared__ float part[32][33];
     const int i = blockIdx.x * 32 + threadIdx.x;
     const int stride = n * n_out;
     float s = 0.f;
-    if (i < stride) {
-        int b = threadIdx.y;
-        for (; b + 24 < nblk; b += 32) {   // four independent loads in flight
-            const float a0 = partial[(long long)b * stride + i];
-            const float a1 = partial[(long long)(b + 8) * stride + i];
-            const float a2 = partial[(long long)(b + 16) * stride + i];
-            const float a3 = partial[(long long)(b + 24) * stride + i];
-            s += (a0 + a1) + (a2 + a3);
-        }
-        for (; b < nblk; b += 8) s += partial[(long long)b * stride + i];
-    }
+    if (i < stride)
+        for (int b = threadIdx.y; b < nblk; b += 32) s += partial[(long long)b * stride + i];
     part[threadIdx.y][threadIdx.x] = s;
     __syncthreads();
     if (threadIdx.y == 0 && i < stride) {
         float t = 0.f;
 #pragma unroll
-        for (int g = 0; g < 8; ++g) t += part[g][threadIdx.x];
+        for (int g = 0; g < 32; ++g) t += part[g][threadIdx.x];
         const int k = i / n, j = i % n;
         float* out = k == 0 ? out0 : (k == 1 ? out1 : out2);
         if (out) out[j] += t;
@@ -332,15 +306,15 @@ __global__ void colsum_partial_kernel(const T* __restrict__ in, int rows, int co
     const int r1 = min(rows, r0 + rows_per_block);
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     int r = r0;
-    for (; r + 4 <= r1; r += 4) {   // four rows of loads in flight
-        float v[4][8];
+    for (; r + 8 <= r1; r += 8) {   // eight rows of loads in flight
+        float v[8][8];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < 8; ++k) {
             load4(in + (long long)(r + k) * cols + col, v[k]);
             load4(in + (long long)(r + k) * cols + col + 4, v[k] + 4);
         }
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
+        for (int k = 0; k < 8; ++k)
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j] += v[k][j];
     }
@@ -437,8 +411,8 @@ void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const flo
         default: break;
     }
 #undef LNB_CASE
-    colred_finalize_kernel<<<ceil_div(3 * C, 32), dim3(32, 8), 0, ctx.stream>>>(scratch, blocks, C, 3, dw, db,
-                                                                                 dbias_next);
+    colred_finalize_kernel<<<ceil_div(3 * C, 32), dim3(32, 32), 0, ctx.stream>>>(scratch, blocks, C, 3, dw, db,
+                                                                                  dbias_next);
     *ctx.launches += 2;
 }
 
@@ -460,8 +434,8 @@ void launch_colsum(const Ctx& ctx, const T* in, int rows, int cols, float* out, 
     const int rpb = ceil_div(rows, nblk);
     dim3 grid(ceil_div(cols, 8 * 128), nblk);
     colsum_partial_kernel<T><<<grid, 128, 0, ctx.stream>>>(in, rows, cols, rpb, scratch);
-    colred_finalize_kernel<<<ceil_div(cols, 32), dim3(32, 8), 0, ctx.stream>>>(scratch, nblk, cols, 1, out,
-                                                                               nullptr, nullptr);
+    colred_finalize_kernel<<<ceil_div(cols, 32), dim3(32, 32), 0, ctx.stream>>>(scratch, nblk, cols, 1, out,
+                                                                                nullptr, nullptr);
     *ctx.launches += 2;
 }
 

@@ -62,9 +62,11 @@ int check_attention_args(int dtype, int B, int T, int H, int hd, int engine, con
     if (dtype != GPT2K_F32 && dtype != GPT2K_BF16) return set_error(GPT2_ERR_INVALID_ARG, "unknown dtype");
     if (B < 1 || T < 1 || H < 1) return set_error(GPT2_ERR_INVALID_ARG, "B, T, H must be >= 1");
     if (hd != 32 && hd != 64) return set_error(GPT2_ERR_INVALID_ARG, "head width must be 32 or 64");
-    if (engine != 0 && engine != 1) return set_error(GPT2_ERR_INVALID_ARG, "unknown attention engine");
-    if (engine == 1 && dtype != GPT2K_BF16)
-        return set_error(GPT2_ERR_INVALID_ARG, "the tensor-core attention engine takes bf16 operands");
+    if (engine < 0 || engine > 2) return set_error(GPT2_ERR_INVALID_ARG, "unknown attention engine");
+    if (engine >= 1 && dtype != GPT2K_BF16)
+        return set_error(GPT2_ERR_INVALID_ARG, "the tensor-core attention engines take bf16 operands");
+    if (engine == 2 && hd != 64)
+        return set_error(GPT2_ERR_INVALID_ARG, "the tcgen05 attention engine needs head width 64");
     if (!a || !b || !c || !status) return set_error(GPT2_ERR_INVALID_ARG, "NULL operand");
     return GPT2_OK;
 }
@@ -85,7 +87,10 @@ extern "C" int gpt2k_attention_fwd(int dtype, const void* qkv, void* out, float*
     if (rc) return rc;
     long long launches = 0;
     Ctx c = kctx(stream, status_dev, &launches);
-    if (engine == 1)
+    if (engine == 2) {
+        if (!launch_attention_fwd_tc(c, (const bf16*)qkv, (bf16*)out, lse, B, T, H))
+            return set_error(GPT2_ERR_CUDA, "tensor-map encoding failed");
+    } else if (engine == 1)
         launch_attention_fwd_mma(c, (const bf16*)qkv, (bf16*)out, lse, B, T, H, hd);
     else if (dtype == GPT2K_F32)
         launch_attention_fwd_simt<float>(c, (const float*)qkv, (float*)out, lse, B, T, H, hd);
@@ -104,7 +109,7 @@ extern "C" int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, 
     if (!lse || !dqkv || !workspace_dev) return set_error(GPT2_ERR_INVALID_ARG, "NULL operand");
     long long launches = 0;
     Ctx c = kctx(stream, status_dev, &launches);
-    if (engine == 1)
+    if (engine >= 1)
         launch_attention_bwd_mma(c, (const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, workspace_dev,
                                  (bf16*)dqkv, B, T, H, hd);
     else if (dtype == GPT2K_F32)

@@ -86,7 +86,7 @@ void launch_classifier(const Ctx& ctx, T* logits, const int* targets, int rows, 
                        float scale, double* loss_accum, int write_grad);
 // Column sums: out[c] += sum_r in[r, c], through colsum_row_blocks(rows) x cols
 // partials in scratch and a fixed-order finalize. cols is a multiple of 8.
-inline int colsum_row_blocks(int rows) { return (rows + 127) / 128; }
+inline int colsum_row_blocks(int rows) { return (rows + 63) / 64; }
 template <typename T>
 void launch_colsum(const Ctx& ctx, const T* in, int rows, int cols, float* out, float* scratch);
 // dwte[idx[r]] += dx[r]; dwpe[t] += sum_b dx[b, t].
@@ -107,6 +107,11 @@ void launch_attention_fwd_mma(const Ctx& ctx, const bf16* qkv, bf16* out, float*
                               int hd);
 void launch_attention_bwd_mma(const Ctx& ctx, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
                               float* dpre, bf16* dqkv, int B, int Tn, int H, int hd);
+
+// tcgen05 flash attention forward (head width 64). Returns false if a tensor map
+// could not be encoded (nothing launched).
+bool attention_tc_supported(int hd);
+bool launch_attention_fwd_tc(const Ctx& ctx, const bf16* qkv, bf16* out, float* lse, int B, int Tn, int H);
 
 // ----------------------------------------------------------------------------
 // Optimiser and parameter utilities.

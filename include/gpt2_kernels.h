@@ -73,14 +73,15 @@ int gpt2k_matmul_bf16(int layout, const void* A, const void* B, int M, int N, in
  * dtype: GPT2K_F32 or GPT2K_BF16 (qkv, out); arithmetic is fp32.
  * engine: 0 = SIMT kernel (fp32 arithmetic throughout); 1 = tensor-core flash
  *         kernel (bf16 only: mma.sync bf16 products, fp32 accumulation and
- *         softmax). hd must be 32 or 64; T >= 1. */
+ *         softmax); 2 = tcgen05 flash kernel (bf16, hd = 64 only: TMA loads,
+ *         S and P*V in tensor memory, fp32 softmax). hd must be 32 or 64; T >= 1. */
 int gpt2k_attention_fwd(int dtype, const void* qkv, void* out, float* lse, int B, int T, int H, int hd,
                         int engine, uint32_t* status_dev, void* stream);
 
 /* Backward of gpt2k_attention_fwd: dqkv (B, T, 3C) = [dq | dk | dv] from qkv,
  * out, dout (B, T, C) and lse.
  * workspace_dev: caller-owned scratch of B*H*T floats (D = rowsum(dout * out)).
- * engine: 0 = SIMT kernel; 1 = tensor-core kernels (bf16 only). */
+ * engine: 0 = SIMT kernel; 1 or 2 = tensor-core kernels (bf16 only). */
 int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, const void* dout, const float* lse,
                         void* dqkv, int B, int T, int H, int hd, float* workspace_dev, int engine,
                         uint32_t* status_dev, void* stream);
