@@ -181,7 +181,7 @@ def kernel_source_sha(name: str) -> str:
     return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16] if os.path.exists(p) else ""
 
 
-SITE_SOURCES = [("gemm", "k_gemm_tc.cu"), ("attention", "k_attention_simt.cu"), ("layernorm", "k_rowwise.cu"),
+SITE_SOURCES = [("gemm", "k_gemm_tc.cu"), ("attention", "k_attention_mma.cu"), ("layernorm", "k_rowwise.cu"),
                 ("classifier", "k_rowwise.cu"), ("adamw", "k_optim.cu"), ("grad norm", "k_optim.cu"),
                 ("embed", "k_rowwise.cu"), ("bias colsum", "k_rowwise.cu")]
 

@@ -70,36 +70,57 @@ struct Units {
     }
 };
 
+template <int KIND>
+struct EpiTraits {
+    static constexpr bool F32 = (KIND == EPI_BIAS_RESID || KIND == EPI_ACCUM_F32);   // fp32 result
+    static constexpr int CW = F32 ? 32 : 64;       // columns per chunk: 128 bytes of results per row
+    static constexpr int EPS = F32 ? 4 : 8;        // elements per 16-byte segment
+    static constexpr int ES = F32 ? 4 : 2;         // element size
+    static constexpr bool HAS_IN = (KIND == EPI_BIAS_RESID || KIND == EPI_DGELU);
+    static constexpr bool HAS_BIAS = (KIND == EPI_BIAS || KIND == EPI_BIAS_GELU || KIND == EPI_BIAS_RESID);
+};
+
+// Start the coalesced loads of one input chunk (the residual, or the GELU
+// pre-activation) into registers: lane = 8 lanes per row, 4 rows per step.
+template <int KIND>
+__device__ __forceinline__ void prefetch_in(const Epilogue& ep, uint4 (&pre)[8], int row0, int col0, int M, int N) {
+    using E = EpiTraits<KIND>;
+    const int lane = threadIdx.x & 31;
+    const int lrow = lane >> 3, lseg = lane & 7;
+    const char* src = KIND == EPI_BIAS_RESID ? reinterpret_cast<const char*>(ep.resid)
+                                             : reinterpret_cast<const char*>(ep.aux);
+#pragma unroll
+    for (int st = 0; st < 8; ++st) {
+        const int r = st * 4 + lrow;
+        const int c = col0 + lseg * E::EPS;
+        pre[st] = make_uint4(0, 0, 0, 0);
+        if (row0 + r < M && c < N)
+            pre[st] = *reinterpret_cast<const uint4*>(src + ((long long)(row0 + r) * ep.ldo + c) * E::ES);
+    }
+}
+
 // One chunk of the epilogue for the calling warp: rows row0 .. row0+31 (lane =
-// row of acc) by CW columns from col0, CW = 64 for bf16 results and 32 for fp32
-// results, i.e. 128 bytes per row. Results (and the residual / GELU' inputs,
-// which have the same shape as the result) pass through the warp's
-// shared-memory buffer, so global memory is read and written in whole 128-byte
-// rows, four rows per instruction; each lane updates its row's 16-byte
-// segments in place in the buffer.
+// row of acc) by CW columns from col0. Results (and the prefetched residual /
+// GELU' inputs, which have the same shape as the result) pass through the
+// warp's shared-memory buffer, so global memory is read and written in whole
+// 128-byte rows, four rows per instruction; each lane updates its row's
+// 16-byte segments in place in the buffer. If next_col0 >= 0, the input chunk
+// at next_col0 is prefetched into `pre` while this chunk is computed.
 template <int KIND>
 __device__ __forceinline__ void epilogue_chunk(const Epilogue& ep, float* acc, int row0, int col0, int M, int N,
-                                               uint8_t* buf) {
-    constexpr bool F32 = (KIND == EPI_BIAS_RESID || KIND == EPI_ACCUM_F32);
-    constexpr int EPS = F32 ? 4 : 8;           // elements per 16-byte segment
-    constexpr int ES = F32 ? 4 : 2;            // element size
+                                               uint8_t* buf, uint4 (&pre)[8], int next_col0) {
+    using E = EpiTraits<KIND>;
+    constexpr bool F32 = E::F32;
+    constexpr int EPS = E::EPS;
+    constexpr int ES = E::ES;
     constexpr int kind = KIND;
     const int lane = threadIdx.x & 31;
     const int lrow = lane >> 3, lseg = lane & 7;   // copy pattern: 8 lanes per row, 4 rows per step
-    constexpr bool has_in = (kind == EPI_BIAS_RESID || kind == EPI_DGELU);
-    constexpr bool has_bias = (kind == EPI_BIAS || kind == EPI_BIAS_GELU || kind == EPI_BIAS_RESID);
-    if (has_in) {
-        const char* src = kind == EPI_BIAS_RESID ? reinterpret_cast<const char*>(ep.resid)
-                                                 : reinterpret_cast<const char*>(ep.aux);
+    if (E::HAS_IN) {
 #pragma unroll
-        for (int st = 0; st < 8; ++st) {
-            const int r = st * 4 + lrow;
-            const int c = col0 + lseg * EPS;
-            uint4 q = make_uint4(0, 0, 0, 0);
-            if (row0 + r < M && c < N) q = *reinterpret_cast<const uint4*>(src + ((long long)(row0 + r) * ep.ldo + c) * ES);
-            *reinterpret_cast<uint4*>(buf + swz(r, lseg)) = q;
-        }
+        for (int st = 0; st < 8; ++st) *reinterpret_cast<uint4*>(buf + swz(st * 4 + lrow, lseg)) = pre[st];
         __syncwarp();
+        if (next_col0 >= 0) prefetch_in<KIND>(ep, pre, row0, next_col0, M, N);
     }
     constexpr int npass = kind == EPI_BIAS_GELU ? 2 : 1;   // GELU: u (out2), then gelu(u) (out)
 #pragma unroll
@@ -108,7 +129,7 @@ __device__ __forceinline__ void epilogue_chunk(const Epilogue& ep, float* acc, i
         for (int c = 0; c < 8; ++c) {
             float* x = acc + c * EPS;
             float in[EPS], b[EPS];
-            if (has_in) {
+            if (E::HAS_IN) {
                 if (F32) {
                     const float4 q = *reinterpret_cast<const float4*>(buf + swz(lane, c));
                     in[0] = q.x; in[1] = q.y; in[2] = q.z; in[3] = q.w;
@@ -116,7 +137,7 @@ __device__ __forceinline__ void epilogue_chunk(const Epilogue& ep, float* acc, i
                     load8(reinterpret_cast<const bf16*>(buf + swz(lane, c)), in);
                 }
             }
-            if (has_bias && pass == 0) {
+            if (E::HAS_BIAS && pass == 0) {
 #pragma unroll
                 for (int g = 0; g < EPS / 4; ++g) {
                     float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -294,21 +315,24 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
         const int col_half = ew >> 2;            // columns [half*BN/2, half*BN/2 + BN/2)
         uint8_t* buf = epi_smem + ew * EBUF;
-        constexpr bool f32_out = (KIND == EPI_BIAS_RESID || KIND == EPI_ACCUM_F32);
+        using E = EpiTraits<KIND>;
+        constexpr int CW = E::CW;
+        uint4 pre[8];
         uint32_t acc_it = 0;
         for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++acc_it) {
             int mb, nb, kb0, kb1;
             units.decode(u, mb, nb, kb0, kb1);
             const uint32_t ab = acc_it & 1, aph = (acc_it >> 1) & 1;
+            const int row0 = mb * BM + quarter * 32;
+            const int cbase = col_half * (BN / 2);
+            // the first input chunk of this tile is requested before waiting for the accumulator
+            if (E::HAS_IN && row0 < M) prefetch_in<KIND>(ep, pre, row0, nb * BN + cbase, M, N);
             uint32_t ok = 0;
             if (lane == 0) ok = tc::mbar_wait(&ctl->acc_full[ab], aph, abort, status) ? 1u : 0u;
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc::fence_after_sync();
-            const int row0 = mb * BM + quarter * 32;
-            const int cbase = col_half * (BN / 2);
             const uint32_t taddr = tmem + ab * BN + cbase + ((uint32_t)(quarter * 32) << 16);
-            constexpr int CW = f32_out ? 32 : 64;   // columns per chunk (128 bytes of results per row)
 #pragma unroll 1
             for (int c = 0; c < BN / 2; c += CW) {
                 const int col0 = nb * BN + cbase + c;
@@ -316,7 +340,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 float acc[CW];
                 tc::tmem_ld_32x32b_x32(taddr + (uint32_t)c, acc);
                 if (CW == 64) tc::tmem_ld_32x32b_x32(taddr + (uint32_t)c + 32, acc + 32);
-                if (row0 < M) epilogue_chunk<KIND>(ep, acc, row0, col0, M, N, buf);
+                const int next = (c + CW < BN / 2 && col0 + CW < N) ? col0 + CW : -1;
+                if (row0 < M) epilogue_chunk<KIND>(ep, acc, row0, col0, M, N, buf, pre, next);
             }
             tc::fence_before_sync();
             __syncwarp();
