@@ -99,6 +99,13 @@ __device__ __forceinline__ float gelu_fast_grad(float u) {
     const float s = gelu_sigmoid_s(u);
     return fmaf(2.0f * u * s * (1.0f - s) * c, fmaf(3.0f * 0.044715f * u, u, 1.0f), s);
 }
+// GELU and its derivative from one exponential (logistic form).
+__device__ __forceinline__ void gelu_fast_both(float u, float& g, float& dg) {
+    const float c = 0.7978845608028654f;
+    const float s = gelu_sigmoid_s(u);
+    g = u * s;
+    dg = fmaf(2.0f * u * s * (1.0f - s) * c, fmaf(3.0f * 0.044715f * u, u, 1.0f), s);
+}
 // GELU and its derivative for an output element type: exact tanh form for fp32
 // results, the logistic form for bf16 results.
 template <typename T> __device__ __forceinline__ float gelu_for(float u);

@@ -16,19 +16,17 @@ __device__ __forceinline__ void epilogue_scalar(const Epilogue& ep, long long ro
         case EPI_STORE: reinterpret_cast<T*>(ep.out)[base + j] = from_f<T>(a); break;
         case EPI_BIAS: reinterpret_cast<T*>(ep.out)[base + j] = from_f<T>(a + ep.bias[col + j]); break;
         case EPI_BIAS_GELU: {
-            T u = from_f<T>(a + ep.bias[col + j]);   // stored pre-activation
-            reinterpret_cast<T*>(ep.out2)[base + j] = u;
-            reinterpret_cast<T*>(ep.out)[base + j] = from_f<T>(gelu_for<T>(to_f(u)));
+            const float u = to_f(from_f<T>(a + ep.bias[col + j]));   // pre-activation as rounded
+            reinterpret_cast<T*>(ep.out2)[base + j] = from_f<T>(gelu_grad_for<T>(u));
+            reinterpret_cast<T*>(ep.out)[base + j] = from_f<T>(gelu_for<T>(u));
             break;
         }
         case EPI_BIAS_RESID:
             reinterpret_cast<float*>(ep.out)[base + j] = ep.resid[base + j] + (a + ep.bias[col + j]);
             break;
-        case EPI_DGELU: {
-            const T u = reinterpret_cast<const T*>(ep.aux)[base + j];
-            reinterpret_cast<T*>(ep.out)[base + j] = from_f<T>(a * gelu_grad_for<T>(to_f(u)));
+        case EPI_MUL:
+            reinterpret_cast<T*>(ep.out)[base + j] = from_f<T>(a * to_f(reinterpret_cast<const T*>(ep.aux)[base + j]));
             break;
-        }
         case EPI_ACCUM_F32: {
             float* o = reinterpret_cast<float*>(ep.out) + base + j;
             if (ep.split_atomic) atomicAdd(o, a);
@@ -54,10 +52,14 @@ __device__ __forceinline__ void epilogue_vec4(const Epilogue& ep, long long base
         store4(reinterpret_cast<T*>(ep.out) + base, v);
         break;
     case EPI_BIAS_GELU: {
+        float d[4];
         load4(ep.bias + col, b);
-        for (int j = 0; j < 4; ++j) v[j] = to_f(from_f<T>(acc[j] + b[j]));   // value as stored
-        store4(reinterpret_cast<T*>(ep.out2) + base, v);
-        for (int j = 0; j < 4; ++j) v[j] = gelu_for<T>(v[j]);
+        for (int j = 0; j < 4; ++j) {
+            const float u = to_f(from_f<T>(acc[j] + b[j]));   // pre-activation as rounded
+            v[j] = gelu_for<T>(u);
+            d[j] = gelu_grad_for<T>(u);
+        }
+        store4(reinterpret_cast<T*>(ep.out2) + base, d);
         store4(reinterpret_cast<T*>(ep.out) + base, v);
         break;
     }
@@ -69,10 +71,10 @@ __device__ __forceinline__ void epilogue_vec4(const Epilogue& ep, long long base
         store4(reinterpret_cast<float*>(ep.out) + base, v);
         break;
     }
-    case EPI_DGELU: {
+    case EPI_MUL: {
         float u[4];
         load4(reinterpret_cast<const T*>(ep.aux) + base, u);
-        for (int j = 0; j < 4; ++j) v[j] = acc[j] * gelu_grad_for<T>(u[j]);
+        for (int j = 0; j < 4; ++j) v[j] = acc[j] * u[j];
         store4(reinterpret_cast<T*>(ep.out) + base, v);
         break;
     }
@@ -133,20 +135,20 @@ __device__ __forceinline__ void epilogue_vec8_bf16(const Epilogue& ep, long long
         for (int j = 0; j < 8; ++j) v[j] = acc[j] + b[j];
         store8(reinterpret_cast<bf16*>(ep.out) + base, v);
         break;
-    case EPI_BIAS_GELU:
+    case EPI_BIAS_GELU: {
+        float d[8];
         load4(ep.bias + col, b);
         load4(ep.bias + col + 4, b + 4);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = __bfloat162float(__float2bfloat16_rn(acc[j] + b[j]));
-        store8(reinterpret_cast<bf16*>(ep.out2) + base, v);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = gelu_fast(v[j]);
+        for (int j = 0; j < 8; ++j) gelu_fast_both(__bfloat162float(__float2bfloat16_rn(acc[j] + b[j])), v[j], d[j]);
+        store8(reinterpret_cast<bf16*>(ep.out2) + base, d);
         store8(reinterpret_cast<bf16*>(ep.out) + base, v);
         break;
-    case EPI_DGELU:
+    }
+    case EPI_MUL:
         load8(reinterpret_cast<const bf16*>(ep.aux) + base, b);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = acc[j] * gelu_fast_grad(b[j]);
+        for (int j = 0; j < 8; ++j) v[j] = acc[j] * b[j];
         store8(reinterpret_cast<bf16*>(ep.out) + base, v);
         break;
     default:   // fp32 outputs

@@ -97,7 +97,7 @@ struct gpt2_handle {
     char* act_pool = nullptr;
     std::vector<float*> resid;          // 2L+1 of (BT, C) fp32
     std::vector<float*> ln_mean, ln_rstd;  // 2L+1 of (BT)
-    std::vector<void*> ln1, ln2, qkv, att, fch, fcg;  // per layer
+    std::vector<void*> ln1, ln2, qkv, att, fch, fcg;  // per layer; fch = gelu'(u), fcg = gelu(u)
     std::vector<float*> lse;            // per layer (B, H, T)
     void* lnf = nullptr;
     void* logits = nullptr;
@@ -335,7 +335,7 @@ double gemm_bytes(int M, int N, int K, size_t es, const Epilogue& ep) {
     switch (ep.kind) {
     case EPI_BIAS_GELU: b += 2 * mn * es; break;
     case EPI_BIAS_RESID: b += 2 * mn * 4; break;
-    case EPI_DGELU: b += 2 * mn * es; break;
+    case EPI_MUL: b += 2 * mn * es; break;
     case EPI_ACCUM_F32: b += (ep.beta != 0.f ? 2 : 1) * mn * 4; break;
     default: b += mn * es; break;
     }
@@ -474,9 +474,9 @@ void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
         acc = epi(EPI_ACCUM_F32, G + o.wfcp, 4 * C);
         acc.beta = 1.f;
         gemm<A>(h, "gemm wgrad mlp.c_proj", GEMM_TN, h->dres_act, h->fcg[l], C, 4 * C, BT, acc);
-        Epilogue e = epi(EPI_DGELU, h->du, 4 * C);
+        Epilogue e = epi(EPI_MUL, h->du, 4 * C);   // du = (dY W) * gelu'(u), gelu'(u) stored by the forward
         e.aux = h->fch[l];
-        gemm<A>(h, "gemm dgrad mlp.c_proj+dgelu", GEMM_NN, h->dres_act, wop<A>(h, o.wfcp), BT, 4 * C, C, e);
+        gemm<A>(h, "gemm dgrad mlp.c_proj*gelu'", GEMM_NN, h->dres_act, wop<A>(h, o.wfcp), BT, 4 * C, C, e);
         PROF("bias colsum", 0, 0, 0, 0.0, (double)BT * 4 * C * es,
              launch_colsum<A>(c, (const A*)h->du, BT, 4 * C, G + o.bfc, h->red_scratch));
         // mlp.c_fc: dW += du^T ln2 ; dln2 = du W
@@ -678,7 +678,7 @@ int gpt2_create(const gpt2_config* cfg, void* stream, gpt2_handle** out) {
     plan.push_back({&h->du, BT * 4 * C * es});
     plan.push_back({(void**)&h->dpre, BHT * 4});
     {
-        const size_t ln_part = (size_t)ln_bwd_blocks(h->num_sms) * 3 * C;
+        const size_t ln_part = (size_t)ln_bwd_col_blocks((int)BT) * 3 * C;
         const size_t cs_part = (size_t)colsum_row_blocks((int)BT) * 4 * C;
         plan.push_back({(void**)&h->red_scratch, std::max(ln_part, cs_part) * 4});
     }

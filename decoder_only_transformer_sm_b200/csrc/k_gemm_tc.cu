@@ -76,8 +76,9 @@ struct EpiTraits {
     static constexpr int CW = F32 ? 32 : 64;       // columns per chunk: 128 bytes of results per row
     static constexpr int EPS = F32 ? 4 : 8;        // elements per 16-byte segment
     static constexpr int ES = F32 ? 4 : 2;         // element size
-    static constexpr bool HAS_IN = (KIND == EPI_BIAS_RESID || KIND == EPI_DGELU);
+    static constexpr bool HAS_IN = (KIND == EPI_BIAS_RESID || KIND == EPI_MUL);
     static constexpr bool HAS_BIAS = (KIND == EPI_BIAS || KIND == EPI_BIAS_GELU || KIND == EPI_BIAS_RESID);
+    static constexpr int DEPTH = F32 ? 2 : 1;      // input chunks prefetched ahead (fp32 chunks are narrower)
 };
 
 // Start the coalesced loads of one input chunk (the residual, or the GELU
@@ -122,7 +123,7 @@ __device__ __forceinline__ void epilogue_chunk(const Epilogue& ep, float* acc, i
         __syncwarp();
         if (next_col0 >= 0) prefetch_in<KIND>(ep, pre, row0, next_col0, M, N);
     }
-    constexpr int npass = kind == EPI_BIAS_GELU ? 2 : 1;   // GELU: u (out2), then gelu(u) (out)
+    constexpr int npass = kind == EPI_BIAS_GELU ? 2 : 1;   // GELU: gelu'(u) (out2), then gelu(u) (out)
 #pragma unroll
     for (int pass = 0; pass < npass; ++pass) {
 #pragma unroll
@@ -151,15 +152,16 @@ __device__ __forceinline__ void epilogue_chunk(const Epilogue& ep, float* acc, i
                 switch (kind) {
                 case EPI_BIAS: v[j] = x[j] + b[j]; break;
                 case EPI_BIAS_GELU:
-                    if (pass == 0) {
-                        x[j] = __bfloat162float(__float2bfloat16_rn(x[j] + b[j]));   // u as stored
-                        v[j] = x[j];
+                    if (pass == 0) {   // u as rounded to bf16; keep gelu(u) for the second pass
+                        float g;
+                        gelu_fast_both(__bfloat162float(__float2bfloat16_rn(x[j] + b[j])), g, v[j]);
+                        x[j] = g;
                     } else {
-                        v[j] = gelu_fast(x[j]);
+                        v[j] = x[j];
                     }
                     break;
                 case EPI_BIAS_RESID: v[j] = in[j] + (x[j] + b[j]); break;
-                case EPI_DGELU: v[j] = x[j] * gelu_fast_grad(in[j]); break;
+                case EPI_MUL: v[j] = x[j] * in[j]; break;
                 default: v[j] = x[j]; break;
                 }
             }
@@ -317,7 +319,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint8_t* buf = epi_smem + ew * EBUF;
         using E = EpiTraits<KIND>;
         constexpr int CW = E::CW;
-        uint4 pre[8];
+        constexpr int NCH = (BN / 2) / CW;       // chunks per warp and tile
+        uint4 pre[E::DEPTH][8];                  // input chunks in flight (ring)
         uint32_t acc_it = 0;
         for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++acc_it) {
             int mb, nb, kb0, kb1;
@@ -325,23 +328,29 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t ab = acc_it & 1, aph = (acc_it >> 1) & 1;
             const int row0 = mb * BM + quarter * 32;
             const int cbase = col_half * (BN / 2);
-            // the first input chunk of this tile is requested before waiting for the accumulator
-            if (E::HAS_IN && row0 < M) prefetch_in<KIND>(ep, pre, row0, nb * BN + cbase, M, N);
+            // the first input chunks of this tile are requested before waiting for the accumulator
+            if (E::HAS_IN && row0 < M) {
+#pragma unroll
+                for (int d = 0; d < E::DEPTH; ++d)
+                    if (d < NCH) prefetch_in<KIND>(ep, pre[d], row0, nb * BN + cbase + d * CW, M, N);
+            }
             uint32_t ok = 0;
             if (lane == 0) ok = tc::mbar_wait(&ctl->acc_full[ab], aph, abort, status) ? 1u : 0u;
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc::fence_after_sync();
             const uint32_t taddr = tmem + ab * BN + cbase + ((uint32_t)(quarter * 32) << 16);
-#pragma unroll 1
-            for (int c = 0; c < BN / 2; c += CW) {
+#pragma unroll
+            for (int ci = 0; ci < NCH; ++ci) {
+                const int c = ci * CW;
                 const int col0 = nb * BN + cbase + c;
                 if (col0 >= N) break;
                 float acc[CW];
                 tc::tmem_ld_32x32b_x32(taddr + (uint32_t)c, acc);
                 if (CW == 64) tc::tmem_ld_32x32b_x32(taddr + (uint32_t)c + 32, acc + 32);
-                const int next = (c + CW < BN / 2 && col0 + CW < N) ? col0 + CW : -1;
-                if (row0 < M) epilogue_chunk<KIND>(ep, acc, row0, col0, M, N, buf, pre, next);
+                const int nc = c + E::DEPTH * CW;     // chunk whose input this buffer prefetches next
+                const int next = (nc < BN / 2 && nb * BN + cbase + nc < N) ? nb * BN + cbase + nc : -1;
+                if (row0 < M) epilogue_chunk<KIND>(ep, acc, row0, col0, M, N, buf, pre[ci % E::DEPTH], next);
             }
             tc::fence_before_sync();
             __syncwarp();
@@ -437,7 +446,7 @@ bool launch_variant(const Ctx& ctx, const CUtensorMap& ta, const CUtensorMap& tb
     case EPI_BIAS_RESID:
         launch_kernel<A_MN, B_MN, EPI_BIAS_RESID>(grid, ctx.stream, ta, tb, M, N, u, ep, ctx.status);
         break;
-    case EPI_DGELU: launch_kernel<A_MN, B_MN, EPI_DGELU>(grid, ctx.stream, ta, tb, M, N, u, ep, ctx.status); break;
+    case EPI_MUL: launch_kernel<A_MN, B_MN, EPI_MUL>(grid, ctx.stream, ta, tb, M, N, u, ep, ctx.status); break;
     case EPI_ACCUM_F32:
         launch_kernel<A_MN, B_MN, EPI_ACCUM_F32>(grid, ctx.stream, ta, tb, M, N, u, ep, ctx.status);
         break;

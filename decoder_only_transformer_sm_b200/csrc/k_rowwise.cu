@@ -95,64 +95,107 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const int* __restrict__ idx
     if (lane == 0) { mean[row] = mu; rstd[row] = rs; }
 }
 
+// LayerNorm backward, row part: one warp per row computes
+// dx = rstd (dxhat - mean(dxhat) - xhat mean(dxhat xhat)) + dres_in, dxhat = dy * w,
+// and writes it as fp32 (residual gradient) and in the GEMM operand type.
 template <typename T, int NV>
-__global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, const float* __restrict__ x,
-                                                      const float* __restrict__ mean, const float* __restrict__ rstd,
-                                                      const float* __restrict__ w, const float* dres_in,
-                                                      float* dres_out, T* __restrict__ dres_act,
-                                                      float* __restrict__ partial, int rows, int C) {
-    // [3][C]: sum dy*xhat, sum dy, sum dres_out over this block's rows, added
-    // per row with shared-memory atomics (keeps registers low: several blocks per SM)
-    extern __shared__ float red[];
-    for (int i = threadIdx.x; i < 3 * C; i += blockDim.x) red[i] = 0.f;
-    __syncthreads();
+__global__ void __launch_bounds__(256) ln_bwd_rows_kernel(const T* __restrict__ dy, const float* __restrict__ x,
+                                                           const float* __restrict__ mean,
+                                                           const float* __restrict__ rstd,
+                                                           const float* __restrict__ w, const float* dres_in,
+                                                           float* dres_out, T* __restrict__ dres_act, int rows,
+                                                           int C) {
+    const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
-    const int warps_total = (gridDim.x * blockDim.x) >> 5;
-    for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < rows; row += warps_total) {
-        const float mu = mean[row], rs = rstd[row];
-        float g[NV][4], xh[NV][4];
-        float s1 = 0.f, s2 = 0.f;
+    if (row >= rows) return;
+    const float mu = mean[row], rs = rstd[row];
+    float dxh[NV][4], xh[NV][4];
+    float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-        for (int i = 0; i < NV; ++i) {
-            const int c = (lane + 32 * i) * 4;
-            if (c < C) {
-                float xx[4], ww[4];
-                load4(dy + (long long)row * C + c, g[i]);
-                load4(x + (long long)row * C + c, xx);
-                load4(w + c, ww);
+    for (int i = 0; i < NV; ++i) {
+        const int c = (lane + 32 * i) * 4;
+        if (c < C) {
+            float g[4], xx[4], ww[4];
+            load4(dy + (long long)row * C + c, g);
+            load4(x + (long long)row * C + c, xx);
+            load4(w + c, ww);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    xh[i][j] = (xx[j] - mu) * rs;
-                    const float d = g[i][j] * ww[j];
-                    s1 += d;
-                    s2 += d * xh[i][j];
-                }
-            }
-        }
-        s1 = warp_sum(s1) / C;
-        s2 = warp_sum(s2) / C;
-#pragma unroll
-        for (int i = 0; i < NV; ++i) {
-            const int c = (lane + 32 * i) * 4;
-            if (c < C) {
-                float ww[4], o[4], r[4] = {0.f, 0.f, 0.f, 0.f};
-                load4(w + c, ww);
-                if (dres_in) load4(dres_in + (long long)row * C + c, r);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    o[j] = rs * (g[i][j] * ww[j] - s1 - xh[i][j] * s2) + r[j];
-                    atomicAdd(&red[c + j], g[i][j] * xh[i][j]);
-                    atomicAdd(&red[C + c + j], g[i][j]);
-                    atomicAdd(&red[2 * C + c + j], o[j]);
-                }
-                store4(dres_out + (long long)row * C + c, o);
-                if (dres_act) store4(dres_act + (long long)row * C + c, o);
+            for (int j = 0; j < 4; ++j) {
+                xh[i][j] = (xx[j] - mu) * rs;
+                dxh[i][j] = g[j] * ww[j];
+                s1 += dxh[i][j];
+                s2 += dxh[i][j] * xh[i][j];
             }
         }
     }
+    s1 = warp_sum(s1) / C;
+    s2 = warp_sum(s2) / C;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c = (lane + 32 * i) * 4;
+        if (c < C) {
+            float o[4], r[4] = {0.f, 0.f, 0.f, 0.f};
+            if (dres_in) load4(dres_in + (long long)row * C + c, r);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o[j] = rs * (dxh[i][j] - s1 - xh[i][j] * s2) + r[j];
+            store4(dres_out + (long long)row * C + c, o);
+            if (dres_act) store4(dres_act + (long long)row * C + c, o);
+        }
+    }
+}
+
+// LayerNorm backward, column part: per block of rows, the partial sums
+// sum dy * xhat (weight gradient), sum dy (bias gradient) and sum dres_out
+// (bias gradient of the GEMM that produced this LayerNorm's input) for each
+// column. Thread (tx, ty) owns columns 8 tx .. 8 tx + 7 and every blockDim.y-th
+// row; the ty partials are added in a fixed order (deterministic).
+template <typename T>
+__global__ void ln_bwd_cols_kernel(const T* __restrict__ dy, const float* __restrict__ x,
+                                   const float* __restrict__ mean, const float* __restrict__ rstd,
+                                   const float* __restrict__ dres_out, int rows, int C, int rows_per_block,
+                                   float* __restrict__ partial) {
+    extern __shared__ float red[];   // [blockDim.y][3][C]
+    const int col = threadIdx.x * 8;
+    const int r0 = blockIdx.x * rows_per_block;
+    const int r1 = min(rows, r0 + rows_per_block);
+    float aw[8], ab[8], an[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) aw[j] = ab[j] = an[j] = 0.f;
+    for (int r = r0 + threadIdx.y; r < r1; r += blockDim.y) {
+        float g[8], xx[8], d[8];
+        load4(dy + (long long)r * C + col, g);
+        load4(dy + (long long)r * C + col + 4, g + 4);
+        load4(x + (long long)r * C + col, xx);
+        load4(x + (long long)r * C + col + 4, xx + 4);
+        load4(dres_out + (long long)r * C + col, d);
+        load4(dres_out + (long long)r * C + col + 4, d + 4);
+        const float mu = mean[r], rs = rstd[r];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            aw[j] += g[j] * ((xx[j] - mu) * rs);
+            ab[j] += g[j];
+            an[j] += d[j];
+        }
+    }
+    float* mine = red + threadIdx.y * 3 * C;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        mine[col + j] = aw[j];
+        mine[C + col + j] = ab[j];
+        mine[2 * C + col + j] = an[j];
+    }
     __syncthreads();
-    float* part = partial + (long long)blockIdx.x * 3 * C;
-    for (int i = threadIdx.x; i < 3 * C; i += blockDim.x) part[i] = red[i];
+    if (threadIdx.y == 0) {
+        float* part = partial + (long long)blockIdx.x * 3 * C;
+#pragma unroll
+        for (int k = 0; k < 3; ++k)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float t = 0.f;
+                for (int y = 0; y < (int)blockDim.y; ++y) t += red[(y * 3 + k) * C + col + j];
+                part[k * C + col + j] = t;
+            }
+    }
 }
 
 // out_k[j] += sum over nblk partial rows of partial[b][k * n + j], k < n_out;
@@ -396,13 +439,12 @@ void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const flo
                           const float* w, const float* dres_in, float* dres_out, T* dres_act, float* dw,
                           float* db, float* dbias_next, int rows, int C, float* scratch) {
     const int threads = 256;
-    const int blocks = min(ceil_div(rows, threads / 32), ln_bwd_blocks(ctx.num_sms));
-    const size_t smem = 3 * C * sizeof(float);
+    const int blocks = ceil_div(rows, threads / 32);
     const int nv = ceil_div(C, 128);
-#define LNB_CASE(N)                                                                                      \
-    case N:                                                                                              \
-        ln_bwd_kernel<T, N><<<blocks, threads, smem, ctx.stream>>>(dy, x, mean, rstd, w, dres_in, dres_out, \
-                                                                   dres_act, scratch, rows, C);            \
+#define LNB_CASE(N)                                                                                           \
+    case N:                                                                                                   \
+        ln_bwd_rows_kernel<T, N><<<blocks, threads, 0, ctx.stream>>>(dy, x, mean, rstd, w, dres_in, dres_out, \
+                                                                     dres_act, rows, C);                      \
         break;
     switch (nv) {
         LNB_CASE(1) LNB_CASE(2) LNB_CASE(3) LNB_CASE(4) LNB_CASE(5) LNB_CASE(6) LNB_CASE(7)
@@ -411,9 +453,21 @@ void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const flo
         default: break;
     }
 #undef LNB_CASE
-    colred_finalize_kernel<<<ceil_div(3 * C, 32), dim3(32, 32), 0, ctx.stream>>>(scratch, blocks, C, 3, dw, db,
+    const int tx = C / 8;
+    const int ty = max(1, min(8, 1024 / tx));
+    const int nblk = ln_bwd_col_blocks(rows);
+    const int rpb = ceil_div(rows, nblk);
+    const size_t smem = (size_t)ty * 3 * C * sizeof(float);
+    static bool configured = false;
+    if (!configured) {
+        cudaFuncSetAttribute(ln_bwd_cols_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        configured = true;
+    }
+    ln_bwd_cols_kernel<T><<<nblk, dim3(tx, ty), smem, ctx.stream>>>(dy, x, mean, rstd, dres_out, rows, C, rpb,
+                                                                     scratch);
+    colred_finalize_kernel<<<ceil_div(3 * C, 32), dim3(32, 32), 0, ctx.stream>>>(scratch, nblk, C, 3, dw, db,
                                                                                   dbias_next);
-    *ctx.launches += 2;
+    *ctx.launches += 3;
 }
 
 void launch_count_targets(const Ctx& ctx, const int* targets, int n, int V, int* n_valid) {

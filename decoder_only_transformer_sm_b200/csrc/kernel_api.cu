@@ -22,7 +22,7 @@ extern "C" int gpt2k_matmul_bf16(int layout, const void* A, const void* B, int M
     const bool needs_bias = epilogue == GPT2K_EPI_BIAS || epilogue == GPT2K_EPI_BIAS_GELU ||
                             epilogue == GPT2K_EPI_BIAS_RESID;
     if ((needs_bias && !bias) || (epilogue == GPT2K_EPI_BIAS_GELU && !out2) ||
-        (epilogue == GPT2K_EPI_BIAS_RESID && !resid) || (epilogue == GPT2K_EPI_DGELU && !aux))
+        (epilogue == GPT2K_EPI_BIAS_RESID && !resid) || (epilogue == GPT2K_EPI_MUL && !aux))
         return set_error(GPT2_ERR_INVALID_ARG, "epilogue operand missing");
     long long launches = 0;
     Ctx c;

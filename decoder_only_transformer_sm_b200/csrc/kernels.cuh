@@ -20,9 +20,9 @@ struct Ctx {
 enum EpiKind {
     EPI_STORE = 0,       // out[act]  = acc
     EPI_BIAS = 1,        // out[act]  = acc + bias[col]
-    EPI_BIAS_GELU = 2,   // out2[act] = u = acc + bias[col];  out[act] = gelu(u)
+    EPI_BIAS_GELU = 2,   // u = acc + bias[col] (rounded to act);  out[act] = gelu(u);  out2[act] = gelu'(u)
     EPI_BIAS_RESID = 3,  // out[f32]  = resid[f32] + acc + bias[col]
-    EPI_DGELU = 4,       // out[act]  = acc * gelu'(aux[act])
+    EPI_MUL = 4,         // out[act]  = acc * aux[act]   (aux = the stored gelu'(u): the GELU backward)
     EPI_ACCUM_F32 = 5,   // out[f32]  = beta * out + acc
 };
 
@@ -30,10 +30,10 @@ struct Epilogue {
     int kind = EPI_STORE;
     void* out = nullptr;
     long long ldo = 0;
-    void* out2 = nullptr;          // EPI_BIAS_GELU pre-activation output (ld = ldo)
+    void* out2 = nullptr;          // EPI_BIAS_GELU derivative output gelu'(u) (ld = ldo)
     const float* bias = nullptr;
     const float* resid = nullptr;  // EPI_BIAS_RESID input (ld = ldo)
-    const void* aux = nullptr;     // EPI_DGELU pre-activation input (ld = ldo)
+    const void* aux = nullptr;     // EPI_MUL factor (ld = ldo)
     float beta = 0.f;
     int split_atomic = 0;          // EPI_ACCUM_F32 partial sums of a K split: atomicAdd into out
 };
@@ -69,9 +69,10 @@ void launch_layernorm_fwd(const Ctx& ctx, const float* x, const float* w, const 
                           float* rstd, int rows, int C);
 // dx = LN'(x)^T dy (+ dres_in); writes dres_out (fp32) and dres_act (operand copy);
 // accumulates dw += sum dy*xhat, db += sum dy and, if dbias_next != null,
-// dbias_next += sum_rows dres_out. Column sums go through per-block partials in
-// scratch (ln_bwd_blocks(num_sms) x 3C floats) and a fixed-order finalize.
-inline int ln_bwd_blocks(int num_sms) { return 2 * num_sms; }
+// dbias_next += sum_rows dres_out. A row kernel writes dres; a column kernel
+// writes per-block partial sums to scratch (ln_bwd_col_blocks(rows) x 3C floats)
+// that a fixed-order finalize adds to dw, db, dbias_next. C % 8 == 0.
+inline int ln_bwd_col_blocks(int rows) { return (rows + 63) / 64; }
 template <typename T>
 void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const float* mean, const float* rstd,
                           const float* w, const float* dres_in, float* dres_out, T* dres_act, float* dw,

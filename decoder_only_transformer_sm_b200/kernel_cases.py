@@ -43,7 +43,7 @@ def gemm_case(args):
     out2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda") if ep == "bias_gelu" else None
     bias = torch.randn(N, device="cuda") if ep.startswith("bias") else None
     resid = torch.randn((M, N), device="cuda") if ep == "bias_resid" else None
-    aux = torch.randn((M, N), device="cuda").to(torch.bfloat16) if ep == "dgelu" else None
+    aux = torch.randn((M, N), device="cuda").to(torch.bfloat16) if ep == "mul" else None
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     fn = lambda: native.matmul_bf16(args.layout, A, B, M, N, K, ep, out, out2=out2, bias=bias,  # noqa: E731
                                     resid=resid, aux=aux, beta=1.0, engine="tc" if args.engine else "simt",

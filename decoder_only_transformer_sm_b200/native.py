@@ -243,7 +243,7 @@ class GPT2:
 # Kernel-level entry points (include/gpt2_kernels.h).
 # ---------------------------------------------------------------------------
 LAYOUT = {"NT": 0, "NN": 1, "TN": 2}
-EPILOGUE = {"store": 0, "bias": 1, "bias_gelu": 2, "bias_resid": 3, "dgelu": 4, "accum_f32": 5}
+EPILOGUE = {"store": 0, "bias": 1, "bias_gelu": 2, "bias_resid": 3, "mul": 4, "accum_f32": 5}
 
 
 def matmul_bf16(layout: str, A, B, M: int, N: int, K: int, epilogue: str, out, ldo: int | None = None,

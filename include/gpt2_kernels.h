@@ -32,24 +32,25 @@ extern "C" {
  * "The Block: pre-LN and residuals"):
  *   GPT2K_EPI_STORE      out = acc                                (bf16)
  *   GPT2K_EPI_BIAS       out = acc + bias[n]                      (bf16)
- *   GPT2K_EPI_BIAS_GELU  out2 = u = acc + bias[n]; out = gelu_tanh(u) (bf16)
+ *   GPT2K_EPI_BIAS_GELU  u = acc + bias[n] rounded to bf16; out = gelu_tanh(u),
+ *                        out2 = gelu_tanh'(u), the factor the backward needs (bf16)
  *   GPT2K_EPI_BIAS_RESID out = resid + acc + bias[n]              (fp32)
- *   GPT2K_EPI_DGELU      out = acc * gelu_tanh'(aux)              (bf16)
+ *   GPT2K_EPI_MUL        out = acc * aux (the GELU backward: aux = gelu_tanh'(u)) (bf16)
  *   GPT2K_EPI_ACCUM_F32  out = beta * out + acc                   (fp32)      */
 #define GPT2K_EPI_STORE 0
 #define GPT2K_EPI_BIAS 1
 #define GPT2K_EPI_BIAS_GELU 2
 #define GPT2K_EPI_BIAS_RESID 3
-#define GPT2K_EPI_DGELU 4
+#define GPT2K_EPI_MUL 4
 #define GPT2K_EPI_ACCUM_F32 5
 
 /* bf16 GEMM with fp32 accumulation and a fused epilogue.
  * A, B        : bf16 operands in the given layout.
  * out, ldo    : result matrix [M, N] with row stride ldo (elements).
- * out2        : pre-activation output of GPT2K_EPI_BIAS_GELU (same ldo), else NULL.
+ * out2        : derivative output of GPT2K_EPI_BIAS_GELU (same ldo), else NULL.
  * bias        : fp32 [N] for the BIAS* epilogues, else NULL.
  * resid       : fp32 [M, N] (stride ldo) for GPT2K_EPI_BIAS_RESID, else NULL.
- * aux         : bf16 [M, N] (stride ldo) pre-activation for GPT2K_EPI_DGELU, else NULL.
+ * aux         : bf16 [M, N] (stride ldo) factor for GPT2K_EPI_MUL, else NULL.
  * engine      : 1 = tcgen05 tensor cores (TMA + TMEM), 0 = SIMT fp32-FMA kernel.
  * Errors: INVALID_ARG (sizes < 1, unknown layout/epilogue, a required pointer
  * NULL, or engine 1 with K, N, ldo (or M for TN) not a multiple of 8, or

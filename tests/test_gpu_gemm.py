@@ -75,24 +75,25 @@ def test_gemm_fused_epilogues(shape):
     # bias
     out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     native.matmul_bf16("NT", A, B, M, N, K, "bias", out, bias=bias)
-    # bias + gelu
+    # bias + gelu: out = gelu(u), out2 = gelu'(u), u = bias + acc rounded to bf16
     g_out = torch.empty_like(out)
-    u_out = torch.empty_like(out)
-    native.matmul_bf16("NT", A, B, M, N, K, "bias_gelu", g_out, out2=u_out, bias=bias)
+    d_out2 = torch.empty_like(out)
+    native.matmul_bf16("NT", A, B, M, N, K, "bias_gelu", g_out, out2=d_out2, bias=bias)
     # bias + residual (fp32)
     resid = torch.randn((M, N), generator=g).cuda()
     r_out = torch.empty((M, N), dtype=torch.float32, device="cuda")
     native.matmul_bf16("NT", A, B, M, N, K, "bias_resid", r_out, bias=bias, resid=resid)
-    # dgelu with the stored pre-activation
-    d_out = torch.empty_like(out)
-    native.matmul_bf16("NT", A, B, M, N, K, "dgelu", d_out, aux=u_out)
+    # multiply by a stored factor (the GELU backward)
+    aux = torch.randn((M, N), generator=g).to(torch.bfloat16).cuda()
+    m_out = torch.empty_like(out)
+    native.matmul_bf16("NT", A, B, M, N, K, "mul", m_out, aux=aux)
     torch.cuda.synchronize()
     assert _relerr(_np(out), ref) < 8e-3
-    u = _np(u_out)
-    assert _relerr(u, ref) < 8e-3
+    u = _np(out)                       # bf16-rounded pre-activation
     assert _relerr(_np(g_out), O.gelu_tanh(u)) < 8e-3
+    assert _relerr(_np(d_out2), O.gelu_tanh_grad(u)) < 8e-3
     assert _relerr(r_out.cpu().numpy(), resid.cpu().numpy() + ref) < 1e-5
-    assert _relerr(_np(d_out), _ref("NT", A, B) * O.gelu_tanh_grad(u)) < 8e-3
+    assert _relerr(_np(m_out), _ref("NT", A, B) * _np(aux)) < 8e-3
 
 
 def test_tc_rejects_unaligned_shapes():
