@@ -118,7 +118,8 @@ struct gpt2_handle {
     long long launches = 0;
     bool use_tc_gemm = true;
     bool use_tc_attention = true;
-    bool use_tcgen05_attention = false;   // tcgen05 forward (slower than the mma.sync kernel so far)
+    bool use_tcgen05_attention = false;       // tcgen05 forward (slower than the mma.sync kernel so far)
+    bool use_tcgen05_attention_bwd = true;    // tcgen05 backward (faster than the mma.sync kernels)
     std::string host_error;   // set by enqueue helpers that cannot report a status
 
     bool profiling = false;
@@ -377,7 +378,10 @@ void attn_bwd<float>(gpt2_handle* h, const float* qkv, const float* out, const f
 template <>
 void attn_bwd<bf16>(gpt2_handle* h, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
                     bf16* dqkv, int B, int T) {
-    if (h->use_tc_attention)
+    if (h->use_tc_attention && h->use_tcgen05_attention_bwd && attention_tc_supported(h->hd)) {
+        if (!launch_attention_bwd_tc(h->ctx(), qkv, out, dout, lse, h->dpre, dqkv, B, T, h->H))
+            h->host_error = "tensor-map encoding failed for the attention backward";
+    } else if (h->use_tc_attention)
         launch_attention_bwd_mma(h->ctx(), qkv, out, dout, lse, h->dpre, dqkv, B, T, h->H, h->hd);
     else
         launch_attention_bwd_simt<bf16>(h->ctx(), qkv, out, dout, lse, h->dpre, dqkv, B, T, h->H, h->hd);
@@ -617,6 +621,7 @@ int gpt2_create(const gpt2_config* cfg, void* stream, gpt2_handle** out) {
     if (const char* e = getenv("GPT2_B200_SIMT_GEMM")) h->use_tc_gemm = (e[0] == '0');
     if (const char* e = getenv("GPT2_B200_SIMT_ATTENTION")) h->use_tc_attention = (e[0] == '0');
     if (const char* e = getenv("GPT2_B200_TCGEN05_ATTENTION")) h->use_tcgen05_attention = (e[0] == '1');
+    if (const char* e = getenv("GPT2_B200_TCGEN05_ATTENTION_BWD")) h->use_tcgen05_attention_bwd = (e[0] == '1');
     build_layout(h);
 
     auto cleanup_fail = [&](int code, const std::string& msg) {

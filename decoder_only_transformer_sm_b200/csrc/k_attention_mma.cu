@@ -502,6 +502,16 @@ void bwd_launch(const Ctx& ctx, const bf16* qkv, const bf16* out, const bf16* do
 
 }  // namespace
 
+void launch_attention_bwd_pre(const Ctx& ctx, const bf16* out, const bf16* dout, float* dpre, int B, int Tn, int H,
+                              int hd) {
+    const long long n = (long long)B * H * Tn;
+    if (hd == 64)
+        flash_bwd_pre_kernel<64><<<(unsigned)ceil_div_ll(n, 256), 256, 0, ctx.stream>>>(out, dout, dpre, B, Tn, H);
+    else
+        flash_bwd_pre_kernel<32><<<(unsigned)ceil_div_ll(n, 256), 256, 0, ctx.stream>>>(out, dout, dpre, B, Tn, H);
+    ++*ctx.launches;
+}
+
 void launch_attention_fwd_mma(const Ctx& ctx, const bf16* qkv, bf16* out, float* lse, int B, int Tn, int H,
                               int hd) {
     if (hd == 64) fwd_launch<64>(ctx, qkv, out, lse, B, Tn, H);

@@ -13,9 +13,13 @@
 // 2-stage TMA ring; warp 1 issues, from one thread, S_j = Q K_j^T (M=128,
 // N=128, K=64) into one of two TMEM S buffers and PV_j = P_j V_j (M=128, N=64,
 // K=128; V described as an N-major operand) into one of two TMEM PV buffers;
-// warps 2..5 read S_j from TMEM (two passes: row max, then exp2 / row sum /
-// bf16 P into a 128-byte-swizzled K-major shared tile), then fold PV_{j-1}
-// into the register-resident output row: O = O * exp2(m_{j-2} - m_{j-1}) + PV.
+// warps 2..9 are the softmax warps, two per TMEM lane quarter: each owns 64 of
+// the 128 keys of S_j (one 64-key swizzle atom of P) and 32 of the 64 output
+// columns. They read S_j from TMEM in two passes (partial row max, exchanged
+// with the pair through shared memory; then exp2 / partial row sum / bf16 P
+// into the 128-byte-swizzled K-major shared tile), then fold their half of
+// PV_{j-1} into the register-resident output row:
+// O = O * exp2(m_{j-2} - m_{j-1}) + PV. The pair's row sums meet once at the end.
 // Every wait is bounded (2 s) and reports a timeout in the status word.
 #include <cudaTypedefs.h>
 
@@ -29,7 +33,8 @@ namespace {
 constexpr int HD = 64;
 constexpr int BQ = 128, BKV = 128;
 constexpr int KV_STAGES = 2;
-constexpr int THREADS = 192;
+constexpr int SM_WARPS = 8;                       // softmax warps: 2 per TMEM lane quarter
+constexpr int THREADS = 64 + 32 * SM_WARPS;
 constexpr int TILE_BYTES = 128 * HD * 2;          // 16 KB: 128 rows x 128 bytes
 constexpr int P_BYTES = BQ * BKV * 2;             // 32 KB: two 64-key swizzle atoms of 16 KB
 constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_PV0 = 256, TM_PV1 = 320;
@@ -44,6 +49,8 @@ struct Ctl {
     uint64_t drain;
     uint32_t tmem_base;
     uint32_t abort;
+    float mx[2][2][BQ];                           // [tile parity][column half][row]: partial row max
+    float lsum[2][BQ];                            // [column half][row]: partial row sum at the end
 };
 
 // smem: Q | K[2] | V[2] | P[2] | ctl
@@ -55,6 +62,29 @@ constexpr int OFF_CTL = OFF_P + 2 * P_BYTES;
 constexpr size_t SMEM_BYTES = OFF_CTL + sizeof(Ctl) + 1024;
 
 __device__ __forceinline__ uint32_t swz128(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
+
+// 2^x with the hardware approximation (ex2.approx; 2^-inf = 0). Its relative
+// error (about 2^-22) is far below the bf16 rounding of P and dS.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void ew_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ uint4 pack8_bf16(const float* v) {
+    uint4 q;
+    __nv_bfloat162 t0 = __floats2bfloat162_rn(v[0], v[1]);
+    __nv_bfloat162 t1 = __floats2bfloat162_rn(v[2], v[3]);
+    __nv_bfloat162 t2 = __floats2bfloat162_rn(v[4], v[5]);
+    __nv_bfloat162 t3 = __floats2bfloat162_rn(v[6], v[7]);
+    q.x = *reinterpret_cast<uint32_t*>(&t0);
+    q.y = *reinterpret_cast<uint32_t*>(&t1);
+    q.z = *reinterpret_cast<uint32_t*>(&t2);
+    q.w = *reinterpret_cast<uint32_t*>(&t3);
+    return q;
+}
 
 __global__ void __launch_bounds__(THREADS, 1)
     flash_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse,
@@ -80,10 +110,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&ctl->s_full[i], 1);
-            tc::mbar_init(&ctl->s_empty[i], 4);
-            tc::mbar_init(&ctl->p_full[i], 4);
+            tc::mbar_init(&ctl->s_empty[i], SM_WARPS);
+            tc::mbar_init(&ctl->p_full[i], SM_WARPS);
             tc::mbar_init(&ctl->pv_full[i], 1);
-            tc::mbar_init(&ctl->pv_empty[i], 4);
+            tc::mbar_init(&ctl->pv_empty[i], SM_WARPS);
         }
         tc::mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
@@ -159,14 +189,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else {
         // ---------------------------------------------------- softmax / output
+        // Warp pair (chalf 0/1) of a lane quarter shares 32 query rows: each warp
+        // owns 64 of the 128 keys of an S tile (one swizzle atom of P) and 32 of
+        // the 64 output columns. Only the row max is exchanged per tile.
         const int quarter = warp & 3;
+        const int chalf = (warp - 2) >> 2;
         const int r = quarter * 32 + lane;            // query row within the tile = TMEM lane
         const int q = q0 + r;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const float sl2 = LOG2E * 0.125f;             // log2(e) / sqrt(64)
-        float o[HD];
+        float o[32];
 #pragma unroll
-        for (int d = 0; d < HD; ++d) o[d] = 0.f;
+        for (int d = 0; d < 32; ++d) o[d] = 0.f;
         float m = -INFINITY, l = 0.f, corr_prev = 1.f;
         bool ok = true;
         auto consume_pv = [&](int j) -> bool {
@@ -177,69 +211,60 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!w) return false;
             tc::fence_after_sync();
             float pv[32];
+            tc::tmem_ld_32x32b_x32(tmem + (pb ? TM_PV1 : TM_PV0) + chalf * 32 + lane_off, pv);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                tc::tmem_ld_32x32b_x32(tmem + (pb ? TM_PV1 : TM_PV0) + half * 32 + lane_off, pv);
-#pragma unroll
-                for (int d = 0; d < 32; ++d) o[half * 32 + d] = fmaf(o[half * 32 + d], corr_prev, pv[d]);
-            }
+            for (int d = 0; d < 32; ++d) o[d] = fmaf(o[d], corr_prev, pv[d]);
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&ctl->pv_empty[pb]);
             return true;
         };
+        // Every softmax warp passes the named barrier once per tile and twice after
+        // the loop, also after a failed wait (then without work), so that none of
+        // them is left waiting there.
         for (int j = 0; j < n_kv; ++j) {
             const int sb = j & 1;
             uint32_t w = 0;
-            if (lane == 0) w = tc::mbar_wait(&ctl->s_full[sb], (j >> 1) & 1, abort, status) ? 1u : 0u;
+            if (lane == 0 && ok) w = tc::mbar_wait(&ctl->s_full[sb], (j >> 1) & 1, abort, status) ? 1u : 0u;
             w = __shfl_sync(0xffffffffu, w, 0);
-            if (!w) { ok = false; break; }
-            tc::fence_after_sync();
-            const uint32_t s_addr = tmem + (sb ? TM_S1 : TM_S0) + lane_off;
-            const bool diag = (j * BKV + BKV > q0);   // tile reaches past the first query of the block
-            // pass 1: row max
+            const uint32_t s_addr = tmem + (sb ? TM_S1 : TM_S0) + chalf * 64 + lane_off;
+            const int kbase = j * BKV + chalf * 64;   // first key of this warp's columns
+            const bool diag = (j * BKV + BKV > q0);
+            // pass 1: partial row max over this warp's 64 keys, exchanged with the pair
             float mx = -INFINITY;
-#pragma unroll 1
-            for (int c = 0; c < BKV; c += 32) {
-                float sv[32];
-                tc::tmem_ld_32x32b_x32(s_addr + c, sv);
+            if (w) {
+                tc::fence_after_sync();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int key = j * BKV + c + e;
-                    if (!diag || key <= q) mx = fmaxf(mx, sv[e]);
+                for (int c = 0; c < 64; c += 32) {
+                    float sv[32];
+                    tc::tmem_ld_32x32b_x32(s_addr + c, sv);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (!diag || kbase + c + e <= q) mx = fmaxf(mx, sv[e]);
                 }
             }
+            ctl->mx[sb][chalf][r] = mx;
+            ew_bar();
+            if (!w) { ok = false; continue; }
+            mx = fmaxf(mx, ctl->mx[sb][chalf ^ 1][r]);
             const float m_new = fmaxf(m, mx * sl2);
-            const float corr = exp2f(m - m_new);   // m = -inf at the start: 0
-            // pass 2: P = exp2(s * sl2 - m_new) as bf16 into the K-major swizzled tile
-            uint8_t* pt = smem + OFF_P + sb * P_BYTES;
+            const float corr = ex2(m - m_new);   // m = -inf at the start: 0
+            // pass 2: P = exp2(s * sl2 - m_new) as bf16 into this warp's 64-key atom of P
+            uint8_t* pt = smem + OFF_P + sb * P_BYTES + chalf * TILE_BYTES;
             float rs = 0.f;
-#pragma unroll 1
-            for (int c = 0; c < BKV; c += 32) {
+#pragma unroll
+            for (int c = 0; c < 64; c += 32) {
                 float sv[32];
                 tc::tmem_ld_32x32b_x32(s_addr + c, sv);
-                float p[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const int key = j * BKV + c + e;
-                    p[e] = (!diag || key <= q) ? exp2f(fmaf(sv[e], sl2, -m_new)) : 0.f;
-                    rs += p[e];
+                    const float p = (!diag || kbase + c + e <= q) ? ex2(fmaf(sv[e], sl2, -m_new)) : 0.f;
+                    sv[e] = p;
+                    rs += p;
                 }
-                const int atom = c >> 6;
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const int chunk = ((c & 63) >> 3) + g;   // 16-byte chunk within the 128-byte atom row
-                    uint4 v;
-                    __nv_bfloat162 t0 = __floats2bfloat162_rn(p[8 * g + 0], p[8 * g + 1]);
-                    __nv_bfloat162 t1 = __floats2bfloat162_rn(p[8 * g + 2], p[8 * g + 3]);
-                    __nv_bfloat162 t2 = __floats2bfloat162_rn(p[8 * g + 4], p[8 * g + 5]);
-                    __nv_bfloat162 t3 = __floats2bfloat162_rn(p[8 * g + 6], p[8 * g + 7]);
-                    v.x = *reinterpret_cast<uint32_t*>(&t0);
-                    v.y = *reinterpret_cast<uint32_t*>(&t1);
-                    v.z = *reinterpret_cast<uint32_t*>(&t2);
-                    v.w = *reinterpret_cast<uint32_t*>(&t3);
-                    *reinterpret_cast<uint4*>(pt + atom * TILE_BYTES + swz128(r, chunk)) = v;
-                }
+                for (int g = 0; g < 4; ++g)
+                    *reinterpret_cast<uint4*>(pt + swz128(r, (c >> 3) + g)) = pack8_bf16(sv + 8 * g);
             }
             l = l * corr + rs;
             m = m_new;
@@ -250,30 +275,30 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tc::mbar_arrive(&ctl->p_full[sb]);
                 tc::mbar_arrive(&ctl->s_empty[sb]);
             }
-            if (j > 0 && !consume_pv(j - 1)) { ok = false; break; }
+            if (j > 0 && !consume_pv(j - 1)) { ok = false; continue; }
             corr_prev = corr;
         }
         if (ok && n_kv > 0) ok = consume_pv(n_kv - 1);
+        // row sum of both halves (the barrier is reached by every softmax warp)
+        ctl->lsum[chalf][r] = l;
+        ew_bar();
+        const float l_tot = l + ctl->lsum[chalf ^ 1][r];
         if (ok) {
             // out row q: O / l, staged through the Q tile (free now) for 128-byte row stores
-            const float inv = 1.f / l;
+            const float inv = 1.f / l_tot;
             uint8_t* stage = smem + OFF_Q;
-            __syncwarp();
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint4 v;
-                __nv_bfloat162 t0 = __floats2bfloat162_rn(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
-                __nv_bfloat162 t1 = __floats2bfloat162_rn(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
-                __nv_bfloat162 t2 = __floats2bfloat162_rn(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
-                __nv_bfloat162 t3 = __floats2bfloat162_rn(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
-                v.x = *reinterpret_cast<uint32_t*>(&t0);
-                v.y = *reinterpret_cast<uint32_t*>(&t1);
-                v.z = *reinterpret_cast<uint32_t*>(&t2);
-                v.w = *reinterpret_cast<uint32_t*>(&t3);
-                *reinterpret_cast<uint4*>(stage + swz128(r, c)) = v;
+            for (int g = 0; g < 4; ++g) {
+                float t[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) t[e] = o[8 * g + e] * inv;
+                *reinterpret_cast<uint4*>(stage + swz128(r, chalf * 4 + g)) = pack8_bf16(t);
             }
-            if (q < Tn) lse[(long long)bh * Tn + q] = (m + log2f(l)) / LOG2E;
-            __syncwarp();
+            if (chalf == 0 && q < Tn) lse[(long long)bh * Tn + q] = (m + log2f(l_tot)) / LOG2E;
+        }
+        ew_bar();
+        if (ok && chalf == 0) {
+            uint8_t* stage = smem + OFF_Q;
             const int lrow = lane >> 3, lseg = lane & 7;
 #pragma unroll
             for (int st = 0; st < 8; ++st) {
@@ -281,6 +306,461 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (q0 + rr < Tn)
                     *reinterpret_cast<uint4*>(out + ((long long)b * Tn + q0 + rr) * C + h * HD + lseg * 8) =
                         *reinterpret_cast<const uint4*>(stage + swz128(rr, lseg));
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) tc::tmem_dealloc(tmem, 512);
+}
+
+// ============================================================================
+// Backward. D = rowsum(dO * O) comes from the pre-pass kernel. With
+// P = exp(S - lse) recomputed from the saved lse:
+//   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),
+//   dK = dS^T Q / sqrt(64),  dQ = dS K / sqrt(64).
+// dK/dV kernel: one CTA per (b, h, 128-key tile); it walks the 64-query tiles
+// at or after the key tile. S^T = K Q^T and dP^T = V dO^T (M=128 keys, N=64
+// queries) go to double-buffered TMEM so the tensor core computes tile i+1
+// while 4 warps turn tile i into P^T and dS^T (bf16, K-major shared tiles);
+// dV += P^T dO and dK += dS^T Q (dO and Q as N-major operands) accumulate in
+// TMEM. dQ kernel: one CTA per (b, h, 128-query tile) over the 64-key tiles at
+// or before it: S = Q K^T, dP = dO V^T, dS, then dQ += dS K in TMEM.
+// ============================================================================
+constexpr int BW_EW_WARPS = 8;                     // 2 warps per TMEM lane quarter, 32 columns each
+constexpr int BW_THREADS = 64 + 32 * BW_EW_WARPS;
+constexpr int T64_BYTES = 64 * HD * 2;      // 8 KB: 64 rows x 128 bytes
+constexpr int T128_BYTES = 128 * HD * 2;    // 16 KB
+
+// Write one 64-column bf16 result row (128 bytes) per thread of a 4-warp group
+// through a swizzled 128-row staging tile, then copy whole rows to global
+// memory: dst(row) = base + row * ld (elements), rows >= n_rows skipped.
+__device__ __forceinline__ void store_rows_64(uint8_t* stage, int r, const float* v, float scale, bf16* base,
+                                              long long ld, int n_rows) {
+    const int lane = threadIdx.x & 31, quarter = (threadIdx.x >> 5) & 3;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        float t[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t[e] = v[8 * c + e] * scale;
+        *reinterpret_cast<uint4*>(stage + swz128(r, c)) = pack8_bf16(t);
+    }
+    __syncwarp();
+    const int lrow = lane >> 3, lseg = lane & 7;
+#pragma unroll
+    for (int st = 0; st < 8; ++st) {
+        const int rr = quarter * 32 + st * 4 + lrow;
+        if (rr < n_rows)
+            *reinterpret_cast<uint4*>(base + (long long)rr * ld + lseg * 8) =
+                *reinterpret_cast<const uint4*>(stage + swz128(rr, lseg));
+    }
+    __syncwarp();
+}
+
+constexpr int DKV_STAGES = 3;
+struct CtlDkv {
+    uint64_t kv_full;
+    uint64_t q_full[DKV_STAGES], q_empty[DKV_STAGES];
+    uint64_t st_full[2], st_empty[2];
+    uint64_t ew_done[2], pds_free[2];
+    uint64_t acc_done;
+    uint64_t drain;
+    uint32_t tmem_base;
+    uint32_t abort;
+    float lse2[2][64];
+    float dd[2][64];
+};
+// smem: K | V | (Q | dO) stages | Pt[2] | dSt[2] | ctl
+constexpr int DKV_OFF_K = 0;
+constexpr int DKV_OFF_V = DKV_OFF_K + T128_BYTES;
+constexpr int DKV_OFF_Q = DKV_OFF_V + T128_BYTES;
+constexpr int DKV_STAGE_BYTES = 2 * T64_BYTES;                  // Q tile + dO tile
+constexpr int DKV_OFF_PT = DKV_OFF_Q + DKV_STAGES * DKV_STAGE_BYTES;
+constexpr int DKV_OFF_DST = DKV_OFF_PT + 2 * T128_BYTES;        // 128 keys x 64 queries bf16 = 16 KB each
+constexpr int DKV_OFF_CTL = DKV_OFF_DST + 2 * T128_BYTES;
+constexpr size_t DKV_SMEM = DKV_OFF_CTL + sizeof(CtlDkv) + 1024;
+// TMEM columns
+constexpr uint32_t DKV_ST = 0, DKV_DPT = 128, DKV_DV = 256, DKV_DK = 320;
+
+__global__ void __launch_bounds__(BW_THREADS, 1)
+    flash_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q,
+                            const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ lse,
+                            const float* __restrict__ dpre, bf16* __restrict__ dqkv, int Tn, int H,
+                            unsigned* status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    CtlDkv* ctl = reinterpret_cast<CtlDkv*>(smem + DKV_OFF_CTL);
+    volatile uint32_t* abort = &ctl->abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_kt = gridDim.x;
+    const int kt = n_kt - 1 - blockIdx.x;               // longest query ranges first
+    const int bh = blockIdx.y, b = bh / H, h = bh % H;
+    const int C = H * HD;
+    const int k0 = kt * 128;
+    const int n_q64 = (Tn + 63) / 64;
+    const int it0 = k0 / 64;                            // first 64-query tile that sees these keys
+    const int n_it = n_q64 - it0;
+    const int row_base = b * Tn;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&ctl->kv_full, 1);
+        for (int s = 0; s < DKV_STAGES; ++s) {
+            tc::mbar_init(&ctl->q_full[s], 1);
+            tc::mbar_init(&ctl->q_empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&ctl->st_full[i], 1);
+            tc::mbar_init(&ctl->st_empty[i], BW_EW_WARPS);
+            tc::mbar_init(&ctl->ew_done[i], BW_EW_WARPS);
+            tc::mbar_init(&ctl->pds_free[i], 1);
+        }
+        tc::mbar_init(&ctl->acc_done, 1);
+        tc::mbar_init(&ctl->drain, 1);
+        ctl->abort = 0;
+        tc::fence_barrier_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(&ctl->tmem_base, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = ctl->tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tc::tma_prefetch_desc(&tm_kv);
+            tc::tma_prefetch_desc(&tm_q);
+            tc::tma_prefetch_desc(&tm_do);
+            tc::mbar_expect_tx(&ctl->kv_full, 2 * T128_BYTES);
+            tc::tma_load_2d(smem + DKV_OFF_K, &tm_kv, C + h * HD, row_base + k0, &ctl->kv_full);
+            tc::tma_load_2d(smem + DKV_OFF_V, &tm_kv, 2 * C + h * HD, row_base + k0, &ctl->kv_full);
+            for (int it = 0; it < n_it; ++it) {
+                const int s = it % DKV_STAGES;
+                if (!tc::mbar_wait(&ctl->q_empty[s], ((it / DKV_STAGES) & 1) ^ 1, abort, status)) break;
+                const int q0 = (it0 + it) * 64;
+                uint8_t* st = smem + DKV_OFF_Q + s * DKV_STAGE_BYTES;
+                tc::mbar_expect_tx(&ctl->q_full[s], 2 * T64_BYTES);
+                tc::tma_load_2d(st, &tm_q, h * HD, row_base + q0, &ctl->q_full[s]);
+                tc::tma_load_2d(st + T64_BYTES, &tm_do, h * HD, row_base + q0, &ctl->q_full[s]);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc_st = tc::idesc_bf16_f32(128, 64, 0, 0);   // K Q^T, V dO^T
+            constexpr uint32_t idesc_acc = tc::idesc_bf16_f32(128, 64, 0, 1);  // P^T dO, dS^T Q
+            const uint32_t k_addr = tc::smem_u32(smem + DKV_OFF_K), v_addr = tc::smem_u32(smem + DKV_OFF_V);
+            bool ok = tc::mbar_wait(&ctl->kv_full, 0, abort, status);
+            auto accumulate = [&](int it) -> bool {   // dV += P^T dO, dK += dS^T Q for tile it
+                const int r = it & 1, s = it % DKV_STAGES;
+                if (!tc::mbar_wait(&ctl->ew_done[r], (it >> 1) & 1, abort, status)) return false;
+                tc::fence_after_sync();
+                const uint32_t q_addr = tc::smem_u32(smem + DKV_OFF_Q + s * DKV_STAGE_BYTES);
+                const uint32_t do_addr = q_addr + T64_BYTES;
+                const uint32_t pt = tc::smem_u32(smem + DKV_OFF_PT + r * T128_BYTES);
+                const uint32_t dst = tc::smem_u32(smem + DKV_OFF_DST + r * T128_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {   // K = 64 queries
+                    const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+                    tc::mma_bf16(tmem + DKV_DV, tc::smem_desc_sw128(pt + kk * 32, 16, 1024),
+                                 tc::smem_desc_sw128(do_addr + kk * 2048, T64_BYTES, 1024), idesc_acc, acc);
+                    tc::mma_bf16(tmem + DKV_DK, tc::smem_desc_sw128(dst + kk * 32, 16, 1024),
+                                 tc::smem_desc_sw128(q_addr + kk * 2048, T64_BYTES, 1024), idesc_acc, acc);
+                }
+                tc::mma_commit(&ctl->pds_free[r]);
+                tc::mma_commit(&ctl->q_empty[s]);
+                return true;
+            };
+            for (int it = 0; it < n_it && ok; ++it) {
+                const int r = it & 1, s = it % DKV_STAGES;
+                if (!tc::mbar_wait(&ctl->q_full[s], (it / DKV_STAGES) & 1, abort, status)) break;
+                if (!tc::mbar_wait(&ctl->st_empty[r], ((it >> 1) & 1) ^ 1, abort, status)) break;
+                tc::fence_after_sync();
+                const uint32_t q_addr = tc::smem_u32(smem + DKV_OFF_Q + s * DKV_STAGE_BYTES);
+                const uint32_t do_addr = q_addr + T64_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    tc::mma_bf16(tmem + DKV_ST + r * 64, tc::smem_desc_sw128(k_addr + kk * 32, 16, 1024),
+                                 tc::smem_desc_sw128(q_addr + kk * 32, 16, 1024), idesc_st, kk > 0 ? 1u : 0u);
+                    tc::mma_bf16(tmem + DKV_DPT + r * 64, tc::smem_desc_sw128(v_addr + kk * 32, 16, 1024),
+                                 tc::smem_desc_sw128(do_addr + kk * 32, 16, 1024), idesc_st, kk > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(&ctl->st_full[r]);
+                if (it > 0 && !accumulate(it - 1)) { ok = false; break; }
+            }
+            if (ok && n_it > 0) ok = accumulate(n_it - 1);
+            tc::mma_commit(&ctl->acc_done);
+            volatile uint32_t no_abort = 0;
+            tc::mma_commit(&ctl->drain);
+            tc::mbar_wait(&ctl->drain, 0, &no_abort, status);
+        }
+    } else {
+        // ------------------------------------------- P^T, dS^T (thread = key row)
+        const int quarter = warp & 3;
+        const int chalf = (warp - 2) >> 2;              // query columns [32 chalf, 32 chalf + 32)
+        const int r = quarter * 32 + lane;              // key row in the tile = TMEM lane
+        const int key = k0 + r;
+        const int et = threadIdx.x - 64;                // 0..255 within the element-wise warps
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const float sl2 = LOG2E * 0.125f;
+        // per-query lse (log2 units) and D of the next tile, one value per thread
+        auto fetch = [&](int it) -> float {
+            const int q = (it0 + it) * 64 + (et & 63);
+            if (et < 64) return q < Tn ? lse[(long long)bh * Tn + q] * LOG2E : INFINITY;
+            if (et < 128) return q < Tn ? dpre[(long long)bh * Tn + q] : 0.f;
+            return 0.f;
+        };
+        float nxt = n_it > 0 ? fetch(0) : 0.f;
+        bool ok = true;
+        for (int it = 0; it < n_it; ++it) {
+            const int rb = it & 1;
+            const int q0 = (it0 + it) * 64;
+            if (et < 64) ctl->lse2[rb][et] = nxt;
+            else if (et < 128) ctl->dd[rb][et - 64] = nxt;
+            ew_bar();
+            if (it + 1 < n_it) nxt = fetch(it + 1);
+            uint32_t w = 0;
+            if (lane == 0 && ok) {
+                w = tc::mbar_wait(&ctl->st_full[rb], (it >> 1) & 1, abort, status) ? 1u : 0u;
+                if (w) w = tc::mbar_wait(&ctl->pds_free[rb], ((it >> 1) & 1) ^ 1, abort, status) ? 1u : 0u;
+            }
+            w = __shfl_sync(0xffffffffu, w, 0);
+            // after a failed wait keep looping without work, so that every
+            // element-wise warp reaches the named barrier equally often
+            if (!w) { ok = false; continue; }
+            tc::fence_after_sync();
+            const bool diag = (q0 < k0 + 128);          // some queries of the tile precede some keys
+            uint8_t* pt = smem + DKV_OFF_PT + rb * T128_BYTES;
+            uint8_t* dst = smem + DKV_OFF_DST + rb * T128_BYTES;
+            float sv[32], dp[32];
+            tc::tmem_ld_32x32b_x32(tmem + DKV_ST + rb * 64 + chalf * 32 + lane_off, sv);
+            tc::tmem_ld_32x32b_x32(tmem + DKV_DPT + rb * 64 + chalf * 32 + lane_off, dp);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int qi = chalf * 32 + e;
+                float p = ex2(fmaf(sv[e], sl2, -ctl->lse2[rb][qi]));
+                if (diag && key > q0 + qi) p = 0.f;
+                sv[e] = p;
+                dp[e] = p * (dp[e] - ctl->dd[rb][qi]);
+            }
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                const int chunk = chalf * 4 + g;
+                *reinterpret_cast<uint4*>(pt + swz128(r, chunk)) = pack8_bf16(sv + 8 * g);
+                *reinterpret_cast<uint4*>(dst + swz128(r, chunk)) = pack8_bf16(dp + 8 * g);
+            }
+            tc::fence_proxy_async_smem();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_arrive(&ctl->st_empty[rb]);
+                tc::mbar_arrive(&ctl->ew_done[rb]);
+            }
+        }
+        if (ok && chalf == 0) {
+            uint32_t w = 0;
+            if (lane == 0) w = tc::mbar_wait(&ctl->acc_done, 0, abort, status) ? 1u : 0u;
+            w = __shfl_sync(0xffffffffu, w, 0);
+            if (w) {
+                tc::fence_after_sync();
+                float v[64];
+                tc::tmem_ld_32x32b_x32(tmem + DKV_DK + lane_off, v);
+                tc::tmem_ld_32x32b_x32(tmem + DKV_DK + 32 + lane_off, v + 32);
+                bf16* kbase = dqkv + ((long long)row_base + k0) * 3 * C + C + h * HD;
+                uint8_t* stage = smem + DKV_OFF_PT;     // free: every MMA has completed
+                store_rows_64(stage, r, v, 0.125f, kbase, 3LL * C, Tn - k0);
+                tc::tmem_ld_32x32b_x32(tmem + DKV_DV + lane_off, v);
+                tc::tmem_ld_32x32b_x32(tmem + DKV_DV + 32 + lane_off, v + 32);
+                store_rows_64(stage, r, v, 1.0f, kbase + C, 3LL * C, Tn - k0);
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) tc::tmem_dealloc(tmem, 512);
+}
+
+constexpr int DQ_STAGES = 3;
+struct CtlDq {
+    uint64_t q_full;
+    uint64_t kv_full[DQ_STAGES], kv_empty[DQ_STAGES];
+    uint64_t s_full[2], s_empty[2];
+    uint64_t ds_full[2], ds_free[2];
+    uint64_t acc_done;
+    uint64_t drain;
+    uint32_t tmem_base;
+    uint32_t abort;
+};
+// smem: Q | dO | (K | V) stages | dS[2] | ctl
+constexpr int DQ_OFF_Q = 0;
+constexpr int DQ_OFF_DO = DQ_OFF_Q + T128_BYTES;
+constexpr int DQ_OFF_KV = DQ_OFF_DO + T128_BYTES;
+constexpr int DQ_STAGE_BYTES = 2 * T64_BYTES;
+constexpr int DQ_OFF_DS = DQ_OFF_KV + DQ_STAGES * DQ_STAGE_BYTES;
+constexpr int DQ_OFF_CTL = DQ_OFF_DS + 2 * T128_BYTES;   // 128 queries x 64 keys bf16 = 16 KB each
+constexpr size_t DQ_SMEM = DQ_OFF_CTL + sizeof(CtlDq) + 1024;
+constexpr uint32_t DQ_S = 0, DQ_DP = 128, DQ_DQ = 256;
+
+__global__ void __launch_bounds__(BW_THREADS, 1)
+    flash_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q128, const __grid_constant__ CUtensorMap tm_kv64,
+                           const __grid_constant__ CUtensorMap tm_do128, const float* __restrict__ lse,
+                           const float* __restrict__ dpre, bf16* __restrict__ dqkv, int Tn, int H,
+                           unsigned* status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    CtlDq* ctl = reinterpret_cast<CtlDq*>(smem + DQ_OFF_CTL);
+    volatile uint32_t* abort = &ctl->abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_qt = gridDim.x;
+    const int qt = n_qt - 1 - blockIdx.x;
+    const int bh = blockIdx.y, b = bh / H, h = bh % H;
+    const int C = H * HD;
+    const int q0 = qt * 128;
+    const int n_k64 = (min(Tn, q0 + 128) + 63) / 64;    // key tiles that some query of the tile sees
+    const int row_base = b * Tn;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&ctl->q_full, 1);
+        for (int s = 0; s < DQ_STAGES; ++s) {
+            tc::mbar_init(&ctl->kv_full[s], 1);
+            tc::mbar_init(&ctl->kv_empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&ctl->s_full[i], 1);
+            tc::mbar_init(&ctl->s_empty[i], BW_EW_WARPS);
+            tc::mbar_init(&ctl->ds_full[i], BW_EW_WARPS);
+            tc::mbar_init(&ctl->ds_free[i], 1);
+        }
+        tc::mbar_init(&ctl->acc_done, 1);
+        tc::mbar_init(&ctl->drain, 1);
+        ctl->abort = 0;
+        tc::fence_barrier_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(&ctl->tmem_base, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = ctl->tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tc::tma_prefetch_desc(&tm_q128);
+            tc::tma_prefetch_desc(&tm_kv64);
+            tc::tma_prefetch_desc(&tm_do128);
+            tc::mbar_expect_tx(&ctl->q_full, 2 * T128_BYTES);
+            tc::tma_load_2d(smem + DQ_OFF_Q, &tm_q128, h * HD, row_base + q0, &ctl->q_full);
+            tc::tma_load_2d(smem + DQ_OFF_DO, &tm_do128, h * HD, row_base + q0, &ctl->q_full);
+            for (int j = 0; j < n_k64; ++j) {
+                const int s = j % DQ_STAGES;
+                if (!tc::mbar_wait(&ctl->kv_empty[s], ((j / DQ_STAGES) & 1) ^ 1, abort, status)) break;
+                uint8_t* st = smem + DQ_OFF_KV + s * DQ_STAGE_BYTES;
+                tc::mbar_expect_tx(&ctl->kv_full[s], 2 * T64_BYTES);
+                tc::tma_load_2d(st, &tm_kv64, C + h * HD, row_base + j * 64, &ctl->kv_full[s]);
+                tc::tma_load_2d(st + T64_BYTES, &tm_kv64, 2 * C + h * HD, row_base + j * 64, &ctl->kv_full[s]);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 64, 0, 0);    // Q K^T, dO V^T
+            constexpr uint32_t idesc_dq = tc::idesc_bf16_f32(128, 64, 0, 1);   // dS K
+            const uint32_t q_addr = tc::smem_u32(smem + DQ_OFF_Q), do_addr = tc::smem_u32(smem + DQ_OFF_DO);
+            bool ok = tc::mbar_wait(&ctl->q_full, 0, abort, status);
+            auto accumulate = [&](int j) -> bool {   // dQ += dS K for key tile j
+                const int r = j & 1, s = j % DQ_STAGES;
+                if (!tc::mbar_wait(&ctl->ds_full[r], (j >> 1) & 1, abort, status)) return false;
+                tc::fence_after_sync();
+                const uint32_t k_addr = tc::smem_u32(smem + DQ_OFF_KV + s * DQ_STAGE_BYTES);
+                const uint32_t ds = tc::smem_u32(smem + DQ_OFF_DS + r * T128_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)   // K = 64 keys
+                    tc::mma_bf16(tmem + DQ_DQ, tc::smem_desc_sw128(ds + kk * 32, 16, 1024),
+                                 tc::smem_desc_sw128(k_addr + kk * 2048, T64_BYTES, 1024), idesc_dq,
+                                 (j > 0 || kk > 0) ? 1u : 0u);
+                tc::mma_commit(&ctl->ds_free[r]);
+                tc::mma_commit(&ctl->kv_empty[s]);
+                return true;
+            };
+            for (int j = 0; j < n_k64 && ok; ++j) {
+                const int r = j & 1, s = j % DQ_STAGES;
+                if (!tc::mbar_wait(&ctl->kv_full[s], (j / DQ_STAGES) & 1, abort, status)) break;
+                if (!tc::mbar_wait(&ctl->s_empty[r], ((j >> 1) & 1) ^ 1, abort, status)) break;
+                tc::fence_after_sync();
+                const uint32_t k_addr = tc::smem_u32(smem + DQ_OFF_KV + s * DQ_STAGE_BYTES);
+                const uint32_t v_addr = k_addr + T64_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    tc::mma_bf16(tmem + DQ_S + r * 64, tc::smem_desc_sw128(q_addr + kk * 32, 16, 1024),
+                                 tc::smem_desc_sw128(k_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                    tc::mma_bf16(tmem + DQ_DP + r * 64, tc::smem_desc_sw128(do_addr + kk * 32, 16, 1024),
+                                 tc::smem_desc_sw128(v_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(&ctl->s_full[r]);
+                if (j > 0 && !accumulate(j - 1)) { ok = false; break; }
+            }
+            if (ok && n_k64 > 0) ok = accumulate(n_k64 - 1);
+            tc::mma_commit(&ctl->acc_done);
+            volatile uint32_t no_abort = 0;
+            tc::mma_commit(&ctl->drain);
+            tc::mbar_wait(&ctl->drain, 0, &no_abort, status);
+        }
+    } else {
+        // --------------------------------------------------- dS (thread = query row)
+        const int quarter = warp & 3;
+        const int chalf = (warp - 2) >> 2;              // key columns [32 chalf, 32 chalf + 32)
+        const int r = quarter * 32 + lane;
+        const int q = q0 + r;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const float sl2 = LOG2E * 0.125f;
+        const float L2 = q < Tn ? lse[(long long)bh * Tn + q] * LOG2E : INFINITY;
+        const float Dv = q < Tn ? dpre[(long long)bh * Tn + q] : 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_k64; ++j) {
+            const int rb = j & 1;
+            uint32_t w = 0;
+            if (lane == 0) {
+                w = tc::mbar_wait(&ctl->s_full[rb], (j >> 1) & 1, abort, status) ? 1u : 0u;
+                if (w) w = tc::mbar_wait(&ctl->ds_free[rb], ((j >> 1) & 1) ^ 1, abort, status) ? 1u : 0u;
+            }
+            w = __shfl_sync(0xffffffffu, w, 0);
+            if (!w) { ok = false; break; }
+            tc::fence_after_sync();
+            const bool diag = (j * 64 + 64 > q0);
+            uint8_t* ds = smem + DQ_OFF_DS + rb * T128_BYTES;
+            float sv[32], dp[32];
+            tc::tmem_ld_32x32b_x32(tmem + DQ_S + rb * 64 + chalf * 32 + lane_off, sv);
+            tc::tmem_ld_32x32b_x32(tmem + DQ_DP + rb * 64 + chalf * 32 + lane_off, dp);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                float p = ex2(fmaf(sv[e], sl2, -L2));
+                if (diag && j * 64 + chalf * 32 + e > q) p = 0.f;
+                dp[e] = p * (dp[e] - Dv);
+            }
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+                *reinterpret_cast<uint4*>(ds + swz128(r, chalf * 4 + g)) = pack8_bf16(dp + 8 * g);
+            tc::fence_proxy_async_smem();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_arrive(&ctl->s_empty[rb]);
+                tc::mbar_arrive(&ctl->ds_full[rb]);
+            }
+        }
+        if (ok && chalf == 0) {
+            uint32_t w = 0;
+            if (lane == 0) w = tc::mbar_wait(&ctl->acc_done, 0, abort, status) ? 1u : 0u;
+            w = __shfl_sync(0xffffffffu, w, 0);
+            if (w) {
+                tc::fence_after_sync();
+                float v[64];
+                tc::tmem_ld_32x32b_x32(tmem + DQ_DQ + lane_off, v);
+                tc::tmem_ld_32x32b_x32(tmem + DQ_DQ + 32 + lane_off, v + 32);
+                bf16* qbase = dqkv + ((long long)row_base + q0) * 3 * C + h * HD;
+                store_rows_64(smem + DQ_OFF_DS, r, v, 0.125f, qbase, 3LL * C, Tn - q0);
             }
         }
     }
@@ -326,6 +806,40 @@ bool launch_attention_fwd_tc(const Ctx& ctx, const bf16* qkv, bf16* out, float* 
     dim3 grid(ceil_div(Tn, BQ), B * H);
     flash_fwd_tc_kernel<<<grid, THREADS, SMEM_BYTES, ctx.stream>>>(m, out, lse, Tn, H, ctx.status);
     ++*ctx.launches;
+    return true;
+}
+
+bool launch_attention_bwd_tc(const Ctx& ctx, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
+                             float* dpre, bf16* dqkv, int B, int Tn, int H) {
+    auto fn = encode_fn_attn();
+    if (!fn) return false;
+    const long long C = (long long)H * HD;
+    auto make = [&](CUtensorMap* m, const bf16* base, long long cols, int box_rows) {
+        cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)B * Tn};
+        cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+        cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+        cuuint32_t estr[2] = {1, 1};
+        return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<bf16*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    };
+    CUtensorMap qkv128, qkv64, do64, do128;
+    if (!make(&qkv128, qkv, 3 * C, 128) || !make(&qkv64, qkv, 3 * C, 64) || !make(&do64, dout, C, 64) ||
+        !make(&do128, dout, C, 128))
+        return false;
+    static bool configured = false;
+    if (!configured) {
+        cudaFuncSetAttribute(flash_bwd_dkv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DKV_SMEM);
+        cudaFuncSetAttribute(flash_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DQ_SMEM);
+        configured = true;
+    }
+    launch_attention_bwd_pre(ctx, out, dout, dpre, B, Tn, H, HD);
+    const dim3 grid(ceil_div(Tn, 128), B * H);
+    flash_bwd_dkv_tc_kernel<<<grid, BW_THREADS, DKV_SMEM, ctx.stream>>>(qkv128, qkv64, do64, lse, dpre, dqkv, Tn, H,
+                                                                         ctx.status);
+    flash_bwd_dq_tc_kernel<<<grid, BW_THREADS, DQ_SMEM, ctx.stream>>>(qkv128, qkv64, do128, lse, dpre, dqkv, Tn, H,
+                                                                       ctx.status);
+    *ctx.launches += 2;
     return true;
 }
 

@@ -109,7 +109,11 @@ extern "C" int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, 
     if (!lse || !dqkv || !workspace_dev) return set_error(GPT2_ERR_INVALID_ARG, "NULL operand");
     long long launches = 0;
     Ctx c = kctx(stream, status_dev, &launches);
-    if (engine >= 1)
+    if (engine == 2) {
+        if (!launch_attention_bwd_tc(c, (const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, workspace_dev,
+                                     (bf16*)dqkv, B, T, H))
+            return set_error(GPT2_ERR_CUDA, "tensor-map encoding failed");
+    } else if (engine == 1)
         launch_attention_bwd_mma(c, (const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, workspace_dev,
                                  (bf16*)dqkv, B, T, H, hd);
     else if (dtype == GPT2K_F32)

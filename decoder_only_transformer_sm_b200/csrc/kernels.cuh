@@ -113,6 +113,12 @@ void launch_attention_bwd_mma(const Ctx& ctx, const bf16* qkv, const bf16* out, 
 // could not be encoded (nothing launched).
 bool attention_tc_supported(int hd);
 bool launch_attention_fwd_tc(const Ctx& ctx, const bf16* qkv, bf16* out, float* lse, int B, int Tn, int H);
+// tcgen05 flash attention backward (head width 64): D pre-pass, dK/dV kernel, dQ kernel.
+bool launch_attention_bwd_tc(const Ctx& ctx, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
+                             float* dpre, bf16* dqkv, int B, int Tn, int H);
+// D = rowsum(dout * out) per (b, h, t) (the backward's pre-pass).
+void launch_attention_bwd_pre(const Ctx& ctx, const bf16* out, const bf16* dout, float* dpre, int B, int Tn, int H,
+                              int hd);
 
 // ----------------------------------------------------------------------------
 // Optimiser and parameter utilities.

@@ -82,7 +82,8 @@ int gpt2k_attention_fwd(int dtype, const void* qkv, void* out, float* lse, int B
 /* Backward of gpt2k_attention_fwd: dqkv (B, T, 3C) = [dq | dk | dv] from qkv,
  * out, dout (B, T, C) and lse.
  * workspace_dev: caller-owned scratch of B*H*T floats (D = rowsum(dout * out)).
- * engine: 0 = SIMT kernel; 1 or 2 = tensor-core kernels (bf16 only). */
+ * engine: 0 = SIMT kernel; 1 = mma.sync tensor-core kernels (bf16); 2 = tcgen05
+ *         kernels (bf16, hd = 64: TMEM accumulators for dK, dV, dQ). */
 int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, const void* dout, const float* lse,
                         void* dqkv, int B, int T, int H, int hd, float* workspace_dev, int engine,
                         uint32_t* status_dev, void* stream);
