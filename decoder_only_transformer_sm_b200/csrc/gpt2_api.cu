@@ -343,6 +343,16 @@ double gemm_bytes(int M, int N, int K, size_t es, const Epilogue& ep) {
     return b;
 }
 
+// Whether gemm_raw<A> takes the tensor-core path for this shape.
+template <typename A>
+bool gemm_on_tc(gpt2_handle*, GemmLayout, int, int, int) {
+    return false;
+}
+template <>
+bool gemm_on_tc<bf16>(gpt2_handle* h, GemmLayout layout, int M, int N, int K) {
+    return h->use_tc_gemm && gemm_tc_supported(layout, M, N, K);
+}
+
 template <typename A>
 void gemm(gpt2_handle* h, const char* site, GemmLayout layout, const void* a, const void* b, int M, int N, int K,
           const Epilogue& ep) {
@@ -480,9 +490,18 @@ void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
         gemm<A>(h, "gemm wgrad mlp.c_proj", GEMM_TN, h->dres_act, h->fcg[l], C, 4 * C, BT, acc);
         Epilogue e = epi(EPI_MUL, h->du, 4 * C);   // du = (dY W) * gelu'(u), gelu'(u) stored by the forward
         e.aux = h->fch[l];
+        // on the tensor-core path the epilogue also leaves per-32-row column sums of du
+        // (the c_fc bias gradient) in red_scratch
+        const bool fused_colsum = gemm_on_tc<A>(h, GEMM_NN, BT, 4 * C, C);
+        if (fused_colsum) e.colsum_part = h->red_scratch;
         gemm<A>(h, "gemm dgrad mlp.c_proj*gelu'", GEMM_NN, h->dres_act, wop<A>(h, o.wfcp), BT, 4 * C, C, e);
-        PROF("bias colsum", 0, 0, 0, 0.0, (double)BT * 4 * C * es,
-             launch_colsum<A>(c, (const A*)h->du, BT, 4 * C, G + o.bfc, h->red_scratch));
+        if (fused_colsum) {
+            PROF("bias colsum", 0, 0, 0, 0.0, (double)ceil_div(BT, 32) * 4 * C * 4,
+                 launch_colred_finalize(c, h->red_scratch, ceil_div(BT, 32), 4 * C, G + o.bfc));
+        } else {
+            PROF("bias colsum", 0, 0, 0, 0.0, (double)BT * 4 * C * es,
+                 launch_colsum<A>(c, (const A*)h->du, BT, 4 * C, G + o.bfc, h->red_scratch));
+        }
         // mlp.c_fc: dW += du^T ln2 ; dln2 = du W
         acc = epi(EPI_ACCUM_F32, G + o.wfc, C);
         acc.beta = 1.f;
@@ -685,7 +704,8 @@ int gpt2_create(const gpt2_config* cfg, void* stream, gpt2_handle** out) {
     {
         const size_t ln_part = (size_t)ln_bwd_col_blocks((int)BT) * 3 * C;
         const size_t cs_part = (size_t)colsum_row_blocks((int)BT) * 4 * C;
-        plan.push_back({(void**)&h->red_scratch, std::max(ln_part, cs_part) * 4});
+        const size_t mul_part = (size_t)ceil_div((int)BT, 32) * 4 * C;   // fused colsum of the GELU backward
+        plan.push_back({(void**)&h->red_scratch, std::max(std::max(ln_part, cs_part), mul_part) * 4});
     }
     plan.push_back({(void**)&h->d_tokens, 2 * BT * 4});
     size_t total = 0;

@@ -197,6 +197,22 @@ __device__ __forceinline__ void epilogue_chunk(const Epilogue& ep, float* acc, i
                 }
             }
         }
+        if (kind == EPI_MUL && ep.colsum_part) {
+            // column sums of the warp's 32 rows: lane = columns 2 lane, 2 lane + 1 of the chunk
+            float s0 = 0.f, s1 = 0.f;
+            const int rmax = M - row0;
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                if (r < rmax) {
+                    const uint32_t w2 = *reinterpret_cast<const uint32_t*>(buf + swz(r, lane >> 2) + (lane & 3) * 4);
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w2));
+                    s0 += f.x;
+                    s1 += f.y;
+                }
+            }
+            const int c = col0 + 2 * lane;
+            if (c < N) *reinterpret_cast<float2*>(ep.colsum_part + (long long)(row0 >> 5) * N + c) = make_float2(s0, s1);
+        }
         __syncwarp();
     }
 }

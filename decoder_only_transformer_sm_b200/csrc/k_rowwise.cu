@@ -95,106 +95,88 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const int* __restrict__ idx
     if (lane == 0) { mean[row] = mu; rstd[row] = rs; }
 }
 
-// LayerNorm backward, row part: one warp per row computes
+// LayerNorm backward, one pass over the rows. A warp per row computes
 // dx = rstd (dxhat - mean(dxhat) - xhat mean(dxhat xhat)) + dres_in, dxhat = dy * w,
-// and writes it as fp32 (residual gradient) and in the GEMM operand type.
+// and writes it as fp32 (residual gradient) and in the GEMM operand type. The
+// same pass adds, per column, dy * xhat (weight gradient), dy (bias gradient)
+// and dx (bias gradient of the GEMM that produced this LayerNorm's input) into
+// the warp's own shared-memory row of partial sums (lane-owned columns, no
+// atomics). At the end the block adds its 8 warp rows in a fixed order and
+// writes one partial row per block; colred_finalize_kernel adds those
+// (deterministic). Block b owns rows [b rows_per_block, (b + 1) rows_per_block).
+constexpr int LNB_WARPS = 8;
 template <typename T, int NV>
-__global__ void __launch_bounds__(256) ln_bwd_rows_kernel(const T* __restrict__ dy, const float* __restrict__ x,
-                                                           const float* __restrict__ mean,
-                                                           const float* __restrict__ rstd,
-                                                           const float* __restrict__ w, const float* dres_in,
-                                                           float* dres_out, T* __restrict__ dres_act, int rows,
-                                                           int C) {
-    const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
-    const float mu = mean[row], rs = rstd[row];
-    float dxh[NV][4], xh[NV][4];
-    float s1 = 0.f, s2 = 0.f;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        const int c = (lane + 32 * i) * 4;
-        if (c < C) {
-            float g[4], xx[4], ww[4];
-            load4(dy + (long long)row * C + c, g);
-            load4(x + (long long)row * C + c, xx);
-            load4(w + c, ww);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                xh[i][j] = (xx[j] - mu) * rs;
-                dxh[i][j] = g[j] * ww[j];
-                s1 += dxh[i][j];
-                s2 += dxh[i][j] * xh[i][j];
-            }
-        }
-    }
-    s1 = warp_sum(s1) / C;
-    s2 = warp_sum(s2) / C;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        const int c = (lane + 32 * i) * 4;
-        if (c < C) {
-            float o[4], r[4] = {0.f, 0.f, 0.f, 0.f};
-            if (dres_in) load4(dres_in + (long long)row * C + c, r);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) o[j] = rs * (dxh[i][j] - s1 - xh[i][j] * s2) + r[j];
-            store4(dres_out + (long long)row * C + c, o);
-            if (dres_act) store4(dres_act + (long long)row * C + c, o);
-        }
-    }
-}
-
-// LayerNorm backward, column part: per block of rows, the partial sums
-// sum dy * xhat (weight gradient), sum dy (bias gradient) and sum dres_out
-// (bias gradient of the GEMM that produced this LayerNorm's input) for each
-// column. Thread (tx, ty) owns columns 8 tx .. 8 tx + 7 and every blockDim.y-th
-// row; the ty partials are added in a fixed order (deterministic).
-template <typename T>
-__global__ void ln_bwd_cols_kernel(const T* __restrict__ dy, const float* __restrict__ x,
-                                   const float* __restrict__ mean, const float* __restrict__ rstd,
-                                   const float* __restrict__ dres_out, int rows, int C, int rows_per_block,
-                                   float* __restrict__ partial) {
-    extern __shared__ float red[];   // [blockDim.y][3][C]
-    const int col = threadIdx.x * 8;
+__global__ void __launch_bounds__(32 * LNB_WARPS, NV <= 8 ? 2 : 1)
+    ln_bwd_kernel(const T* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ mean,
+                  const float* __restrict__ rstd, const float* __restrict__ w, const float* dres_in, float* dres_out,
+                  T* __restrict__ dres_act, int rows, int C, int rows_per_block, int want_dx_sum,
+                  float* __restrict__ partial) {
+    extern __shared__ float4 acc4[];   // [LNB_WARPS][3][C / 4]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int C4 = C >> 2;
+    float4* mine = acc4 + warp * 3 * C4;
+    for (int i = lane; i < 3 * C4; i += 32) mine[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     const int r0 = blockIdx.x * rows_per_block;
     const int r1 = min(rows, r0 + rows_per_block);
-    float aw[8], ab[8], an[8];
+    for (int row = r0 + warp; row < r1; row += LNB_WARPS) {
+        const float mu = mean[row], rs = rstd[row];
+        float dxh[NV][4], xh[NV][4], res[NV][4];
+        float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) aw[j] = ab[j] = an[j] = 0.f;
-    for (int r = r0 + threadIdx.y; r < r1; r += blockDim.y) {
-        float g[8], xx[8], d[8];
-        load4(dy + (long long)r * C + col, g);
-        load4(dy + (long long)r * C + col + 4, g + 4);
-        load4(x + (long long)r * C + col, xx);
-        load4(x + (long long)r * C + col + 4, xx + 4);
-        load4(dres_out + (long long)r * C + col, d);
-        load4(dres_out + (long long)r * C + col + 4, d + 4);
-        const float mu = mean[r], rs = rstd[r];
+        for (int i = 0; i < NV; ++i) {
+            const int c4 = lane + 32 * i;
+            if (c4 < C4) {
+                const int c = 4 * c4;
+                float g[4], xx[4], ww[4];
+                load4(dy + (long long)row * C + c, g);
+                load4(x + (long long)row * C + c, xx);
+                load4(w + c, ww);
+                if (dres_in) load4(dres_in + (long long)row * C + c, res[i]);
+                else res[i][0] = res[i][1] = res[i][2] = res[i][3] = 0.f;
+                float4 aw = mine[c4], ab = mine[C4 + c4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            aw[j] += g[j] * ((xx[j] - mu) * rs);
-            ab[j] += g[j];
-            an[j] += d[j];
+                for (int j = 0; j < 4; ++j) {
+                    xh[i][j] = (xx[j] - mu) * rs;
+                    dxh[i][j] = g[j] * ww[j];
+                    s1 += dxh[i][j];
+                    s2 += dxh[i][j] * xh[i][j];
+                }
+                aw.x += g[0] * xh[i][0]; aw.y += g[1] * xh[i][1]; aw.z += g[2] * xh[i][2]; aw.w += g[3] * xh[i][3];
+                ab.x += g[0]; ab.y += g[1]; ab.z += g[2]; ab.w += g[3];
+                mine[c4] = aw;
+                mine[C4 + c4] = ab;
+            }
+        }
+        s1 = warp_sum(s1) / C;
+        s2 = warp_sum(s2) / C;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int c4 = lane + 32 * i;
+            if (c4 < C4) {
+                const int c = 4 * c4;
+                float o[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) o[j] = rs * (dxh[i][j] - s1 - xh[i][j] * s2) + res[i][j];
+                store4(dres_out + (long long)row * C + c, o);
+                if (dres_act) store4(dres_act + (long long)row * C + c, o);
+                if (want_dx_sum) {
+                    float4 an = mine[2 * C4 + c4];
+                    an.x += o[0]; an.y += o[1]; an.z += o[2]; an.w += o[3];
+                    mine[2 * C4 + c4] = an;
+                }
+            }
         }
     }
-    float* mine = red + threadIdx.y * 3 * C;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        mine[col + j] = aw[j];
-        mine[C + col + j] = ab[j];
-        mine[2 * C + col + j] = an[j];
-    }
     __syncthreads();
-    if (threadIdx.y == 0) {
-        float* part = partial + (long long)blockIdx.x * 3 * C;
+    float4* part = reinterpret_cast<float4*>(partial + (long long)blockIdx.x * 3 * C);
+    for (int i = threadIdx.x; i < 3 * C4; i += blockDim.x) {
+        float4 t = acc4[i];
 #pragma unroll
-        for (int k = 0; k < 3; ++k)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                float t = 0.f;
-                for (int y = 0; y < (int)blockDim.y; ++y) t += red[(y * 3 + k) * C + col + j];
-                part[k * C + col + j] = t;
-            }
+        for (int k = 1; k < LNB_WARPS; ++k) {
+            const float4 u = acc4[k * 3 * C4 + i];
+            t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
+        }
+        part[i] = t;
     }
 }
 
@@ -438,14 +420,24 @@ template <typename T>
 void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const float* mean, const float* rstd,
                           const float* w, const float* dres_in, float* dres_out, T* dres_act, float* dw,
                           float* db, float* dbias_next, int rows, int C, float* scratch) {
-    const int threads = 256;
-    const int blocks = ceil_div(rows, threads / 32);
     const int nv = ceil_div(C, 128);
-#define LNB_CASE(N)                                                                                           \
-    case N:                                                                                                   \
-        ln_bwd_rows_kernel<T, N><<<blocks, threads, 0, ctx.stream>>>(dy, x, mean, rstd, w, dres_in, dres_out, \
-                                                                     dres_act, rows, C);                      \
-        break;
+    const int nblk = ln_bwd_col_blocks(rows);
+    const int rpb = ceil_div(rows, nblk);
+    const size_t smem = (size_t)LNB_WARPS * 3 * C * sizeof(float);
+    const int want = dbias_next != nullptr;
+#define LNB_CASE(N)                                                                                         \
+    case N: {                                                                                               \
+        static bool configured = false;                                                                     \
+        if (!configured) {                                                                                  \
+            cudaFuncSetAttribute(ln_bwd_kernel<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,          \
+                                 (int)(LNB_WARPS * 3 * 128 * N * sizeof(float)));                           \
+            configured = true;                                                                              \
+        }                                                                                                   \
+        ln_bwd_kernel<T, N><<<nblk, 32 * LNB_WARPS, smem, ctx.stream>>>(dy, x, mean, rstd, w, dres_in,      \
+                                                                        dres_out, dres_act, rows, C, rpb,   \
+                                                                        want, scratch);                     \
+        break;                                                                                              \
+    }
     switch (nv) {
         LNB_CASE(1) LNB_CASE(2) LNB_CASE(3) LNB_CASE(4) LNB_CASE(5) LNB_CASE(6) LNB_CASE(7)
         LNB_CASE(8) LNB_CASE(9) LNB_CASE(10) LNB_CASE(11) LNB_CASE(12) LNB_CASE(13) LNB_CASE(14)
@@ -453,21 +445,15 @@ void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const flo
         default: break;
     }
 #undef LNB_CASE
-    const int tx = C / 8;
-    const int ty = max(1, min(8, 1024 / tx));
-    const int nblk = ln_bwd_col_blocks(rows);
-    const int rpb = ceil_div(rows, nblk);
-    const size_t smem = (size_t)ty * 3 * C * sizeof(float);
-    static bool configured = false;
-    if (!configured) {
-        cudaFuncSetAttribute(ln_bwd_cols_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-        configured = true;
-    }
-    ln_bwd_cols_kernel<T><<<nblk, dim3(tx, ty), smem, ctx.stream>>>(dy, x, mean, rstd, dres_out, rows, C, rpb,
-                                                                     scratch);
     colred_finalize_kernel<<<ceil_div(3 * C, 32), dim3(32, 32), 0, ctx.stream>>>(scratch, nblk, C, 3, dw, db,
                                                                                   dbias_next);
-    *ctx.launches += 3;
+    *ctx.launches += 2;
+}
+
+void launch_colred_finalize(const Ctx& ctx, const float* partial, int nblk, int n, float* out) {
+    colred_finalize_kernel<<<ceil_div(n, 32), dim3(32, 32), 0, ctx.stream>>>(partial, nblk, n, 1, out, nullptr,
+                                                                              nullptr);
+    ++*ctx.launches;
 }
 
 void launch_count_targets(const Ctx& ctx, const int* targets, int n, int V, int* n_valid) {

@@ -13,7 +13,8 @@ int set_error(int code, const char* msg);   // defined in gpt2_api.cu
 
 extern "C" int gpt2k_matmul_bf16(int layout, const void* A, const void* B, int M, int N, int K, int epilogue,
                                  void* out, int64_t ldo, void* out2, const float* bias, const float* resid,
-                                 const void* aux, float beta, int engine, uint32_t* status_dev, void* stream) {
+                                 const void* aux, float* colsum_part, float beta, int engine,
+                                 uint32_t* status_dev, void* stream) {
     if (layout < GPT2K_NT || layout > GPT2K_TN) return set_error(GPT2_ERR_INVALID_ARG, "unknown layout");
     if (epilogue < GPT2K_EPI_STORE || epilogue > GPT2K_EPI_ACCUM_F32)
         return set_error(GPT2_ERR_INVALID_ARG, "unknown epilogue");
@@ -24,6 +25,8 @@ extern "C" int gpt2k_matmul_bf16(int layout, const void* A, const void* B, int M
     if ((needs_bias && !bias) || (epilogue == GPT2K_EPI_BIAS_GELU && !out2) ||
         (epilogue == GPT2K_EPI_BIAS_RESID && !resid) || (epilogue == GPT2K_EPI_MUL && !aux))
         return set_error(GPT2_ERR_INVALID_ARG, "epilogue operand missing");
+    if (colsum_part && (epilogue != GPT2K_EPI_MUL || engine != 1))
+        return set_error(GPT2_ERR_INVALID_ARG, "column sums come only with the tensor-core GPT2K_EPI_MUL epilogue");
     long long launches = 0;
     Ctx c;
     c.stream = (cudaStream_t)stream;
@@ -38,6 +41,7 @@ extern "C" int gpt2k_matmul_bf16(int layout, const void* A, const void* B, int M
     e.bias = bias;
     e.resid = resid;
     e.aux = aux;
+    e.colsum_part = colsum_part;
     e.beta = beta;
     const GemmLayout L = (GemmLayout)layout;
     if (engine == 1) {

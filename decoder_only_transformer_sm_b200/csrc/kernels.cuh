@@ -36,6 +36,10 @@ struct Epilogue {
     const void* aux = nullptr;     // EPI_MUL factor (ld = ldo)
     float beta = 0.f;
     int split_atomic = 0;          // EPI_ACCUM_F32 partial sums of a K split: atomicAdd into out
+    // EPI_MUL on the tensor-core path only: if set, per 32-row group g the
+    // column sums of the bf16 results go to colsum_part[g * N + col]
+    // (ceil(M / 32) x N floats); launch_colred_finalize adds them up.
+    float* colsum_part = nullptr;
 };
 
 // Operand layouts of C[M,N] = sum_k A(m,k) B(n,k):
@@ -69,10 +73,12 @@ void launch_layernorm_fwd(const Ctx& ctx, const float* x, const float* w, const 
                           float* rstd, int rows, int C);
 // dx = LN'(x)^T dy (+ dres_in); writes dres_out (fp32) and dres_act (operand copy);
 // accumulates dw += sum dy*xhat, db += sum dy and, if dbias_next != null,
-// dbias_next += sum_rows dres_out. A row kernel writes dres; a column kernel
-// writes per-block partial sums to scratch (ln_bwd_col_blocks(rows) x 3C floats)
-// that a fixed-order finalize adds to dw, db, dbias_next. C % 8 == 0.
-inline int ln_bwd_col_blocks(int rows) { return (rows + 63) / 64; }
+// dbias_next += sum_rows dres_out. One pass over the rows writes dres and
+// per-block partial column sums to scratch (ln_bwd_col_blocks(rows) x 3C
+// floats) that a fixed-order finalize adds to dw, db, dbias_next. C % 4 == 0,
+// C <= 2048. The block count is fixed (2 blocks on each of 148 SMs at most),
+// so the summation order does not depend on the device.
+inline int ln_bwd_col_blocks(int rows) { return rows < 8 * 296 ? (rows + 7) / 8 : 296; }
 template <typename T>
 void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const float* mean, const float* rstd,
                           const float* w, const float* dres_in, float* dres_out, T* dres_act, float* dw,
@@ -90,6 +96,8 @@ void launch_classifier(const Ctx& ctx, T* logits, const int* targets, int rows, 
 inline int colsum_row_blocks(int rows) { return (rows + 63) / 64; }
 template <typename T>
 void launch_colsum(const Ctx& ctx, const T* in, int rows, int cols, float* out, float* scratch);
+// out[j] += sum_b partial[b * n + j], b < nblk, in a fixed order.
+void launch_colred_finalize(const Ctx& ctx, const float* partial, int nblk, int n, float* out);
 // dwte[idx[r]] += dx[r]; dwpe[t] += sum_b dx[b, t].
 void launch_embed_bwd(const Ctx& ctx, const int* idx, const float* dx, int B, int Tn, int C, int V, float* dwte,
                       float* dwpe);

@@ -84,7 +84,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gpt2_last_launch_count": (I, [P, ctypes.POINTER(ctypes.c_int64)]),
         "gpt2_profile": (I, [P, I]),
         "gpt2_profile_read": (I, [P, P, I, ctypes.POINTER(I)]),
-        "gpt2k_matmul_bf16": (I, [I, P, P, I, I, I, I, P, ctypes.c_int64, P, P, P, P, F, I, P, P]),
+        "gpt2k_matmul_bf16": (I, [I, P, P, I, I, I, I, P, ctypes.c_int64, P, P, P, P, P, F, I, P, P]),
         "gpt2k_attention_fwd": (I, [I, P, P, P, I, I, I, I, I, P, P]),
         "gpt2k_attention_bwd": (I, [I, P, P, P, P, P, I, I, I, I, P, I, P, P]),
     }
@@ -248,7 +248,7 @@ EPILOGUE = {"store": 0, "bias": 1, "bias_gelu": 2, "bias_resid": 3, "mul": 4, "a
 
 def matmul_bf16(layout: str, A, B, M: int, N: int, K: int, epilogue: str, out, ldo: int | None = None,
                 out2=None, bias=None, resid=None, aux=None, beta: float = 0.0, engine: str = "tc",
-                status=None, stream=None):
+                status=None, stream=None, colsum_part=None):
     """gpt2k_matmul_bf16 on torch device tensors; returns the device status tensor."""
     import torch
     lib = load_library()
@@ -258,7 +258,7 @@ def matmul_bf16(layout: str, A, B, M: int, N: int, K: int, epilogue: str, out, l
         stream = torch.cuda.current_stream().cuda_stream
     rc = lib.gpt2k_matmul_bf16(LAYOUT[layout], _ptr(A), _ptr(B), M, N, K, EPILOGUE[epilogue], _ptr(out),
                                ldo if ldo is not None else N, _ptr(out2), _ptr(bias), _ptr(resid), _ptr(aux),
-                               beta, 1 if engine == "tc" else 0, _ptr(status), stream)
+                               _ptr(colsum_part), beta, 1 if engine == "tc" else 0, _ptr(status), stream)
     _check(rc)
     return status
 

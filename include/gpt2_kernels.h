@@ -51,13 +51,19 @@ extern "C" {
  * bias        : fp32 [N] for the BIAS* epilogues, else NULL.
  * resid       : fp32 [M, N] (stride ldo) for GPT2K_EPI_BIAS_RESID, else NULL.
  * aux         : bf16 [M, N] (stride ldo) factor for GPT2K_EPI_MUL, else NULL.
+ * colsum_part : GPT2K_EPI_MUL with engine 1 only, else NULL: fp32
+ *               [ceil(M / 32), N] (stride N), written with the column sums of
+ *               the bf16 results over each group of 32 rows (rows g*32 ..
+ *               g*32+31 below M); adding its rows gives the bias gradient of
+ *               the layer whose input gradient the GEMM produces.
  * engine      : 1 = tcgen05 tensor cores (TMA + TMEM), 0 = SIMT fp32-FMA kernel.
  * Errors: INVALID_ARG (sizes < 1, unknown layout/epilogue, a required pointer
  * NULL, or engine 1 with K, N, ldo (or M for TN) not a multiple of 8, or
- * GPT2K_EPI_ACCUM_F32 with beta other than 0 or 1). */
+ * GPT2K_EPI_ACCUM_F32 with beta other than 0 or 1, or colsum_part given with
+ * another epilogue or engine 0). */
 int gpt2k_matmul_bf16(int layout, const void* A, const void* B, int M, int N, int K, int epilogue, void* out,
-                      int64_t ldo, void* out2, const float* bias, const float* resid, const void* aux, float beta,
-                      int engine, uint32_t* status_dev, void* stream);
+                      int64_t ldo, void* out2, const float* bias, const float* resid, const void* aux,
+                      float* colsum_part, float beta, int engine, uint32_t* status_dev, void* stream);
 
 /* Element types of activation operands. */
 #define GPT2K_F32 0

@@ -96,6 +96,44 @@ def test_gemm_fused_epilogues(shape):
     assert _relerr(_np(m_out), _ref("NT", A, B) * _np(aux)) < 8e-3
 
 
+@pytest.mark.parametrize("shape", [(296, 200, 72), (1000, 3072, 768), (16384, 3072, 768)])
+def test_gemm_mul_column_sums(shape):
+    """GPT2K_EPI_MUL with colsum_part: per 32-row group, the column sums of the
+    stored bf16 results (checked against sums of the stored output itself, so
+    only summation order separates the two: 1e-5 of the group's absolute sum)."""
+    from decoder_only_transformer_sm_b200 import native
+    M, N, K = shape
+    g = torch.Generator().manual_seed(5)
+    A, B = _operands("NN", M, N, K, g)
+    aux = torch.randn((M, N), generator=g).to(torch.bfloat16).cuda()
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ng = (M + 31) // 32
+    part = torch.full((ng, N), float("nan"), device="cuda")
+    st = native.matmul_bf16("NN", A, B, M, N, K, "mul", out, aux=aux, colsum_part=part)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    o = _np(out)
+    pad = np.zeros((ng * 32, N))
+    pad[:M] = o
+    ref = pad.reshape(ng, 32, N).sum(axis=1)
+    scale = np.abs(pad).reshape(ng, 32, N).sum(axis=1) + 1e-30
+    got = part.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(got))
+    assert np.max(np.abs(got - ref) / scale) < 1e-5
+    assert _relerr(o, _ref("NN", A, B) * _np(aux)) < 8e-3
+
+
+def test_colsum_needs_tc_mul():
+    from decoder_only_transformer_sm_b200 import native
+    A = torch.zeros((64, 64), dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros((64, 64), dtype=torch.bfloat16, device="cuda")
+    part = torch.zeros((2, 64), device="cuda")
+    with pytest.raises(native.Gpt2Error):
+        native.matmul_bf16("NT", A, A, 64, 64, 64, "store", out, colsum_part=part)
+    with pytest.raises(native.Gpt2Error):
+        native.matmul_bf16("NT", A, A, 64, 64, 64, "mul", out, aux=A, colsum_part=part, engine="simt")
+
+
 def test_tc_rejects_unaligned_shapes():
     from decoder_only_transformer_sm_b200 import native
     A = torch.zeros((16, 12), dtype=torch.bfloat16, device="cuda")

@@ -103,6 +103,36 @@ def test_tiny_fp32_step_matches_oracle(kind):
     m.close()
 
 
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_gpt2_width_one_layer_grads(precision):
+    """GPT-2 small's width (C = 768, 12 heads, the 124M row layout of every
+    row-wise kernel) in one layer with a small vocabulary, ragged T."""
+    s = S.ModelShape(n_layer=1, n_head=12, n_embd=768, vocab_size=512, block_size=64)
+    B, T = 3, 37
+    idx, tgt = S.uniform_tokens(B, T, s.vocab_size, seed=77)
+    tgt[1, :5] = -1
+    flat = S.random_params(s, seed=78)
+    P = O.unflatten(_oshape(s), flat.astype(np.float64))
+    Mo, Vo = O.zeros_like(_oshape(s)), O.zeros_like(_oshape(s))
+    ref_loss, ref_norm, G = O.train_step(_oshape(s), P, Mo, Vo, 1, idx, tgt, lr=1e-4)
+    m = _model(s, precision, B, T)
+    m.set_params(flat)
+    loss, norm = m.step(_dev(idx), _dev(tgt), 1e-4)
+    Gg = _split(s, m.get_grads())
+    if precision == "fp32":
+        assert abs(loss - ref_loss) / ref_loss < 1e-5
+        assert abs(norm - ref_norm) / ref_norm < 1e-4
+        for name in G:
+            assert _rel(Gg[name], G[name]) < 1e-4, (name, _rel(Gg[name], G[name]))
+    else:
+        assert abs(loss - ref_loss) < 2e-2
+        for name in G:
+            assert _cos(Gg[name], G[name]) >= 0.999, name
+            nr, ng = np.linalg.norm(G[name]), np.linalg.norm(Gg[name].astype(np.float64))
+            assert nr == 0 or abs(ng / nr - 1.0) < 1e-2, (name, ng, nr)
+    m.close()
+
+
 def test_tiny_fp32_three_steps_and_ragged_shape():
     """B=3, T=37: partial attention tiles and GEMM edges; AdamW steps 1..3.
 
@@ -238,6 +268,12 @@ def _bf16_check(s, flat, idx, tgt, lr=6e-4):
     Gg = _split(s, g)
     worst = min((_cos(Gg[n], G[n]), n) for n in G)
     assert worst[0] >= 0.999, worst
+    # cosine ignores scale: the norms must agree too (bf16 roundings are about
+    # 2^-8 relative and largely cancel in a norm; 1e-2 leaves a wide margin)
+    for n in G:
+        nr, ng = np.linalg.norm(G[n]), np.linalg.norm(Gg[n].astype(np.float64))
+        if nr > 0:
+            assert abs(ng / nr - 1.0) < 1e-2, (n, ng, nr)
     m.close()
     return loss, ref_loss, worst
 
