@@ -106,6 +106,66 @@ __device__ __forceinline__ void gelu_fast_both(float u, float& g, float& dg) {
     g = u * s;
     dg = fmaf(2.0f * u * s * (1.0f - s) * c, fmaf(3.0f * 0.044715f * u, u, 1.0f), s);
 }
+// Pairs of fp32 values in one 64-bit register, for the sm_100 packed fp32
+// instructions (fma/mul/add .f32x2: one instruction per pair, IEEE
+// round-to-nearest per lane like the scalar forms).
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 pk2(float a, float b) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void upk2(f32x2 v, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ float ex2_approx(float x) {   // hardware 2^x (ex2.approx), 2^-inf = 0
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// GELU (tanh form) and its derivative for two pre-activations, in the logistic
+// form used by gelu_fast_both: s = 1 / (1 + 2^(u (K1 + K2 u^2))) with
+// K1 = -2 c log2(e), K2 = 0.044715 K1 (so s = sigmoid(2 z), z = c (u + 0.044715 u^3));
+// gelu = u s; gelu' = s + u s (1 - s) (2c + 6c 0.044715 u^2).
+__device__ __forceinline__ void gelu_both_x2(float u0, float u1, float& g0, float& g1, float& d0, float& d1) {
+    constexpr float c = 0.7978845608028654f;
+    constexpr float K1 = -2.0f * c * 1.4426950408889634f;
+    constexpr float K2 = K1 * 0.044715f;
+    constexpr float K3 = 2.0f * c;
+    constexpr float K4 = 6.0f * c * 0.044715f;
+    const f32x2 U = pk2(u0, u1);
+    const f32x2 U2 = mul2(U, U);
+    const f32x2 Z = mul2(U, fma2(U2, pk2(K2, K2), pk2(K1, K1)));
+    float z0, z1;
+    upk2(Z, z0, z1);
+    const f32x2 D = add2(pk2(ex2_approx(z0), ex2_approx(z1)), pk2(1.0f, 1.0f));
+    float e0, e1;
+    upk2(D, e0, e1);
+    const f32x2 S = pk2(rcp_approx(e0), rcp_approx(e1));
+    const f32x2 G = mul2(U, S);
+    const f32x2 OMS = fma2(S, pk2(-1.0f, -1.0f), pk2(1.0f, 1.0f));
+    const f32x2 Q = fma2(U2, pk2(K4, K4), pk2(K3, K3));
+    const f32x2 DG = fma2(mul2(G, OMS), Q, S);
+    upk2(G, g0, g1);
+    upk2(DG, d0, d1);
+}
+
 // GELU and its derivative for an output element type: exact tanh form for fp32
 // results, the logistic form for bf16 results.
 template <typename T> __device__ __forceinline__ float gelu_for(float u);

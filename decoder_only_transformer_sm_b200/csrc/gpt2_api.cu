@@ -118,7 +118,7 @@ struct gpt2_handle {
     long long launches = 0;
     bool use_tc_gemm = true;
     bool use_tc_attention = true;
-    bool use_tcgen05_attention = false;       // tcgen05 forward (slower than the mma.sync kernel so far)
+    bool use_tcgen05_attention = true;        // tcgen05 forward for head width 64 (else the mma.sync kernel)
     bool use_tcgen05_attention_bwd = true;    // tcgen05 backward (faster than the mma.sync kernels)
     std::string host_error;   // set by enqueue helpers that cannot report a status
 

@@ -10,7 +10,7 @@
 //
 // One CTA = one (b, h) and 128 queries (one query per softmax thread and TMEM
 // lane). Warp 0 loads Q once and the K/V tiles of the causal prefix through a
-// 2-stage TMA ring; warp 1 issues, from one thread, S_j = Q K_j^T (M=128,
+// 3-stage TMA ring; warp 1 issues, from one thread, S_j = Q K_j^T (M=128,
 // N=128, K=64) into one of two TMEM S buffers and PV_j = P_j V_j (M=128, N=64,
 // K=128; V described as an N-major operand) into one of two TMEM PV buffers;
 // warps 2..9 are the softmax warps, two per TMEM lane quarter: each owns 64 of
@@ -32,7 +32,7 @@ namespace {
 
 constexpr int HD = 64;
 constexpr int BQ = 128, BKV = 128;
-constexpr int KV_STAGES = 2;
+constexpr int KV_STAGES = 3;
 constexpr int SM_WARPS = 8;                       // softmax warps: 2 per TMEM lane quarter
 constexpr int THREADS = 64 + 32 * SM_WARPS;
 constexpr int TILE_BYTES = 128 * HD * 2;          // 16 KB: 128 rows x 128 bytes
@@ -94,9 +94,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     Ctl* ctl = reinterpret_cast<Ctl*>(smem + OFF_CTL);
     volatile uint32_t* abort = &ctl->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_qt = gridDim.x;
-    const int qt = n_qt - 1 - blockIdx.x;            // longest causal prefixes first
-    const int bh = blockIdx.y, b = bh / H, h = bh % H;
+    // grid (B H, query tiles): blocks are dispatched in linear order, so every
+    // head's longest causal prefix comes first (longest-first over the grid)
+    const int n_qt = gridDim.y;
+    const int qt = n_qt - 1 - blockIdx.y;
+    const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const int C = H * HD;
     const int q0 = qt * BQ;
     const int n_kv = (min(Tn, q0 + BQ) + BKV - 1) / BKV;   // key tiles 0 .. n_kv-1
@@ -392,9 +394,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     CtlDkv* ctl = reinterpret_cast<CtlDkv*>(smem + DKV_OFF_CTL);
     volatile uint32_t* abort = &ctl->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_kt = gridDim.x;
-    const int kt = n_kt - 1 - blockIdx.x;               // longest query ranges first
-    const int bh = blockIdx.y, b = bh / H, h = bh % H;
+    // grid (B H, key tiles): key tile 0 sees the most queries and is dispatched first
+    const int kt = blockIdx.y;
+    const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const int C = H * HD;
     const int k0 = kt * 128;
     const int n_q64 = (Tn + 63) / 64;
@@ -612,9 +614,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     CtlDq* ctl = reinterpret_cast<CtlDq*>(smem + DQ_OFF_CTL);
     volatile uint32_t* abort = &ctl->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_qt = gridDim.x;
-    const int qt = n_qt - 1 - blockIdx.x;
-    const int bh = blockIdx.y, b = bh / H, h = bh % H;
+    // grid (B H, query tiles): the last query tile sees the most keys and is dispatched first
+    const int n_qt = gridDim.y;
+    const int qt = n_qt - 1 - blockIdx.y;
+    const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const int C = H * HD;
     const int q0 = qt * 128;
     const int n_k64 = (min(Tn, q0 + 128) + 63) / 64;    // key tiles that some query of the tile sees
@@ -803,7 +806,7 @@ bool launch_attention_fwd_tc(const Ctx& ctx, const bf16* qkv, bf16* out, float* 
         cudaFuncSetAttribute(flash_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
         configured = true;
     }
-    dim3 grid(ceil_div(Tn, BQ), B * H);
+    dim3 grid(B * H, ceil_div(Tn, BQ));
     flash_fwd_tc_kernel<<<grid, THREADS, SMEM_BYTES, ctx.stream>>>(m, out, lse, Tn, H, ctx.status);
     ++*ctx.launches;
     return true;
@@ -834,7 +837,7 @@ bool launch_attention_bwd_tc(const Ctx& ctx, const bf16* qkv, const bf16* out, c
         configured = true;
     }
     launch_attention_bwd_pre(ctx, out, dout, dpre, B, Tn, H, HD);
-    const dim3 grid(ceil_div(Tn, 128), B * H);
+    const dim3 grid(B * H, ceil_div(Tn, 128));
     flash_bwd_dkv_tc_kernel<<<grid, BW_THREADS, DKV_SMEM, ctx.stream>>>(qkv128, qkv64, do64, lse, dpre, dqkv, Tn, H,
                                                                          ctx.status);
     flash_bwd_dq_tc_kernel<<<grid, BW_THREADS, DQ_SMEM, ctx.stream>>>(qkv128, qkv64, do128, lse, dpre, dqkv, Tn, H,

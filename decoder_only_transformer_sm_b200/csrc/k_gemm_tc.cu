@@ -147,6 +147,14 @@ __device__ __forceinline__ void epilogue_chunk(const Epilogue& ep, float* acc, i
                 }
             }
             float v[EPS];
+            if (kind == EPI_BIAS_GELU && pass == 0) {
+                // u = acc + bias rounded to bf16; gelu(u) kept in x for pass 1, gelu'(u) out now
+#pragma unroll
+                for (int j = 0; j < EPS; j += 2) {
+                    const float2 u = __bfloat1622float2(__floats2bfloat162_rn(x[j] + b[j], x[j + 1] + b[j + 1]));
+                    gelu_both_x2(u.x, u.y, x[j], x[j + 1], v[j], v[j + 1]);
+                }
+            } else {
 #pragma unroll
             for (int j = 0; j < EPS; ++j) {
                 switch (kind) {
@@ -164,6 +172,7 @@ __device__ __forceinline__ void epilogue_chunk(const Epilogue& ep, float* acc, i
                 case EPI_MUL: v[j] = x[j] * in[j]; break;
                 default: v[j] = x[j]; break;
                 }
+            }
             }
             if (F32) {
                 *reinterpret_cast<float4*>(buf + swz(lane, c)) = make_float4(v[0], v[1], v[2], v[3]);
