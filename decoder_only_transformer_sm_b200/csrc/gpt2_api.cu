@@ -122,6 +122,15 @@ struct gpt2_handle {
     bool use_tcgen05_attention_bwd = true;    // tcgen05 backward (faster than the mma.sync kernels)
     std::string host_error;   // set by enqueue helpers that cannot report a status
 
+    // CUDA graph of zero_grad + forward + backward for one (B, T), captured on the
+    // second step with that shape (the first runs eagerly, so one-time setup such
+    // as kernel attributes happens outside a capture) and replayed afterwards.
+    bool use_graphs = true;
+    cudaStream_t cap_stream = nullptr;
+    cudaGraphExec_t graph_exec = nullptr;
+    int graph_B = 0, graph_T = 0;
+    long long graph_launches = 0;
+
     bool profiling = false;
     std::vector<ProfSite> psites;
     std::unordered_map<std::string, int> pidx;
@@ -579,6 +588,55 @@ int zero_grad_impl(gpt2_handle* h) {
     return GPT2_OK;
 }
 
+// zero_grad + forward + backward of one step on the tokens in the handle's own
+// buffer (idx at d_tokens, targets at d_tokens + maxBT), through the step graph
+// when graphs are on and the profiler is off.
+int grad_pass_impl(gpt2_handle* h, int B, int T) {
+    const int* idx = h->d_tokens;
+    const int* tgt = h->d_tokens + h->maxBT;
+    auto eager = [&]() {
+        int rc = zero_grad_impl(h);
+        if (!rc) rc = accumulate_impl(h, idx, tgt, B, T, 1.f);
+        return rc;
+    };
+    if (!h->use_graphs || h->profiling) return eager();
+    if (h->graph_exec && h->graph_B == B && h->graph_T == T) {
+        CK(cudaGraphLaunch(h->graph_exec, h->stream));
+        h->launches += h->graph_launches;
+        return GPT2_OK;
+    }
+    if (h->graph_B != B || h->graph_T != T) {   // first step with this shape: eager
+        if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
+        h->graph_exec = nullptr;
+        h->graph_B = B;
+        h->graph_T = T;
+        return eager();
+    }
+    // second step with this shape: capture on a private stream (the caller's may be
+    // the legacy default stream, which cannot be captured), then launch on the caller's
+    if (!h->cap_stream) CK(cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking));
+    cudaStream_t user = h->stream;
+    const long long l0 = h->launches;
+    CK(cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal));
+    h->stream = h->cap_stream;
+    int rc = eager();
+    h->stream = user;
+    cudaGraph_t g = nullptr;
+    cudaError_t e = cudaStreamEndCapture(h->cap_stream, &g);
+    if (!rc && e == cudaSuccess) e = cudaGraphInstantiate(&h->graph_exec, g, 0);
+    if (g) cudaGraphDestroy(g);
+    if (rc) return rc;
+    if (e != cudaSuccess) {
+        h->graph_exec = nullptr;
+        return fail(GPT2_ERR_CUDA, std::string("step graph capture failed: ") + cudaGetErrorString(e));
+    }
+    h->graph_launches = h->launches - l0;
+    h->launches = l0;
+    CK(cudaGraphLaunch(h->graph_exec, h->stream));
+    h->launches += h->graph_launches;
+    return GPT2_OK;
+}
+
 int update_impl(gpt2_handle* h, float lr, float* loss_host, float* norm_host) {
     Ctx c = h->ctx();
     CK(cudaMemsetAsync(&h->d_sc->sumsq, 0, sizeof(double), h->stream));
@@ -638,6 +696,7 @@ int gpt2_create(const gpt2_config* cfg, void* stream, gpt2_handle** out) {
     h->V = cfg->vocab_size;
     h->maxBT = cfg->max_B * cfg->max_T;
     if (const char* e = getenv("GPT2_B200_SIMT_GEMM")) h->use_tc_gemm = (e[0] == '0');
+    if (const char* e = getenv("GPT2_B200_NO_GRAPH")) h->use_graphs = (e[0] == '0');
     if (const char* e = getenv("GPT2_B200_SIMT_ATTENTION")) h->use_tc_attention = (e[0] == '0');
     if (const char* e = getenv("GPT2_B200_TCGEN05_ATTENTION")) h->use_tcgen05_attention = (e[0] == '1');
     if (const char* e = getenv("GPT2_B200_TCGEN05_ATTENTION_BWD")) h->use_tcgen05_attention_bwd = (e[0] == '1');
@@ -739,6 +798,8 @@ int gpt2_create(const gpt2_config* cfg, void* stream, gpt2_handle** out) {
 void gpt2_destroy(gpt2_handle* h) {
     if (!h) return;
     cudaStreamSynchronize(h->stream);
+    if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
+    if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
     cudaFree(h->params);
     cudaFree(h->grads);
     cudaFree(h->mom1);
@@ -876,9 +937,11 @@ int gpt2_step(gpt2_handle* h, const int32_t* idx, const int32_t* targets, int B,
     if (!h || !idx || !targets) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
     int rc = check_bt(h, B, T);
     if (rc) return rc;
+    const size_t n = (size_t)B * T;
+    CK(cudaMemcpyAsync(h->d_tokens, idx, n * 4, cudaMemcpyDeviceToDevice, h->stream));
+    CK(cudaMemcpyAsync(h->d_tokens + h->maxBT, targets, n * 4, cudaMemcpyDeviceToDevice, h->stream));
     h->launches = 0;
-    rc = zero_grad_impl(h);
-    if (!rc) rc = accumulate_impl(h, idx, targets, B, T, 1.f);
+    rc = grad_pass_impl(h, B, T);
     if (!rc) rc = update_impl(h, lr, loss_host, grad_norm_host);
     return rc;
 }
@@ -890,10 +953,9 @@ int gpt2_step_host(gpt2_handle* h, const int32_t* idx_host, const int32_t* targe
     if (rc) return rc;
     const size_t n = (size_t)B * T;
     CK(cudaMemcpyAsync(h->d_tokens, idx_host, n * 4, cudaMemcpyHostToDevice, h->stream));
-    CK(cudaMemcpyAsync(h->d_tokens + n, targets_host, n * 4, cudaMemcpyHostToDevice, h->stream));
+    CK(cudaMemcpyAsync(h->d_tokens + h->maxBT, targets_host, n * 4, cudaMemcpyHostToDevice, h->stream));
     h->launches = 0;
-    rc = zero_grad_impl(h);
-    if (!rc) rc = accumulate_impl(h, h->d_tokens, h->d_tokens + n, B, T, 1.f);
+    rc = grad_pass_impl(h, B, T);
     if (!rc) rc = update_impl(h, lr, loss_host, grad_norm_host);
     return rc;
 }

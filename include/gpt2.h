@@ -159,13 +159,20 @@ int gpt2_accumulate(gpt2_handle* h, const int32_t* idx_dev, const int32_t* targe
 int gpt2_update(gpt2_handle* h, float lr, float* loss_host, float* grad_norm_host);
 
 /* One full training step: zero_grad, accumulate(loss_scale = 1), update.
- * Device-resident inputs. */
+ * Device-resident inputs. The ids and targets are first copied (on the
+ * handle's stream) into a buffer the handle owns. The first step with a given
+ * (B, T) runs eagerly; the second captures its zero_grad/forward/backward
+ * launches into a CUDA graph (on a private stream), and later steps with the
+ * same (B, T) replay that graph on the handle's stream; the update always runs
+ * eagerly. A step with another (B, T) drops the graph. The environment variable
+ * GPT2_B200_NO_GRAPH=1 at gpt2_create turns graphs off; so does profiling. */
 int gpt2_step(gpt2_handle* h, const int32_t* idx_dev, const int32_t* targets_dev,
               int B, int T, float lr, float* loss_host, float* grad_norm_host);
 
 /* The same step taking HOST token buffers: the ids and targets are copied to the
  * device on the handle's stream inside the call (pinned memory gives an
- * asynchronous copy), then the step runs and the two scalars are read back. */
+ * asynchronous copy), then the step runs (graph replay as for gpt2_step) and
+ * the two scalars are read back. */
 int gpt2_step_host(gpt2_handle* h, const int32_t* idx_host, const int32_t* targets_host,
                    int B, int T, float lr, float* loss_host, float* grad_norm_host);
 
