@@ -8,9 +8,11 @@
 // and row sum l, so no T x T matrix is stored; lse = m + log(l) is kept for
 // the backward.
 //
-// One CTA = one (b, h) and 128 queries (one query per softmax thread and TMEM
-// lane). Warp 0 loads Q once and the K/V tiles of the causal prefix through a
-// 3-stage TMA ring; warp 1 issues, from one thread, S_j = Q K_j^T (M=128,
+// Work item = one (b, h) and 128 queries (one query row per TMEM lane). The
+// kernel is persistent: one CTA per SM walks the items, longest causal prefix
+// first. Warp 0 loads each item's Q (double-buffered, so the next item's Q
+// arrives during the current one) and the K/V tiles of its causal prefix
+// through a 3-stage TMA ring; warp 1 issues, from one thread, S_j = Q K_j^T (M=128,
 // N=128, K=64) into one of two TMEM S buffers and PV_j = P_j V_j (M=128, N=64,
 // K=128; V described as an N-major operand) into one of two TMEM PV buffers;
 // warps 2..9 are the softmax warps, two per TMEM lane quarter: each owns 64 of
@@ -41,7 +43,7 @@ constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_PV0 = 256, TM_PV1 = 320;
 constexpr float LOG2E = 1.4426950408889634f;
 
 struct Ctl {
-    uint64_t q_full;
+    uint64_t q_full[2], q_empty[2];
     uint64_t kv_full[KV_STAGES], kv_empty[KV_STAGES];
     uint64_t s_full[2], s_empty[2];
     uint64_t p_full[2];
@@ -53,9 +55,9 @@ struct Ctl {
     float lsum[2][BQ];                            // [column half][row]: partial row sum at the end
 };
 
-// smem: Q | K[2] | V[2] | P[2] | ctl
+// smem: Q[2] | K[3] | V[3] | P[2] | ctl
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + TILE_BYTES;
+constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
 constexpr int OFF_V = OFF_K + KV_STAGES * TILE_BYTES;
 constexpr int OFF_P = OFF_V + KV_STAGES * TILE_BYTES;
 constexpr int OFF_CTL = OFF_P + 2 * P_BYTES;
@@ -86,36 +88,48 @@ __device__ __forceinline__ uint4 pack8_bf16(const float* v) {
     return q;
 }
 
+// Work item i of the forward (longest causal prefixes first over the whole
+// grid): query tile n_qt - 1 - i / BH of head-sequence i % BH.
+struct FwdItem {
+    int bh, q0, n_kv;
+};
+__device__ __forceinline__ FwdItem fwd_item(int i, int BH, int n_qt, int Tn) {
+    FwdItem it;
+    it.bh = i % BH;
+    it.q0 = (n_qt - 1 - i / BH) * BQ;
+    it.n_kv = (min(Tn, it.q0 + BQ) + BKV - 1) / BKV;   // key tiles 0 .. n_kv-1
+    return it;
+}
+
+// Persistent: gridDim.x CTAs (at most one per SM) walk the items
+// blockIdx.x, blockIdx.x + gridDim.x, ... Every ring and buffer parity runs on
+// counters over all the CTA's tiles, so the loads and S MMAs of the next item
+// overlap the softmax and output of the current one.
 __global__ void __launch_bounds__(THREADS, 1)
     flash_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse,
-                        int Tn, int H, unsigned* status) {
+                        int Tn, int H, int BH, unsigned* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Ctl* ctl = reinterpret_cast<Ctl*>(smem + OFF_CTL);
     volatile uint32_t* abort = &ctl->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // grid (B H, query tiles): blocks are dispatched in linear order, so every
-    // head's longest causal prefix comes first (longest-first over the grid)
-    const int n_qt = gridDim.y;
-    const int qt = n_qt - 1 - blockIdx.y;
-    const int bh = blockIdx.x, b = bh / H, h = bh % H;
+    const int n_qt = (Tn + BQ - 1) / BQ;
+    const int n_items = BH * n_qt;
     const int C = H * HD;
-    const int q0 = qt * BQ;
-    const int n_kv = (min(Tn, q0 + BQ) + BKV - 1) / BKV;   // key tiles 0 .. n_kv-1
-    const int row_base = b * Tn;                      // first row of this sequence in qkv
 
     if (threadIdx.x == 0) {
-        tc::mbar_init(&ctl->q_full, 1);
-        for (int s = 0; s < KV_STAGES; ++s) {
-            tc::mbar_init(&ctl->kv_full[s], 1);
-            tc::mbar_init(&ctl->kv_empty[s], 1);
-        }
         for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&ctl->q_full[i], 1);
+            tc::mbar_init(&ctl->q_empty[i], 1);
             tc::mbar_init(&ctl->s_full[i], 1);
             tc::mbar_init(&ctl->s_empty[i], SM_WARPS);
             tc::mbar_init(&ctl->p_full[i], SM_WARPS);
             tc::mbar_init(&ctl->pv_full[i], 1);
             tc::mbar_init(&ctl->pv_empty[i], SM_WARPS);
+        }
+        for (int s = 0; s < KV_STAGES; ++s) {
+            tc::mbar_init(&ctl->kv_full[s], 1);
+            tc::mbar_init(&ctl->kv_empty[s], 1);
         }
         tc::mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
@@ -134,17 +148,26 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0) {
             // --------------------------------------------------------------- TMA
             tc::tma_prefetch_desc(&tm_qkv);
-            tc::mbar_expect_tx(&ctl->q_full, TILE_BYTES);
-            tc::tma_load_2d(smem + OFF_Q, &tm_qkv, h * HD, row_base + q0, &ctl->q_full);
-            for (int j = 0; j < n_kv; ++j) {
-                const int s = j % KV_STAGES;
-                const uint32_t ph = (j / KV_STAGES) & 1;
-                if (!tc::mbar_wait(&ctl->kv_empty[s], ph ^ 1, abort, status)) break;
-                tc::mbar_expect_tx(&ctl->kv_full[s], 2 * TILE_BYTES);
-                tc::tma_load_2d(smem + OFF_K + s * TILE_BYTES, &tm_qkv, C + h * HD, row_base + j * BKV,
-                                &ctl->kv_full[s]);
-                tc::tma_load_2d(smem + OFF_V + s * TILE_BYTES, &tm_qkv, 2 * C + h * HD, row_base + j * BKV,
-                                &ctl->kv_full[s]);
+            uint32_t g = 0;                           // K/V tile counter over all items
+            uint32_t ord = 0;                         // item counter (Q buffer ring)
+            bool ok = true;
+            for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, ++ord) {
+                const FwdItem it = fwd_item(i, BH, n_qt, Tn);
+                const int row_base = (it.bh / H) * Tn, h = it.bh % H;
+                const int qb = ord & 1;
+                if (!tc::mbar_wait(&ctl->q_empty[qb], ((ord >> 1) & 1) ^ 1, abort, status)) break;
+                tc::mbar_expect_tx(&ctl->q_full[qb], TILE_BYTES);
+                tc::tma_load_2d(smem + OFF_Q + qb * TILE_BYTES, &tm_qkv, h * HD, row_base + it.q0, &ctl->q_full[qb]);
+                for (int j = 0; j < it.n_kv; ++j, ++g) {
+                    const int s = g % KV_STAGES;
+                    const uint32_t ph = (g / KV_STAGES) & 1;
+                    if (!tc::mbar_wait(&ctl->kv_empty[s], ph ^ 1, abort, status)) { ok = false; break; }
+                    tc::mbar_expect_tx(&ctl->kv_full[s], 2 * TILE_BYTES);
+                    tc::tma_load_2d(smem + OFF_K + s * TILE_BYTES, &tm_qkv, C + h * HD, row_base + j * BKV,
+                                    &ctl->kv_full[s]);
+                    tc::tma_load_2d(smem + OFF_V + s * TILE_BYTES, &tm_qkv, 2 * C + h * HD, row_base + j * BKV,
+                                    &ctl->kv_full[s]);
+                }
             }
         }
     } else if (warp == 1) {
@@ -152,27 +175,49 @@ __global__ void __launch_bounds__(THREADS, 1)
             // --------------------------------------------------------------- MMA
             constexpr uint32_t idesc_s = tc::idesc_bf16_f32(BQ, BKV, 0, 0);
             constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(BQ, HD, 0, 1);
-            const uint32_t q_addr = tc::smem_u32(smem + OFF_Q);
-            bool ok = tc::mbar_wait(&ctl->q_full, 0, abort, status);
-            auto issue_s = [&](int j) -> bool {
-                const int s = j % KV_STAGES, sb = j & 1;
-                if (!tc::mbar_wait(&ctl->kv_full[s], (j / KV_STAGES) & 1, abort, status)) return false;
-                if (!tc::mbar_wait(&ctl->s_empty[sb], ((j >> 1) & 1) ^ 1, abort, status)) return false;
+            // tile cursor over (item, key tile) in the CTA's order
+            struct Cur {
+                int i, j, n_kv;
+                uint32_t ord;
+            };
+            auto start = [&](Cur& c, int i, uint32_t ord) {
+                c.i = i;
+                c.j = 0;
+                c.ord = ord;
+                c.n_kv = i < n_items ? fwd_item(i, BH, n_qt, Tn).n_kv : 0;
+            };
+            auto advance = [&](Cur c) {
+                Cur n = c;
+                if (++n.j == n.n_kv) start(n, c.i + (int)gridDim.x, c.ord + 1);
+                return n;
+            };
+            // S_g = Q K_g^T for the tile at cursor c (global tile index g)
+            auto issue_s = [&](const Cur& c, uint32_t g) -> bool {
+                const int s = g % KV_STAGES, sb = g & 1, qb = c.ord & 1;
+                if (c.j == 0 && !tc::mbar_wait(&ctl->q_full[qb], (c.ord >> 1) & 1, abort, status)) return false;
+                if (!tc::mbar_wait(&ctl->kv_full[s], (g / KV_STAGES) & 1, abort, status)) return false;
+                if (!tc::mbar_wait(&ctl->s_empty[sb], ((g >> 1) & 1) ^ 1, abort, status)) return false;
                 tc::fence_after_sync();
+                const uint32_t q_addr = tc::smem_u32(smem + OFF_Q + qb * TILE_BYTES);
                 const uint32_t k_addr = tc::smem_u32(smem + OFF_K + s * TILE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk)
                     tc::mma_bf16(tmem + (sb ? TM_S1 : TM_S0), tc::smem_desc_sw128(q_addr + kk * 32, 16, 1024),
                                  tc::smem_desc_sw128(k_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
                 tc::mma_commit(&ctl->s_full[sb]);
+                if (c.j == c.n_kv - 1) tc::mma_commit(&ctl->q_empty[qb]);   // Q done once this S completes
                 return true;
             };
-            if (ok && n_kv > 0) ok = issue_s(0);
-            for (int j = 0; j < n_kv && ok; ++j) {
-                if (j + 1 < n_kv && !issue_s(j + 1)) break;
-                const int s = j % KV_STAGES, pb = j & 1;
-                if (!tc::mbar_wait(&ctl->p_full[pb], (j >> 1) & 1, abort, status)) break;
-                if (!tc::mbar_wait(&ctl->pv_empty[pb], ((j >> 1) & 1) ^ 1, abort, status)) break;
+            Cur cur;
+            start(cur, blockIdx.x, 0);
+            uint32_t g = 0;
+            bool ok = cur.i < n_items ? issue_s(cur, 0) : false;
+            while (ok && cur.i < n_items) {
+                const Cur nxt = advance(cur);
+                if (nxt.i < n_items && !issue_s(nxt, g + 1)) break;
+                const int s = g % KV_STAGES, pb = g & 1;
+                if (!tc::mbar_wait(&ctl->p_full[pb], (g >> 1) & 1, abort, status)) break;
+                if (!tc::mbar_wait(&ctl->pv_empty[pb], ((g >> 1) & 1) ^ 1, abort, status)) break;
                 tc::fence_after_sync();
                 const uint32_t p_addr = tc::smem_u32(smem + OFF_P + pb * P_BYTES);
                 const uint32_t v_addr = tc::smem_u32(smem + OFF_V + s * TILE_BYTES);
@@ -184,6 +229,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                                  kk > 0 ? 1u : 0u);
                 tc::mma_commit(&ctl->pv_full[pb]);
                 tc::mma_commit(&ctl->kv_empty[s]);
+                cur = nxt;
+                ++g;
             }
             volatile uint32_t no_abort = 0;
             tc::mma_commit(&ctl->drain);
@@ -197,18 +244,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int quarter = warp & 3;
         const int chalf = (warp - 2) >> 2;
         const int r = quarter * 32 + lane;            // query row within the tile = TMEM lane
-        const int q = q0 + r;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const float sl2 = LOG2E * 0.125f;             // log2(e) / sqrt(64)
-        float o[32];
-#pragma unroll
-        for (int d = 0; d < 32; ++d) o[d] = 0.f;
-        float m = -INFINITY, l = 0.f, corr_prev = 1.f;
         bool ok = true;
-        auto consume_pv = [&](int j) -> bool {
-            const int pb = j & 1;
+        uint32_t g = 0;                               // tile counter over all items
+        float o[32];
+        float corr_prev = 1.f;
+        auto consume_pv = [&](uint32_t gt) -> bool {
+            const int pb = gt & 1;
             uint32_t w = 0;
-            if (lane == 0) w = tc::mbar_wait(&ctl->pv_full[pb], (j >> 1) & 1, abort, status) ? 1u : 0u;
+            if (lane == 0) w = tc::mbar_wait(&ctl->pv_full[pb], (gt >> 1) & 1, abort, status) ? 1u : 0u;
             w = __shfl_sync(0xffffffffu, w, 0);
             if (!w) return false;
             tc::fence_after_sync();
@@ -221,93 +266,103 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (lane == 0) tc::mbar_arrive(&ctl->pv_empty[pb]);
             return true;
         };
-        // Every softmax warp passes the named barrier once per tile and twice after
-        // the loop, also after a failed wait (then without work), so that none of
-        // them is left waiting there.
-        for (int j = 0; j < n_kv; ++j) {
-            const int sb = j & 1;
-            uint32_t w = 0;
-            if (lane == 0 && ok) w = tc::mbar_wait(&ctl->s_full[sb], (j >> 1) & 1, abort, status) ? 1u : 0u;
-            w = __shfl_sync(0xffffffffu, w, 0);
-            const uint32_t s_addr = tmem + (sb ? TM_S1 : TM_S0) + chalf * 64 + lane_off;
-            const int kbase = j * BKV + chalf * 64;   // first key of this warp's columns
-            const bool diag = (j * BKV + BKV > q0);
-            // pass 1: partial row max over this warp's 64 keys, exchanged with the pair
-            float mx = -INFINITY;
-            if (w) {
-                tc::fence_after_sync();
+        // Every softmax warp passes the named barrier n_kv + 2 times per item, also
+        // after a failed wait (then without work), so none is left waiting there.
+        for (int i = blockIdx.x; i < n_items; i += gridDim.x) {
+            const FwdItem it = fwd_item(i, BH, n_qt, Tn);
+            const int q0 = it.q0, n_kv = it.n_kv;
+            const int q = q0 + r;
+#pragma unroll
+            for (int d = 0; d < 32; ++d) o[d] = 0.f;
+            float m = -INFINITY, l = 0.f;
+            corr_prev = 1.f;
+            for (int j = 0; j < n_kv; ++j, ++g) {
+                const int sb = g & 1;
+                uint32_t w = 0;
+                if (lane == 0 && ok) w = tc::mbar_wait(&ctl->s_full[sb], (g >> 1) & 1, abort, status) ? 1u : 0u;
+                w = __shfl_sync(0xffffffffu, w, 0);
+                const uint32_t s_addr = tmem + (sb ? TM_S1 : TM_S0) + chalf * 64 + lane_off;
+                const int kbase = j * BKV + chalf * 64;   // first key of this warp's columns
+                const bool diag = (j * BKV + BKV > q0);
+                // pass 1: partial row max over this warp's 64 keys, exchanged with the pair
+                float mx = -INFINITY;
+                if (w) {
+                    tc::fence_after_sync();
+#pragma unroll
+                    for (int c = 0; c < 64; c += 32) {
+                        float sv[32];
+                        tc::tmem_ld_32x32b_x32(s_addr + c, sv);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (!diag || kbase + c + e <= q) mx = fmaxf(mx, sv[e]);
+                    }
+                }
+                ctl->mx[sb][chalf][r] = mx;
+                ew_bar();
+                if (!w) { ok = false; continue; }
+                mx = fmaxf(mx, ctl->mx[sb][chalf ^ 1][r]);
+                const float m_new = fmaxf(m, mx * sl2);
+                const float corr = ex2(m - m_new);   // m = -inf at an item's start: 0
+                // pass 2: P = exp2(s * sl2 - m_new) as bf16 into this warp's 64-key atom of P
+                uint8_t* pt = smem + OFF_P + sb * P_BYTES + chalf * TILE_BYTES;
+                float rs = 0.f;
 #pragma unroll
                 for (int c = 0; c < 64; c += 32) {
                     float sv[32];
                     tc::tmem_ld_32x32b_x32(s_addr + c, sv);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (!diag || kbase + c + e <= q) mx = fmaxf(mx, sv[e]);
+                    for (int e = 0; e < 32; ++e) {
+                        const float p = (!diag || kbase + c + e <= q) ? ex2(fmaf(sv[e], sl2, -m_new)) : 0.f;
+                        sv[e] = p;
+                        rs += p;
+                    }
+#pragma unroll
+                    for (int gg = 0; gg < 4; ++gg)
+                        *reinterpret_cast<uint4*>(pt + swz128(r, (c >> 3) + gg)) = pack8_bf16(sv + 8 * gg);
                 }
+                l = l * corr + rs;
+                m = m_new;
+                tc::fence_proxy_async_smem();      // P visible to the tensor core
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) {
+                    tc::mbar_arrive(&ctl->p_full[sb]);
+                    tc::mbar_arrive(&ctl->s_empty[sb]);
+                }
+                if (j > 0 && !consume_pv(g - 1)) { ok = false; continue; }
+                corr_prev = corr;
             }
-            ctl->mx[sb][chalf][r] = mx;
+            if (ok && n_kv > 0) ok = consume_pv(g - 1);
+            // row sum of both halves
+            ctl->lsum[chalf][r] = l;
             ew_bar();
-            if (!w) { ok = false; continue; }
-            mx = fmaxf(mx, ctl->mx[sb][chalf ^ 1][r]);
-            const float m_new = fmaxf(m, mx * sl2);
-            const float corr = ex2(m - m_new);   // m = -inf at the start: 0
-            // pass 2: P = exp2(s * sl2 - m_new) as bf16 into this warp's 64-key atom of P
-            uint8_t* pt = smem + OFF_P + sb * P_BYTES + chalf * TILE_BYTES;
-            float rs = 0.f;
+            const float l_tot = l + ctl->lsum[chalf ^ 1][r];
+            // out rows: O / l, staged in the first 64-key atom of P buffer 0 (every PV MMA of
+            // this item has completed; only these warps write P, and only after this store)
+            uint8_t* stage = smem + OFF_P;
+            if (ok) {
+                const float inv = 1.f / l_tot;
 #pragma unroll
-            for (int c = 0; c < 64; c += 32) {
-                float sv[32];
-                tc::tmem_ld_32x32b_x32(s_addr + c, sv);
+                for (int gg = 0; gg < 4; ++gg) {
+                    float t[8];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float p = (!diag || kbase + c + e <= q) ? ex2(fmaf(sv[e], sl2, -m_new)) : 0.f;
-                    sv[e] = p;
-                    rs += p;
+                    for (int e = 0; e < 8; ++e) t[e] = o[8 * gg + e] * inv;
+                    *reinterpret_cast<uint4*>(stage + swz128(r, chalf * 4 + gg)) = pack8_bf16(t);
                 }
-#pragma unroll
-                for (int g = 0; g < 4; ++g)
-                    *reinterpret_cast<uint4*>(pt + swz128(r, (c >> 3) + g)) = pack8_bf16(sv + 8 * g);
+                if (chalf == 0 && q < Tn) lse[(long long)it.bh * Tn + q] = (m + log2f(l_tot)) / LOG2E;
             }
-            l = l * corr + rs;
-            m = m_new;
-            tc::fence_proxy_async_smem();      // P visible to the tensor core
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) {
-                tc::mbar_arrive(&ctl->p_full[sb]);
-                tc::mbar_arrive(&ctl->s_empty[sb]);
-            }
-            if (j > 0 && !consume_pv(j - 1)) { ok = false; continue; }
-            corr_prev = corr;
-        }
-        if (ok && n_kv > 0) ok = consume_pv(n_kv - 1);
-        // row sum of both halves (the barrier is reached by every softmax warp)
-        ctl->lsum[chalf][r] = l;
-        ew_bar();
-        const float l_tot = l + ctl->lsum[chalf ^ 1][r];
-        if (ok) {
-            // out row q: O / l, staged through the Q tile (free now) for 128-byte row stores
-            const float inv = 1.f / l_tot;
-            uint8_t* stage = smem + OFF_Q;
+            ew_bar();
+            if (ok && chalf == 0) {
+                const int b = it.bh / H, h = it.bh % H;
+                const int lrow = lane >> 3, lseg = lane & 7;
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                float t[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) t[e] = o[8 * g + e] * inv;
-                *reinterpret_cast<uint4*>(stage + swz128(r, chalf * 4 + g)) = pack8_bf16(t);
-            }
-            if (chalf == 0 && q < Tn) lse[(long long)bh * Tn + q] = (m + log2f(l_tot)) / LOG2E;
-        }
-        ew_bar();
-        if (ok && chalf == 0) {
-            uint8_t* stage = smem + OFF_Q;
-            const int lrow = lane >> 3, lseg = lane & 7;
-#pragma unroll
-            for (int st = 0; st < 8; ++st) {
-                const int rr = quarter * 32 + st * 4 + lrow;
-                if (q0 + rr < Tn)
-                    *reinterpret_cast<uint4*>(out + ((long long)b * Tn + q0 + rr) * C + h * HD + lseg * 8) =
-                        *reinterpret_cast<const uint4*>(stage + swz128(rr, lseg));
+                for (int st = 0; st < 8; ++st) {
+                    const int rr = quarter * 32 + st * 4 + lrow;
+                    if (q0 + rr < Tn)
+                        *reinterpret_cast<uint4*>(out + ((long long)b * Tn + q0 + rr) * C + h * HD + lseg * 8) =
+                            *reinterpret_cast<const uint4*>(stage + swz128(rr, lseg));
+                }
+                __syncwarp();
             }
         }
     }
@@ -513,7 +568,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             if (et < 128) return q < Tn ? dpre[(long long)bh * Tn + q] : 0.f;
             return 0.f;
         };
+        // two tiles of lookahead: a global load's latency exceeds one tile's work
         float nxt = n_it > 0 ? fetch(0) : 0.f;
+        float nxt2 = n_it > 1 ? fetch(1) : 0.f;
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             const int rb = it & 1;
@@ -521,7 +578,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             if (et < 64) ctl->lse2[rb][et] = nxt;
             else if (et < 128) ctl->dd[rb][et - 64] = nxt;
             ew_bar();
-            if (it + 1 < n_it) nxt = fetch(it + 1);
+            nxt = nxt2;
+            if (it + 2 < n_it) nxt2 = fetch(it + 2);
             uint32_t w = 0;
             if (lane == 0 && ok) {
                 w = tc::mbar_wait(&ctl->st_full[rb], (it >> 1) & 1, abort, status) ? 1u : 0u;
@@ -536,8 +594,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             uint8_t* pt = smem + DKV_OFF_PT + rb * T128_BYTES;
             uint8_t* dst = smem + DKV_OFF_DST + rb * T128_BYTES;
             float sv[32], dp[32];
-            tc::tmem_ld_32x32b_x32(tmem + DKV_ST + rb * 64 + chalf * 32 + lane_off, sv);
-            tc::tmem_ld_32x32b_x32(tmem + DKV_DPT + rb * 64 + chalf * 32 + lane_off, dp);
+            tc::tmem_ld2_32x32b_x32(tmem + DKV_ST + rb * 64 + chalf * 32 + lane_off,
+                                    tmem + DKV_DPT + rb * 64 + chalf * 32 + lane_off, sv, dp);
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
                 const int qi = chalf * 32 + e;
@@ -567,13 +625,11 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             if (w) {
                 tc::fence_after_sync();
                 float v[64];
-                tc::tmem_ld_32x32b_x32(tmem + DKV_DK + lane_off, v);
-                tc::tmem_ld_32x32b_x32(tmem + DKV_DK + 32 + lane_off, v + 32);
+                tc::tmem_ld_32x32b_x64(tmem + DKV_DK + lane_off, v);
                 bf16* kbase = dqkv + ((long long)row_base + k0) * 3 * C + C + h * HD;
                 uint8_t* stage = smem + DKV_OFF_PT;     // free: every MMA has completed
                 store_rows_64(stage, r, v, 0.125f, kbase, 3LL * C, Tn - k0);
-                tc::tmem_ld_32x32b_x32(tmem + DKV_DV + lane_off, v);
-                tc::tmem_ld_32x32b_x32(tmem + DKV_DV + 32 + lane_off, v + 32);
+                tc::tmem_ld_32x32b_x64(tmem + DKV_DV + lane_off, v);
                 store_rows_64(stage, r, v, 1.0f, kbase + C, 3LL * C, Tn - k0);
             }
         }
@@ -734,8 +790,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             const bool diag = (j * 64 + 64 > q0);
             uint8_t* ds = smem + DQ_OFF_DS + rb * T128_BYTES;
             float sv[32], dp[32];
-            tc::tmem_ld_32x32b_x32(tmem + DQ_S + rb * 64 + chalf * 32 + lane_off, sv);
-            tc::tmem_ld_32x32b_x32(tmem + DQ_DP + rb * 64 + chalf * 32 + lane_off, dp);
+            tc::tmem_ld2_32x32b_x32(tmem + DQ_S + rb * 64 + chalf * 32 + lane_off,
+                                    tmem + DQ_DP + rb * 64 + chalf * 32 + lane_off, sv, dp);
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
                 float p = ex2(fmaf(sv[e], sl2, -L2));
@@ -760,8 +816,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             if (w) {
                 tc::fence_after_sync();
                 float v[64];
-                tc::tmem_ld_32x32b_x32(tmem + DQ_DQ + lane_off, v);
-                tc::tmem_ld_32x32b_x32(tmem + DQ_DQ + 32 + lane_off, v + 32);
+                tc::tmem_ld_32x32b_x64(tmem + DQ_DQ + lane_off, v);
                 bf16* qbase = dqkv + ((long long)row_base + q0) * 3 * C + h * HD;
                 store_rows_64(smem + DQ_OFF_DS, r, v, 0.125f, qbase, 3LL * C, Tn - q0);
             }
@@ -806,8 +861,9 @@ bool launch_attention_fwd_tc(const Ctx& ctx, const bf16* qkv, bf16* out, float* 
         cudaFuncSetAttribute(flash_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
         configured = true;
     }
-    dim3 grid(B * H, ceil_div(Tn, BQ));
-    flash_fwd_tc_kernel<<<grid, THREADS, SMEM_BYTES, ctx.stream>>>(m, out, lse, Tn, H, ctx.status);
+    const int n_items = B * H * ceil_div(Tn, BQ);
+    const int grid = min(n_items, ctx.num_sms > 0 ? ctx.num_sms : 148);
+    flash_fwd_tc_kernel<<<grid, THREADS, SMEM_BYTES, ctx.stream>>>(m, out, lse, Tn, H, B * H, ctx.status);
     ++*ctx.launches;
     return true;
 }

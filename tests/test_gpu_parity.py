@@ -293,30 +293,31 @@ def test_tiny_bf16_ragged():
 
 def test_step_graph_replay_matches_eager(monkeypatch):
     """Steps 3+ with one (B, T) replay a captured CUDA graph; a shape change drops
-    it. Against a model created with graphs off: the same per-step loss and
-    gradient norm (as returned, float32) over ten steps with shape changes, the
-    same launch count, and final gradients within 1e-5 of their max. (Bitwise
-    parameter equality is not expected: the split-K weight-gradient GEMMs add
-    their K partials with fp32 atomics, so the last bits of a gradient depend
-    on arrival order.)"""
-    from decoder_only_transformer_sm_b200 import native
+    it. A graph model and an eager model (graphs off) take the same ten steps,
+    shape changes included; before each step the graph model is given the eager
+    model's parameters and optimiser state, so each step starts from one state.
+    Per step: loss 1e-6 and gradient norm 1e-5 relative, gradients 1e-5 of their
+    max (not bitwise: the split-K weight-gradient GEMMs add their K partials
+    with fp32 atomics, so a gradient's last bits depend on arrival order), and
+    the same launch count."""
     s = TINY
     flat = S.random_params(s, seed=31)
     shapes = [(4, 64), (4, 64), (4, 64), (4, 64), (3, 17), (3, 17), (3, 17), (4, 64), (4, 64), (4, 64)]
-    runs = []
-    for no_graph in ("0", "1"):
-        monkeypatch.setenv("GPT2_B200_NO_GRAPH", no_graph)
-        m = _model(s, "bf16", 4, 64)
-        m.set_params(flat)
-        out = []
-        for i, (B, T) in enumerate(shapes):
-            idx, tgt = S.uniform_tokens(B, T, s.vocab_size, seed=500 + i)
-            out.append(m.step(_dev(idx), _dev(tgt), 3e-4))
-        runs.append((out, m.get_params(), m.get_grads(), m.last_launch_count()))
-        m.close()
-    (o_g, p_g, g_g, n_g), (o_e, p_e, g_e, n_e) = runs
-    for (lg, ng), (le, ne) in zip(o_g, o_e):
-        assert abs(lg - le) <= 1e-6 * abs(le), (lg, le)
-        assert abs(ng - ne) <= 1e-5 * abs(ne), (ng, ne)
-    assert _rel(g_g, g_e) < 1e-5
-    assert n_g == n_e
+    monkeypatch.setenv("GPT2_B200_NO_GRAPH", "0")
+    mg = _model(s, "bf16", 4, 64)
+    monkeypatch.setenv("GPT2_B200_NO_GRAPH", "1")
+    me = _model(s, "bf16", 4, 64)
+    me.set_params(flat)
+    for i, (B, T) in enumerate(shapes):
+        mg.set_params(me.get_params())
+        m1, v1, t1 = me.get_opt_state()
+        mg.set_opt_state(m1, v1, t1)
+        idx, tgt = S.uniform_tokens(B, T, s.vocab_size, seed=500 + i)
+        lg, ng = mg.step(_dev(idx), _dev(tgt), 3e-4)
+        le, ne = me.step(_dev(idx), _dev(tgt), 3e-4)
+        assert abs(lg - le) <= 1e-6 * abs(le), (i, lg, le)
+        assert abs(ng - ne) <= 1e-5 * abs(ne), (i, ng, ne)
+        assert _rel(mg.get_grads(), me.get_grads()) < 1e-5, i
+        assert mg.last_launch_count() == me.last_launch_count(), i
+    mg.close()
+    me.close()
