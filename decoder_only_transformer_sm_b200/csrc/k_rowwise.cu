@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(32 * LNB_WARPS, NV <= 8 ? 2 : 1)
                 load4(dy + (long long)row * C + c, g);
                 load4(x + (long long)row * C + c, xx);
                 load4(w + c, ww);
-                if (dres_in) load4(dres_in + (long long)row * C + c, res[i]);
+                if (dres_in) load4(dres_in + (long long)row * C + c, res[i]);   // with the row's other loads
                 else res[i][0] = res[i][1] = res[i][2] = res[i][3] = 0.f;
                 float4 aw = mine[c4], ab = mine[C4 + c4];
 #pragma unroll
@@ -320,6 +320,114 @@ __global__ void __launch_bounds__(512) classifier_kernel(T* logits, const int* _
     }
 }
 
+// The classifier for bf16 logits: the same two passes with fewer instructions
+// per element, since the fp32 version is issue-bound. The maximum of each
+// 8-element chunk comes from packed bf16x2 max; exponentials are taken in
+// log2 units, 2^(v log2(e) - m log2(e)), with one packed fma.f32x2 per pair
+// and ex2.approx per element; sums and the gradient scale use packed pairs; the
+// one target column of the row is patched after the chunk that holds it.
+__device__ __forceinline__ void bf16x8_unpack(const uint4& q, f32x2 (&v)[4]) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
+        v[k] = pk2(f.x, f.y);
+    }
+}
+__global__ void __launch_bounds__(512) classifier_bf16_kernel(bf16* logits, const int* __restrict__ targets, int V,
+                                                               const int* __restrict__ n_valid, float scale,
+                                                               double* loss_accum, int write_grad) {
+    constexpr float LOG2E = 1.4426950408889634f;
+    const long long row = blockIdx.x;
+    bf16* lr = logits + row * V;
+    const int tgt = targets[row];
+    const bool valid = (tgt >= 0 && tgt < V);
+    float lt = 0.f;
+    if (threadIdx.x == 0 && valid) lt = __bfloat162float(lr[tgt]);
+    const f32x2 L2E = pk2(LOG2E, LOG2E);
+    float m = -INFINITY;
+    f32x2 S = pk2(0.f, 0.f);
+    for (int c = threadIdx.x * 8; c < V; c += blockDim.x * 8) {
+        const uint4 q = *reinterpret_cast<const uint4*>(lr + c);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+        const __nv_bfloat162 hm = __hmax2(__hmax2(h[0], h[1]), __hmax2(h[2], h[3]));
+        const float mx = fmaxf(__low2float(hm), __high2float(hm));
+        if (mx > m) {
+            const float cr = ex2_approx((m - mx) * LOG2E);   // m = -inf at the start: 0
+            S = mul2(S, pk2(cr, cr));
+            m = mx;
+        }
+        const float nm = -m * LOG2E;
+        const f32x2 NM = pk2(nm, nm);
+        f32x2 v[4];
+        bf16x8_unpack(q, v);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float t0, t1;
+            upk2(fma2(v[k], L2E, NM), t0, t1);
+            S = add2(S, pk2(ex2_approx(t0), ex2_approx(t1)));
+        }
+    }
+    float s0, s1;
+    upk2(S, s0, s1);
+    float s = s0 + s1;
+    // block reduction of (m, s)
+    __shared__ float sm[32], ssum[32];
+    __shared__ float s_lse;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+        float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+        float mm = fmaxf(m, m2);
+        s = (m == -INFINITY ? 0.f : s * expf(m - mm)) + (m2 == -INFINITY ? 0.f : s2 * expf(m2 - mm));
+        m = mm;
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    if (lane == 0) { sm[warp] = m; ssum[warp] = s; }
+    __syncthreads();
+    if (warp == 0) {
+        m = lane < nw ? sm[lane] : -INFINITY;
+        s = lane < nw ? ssum[lane] : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+            float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+            float mm = fmaxf(m, m2);
+            s = (m == -INFINITY ? 0.f : s * expf(m - mm)) + (m2 == -INFINITY ? 0.f : s2 * expf(m2 - mm));
+            m = mm;
+        }
+        if (lane == 0) s_lse = m + logf(s);
+    }
+    __syncthreads();
+    const float lse = s_lse;
+    const int nv = *n_valid;
+    if (threadIdx.x == 0 && valid && nv > 0)
+        atomicAdd(loss_accum, (double)scale * (double)(lse - lt) / (double)nv);
+    if (!write_grad) return;
+    const float gs = (valid && nv > 0) ? scale / (float)nv : 0.f;
+    const float nl = -lse * LOG2E;
+    const f32x2 NL = pk2(nl, nl), GS = pk2(gs, gs);
+    for (int c = threadIdx.x * 8; c < V; c += blockDim.x * 8) {
+        const uint4 q = *reinterpret_cast<const uint4*>(lr + c);
+        f32x2 v[4];
+        bf16x8_unpack(q, v);
+        float g[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float t0, t1;
+            upk2(fma2(v[k], L2E, NL), t0, t1);
+            upk2(mul2(pk2(ex2_approx(t0), ex2_approx(t1)), GS), g[2 * k], g[2 * k + 1]);
+        }
+        const int tj = tgt - c;
+        if ((unsigned)tj < 8u) {   // the target column: softmax - 1
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j == tj) g[j] -= gs;
+        }
+        store8v(lr + c, g);
+    }
+}
+
 // Partial column sums of in[rows][cols] over blocks of rows: each thread owns 8
 // consecutive columns and walks the block's rows with 16-byte loads.
 template <typename T>
@@ -431,6 +539,7 @@ void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const flo
         if (!configured) {                                                                                  \
             cudaFuncSetAttribute(ln_bwd_kernel<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,          \
                                  (int)(LNB_WARPS * 3 * 128 * N * sizeof(float)));                           \
+            cudaFuncSetAttribute(ln_bwd_kernel<T, N>, cudaFuncAttributePreferredSharedMemoryCarveout, 100); \
             configured = true;                                                                              \
         }                                                                                                   \
         ln_bwd_kernel<T, N><<<nblk, 32 * LNB_WARPS, smem, ctx.stream>>>(dy, x, mean, rstd, w, dres_in,      \
@@ -464,7 +573,11 @@ void launch_count_targets(const Ctx& ctx, const int* targets, int n, int V, int*
 template <typename T>
 void launch_classifier(const Ctx& ctx, T* logits, const int* targets, int rows, int V, const int* n_valid,
                        float scale, double* loss_accum, int write_grad) {
-    classifier_kernel<T><<<rows, 512, 0, ctx.stream>>>(logits, targets, V, n_valid, scale, loss_accum, write_grad);
+    if (sizeof(T) == 2)
+        classifier_bf16_kernel<<<rows, 512, 0, ctx.stream>>>(reinterpret_cast<bf16*>(logits), targets, V, n_valid,
+                                                              scale, loss_accum, write_grad);
+    else
+        classifier_kernel<T><<<rows, 512, 0, ctx.stream>>>(logits, targets, V, n_valid, scale, loss_accum, write_grad);
     ++*ctx.launches;
 }
 
@@ -472,8 +585,8 @@ template <typename T>
 void launch_colsum(const Ctx& ctx, const T* in, int rows, int cols, float* out, float* scratch) {
     const int nblk = colsum_row_blocks(rows);
     const int rpb = ceil_div(rows, nblk);
-    dim3 grid(ceil_div(cols, 8 * 128), nblk);
-    colsum_partial_kernel<T><<<grid, 128, 0, ctx.stream>>>(in, rows, cols, rpb, scratch);
+    dim3 grid(ceil_div(cols, 8 * 64), nblk);   // many small blocks: enough loads in flight on every SM
+    colsum_partial_kernel<T><<<grid, 64, 0, ctx.stream>>>(in, rows, cols, rpb, scratch);
     colred_finalize_kernel<<<ceil_div(cols, 32), dim3(32, 32), 0, ctx.stream>>>(scratch, nblk, cols, 1, out,
                                                                                 nullptr, nullptr);
     *ctx.launches += 2;

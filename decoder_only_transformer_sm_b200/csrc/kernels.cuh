@@ -93,7 +93,7 @@ void launch_classifier(const Ctx& ctx, T* logits, const int* targets, int rows, 
                        float scale, double* loss_accum, int write_grad);
 // Column sums: out[c] += sum_r in[r, c], through colsum_row_blocks(rows) x cols
 // partials in scratch and a fixed-order finalize. cols is a multiple of 8.
-inline int colsum_row_blocks(int rows) { return (rows + 63) / 64; }
+inline int colsum_row_blocks(int rows) { return (rows + 31) / 32; }
 template <typename T>
 void launch_colsum(const Ctx& ctx, const T* in, int rows, int cols, float* out, float* scratch);
 // out[j] += sum_b partial[b * n + j], b < nblk, in a fixed order.
