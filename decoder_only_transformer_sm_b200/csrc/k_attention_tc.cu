@@ -75,6 +75,26 @@ __device__ __forceinline__ float ex2(float x) {
 
 __device__ __forceinline__ void ew_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
+// max(a, b, c) in one instruction (sm_100 three-input max.f32)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Max of 32 values in four independent chains of three-input max.
+__device__ __forceinline__ float max32(const float* v, float init) {
+    float p0 = init, p1 = init, p2 = init, p3 = init;
+#pragma unroll
+    for (int e = 0; e < 32; e += 8) {
+        p0 = max3f(p0, v[e], v[e + 1]);
+        p1 = max3f(p1, v[e + 2], v[e + 3]);
+        p2 = max3f(p2, v[e + 4], v[e + 5]);
+        p3 = max3f(p3, v[e + 6], v[e + 7]);
+    }
+    return fmaxf(fmaxf(p0, p1), fmaxf(p2, p3));
+}
+
 __device__ __forceinline__ uint4 pack8_bf16(const float* v) {
     uint4 q;
     __nv_bfloat162 t0 = __floats2bfloat162_rn(v[0], v[1]);
@@ -259,8 +279,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::fence_after_sync();
             float pv[32];
             tc::tmem_ld_32x32b_x32(tmem + (pb ? TM_PV1 : TM_PV0) + chalf * 32 + lane_off, pv);
+            const f32x2 CP = pk2(corr_prev, corr_prev);
 #pragma unroll
-            for (int d = 0; d < 32; ++d) o[d] = fmaf(o[d], corr_prev, pv[d]);
+            for (int d = 0; d < 32; d += 2)
+                upk2(fma2(pk2(o[d], o[d + 1]), CP, pk2(pv[d], pv[d + 1])), o[d], o[d + 1]);
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&ctl->pv_empty[pb]);
@@ -292,9 +314,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                     for (int c = 0; c < 64; c += 32) {
                         float sv[32];
                         tc::tmem_ld_32x32b_x32(s_addr + c, sv);
+                        if (diag) {   // keys after the query do not count
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (!diag || kbase + c + e <= q) mx = fmaxf(mx, sv[e]);
+                            for (int e = 0; e < 32; ++e)
+                                if (kbase + c + e > q) sv[e] = -INFINITY;
+                        }
+                        mx = max32(sv, mx);
                     }
                 }
                 ctl->mx[sb][chalf][r] = mx;
@@ -305,21 +330,34 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const float corr = ex2(m - m_new);   // m = -inf at an item's start: 0
                 // pass 2: P = exp2(s * sl2 - m_new) as bf16 into this warp's 64-key atom of P
                 uint8_t* pt = smem + OFF_P + sb * P_BYTES + chalf * TILE_BYTES;
-                float rs = 0.f;
+                // the exponent s * sl2 - m_new and the row sum on packed pairs
+                const f32x2 SL = pk2(sl2, sl2), NM = pk2(-m_new, -m_new);
+                f32x2 RS = pk2(0.f, 0.f);
 #pragma unroll
                 for (int c = 0; c < 64; c += 32) {
                     float sv[32];
                     tc::tmem_ld_32x32b_x32(s_addr + c, sv);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float p = (!diag || kbase + c + e <= q) ? ex2(fmaf(sv[e], sl2, -m_new)) : 0.f;
-                        sv[e] = p;
-                        rs += p;
+                    for (int e = 0; e < 32; e += 2) {
+                        float t0, t1;
+                        upk2(fma2(pk2(sv[e], sv[e + 1]), SL, NM), t0, t1);
+                        sv[e] = ex2(t0);
+                        sv[e + 1] = ex2(t1);
                     }
+                    if (diag) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (kbase + c + e > q) sv[e] = 0.f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) RS = add2(RS, pk2(sv[e], sv[e + 1]));
 #pragma unroll
                     for (int gg = 0; gg < 4; ++gg)
                         *reinterpret_cast<uint4*>(pt + swz128(r, (c >> 3) + gg)) = pack8_bf16(sv + 8 * gg);
                 }
+                float rs0, rs1;
+                upk2(RS, rs0, rs1);
+                const float rs = rs0 + rs1;
                 l = l * corr + rs;
                 m = m_new;
                 tc::fence_proxy_async_smem();      // P visible to the tensor core
@@ -424,8 +462,8 @@ struct CtlDkv {
     uint64_t drain;
     uint32_t tmem_base;
     uint32_t abort;
-    float lse2[2][64];
-    float dd[2][64];
+    alignas(16) float lse2[2][64];   // negated, log2 units (read as float2 pairs)
+    alignas(16) float dd[2][64];     // negated D
 };
 // smem: K | V | (Q | dO) stages | Pt[2] | dSt[2] | ctl
 constexpr int DKV_OFF_K = 0;
@@ -562,10 +600,11 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const float sl2 = LOG2E * 0.125f;
         // per-query lse (log2 units) and D of the next tile, one value per thread
+        // stored negated, the form the packed exponent and dS arithmetic take
         auto fetch = [&](int it) -> float {
             const int q = (it0 + it) * 64 + (et & 63);
-            if (et < 64) return q < Tn ? lse[(long long)bh * Tn + q] * LOG2E : INFINITY;
-            if (et < 128) return q < Tn ? dpre[(long long)bh * Tn + q] : 0.f;
+            if (et < 64) return q < Tn ? -lse[(long long)bh * Tn + q] * LOG2E : -INFINITY;
+            if (et < 128) return q < Tn ? -dpre[(long long)bh * Tn + q] : 0.f;
             return 0.f;
         };
         // two tiles of lookahead: a global load's latency exceeds one tile's work
@@ -596,13 +635,22 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             float sv[32], dp[32];
             tc::tmem_ld2_32x32b_x32(tmem + DKV_ST + rb * 64 + chalf * 32 + lane_off,
                                     tmem + DKV_DPT + rb * 64 + chalf * 32 + lane_off, sv, dp);
+            // P^T = 2^(s sl2 - lse2), dS^T = P^T (dP^T - D) on packed pairs of queries
+            const f32x2 SL = pk2(sl2, sl2);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
+            for (int e = 0; e < 32; e += 2) {
                 const int qi = chalf * 32 + e;
-                float p = ex2(fmaf(sv[e], sl2, -ctl->lse2[rb][qi]));
-                if (diag && key > q0 + qi) p = 0.f;
-                sv[e] = p;
-                dp[e] = p * (dp[e] - ctl->dd[rb][qi]);
+                const float2 nl = *reinterpret_cast<const float2*>(&ctl->lse2[rb][qi]);
+                const float2 nd = *reinterpret_cast<const float2*>(&ctl->dd[rb][qi]);
+                float t0, t1;
+                upk2(fma2(pk2(sv[e], sv[e + 1]), SL, pk2(nl.x, nl.y)), t0, t1);
+                sv[e] = ex2(t0);
+                sv[e + 1] = ex2(t1);
+                if (diag) {   // queries before this key
+                    if (key > q0 + qi) sv[e] = 0.f;
+                    if (key > q0 + qi + 1) sv[e + 1] = 0.f;
+                }
+                upk2(mul2(pk2(sv[e], sv[e + 1]), add2(pk2(dp[e], dp[e + 1]), pk2(nd.x, nd.y))), dp[e], dp[e + 1]);
             }
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
@@ -792,11 +840,18 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             float sv[32], dp[32];
             tc::tmem_ld2_32x32b_x32(tmem + DQ_S + rb * 64 + chalf * 32 + lane_off,
                                     tmem + DQ_DP + rb * 64 + chalf * 32 + lane_off, sv, dp);
+            // dS = 2^(s sl2 - lse2) (dP - D) on packed pairs of keys
+            const f32x2 SL = pk2(sl2, sl2), NL = pk2(-L2, -L2), ND = pk2(-Dv, -Dv);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                float p = ex2(fmaf(sv[e], sl2, -L2));
-                if (diag && j * 64 + chalf * 32 + e > q) p = 0.f;
-                dp[e] = p * (dp[e] - Dv);
+            for (int e = 0; e < 32; e += 2) {
+                float t0, t1;
+                upk2(fma2(pk2(sv[e], sv[e + 1]), SL, NL), t0, t1);
+                float p0 = ex2(t0), p1 = ex2(t1);
+                if (diag) {   // keys after this query
+                    if (j * 64 + chalf * 32 + e > q) p0 = 0.f;
+                    if (j * 64 + chalf * 32 + e + 1 > q) p1 = 0.f;
+                }
+                upk2(mul2(pk2(p0, p1), add2(pk2(dp[e], dp[e + 1]), ND)), dp[e], dp[e + 1]);
             }
 #pragma unroll
             for (int g = 0; g < 4; ++g)
