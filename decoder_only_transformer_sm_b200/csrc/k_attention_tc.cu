@@ -415,11 +415,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 //   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),
 //   dK = dS^T Q / sqrt(64),  dQ = dS K / sqrt(64).
 // dK/dV kernel: one CTA per (b, h, 128-key tile); it walks the 64-query tiles
-// at or after the key tile. S^T = K Q^T and dP^T = V dO^T (M=128 keys, N=64
-// queries) go to double-buffered TMEM so the tensor core computes tile i+1
-// while 4 warps turn tile i into P^T and dS^T (bf16, K-major shared tiles);
-// dV += P^T dO and dK += dS^T Q (dO and Q as N-major operands) accumulate in
-// TMEM. dQ kernel: one CTA per (b, h, 128-query tile) over the 64-key tiles at
+// at or after the key tile. K and V are copied once into TMEM as packed bf16
+// A operands, so the N=64 MMAs read only their B operand from shared memory
+// (with both operands there they are limited by shared-memory bandwidth).
+// S^T = K Q^T and dP^T = V dO^T (M=128 keys, N=64 queries) go to
+// double-buffered TMEM so the tensor core computes tile i+1 while 8 warps turn
+// tile i into P^T and dS^T, written back as packed bf16 over the S^T / dP^T
+// columns they came from; dV += P^T dO and dK += dS^T Q (A from TMEM; dO and Q
+// as N-major shared operands) accumulate in TMEM. dQ kernel: one CTA per (b, h, 128-query tile) over the 64-key tiles at
 // or before it: S = Q K^T, dP = dO V^T, dS, then dQ += dS K in TMEM.
 // ============================================================================
 constexpr int BW_EW_WARPS = 8;                     // 2 warps per TMEM lane quarter, 32 columns each
@@ -452,12 +455,13 @@ __device__ __forceinline__ void store_rows_64(uint8_t* stage, int r, const float
     __syncwarp();
 }
 
-constexpr int DKV_STAGES = 3;
+constexpr int DKV_STAGES = 6;   // Q/dO ring deep enough to cover a ~1.3 us tile load
 struct CtlDkv {
     uint64_t kv_full;
     uint64_t q_full[DKV_STAGES], q_empty[DKV_STAGES];
     uint64_t st_full[2], st_empty[2];
-    uint64_t ew_done[2], pds_free[2];
+    uint64_t ew_done[2];
+    uint64_t kv_tmem;                            // K and V copied into TMEM (A operands)
     uint64_t acc_done;
     uint64_t drain;
     uint32_t tmem_base;
@@ -465,17 +469,20 @@ struct CtlDkv {
     alignas(16) float lse2[2][64];   // negated, log2 units (read as float2 pairs)
     alignas(16) float dd[2][64];     // negated D
 };
-// smem: K | V | (Q | dO) stages | Pt[2] | dSt[2] | ctl
+// smem: K | V | (Q | dO) stages | output staging | ctl
 constexpr int DKV_OFF_K = 0;
 constexpr int DKV_OFF_V = DKV_OFF_K + T128_BYTES;
 constexpr int DKV_OFF_Q = DKV_OFF_V + T128_BYTES;
 constexpr int DKV_STAGE_BYTES = 2 * T64_BYTES;                  // Q tile + dO tile
-constexpr int DKV_OFF_PT = DKV_OFF_Q + DKV_STAGES * DKV_STAGE_BYTES;
-constexpr int DKV_OFF_DST = DKV_OFF_PT + 2 * T128_BYTES;        // 128 keys x 64 queries bf16 = 16 KB each
-constexpr int DKV_OFF_CTL = DKV_OFF_DST + 2 * T128_BYTES;
+constexpr int DKV_OFF_STAGE = DKV_OFF_Q + DKV_STAGES * DKV_STAGE_BYTES;   // dK / dV output staging
+constexpr int DKV_OFF_CTL = DKV_OFF_STAGE + T128_BYTES;
 constexpr size_t DKV_SMEM = DKV_OFF_CTL + sizeof(CtlDkv) + 1024;
 // TMEM columns
-constexpr uint32_t DKV_ST = 0, DKV_DPT = 128, DKV_DV = 256, DKV_DK = 320;
+// TMEM columns: S^T and dP^T (fp32, double-buffered; after the element-wise step
+// the first 16 columns of each 32-column half hold that half's P^T / dS^T as
+// packed bf16, the A operand of the dV / dK MMAs), the dV and dK accumulators,
+// and K and V as packed bf16 A operands of the S^T and dP^T MMAs.
+constexpr uint32_t DKV_ST = 0, DKV_DPT = 128, DKV_DV = 256, DKV_DK = 320, DKV_KT = 384, DKV_VT = 416;
 
 __global__ void __launch_bounds__(BW_THREADS, 1)
     flash_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q,
@@ -507,8 +514,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             tc::mbar_init(&ctl->st_full[i], 1);
             tc::mbar_init(&ctl->st_empty[i], BW_EW_WARPS);
             tc::mbar_init(&ctl->ew_done[i], BW_EW_WARPS);
-            tc::mbar_init(&ctl->pds_free[i], 1);
         }
+        tc::mbar_init(&ctl->kv_tmem, BW_EW_WARPS);
         tc::mbar_init(&ctl->acc_done, 1);
         tc::mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
@@ -545,25 +552,22 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_st = tc::idesc_bf16_f32(128, 64, 0, 0);   // K Q^T, V dO^T
             constexpr uint32_t idesc_acc = tc::idesc_bf16_f32(128, 64, 0, 1);  // P^T dO, dS^T Q
-            const uint32_t k_addr = tc::smem_u32(smem + DKV_OFF_K), v_addr = tc::smem_u32(smem + DKV_OFF_V);
-            bool ok = tc::mbar_wait(&ctl->kv_full, 0, abort, status);
+            bool ok = tc::mbar_wait(&ctl->kv_tmem, 0, abort, status);
             auto accumulate = [&](int it) -> bool {   // dV += P^T dO, dK += dS^T Q for tile it
                 const int r = it & 1, s = it % DKV_STAGES;
                 if (!tc::mbar_wait(&ctl->ew_done[r], (it >> 1) & 1, abort, status)) return false;
                 tc::fence_after_sync();
                 const uint32_t q_addr = tc::smem_u32(smem + DKV_OFF_Q + s * DKV_STAGE_BYTES);
                 const uint32_t do_addr = q_addr + T64_BYTES;
-                const uint32_t pt = tc::smem_u32(smem + DKV_OFF_PT + r * T128_BYTES);
-                const uint32_t dst = tc::smem_u32(smem + DKV_OFF_DST + r * T128_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {   // K = 64 queries
+                for (int kk = 0; kk < 4; ++kk) {   // K = 64 queries: 16 per MMA, 8 packed columns
                     const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    tc::mma_bf16(tmem + DKV_DV, tc::smem_desc_sw128(pt + kk * 32, 16, 1024),
-                                 tc::smem_desc_sw128(do_addr + kk * 2048, T64_BYTES, 1024), idesc_acc, acc);
-                    tc::mma_bf16(tmem + DKV_DK, tc::smem_desc_sw128(dst + kk * 32, 16, 1024),
-                                 tc::smem_desc_sw128(q_addr + kk * 2048, T64_BYTES, 1024), idesc_acc, acc);
+                    const uint32_t col = r * 64 + (kk >> 1) * 32 + (kk & 1) * 8;
+                    tc::mma_bf16_ts(tmem + DKV_DV, tmem + DKV_ST + col,
+                                    tc::smem_desc_sw128(do_addr + kk * 2048, T64_BYTES, 1024), idesc_acc, acc);
+                    tc::mma_bf16_ts(tmem + DKV_DK, tmem + DKV_DPT + col,
+                                    tc::smem_desc_sw128(q_addr + kk * 2048, T64_BYTES, 1024), idesc_acc, acc);
                 }
-                tc::mma_commit(&ctl->pds_free[r]);
                 tc::mma_commit(&ctl->q_empty[s]);
                 return true;
             };
@@ -576,10 +580,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 const uint32_t do_addr = q_addr + T64_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
-                    tc::mma_bf16(tmem + DKV_ST + r * 64, tc::smem_desc_sw128(k_addr + kk * 32, 16, 1024),
-                                 tc::smem_desc_sw128(q_addr + kk * 32, 16, 1024), idesc_st, kk > 0 ? 1u : 0u);
-                    tc::mma_bf16(tmem + DKV_DPT + r * 64, tc::smem_desc_sw128(v_addr + kk * 32, 16, 1024),
-                                 tc::smem_desc_sw128(do_addr + kk * 32, 16, 1024), idesc_st, kk > 0 ? 1u : 0u);
+                    tc::mma_bf16_ts(tmem + DKV_ST + r * 64, tmem + DKV_KT + kk * 8,
+                                    tc::smem_desc_sw128(q_addr + kk * 32, 16, 1024), idesc_st, kk > 0 ? 1u : 0u);
+                    tc::mma_bf16_ts(tmem + DKV_DPT + r * 64, tmem + DKV_VT + kk * 8,
+                                    tc::smem_desc_sw128(do_addr + kk * 32, 16, 1024), idesc_st, kk > 0 ? 1u : 0u);
                 }
                 tc::mma_commit(&ctl->st_full[r]);
                 if (it > 0 && !accumulate(it - 1)) { ok = false; break; }
@@ -611,6 +615,31 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         float nxt = n_it > 0 ? fetch(0) : 0.f;
         float nxt2 = n_it > 1 ? fetch(1) : 0.f;
         bool ok = true;
+        {
+            // K and V rows into TMEM as the packed bf16 A operands of the S^T and dP^T MMAs:
+            // this thread's key row, head columns [32 chalf, 32 chalf + 32) = 16 columns
+            uint32_t w = 0;
+            if (lane == 0) w = tc::mbar_wait(&ctl->kv_full, 0, abort, status) ? 1u : 0u;
+            w = __shfl_sync(0xffffffffu, w, 0);
+            if (w) {
+                uint32_t kw[16], vw[16];
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const uint4 kq = *reinterpret_cast<const uint4*>(smem + DKV_OFF_K + swz128(r, chalf * 4 + g));
+                    const uint4 vq = *reinterpret_cast<const uint4*>(smem + DKV_OFF_V + swz128(r, chalf * 4 + g));
+                    kw[4 * g] = kq.x; kw[4 * g + 1] = kq.y; kw[4 * g + 2] = kq.z; kw[4 * g + 3] = kq.w;
+                    vw[4 * g] = vq.x; vw[4 * g + 1] = vq.y; vw[4 * g + 2] = vq.z; vw[4 * g + 3] = vq.w;
+                }
+                tc::tmem_st_32x32b_x16(tmem + DKV_KT + chalf * 16 + lane_off, kw);
+                tc::tmem_st_32x32b_x16(tmem + DKV_VT + chalf * 16 + lane_off, vw);
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&ctl->kv_tmem);
+            } else {
+                ok = false;
+            }
+        }
         for (int it = 0; it < n_it; ++it) {
             const int rb = it & 1;
             const int q0 = (it0 + it) * 64;
@@ -620,18 +649,15 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             nxt = nxt2;
             if (it + 2 < n_it) nxt2 = fetch(it + 2);
             uint32_t w = 0;
-            if (lane == 0 && ok) {
-                w = tc::mbar_wait(&ctl->st_full[rb], (it >> 1) & 1, abort, status) ? 1u : 0u;
-                if (w) w = tc::mbar_wait(&ctl->pds_free[rb], ((it >> 1) & 1) ^ 1, abort, status) ? 1u : 0u;
-            }
+            // st_full also means every earlier MMA is done, among them the dV/dK MMAs that
+            // read this buffer's P^T / dS^T two tiles ago
+            if (lane == 0 && ok) w = tc::mbar_wait(&ctl->st_full[rb], (it >> 1) & 1, abort, status) ? 1u : 0u;
             w = __shfl_sync(0xffffffffu, w, 0);
             // after a failed wait keep looping without work, so that every
             // element-wise warp reaches the named barrier equally often
             if (!w) { ok = false; continue; }
             tc::fence_after_sync();
             const bool diag = (q0 < k0 + 128);          // some queries of the tile precede some keys
-            uint8_t* pt = smem + DKV_OFF_PT + rb * T128_BYTES;
-            uint8_t* dst = smem + DKV_OFF_DST + rb * T128_BYTES;
             float sv[32], dp[32];
             tc::tmem_ld2_32x32b_x32(tmem + DKV_ST + rb * 64 + chalf * 32 + lane_off,
                                     tmem + DKV_DPT + rb * 64 + chalf * 32 + lane_off, sv, dp);
@@ -652,13 +678,17 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 }
                 upk2(mul2(pk2(sv[e], sv[e + 1]), add2(pk2(dp[e], dp[e + 1]), pk2(nd.x, nd.y))), dp[e], dp[e + 1]);
             }
+            // P^T and dS^T as packed bf16 over the first 16 columns of this warp's S^T / dP^T half
+            uint32_t pw[16], dw[16];
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
-                const int chunk = chalf * 4 + g;
-                *reinterpret_cast<uint4*>(pt + swz128(r, chunk)) = pack8_bf16(sv + 8 * g);
-                *reinterpret_cast<uint4*>(dst + swz128(r, chunk)) = pack8_bf16(dp + 8 * g);
+                const uint4 a = pack8_bf16(sv + 8 * g), d = pack8_bf16(dp + 8 * g);
+                pw[4 * g] = a.x; pw[4 * g + 1] = a.y; pw[4 * g + 2] = a.z; pw[4 * g + 3] = a.w;
+                dw[4 * g] = d.x; dw[4 * g + 1] = d.y; dw[4 * g + 2] = d.z; dw[4 * g + 3] = d.w;
             }
-            tc::fence_proxy_async_smem();
+            tc::tmem_st_32x32b_x16(tmem + DKV_ST + rb * 64 + chalf * 32 + lane_off, pw);
+            tc::tmem_st_32x32b_x16(tmem + DKV_DPT + rb * 64 + chalf * 32 + lane_off, dw);
+            tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) {
@@ -675,7 +705,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 float v[64];
                 tc::tmem_ld_32x32b_x64(tmem + DKV_DK + lane_off, v);
                 bf16* kbase = dqkv + ((long long)row_base + k0) * 3 * C + C + h * HD;
-                uint8_t* stage = smem + DKV_OFF_PT;     // free: every MMA has completed
+                uint8_t* stage = smem + DKV_OFF_STAGE;
                 store_rows_64(stage, r, v, 0.125f, kbase, 3LL * C, Tn - k0);
                 tc::tmem_ld_32x32b_x64(tmem + DKV_DV + lane_off, v);
                 store_rows_64(stage, r, v, 1.0f, kbase + C, 3LL * C, Tn - k0);
@@ -687,7 +717,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     if (warp == 1) tc::tmem_dealloc(tmem, 512);
 }
 
-constexpr int DQ_STAGES = 3;
+constexpr int DQ_STAGES = 6;    // K/V ring, likewise
 struct CtlDq {
     uint64_t q_full;
     uint64_t kv_full[DQ_STAGES], kv_empty[DQ_STAGES];
