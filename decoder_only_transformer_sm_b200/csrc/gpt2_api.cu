@@ -388,17 +388,28 @@ void attn_fwd<bf16>(gpt2_handle* h, const bf16* qkv, bf16* out, float* lse, int 
     }
 }
 template <typename A>
-void attn_bwd(gpt2_handle* h, const A* qkv, const A* out, const A* dout, const float* lse, A* dqkv, int B, int T);
+void attn_bwd(gpt2_handle* h, const A* qkv, const A* out, const A* dout, const float* lse, A* dqkv, int B, int T,
+              float* colsum_part);
+// Whether attn_bwd<A> takes the tcgen05 path, which can also leave the column
+// sums of dqkv (per 32-row group) in colsum_part.
+template <typename A>
+bool attn_bwd_sums(gpt2_handle*) {
+    return false;
+}
+template <>
+bool attn_bwd_sums<bf16>(gpt2_handle* h) {
+    return h->use_tc_attention && h->use_tcgen05_attention_bwd && attention_tc_supported(h->hd);
+}
 template <>
 void attn_bwd<float>(gpt2_handle* h, const float* qkv, const float* out, const float* dout, const float* lse,
-                     float* dqkv, int B, int T) {
+                     float* dqkv, int B, int T, float*) {
     launch_attention_bwd_simt<float>(h->ctx(), qkv, out, dout, lse, h->dpre, dqkv, B, T, h->H, h->hd);
 }
 template <>
 void attn_bwd<bf16>(gpt2_handle* h, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
-                    bf16* dqkv, int B, int T) {
-    if (h->use_tc_attention && h->use_tcgen05_attention_bwd && attention_tc_supported(h->hd)) {
-        if (!launch_attention_bwd_tc(h->ctx(), qkv, out, dout, lse, h->dpre, dqkv, B, T, h->H))
+                    bf16* dqkv, int B, int T, float* colsum_part) {
+    if (attn_bwd_sums<bf16>(h)) {
+        if (!launch_attention_bwd_tc(h->ctx(), qkv, out, dout, lse, h->dpre, dqkv, B, T, h->H, colsum_part))
             h->host_error = "tensor-map encoding failed for the attention backward";
     } else if (h->use_tc_attention)
         launch_attention_bwd_mma(h->ctx(), qkv, out, dout, lse, h->dpre, dqkv, B, T, h->H, h->hd);
@@ -528,11 +539,20 @@ void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
         gemm<A>(h, "gemm dgrad attn.c_proj", GEMM_NN, h->dres_act, wop<A>(h, o.wproj), BT, C, C,
                 epi(EPI_STORE, h->dO, C));
         // attention
+        // on the tcgen05 path the backward also leaves per-32-row column sums of dqkv
+        // (the c_attn bias gradient) in red_scratch
+        const bool attn_sums = attn_bwd_sums<A>(h);
         PROF("attention bwd", 0, 0, 0, att_bwd_flops, (double)BT * C * es * 8,
              attn_bwd<A>(h, (const A*)h->qkv[l], (const A*)h->att[l], (const A*)h->dO, h->lse[l], (A*)h->dqkv, B,
-                         T));
-        PROF("bias colsum", 0, 0, 0, 0.0, (double)BT * 3 * C * es,
-             launch_colsum<A>(c, (const A*)h->dqkv, BT, 3 * C, G + o.bqkv, h->red_scratch));
+                         T, attn_sums ? h->red_scratch : nullptr));
+        if (attn_sums) {
+            const int groups = B * ceil_div(T, 32);
+            PROF("bias colsum", 0, 0, 0, 0.0, (double)groups * 3 * C * 4,
+                 launch_colred_finalize(c, h->red_scratch, groups, 3 * C, G + o.bqkv));
+        } else {
+            PROF("bias colsum", 0, 0, 0, 0.0, (double)BT * 3 * C * es,
+                 launch_colsum<A>(c, (const A*)h->dqkv, BT, 3 * C, G + o.bqkv, h->red_scratch));
+        }
         // attn.c_attn
         acc = epi(EPI_ACCUM_F32, G + o.wqkv, C);
         acc.beta = 1.f;
@@ -764,7 +784,8 @@ int gpt2_create(const gpt2_config* cfg, void* stream, gpt2_handle** out) {
         const size_t ln_part = (size_t)ln_bwd_col_blocks((int)BT) * 3 * C;
         const size_t cs_part = (size_t)colsum_row_blocks((int)BT) * 4 * C;
         const size_t mul_part = (size_t)ceil_div((int)BT, 32) * 4 * C;   // fused colsum of the GELU backward
-        plan.push_back({(void**)&h->red_scratch, std::max(std::max(ln_part, cs_part), mul_part) * 4});
+        const size_t att_part = (size_t)cfg->max_B * ceil_div(cfg->max_T, 32) * 3 * C;   // ... of the attention bwd
+        plan.push_back({(void**)&h->red_scratch, std::max(std::max(ln_part, cs_part), std::max(mul_part, att_part)) * 4});
     }
     plan.push_back({(void**)&h->d_tokens, 2 * BT * 4});
     size_t total = 0;

@@ -433,8 +433,11 @@ constexpr int T128_BYTES = 128 * HD * 2;    // 16 KB
 // Write one 64-column bf16 result row (128 bytes) per thread of a 4-warp group
 // through a swizzled 128-row staging tile, then copy whole rows to global
 // memory: dst(row) = base + row * ld (elements), rows >= n_rows skipped.
+// If csum is non-null, the warp also writes the column sums of its 32 rows
+// (rows at or beyond n_rows excluded) of the stored bf16 values as 64 floats
+// at csum; a warp whose rows all lie beyond n_rows writes nothing.
 __device__ __forceinline__ void store_rows_64(uint8_t* stage, int r, const float* v, float scale, bf16* base,
-                                              long long ld, int n_rows) {
+                                              long long ld, int n_rows, float* csum) {
     const int lane = threadIdx.x & 31, quarter = (threadIdx.x >> 5) & 3;
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -451,6 +454,20 @@ __device__ __forceinline__ void store_rows_64(uint8_t* stage, int r, const float
         if (rr < n_rows)
             *reinterpret_cast<uint4*>(base + (long long)rr * ld + lseg * 8) =
                 *reinterpret_cast<const uint4*>(stage + swz128(rr, lseg));
+    }
+    if (csum && quarter * 32 < n_rows) {   // lane = columns 2 lane, 2 lane + 1
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int rr = quarter * 32 + i;
+            if (rr < n_rows) {
+                const uint32_t w2 = *reinterpret_cast<const uint32_t*>(stage + swz128(rr, lane >> 2) + (lane & 3) * 4);
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w2));
+                s0 += f.x;
+                s1 += f.y;
+            }
+        }
+        *reinterpret_cast<float2*>(csum + 2 * lane) = make_float2(s0, s1);
     }
     __syncwarp();
 }
@@ -488,7 +505,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     flash_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q,
                             const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ lse,
                             const float* __restrict__ dpre, bf16* __restrict__ dqkv, int Tn, int H,
-                            unsigned* status) {
+                            float* __restrict__ colsum_part, unsigned* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     CtlDkv* ctl = reinterpret_cast<CtlDkv*>(smem + DKV_OFF_CTL);
@@ -706,9 +723,12 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 tc::tmem_ld_32x32b_x64(tmem + DKV_DK + lane_off, v);
                 bf16* kbase = dqkv + ((long long)row_base + k0) * 3 * C + C + h * HD;
                 uint8_t* stage = smem + DKV_OFF_STAGE;
-                store_rows_64(stage, r, v, 0.125f, kbase, 3LL * C, Tn - k0);
+                // column sums (the c_attn bias gradient) of this warp's 32-row group
+                float* cs = colsum_part ? colsum_part + ((long long)b * ((Tn + 31) / 32) + kt * 4 + quarter) * 3 * C
+                                        : nullptr;
+                store_rows_64(stage, r, v, 0.125f, kbase, 3LL * C, Tn - k0, cs ? cs + C + h * HD : nullptr);
                 tc::tmem_ld_32x32b_x64(tmem + DKV_DV + lane_off, v);
-                store_rows_64(stage, r, v, 1.0f, kbase + C, 3LL * C, Tn - k0);
+                store_rows_64(stage, r, v, 1.0f, kbase + C, 3LL * C, Tn - k0, cs ? cs + 2 * C + h * HD : nullptr);
             }
         }
     }
@@ -742,7 +762,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     flash_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q128, const __grid_constant__ CUtensorMap tm_kv64,
                            const __grid_constant__ CUtensorMap tm_do128, const float* __restrict__ lse,
                            const float* __restrict__ dpre, bf16* __restrict__ dqkv, int Tn, int H,
-                           unsigned* status) {
+                           float* __restrict__ colsum_part, unsigned* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     CtlDq* ctl = reinterpret_cast<CtlDq*>(smem + DQ_OFF_CTL);
@@ -903,7 +923,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 float v[64];
                 tc::tmem_ld_32x32b_x64(tmem + DQ_DQ + lane_off, v);
                 bf16* qbase = dqkv + ((long long)row_base + q0) * 3 * C + h * HD;
-                store_rows_64(smem + DQ_OFF_DS, r, v, 0.125f, qbase, 3LL * C, Tn - q0);
+                float* cs = colsum_part ? colsum_part + ((long long)b * ((Tn + 31) / 32) + qt * 4 + quarter) * 3 * C
+                                        : nullptr;
+                store_rows_64(smem + DQ_OFF_DS, r, v, 0.125f, qbase, 3LL * C, Tn - q0, cs ? cs + h * HD : nullptr);
             }
         }
     }
@@ -954,7 +976,7 @@ bool launch_attention_fwd_tc(const Ctx& ctx, const bf16* qkv, bf16* out, float* 
 }
 
 bool launch_attention_bwd_tc(const Ctx& ctx, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
-                             float* dpre, bf16* dqkv, int B, int Tn, int H) {
+                             float* dpre, bf16* dqkv, int B, int Tn, int H, float* colsum_part) {
     auto fn = encode_fn_attn();
     if (!fn) return false;
     const long long C = (long long)H * HD;
@@ -980,9 +1002,9 @@ bool launch_attention_bwd_tc(const Ctx& ctx, const bf16* qkv, const bf16* out, c
     launch_attention_bwd_pre(ctx, out, dout, dpre, B, Tn, H, HD);
     const dim3 grid(B * H, ceil_div(Tn, 128));
     flash_bwd_dkv_tc_kernel<<<grid, BW_THREADS, DKV_SMEM, ctx.stream>>>(qkv128, qkv64, do64, lse, dpre, dqkv, Tn, H,
-                                                                         ctx.status);
+                                                                         colsum_part, ctx.status);
     flash_bwd_dq_tc_kernel<<<grid, BW_THREADS, DQ_SMEM, ctx.stream>>>(qkv128, qkv64, do128, lse, dpre, dqkv, Tn, H,
-                                                                       ctx.status);
+                                                                       colsum_part, ctx.status);
     *ctx.launches += 2;
     return true;
 }

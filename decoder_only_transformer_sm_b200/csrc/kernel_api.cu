@@ -106,16 +106,18 @@ extern "C" int gpt2k_attention_fwd(int dtype, const void* qkv, void* out, float*
 }
 
 extern "C" int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, const void* dout, const float* lse,
-                                   void* dqkv, int B, int T, int H, int hd, float* workspace_dev, int engine,
-                                   uint32_t* status_dev, void* stream) {
+                                   void* dqkv, int B, int T, int H, int hd, float* workspace_dev,
+                                   float* colsum_part, int engine, uint32_t* status_dev, void* stream) {
     int rc = check_attention_args(dtype, B, T, H, hd, engine, qkv, out, dout, status_dev);
     if (rc) return rc;
     if (!lse || !dqkv || !workspace_dev) return set_error(GPT2_ERR_INVALID_ARG, "NULL operand");
+    if (colsum_part && engine != 2)
+        return set_error(GPT2_ERR_INVALID_ARG, "column sums come only with the tcgen05 attention backward");
     long long launches = 0;
     Ctx c = kctx(stream, status_dev, &launches);
     if (engine == 2) {
         if (!launch_attention_bwd_tc(c, (const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, workspace_dev,
-                                     (bf16*)dqkv, B, T, H))
+                                     (bf16*)dqkv, B, T, H, colsum_part))
             return set_error(GPT2_ERR_CUDA, "tensor-map encoding failed");
     } else if (engine == 1)
         launch_attention_bwd_mma(c, (const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, workspace_dev,

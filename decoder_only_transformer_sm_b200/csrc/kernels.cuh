@@ -122,8 +122,10 @@ void launch_attention_bwd_mma(const Ctx& ctx, const bf16* qkv, const bf16* out, 
 bool attention_tc_supported(int hd);
 bool launch_attention_fwd_tc(const Ctx& ctx, const bf16* qkv, bf16* out, float* lse, int B, int Tn, int H);
 // tcgen05 flash attention backward (head width 64): D pre-pass, dK/dV kernel, dQ kernel.
+// colsum_part (nullable): fp32 [B * ceil(Tn / 32)][3C]; row b * ceil(Tn / 32) + g
+// receives the column sums of dqkv rows 32 g .. 32 g + 31 of sequence b.
 bool launch_attention_bwd_tc(const Ctx& ctx, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
-                             float* dpre, bf16* dqkv, int B, int Tn, int H);
+                             float* dpre, bf16* dqkv, int B, int Tn, int H, float* colsum_part);
 // D = rowsum(dout * out) per (b, h, t) (the backward's pre-pass).
 void launch_attention_bwd_pre(const Ctx& ctx, const bf16* out, const bf16* dout, float* dpre, int B, int Tn, int H,
                               int hd);

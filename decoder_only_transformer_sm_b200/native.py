@@ -86,7 +86,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gpt2_profile_read": (I, [P, P, I, ctypes.POINTER(I)]),
         "gpt2k_matmul_bf16": (I, [I, P, P, I, I, I, I, P, ctypes.c_int64, P, P, P, P, P, F, I, P, P]),
         "gpt2k_attention_fwd": (I, [I, P, P, P, I, I, I, I, I, P, P]),
-        "gpt2k_attention_bwd": (I, [I, P, P, P, P, P, I, I, I, I, P, I, P, P]),
+        "gpt2k_attention_bwd": (I, [I, P, P, P, P, P, I, I, I, I, P, P, I, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -286,12 +286,12 @@ def attention_fwd(qkv, out, lse, B: int, T: int, H: int, hd: int, engine: int = 
 
 
 def attention_bwd(qkv, out, dout, lse, dqkv, B: int, T: int, H: int, hd: int, workspace, engine: int = 0,
-                  status=None, stream=None):
+                  status=None, stream=None, colsum_part=None):
     """gpt2k_attention_bwd on torch device tensors (workspace: B*H*T float32)."""
     status, stream = _stream_and_status(qkv, status, stream)
     _check(load_library().gpt2k_attention_bwd(_dtype_code(qkv), _ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse),
-                                              _ptr(dqkv), B, T, H, hd, _ptr(workspace), engine, _ptr(status),
-                                              stream))
+                                              _ptr(dqkv), B, T, H, hd, _ptr(workspace), _ptr(colsum_part), engine,
+                                              _ptr(status), stream))
     return status
 
 

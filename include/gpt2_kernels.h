@@ -88,11 +88,15 @@ int gpt2k_attention_fwd(int dtype, const void* qkv, void* out, float* lse, int B
 /* Backward of gpt2k_attention_fwd: dqkv (B, T, 3C) = [dq | dk | dv] from qkv,
  * out, dout (B, T, C) and lse.
  * workspace_dev: caller-owned scratch of B*H*T floats (D = rowsum(dout * out)).
+ * colsum_part: engine 2 only, else NULL: fp32 [B * ceil(T / 32), 3C] (stride
+ *         3C); row b * ceil(T / 32) + g receives the column sums of the stored
+ *         dqkv rows 32 g .. min(32 g + 31, T - 1) of sequence b. Adding its rows
+ *         gives the bias gradient of the layer that produced qkv.
  * engine: 0 = SIMT kernel; 1 = mma.sync tensor-core kernels (bf16); 2 = tcgen05
  *         kernels (bf16, hd = 64: TMEM accumulators for dK, dV, dQ). */
 int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, const void* dout, const float* lse,
-                        void* dqkv, int B, int T, int H, int hd, float* workspace_dev, int engine,
-                        uint32_t* status_dev, void* stream);
+                        void* dqkv, int B, int T, int H, int hd, float* workspace_dev, float* colsum_part,
+                        int engine, uint32_t* status_dev, void* stream);
 
 /* gpt2k_attention_bwd without a workspace argument, for callers that cannot
  * allocate device memory (a framework whose caching allocator owns the GPU's

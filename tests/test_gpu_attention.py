@@ -66,6 +66,50 @@ def test_attention_fwd_bwd_vs_oracle(dtype, engine, case):
         assert _rel(got[..., i * C:(i + 1) * C], _merge(ref, B, T, H, hd)) < tol, i
 
 
+@pytest.mark.parametrize("case", [(2, 200, 12, 64), (3, 37, 2, 64), (1, 1, 3, 64), (16, 1024, 12, 64)])
+def test_tcgen05_backward_column_sums(case):
+    """colsum_part of the tcgen05 backward: per sequence and 32-row group, the
+    column sums of the stored dqkv rows (compared with sums of the stored dqkv
+    itself, so only the summation order separates them: 1e-5 of the group's
+    absolute sum); ragged T leaves a short last group."""
+    from decoder_only_transformer_sm_b200 import native
+    B, T, H, hd = case
+    C = H * hd
+    g = torch.Generator().manual_seed(7 * T + H)
+    qkv = torch.randn((B, T, 3 * C), generator=g).to(torch.bfloat16).cuda()
+    dout = torch.randn((B, T, C), generator=g).to(torch.bfloat16).cuda()
+    out = torch.empty((B, T, C), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
+    dqkv = torch.empty_like(qkv)
+    ws = torch.empty((B * H * T,), dtype=torch.float32, device="cuda")
+    G = (T + 31) // 32
+    part = torch.full((B * G, 3 * C), float("nan"), device="cuda")
+    st = native.attention_fwd(qkv, out, lse, B, T, H, hd, engine=2)
+    native.attention_bwd(qkv, out, dout, lse, dqkv, B, T, H, hd, ws, engine=2, status=st, colsum_part=part)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    d = dqkv.float().cpu().numpy().astype(np.float64)
+    pad = np.zeros((B, G * 32, 3 * C))
+    pad[:, :T] = d
+    ref = pad.reshape(B * G, 32, 3 * C).sum(axis=1)
+    scale = np.abs(pad).reshape(B * G, 32, 3 * C).sum(axis=1) + 1e-30
+    got = part.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(got))
+    assert np.max(np.abs(got - ref) / scale) < 1e-5
+
+
+def test_column_sums_need_tcgen05_backward():
+    from decoder_only_transformer_sm_b200 import native
+    B, T, H, hd = 1, 64, 1, 64
+    x = torch.zeros((B, T, 3 * H * hd), dtype=torch.bfloat16, device="cuda")
+    o = torch.zeros((B, T, H * hd), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((B, H, T), device="cuda")
+    ws = torch.zeros(B * H * T, device="cuda")
+    part = torch.zeros((2, 3 * H * hd), device="cuda")
+    with pytest.raises(native.Gpt2Error):
+        native.attention_bwd(x, o, o, lse, torch.zeros_like(x), B, T, H, hd, ws, engine=1, colsum_part=part)
+
+
 def test_attention_rejects_bad_head_width():
     from decoder_only_transformer_sm_b200 import native
     x = torch.zeros((1, 4, 3 * 48), device="cuda")
