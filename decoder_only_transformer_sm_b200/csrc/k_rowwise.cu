@@ -190,8 +190,18 @@ __global__ void __launch_bounds__(1024) colred_finalize_kernel(const float* __re
     const int i = blockIdx.x * 32 + threadIdx.x;
     const int stride = n * n_out;
     float s = 0.f;
-    if (i < stride)
-        for (int b = threadIdx.y; b < nblk; b += 32) s += partial[(long long)b * stride + i];
+    if (i < stride) {
+        // eight loads in flight per step; the additions keep their order
+        int b = threadIdx.y;
+        for (; b + 7 * 32 < nblk; b += 8 * 32) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = partial[(long long)(b + 32 * u) * stride + i];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) s += v[u];
+        }
+        for (; b < nblk; b += 32) s += partial[(long long)b * stride + i];
+    }
     part[threadIdx.y][threadIdx.x] = s;
     __syncthreads();
     if (threadIdx.y == 0 && i < stride) {
