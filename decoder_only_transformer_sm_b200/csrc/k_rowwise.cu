@@ -180,6 +180,139 @@ __global__ void __launch_bounds__(32 * LNB_WARPS, NV <= 8 ? 2 : 1)
     }
 }
 
+// The same LayerNorm backward with each warp's next row (dy, x, dres_in) copied
+// into a two-slot shared-memory ring by cp.async while the current row is
+// processed, so every warp keeps a row of loads in flight. Shared memory:
+// 8 warps x (3 partial rows + 2 ring rows) = 256 C bytes for bf16 dy, so
+// C <= 880; one block per SM. Lane-owned columns: each lane reads back exactly
+// the chunks it copied, so the ring needs no synchronisation across lanes.
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_8(void* smem_dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+constexpr int LNB_RING_BLOCKS = 148;   // one block per SM of a B200; a fixed count keeps the sum order fixed
+template <typename T, int NV>
+__global__ void __launch_bounds__(32 * LNB_WARPS, 1)
+    ln_bwd_ring_kernel(const T* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ mean,
+                       const float* __restrict__ rstd, const float* __restrict__ w, const float* dres_in,
+                       float* dres_out, T* __restrict__ dres_act, int rows, int C, int rows_per_block,
+                       int want_dx_sum, float* __restrict__ partial) {
+    extern __shared__ float4 smem4[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int C4 = C >> 2;
+    float4* acc4 = smem4;                              // [LNB_WARPS][3][C / 4]
+    float4* mine = acc4 + warp * 3 * C4;
+    const size_t row_bytes = (size_t)C * (sizeof(T) + 8);   // dy | x | dres_in
+    uint8_t* ring = reinterpret_cast<uint8_t*>(smem4 + LNB_WARPS * 3 * C4) + (size_t)warp * 2 * row_bytes;
+    for (int i = lane; i < 3 * C4; i += 32) mine[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float ww[NV][4];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c4 = lane + 32 * i;
+        if (c4 < C4) load4(w + 4 * c4, ww[i]);
+    }
+    auto issue = [&](int row, int slot) {
+        uint8_t* b = ring + slot * row_bytes;
+        T* sdy = reinterpret_cast<T*>(b);
+        float* sx = reinterpret_cast<float*>(b + (size_t)C * sizeof(T));
+        float* sres = sx + C;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int c4 = lane + 32 * i;
+            if (c4 < C4) {
+                const long long g = (long long)row * C + 4 * c4;
+                if (sizeof(T) == 2) cp_async_8(sdy + 4 * c4, dy + g);
+                else cp_async_16(sdy + 4 * c4, dy + g);
+                cp_async_16(sx + 4 * c4, x + g);
+                if (dres_in) cp_async_16(sres + 4 * c4, dres_in + g);
+            }
+        }
+        cp_async_commit_group();
+    };
+    const int r0 = blockIdx.x * rows_per_block;
+    const int r1 = min(rows, r0 + rows_per_block);
+    if (r0 + warp < r1) issue(r0 + warp, 0);
+    int slot = 0;
+    for (int row = r0 + warp; row < r1; row += LNB_WARPS, slot ^= 1) {
+        const int nxt = row + LNB_WARPS;
+        const float mu = mean[row], rs = rstd[row];
+        if (nxt < r1) {
+            issue(nxt, slot ^ 1);
+            cp_async_wait_group<1>();
+        } else {
+            cp_async_wait_group<0>();
+        }
+        const uint8_t* b = ring + slot * row_bytes;
+        const T* sdy = reinterpret_cast<const T*>(b);
+        const float* sx = reinterpret_cast<const float*>(b + (size_t)C * sizeof(T));
+        const float* sres = sx + C;
+        float dxh[NV][4], xh[NV][4];
+        float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int c4 = lane + 32 * i;
+            if (c4 < C4) {
+                float g[4], xx[4];
+                load4(sdy + 4 * c4, g);
+                load4(sx + 4 * c4, xx);
+                float4 aw = mine[c4], ab = mine[C4 + c4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    xh[i][j] = (xx[j] - mu) * rs;
+                    dxh[i][j] = g[j] * ww[i][j];
+                    s1 += dxh[i][j];
+                    s2 += dxh[i][j] * xh[i][j];
+                }
+                aw.x += g[0] * xh[i][0]; aw.y += g[1] * xh[i][1]; aw.z += g[2] * xh[i][2]; aw.w += g[3] * xh[i][3];
+                ab.x += g[0]; ab.y += g[1]; ab.z += g[2]; ab.w += g[3];
+                mine[c4] = aw;
+                mine[C4 + c4] = ab;
+            }
+        }
+        s1 = warp_sum(s1) / C;
+        s2 = warp_sum(s2) / C;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int c4 = lane + 32 * i;
+            if (c4 < C4) {
+                const int c = 4 * c4;
+                float o[4], res[4] = {0.f, 0.f, 0.f, 0.f};
+                if (dres_in) load4(sres + c, res);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) o[j] = rs * (dxh[i][j] - s1 - xh[i][j] * s2) + res[j];
+                store4(dres_out + (long long)row * C + c, o);
+                if (dres_act) store4(dres_act + (long long)row * C + c, o);
+                if (want_dx_sum) {
+                    float4 an = mine[2 * C4 + c4];
+                    an.x += o[0]; an.y += o[1]; an.z += o[2]; an.w += o[3];
+                    mine[2 * C4 + c4] = an;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    float4* part = reinterpret_cast<float4*>(partial + (long long)blockIdx.x * 3 * C);
+    for (int i = threadIdx.x; i < 3 * C4; i += blockDim.x) {
+        float4 t = acc4[i];
+#pragma unroll
+        for (int k = 1; k < LNB_WARPS; ++k) {
+            const float4 u = acc4[k * 3 * C4 + i];
+            t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
+        }
+        part[i] = t;
+    }
+}
+
 // out_k[j] += sum over nblk partial rows of partial[b][k * n + j], k < n_out;
 // a null out_k is skipped. Block = 32 columns x 32 row groups: each thread sums
 // every 32nd partial row of its column (coalesced across the warp), then the
@@ -539,10 +672,36 @@ void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const flo
                           const float* w, const float* dres_in, float* dres_out, T* dres_act, float* dw,
                           float* db, float* dbias_next, int rows, int C, float* scratch) {
     const int nv = ceil_div(C, 128);
+    const int want = dbias_next != nullptr;
+    const size_t ring_smem = (size_t)LNB_WARPS * (3 * C * sizeof(float) + 2 * C * (sizeof(T) + 8));
+    if (ring_smem <= 220 * 1024 && nv <= 8) {
+        const int nblk = min(ceil_div(rows, LNB_WARPS), LNB_RING_BLOCKS);
+        const int rpb = ceil_div(rows, nblk);
+#define LNR_CASE(N)                                                                                         \
+    case N: {                                                                                               \
+        static bool configured = false;                                                                     \
+        if (!configured) {                                                                                  \
+            cudaFuncSetAttribute(ln_bwd_ring_kernel<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,     \
+                                 220 * 1024);                                                               \
+            configured = true;                                                                              \
+        }                                                                                                   \
+        ln_bwd_ring_kernel<T, N><<<nblk, 32 * LNB_WARPS, ring_smem, ctx.stream>>>(                          \
+            dy, x, mean, rstd, w, dres_in, dres_out, dres_act, rows, C, rpb, want, scratch);                \
+        break;                                                                                              \
+    }
+        switch (nv) {
+            LNR_CASE(1) LNR_CASE(2) LNR_CASE(3) LNR_CASE(4) LNR_CASE(5) LNR_CASE(6) LNR_CASE(7) LNR_CASE(8)
+            default: break;
+        }
+#undef LNR_CASE
+        colred_finalize_kernel<<<ceil_div(3 * C, 32), dim3(32, 32), 0, ctx.stream>>>(scratch, nblk, C, 3, dw, db,
+                                                                                      dbias_next);
+        *ctx.launches += 2;
+        return;
+    }
     const int nblk = ln_bwd_col_blocks(rows);
     const int rpb = ceil_div(rows, nblk);
     const size_t smem = (size_t)LNB_WARPS * 3 * C * sizeof(float);
-    const int want = dbias_next != nullptr;
 #define LNB_CASE(N)                                                                                         \
     case N: {                                                                                               \
         static bool configured = false;                                                                     \
