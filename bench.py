@@ -213,12 +213,33 @@ def traffic_for(site: str):
     return e.get("bytes_per_launch")
 
 
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The largest of every rank's x (the job's time is that of its slowest rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_tokens(rank: int, B: int, T: int, vocab_real: int, nb: int = 2):
+    """The nb synthetic batches of one replica: each rank draws its own seeded Zipf stream."""
+    from decoder_only_transformer_sm_b200 import synthetic as S
+    return [S.zipf_tokens(B, T, vocab_real, seed=1001 + 97 * rank + i) for i in range(nb)]
+
+
+def job_throughput(ms_per_step_max: float, B: int, T: int, world: int) -> float:
+    """Whole-job tokens/s: every replica's tokens over the slowest rank's step time."""
+    return B * T * world / (ms_per_step_max / 1000.0)
+
+
 def run_ours(args):
-    import numpy as np
     import torch
     import torch.distributed as dist
 
-    from decoder_only_transformer_sm_b200 import native, synthetic as S
+    from decoder_only_transformer_sm_b200 import native
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -231,7 +252,7 @@ def run_ours(args):
     m = native.GPT2(w["n_layer"], w["n_head"], w["n_embd"], w["vocab_size"], w["block_size"], B, T,
                     precision="bf16", seed=1234 + rank, stream=stream.cuda_stream)
     nb = 2
-    host = [S.zipf_tokens(B, T, w["vocab_real"], seed=1001 + 97 * rank + i) for i in range(nb)]
+    host = replica_tokens(rank, B, T, w["vocab_real"], nb)
     pin = [(torch.from_numpy(i).pin_memory(), torch.from_numpy(t).pin_memory()) for i, t in host]
     dev = [(i.cuda(), t.cuda()) for i, t in pin]
     torch.cuda.synchronize()
@@ -239,13 +260,6 @@ def run_ours(args):
     def barrier():
         if world > 1:
             dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     for k in range(args.warmup):
         m.step(*dev[k % nb], LR)
@@ -267,7 +281,7 @@ def run_ours(args):
         torch.cuda.synchronize()
     barrier()
     clocks = clk.summary()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
 
     # ---- end to end: host (pinned) token buffers through gpt2_step_host ----
     barrier()
@@ -279,7 +293,7 @@ def run_ours(args):
     e3.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms_e2e = max_over_ranks(e2.elapsed_time(e3) / args.steps)
+    ms_e2e = max_over_ranks(e2.elapsed_time(e3) / args.steps, world)
 
     # ---- per-launch-site device times (CUDA events on the launching stream) ----
     m.profile(True)
@@ -295,8 +309,7 @@ def run_ours(args):
         return
 
     peaks, peak_src = load_peaks()
-    tokens = B * T * world
-    value = tokens / (ms / 1000.0)
+    value = job_throughput(ms, B, T, world)
     fpt = flops_per_token(w)
     total_ms = sum(s["total_ms"] for s in stats) / args.steps
     sites = sorted(stats, key=lambda s: -s["total_ms"])
@@ -342,7 +355,7 @@ def run_ours(args):
                      "per_launch_ms": per_launch_ms, "peak_note": peak_note},
         "kernels": breakdown,
         "cpu_baseline": cpu,
-        "e2e": {"value": tokens / (ms_e2e / 1000.0), "unit": "tokens/s",
+        "e2e": {"value": job_throughput(ms_e2e, B, T, world), "unit": "tokens/s",
                 "h2d_bytes_per_step": 2 * B * T * 4, "d2h_bytes_per_step": 40},
         "gpu_launches": launches,
         "clocks": clocks,
