@@ -100,6 +100,14 @@ const char* gpt2_last_error(void);
  * 0.02, and the residual scaling"): N(0, 0.02) for wte, wpe and the Linear
  * weights, N(0, 0.02/sqrt(2 n_layer)) for both c_proj weights, zero biases,
  * LayerNorm weight 1, bias 0. AdamW moments and the step counter start at 0.
+ * Kernel choice in bf16 mode (read from the environment here, once per handle;
+ * the defaults are the fastest measured):
+ *   GPT2_B200_SIMT_GEMM=1             SIMT GEMMs instead of the tcgen05 ones
+ *   GPT2_B200_SIMT_ATTENTION=1        SIMT attention instead of the tensor-core kernels
+ *   GPT2_B200_TCGEN05_ATTENTION=0     mma.sync attention forward instead of tcgen05
+ *   GPT2_B200_TCGEN05_ATTENTION_BWD=0 mma.sync attention backward instead of tcgen05
+ *   GPT2_B200_NO_GRAPH=1              no CUDA-graph replay of the step (see gpt2_step)
+ * fp32 mode always uses the SIMT kernels.
  * Errors: INVALID_ARG (sizes), UNSUPPORTED_ARCH, OOM, CUDA. */
 int gpt2_create(const gpt2_config* cfg, void* stream, gpt2_handle** out);
 
