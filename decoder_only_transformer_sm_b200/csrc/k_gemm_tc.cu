@@ -458,9 +458,12 @@ bool launch_variant(const Ctx& ctx, const CUtensorMap& ta, const CUtensorMap& tb
     u.splits = 1;
     const int tiles = u.tiles_m * u.tiles_n;
     // Split K when the output has too few tiles to fill the GPU and the epilogue
-    // accumulates into fp32 (partials are then added with atomics).
+    // accumulates into fp32 (partials are then added with atomics). Every extra
+    // split adds a full tile of fp32 atomics, so one wave of units when that
+    // fills at least 85% of the SMs, else about two waves.
     if (ep.kind == EPI_ACCUM_F32 && ep.beta == 1.f && tiles < g_num_sms) {
-        int s = (2 * g_num_sms + tiles / 2) / tiles;
+        int s = g_num_sms / tiles;
+        if (tiles * s * 100 < 85 * g_num_sms) s = (2 * g_num_sms + tiles / 2) / tiles;
         s = min(s, max(1, u.kb_total / 8));
         u.splits = max(1, s);
     }
