@@ -235,6 +235,53 @@ def job_throughput(ms_per_step_max: float, B: int, T: int, world: int) -> float:
     return B * T * world / (ms_per_step_max / 1000.0)
 
 
+def run_eval(args):
+    """Forward-only throughput on the benchmark's shapes: held-out loss (forward +
+    cross-entropy, no gradients) and the last-position forward that feeds
+    next-token sampling. Device-resident inputs, CUDA events, one GPU."""
+    import torch
+
+    from decoder_only_transformer_sm_b200 import native
+
+    w = WORKLOAD
+    B, T = args.batch, w["T"]
+    stream = torch.cuda.current_stream()
+    m = native.GPT2(w["n_layer"], w["n_head"], w["n_embd"], w["vocab_size"], w["block_size"], B, T,
+                    precision="bf16", seed=1234, stream=stream.cuda_stream)
+    idx, tgt = (torch.from_numpy(a).cuda() for a in replica_tokens(0, B, T, w["vocab_real"], 1)[0])
+    last = torch.empty((B, w["vocab_size"]), dtype=torch.bfloat16, device="cuda")
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    losses = []
+    ms_loss = timed(lambda: losses.append(m.forward(idx, tgt)))
+    ms_last = timed(lambda: m.forward_last(idx, last))
+    m.close()
+    line = {
+        "metric": "eval tokens/sec (GPT-2 124M, B=16, T=1024, bf16 forward + loss)",
+        "value": B * T / (ms_loss / 1000.0), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_loss, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic Zipf(1.1) tokens, random-init weights",
+        "workload": "eval",
+        "config": dict(workload_config(B, T, 1),
+                       workload="gpt2-124m eval: forward + CE loss, no gradients; B=16 T=1024 V=50304 bf16"),
+        "forward_last": {"ms_per_call": ms_last, "tokens_per_s": B * T / (ms_last / 1000.0),
+                         "note": "blocks + ln_f on all B*T positions, lm_head on the B last rows"},
+        "loss": losses[-1],
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -370,6 +417,9 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["train", "eval"], default="train",
+                    help="train: the training step (the benchmark line); eval: forward + loss and the "
+                         "last-position forward of generation, one GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=WORKLOAD["B"],
                     help="sequences per step (default 16, the benchmark workload); smaller values are for "
@@ -379,6 +429,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "eval":
+        run_eval(args)
     else:
         run_ours(args)
 

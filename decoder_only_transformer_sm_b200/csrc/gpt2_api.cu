@@ -433,7 +433,7 @@ template <> const bf16* wop<bf16>(gpt2_handle* h, long long off) { return h->sha
 // ------------------------------------------------------------------ forward
 template <typename A>
 void forward_impl(gpt2_handle* h, const int* idx, const int* targets, int B, int T, A* logits_out,
-                  double* loss_slot, float loss_scale, bool write_grad) {
+                  double* loss_slot, float loss_scale, bool write_grad, bool last_only = false) {
     Ctx c = h->ctx();
     const int BT = B * T, C = h->C, V = h->V, L = h->L, H = h->H, hd = h->hd;
     const double es = sizeof(A);
@@ -471,6 +471,13 @@ void forward_impl(gpt2_handle* h, const int* idx, const int* targets, int B, int
                                      last ? P + h->off_lnfb : P + h->lo[l + 1].ln1b,
                                      last ? (A*)h->lnf : (A*)h->ln1[l + 1], h->ln_mean[2 * l + 2],
                                      h->ln_rstd[2 * l + 2], BT, C));
+    }
+    if (last_only) {   // logits of each sequence's last position only: (B, V)
+        PROF("gather last rows", 0, 0, 0, 0.0, 2.0 * B * C * es,
+             launch_gather_last_rows<A>(c, (const A*)h->lnf, B, T, C, (A*)h->dtmp));
+        gemm<A>(h, "gemm fwd lm_head (last position)", GEMM_NT, h->dtmp, wop<A>(h, h->off_wte), B, V, C,
+                epi(EPI_STORE, logits_out, V));
+        return;
     }
     A* lg = logits_out ? logits_out : (A*)h->logits;
     gemm<A>(h, "gemm fwd lm_head", GEMM_NT, h->lnf, wop<A>(h, h->off_wte), BT, V, C, epi(EPI_STORE, lg, V));
@@ -932,6 +939,23 @@ int gpt2_forward(gpt2_handle* h, const int32_t* idx, const int32_t* targets, int
         return status_error(h);
     }
     return GPT2_OK;
+}
+
+int gpt2_forward_last(gpt2_handle* h, const int32_t* idx, int B, int T, void* logits_dev) {
+    if (!h || !idx || !logits_dev) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    int rc = check_bt(h, B, T);
+    if (rc) return rc;
+    h->launches = 0;
+    if (h->bf16_mode)
+        forward_impl<bf16>(h, idx, nullptr, B, T, (bf16*)logits_dev, nullptr, 1.f, false, true);
+    else
+        forward_impl<float>(h, idx, nullptr, B, T, (float*)logits_dev, nullptr, 1.f, false, true);
+    CK(cudaGetLastError());
+    rc = pending_error(h);
+    if (rc) return rc;
+    rc = read_scalars(h);   // synchronises; reports a bad token id
+    if (rc) return rc;
+    return status_error(h);
 }
 
 int gpt2_zero_grad(gpt2_handle* h) {

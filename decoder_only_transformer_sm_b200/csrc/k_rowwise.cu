@@ -734,6 +734,20 @@ void launch_colred_finalize(const Ctx& ctx, const float* partial, int nblk, int 
     ++*ctx.launches;
 }
 
+template <typename T>
+__global__ void gather_last_rows_kernel(const T* __restrict__ src, int Tn, int C, T* __restrict__ dst) {
+    const int b = blockIdx.x;
+    const uint4* s = reinterpret_cast<const uint4*>(src + ((long long)b * Tn + Tn - 1) * C);
+    uint4* d = reinterpret_cast<uint4*>(dst + (long long)b * C);
+    for (int i = threadIdx.x; i < C * (int)sizeof(T) / 16; i += blockDim.x) d[i] = s[i];
+}
+
+template <typename T>
+void launch_gather_last_rows(const Ctx& ctx, const T* src, int B, int Tn, int C, T* dst) {
+    gather_last_rows_kernel<T><<<B, 128, 0, ctx.stream>>>(src, Tn, C, dst);
+    ++*ctx.launches;
+}
+
 void launch_count_targets(const Ctx& ctx, const int* targets, int n, int V, int* n_valid) {
     count_targets_kernel<<<1, 1024, 0, ctx.stream>>>(targets, n, V, n_valid, ctx.status);
     ++*ctx.launches;
@@ -778,7 +792,8 @@ void launch_embed_bwd(const Ctx& ctx, const int* idx, const float* dx, int B, in
                                           const float*, const float*, float*, T*, float*, float*, float*, int, \
                                           int, float*);                                                        \
     template void launch_classifier<T>(const Ctx&, T*, const int*, int, int, const int*, float, double*, int); \
-    template void launch_colsum<T>(const Ctx&, const T*, int, int, float*, float*);
+    template void launch_colsum<T>(const Ctx&, const T*, int, int, float*, float*);                          \
+    template void launch_gather_last_rows<T>(const Ctx&, const T*, int, int, int, T*);
 INST(float)
 INST(bf16)
 #undef INST

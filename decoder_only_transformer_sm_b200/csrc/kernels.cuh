@@ -91,6 +91,9 @@ void launch_count_targets(const Ctx& ctx, const int* targets, int n, int V, int*
 template <typename T>
 void launch_classifier(const Ctx& ctx, T* logits, const int* targets, int rows, int V, const int* n_valid,
                        float scale, double* loss_accum, int write_grad);
+// dst[b, :] = src[b * Tn + Tn - 1, :] for b < B (each sequence's last row; C % 8 == 0).
+template <typename T>
+void launch_gather_last_rows(const Ctx& ctx, const T* src, int B, int Tn, int C, T* dst);
 // Column sums: out[c] += sum_r in[r, c], through colsum_row_blocks(rows) x cols
 // partials in scratch and a fixed-order finalize. cols is a multiple of 8.
 inline int colsum_row_blocks(int rows) { return (rows + 31) / 32; }

@@ -76,6 +76,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gpt2_get_opt_state": (I, [P, P, P, ctypes.POINTER(ctypes.c_int64), I]),
         "gpt2_set_opt_state": (I, [P, P, P, ctypes.c_int64, I]),
         "gpt2_forward": (I, [P, P, P, I, I, P, ctypes.POINTER(F)]),
+        "gpt2_forward_last": (I, [P, P, I, I, P]),
         "gpt2_zero_grad": (I, [P]),
         "gpt2_accumulate": (I, [P, P, P, I, I, F]),
         "gpt2_update": (I, [P, F, ctypes.POINTER(F), ctypes.POINTER(F)]),
@@ -193,6 +194,11 @@ class GPT2:
         _check(self._lib.gpt2_forward(self._h, _ptr(idx), _ptr(targets), B, T, _ptr(logits),
                                       ctypes.byref(loss) if targets is not None else None))
         return loss.value if targets is not None else None
+
+    def forward_last(self, idx, logits):
+        """Logits (B, vocab_size) of each sequence's last position (gpt2_forward_last)."""
+        B, T = idx.shape
+        _check(self._lib.gpt2_forward_last(self._h, _ptr(idx), B, T, _ptr(logits)))
 
     def zero_grad(self):
         _check(self._lib.gpt2_zero_grad(self._h))

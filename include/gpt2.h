@@ -150,6 +150,20 @@ int gpt2_set_opt_state(gpt2_handle* h, const float* m, const float* v, int64_t s
 int gpt2_forward(gpt2_handle* h, const int32_t* idx_dev, const int32_t* targets_dev,
                  int B, int T, void* logits_dev, float* loss_host);
 
+/* Forward pass with the logits of each sequence's last position only, the
+ * input of next-token sampling ("GPT-2 from Scratch", "A generation loop": the
+ * forward without targets keeps only the last position's logits, from which
+ * the next token is drawn).
+ * The blocks and ln_f run on all T positions (causal attention needs them);
+ * the tied lm_head runs on the B last rows, so no (B, T, vocab_size) tensor is
+ * formed.
+ * idx_dev    : (B, T) int32 token ids on the device.
+ * logits_dev : device buffer for (B, vocab_size) logits: fp32 in fp32 mode,
+ *              bf16 in bf16 mode; row b = position T - 1 of sequence b.
+ * Synchronises once at the end. Errors: as gpt2_forward; BAD_TOKEN for an id
+ * outside [0, vocab_size). */
+int gpt2_forward_last(gpt2_handle* h, const int32_t* idx_dev, int B, int T, void* logits_dev);
+
 /* Set every gradient to zero and clear the accumulated loss. Asynchronous. */
 int gpt2_zero_grad(gpt2_handle* h);
 

@@ -321,3 +321,30 @@ def test_step_graph_replay_matches_eager(monkeypatch):
         assert mg.last_launch_count() == me.last_launch_count(), i
     mg.close()
     me.close()
+
+
+@pytest.mark.parametrize("precision,T", [("fp32", 64), ("fp32", 23), ("bf16", 64), ("bf16", 23)])
+def test_forward_last_position_logits(precision, T):
+    """gpt2_forward_last: each sequence's last-position logits against the
+    oracle's full forward (fp32: 1e-4 of max |logit|; bf16: 2e-2, the bf16
+    tolerance), and within 1e-6 of the same row of the GPU's own full-logits
+    forward in fp32 mode (the same arithmetic on the same rows)."""
+    s = TINY
+    B = 3
+    idx, _ = S.uniform_tokens(B, T, s.vocab_size, seed=900 + T)
+    flat = S.random_params(s, seed=901)
+    m = _model(s, precision, 4, 64)
+    m.set_params(flat)
+    tdt = torch.float32 if precision == "fp32" else torch.bfloat16
+    last = torch.empty((B, s.vocab_size), dtype=tdt, device="cuda")
+    m.forward_last(_dev(idx), last)
+    full = torch.empty((B, T, s.vocab_size), dtype=tdt, device="cuda")
+    m.forward(_dev(idx), None, full)
+    P = O.unflatten(_oshape(s), flat.astype(np.float64))
+    _, ref_logits, _ = O.forward(_oshape(s), P, idx)
+    got = last.float().cpu().numpy()
+    tol = 1e-4 if precision == "fp32" else 2e-2
+    assert _rel(got, ref_logits[:, -1, :]) < tol
+    if precision == "fp32":
+        assert _rel(got, full[:, -1, :].cpu().numpy()) < 1e-6
+    m.close()
