@@ -34,8 +34,24 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-WORKLOAD = dict(n_layer=12, n_head=12, n_embd=768, vocab_size=50304, vocab_real=50257, block_size=1024,
-                B=16, T=1024)
+MODELS = {
+    "124m": dict(name="GPT-2 124M", n_layer=12, n_head=12, n_embd=768, vocab_size=50304, vocab_real=50257,
+                 block_size=1024, B=16, T=1024),
+    "medium": dict(name="GPT-2 medium", n_layer=24, n_head=16, n_embd=1024, vocab_size=50304, vocab_real=50257,
+                   block_size=1024, B=8, T=1024),
+    "large": dict(name="GPT-2 large", n_layer=36, n_head=20, n_embd=1280, vocab_size=50304, vocab_real=50257,
+                  block_size=1024, B=8, T=1024),
+    "xl": dict(name="GPT-2 XL", n_layer=48, n_head=25, n_embd=1600, vocab_size=50304, vocab_real=50257,
+               block_size=1024, B=4, T=1024),
+}
+WORKLOAD = MODELS["124m"]   # the benchmark workload
+METRIC = "training tokens/sec and MFU at GPT-2 124M (B=16,T=1024, bf16), 1×B200"
+
+
+def metric_for(w, B: int, T: int) -> str:
+    if w is WORKLOAD and B == w["B"] and T == w["T"]:
+        return METRIC
+    return f"training tokens/sec and MFU at {w['name']} (B={B},T={T}, bf16)"
 LR = 6e-4
 NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -151,8 +167,9 @@ def oracle_step_time(T_sample: int, warm: int, steps: int):
     return times, threads
 
 
-def workload_config(B: int, T: int, world: int) -> dict:
-    return {"workload": "gpt2-124m train step (fwd+CE+bwd+clip+AdamW), B=16 T=1024 V=50304 bf16",
+def workload_config(B: int, T: int, world: int, w=None) -> dict:
+    w = w or WORKLOAD
+    return {"workload": f"{w['name']} train step (fwd+CE+bwd+clip+AdamW), B={B} T={T} V={w['vocab_size']} bf16",
             "B": B, "T": T, "tokens_per_step_per_gpu": B * T,
             "parallelism": "replicas" if world > 1 else "single-gpu",
             "l2": "working set (6+ GB of activations per step) larger than the 126 MB L2; no flush"}
@@ -170,7 +187,7 @@ def run_reference(args):
               f"backward, clip, AdamW on all 124.5M parameters) on B=1 x T={T_sample} Zipf tokens; warm-up "
               f"steps are forward passes on 16 tokens; value = sampled tokens / oracle seconds")
     line = {
-        "metric": "training tokens/sec (GPT-2 124M, B=16, T=1024, bf16 step)",
+        "metric": METRIC,
         "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * sec, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic Zipf(1.1) tokens", "impl": "reference",
@@ -244,7 +261,7 @@ def run_eval(args):
     from decoder_only_transformer_sm_b200 import native
 
     w = WORKLOAD
-    B, T = args.batch, w["T"]
+    B, T = args.batch or w["B"], w["T"]
     stream = torch.cuda.current_stream()
     m = native.GPT2(w["n_layer"], w["n_head"], w["n_embd"], w["vocab_size"], w["block_size"], B, T,
                     precision="bf16", seed=1234, stream=stream.cuda_stream)
@@ -293,8 +310,8 @@ def run_ours(args):
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
-    w = WORKLOAD
-    B, T = args.batch, w["T"]
+    w = MODELS[args.model]
+    B, T = args.batch or w["B"], w["T"]
     stream = torch.cuda.current_stream()
     m = native.GPT2(w["n_layer"], w["n_head"], w["n_embd"], w["vocab_size"], w["block_size"], B, T,
                     precision="bf16", seed=1234 + rank, stream=stream.cuda_stream)
@@ -383,17 +400,17 @@ def run_ours(args):
             row["gbs"] = round(s["bytes"] / (s["total_ms"] / 1e3) / 1e9, 1)
         breakdown.append(row)
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and w is WORKLOAD:
         times, threads = oracle_step_time(1024, 0, 1)
         cpu = {"value": 1024 / times[0], "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": "one float64 oracle step (forward, loss, backward, clip, AdamW on all 124.5M "
                          "parameters) on B=1 x T=1024 Zipf tokens, timed on this host"}
     line = {
-        "metric": "training tokens/sec (GPT-2 124M, B=16, T=1024, bf16 step)",
+        "metric": metric_for(w, B, T),
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic Zipf(1.1) tokens, random-init weights",
-        "config": workload_config(B, T, world),
+        "config": workload_config(B, T, world, w),
         "mfu": {"flops_per_token": fpt, "vs_nominal_2250": value * fpt / world / (NOMINAL_BF16_TFLOPS * 1e12),
                 "vs_measured_sustained": value * fpt / world / (peaks.get("bf16_tflops_sustained", 1400.0) * 1e12),
                 "peak_source": peak_src},
@@ -421,9 +438,13 @@ def main():
                     help="train: the training step (the benchmark line); eval: forward + loss and the "
                          "last-position forward of generation, one GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--batch", type=int, default=WORKLOAD["B"],
-                    help="sequences per step (default 16, the benchmark workload); smaller values are for "
-                         "small-footprint profiler captures and do not produce the benchmark number")
+    ap.add_argument("--model", choices=sorted(MODELS), default="124m",
+                    help="124m is the benchmark workload; the others are the same step at GPT-2 medium, "
+                         "large and XL sizes (B = 8, 8, 4)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="sequences per step (default: the model's B, 16 for the 124m benchmark workload); "
+                         "other values are for small-footprint profiler captures and do not produce the "
+                         "benchmark number")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

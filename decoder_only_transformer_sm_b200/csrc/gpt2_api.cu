@@ -1005,6 +1005,22 @@ int gpt2_step_host(gpt2_handle* h, const int32_t* idx_host, const int32_t* targe
     return rc;
 }
 
+int gpt2_lr_at(int64_t step, float max_lr, float min_lr, int64_t warmup, int64_t max_steps, float* lr_out) {
+    if (!lr_out || step < 0 || warmup < 1 || max_steps < warmup)
+        return fail(GPT2_ERR_INVALID_ARG, "lr schedule: need step >= 0, warmup >= 1, max_steps >= warmup");
+    double lr;
+    if (step < warmup) {
+        lr = (double)max_lr * (double)(step + 1) / (double)warmup;
+    } else if (step > max_steps) {
+        lr = min_lr;
+    } else {
+        const double f = (double)(step - warmup) / (double)std::max<int64_t>(1, max_steps - warmup);
+        lr = min_lr + ((double)max_lr - min_lr) * 0.5 * (1.0 + cos(M_PI * f));
+    }
+    *lr_out = (float)lr;
+    return GPT2_OK;
+}
+
 int gpt2_profile(gpt2_handle* h, int enable) {
     if (!h) return fail(GPT2_ERR_INVALID_ARG, "NULL handle");
     CK(cudaStreamSynchronize(h->stream));

@@ -77,6 +77,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gpt2_set_opt_state": (I, [P, P, P, ctypes.c_int64, I]),
         "gpt2_forward": (I, [P, P, P, I, I, P, ctypes.POINTER(F)]),
         "gpt2_forward_last": (I, [P, P, I, I, P]),
+        "gpt2_lr_at": (I, [ctypes.c_int64, F, F, ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(F)]),
         "gpt2_zero_grad": (I, [P]),
         "gpt2_accumulate": (I, [P, P, P, I, I, F]),
         "gpt2_update": (I, [P, F, ctypes.POINTER(F), ctypes.POINTER(F)]),
@@ -267,6 +268,13 @@ def matmul_bf16(layout: str, A, B, M: int, N: int, K: int, epilogue: str, out, l
                                _ptr(colsum_part), beta, 1 if engine == "tc" else 0, _ptr(status), stream)
     _check(rc)
     return status
+
+
+def lr_at(step: int, max_lr: float, min_lr: float, warmup: int, max_steps: int) -> float:
+    """gpt2_lr_at: the warmup + cosine learning-rate schedule (host only, no GPU)."""
+    out = ctypes.c_float()
+    _check(load_library().gpt2_lr_at(step, max_lr, min_lr, warmup, max_steps, ctypes.byref(out)))
+    return out.value
 
 
 def _dtype_code(t) -> int:

@@ -198,6 +198,15 @@ int gpt2_step(gpt2_handle* h, const int32_t* idx_dev, const int32_t* targets_dev
 int gpt2_step_host(gpt2_handle* h, const int32_t* idx_host, const int32_t* targets_host,
                    int B, int T, float lr, float* loss_host, float* grad_norm_host);
 
+/* Learning rate for a 0-based step ("GPT-2 from Scratch", "Warmup and cosine
+ * decay"; "Let's reproduce GPT-2 (124M)": 6e-4 peak, 10% floor, 715 warmup steps
+ * for 124M): max_lr * (step + 1) / warmup during the first `warmup` steps, then
+ * min_lr + (max_lr - min_lr) (1 + cos(pi f)) / 2 with f = (step - warmup) /
+ * max(1, max_steps - warmup), and min_lr after max_steps. A host-side scalar for
+ * the lr argument of gpt2_step / gpt2_update; needs no handle and no GPU.
+ * Errors: INVALID_ARG (step < 0, warmup < 1, max_steps < warmup, lr_out NULL). */
+int gpt2_lr_at(int64_t step, float max_lr, float min_lr, int64_t warmup, int64_t max_steps, float* lr_out);
+
 /* Number of kernel launches the last forward/accumulate/update/step issued. */
 int gpt2_last_launch_count(const gpt2_handle* h, int64_t* n);
 

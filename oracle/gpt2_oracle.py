@@ -16,7 +16,8 @@ Sources (page title, section):
     output projection), "The MLP and GPT-2's GELU", "The Block: pre-LN and
     residuals", "Forward: logits, and loss when targets are given",
     "Weight tying", "AdamW, and weight decay on matrices only",
-    "Gradient clipping", "How to scale up" (gradient accumulation).
+    "Gradient clipping", "How to scale up" (gradient accumulation),
+    "Warmup and cosine decay" (the learning-rate schedule).
   * "Let's reproduce GPT-2 (124M)" synopsis: "Matching GPT-3's optimization
     hyperparameters" (betas, eps, clip 1.0, decay on 2-D tensors only) and
     "Gradient accumulation, and the bug in getting it right".
@@ -320,6 +321,21 @@ def adamw_update(s: Shape, P: dict, G: dict, M: dict, V: dict, t: int, lr: float
 
 def zeros_like(s: Shape) -> dict:
     return {name: np.zeros(shp) for name, shp in layout(s)}
+
+
+def lr_schedule(step: int, max_lr: float, min_lr: float, warmup: int, max_steps: int) -> float:
+    """Learning rate at a 0-based step ("GPT-2 from Scratch", "Warmup and cosine
+    decay"): a linear ramp over the first `warmup` steps, reaching
+    max_lr * (step + 1) / warmup at step `step`; then a half cosine from max_lr
+    at step == warmup (cos 0 = 1) down to min_lr at step == max_steps (cos pi = -1),
+    the midpoint halfway; min_lr after max_steps. The decay interval counts at
+    least one step."""
+    if step < warmup:
+        return max_lr * (step + 1) / warmup
+    if step > max_steps:
+        return min_lr
+    frac = (step - warmup) / max(1, max_steps - warmup)
+    return min_lr + (max_lr - min_lr) * 0.5 * (1.0 + np.cos(np.pi * frac))
 
 
 def train_step(s: Shape, P: dict, M: dict, V: dict, t: int, idx, targets, lr: float,

@@ -74,3 +74,16 @@ def test_null_arguments():
     lib.gpt2_destroy(None)   # no-op
     n = ctypes.c_int64()
     assert lib.gpt2_num_params(None, ctypes.byref(n)) == -1
+
+
+def test_lr_schedule_entry_matches_oracle():
+    """gpt2_lr_at (host only: runs without a GPU) against the oracle's schedule,
+    float32 rounding apart, over the 124M run's steps; bad arguments rejected."""
+    from decoder_only_transformer_sm_b200 import native
+    from oracle import gpt2_oracle as O
+    mx, mn, tw, tm = 6e-4, 6e-5, 715, 19073
+    for k in list(range(0, 800, 7)) + list(range(700, 19200, 211)) + [tw - 1, tw, tm, tm + 1, 50000]:
+        assert native.lr_at(k, mx, mn, tw, tm) == pytest.approx(O.lr_schedule(k, mx, mn, tw, tm), rel=1e-6)
+    for bad in [(-1, mx, mn, tw, tm), (0, mx, mn, 0, tm), (0, mx, mn, tw, tw - 1)]:
+        with pytest.raises(native.Gpt2Error):
+            native.lr_at(*bad)

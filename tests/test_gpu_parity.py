@@ -104,10 +104,12 @@ def test_tiny_fp32_step_matches_oracle(kind):
 
 
 @pytest.mark.parametrize("precision", ["fp32", "bf16"])
-def test_gpt2_width_one_layer_grads(precision):
-    """GPT-2 small's width (C = 768, 12 heads, the 124M row layout of every
-    row-wise kernel) in one layer with a small vocabulary, ragged T."""
-    s = S.ModelShape(n_layer=1, n_head=12, n_embd=768, vocab_size=512, block_size=64)
+@pytest.mark.parametrize("C,H", [(768, 12), (1024, 16), (1280, 20), (1600, 25)])
+def test_gpt2_width_one_layer_grads(precision, C, H):
+    """The widths of GPT-2 small, medium, large and XL (head width 64; C = 1600
+    is not a multiple of 128, so the row kernels' last lane group is partial),
+    one layer each with a small vocabulary and ragged T."""
+    s = S.ModelShape(n_layer=1, n_head=H, n_embd=C, vocab_size=512, block_size=64)
     B, T = 3, 37
     idx, tgt = S.uniform_tokens(B, T, s.vocab_size, seed=77)
     tgt[1, :5] = -1

@@ -455,3 +455,38 @@ def test_planted_mistakes_are_caught(monkeypatch, mutation):
     idx, tgt = S.uniform_tokens(2, 8, 64, seed=31)
     with pytest.raises(AssertionError):
         _fd_check(s, P, idx, tgt, 8, np.random.default_rng(2))
+
+
+# ----------------------------------------------------------------------------
+# Learning-rate schedule ("GPT-2 from Scratch", "Warmup and cosine decay")
+# ----------------------------------------------------------------------------
+def test_lr_schedule_page_properties():
+    """The page fixes: a linear ramp from zero over the warmup, the peak at
+    t = t_w (cos 0 = 1), the floor at t = t_max (cos pi = -1), the midpoint
+    halfway, and a floor of 10% of the peak; the 124M run's numbers."""
+    g = GOLDEN["lr_schedule"]
+    r = GOLDEN["lr_schedule_124m_run"]
+    mx, mn, tw, tm = r["max_lr"], r["min_lr"], r["warmup_steps"], r["max_steps"]
+    assert mx == g["max_lr"] and mn == g["min_lr"] and abs(mn - 0.1 * mx) < 1e-18
+    lr = lambda k: O.lr_schedule(k, mx, mn, tw, tm)   # noqa: E731
+    assert lr(0) == pytest.approx(mx / tw)              # first step of the ramp
+    assert lr(tw - 1) == pytest.approx(mx)              # end of the ramp
+    ramp = [lr(k) for k in range(tw)]
+    assert all(b - a == pytest.approx(mx / tw) for a, b in zip(ramp, ramp[1:]))   # linear
+    assert lr(tw) == pytest.approx(mx)                  # cos 0 = 1
+    assert lr(tm) == pytest.approx(mn)                  # cos pi = -1
+    assert lr((tw + tm) / 2) == pytest.approx((mx + mn) / 2)
+    assert lr(tm + 1) == mn and lr(10 * tm) == mn
+    decay = [lr(k) for k in range(tw, tm + 1, 97)]
+    assert all(b <= a for a, b in zip(decay, decay[1:]))
+
+
+def test_lr_schedule_planted_mistakes_are_caught():
+    """A schedule that forgets the +1 of the ramp, or decays with the full
+    cosine period, or floors at zero, breaks one of the page's properties."""
+    mx, mn, tw, tm = 6e-4, 6e-5, 10, 110
+    wrong_ramp = lambda k: mx * k / tw if k < tw else O.lr_schedule(k, mx, mn, tw, tm)   # noqa: E731
+    assert wrong_ramp(tw - 1) != pytest.approx(mx)
+    wrong_period = lambda k: mn + (mx - mn) * 0.5 * (1 + np.cos(2 * np.pi * (k - tw) / (tm - tw)))   # noqa: E731
+    assert wrong_period(tm) != pytest.approx(O.lr_schedule(tm, mx, mn, tw, tm))
+    assert O.lr_schedule(tm, mx, 0.0, tw, tm) != pytest.approx(mn)
