@@ -299,6 +299,60 @@ def run_eval(args):
     print(json.dumps(line), flush=True)
 
 
+def run_accum(args):
+    """Gradient accumulation on the benchmark's micro-batch: zero_grad, 32 x
+    accumulate (loss scale 1/32; the second half of the micro-batches with
+    SFT-style masked target prefixes), one clip + AdamW update. A step here is one
+    update (32 x B x T tokens). Device-resident inputs, CUDA events, one GPU."""
+    import torch
+
+    from decoder_only_transformer_sm_b200 import native, synthetic as S
+
+    w = WORKLOAD
+    B, T, n_micro = args.batch or w["B"], w["T"], 32
+    stream = torch.cuda.current_stream()
+    m = native.GPT2(w["n_layer"], w["n_head"], w["n_embd"], w["vocab_size"], w["block_size"], B, T,
+                    precision="bf16", seed=1234, stream=stream.cuda_stream)
+    dev = [(torch.from_numpy(i).cuda(), torch.from_numpy(t).cuda())
+           for i, t in S.accumulation_batches(n_micro, B, T, w["vocab_real"], seed=1002)]
+    out = []
+
+    def update():
+        m.zero_grad()
+        for i, t in dev:
+            m.accumulate(i, t, 1.0 / n_micro)
+        out.append(m.update(LR))
+
+    for _ in range(args.warmup):
+        update()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            update()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    m.close()
+    fpt = flops_per_token(w)
+    tokens = n_micro * B * T
+    line = {
+        "metric": f"training tokens/sec and MFU at GPT-2 124M ({n_micro} x B={B},T={T} accumulation, bf16)",
+        "value": tokens / (ms / 1000.0), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic Zipf(1.1) tokens, random-init weights",
+        "workload": "accum",
+        "config": dict(workload_config(B, T, 1), tokens_per_step_per_gpu=tokens,
+                       workload=f"GPT-2 124M: zero_grad + {n_micro} x accumulate(1/{n_micro}) + update; "
+                                f"micro-batches {n_micro // 2}-{n_micro - 1} with masked target prefixes"),
+        "mfu": {"flops_per_token": fpt, "vs_nominal_2250": tokens / (ms / 1000.0) * fpt / (NOMINAL_BF16_TFLOPS * 1e12)},
+        "clocks": clk.summary(),
+        "loss_norm_last": list(out[-1]),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -434,9 +488,10 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["train", "eval"], default="train",
+    ap.add_argument("--workload", choices=["train", "eval", "accum"], default="train",
                     help="train: the training step (the benchmark line); eval: forward + loss and the "
-                         "last-position forward of generation, one GPU")
+                         "last-position forward of generation; accum: one update over 32 accumulated "
+                         "micro-batches (524,288 tokens); eval and accum on one GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--model", choices=sorted(MODELS), default="124m",
                     help="124m is the benchmark workload; the others are the same step at GPT-2 medium, "
@@ -452,6 +507,8 @@ def main():
         run_reference(args)
     elif args.workload == "eval":
         run_eval(args)
+    elif args.workload == "accum":
+        run_accum(args)
     else:
         run_ours(args)
 
