@@ -1,0 +1,49 @@
+"""Host logic of bench.py that needs no GPU: the clock record taken during the
+timed region (nvidia-smi rows, here written by the test) and the JSON line's
+shape helpers."""
+import os
+
+import pytest
+
+import bench
+
+
+def _sampler_with(rows, tmp_path):
+    s = bench.ClockSampler(0)
+    p = tmp_path / "clocks.csv"
+    p.write_text("".join(r + "\n" for r in rows))
+    s.path = str(p)
+    return s
+
+
+def test_clock_summary_uses_loaded_samples_and_active_reasons(tmp_path):
+    idle = "0, 1965, 1965, 120.0, 0x0, Not Active, Not Active, Not Active, Not Active"
+    busy = "0, 1900, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, Active"
+    busy2 = "0, 1800, 1965, 980.0, 0x4, Not Active, Not Active, Not Active, Active"
+    s = _sampler_with([idle, busy, busy2, "garbage line", idle], tmp_path)
+    out = s.summary()
+    assert out["samples"] == 2                       # idle samples (below half the peak power) left out
+    assert out["sm_mhz"] == pytest.approx(1850.0)    # median of the loaded samples
+    assert out["sm_max_mhz"] == 1965.0
+    assert out["reasons"] == ["sw_power_cap"]        # "Not Active" is not a reason
+    assert out["power_w_max"] == 980.0
+    assert not os.path.exists(s.path)                # the temporary record is removed
+
+
+def test_clock_summary_reports_throttling_and_missing_record(tmp_path):
+    hot = "0, 1200, 1965, 950.0, 0x48, Active, Not Active, Active, Not Active"
+    out = _sampler_with([hot, hot], tmp_path).summary()
+    assert out["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    empty = bench.ClockSampler(0)
+    assert empty.summary()["reasons"] == ["unsampled"]
+
+
+def test_workload_config_and_metric_names():
+    w = bench.WORKLOAD
+    c = bench.workload_config(w["B"], w["T"], 1)
+    assert c["tokens_per_step_per_gpu"] == w["B"] * w["T"] and c["parallelism"] == "single-gpu"
+    assert bench.workload_config(w["B"], w["T"], 8)["parallelism"] == "replicas"
+    assert bench.metric_for(w, w["B"], w["T"]) == bench.METRIC
+    assert bench.metric_for(bench.MODELS["xl"], 4, 1024) != bench.METRIC
+    # 6N + 12 L C T with the tied wte counted once at the padded vocabulary
+    assert bench.flops_per_token(w) == pytest.approx(8.601e8, rel=1e-3)
