@@ -153,3 +153,9 @@ def accumulation_batches(n_micro: int, B: int, T: int, vocab: int, seed: int):
             tgt = masked_prefix(tgt, rng)
         out.append((idx, tgt))
     return out
+
+
+def uniforms(n_steps: int, B: int, seed: int) -> np.ndarray:
+    """(n_steps, B) float32 uniforms in [0, 1) from default_rng(seed): the random
+    numbers of the multinomial draws of generation, one per drawn token."""
+    return np.random.default_rng(seed).random((n_steps, B)).astype(np.float32)

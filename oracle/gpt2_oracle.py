@@ -17,7 +17,9 @@ Sources (page title, section):
     residuals", "Forward: logits, and loss when targets are given",
     "Weight tying", "AdamW, and weight decay on matrices only",
     "Gradient clipping", "How to scale up" (gradient accumulation),
-    "Warmup and cosine decay" (the learning-rate schedule).
+    "Warmup and cosine decay" (the learning-rate schedule), "A generation
+    loop" (temperature, top-k, one multinomial draw per step, the context
+    cropped to block_size).
   * "Let's reproduce GPT-2 (124M)" synopsis: "Matching GPT-3's optimization
     hyperparameters" (betas, eps, clip 1.0, decay on 2-D tensors only) and
     "Gradient accumulation, and the bug in getting it right".
@@ -36,13 +38,19 @@ Readings where the pages are silent or the extraction lost the formula:
   * Clip: coef = min(1, max_norm / (norm + 1e-6)); the reported norm is pre-clip.
   * AdamW: decoupled decay scaled by lr, bias correction on both moments,
     eps added after the square root, step counter starting at 1.
+  * Sampling: the multinomial draw is an inverse CDF in vocabulary order with
+    the uniform number passed in; the k-th largest is taken on the logits
+    before the temperature division (same order for temperature > 0).
 
 Pins (tests/test_oracle_pins.py): finite differences, a torch float64
 autograd model plus torch's own cross_entropy / clip_grad_norm_ / AdamW,
 closed forms (initial loss, CE of equal logits, AdamW step 1, clip), the
 causal invariant, the T = 1 attention case, GELU identities, LN moments,
 the parameter count of "Counting parameters: 124,439,808", accumulation
-equivalence and single-batch overfitting. Parity pinned for every function.
+equivalence and single-batch overfitting; for sampling, draw frequencies
+over a grid of uniforms against torch's softmax, top-1 = argmax, kept ties,
+and greedy generation against the torch library model. Parity pinned for
+every function.
 """
 from __future__ import annotations
 
@@ -336,6 +344,64 @@ def lr_schedule(step: int, max_lr: float, min_lr: float, warmup: int, max_steps:
         return min_lr
     frac = (step - warmup) / max(1, max_steps - warmup)
     return min_lr + (max_lr - min_lr) * 0.5 * (1.0 + np.cos(np.pi * frac))
+
+
+# ----------------------------------------------------------------------------
+# Sampling ("GPT-2 from Scratch", "A generation loop").
+# ----------------------------------------------------------------------------
+def sample_next(logits, temperature: float, top_k: int, u: float):
+    """One draw from a row of last-position logits.
+
+    The row is divided by the temperature. With top_k >= 1, every entry below
+    the k-th largest (k = min(top_k, V)) becomes -inf; entries equal to the
+    k-th largest stay. The kept entries go through a softmax, and one index is
+    drawn from it. The draw is by inverse CDF in vocabulary order: u in
+    [0, 1) is given, and the result is the first j whose cumulative probability
+    (inclusive) exceeds u; if rounding leaves u at or above the last cumulative
+    value, the last kept index. top_k <= 0 keeps every entry. The k-th largest
+    is found on the row before the division, which orders the entries the same
+    way for any temperature > 0.
+
+    Returns (j, probs, margin): probs in vocabulary order, and margin = the
+    distance from u to the nearer end of the interval [cdf[j-1], cdf[j]) that
+    selected j (a decision closer than the rounding of the cumulative sums to
+    an end could go either way)."""
+    x = np.asarray(logits, dtype=np.float64).reshape(-1)
+    V = x.shape[0]
+    keep = np.ones(V, dtype=bool)
+    if top_k >= 1 and top_k < V:
+        kth = np.sort(x)[::-1][top_k - 1]
+        keep = x >= kth
+    z = np.where(keep, x / temperature, -np.inf)
+    e = np.exp(z - z.max())
+    probs = e / e.sum()
+    cdf = np.cumsum(probs)
+    over = np.nonzero(cdf > u)[0]
+    j = int(over[0]) if over.size else int(np.nonzero(keep)[0][-1])
+    lo = cdf[j - 1] if j > 0 else 0.0
+    margin = float(min(u - lo, cdf[j] - u))
+    return j, probs, margin
+
+
+def generate(s: Shape, P: dict, idx, max_new_tokens: int, temperature: float, top_k: int, u):
+    """The pages' generation loop: crop the running sequence to its last
+    block_size tokens, run the forward, take the last position's logits, draw
+    the next token (sample_next) and append it; repeat. Every step recomputes
+    the whole window (no cache). u: (max_new_tokens, B) uniforms in [0, 1),
+    one per drawn token. Returns (tokens (B, T0 + max_new_tokens), margins
+    (max_new_tokens, B))."""
+    seq = np.asarray(idx).copy()
+    u = np.asarray(u, dtype=np.float64)
+    B = seq.shape[0]
+    margins = np.zeros((max_new_tokens, B))
+    for step in range(max_new_tokens):
+        cond = seq[:, -s.block_size:]
+        _, logits, _ = forward(s, P, cond)
+        nxt = np.zeros((B, 1), dtype=seq.dtype)
+        for b in range(B):
+            nxt[b, 0], _, margins[step, b] = sample_next(logits[b, -1], temperature, top_k, u[step, b])
+        seq = np.concatenate([seq, nxt], axis=1)
+    return seq, margins
 
 
 def train_step(s: Shape, P: dict, M: dict, V: dict, t: int, idx, targets, lr: float,

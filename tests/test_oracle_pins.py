@@ -490,3 +490,126 @@ def test_lr_schedule_planted_mistakes_are_caught():
     wrong_period = lambda k: mn + (mx - mn) * 0.5 * (1 + np.cos(2 * np.pi * (k - tw) / (tm - tw)))   # noqa: E731
     assert wrong_period(tm) != pytest.approx(O.lr_schedule(tm, mx, mn, tw, tm))
     assert O.lr_schedule(tm, mx, 0.0, tw, tm) != pytest.approx(mn)
+
+
+# ----------------------------------------------------------------------------
+# Sampling and generation ("GPT-2 from Scratch", "A generation loop").
+# ----------------------------------------------------------------------------
+def _torch_topk_softmax(logits, temperature, top_k):
+    torch = pytest.importorskip("torch")
+    x = torch.tensor(logits, dtype=torch.float64) / temperature
+    if top_k >= 1:
+        v, _ = torch.topk(x, min(top_k, x.numel()))
+        x = torch.where(x < v[-1], torch.tensor(float("-inf"), dtype=torch.float64), x)
+    return torch.softmax(x, dim=-1).numpy()
+
+
+@pytest.mark.parametrize("temperature,top_k", [(1.0, 0), (0.7, 5), (1.6, 12), (0.8, 40)])
+def test_sample_frequencies_match_torch_softmax(temperature, top_k):
+    """Over a uniform grid of u, each index is drawn with the probability torch's
+    softmax of the temperature-scaled, top-k-masked row gives it: this fixes the
+    temperature (divide), the mask (drop below the k-th, keep the rest) and the
+    order of the inverse CDF (inclusive, vocabulary order)."""
+    rng = np.random.default_rng(31)
+    logits = rng.normal(0.0, 1.5, 48)
+    n = 20_000
+    us = (np.arange(n) + 0.5) / n
+    counts = np.zeros(48)
+    draws = []
+    for u in us:
+        j, probs, _ = O.sample_next(logits, temperature, top_k, u)
+        counts[j] += 1
+        draws.append(j)
+    ref = _torch_topk_softmax(logits, temperature, top_k)
+    assert np.max(np.abs(counts / n - ref)) <= 1.0 / n + 1e-12
+    assert np.max(np.abs(probs - ref)) < 1e-12
+    # inverse CDF in vocabulary order: the draw never decreases as u grows
+    assert all(a <= b for a, b in zip(draws, draws[1:]))
+
+
+def test_sample_top1_is_argmax_and_ties_at_kth_stay():
+    rng = np.random.default_rng(32)
+    x = rng.normal(size=100)
+    for u in (0.0, 0.3, 0.999999):
+        assert O.sample_next(x, 0.9, 1, u)[0] == int(np.argmax(x))
+    # three entries equal to the 2nd largest value all stay with top_k = 2
+    x = np.array([0.0, 4.0, 1.0, 4.0, 5.0, 4.0, -1.0])
+    _, probs, _ = O.sample_next(x, 1.0, 2, 0.5)
+    kept = np.nonzero(probs > 0)[0].tolist()
+    assert kept == [1, 3, 4, 5]
+    e = np.exp(np.array([4.0, 4.0, 5.0, 4.0]) - 5.0)
+    assert np.allclose(probs[kept], e / e.sum(), rtol=1e-14)
+    # top_k >= V and top_k <= 0 keep everything
+    for k in (0, -3, 7, 50):
+        assert np.all(O.sample_next(x, 1.0, k, 0.5)[1] > 0)
+
+
+def test_sample_margin_and_last_index():
+    x = np.log(np.array([0.25, 0.25, 0.5]))
+    j, probs, margin = O.sample_next(x, 1.0, 0, 0.3)
+    assert j == 1 and abs(margin - 0.05) < 1e-12          # interval [0.25, 0.5)
+    assert O.sample_next(x, 1.0, 0, 0.5)[0] == 2          # u on a boundary: the next index
+    assert O.sample_next(x, 1.0, 0, 0.0)[0] == 0
+    # with top-k the masked tail is never drawn, even at u -> 1
+    assert O.sample_next(np.array([3.0, 2.0, 1.0, 0.0]), 1.0, 2, 1.0 - 1e-15)[0] == 1
+
+
+def _torch_last_logits(s, flat, idx):
+    torch = pytest.importorskip("torch")
+    F = torch.nn.functional
+    P, off = {}, 0
+    for n, shp in O.layout(s):
+        k = int(np.prod(shp))
+        P[n] = torch.tensor(flat[off:off + k].reshape(shp), dtype=torch.float64)
+        off += k
+    C, H = s.n_embd, s.n_head
+    x_idx = torch.tensor(idx, dtype=torch.long)
+    B, T = x_idx.shape
+    x = F.embedding(x_idx, P["wte"]) + F.embedding(torch.arange(T), P["wpe"])
+    for l in range(s.n_layer):
+        p = f"h.{l}."
+        a = F.layer_norm(x, (C,), P[p + "ln_1.weight"], P[p + "ln_1.bias"], eps=1e-5)
+        q, k, v = F.linear(a, P[p + "attn.c_attn.weight"], P[p + "attn.c_attn.bias"]).split(C, dim=2)
+        q, k, v = (z.view(B, T, H, C // H).transpose(1, 2) for z in (q, k, v))
+        y = F.scaled_dot_product_attention(q, k, v, is_causal=True).transpose(1, 2).reshape(B, T, C)
+        x = x + F.linear(y, P[p + "attn.c_proj.weight"], P[p + "attn.c_proj.bias"])
+        m = F.layer_norm(x, (C,), P[p + "ln_2.weight"], P[p + "ln_2.bias"], eps=1e-5)
+        u = F.gelu(F.linear(m, P[p + "mlp.c_fc.weight"], P[p + "mlp.c_fc.bias"]), approximate="tanh")
+        x = x + F.linear(u, P[p + "mlp.c_proj.weight"], P[p + "mlp.c_proj.bias"])
+    f = F.layer_norm(x, (C,), P["ln_f.weight"], P["ln_f.bias"], eps=1e-5)
+    return F.linear(f[:, -1, :], P["wte"]).numpy()
+
+
+def test_generate_top1_matches_greedy_torch_model_past_block_size():
+    """top_k = 1 makes every draw the argmax: the oracle's loop must then equal
+    greedy decoding with torch's library layers, including the crop to the
+    last block_size tokens once the sequence outgrows the block."""
+    s = MICRO
+    flat = S.random_params(_syn(s), seed=33).astype(np.float64)
+    P = O.unflatten(s, flat)
+    idx, _ = S.uniform_tokens(2, 5, s.vocab_size, seed=34)
+    n_new = 7                                   # 5 + 7 > block_size = 8
+    u = np.random.default_rng(35).random((n_new, 2))
+    seq, margins = O.generate(s, P, idx, n_new, 0.9, 1, u)
+    ref = np.asarray(idx).copy()
+    for _ in range(n_new):
+        lg = _torch_last_logits(s, flat, ref[:, -s.block_size:])
+        ref = np.concatenate([ref, lg.argmax(axis=-1)[:, None]], axis=1)
+    assert seq.shape == (2, 12)
+    assert np.array_equal(seq, ref)
+    assert np.all(margins >= 0)
+
+
+def test_generate_draws_follow_torch_probabilities():
+    """One draw of the loop at a given u is the inverse CDF of torch's softmax of
+    the last-position logits of the torch model (temperature and top-k applied)."""
+    s = MICRO
+    flat = S.random_params(_syn(s), seed=36).astype(np.float64)
+    P = O.unflatten(s, flat)
+    idx, _ = S.uniform_tokens(3, 6, s.vocab_size, seed=37)
+    u = np.random.default_rng(38).random((1, 3))
+    seq, _ = O.generate(s, P, idx, 1, 0.8, 10, u)
+    lg = _torch_last_logits(s, flat, idx)
+    for b in range(3):
+        cdf = np.cumsum(_torch_topk_softmax(lg[b], 0.8, 10))
+        assert seq[b, -1] == int(np.searchsorted(cdf, u[0, b], side="right"))
