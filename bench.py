@@ -206,7 +206,7 @@ def kernel_source_sha(name: str) -> str:
     return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16] if os.path.exists(p) else ""
 
 
-SITE_SOURCES = [("gemm", "k_gemm_tc.cu"), ("attention", "k_attention_tc.cu"), ("layernorm", "k_rowwise.cu"),
+SITE_SOURCES = [("decode attention", "k_decode.cu"), ("sample", "k_decode.cu"), ("gemm", "k_gemm_tc.cu"), ("attention", "k_attention_tc.cu"), ("layernorm", "k_rowwise.cu"),
                 ("classifier", "k_rowwise.cu"), ("adamw", "k_optim.cu"), ("grad norm", "k_optim.cu"),
                 ("embed", "k_rowwise.cu"), ("bias colsum", "k_rowwise.cu")]
 
@@ -295,6 +295,83 @@ def run_eval(args):
         "forward_last": {"ms_per_call": ms_last, "tokens_per_s": B * T / (ms_last / 1000.0),
                          "note": "blocks + ln_f on all B*T positions, lm_head on the B last rows"},
         "loss": losses[-1],
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_generate(args):
+    """Generation throughput ("GPT-2 from Scratch", "A generation loop"): the
+    pages' sampling call (a short prompt, 40 new tokens, temperature 0.8,
+    top-k 40) through gpt2_generate on GPT-2 124M bf16: one prefill that fills
+    the key/value cache, then per token one decode step and one draw.
+    Device-resident prompt and uniforms; CUDA events around whole calls (each
+    call ends with one synchronisation). The bf16 weights (250 MB) exceed the
+    L2, so every decode step streams them from HBM."""
+    import torch
+
+    from decoder_only_transformer_sm_b200 import native
+    from decoder_only_transformer_sm_b200 import synthetic as S
+
+    w = WORKLOAD
+    B, T0, n_new, temperature, top_k = args.batch or 1, 4, 40, 0.8, 40
+    stream = torch.cuda.current_stream()
+    m = native.GPT2(w["n_layer"], w["n_head"], w["n_embd"], w["vocab_size"], w["block_size"], B, w["T"],
+                    precision="bf16", seed=1234, stream=stream.cuda_stream)
+    prompt = torch.from_numpy(S.zipf_tokens(B, T0, w["vocab_real"], seed=1001)[0]).cuda()
+    u = torch.from_numpy(S.uniforms(n_new, B, seed=1002)).cuda()
+    out = torch.empty((B, T0 + n_new), dtype=torch.int32, device="cuda")
+
+    def call():
+        m.generate(prompt, n_new, temperature, top_k, u, out)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches = 0
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            call()
+            launches += m.last_launch_count()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    clocks = clk.summary()
+    ms = e0.elapsed_time(e1) / args.steps
+    m.profile(True)
+    call()
+    stats = m.profile_read()
+    m.profile(False)
+    m.close()
+
+    peaks, peak_src = load_peaks()
+    total_ms = sum(s["total_ms"] for s in stats)
+    sites = sorted(stats, key=lambda s: -s["total_ms"])
+    dom = sites[0]
+    per_launch_ms = dom["total_ms"] / dom["launches"]
+    achieved = dom["bytes"] / dom["launches"] / (per_launch_ms / 1e3) / 1e9
+    peak = peaks.get("hbm_gbs")
+    breakdown = [{"site": s["name"], "ms_per_call": round(s["total_ms"], 4), "share": round(s["total_ms"] / total_ms, 4),
+                  "launches_per_call": s["launches"],
+                  "gbs": round(s["bytes"] / (s["total_ms"] / 1e3) / 1e9, 1) if s["bytes"] > 0 else None}
+                 for s in sites]
+    line = {
+        "metric": "generated tokens/sec (GPT-2 124M bf16; prompt 4, 40 new tokens, temperature 0.8, top-k 40)",
+        "value": B * n_new / (ms / 1000.0), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic Zipf(1.1) prompt, seeded uniforms for the draws, random-init weights",
+        "workload": "generate",
+        "config": {"workload": f"gpt2-124m generation: gpt2_generate, B={B}, prompt {T0}, {n_new} new tokens, "
+                               f"temperature {temperature}, top-k {top_k}; key/value cache; bf16 weights "
+                               "(250 MB) larger than L2", "global_batch": B, "seq_len": T0 + n_new,
+                   "parallelism": "single GPU"},
+        "roofline": {"kernel": dom["name"], "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak if peak else None, "traffic": None, "per_launch_ms": per_launch_ms,
+                     "peak_note": f"hbm_gbs of {peak_src}"},
+        "kernels": breakdown,
+        "gpu_launches": launches,
+        "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
 
@@ -488,10 +565,11 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["train", "eval", "accum"], default="train",
+    ap.add_argument("--workload", choices=["train", "eval", "accum", "generate"], default="train",
                     help="train: the training step (the benchmark line); eval: forward + loss and the "
                          "last-position forward of generation; accum: one update over 32 accumulated "
-                         "micro-batches (524,288 tokens); eval and accum on one GPU")
+                         "micro-batches (524,288 tokens); generate: the pages' sampling call with a "
+                         "key/value cache (--batch sets B, default 1); eval, accum and generate on one GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--model", choices=sorted(MODELS), default="124m",
                     help="124m is the benchmark workload; the others are the same step at GPT-2 medium, "
@@ -509,6 +587,8 @@ def main():
         run_eval(args)
     elif args.workload == "accum":
         run_accum(args)
+    elif args.workload == "generate":
+        run_generate(args)
     else:
         run_ours(args)
 

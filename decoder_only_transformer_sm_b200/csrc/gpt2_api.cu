@@ -131,6 +131,18 @@ struct gpt2_handle {
     int graph_B = 0, graph_T = 0;
     long long graph_launches = 0;
 
+    // Generation ("A generation loop"): per layer a key/value cache of
+    // (max_B, block_size, 3C) rows [q | k | v] in the activation type (the q
+    // block of a row is written by the decode step's qkv GEMM and read only for
+    // that row), allocated by the first prefill.
+    char* gen_pool = nullptr;
+    std::vector<void*> kv;
+    void** d_layer_ptrs = nullptr;   // device [qkv[0..L-1], kv[0..L-1]] for the cache fill
+    float* dec_part = nullptr;       // decode attention partial sums
+    int* d_next = nullptr;           // last drawn token per row (max_B): the next decode step's input
+    int* d_window = nullptr;         // contiguous token window of a prefill inside gpt2_generate (maxBT)
+    int kv_B = 0, kv_len = 0;        // rows and positions the cache holds
+
     bool profiling = false;
     std::vector<ProfSite> psites;
     std::unordered_map<std::string, int> pidx;
@@ -576,6 +588,114 @@ void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
          launch_embed_bwd(c, idx, h->dres, B, T, C, V, G + h->off_wte, G + h->off_wpe));
 }
 
+// -------------------------------------------------------------- generation
+// Cache and scratch of the generation calls, allocated on first use.
+int ensure_gen(gpt2_handle* h) {
+    if (h->gen_pool) return GPT2_OK;
+    const size_t es = h->bf16_mode ? 2 : 4;
+    const size_t L = h->L, C = h->C, Tc = h->cfg.block_size, Bm = h->cfg.max_B;
+    const size_t layer = align_up(Bm * Tc * 3 * C * es);
+    const size_t part = align_up((size_t)decode_part_floats(h->cfg.max_B * h->H, (int)Tc, h->hd) * 4);
+    const size_t ptrs = align_up(2 * L * sizeof(void*));
+    const size_t next = align_up(Bm * 4), win = align_up((size_t)h->maxBT * 4);
+    char* pool = nullptr;
+    if (cudaMalloc((void**)&pool, L * layer + part + ptrs + next + win) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(GPT2_ERR_OOM, "cudaMalloc of the key/value cache failed");
+    }
+    h->gen_pool = pool;
+    h->kv.assign(L, nullptr);
+    size_t off = 0;
+    for (size_t l = 0; l < L; ++l, off += layer) h->kv[l] = pool + off;
+    h->dec_part = (float*)(pool + off);
+    off += part;
+    h->d_layer_ptrs = (void**)(pool + off);
+    off += ptrs;
+    h->d_next = (int*)(pool + off);
+    off += next;
+    h->d_window = (int*)(pool + off);
+    std::vector<void*> tab(2 * L);
+    for (size_t l = 0; l < L; ++l) {
+        tab[l] = h->qkv[l];
+        tab[L + l] = h->kv[l];
+    }
+    CK(cudaMemcpyAsync(h->d_layer_ptrs, tab.data(), tab.size() * sizeof(void*), cudaMemcpyHostToDevice, h->stream));
+    CK(cudaStreamSynchronize(h->stream));
+    return GPT2_OK;
+}
+
+// Forward of (B, T) tokens keeping only the last position's logits (B, V),
+// then k, v of every position of every layer into cache rows 0 .. T-1.
+template <typename A>
+void prefill_impl(gpt2_handle* h, const int* idx, int B, int T, A* logits_out) {
+    forward_impl<A>(h, idx, nullptr, B, T, logits_out, nullptr, 1.f, false, true);
+    const double es = sizeof(A);
+    PROF("kv cache fill", 0, 0, 0, 0.0, 2.0 * h->L * B * T * 2 * h->C * es,
+         launch_kv_store(h->ctx(), (const void* const*)h->d_layer_ptrs, h->d_layer_ptrs + h->L, h->L, B, T,
+                         h->cfg.block_size, h->C, (int)sizeof(A)));
+}
+
+// One new position `pos` of B sequences whose cache holds rows 0 .. pos-1:
+// the blocks' forward for tok (B) at that position, its q, k, v written to
+// cache row pos, attention over rows 0 .. pos, logits (B, V).
+template <typename A>
+void decode_impl(gpt2_handle* h, const int* tok, int B, int pos, A* logits_out) {
+    Ctx c = h->ctx();
+    const int C = h->C, V = h->V, L = h->L, H = h->H, hd = h->hd, Tc = h->cfg.block_size;
+    const long long ld_kv = 3LL * C * Tc;
+    const double es = sizeof(A);
+    const double ln_fwd_bytes = (double)B * C * (4 + es) + 8.0 * B;
+    const int n = pos + 1;
+    float* P = h->params;
+    PROF("decode embed+ln_1", 0, 0, 0, 0.0, (double)B * C * (4 + 4 + 4 + es),
+         launch_embed_ln<A>(c, tok, P + h->off_wte, P + h->off_wpe + (long long)pos * C, B, 1, C, V,
+                            P + h->lo[0].ln1w, P + h->lo[0].ln1b, h->resid[0], (A*)h->ln1[0], h->ln_mean[0],
+                            h->ln_rstd[0]));
+    for (int l = 0; l < L; ++l) {
+        const LayerOff& o = h->lo[l];
+        Epilogue e = epi(EPI_BIAS, (A*)h->kv[l] + (long long)pos * 3 * C, ld_kv);
+        e.bias = P + o.bqkv;
+        gemm<A>(h, "decode gemm c_attn", GEMM_NT, h->ln1[l], wop<A>(h, o.wqkv), B, 3 * C, C, e);
+        PROF("decode attention", 0, 0, 0, 4.0 * B * H * (double)n * hd, (double)B * n * 2 * C * es,
+             launch_attention_decode<A>(c, (const A*)h->kv[l], (A*)h->att[l], h->dec_part, B, H, hd, Tc, n));
+        e = epi(EPI_BIAS_RESID, h->resid[2 * l + 1], C);
+        e.bias = P + o.bproj;
+        e.resid = h->resid[2 * l];
+        gemm<A>(h, "decode gemm attn.c_proj", GEMM_NT, h->att[l], wop<A>(h, o.wproj), B, C, C, e);
+        PROF("decode layernorm", 0, 0, 0, 0.0, ln_fwd_bytes,
+             launch_layernorm_fwd<A>(c, h->resid[2 * l + 1], P + o.ln2w, P + o.ln2b, (A*)h->ln2[l],
+                                     h->ln_mean[2 * l + 1], h->ln_rstd[2 * l + 1], B, C));
+        e = epi(EPI_BIAS_GELU, h->fcg[l], 4 * C);
+        e.out2 = h->fch[l];
+        e.bias = P + o.bfc;
+        gemm<A>(h, "decode gemm c_fc+gelu", GEMM_NT, h->ln2[l], wop<A>(h, o.wfc), B, 4 * C, C, e);
+        e = epi(EPI_BIAS_RESID, h->resid[2 * l + 2], C);
+        e.bias = P + o.bfcp;
+        e.resid = h->resid[2 * l + 1];
+        gemm<A>(h, "decode gemm mlp.c_proj", GEMM_NT, h->fcg[l], wop<A>(h, o.wfcp), B, C, 4 * C, e);
+        const bool last = (l + 1 == L);
+        PROF("decode layernorm", 0, 0, 0, 0.0, ln_fwd_bytes,
+             launch_layernorm_fwd<A>(c, h->resid[2 * l + 2], last ? P + h->off_lnfw : P + h->lo[l + 1].ln1w,
+                                     last ? P + h->off_lnfb : P + h->lo[l + 1].ln1b,
+                                     last ? (A*)h->lnf : (A*)h->ln1[l + 1], h->ln_mean[2 * l + 2],
+                                     h->ln_rstd[2 * l + 2], B, C));
+    }
+    gemm<A>(h, "decode gemm lm_head", GEMM_NT, h->lnf, wop<A>(h, h->off_wte), B, V, C, epi(EPI_STORE, logits_out, V));
+}
+
+template <typename A>
+void sample_impl(gpt2_handle* h, const A* logits, int B, float temperature, int top_k, const float* u, int* next,
+                 int* out, long long out_ld, int out_col) {
+    PROF("sample", 0, 0, 0, 0.0, (double)B * h->V * sizeof(A),
+         launch_sample<A>(h->ctx(), logits, h->V, B, h->V, temperature, top_k, u, next, out, out_ld, out_col));
+}
+
+int check_sampling(float temperature) {
+    if (!(temperature > 0.f) || !std::isfinite(temperature))
+        return fail(GPT2_ERR_INVALID_ARG, "temperature must be finite and > 0");
+    return GPT2_OK;
+}
+
 int read_scalars(gpt2_handle* h) {
     CK(cudaMemcpyAsync(h->h_sc, h->d_sc, sizeof(DevScalars), cudaMemcpyDeviceToHost, h->stream));
     CK(cudaStreamSynchronize(h->stream));
@@ -688,6 +808,33 @@ int update_impl(gpt2_handle* h, float lr, float* loss_host, float* norm_host) {
         return fail(GPT2_ERR_NONFINITE, "loss or gradient norm is not finite; update skipped");
     h->step_t = t;
     return GPT2_OK;
+}
+
+template <typename A>
+int generate_impl(gpt2_handle* h, const int* prompt, int B, int T0, int max_new, float temperature, int top_k,
+                  const float* u, int* out) {
+    const int Tb = h->cfg.block_size, Ttot = T0 + max_new;
+    Ctx c = h->ctx();
+    PROF("token copy", 0, 0, 0, 0.0, 8.0 * B * T0, launch_copy_tokens(c, prompt, T0, out, Ttot, B, T0));
+    A* lg = (A*)h->logits;
+    for (int s = 0; s < max_new; ++s) {
+        const int n = T0 + s;   // tokens so far; the draw is token n
+        if (s == 0 || n > Tb) {
+            const int W = std::min(n, Tb);
+            PROF("token copy", 0, 0, 0, 0.0, 8.0 * B * W,
+                 launch_copy_tokens(c, out + (n - W), Ttot, h->d_window, W, B, W));
+            prefill_impl<A>(h, h->d_window, B, W, lg);
+            h->kv_B = B;
+            h->kv_len = W;
+        } else {
+            decode_impl<A>(h, h->d_next, B, n - 1, lg);
+            h->kv_len = n;
+        }
+        sample_impl<A>(h, lg, B, temperature, top_k, u + (long long)s * B, h->d_next, out, Ttot, n);
+        if (!h->host_error.empty()) break;
+    }
+    CK(cudaGetLastError());
+    return pending_error(h);
 }
 
 }  // namespace
@@ -835,6 +982,7 @@ void gpt2_destroy(gpt2_handle* h) {
     cudaFree(h->shadow);
     cudaFree(h->d_chunks);
     cudaFree(h->act_pool);
+    cudaFree(h->gen_pool);
     cudaFree(h->d_sc);
     if (h->h_sc) cudaFreeHost(h->h_sc);
     for (cudaEvent_t e : h->pev) cudaEventDestroy(e);
@@ -955,6 +1103,86 @@ int gpt2_forward_last(gpt2_handle* h, const int32_t* idx, int B, int T, void* lo
     if (rc) return rc;
     rc = read_scalars(h);   // synchronises; reports a bad token id
     if (rc) return rc;
+    return status_error(h);
+}
+
+int gpt2_prefill(gpt2_handle* h, const int32_t* idx, int B, int T, void* logits_dev) {
+    if (!h || !idx || !logits_dev) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    int rc = check_bt(h, B, T);
+    if (!rc) rc = ensure_gen(h);
+    if (rc) return rc;
+    h->launches = 0;
+    if (h->bf16_mode)
+        prefill_impl<bf16>(h, idx, B, T, (bf16*)logits_dev);
+    else
+        prefill_impl<float>(h, idx, B, T, (float*)logits_dev);
+    CK(cudaGetLastError());
+    rc = pending_error(h);
+    if (rc) return rc;
+    h->kv_B = B;
+    h->kv_len = T;
+    rc = read_scalars(h);   // synchronises; reports a bad token id
+    if (rc) return rc;
+    return status_error(h);
+}
+
+int gpt2_decode(gpt2_handle* h, const int32_t* tokens, int B, int pos, void* logits_dev) {
+    if (!h || !tokens || !logits_dev) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    if (!h->gen_pool || h->kv_len < 1) return fail(GPT2_ERR_INVALID_ARG, "no cache: call gpt2_prefill first");
+    if (B < 1 || B > h->kv_B) return fail(GPT2_ERR_INVALID_ARG, "B must be in [1, rows of the last prefill]");
+    if (pos < 1 || pos > h->kv_len || pos >= h->cfg.block_size)
+        return fail(GPT2_ERR_INVALID_ARG, "pos must be in [1, cached length] and < block_size");
+    h->launches = 0;
+    if (h->bf16_mode)
+        decode_impl<bf16>(h, tokens, B, pos, (bf16*)logits_dev);
+    else
+        decode_impl<float>(h, tokens, B, pos, (float*)logits_dev);
+    CK(cudaGetLastError());
+    int rc = pending_error(h);
+    if (rc) return rc;
+    h->kv_len = pos + 1;
+    rc = read_scalars(h);
+    if (rc) return rc;
+    return status_error(h);
+}
+
+int gpt2_sample(gpt2_handle* h, const void* logits_dev, int B, float temperature, int top_k, const float* u_dev,
+                int32_t* next_dev) {
+    if (!h || !logits_dev || !u_dev || !next_dev) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    if (B < 1) return fail(GPT2_ERR_INVALID_ARG, "B must be >= 1");
+    int rc = check_sampling(temperature);
+    if (rc) return rc;
+    h->launches = 0;
+    if (h->bf16_mode)
+        sample_impl<bf16>(h, (const bf16*)logits_dev, B, temperature, top_k, u_dev, next_dev, nullptr, 0, 0);
+    else
+        sample_impl<float>(h, (const float*)logits_dev, B, temperature, top_k, u_dev, next_dev, nullptr, 0, 0);
+    CK(cudaGetLastError());
+    return GPT2_OK;
+}
+
+
+int gpt2_generate(gpt2_handle* h, const int32_t* prompt, int B, int T0, int max_new_tokens, float temperature,
+                  int top_k, const float* u_dev, int32_t* out_dev) {
+    if (!h || !prompt || !out_dev || (max_new_tokens > 0 && !u_dev))
+        return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    if (B < 1 || B > h->cfg.max_B) return fail(GPT2_ERR_INVALID_ARG, "B must be in [1, max_B]");
+    if (T0 < 1 || max_new_tokens < 0) return fail(GPT2_ERR_INVALID_ARG, "need T0 >= 1 and max_new_tokens >= 0");
+    int rc = check_sampling(temperature);
+    if (rc) return rc;
+    const int Tb = h->cfg.block_size;
+    if (std::min(T0, Tb) > h->cfg.max_T || (T0 + max_new_tokens - 1 > Tb && Tb > h->cfg.max_T))
+        return fail(GPT2_ERR_INVALID_ARG, "a prefill window (min(T0, block_size), or block_size once the "
+                                          "sequence outgrows it) exceeds max_T");
+    rc = ensure_gen(h);
+    if (rc) return rc;
+    h->launches = 0;
+    rc = h->bf16_mode ? generate_impl<bf16>(h, prompt, B, T0, max_new_tokens, temperature, top_k, u_dev, out_dev)
+                      : generate_impl<float>(h, prompt, B, T0, max_new_tokens, temperature, top_k, u_dev, out_dev);
+    if (rc) return rc;
+    rc = read_scalars(h);
+    if (rc) return rc;
+    if (h->profiling) prof_collect(h);
     return status_error(h);
 }
 

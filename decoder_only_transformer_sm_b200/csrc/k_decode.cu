@@ -1,0 +1,406 @@
+// Kernels of autoregressive generation ("GPT-2 from Scratch", "A generation
+// loop"): attention of the newest position against a key/value cache, the
+// sampling draw (temperature, top-k, one multinomial draw), and the row copies
+// that fill the cache and move token windows.
+//
+// Cache layout: per layer (B, Tc, 3C) rows [q | k | v] in the activation type,
+// row (b, j) at (b * Tc + j) * 3C, head h at columns h*hd of each C-wide block.
+// Rows 0 .. n-1 of a sequence are its positions 0 .. n-1; the decode step's
+// qkv GEMM writes row n-1 before the attention runs, and the attention reads q
+// from that row and k, v from rows 0 .. n-1.
+#include <climits>
+
+#include "kernels.cuh"
+
+namespace gpt2 {
+
+namespace {
+
+// 16 bytes of T unpacked to floats.
+template <typename T> struct V16;
+template <> struct V16<float> {
+    static constexpr int N = 4;
+    __device__ static void unpack(const uint4& q, float* f) {
+        f[0] = __uint_as_float(q.x); f[1] = __uint_as_float(q.y);
+        f[2] = __uint_as_float(q.z); f[3] = __uint_as_float(q.w);
+    }
+};
+template <> struct V16<bf16> {
+    static constexpr int N = 8;
+    __device__ static void unpack(const uint4& q, float* f) {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 t = __bfloat1622float2(h[i]);
+            f[2 * i] = t.x;
+            f[2 * i + 1] = t.y;
+        }
+    }
+};
+
+constexpr int DEC_THREADS = 128;
+constexpr int DEC_UNROLL = 4;
+
+// One block: keys [s*chunk, min(n, (s+1)*chunk)) of one (b, h). Groups of G
+// lanes own one key at a time, each lane 16 bytes of its head dims; a group
+// keeps an online softmax (running max m in log2 units, sum l, weighted sum of
+// v); the block merges its groups and writes (m, l, acc[HD]) to part.
+template <typename T, int HD>
+__global__ void __launch_bounds__(DEC_THREADS)
+    attn_decode_partial_kernel(const T* __restrict__ cache, int H, int C, int Tc, int n, int chunk, int S,
+                               float* __restrict__ part) {
+    constexpr int VE = V16<T>::N;
+    constexpr int G = HD / VE;                       // lanes per key
+    constexpr int KPW = 32 / G;                      // keys per warp per step
+    constexpr int NG = (DEC_THREADS / 32) * KPW;     // key groups per block
+    static_assert(G >= 1 && G <= 32 && 32 % G == 0, "head width and type give a bad lane split");
+    __shared__ float sm_m[NG], sm_l[NG];
+    __shared__ float sm_acc[NG][HD];
+
+    const int bh = blockIdx.x, s = blockIdx.y;
+    const int b = bh / H, h = bh % H;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int gw = lane / G, sub = lane % G;
+    const int grp = warp * KPW + gw;
+    const long long ld = 3LL * C;
+    const T* seq = cache + (long long)b * Tc * ld;
+
+    float q[VE];
+    {
+        const uint4 qv = *reinterpret_cast<const uint4*>(seq + (long long)(n - 1) * ld + h * HD + sub * VE);
+        V16<T>::unpack(qv, q);
+        const float sc = rsqrtf((float)HD) * 1.4426950408889634f;   // scores in log2 units
+#pragma unroll
+        for (int i = 0; i < VE; ++i) q[i] *= sc;
+    }
+    const int j0 = s * chunk, j1 = min(n, j0 + chunk);
+    float m = -INFINITY, l = 0.f, acc[VE];
+#pragma unroll
+    for (int i = 0; i < VE; ++i) acc[i] = 0.f;
+
+    // the trip count is the same for every lane of the block (shuffles below)
+    for (int jb = j0; jb < j1; jb += NG * DEC_UNROLL) {
+        uint4 kq[DEC_UNROLL], vq[DEC_UNROLL];
+#pragma unroll
+        for (int u = 0; u < DEC_UNROLL; ++u) {
+            const int j = jb + u * NG + grp;
+            kq[u] = make_uint4(0, 0, 0, 0);
+            vq[u] = make_uint4(0, 0, 0, 0);
+            if (j < j1) {
+                const T* r = seq + (long long)j * ld + h * HD + sub * VE;
+                kq[u] = *reinterpret_cast<const uint4*>(r + C);
+                vq[u] = *reinterpret_cast<const uint4*>(r + 2 * C);
+            }
+        }
+        float sc[DEC_UNROLL];
+#pragma unroll
+        for (int u = 0; u < DEC_UNROLL; ++u) {
+            float k[VE];
+            V16<T>::unpack(kq[u], k);
+            float d = 0.f;
+#pragma unroll
+            for (int i = 0; i < VE; ++i) d = fmaf(q[i], k[i], d);
+#pragma unroll
+            for (int o = G / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+            sc[u] = (jb + u * NG + grp < j1) ? d : -INFINITY;
+        }
+        float mx = m;
+#pragma unroll
+        for (int u = 0; u < DEC_UNROLL; ++u) mx = fmaxf(mx, sc[u]);
+        if (mx != -INFINITY) {   // same value on the G lanes of a group
+            const float corr = exp2f(m - mx);
+            l *= corr;
+#pragma unroll
+            for (int i = 0; i < VE; ++i) acc[i] *= corr;
+#pragma unroll
+            for (int u = 0; u < DEC_UNROLL; ++u) {
+                const float p = exp2f(sc[u] - mx);
+                float v[VE];
+                V16<T>::unpack(vq[u], v);
+                l += p;
+#pragma unroll
+                for (int i = 0; i < VE; ++i) acc[i] = fmaf(p, v[i], acc[i]);
+            }
+            m = mx;
+        }
+    }
+    if (sub == 0) {
+        sm_m[grp] = m;
+        sm_l[grp] = l;
+    }
+#pragma unroll
+    for (int i = 0; i < VE; ++i) sm_acc[grp][sub * VE + i] = acc[i];
+    __syncthreads();
+    if (threadIdx.x < HD) {
+        const int d = threadIdx.x;
+        float M = -INFINITY;
+        for (int g = 0; g < NG; ++g) M = fmaxf(M, sm_m[g]);
+        float L = 0.f, A = 0.f;   // M is finite: the block's key range is not empty
+        for (int g = 0; g < NG; ++g) {
+            const float w = exp2f(sm_m[g] - M);
+            L = fmaf(sm_l[g], w, L);
+            A = fmaf(sm_acc[g][d], w, A);
+        }
+        float* o = part + ((long long)bh * S + s) * (HD + 2);
+        o[2 + d] = A;
+        if (d == 0) {
+            o[0] = M;
+            o[1] = L;
+        }
+    }
+}
+
+// Merge the S partials of each (b, h): out = sum_s acc_s 2^(m_s - M) / sum_s l_s 2^(m_s - M).
+template <typename T, int HD>
+__global__ void attn_decode_combine_kernel(const float* __restrict__ part, int H, int C, int S, T* __restrict__ out) {
+    const int bh = blockIdx.x, d = threadIdx.x;
+    const int b = bh / H, h = bh % H;
+    const float* p = part + (long long)bh * S * (HD + 2);
+    float M = -INFINITY;
+    for (int s = 0; s < S; ++s) M = fmaxf(M, p[s * (HD + 2)]);
+    float L = 0.f, A = 0.f;
+    for (int s = 0; s < S; ++s) {
+        const float w = exp2f(p[s * (HD + 2)] - M);
+        L = fmaf(p[s * (HD + 2) + 1], w, L);
+        A = fmaf(p[s * (HD + 2) + 2 + d], w, A);
+    }
+    out[(long long)b * C + h * HD + d] = from_f<T>(A / L);
+}
+
+// ------------------------------------------------------------------ sampling
+constexpr int SMP_THREADS = 1024;
+
+// Unsigned key with the order of the float values (-0 taken as +0).
+__device__ __forceinline__ unsigned order_key(float f) {
+    if (f == 0.f) f = 0.f;
+    const unsigned u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// One block per row. 1) top_k in [1, V): the key of the k-th largest value by
+// a 4-pass radix select (8 bits a pass, high byte first); entries with a key
+// at or above it are kept (ties at the k-th value stay). 2) The row maximum.
+// 3) e_i = 2^((x_i - max) * log2(e) / temperature) over kept entries; thread t
+// owns the contiguous indices [t*per, (t+1)*per); a block scan of the
+// threads' sums gives each thread's starting cumulative value; the thread
+// whose range holds u * total walks it in order to the first index whose
+// cumulative value exceeds u * total. No thread claiming (rounding at the
+// ends) gives the last kept index.
+template <typename T>
+__global__ void __launch_bounds__(SMP_THREADS)
+    sample_kernel(const T* __restrict__ logits, long long ld, int V, float scale, int top_k,
+                  const float* __restrict__ u, int* __restrict__ next, int* __restrict__ out, long long out_ld,
+                  int out_col) {
+    __shared__ unsigned hist[256];
+    __shared__ unsigned s_prefix, s_krem;
+    __shared__ float s_wred[32];
+    __shared__ int s_wredi[32];
+    __shared__ float s_excl[SMP_THREADS + 1];
+    __shared__ int s_pick;
+    const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const T* x = logits + (long long)row * ld;
+
+    unsigned thr = 0;
+    if (top_k >= 1 && top_k < V) {
+        unsigned prefix = 0, mask = 0, krem = (unsigned)top_k;
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            for (int i = tid; i < 256; i += SMP_THREADS) hist[i] = 0;
+            __syncthreads();
+            for (int i = tid; i < V; i += SMP_THREADS) {
+                const unsigned k = order_key(to_f(x[i]));
+                if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+            }
+            __syncthreads();
+            if (tid == 0) {
+                unsigned cum = 0;
+                int d = 255;
+                for (; d > 0; --d) {
+                    if (cum + hist[d] >= krem) break;
+                    cum += hist[d];
+                }
+                s_prefix = prefix | ((unsigned)d << shift);
+                s_krem = krem - cum;
+            }
+            __syncthreads();
+            prefix = s_prefix;
+            krem = s_krem;
+            mask |= 0xFFu << shift;
+            __syncthreads();
+        }
+        thr = prefix;
+    }
+
+    // row maximum (always kept)
+    float mx = -INFINITY;
+    for (int i = tid; i < V; i += SMP_THREADS) mx = fmaxf(mx, to_f(x[i]));
+    mx = warp_max(mx);
+    if (lane == 0) s_wred[warp] = mx;
+    __syncthreads();
+    if (warp == 0) {
+        float v = s_wred[lane];
+        v = warp_max(v);
+        if (lane == 0) s_wred[0] = v;
+    }
+    __syncthreads();
+    mx = s_wred[0];
+    __syncthreads();
+
+    // per-thread sums over contiguous ranges
+    const int per = (V + SMP_THREADS - 1) / SMP_THREADS;
+    const int i0 = min(V, tid * per), i1 = min(V, i0 + per);
+    float local = 0.f;
+    int last_kept = -1;
+    for (int i = i0; i < i1; ++i) {
+        const float f = to_f(x[i]);
+        if (order_key(f) >= thr) {
+            local += exp2f((f - mx) * scale);
+            last_kept = i;
+        }
+    }
+    // exclusive scan of the thread sums
+    float incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) s_wred[warp] = incl;
+    int lk = last_kept;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lk = max(lk, __shfl_xor_sync(0xffffffffu, lk, o));
+    if (lane == 0) s_wredi[warp] = lk;
+    __syncthreads();
+    if (warp == 0) {
+        float w = s_wred[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float n = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += n;
+        }
+        s_wred[lane] = w;   // inclusive sums over warps
+        int k = s_wredi[lane];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) k = max(k, __shfl_xor_sync(0xffffffffu, k, o));
+        if (lane == 0) {
+            s_wredi[0] = k;
+            s_pick = INT_MAX;
+        }
+    }
+    __syncthreads();
+    const float woff = warp == 0 ? 0.f : s_wred[warp - 1];
+    const float prev = __shfl_up_sync(0xffffffffu, incl, 1);
+    s_excl[tid] = woff + (lane == 0 ? 0.f : prev);
+    if (tid == SMP_THREADS - 1) s_excl[SMP_THREADS] = s_wred[31];
+    __syncthreads();
+    const float total = s_excl[SMP_THREADS];
+    float uu = u[row];
+    if (!(uu >= 0.f)) uu = 0.f;
+    const float target = uu * total;
+    const float lo = s_excl[tid], hi = s_excl[tid + 1];
+    if (local > 0.f && lo <= target && target < hi) {
+        float run = lo;
+        int pick = last_kept;
+        for (int i = i0; i < i1; ++i) {
+            const float f = to_f(x[i]);
+            if (order_key(f) >= thr) {
+                run += exp2f((f - mx) * scale);
+                if (run > target) {
+                    pick = i;
+                    break;
+                }
+            }
+        }
+        atomicMin(&s_pick, pick);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        const int j = s_pick != INT_MAX ? s_pick : s_wredi[0];
+        next[row] = j;
+        if (out) out[(long long)row * out_ld + out_col] = j;
+    }
+}
+
+// ----------------------------------------------------------------- row copies
+// k and v columns [C, 3C) of qkv row (b*Tn + t) of layer l -> cache row (b, t).
+template <typename T>
+__global__ void kv_store_kernel(const void* const* __restrict__ src, void* const* __restrict__ dst, int Tn, int Tc,
+                                int C) {
+    const int r = blockIdx.x, l = blockIdx.y;
+    const int b = r / Tn, t = r % Tn;
+    const long long ld = 3LL * C;
+    const uint4* s = reinterpret_cast<const uint4*>(static_cast<const T*>(src[l]) + (long long)r * ld + C);
+    uint4* d = reinterpret_cast<uint4*>(static_cast<T*>(dst[l]) + ((long long)b * Tc + t) * ld + C);
+    const int n16 = (int)(2LL * C * sizeof(T) / 16);
+    for (int i = threadIdx.x; i < n16; i += blockDim.x) d[i] = s[i];
+}
+
+__global__ void copy_tokens_kernel(const int* __restrict__ src, long long src_ld, int* __restrict__ dst,
+                                   long long dst_ld, int cols) {
+    const long long r = blockIdx.x;
+    for (int c = threadIdx.x; c < cols; c += blockDim.x) dst[r * dst_ld + c] = src[r * src_ld + c];
+}
+
+}  // namespace
+
+void attention_decode_split(int BH, int n, int num_sms, int* splits, int* chunk) {
+    int want = ceil_div(2 * num_sms, BH);
+    if (want < 1) want = 1;
+    int s = min(want, ceil_div(n, DECODE_MIN_KEYS));
+    if (s < 1) s = 1;
+    const int c = ceil_div(n, s);
+    *chunk = c;
+    *splits = ceil_div(n, c);   // every split holds at least one key
+}
+
+template <typename T>
+void launch_attention_decode(const Ctx& ctx, const T* cache, T* out, float* part, int B, int H, int hd, int Tc,
+                             int n) {
+    int S = 1, chunk = n;
+    attention_decode_split(B * H, n, ctx.num_sms, &S, &chunk);
+    const int C = H * hd;
+    const dim3 grid(B * H, S);
+    if (hd == 64) {
+        attn_decode_partial_kernel<T, 64><<<grid, DEC_THREADS, 0, ctx.stream>>>(cache, H, C, Tc, n, chunk, S, part);
+        attn_decode_combine_kernel<T, 64><<<B * H, 64, 0, ctx.stream>>>(part, H, C, S, out);
+    } else {
+        attn_decode_partial_kernel<T, 32><<<grid, DEC_THREADS, 0, ctx.stream>>>(cache, H, C, Tc, n, chunk, S, part);
+        attn_decode_combine_kernel<T, 32><<<B * H, 32, 0, ctx.stream>>>(part, H, C, S, out);
+    }
+    *ctx.launches += 2;
+}
+
+template <typename T>
+void launch_sample(const Ctx& ctx, const T* logits, long long ld, int rows, int V, float temperature, int top_k,
+                   const float* u, int* next, int* out, long long out_ld, int out_col) {
+    const float scale = 1.4426950408889634f / temperature;
+    sample_kernel<T><<<rows, SMP_THREADS, 0, ctx.stream>>>(logits, ld, V, scale, top_k, u, next, out, out_ld,
+                                                          out_col);
+    ++*ctx.launches;
+}
+
+void launch_kv_store(const Ctx& ctx, const void* const* qkv_ptrs, void* const* cache_ptrs, int L, int B, int Tn,
+                     int Tc, int C, int elem_size) {
+    const dim3 grid(B * Tn, L);
+    if (elem_size == 2)
+        kv_store_kernel<bf16><<<grid, 128, 0, ctx.stream>>>(qkv_ptrs, cache_ptrs, Tn, Tc, C);
+    else
+        kv_store_kernel<float><<<grid, 128, 0, ctx.stream>>>(qkv_ptrs, cache_ptrs, Tn, Tc, C);
+    ++*ctx.launches;
+}
+
+void launch_copy_tokens(const Ctx& ctx, const int* src, long long src_ld, int* dst, long long dst_ld, int rows,
+                        int cols) {
+    if (rows < 1 || cols < 1) return;
+    copy_tokens_kernel<<<rows, 256, 0, ctx.stream>>>(src, src_ld, dst, dst_ld, cols);
+    ++*ctx.launches;
+}
+
+#define INST(T)                                                                                                 \
+    template void launch_attention_decode<T>(const Ctx&, const T*, T*, float*, int, int, int, int, int);        \
+    template void launch_sample<T>(const Ctx&, const T*, long long, int, int, float, int, const float*, int*,   \
+                                   int*, long long, int);
+INST(float)
+INST(bf16)
+#undef INST
+
+}  // namespace gpt2

@@ -132,3 +132,40 @@ extern "C" int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, 
     if (err != cudaSuccess) return set_error(GPT2_ERR_CUDA, cudaGetErrorString(err));
     return GPT2_OK;
 }
+
+extern "C" int gpt2k_attention_decode(int dtype, const void* cache, void* out, int B, int H, int hd, int Tc, int n,
+                                      float* workspace_dev, uint32_t* status_dev, void* stream) {
+    if (dtype != GPT2K_F32 && dtype != GPT2K_BF16) return set_error(GPT2_ERR_INVALID_ARG, "unknown dtype");
+    if (B < 1 || H < 1 || Tc < 1 || n < 1 || n > Tc)
+        return set_error(GPT2_ERR_INVALID_ARG, "need B, H >= 1 and 1 <= n <= Tc");
+    if (hd != 32 && hd != 64) return set_error(GPT2_ERR_INVALID_ARG, "head width must be 32 or 64");
+    if ((H * hd) % 64 != 0) return set_error(GPT2_ERR_INVALID_ARG, "C = H * hd must be a multiple of 64");
+    if (!cache || !out || !workspace_dev || !status_dev) return set_error(GPT2_ERR_INVALID_ARG, "NULL operand");
+    long long launches = 0;
+    Ctx c = kctx(stream, status_dev, &launches);
+    if (dtype == GPT2K_F32)
+        launch_attention_decode<float>(c, (const float*)cache, (float*)out, workspace_dev, B, H, hd, Tc, n);
+    else
+        launch_attention_decode<bf16>(c, (const bf16*)cache, (bf16*)out, workspace_dev, B, H, hd, Tc, n);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return set_error(GPT2_ERR_CUDA, cudaGetErrorString(err));
+    return GPT2_OK;
+}
+
+extern "C" int gpt2k_sample(int dtype, const void* logits, int rows, int V, int64_t ld, float temperature,
+                            int top_k, const float* u_dev, int32_t* next_dev, uint32_t* status_dev, void* stream) {
+    if (dtype != GPT2K_F32 && dtype != GPT2K_BF16) return set_error(GPT2_ERR_INVALID_ARG, "unknown dtype");
+    if (rows < 1 || V < 1 || ld < V) return set_error(GPT2_ERR_INVALID_ARG, "need rows, V >= 1 and ld >= V");
+    if (!logits || !u_dev || !next_dev || !status_dev) return set_error(GPT2_ERR_INVALID_ARG, "NULL operand");
+    if (!(temperature > 0.f) || !(temperature < INFINITY))
+        return set_error(GPT2_ERR_INVALID_ARG, "temperature must be finite and > 0");
+    long long launches = 0;
+    Ctx c = kctx(stream, status_dev, &launches);
+    if (dtype == GPT2K_F32)
+        launch_sample<float>(c, (const float*)logits, ld, rows, V, temperature, top_k, u_dev, next_dev, nullptr, 0, 0);
+    else
+        launch_sample<bf16>(c, (const bf16*)logits, ld, rows, V, temperature, top_k, u_dev, next_dev, nullptr, 0, 0);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return set_error(GPT2_ERR_CUDA, cudaGetErrorString(err));
+    return GPT2_OK;
+}

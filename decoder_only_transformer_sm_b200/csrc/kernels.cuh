@@ -134,6 +134,36 @@ void launch_attention_bwd_pre(const Ctx& ctx, const bf16* out, const bf16* dout,
                               int hd);
 
 // ----------------------------------------------------------------------------
+// Generation (k_decode.cu): key/value cache rows (B, Tc, 3C) [q | k | v] per layer.
+// ----------------------------------------------------------------------------
+// Attention of the newest position n-1 of each sequence against cache rows
+// 0 .. n-1 (q from row n-1), heads concatenated into out (B, C). The keys are
+// split over `splits` blocks per (b, h) of at least DECODE_MIN_KEYS keys each
+// (fewer only when n is smaller); part holds the blocks' partial softmax sums,
+// decode_part_floats(B*H, Tc, hd) floats at most.
+constexpr int DECODE_MIN_KEYS = 64;
+inline long long decode_part_floats(int BH, int Tc, int hd) {
+    return (long long)BH * ceil_div(Tc, DECODE_MIN_KEYS) * (hd + 2);
+}
+void attention_decode_split(int BH, int n, int num_sms, int* splits, int* chunk);
+template <typename T>
+void launch_attention_decode(const Ctx& ctx, const T* cache, T* out, float* part, int B, int H, int hd, int Tc,
+                             int n);
+// One draw per row of logits (row stride ld): temperature, top-k (top_k <= 0
+// or >= V keeps every entry), inverse CDF at u[row] in vocabulary order.
+// next[row] = the drawn index; if out != null also out[row * out_ld + out_col].
+template <typename T>
+void launch_sample(const Ctx& ctx, const T* logits, long long ld, int rows, int V, float temperature, int top_k,
+                   const float* u, int* next, int* out, long long out_ld, int out_col);
+// k, v columns of qkv rows (b * Tn + t) of every layer -> cache rows (b, t).
+// qkv_ptrs, cache_ptrs: device arrays of L pointers.
+void launch_kv_store(const Ctx& ctx, const void* const* qkv_ptrs, void* const* cache_ptrs, int L, int B, int Tn,
+                     int Tc, int C, int elem_size);
+// dst[r * dst_ld + c] = src[r * src_ld + c] for r < rows, c < cols (int32 tokens).
+void launch_copy_tokens(const Ctx& ctx, const int* src, long long src_ld, int* dst, long long dst_ld, int rows,
+                        int cols);
+
+// ----------------------------------------------------------------------------
 // Optimiser and parameter utilities.
 // ----------------------------------------------------------------------------
 struct AdamChunk {        // a run of elements inside one tensor

@@ -77,6 +77,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gpt2_set_opt_state": (I, [P, P, P, ctypes.c_int64, I]),
         "gpt2_forward": (I, [P, P, P, I, I, P, ctypes.POINTER(F)]),
         "gpt2_forward_last": (I, [P, P, I, I, P]),
+        "gpt2_prefill": (I, [P, P, I, I, P]),
+        "gpt2_decode": (I, [P, P, I, I, P]),
+        "gpt2_sample": (I, [P, P, I, F, I, P, P]),
+        "gpt2_generate": (I, [P, P, I, I, I, F, I, P, P]),
         "gpt2_lr_at": (I, [ctypes.c_int64, F, F, ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(F)]),
         "gpt2_zero_grad": (I, [P]),
         "gpt2_accumulate": (I, [P, P, P, I, I, F]),
@@ -89,6 +93,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gpt2k_matmul_bf16": (I, [I, P, P, I, I, I, I, P, ctypes.c_int64, P, P, P, P, P, F, I, P, P]),
         "gpt2k_attention_fwd": (I, [I, P, P, P, I, I, I, I, I, P, P]),
         "gpt2k_attention_bwd": (I, [I, P, P, P, P, P, I, I, I, I, P, P, I, P, P]),
+        "gpt2k_attention_decode": (I, [I, P, P, I, I, I, I, I, P, P, P]),
+        "gpt2k_sample": (I, [I, P, I, I, ctypes.c_int64, F, I, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -200,6 +206,27 @@ class GPT2:
         """Logits (B, vocab_size) of each sequence's last position (gpt2_forward_last)."""
         B, T = idx.shape
         _check(self._lib.gpt2_forward_last(self._h, _ptr(idx), B, T, _ptr(logits)))
+
+    # ---- generation (device tensors; "A generation loop") ----
+    def prefill(self, idx, logits):
+        """gpt2_prefill: last-position logits (B, vocab_size) and the k/v cache of idx (B, T)."""
+        B, T = idx.shape
+        _check(self._lib.gpt2_prefill(self._h, _ptr(idx), B, T, _ptr(logits)))
+
+    def decode(self, tokens, pos: int, logits):
+        """gpt2_decode: tokens (B,) at position pos against the cache; logits (B, vocab_size)."""
+        _check(self._lib.gpt2_decode(self._h, _ptr(tokens), tokens.shape[0], pos, _ptr(logits)))
+
+    def sample(self, logits, temperature: float, top_k: int, u, next_tokens):
+        """gpt2_sample: one draw per row of logits (B, vocab_size) at the uniforms u (B,)."""
+        _check(self._lib.gpt2_sample(self._h, _ptr(logits), logits.shape[0], temperature, top_k, _ptr(u),
+                                     _ptr(next_tokens)))
+
+    def generate(self, prompt, max_new_tokens: int, temperature: float, top_k: int, u, out):
+        """gpt2_generate: out (B, T0 + max_new_tokens) = prompt (B, T0) + drawn tokens; u (max_new_tokens, B)."""
+        B, T0 = prompt.shape
+        _check(self._lib.gpt2_generate(self._h, _ptr(prompt), B, T0, max_new_tokens, temperature, top_k, _ptr(u),
+                                       _ptr(out)))
 
     def zero_grad(self):
         _check(self._lib.gpt2_zero_grad(self._h))
@@ -322,4 +349,23 @@ def attention_bwd_noalloc(qkv, out, dout, lse, dqkv, B: int, T: int, H: int, hd:
     status, stream = _stream_and_status(qkv, status, stream)
     _check(fn(_dtype_code(qkv), _ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dqkv), B, T, H, hd, engine,
               _ptr(status), stream))
+    return status
+
+
+def attention_decode(cache, out, B: int, H: int, hd: int, Tc: int, n: int, workspace, status=None, stream=None):
+    """gpt2k_attention_decode: the newest position n-1 of each sequence against cache
+    (B, Tc, 3C); workspace: B*H*ceil(Tc/64)*(hd+2) float32."""
+    status, stream = _stream_and_status(cache, status, stream)
+    _check(load_library().gpt2k_attention_decode(_dtype_code(cache), _ptr(cache), _ptr(out), B, H, hd, Tc, n,
+                                                 _ptr(workspace), _ptr(status), stream))
+    return status
+
+
+def sample(logits, V: int, temperature: float, top_k: int, u, next_tokens, ld: int | None = None, status=None,
+           stream=None):
+    """gpt2k_sample on rows of logits (rows, ld) (first V columns); next_tokens (rows,) int32."""
+    status, stream = _stream_and_status(logits, status, stream)
+    rows = logits.shape[0]
+    _check(load_library().gpt2k_sample(_dtype_code(logits), _ptr(logits), rows, V, ld if ld is not None else V,
+                                       temperature, top_k, _ptr(u), _ptr(next_tokens), _ptr(status), stream))
     return status

@@ -164,6 +164,64 @@ int gpt2_forward(gpt2_handle* h, const int32_t* idx_dev, const int32_t* targets_
  * outside [0, vocab_size). */
 int gpt2_forward_last(gpt2_handle* h, const int32_t* idx_dev, int B, int T, void* logits_dev);
 
+/* ---- Generation ("GPT-2 from Scratch", "A generation loop") ----------------
+ * The pages' loop recomputes the whole (cropped) sequence for every new token;
+ * these calls keep each layer's k and v rows in a key/value cache instead, so
+ * a new token costs one position's forward plus attention over the cached
+ * rows. The results are those of the full recompute (up to rounding). The
+ * cache (per layer max_B x block_size rows of 3 * n_embd elements, in the
+ * precision mode's type) is allocated by the first generation call and freed
+ * by gpt2_destroy. The calls reuse the handle's activation buffers: call them
+ * between training calls, not between gpt2_accumulate and gpt2_update. */
+
+/* Forward of (B, T) tokens as gpt2_forward_last (logits (B, vocab_size) of the
+ * last positions into logits_dev), then every layer's k and v of positions
+ * 0 .. T-1 into cache rows 0 .. T-1 of sequences 0 .. B-1.
+ * Synchronises once at the end. Errors: as gpt2_forward_last; OOM if the cache
+ * cannot be allocated. */
+int gpt2_prefill(gpt2_handle* h, const int32_t* idx_dev, int B, int T, void* logits_dev);
+
+/* One new position: tokens_dev (B) int32 on the device are the tokens at
+ * position pos of sequences 0 .. B-1, whose cache rows 0 .. pos-1 hold the
+ * earlier positions (a gpt2_prefill of length pos, or a prefill followed by
+ * decodes at the positions up to pos - 1). Runs the blocks on the B rows at
+ * position pos, writes their k and v to cache row pos, attends over rows
+ * 0 .. pos, and writes the logits (B, vocab_size) (fp32 or bf16 by mode) to
+ * logits_dev. Afterwards the cache holds pos + 1 positions.
+ * Synchronises once at the end. Errors: INVALID_ARG (no prefill yet, B above
+ * the last prefill's B, pos < 1, pos above the cached length, or pos >=
+ * block_size); BAD_TOKEN for an id outside [0, vocab_size). */
+int gpt2_decode(gpt2_handle* h, const int32_t* tokens_dev, int B, int pos, void* logits_dev);
+
+/* One draw per row of logits_dev (B, vocab_size) (fp32 or bf16 by mode, rows
+ * contiguous): the row divided by temperature; with 1 <= top_k < vocab_size,
+ * entries below the top_k-th largest dropped (entries equal to it kept;
+ * top_k <= 0 or >= vocab_size keeps all); softmax; the index drawn is the
+ * first, in vocabulary order, whose cumulative probability exceeds u_dev[b]
+ * (inverse CDF: u_dev holds B uniforms in [0, 1) drawn by the caller; a value
+ * below 0 counts as 0, one at or above the last cumulative value gives the
+ * last kept index). next_dev (B) int32 receives the indices.
+ * Asynchronous. Errors: INVALID_ARG (NULL pointer, B < 1, temperature not
+ * finite and > 0). The logits must be finite. */
+int gpt2_sample(gpt2_handle* h, const void* logits_dev, int B, float temperature, int top_k,
+                const float* u_dev, int32_t* next_dev);
+
+/* The pages' generation loop on the device: out_dev (B, T0 + max_new_tokens)
+ * int32 receives the prompt (prompt_dev (B, T0) int32) followed by
+ * max_new_tokens drawn tokens. Draw s (0-based) sees the n = T0 + s tokens
+ * so far: while n <= block_size the first draw runs gpt2_prefill on them and
+ * later draws run gpt2_decode at position n - 1; once n > block_size each
+ * draw runs gpt2_prefill on the last block_size tokens (the pages' crop, which
+ * shifts every position, so the cache cannot be reused). Each draw is
+ * gpt2_sample with u = u_dev[s * B + b] (u_dev: (max_new_tokens, B) floats in
+ * [0, 1)). Synchronises once at the end.
+ * Errors: INVALID_ARG (NULL pointer, B outside [1, max_B], T0 < 1,
+ * max_new_tokens < 0, a bad temperature, or a prefill window longer than
+ * max_T: min(T0, block_size), or block_size when the sequence outgrows it);
+ * OOM for the cache; BAD_TOKEN for a prompt id outside [0, vocab_size). */
+int gpt2_generate(gpt2_handle* h, const int32_t* prompt_dev, int B, int T0, int max_new_tokens,
+                  float temperature, int top_k, const float* u_dev, int32_t* out_dev);
+
 /* Set every gradient to zero and clear the accumulated loss. Asynchronous. */
 int gpt2_zero_grad(gpt2_handle* h);
 

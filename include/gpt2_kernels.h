@@ -115,6 +115,28 @@ int gpt2k_attention_bwd_noalloc(int dtype, const void* qkv, const void* out, con
                                 void* dqkv, int B, int T, int H, int hd, int engine, uint32_t* status_dev,
                                 void* stream);
 
+/* Attention of the newest position of each sequence against a key/value cache
+ * ("GPT-2 from Scratch", "A generation loop" and "CausalSelfAttention": the
+ * last row of causal attention, which sees every earlier position).
+ * cache : (B, Tc, 3C) rows [q | k | v], C = H * hd, in dtype; row (b, j) is
+ *         position j of sequence b. q is read from row n - 1, k and v from
+ *         rows 0 .. n - 1 (1 <= n <= Tc).
+ * out   : (B, C) in dtype, heads concatenated in head order.
+ * workspace_dev: caller-owned scratch of B * H * ceil(Tc / 64) * (hd + 2)
+ *         floats (the key range is split over blocks of at least 64 keys).
+ * hd must be 32 or 64, C a multiple of 64. fp32 arithmetic. */
+int gpt2k_attention_decode(int dtype, const void* cache, void* out, int B, int H, int hd, int Tc, int n,
+                           float* workspace_dev, uint32_t* status_dev, void* stream);
+
+/* Next-token draw on rows of logits ("GPT-2 from Scratch", "A generation
+ * loop"): row r is logits[r * ld .. r * ld + V - 1] in dtype; the draw is that
+ * of gpt2_sample (temperature, top-k with ties at the k-th value kept, softmax,
+ * inverse CDF at u_dev[r] in vocabulary order). next_dev (rows) int32 receives
+ * the indices. Errors: INVALID_ARG (unknown dtype, rows or V < 1, ld < V, a
+ * NULL pointer, temperature not finite and > 0). */
+int gpt2k_sample(int dtype, const void* logits, int rows, int V, int64_t ld, float temperature, int top_k,
+                 const float* u_dev, int32_t* next_dev, uint32_t* status_dev, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -87,3 +87,25 @@ def test_lr_schedule_entry_matches_oracle():
     for bad in [(-1, mx, mn, tw, tm), (0, mx, mn, 0, tm), (0, mx, mn, tw, tw - 1)]:
         with pytest.raises(native.Gpt2Error):
             native.lr_at(*bad)
+
+
+def test_generation_entries_reject_bad_arguments_on_host():
+    """The generation entry points validate their arguments before any CUDA
+    call (no GPU needed): NULL handles and pointers, bad sizes, a temperature
+    that is not finite and > 0, a row stride below V, n outside [1, Tc]."""
+    lib = native.load_library()
+    dummy = ctypes.c_void_p(16)   # never dereferenced: validation fails first
+    assert lib.gpt2_prefill(None, dummy, 1, 1, dummy) == -1
+    assert lib.gpt2_decode(None, dummy, 1, 1, dummy) == -1
+    assert lib.gpt2_sample(None, dummy, 1, 1.0, 0, dummy, dummy) == -1
+    assert lib.gpt2_generate(None, dummy, 1, 1, 1, 1.0, 0, dummy, dummy) == -1
+    ok = (1, dummy, 4, 8, 8, 1.0, 0, dummy, dummy, dummy, None)
+    for i, bad in [(0, 7), (2, 0), (3, 0), (4, 7), (5, 0.0), (5, float("nan")), (5, float("inf")), (7, None)]:
+        args = list(ok)
+        args[i] = bad
+        assert lib.gpt2k_sample(*args) == -1, (i, bad)
+    okd = (1, dummy, dummy, 2, 4, 64, 100, 100, dummy, dummy, None)
+    for i, bad in [(0, 3), (3, 0), (5, 48), (6, 0), (7, 0), (7, 101), (8, None)]:
+        args = list(okd)
+        args[i] = bad
+        assert lib.gpt2k_attention_decode(*args) == -1, (i, bad)
