@@ -68,6 +68,18 @@ def flops_per_token(w) -> float:
     return 6.0 * n_params_padded(w) + 12.0 * w["n_layer"] * w["n_embd"] * w["T"]
 
 
+def exact_step_flops(w, B: int, T: int) -> float:
+    """FLOPs one training step performs, with attention counted over the causal
+    triangle only: every Linear layer's forward, input-gradient and weight-gradient
+    GEMMs (3 x 2 M N K), attention forward 2 B H T (T+1) hd (QK^T and PV) and
+    backward 5 B H T (T+1) hd (S recomputed, dV, dP, dQ, dK) per layer."""
+    C, L, V, H = w["n_embd"], w["n_layer"], w["vocab_size"], w["n_head"]
+    BT, hd = B * T, C // H
+    gemm_fwd = L * 2.0 * BT * (3 * C * C + C * C + 4 * C * C + 4 * C * C) + 2.0 * BT * C * V
+    attn = L * 7.0 * B * H * T * (T + 1) * hd
+    return 3.0 * gemm_fwd + attn
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -544,7 +556,9 @@ def run_ours(args):
         "config": workload_config(B, T, world, w),
         "mfu": {"flops_per_token": fpt, "vs_nominal_2250": value * fpt / world / (NOMINAL_BF16_TFLOPS * 1e12),
                 "vs_measured_sustained": value * fpt / world / (peaks.get("bf16_tflops_sustained", 1400.0) * 1e12),
-                "peak_source": peak_src},
+                "peak_source": peak_src,
+                "exact_causal_flops_per_step": exact_step_flops(w, B, T),
+                "exact_causal_tflops_per_gpu": exact_step_flops(w, B, T) / (ms / 1e3) / 1e12},
         "roofline": {"kernel": dom["name"], "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak if peak else None, "traffic": traffic_for(dom["name"]),
                      "per_launch_ms": per_launch_ms, "peak_note": peak_note},

@@ -1,8 +1,8 @@
 /*
  * gpt2_kernels.h -- kernel-level C ABI of libgpt2_b200.so.
  *
- * Single operations of the training step, exposed for unit tests and for
- * callers that assemble their own step. All pointers are CUDA device pointers
+ * Single operations of the training step and of generation, exposed for unit
+ * tests and for callers that assemble their own step. All pointers are CUDA device pointers
  * owned by the caller; every call enqueues on `stream` (a cudaStream_t, NULL =
  * legacy default stream) and returns without synchronising. `status_dev`
  * points to one caller-owned device uint32 that kernels OR error bits into

@@ -47,3 +47,17 @@ def test_workload_config_and_metric_names():
     assert bench.metric_for(bench.MODELS["xl"], 4, 1024) != bench.METRIC
     # 6N + 12 L C T with the tied wte counted once at the padded vocabulary
     assert bench.flops_per_token(w) == pytest.approx(8.601e8, rel=1e-3)
+
+
+def test_exact_causal_flop_count():
+    """The exact causal count of one 124M step: 3 x the forward GEMMs plus 3.5 x
+    the causal attention forward, written out per term and against the ~1.32e13
+    of the hot-path scope table."""
+    w = bench.MODELS["124m"]
+    B, T, C, L, V, H = 16, 1024, 768, 12, 50304, 12
+    gemm = 3 * (L * 2 * B * T * 12 * C * C + 2 * B * T * C * V)
+    attn = L * (2 + 5) * B * H * T * (T + 1) * (C // H)
+    assert bench.exact_step_flops(w, B, T) == pytest.approx(gemm + attn, rel=1e-12)
+    assert bench.exact_step_flops(w, B, T) == pytest.approx(1.32e13, rel=5e-3)
+    # the 6N + 12 L C T convention counts more: non-causal attention and the embeddings' 6N share
+    assert bench.flops_per_token(w) * B * T > bench.exact_step_flops(w, B, T)
