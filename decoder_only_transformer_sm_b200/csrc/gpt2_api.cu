@@ -1049,6 +1049,13 @@ int gpt2_get_grads(gpt2_handle* h, float* flat, int on_device) {
     return copy_flat(h, flat, h->grads, h->n_params * 4, false, on_device);
 }
 
+int gpt2_grads_device(gpt2_handle* h, float** grads_dev, int64_t* n) {
+    if (!h || !grads_dev || !n) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    *grads_dev = h->grads;
+    *n = h->n_params;
+    return GPT2_OK;
+}
+
 int gpt2_get_opt_state(gpt2_handle* h, float* m, float* v, int64_t* step, int on_device) {
     if (!h) return fail(GPT2_ERR_INVALID_ARG, "NULL handle");
     int rc = GPT2_OK;

@@ -73,6 +73,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gpt2_set_params": (I, [P, P, I]),
         "gpt2_get_params": (I, [P, P, I]),
         "gpt2_get_grads": (I, [P, P, I]),
+        "gpt2_grads_device": (I, [P, ctypes.POINTER(P), ctypes.POINTER(ctypes.c_int64)]),
         "gpt2_get_opt_state": (I, [P, P, P, ctypes.POINTER(ctypes.c_int64), I]),
         "gpt2_set_opt_state": (I, [P, P, P, ctypes.c_int64, I]),
         "gpt2_forward": (I, [P, P, P, I, I, P, ctypes.POINTER(F)]),
@@ -118,6 +119,15 @@ def _ptr(x) -> int | None:
         return x.ctypes.data
     assert x.is_contiguous()
     return x.data_ptr()
+
+
+class _DeviceArray:
+    """A device float32 vector the library owns, described by the CUDA array
+    interface so that torch.as_tensor can wrap it without a copy."""
+
+    def __init__(self, ptr: int, n: int):
+        self.__cuda_array_interface__ = {"shape": (n,), "typestr": "<f4", "data": (ptr, False), "version": 3,
+                                         "strides": None}
 
 
 class GPT2:
@@ -181,6 +191,14 @@ class GPT2:
         out = np.empty(self.n_params, np.float32)
         _check(self._lib.gpt2_get_grads(self._h, _ptr(out), 0))
         return out
+
+    def grads_view(self):
+        """The handle's gradient vector as a torch float32 CUDA tensor sharing its
+        memory (gpt2_grads_device; no copy), for in-place collectives."""
+        import torch
+        ptr, n = ctypes.c_void_p(), ctypes.c_int64()
+        _check(self._lib.gpt2_grads_device(self._h, ctypes.byref(ptr), ctypes.byref(n)))
+        return torch.as_tensor(_DeviceArray(ptr.value, n.value), device="cuda")
 
     def get_opt_state(self):
         m = np.empty(self.n_params, np.float32)

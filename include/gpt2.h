@@ -4,7 +4,9 @@
  * One handle owns one GPT-2 model on one CUDA device: fp32 master weights,
  * fp32 gradients, fp32 AdamW moments, a bf16 copy of the weights (bf16 mode),
  * every saved activation and all workspace. All memory is allocated in
- * gpt2_create and released in gpt2_destroy; no other call allocates.
+ * gpt2_create and released in gpt2_destroy; the one other call that allocates
+ * is the first generation call on a handle (gpt2_prefill or gpt2_generate),
+ * which allocates the key/value cache.
  *
  * What a step computes (page title, section of the source pages):
  *   forward      "GPT-2 from Scratch": "Embeddings: tokens and positions",
@@ -24,6 +26,10 @@
  *                "Gradient accumulation, and the bug in getting it right":
  *                each micro-batch's mean loss is multiplied by loss_scale
  *                (1/n_micro) before its gradient is added.
+ *   generation   "A generation loop": temperature, top-k, one multinomial
+ *                draw per new token, the context cropped to block_size; here
+ *                on a key/value cache (gpt2_prefill, gpt2_decode, gpt2_sample,
+ *                gpt2_generate).
  *
  * Conventions
  *   * Every function returns GPT2_OK (0) or a negative GPT2_ERR_* code;
@@ -135,6 +141,15 @@ int gpt2_set_params(gpt2_handle* h, const float* flat, int on_device);
 int gpt2_get_params(gpt2_handle* h, float* flat, int on_device);
 /* Accumulated fp32 gradients (after the last accumulate/step, before clipping). */
 int gpt2_get_grads(gpt2_handle* h, float* flat, int on_device);
+/* The handle's own flat fp32 gradient vector, in place: *grads_dev receives its
+ * device address (n_params floats in gpt2_param_layout order, *n receives
+ * n_params). The handle owns it until gpt2_destroy. Work on it must be ordered
+ * with the handle's stream. Data parallelism uses it ("Let's reproduce GPT-2
+ * (124M)", "Scaling to 8 GPUs with DistributedDataParallel"): between the
+ * last gpt2_accumulate and gpt2_update, the ranks all-reduce (sum) this buffer
+ * in place, each rank having scaled its losses by 1/world, so that every rank
+ * clips and updates with the average gradient. Errors: INVALID_ARG (NULL). */
+int gpt2_grads_device(gpt2_handle* h, float** grads_dev, int64_t* n);
 /* AdamW state: first and second moments (n_params floats each) and the step count. */
 int gpt2_get_opt_state(gpt2_handle* h, float* m, float* v, int64_t* step, int on_device);
 int gpt2_set_opt_state(gpt2_handle* h, const float* m, const float* v, int64_t step, int on_device);
