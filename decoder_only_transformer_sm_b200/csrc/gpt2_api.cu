@@ -603,24 +603,36 @@ int ensure_gen(gpt2_handle* h) {
         cudaGetLastError();
         return fail(GPT2_ERR_OOM, "cudaMalloc of the key/value cache failed");
     }
-    h->gen_pool = pool;
-    h->kv.assign(L, nullptr);
+    std::vector<void*> kv(L, nullptr);
     size_t off = 0;
-    for (size_t l = 0; l < L; ++l, off += layer) h->kv[l] = pool + off;
-    h->dec_part = (float*)(pool + off);
+    for (size_t l = 0; l < L; ++l, off += layer) kv[l] = pool + off;
+    float* dec_part = (float*)(pool + off);
     off += part;
-    h->d_layer_ptrs = (void**)(pool + off);
+    void** layer_ptrs = (void**)(pool + off);
     off += ptrs;
-    h->d_next = (int*)(pool + off);
+    int* d_next = (int*)(pool + off);
     off += next;
-    h->d_window = (int*)(pool + off);
+    int* d_window = (int*)(pool + off);
     std::vector<void*> tab(2 * L);
     for (size_t l = 0; l < L; ++l) {
         tab[l] = h->qkv[l];
-        tab[L + l] = h->kv[l];
+        tab[L + l] = kv[l];
     }
-    CK(cudaMemcpyAsync(h->d_layer_ptrs, tab.data(), tab.size() * sizeof(void*), cudaMemcpyHostToDevice, h->stream));
-    CK(cudaStreamSynchronize(h->stream));
+    // the handle takes the pool only once the pointer table is on the device
+    cudaError_t e = cudaMemcpyAsync(layer_ptrs, tab.data(), tab.size() * sizeof(void*), cudaMemcpyHostToDevice,
+                                    h->stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(h->stream);
+    if (e != cudaSuccess) {
+        cudaFree(pool);
+        return fail(GPT2_ERR_CUDA, std::string("key/value cache setup: ") + cudaGetErrorString(e));
+    }
+    h->gen_pool = pool;
+    h->kv = kv;
+    h->dec_part = dec_part;
+    h->d_layer_ptrs = layer_ptrs;
+    h->d_next = d_next;
+    h->d_window = d_window;
+    h->kv_B = h->kv_len = 0;
     return GPT2_OK;
 }
 
@@ -807,6 +819,7 @@ int update_impl(gpt2_handle* h, float lr, float* loss_host, float* norm_host) {
     if (!std::isfinite(loss) || !std::isfinite(ss))
         return fail(GPT2_ERR_NONFINITE, "loss or gradient norm is not finite; update skipped");
     h->step_t = t;
+    h->kv_len = 0;   // the cached k, v belong to the old weights
     return GPT2_OK;
 }
 
@@ -1030,6 +1043,7 @@ static int copy_flat(gpt2_handle* h, void* dst, const void* src, size_t bytes, b
 
 int gpt2_set_params(gpt2_handle* h, const float* flat, int on_device) {
     if (!h || !flat) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    h->kv_len = 0;   // the cached k, v belong to the old weights
     int rc = copy_flat(h, h->params, flat, h->n_params * 4, true, on_device);
     if (rc) return rc;
     h->launches = 0;

@@ -187,7 +187,9 @@ int gpt2_forward_last(gpt2_handle* h, const int32_t* idx_dev, int B, int T, void
  * cache (per layer max_B x block_size rows of 3 * n_embd elements, in the
  * precision mode's type) is allocated by the first generation call and freed
  * by gpt2_destroy. The calls reuse the handle's activation buffers: call them
- * between training calls, not between gpt2_accumulate and gpt2_update. */
+ * between training calls, not between gpt2_accumulate and gpt2_update. A
+ * weight change (gpt2_update, gpt2_step, gpt2_step_host, gpt2_set_params)
+ * empties the cache: gpt2_decode then needs a new gpt2_prefill. */
 
 /* Forward of (B, T) tokens as gpt2_forward_last (logits (B, vocab_size) of the
  * last positions into logits_dev), then every layer's k and v of positions
