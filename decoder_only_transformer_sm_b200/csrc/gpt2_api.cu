@@ -1070,6 +1070,47 @@ int gpt2_grads_device(gpt2_handle* h, float** grads_dev, int64_t* n) {
     return GPT2_OK;
 }
 
+int gpt2_debug_activation(gpt2_handle* h, int kind, int index, int B, int T, float* out_host) {
+    if (!h || !out_host) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    int rc = check_bt(h, B, T);
+    if (rc) return rc;
+    const int L = h->L;
+    const size_t C = h->C;
+    const void* src = nullptr;
+    size_t width = C;
+    bool fp32 = !h->bf16_mode;
+    auto in = [&](int lo, int hi) { return index >= lo && index <= hi; };
+    switch (kind) {
+    case GPT2_ACT_RESID:
+        if (!in(0, 2 * L)) break;
+        src = h->resid[index];
+        fp32 = true;
+        break;
+    case GPT2_ACT_LN1: if (in(0, L - 1)) src = h->ln1[index]; break;
+    case GPT2_ACT_QKV: if (in(0, L - 1)) { src = h->qkv[index]; width = 3 * C; } break;
+    case GPT2_ACT_ATTN: if (in(0, L - 1)) src = h->att[index]; break;
+    case GPT2_ACT_LN2: if (in(0, L - 1)) src = h->ln2[index]; break;
+    case GPT2_ACT_GELU: if (in(0, L - 1)) { src = h->fcg[index]; width = 4 * C; } break;
+    case GPT2_ACT_LNF: if (index == 0) src = h->lnf; break;
+    default: break;
+    }
+    if (!src) return fail(GPT2_ERR_INVALID_ARG, "unknown activation kind or index out of range");
+    const size_t n = (size_t)B * T * width;
+    if (fp32) {
+        CK(cudaMemcpyAsync(out_host, src, n * 4, cudaMemcpyDeviceToHost, h->stream));
+        CK(cudaStreamSynchronize(h->stream));
+        return GPT2_OK;
+    }
+    std::vector<uint16_t> bits(n);
+    CK(cudaMemcpyAsync(bits.data(), src, n * 2, cudaMemcpyDeviceToHost, h->stream));
+    CK(cudaStreamSynchronize(h->stream));
+    for (size_t i = 0; i < n; ++i) {   // bf16 -> fp32 is exact: the bf16 bits are the high half
+        const uint32_t w = (uint32_t)bits[i] << 16;
+        memcpy(&out_host[i], &w, 4);
+    }
+    return GPT2_OK;
+}
+
 int gpt2_get_opt_state(gpt2_handle* h, float* m, float* v, int64_t* step, int on_device) {
     if (!h) return fail(GPT2_ERR_INVALID_ARG, "NULL handle");
     int rc = GPT2_OK;

@@ -74,6 +74,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gpt2_get_params": (I, [P, P, I]),
         "gpt2_get_grads": (I, [P, P, I]),
         "gpt2_grads_device": (I, [P, ctypes.POINTER(P), ctypes.POINTER(ctypes.c_int64)]),
+        "gpt2_debug_activation": (I, [P, I, I, I, I, P]),
         "gpt2_get_opt_state": (I, [P, P, P, ctypes.POINTER(ctypes.c_int64), I]),
         "gpt2_set_opt_state": (I, [P, P, P, ctypes.c_int64, I]),
         "gpt2_forward": (I, [P, P, P, I, I, P, ctypes.POINTER(F)]),
@@ -190,6 +191,15 @@ class GPT2:
     def get_grads(self) -> np.ndarray:
         out = np.empty(self.n_params, np.float32)
         _check(self._lib.gpt2_get_grads(self._h, _ptr(out), 0))
+        return out
+
+    ACT = {"resid": 0, "ln_1": 1, "qkv": 2, "attn": 3, "ln_2": 4, "gelu": 5, "ln_f": 6}
+
+    def debug_activation(self, kind: str, index: int, B: int, T: int) -> np.ndarray:
+        """gpt2_debug_activation: a saved activation of the last forward as float32 (B, T, width)."""
+        width = {"qkv": 3, "gelu": 4}.get(kind, 1) * self.cfg.n_embd
+        out = np.empty((B, T, width), np.float32)
+        _check(self._lib.gpt2_debug_activation(self._h, self.ACT[kind], index, B, T, _ptr(out)))
         return out
 
     def grads_view(self):

@@ -150,6 +150,32 @@ int gpt2_get_grads(gpt2_handle* h, float* flat, int on_device);
  * in place, each rank having scaled its losses by 1/world, so that every rank
  * clips and updates with the average gradient. Errors: INVALID_ARG (NULL). */
 int gpt2_grads_device(gpt2_handle* h, float** grads_dev, int64_t* n);
+/* Saved activations of the last forward, for a layer-by-layer comparison with a
+ * reference (the debugging advice of the source pages: compare each layer's
+ * activations, where a 1e-6 gap is rounding and a 1e-2 gap is a bug).
+ * kind / index:
+ *   GPT2_ACT_RESID  0..2L  residual stream (fp32): 0 = wte[idx] + wpe[t], 2l+1 =
+ *                          after block l's attention, 2l+2 = after block l's MLP
+ *   GPT2_ACT_LN1    0..L-1 ln_1 output of block l               (B, T, C)
+ *   GPT2_ACT_QKV    0..L-1 c_attn output of block l [q | k | v]  (B, T, 3C)
+ *   GPT2_ACT_ATTN   0..L-1 attention output of block l, heads concatenated, before
+ *                          attn.c_proj                           (B, T, C)
+ *   GPT2_ACT_LN2    0..L-1 ln_2 output of block l               (B, T, C)
+ *   GPT2_ACT_GELU   0..L-1 gelu(c_fc output) of block l         (B, T, 4C)
+ *   GPT2_ACT_LNF    0      ln_f output                           (B, T, C)
+ * B, T: those of the last forward (gpt2_forward, gpt2_accumulate, gpt2_step or
+ * gpt2_forward_last). out_host: B * T * width floats (host), receiving the values
+ * widened to fp32 (exactly, from bf16 in bf16 mode). Synchronous.
+ * Errors: INVALID_ARG (NULL, kind or index out of range, B or T out of range). */
+#define GPT2_ACT_RESID 0
+#define GPT2_ACT_LN1 1
+#define GPT2_ACT_QKV 2
+#define GPT2_ACT_ATTN 3
+#define GPT2_ACT_LN2 4
+#define GPT2_ACT_GELU 5
+#define GPT2_ACT_LNF 6
+int gpt2_debug_activation(gpt2_handle* h, int kind, int index, int B, int T, float* out_host);
+
 /* AdamW state: first and second moments (n_params floats each) and the step count. */
 int gpt2_get_opt_state(gpt2_handle* h, float* m, float* v, int64_t* step, int on_device);
 int gpt2_set_opt_state(gpt2_handle* h, const float* m, const float* v, int64_t step, int on_device);

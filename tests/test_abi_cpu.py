@@ -99,6 +99,8 @@ def test_generation_entries_reject_bad_arguments_on_host():
     assert lib.gpt2_decode(None, dummy, 1, 1, dummy) == -1
     assert lib.gpt2_sample(None, dummy, 1, 1.0, 0, dummy, dummy) == -1
     assert lib.gpt2_generate(None, dummy, 1, 1, 1, 1.0, 0, dummy, dummy) == -1
+    assert lib.gpt2_debug_activation(None, 0, 0, 1, 1, dummy) == -1
+    assert lib.gpt2_grads_device(None, ctypes.byref(ctypes.c_void_p()), ctypes.byref(ctypes.c_int64())) == -1
     ok = (1, dummy, 4, 8, 8, 1.0, 0, dummy, dummy, dummy, None)
     for i, bad in [(0, 7), (2, 0), (3, 0), (4, 7), (5, 0.0), (5, float("nan")), (5, float("inf")), (7, None)]:
         args = list(ok)

@@ -350,3 +350,58 @@ def test_forward_last_position_logits(precision, T):
     if precision == "fp32":
         assert _rel(got, full[:, -1, :].cpu().numpy()) < 1e-6
     m.close()
+
+
+# ----------------------------------------------------------------------------
+# Layer by layer: every saved activation of a forward against the oracle's
+# (the pages' debugging advice: diff each layer's activations).
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_saved_activations_layer_by_layer(precision):
+    """gpt2_debug_activation for every kind and layer against the oracle's forward
+    cache (residual states rebuilt from the oracle's cached branch outputs with
+    its own linear): fp32 1e-4 of max |value| per tensor, bf16 3e-2 and cosine
+    > 0.999."""
+    from decoder_only_transformer_sm_b200 import native
+    s = TINY
+    B, T = 3, 20
+    os_ = _oshape(s)
+    flat = S.random_params(s, seed=950)
+    idx, tgt = S.uniform_tokens(B, T, s.vocab_size, seed=951)
+    m = _model(s, precision, 4, 64)
+    m.set_params(flat)
+    m.forward(_dev(idx), _dev(tgt))
+    P = O.unflatten(os_, flat.astype(np.float64))
+    _, _, cache = O.forward(os_, P, idx)
+    C = s.n_embd
+
+    def flat_heads(z):   # (B, H, T, hd) -> (B, T, C)
+        return z.transpose(0, 2, 1, 3).reshape(B, T, C)
+
+    def check(got, ref, what):
+        if precision == "fp32":
+            assert _rel(got, ref) < 1e-4, what
+        else:
+            assert _rel(got, ref) < 3e-2, what
+            assert _cos(got, ref) > 0.999, what
+
+    x = P["wte"][idx] + P["wpe"][np.arange(T)][None]
+    check(m.debug_activation("resid", 0, B, T), x, "resid 0")
+    for l in range(s.n_layer):
+        c = cache["layers"][l]
+        pre = f"h.{l}."
+        check(m.debug_activation("ln_1", l, B, T), c["a"], ("ln_1", l))
+        qkv = np.concatenate([flat_heads(c["q"]), flat_heads(c["k"]), flat_heads(c["v"])], axis=-1)
+        check(m.debug_activation("qkv", l, B, T), qkv, ("qkv", l))
+        check(m.debug_activation("attn", l, B, T), c["y"], ("attn", l))
+        x = x + O.linear(c["y"], P[pre + "attn.c_proj.weight"], P[pre + "attn.c_proj.bias"])
+        check(m.debug_activation("resid", 2 * l + 1, B, T), x, ("resid", 2 * l + 1))
+        check(m.debug_activation("ln_2", l, B, T), c["m"], ("ln_2", l))
+        check(m.debug_activation("gelu", l, B, T), c["g"], ("gelu", l))
+        x = x + O.linear(c["g"], P[pre + "mlp.c_proj.weight"], P[pre + "mlp.c_proj.bias"])
+        check(m.debug_activation("resid", 2 * l + 2, B, T), x, ("resid", 2 * l + 2))
+    check(m.debug_activation("ln_f", 0, B, T), cache["f"], "ln_f")
+    for kind, index in [("ln_1", s.n_layer), ("resid", 2 * s.n_layer + 1), ("ln_f", 1), ("qkv", -1)]:
+        with pytest.raises(native.Gpt2Error, match="INVALID_ARG"):
+            m.debug_activation(kind, index, B, T)
+    m.close()
