@@ -613,3 +613,18 @@ def test_generate_draws_follow_torch_probabilities():
     for b in range(3):
         cdf = np.cumsum(_torch_topk_softmax(lg[b], 0.8, 10))
         assert seq[b, -1] == int(np.searchsorted(cdf, u[0, b], side="right"))
+
+
+def test_sample_low_temperature_limit_and_empty_generation():
+    """As the temperature goes to 0 the softmax concentrates on the maximum, so
+    every u away from 0 and 1 draws the argmax; a generation of no new tokens
+    returns the prompt unchanged."""
+    x = np.array([0.3, 1.2, -0.5, 1.1, 0.0])
+    for u in (1e-6, 0.25, 0.5, 0.999):
+        j, probs, _ = O.sample_next(x, 1e-3, 0, u)
+        assert j == 1 and probs[1] > 1.0 - 1e-12
+    s = MICRO
+    P = _params(s, seed=3)
+    idx, _ = S.uniform_tokens(2, 4, s.vocab_size, seed=39)
+    seq, margins = O.generate(s, P, idx, 0, 1.0, 0, np.zeros((0, 2)))
+    assert np.array_equal(seq, idx) and margins.shape == (0, 2)
