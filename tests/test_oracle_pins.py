@@ -254,7 +254,10 @@ def test_finite_differences_tiny_sampled():
 # ----------------------------------------------------------------------------
 # Independent model from torch library layers, autograd and torch's optimiser.
 # ----------------------------------------------------------------------------
-def _torch_model_step(s, flat, idx, tgt, lr, steps, max_norm=1.0):
+def _torch_model(s, flat):
+    """The pages' model written with torch library calls in float64 ("GPT-2
+    from Scratch": CausalSelfAttention, MLP, Block, GPT.forward with the tied
+    lm_head and F.cross_entropy(ignore_index=-1)). Returns (params, model)."""
     torch = pytest.importorskip("torch")
     F = torch.nn.functional
     names = [n for n, _ in O.layout(s)]
@@ -267,7 +270,9 @@ def _torch_model_step(s, flat, idx, tgt, lr, steps, max_norm=1.0):
         off += k
     C, H = s.n_embd, s.n_head
 
-    def model(idx_t, tgt_t):
+    def model(idx, tgt):
+        idx_t = torch.tensor(idx, dtype=torch.long)
+        tgt_t = torch.tensor(tgt, dtype=torch.long)
         B, T = idx_t.shape
         x = F.embedding(idx_t, P["wte"]) + F.embedding(torch.arange(T), P["wpe"])
         for l in range(s.n_layer):
@@ -285,6 +290,13 @@ def _torch_model_step(s, flat, idx, tgt, lr, steps, max_norm=1.0):
         logits = F.linear(f, P["wte"])
         return F.cross_entropy(logits.view(-1, logits.size(-1)), tgt_t.view(-1), ignore_index=-1)
 
+    return P, model
+
+
+def _torch_model_step(s, flat, idx, tgt, lr, steps, max_norm=1.0):
+    torch = pytest.importorskip("torch")
+    P, model = _torch_model(s, flat)
+    names = list(P)
     decay = [P[n] for n in names if P[n].dim() >= 2]
     nodecay = [P[n] for n in names if P[n].dim() < 2]
     opt = torch.optim.AdamW([{"params": decay, "weight_decay": 0.1},
@@ -293,7 +305,7 @@ def _torch_model_step(s, flat, idx, tgt, lr, steps, max_norm=1.0):
     out = []
     for _ in range(steps):
         opt.zero_grad(set_to_none=True)
-        loss = model(torch.tensor(idx, dtype=torch.long), torch.tensor(tgt, dtype=torch.long))
+        loss = model(idx, tgt)
         loss.backward()
         grads = {n: P[n].grad.detach().clone().numpy() for n in names}
         norm = torch.nn.utils.clip_grad_norm_(list(P.values()), max_norm)
@@ -379,6 +391,74 @@ def test_accumulation_equals_big_batch():
     assert abs(loss_big - loss_acc) < 1e-12
     for n in G_big:
         assert np.max(np.abs(G_big[n] - G_acc[n])) < 1e-13, n
+
+
+def _masked_micro_batches():
+    """Four micro-batches whose targets carry masked prefixes of different
+    lengths (the supervised fine-tuning masking of "Pretraining and
+    fine-tuning nanoGPT-124M from scratch"), so every micro-batch has its own
+    count of valid targets; the last one is fully valid."""
+    batches = []
+    for k, n_masked in enumerate([3, 11, 0, 17]):
+        idx, tgt = S.uniform_tokens(2, 24, 1024, seed=40 + k)
+        tgt[0, :n_masked] = -1
+        tgt[1, :n_masked // 2] = -1
+        batches.append((idx, tgt))
+    return batches
+
+
+def _torch_accumulation(s, flat, batches):
+    """The pages' accumulation loop with library calls ("Gradient
+    accumulation, and the bug in getting it right"): each micro-batch's
+    F.cross_entropy(ignore_index=-1) divided by the number of micro-batches,
+    backward() adding into .grad; the reported loss is the sum of the scaled
+    micro losses."""
+    P, model = _torch_model(s, flat)
+    total = 0.0
+    for idx, tgt in batches:
+        loss = model(idx, tgt) / len(batches)
+        loss.backward()
+        total += loss.item()
+    return total, {n: P[n].grad.detach().numpy().copy() for n in P}
+
+
+def _max_grad_err(G, ref):
+    return max(np.max(np.abs(G[n] - ref[n])) / max(1.0, np.max(np.abs(ref[n]))) for n in ref)
+
+
+def test_accumulation_with_masks_matches_torch_loop():
+    s = TINY
+    flat = S.random_params(_syn(s), seed=41).astype(np.float64)
+    batches = _masked_micro_batches()
+    assert len({int((t != -1).sum()) for _, t in batches}) == 4   # valid counts all differ
+    ref_loss, ref_G = _torch_accumulation(s, flat, batches)
+    loss, G = O.accumulate_grads(s, O.unflatten(s, flat), batches)
+    assert abs(loss - ref_loss) < 1e-12
+    assert _max_grad_err(G, ref_G) < 1e-12
+
+
+def test_accumulation_token_weighted_mean_is_rejected():
+    """Planted mistake: a token-weighted global mean over all micro-batches
+    (each micro-batch weighted by its share of the valid targets) instead of
+    the per-micro-batch mean divided by the number of micro-batches. With
+    unequal valid counts the two differ, and the torch loop tells them apart."""
+    s = TINY
+    flat = S.random_params(_syn(s), seed=41).astype(np.float64)
+    batches = _masked_micro_batches()
+    ref_loss, ref_G = _torch_accumulation(s, flat, batches)
+    P = O.unflatten(s, flat)
+    n_valid = [int((t != -1).sum()) for _, t in batches]
+    G = O.zeros_like(s)
+    loss = 0.0
+    for (idx, tgt), nv in zip(batches, n_valid):
+        l_k, _, cache = O.forward(s, P, idx, tgt)
+        w = nv / sum(n_valid)
+        g = O.backward(s, P, cache, loss_scale=w)
+        for k in G:
+            G[k] += g[k]
+        loss += w * l_k
+    assert abs(loss - ref_loss) > 1e-4
+    assert _max_grad_err(G, ref_G) > 1e-6
 
 
 # ----------------------------------------------------------------------------
