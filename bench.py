@@ -204,7 +204,8 @@ def run_reference(args):
         "ms_per_step": 1000.0 * sec, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic Zipf(1.1) tokens", "impl": "reference",
         "config": workload_config(16, 1024, args.gpus),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample,
+                         "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -257,6 +258,31 @@ def replica_tokens(rank: int, B: int, T: int, vocab_real: int, nb: int = 2):
     """The nb synthetic batches of one replica: each rank draws its own seeded Zipf stream."""
     from decoder_only_transformer_sm_b200 import synthetic as S
     return [S.zipf_tokens(B, T, vocab_real, seed=1001 + 97 * rank + i) for i in range(nb)]
+
+
+def step_stats(times_ms, world: int) -> dict:
+    """Median, p10, p90 and mean of the per-step device times (each step bracketed
+    by its own CUDA events on the launching stream); for N > 1 each statistic is
+    the max over ranks."""
+    xs = sorted(times_ms)
+
+    def q(f):
+        i = f * (len(xs) - 1)
+        lo, hi = int(math.floor(i)), int(math.ceil(i))
+        return xs[lo] + (xs[hi] - xs[lo]) * (i - lo)
+
+    out = {"median": q(0.5), "p10": q(0.1), "p90": q(0.9), "mean": sum(xs) / len(xs)}
+    return {k: max_over_ranks(v, world) for k, v in out.items()}
+
+
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def job_throughput(ms_per_step_max: float, B: int, T: int, world: int) -> float:
@@ -442,6 +468,84 @@ def run_accum(args):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------
+# --workload kernel: one kernel of the step in isolation, through the kernel-level
+# C ABI (gpt2_kernels.h), timed with CUDA events; the target of ncu captures
+# ----------------------------------------------------------------------------
+def _events(torch, fn, reps: int):
+    times = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    return times
+
+
+def kernel_gemm(args):
+    import torch
+    from decoder_only_transformer_sm_b200 import native
+    M, N, K = args.M, args.N, args.K
+    g = torch.Generator().manual_seed(0)
+    if args.layout == "NT":
+        A, B = torch.randn((M, K), generator=g), torch.randn((N, K), generator=g)
+    elif args.layout == "NN":
+        A, B = torch.randn((M, K), generator=g), torch.randn((K, N), generator=g)
+    else:
+        A, B = torch.randn((K, M), generator=g), torch.randn((K, N), generator=g)
+    A, B = A.to(torch.bfloat16).cuda(), B.to(torch.bfloat16).cuda()
+    ep = args.epilogue
+    f32_out = ep in ("bias_resid", "accum_f32")
+    out = torch.zeros((M, N), dtype=torch.float32 if f32_out else torch.bfloat16, device="cuda")
+    out2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda") if ep == "bias_gelu" else None
+    bias = torch.randn(N, device="cuda") if ep.startswith("bias") else None
+    resid = torch.randn((M, N), device="cuda") if ep == "bias_resid" else None
+    aux = torch.randn((M, N), device="cuda").to(torch.bfloat16) if ep == "mul" else None
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fn = lambda: native.matmul_bf16(args.layout, A, B, M, N, K, ep, out, out2=out2, bias=bias,  # noqa: E731
+                                    resid=resid, aux=aux, beta=1.0, engine="tc" if args.engine else "simt",
+                                    status=st)
+    fn()
+    torch.cuda.synchronize()
+    t = _events(torch, fn, args.reps)
+    best = min(t)
+    print(json.dumps({"case": "gemm", "layout": args.layout, "M": M, "N": N, "K": K, "epilogue": ep,
+                      "ms": t, "tflops_best": 2.0 * M * N * K / best / 1e9, "status": int(st.item())}))
+
+
+def kernel_attention(args):
+    import torch
+    from decoder_only_transformer_sm_b200 import native
+    B, T, H, hd = args.B, args.T, args.H, args.hd
+    C = H * hd
+    g = torch.Generator().manual_seed(0)
+    qkv = torch.randn((B, T, 3 * C), generator=g).to(torch.bfloat16).cuda()
+    dout = torch.randn((B, T, C), generator=g).to(torch.bfloat16).cuda()
+    out = torch.empty((B, T, C), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
+    dqkv = torch.empty_like(qkv)
+    ws = torch.empty(B * H * T, dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fwd = lambda: native.attention_fwd(qkv, out, lse, B, T, H, hd, engine=args.engine, status=st)  # noqa: E731
+    bwd = lambda: native.attention_bwd(qkv, out, dout, lse, dqkv, B, T, H, hd, ws,  # noqa: E731
+                                       engine=args.engine, status=st)
+    fwd()
+    bwd()
+    torch.cuda.synchronize()
+    tf = _events(torch, fwd, args.reps)
+    tb = _events(torch, bwd, args.reps)
+    flops = 2.0 * B * H * T * (T + 1) * hd
+    print(json.dumps({"case": "attention", "B": B, "T": T, "H": H, "hd": hd, "fwd_ms": tf, "bwd_ms": tb,
+                      "fwd_tflops_best": flops / min(tf) / 1e9, "bwd_tflops_best": 2.5 * flops / min(tb) / 1e9,
+                      "status": int(st.item())}))
+
+
+def run_kernel(args):
+    {"gemm": kernel_gemm, "attention": kernel_attention}[args.kernel](args)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -476,19 +580,20 @@ def run_ours(args):
     losses = []
     barrier()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     launches = 0
     with ClockSampler(local) as clk:
-        e0.record(stream)
+        ev[0].record(stream)
         for k in range(args.steps):
             loss, norm = m.step(*dev[k % nb], LR)
             launches += m.last_launch_count()
             losses.append(loss)
-        e1.record(stream)
+            ev[k + 1].record(stream)
         torch.cuda.synchronize()
     barrier()
     clocks = clk.summary()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    ms = max_over_ranks(ev[0].elapsed_time(ev[-1]) / args.steps, world)
+    per_step = step_stats([ev[k].elapsed_time(ev[k + 1]) for k in range(args.steps)], world)
 
     # ---- end to end: host (pinned) token buffers through gpt2_step_host ----
     barrier()
@@ -546,6 +651,7 @@ def run_ours(args):
     if world == 1 and not args.no_cpu_baseline and w is WORKLOAD:
         times, threads = oracle_step_time(1024, 0, 1)
         cpu = {"value": 1024 / times[0], "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "cpu_model": cpu_model(),
                "sample": "one float64 oracle step (forward, loss, backward, clip, AdamW on all 124.5M "
                          "parameters) on B=1 x T=1024 Zipf tokens, timed on this host"}
     line = {
@@ -568,6 +674,7 @@ def run_ours(args):
                 "h2d_bytes_per_step": 2 * B * T * 4, "d2h_bytes_per_step": 40},
         "gpu_launches": launches,
         "clocks": clocks,
+        "step_ms": per_step,
         "loss_first_last": [losses[0], losses[-1]],
     }
     print(json.dumps(line), flush=True)
@@ -579,11 +686,27 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["train", "eval", "accum", "generate"], default="train",
+    ap.add_argument("--workload", choices=["train", "eval", "accum", "generate", "kernel"], default="train",
                     help="train: the training step (the benchmark line); eval: forward + loss and the "
                          "last-position forward of generation; accum: one update over 32 accumulated "
                          "micro-batches (524,288 tokens); generate: the pages' sampling call with a "
-                         "key/value cache (--batch sets B, default 1); eval, accum and generate on one GPU")
+                         "key/value cache (--batch sets B, default 1); kernel: one GEMM or attention "
+                         "call in isolation (--kernel and the shape options below; prints its CUDA-event "
+                         "times); eval, accum, generate and kernel on one GPU")
+    kg = ap.add_argument_group("--workload kernel")
+    kg.add_argument("--kernel", choices=["gemm", "attention"], default="gemm")
+    kg.add_argument("--layout", default="NT", choices=["NT", "NN", "TN"])
+    kg.add_argument("--M", type=int, default=16384)
+    kg.add_argument("--N", type=int, default=3072)
+    kg.add_argument("--K", type=int, default=768)
+    kg.add_argument("--epilogue", default="store")
+    kg.add_argument("--engine", type=int, default=1,
+                    help="gemm: 1 tcgen05, 0 SIMT; attention: 2 tcgen05, 1 mma.sync, 0 SIMT")
+    kg.add_argument("--B", type=int, default=16)
+    kg.add_argument("--T", type=int, default=1024)
+    kg.add_argument("--H", type=int, default=12)
+    kg.add_argument("--hd", type=int, default=64)
+    kg.add_argument("--reps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--model", choices=sorted(MODELS), default="124m",
                     help="124m is the benchmark workload; the others are the same step at GPT-2 medium, "
@@ -603,6 +726,8 @@ def main():
         run_accum(args)
     elif args.workload == "generate":
         run_generate(args)
+    elif args.workload == "kernel":
+        run_kernel(args)
     else:
         run_ours(args)
 

@@ -715,8 +715,13 @@ int read_scalars(gpt2_handle* h) {
     return GPT2_OK;
 }
 
+// Reports the status bits read back by read_scalars, and clears them on the
+// device once reported, so that one bad call does not fail every later one.
 int status_error(gpt2_handle* h) {
     const unsigned s = h->h_sc->status;
+    if (!s) return GPT2_OK;
+    h->h_sc->status = 0;
+    CK(cudaMemsetAsync(&h->d_sc->status, 0, sizeof(unsigned), h->stream));
     if (s & STATUS_TIMEOUT) return fail(GPT2_ERR_TIMEOUT, "a bounded wait inside a kernel gave up");
     if (s & STATUS_BAD_TOKEN) return fail(GPT2_ERR_BAD_TOKEN, "token id or target out of range");
     return GPT2_OK;
@@ -741,9 +746,11 @@ int accumulate_impl(gpt2_handle* h, const int* idx, const int* targets, int B, i
     return pending_error(h);
 }
 
+// Starts a gradient cycle: gradients, accumulated loss and status bits to zero.
 int zero_grad_impl(gpt2_handle* h) {
     CK(cudaMemsetAsync(h->grads, 0, h->n_params * sizeof(float), h->stream));
     CK(cudaMemsetAsync(&h->d_sc->loss_accum, 0, sizeof(double), h->stream));
+    CK(cudaMemsetAsync(&h->d_sc->status, 0, sizeof(unsigned), h->stream));
     return GPT2_OK;
 }
 
@@ -1203,6 +1210,7 @@ int gpt2_decode(gpt2_handle* h, const int32_t* tokens, int B, int pos, void* log
     int rc = pending_error(h);
     if (rc) return rc;
     h->kv_len = pos + 1;
+    h->kv_B = B;   // rows B .. kv_B-1 have no entry at pos: later calls may use at most B rows
     rc = read_scalars(h);
     if (rc) return rc;
     return status_error(h);

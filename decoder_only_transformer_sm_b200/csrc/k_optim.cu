@@ -40,11 +40,16 @@ __global__ void __launch_bounds__(256) adamw_kernel(const AdamChunk* __restrict_
                                                     const float* __restrict__ g, float* __restrict__ m,
                                                     float* __restrict__ v, bf16* __restrict__ shadow,
                                                     const double* __restrict__ sumsq,
-                                                    const double* __restrict__ loss_accum, float lr, float clip,
+                                                    const double* __restrict__ loss_accum,
+                                                    const unsigned* __restrict__ status, float lr, float clip,
                                                     float bc1, float bc2, float wd) {
     const double ss = *sumsq;
     const double loss = *loss_accum;
-    if (!isfinite(ss) || !isfinite(loss)) return;   // the host reports NONFINITE; nothing changes
+    // A step whose forward saw an out-of-range id, or whose kernels gave up a
+    // bounded wait, is reported as an error by the host and must not move the
+    // weights; neither must a non-finite loss or norm (reported as NONFINITE).
+    if (*status & (STATUS_BAD_TOKEN | STATUS_TIMEOUT)) return;
+    if (!isfinite(ss) || !isfinite(loss)) return;
     const float norm = (float)sqrt(ss);
     const float coef = fminf(1.f, clip / (norm + 1e-6f));
     const AdamChunk ch = chunks[blockIdx.x];
@@ -133,8 +138,8 @@ void launch_sumsq(const Ctx& ctx, const float* g, long long n, double* out) {
 void launch_adamw(const Ctx& ctx, const AdamChunk* chunks, int n_chunks, float* p, const float* g, float* m,
                   float* v, bf16* shadow, const double* sumsq, const double* loss_accum, float lr, float clip,
                   float bc1, float bc2, float wd) {
-    adamw_kernel<<<n_chunks, 256, 0, ctx.stream>>>(chunks, p, g, m, v, shadow, sumsq, loss_accum, lr, clip, bc1,
-                                                   bc2, wd);
+    adamw_kernel<<<n_chunks, 256, 0, ctx.stream>>>(chunks, p, g, m, v, shadow, sumsq, loss_accum, ctx.status, lr,
+                                                   clip, bc1, bc2, wd);
     ++*ctx.launches;
 }
 

@@ -172,6 +172,9 @@ struct AdamChunk {        // a run of elements inside one tensor
     int decay;
 };
 void launch_sumsq(const Ctx& ctx, const float* g, long long n, double* out);
+// Clip + AdamW over all chunks. Skips the whole update (nothing written) when
+// *ctx.status has STATUS_BAD_TOKEN or STATUS_TIMEOUT set, or when *sumsq or
+// *loss_accum is not finite.
 void launch_adamw(const Ctx& ctx, const AdamChunk* chunks, int n_chunks, float* p, const float* g, float* m,
                   float* v, bf16* shadow, const double* sumsq, const double* loss_accum, float lr, float clip,
                   float bc1, float bc2, float wd);

@@ -41,6 +41,9 @@
  *     ignored by the loss. Ids must lie in [0, vocab_size); targets in
  *     {-1} U [0, vocab_size). An out-of-range id is clamped on the device and
  *     reported as GPT2_ERR_BAD_TOKEN by the next synchronising call.
+ *   * Device-side error flags (BAD_TOKEN, TIMEOUT) are cleared once a call has
+ *     reported them, and by gpt2_zero_grad (the start of a gradient cycle), so
+ *     one bad call does not fail the calls after it.
  *   * One handle is used from one thread at a time; handles are independent.
  */
 #ifndef GPT2_B200_H
@@ -230,10 +233,11 @@ int gpt2_prefill(gpt2_handle* h, const int32_t* idx_dev, int B, int T, void* log
  * decodes at the positions up to pos - 1). Runs the blocks on the B rows at
  * position pos, writes their k and v to cache row pos, attends over rows
  * 0 .. pos, and writes the logits (B, vocab_size) (fp32 or bf16 by mode) to
- * logits_dev. Afterwards the cache holds pos + 1 positions.
+ * logits_dev. Afterwards the cache holds pos + 1 positions of sequences
+ * 0 .. B-1 only: later decodes may use at most B rows.
  * Synchronises once at the end. Errors: INVALID_ARG (no prefill yet, B above
- * the last prefill's B, pos < 1, pos above the cached length, or pos >=
- * block_size); BAD_TOKEN for an id outside [0, vocab_size). */
+ * the rows of the last prefill or decode, pos < 1, pos above the cached
+ * length, or pos >= block_size); BAD_TOKEN for an id outside [0, vocab_size). */
 int gpt2_decode(gpt2_handle* h, const int32_t* tokens_dev, int B, int pos, void* logits_dev);
 
 /* One draw per row of logits_dev (B, vocab_size) (fp32 or bf16 by mode, rows
@@ -277,11 +281,16 @@ int gpt2_accumulate(gpt2_handle* h, const int32_t* idx_dev, const int32_t* targe
 /* Clip + AdamW on the accumulated gradients, step counter += 1.
  * loss_host / grad_norm_host (nullable host floats) receive the accumulated loss
  * and the pre-clip global gradient norm. Synchronises once at the end.
- * Returns NONFINITE (and leaves parameters, moments, step unchanged) if the
- * norm or the accumulated loss is not finite. */
+ * Returns NONFINITE if the norm or the accumulated loss is not finite, and
+ * BAD_TOKEN / TIMEOUT if a micro-batch since the last gpt2_zero_grad saw an
+ * out-of-range id or target, or a kernel gave up a bounded wait. In all three
+ * cases the update kernel writes nothing: parameters, moments, the bf16 weight
+ * copy and the step counter are unchanged. */
 int gpt2_update(gpt2_handle* h, float lr, float* loss_host, float* grad_norm_host);
 
 /* One full training step: zero_grad, accumulate(loss_scale = 1), update.
+ * A step that returns NONFINITE, BAD_TOKEN or TIMEOUT leaves parameters,
+ * moments and the step counter unchanged (as gpt2_update).
  * Device-resident inputs. The ids and targets are first copied (on the
  * handle's stream) into a buffer the handle owns. The first step with a given
  * (B, T) runs eagerly; the second captures its zero_grad/forward/backward

@@ -109,7 +109,9 @@ int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, const void*
  * call on a device, with that device current, looks up the array's device
  * address (cudaGetSymbolAddress) and caches it; make that first call before
  * any stream capture. Every call shares the array: calls that overlap on the
- * GPU race, and must not be issued. Other arguments and errors as
+ * GPU race, and must not be issued. engine must be 0 (the SIMT kernels: fp32
+ * arithmetic on fp32 or bf16 operands); any other engine returns
+ * GPT2_ERR_INVALID_ARG. No colsum_part output. Other arguments and errors as
  * gpt2k_attention_bwd. */
 int gpt2k_attention_bwd_noalloc(int dtype, const void* qkv, const void* out, const void* dout, const float* lse,
                                 void* dqkv, int B, int T, int H, int hd, int engine, uint32_t* status_dev,

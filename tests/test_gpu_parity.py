@@ -230,15 +230,70 @@ def test_causal_invariance_on_gpu():
     m.close()
 
 
-def test_bad_token_reported():
+def _state(m):
+    mm, vv, t = m.get_opt_state()
+    return m.get_params(), mm, vv, t
+
+
+def _assert_same_state(a, b):
+    """Bit-identical parameters, moments and step counter (NaNs included)."""
+    for x, y in zip(a[:3], b[:3]):
+        assert x.tobytes() == y.tobytes()
+    assert a[3] == b[3]
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_bad_token_leaves_state_unchanged(precision):
+    """A step that reports BAD_TOKEN (an id outside [0, V) in the forward) must
+    not move the weights, the moments or the step counter ("The loop": the
+    update belongs to a valid step), and the report clears the flag: the next
+    valid step succeeds and counts as step 2."""
     from decoder_only_transformer_sm_b200 import native
     s = TINY
-    idx, tgt = S.uniform_tokens(1, 8, s.vocab_size, seed=16)
-    idx[0, 3] = s.vocab_size + 5
-    m = _model(s, "fp32", 1, 8)
+    m = _model(s, precision, 2, 8)
+    m.set_params(S.random_params(s, seed=16))
+    idx, tgt = S.uniform_tokens(2, 8, s.vocab_size, seed=16)
+    m.step(_dev(idx), _dev(tgt), 6e-4)                      # t = 1, moments non-zero
+    before = _state(m)
+    bad = idx.copy()
+    bad[0, 3] = s.vocab_size + 5
+    for _ in range(3):                                      # eager, graph capture, graph replay
+        with pytest.raises(native.Gpt2Error) as e:
+            m.step(_dev(bad), _dev(tgt), 6e-4)
+        assert e.value.code == -6
+        _assert_same_state(before, _state(m))
+    badt = tgt.copy()
+    badt[1, 0] = s.vocab_size
+    with pytest.raises(native.Gpt2Error) as e:              # an out-of-range target
+        m.step(_dev(idx), _dev(badt), 6e-4)
+    assert e.value.code == -6
+    _assert_same_state(before, _state(m))
+    m.step(_dev(idx), _dev(tgt), 6e-4)
+    assert _state(m)[3] == 2
+    m.close()
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_nonfinite_step_leaves_state_unchanged(precision):
+    """A NaN parameter (made on the host through gpt2_set_params) gives a
+    non-finite loss and norm: the step returns NONFINITE and parameters,
+    moments and the step counter stay bit-identical ("Gradient clipping" needs
+    a finite norm)."""
+    from decoder_only_transformer_sm_b200 import native
+    s = TINY
+    m = _model(s, precision, 2, 8)
+    flat = S.random_params(s, seed=23)
+    m.set_params(flat)
+    idx, tgt = S.uniform_tokens(2, 8, s.vocab_size, seed=24)
+    m.step(_dev(idx), _dev(tgt), 6e-4)
+    p = m.get_params()
+    p[12345] = np.nan                                       # inside wte: reaches the logits
+    m.set_params(p)
+    before = _state(m)
     with pytest.raises(native.Gpt2Error) as e:
         m.step(_dev(idx), _dev(tgt), 6e-4)
-    assert e.value.code == -6
+    assert e.value.code == -5
+    _assert_same_state(before, _state(m))
     m.close()
 
 
@@ -291,6 +346,47 @@ def test_tiny_bf16_ragged():
     idx, tgt = S.uniform_tokens(3, 45, s.vocab_size, seed=18)
     tgt[0, :20] = -1
     _bf16_check(s, S.random_params(s, seed=19), idx, tgt)
+
+
+def test_bf16_accumulation_with_masks_matches_oracle():
+    """Gradient accumulation in bf16 mode on the 124M width (one block, C=768,
+    12 heads, head width 64, so the tensor-core GEMMs and attention run):
+    zero_grad + 4 x accumulate(1/4) + update over the accumulation workload's
+    micro-batches, the second half with masked target prefixes ("Gradient
+    accumulation, and the bug in getting it right"; "Supervised fine-tuning").
+    Against oracle.accumulate_grads + adamw_update: loss 2e-2 absolute,
+    per-tensor gradient cosine >= 0.999, gradient norms within 1%, the global
+    norm within 1%, and the post-update parameters within 2*lr of the oracle's
+    (AdamW's first step moves each element by about lr)."""
+    s = S.ModelShape(1, 12, 768, 1024, 128)
+    os_ = _oshape(s)
+    n_micro, B, T, lr = 4, 2, 128, 6e-4
+    flat = S.random_params(s, seed=61)
+    batches = S.accumulation_batches(n_micro, B, T, s.vocab_size, seed=62)
+    assert all((t == -1).any() for _, t in batches[n_micro // 2:])
+    m = _model(s, "bf16", B, T)
+    m.set_params(flat)
+    m.zero_grad()
+    for idx, tgt in batches:
+        m.accumulate(_dev(idx), _dev(tgt), 1.0 / n_micro)
+    g = m.get_grads()
+    loss, norm = m.update(lr)
+    P = O.unflatten(os_, flat.astype(np.float64))
+    ref_loss, G = O.accumulate_grads(os_, P, batches)
+    ref_norm = O.grad_norm(G)
+    assert abs(loss - ref_loss) < 2e-2, (loss, ref_loss)
+    assert abs(norm / ref_norm - 1.0) < 1e-2, (norm, ref_norm)
+    Gg = _split(s, g)
+    worst = min((_cos(Gg[n], G[n]), n) for n in G)
+    assert worst[0] >= 0.999, worst
+    for n in G:
+        nr, ng = np.linalg.norm(G[n]), np.linalg.norm(Gg[n].astype(np.float64))
+        if nr > 0:
+            assert abs(ng / nr - 1.0) < 1e-2, (n, ng, nr)
+    M, V = O.zeros_like(os_), O.zeros_like(os_)
+    O.adamw_update(os_, P, G, M, V, 1, lr)
+    assert np.max(np.abs(m.get_params() - O.flatten(os_, P))) <= 2 * lr + 1e-6
+    m.close()
 
 
 def test_step_graph_replay_matches_eager(monkeypatch):

@@ -204,10 +204,13 @@ def test_decode_argument_errors():
             m.decode(tok, pos, lg)
     with pytest.raises(native.Gpt2Error, match="INVALID_ARG"):   # more rows than the prefill
         m.decode(_dev(np.zeros(3)), 4, lg)
-    m.decode(tok, 4, lg)                                         # the next position is fine
+    m.decode(tok[:1], 4, lg)                                     # one row: row 1 has no entry at 4
+    with pytest.raises(native.Gpt2Error, match="INVALID_ARG"):   # so two rows at 5 are refused
+        m.decode(tok, 5, lg)
+    m.decode(tok[:1], 5, lg)                                     # the next position of row 0 is fine
     m.set_params(m.get_params())                                 # a weight change empties the cache
     with pytest.raises(native.Gpt2Error, match="INVALID_ARG"):
-        m.decode(tok, 5, lg)
+        m.decode(tok[:1], 6, lg)
     out = torch.empty((2, 8), dtype=torch.int32, device="cuda")
     u = torch.zeros((4, 2), device="cuda")
     for temp in (0.0, float("nan")):

@@ -43,8 +43,13 @@ def test_noalloc_matches_workspace_variant_twice(dtype):
         ws = torch.empty((B * H * T,), dtype=torch.float32, device="cuda")
         st = native.attention_bwd(qkv, out, dout, lse, ref, B, T, H, hd, ws)
         got = torch.full_like(qkv, float("nan"))
+        torch.cuda.synchronize()
+        free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
         native.attention_bwd_noalloc(qkv, out, dout, lse, got, B, T, H, hd, status=st)
         torch.cuda.synchronize()
+        if call == 1:   # the first call may load the module; the second must allocate nothing
+            assert torch.cuda.mem_get_info()[0] == free0
+            assert torch.cuda.memory_allocated() == alloc0
         assert int(st.item()) == 0
         assert torch.isfinite(got.float()).all()
         assert _rel(got, ref) <= TOL[dtype], (call, _rel(got, ref))
