@@ -526,7 +526,7 @@ def kernel_attention(args):
     out = torch.empty((B, T, C), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
     dqkv = torch.empty_like(qkv)
-    ws = torch.empty(B * H * T, dtype=torch.float32, device="cuda")
+    ws = torch.empty(native.attention_bwd_workspace(B, T, H, hd, args.engine), dtype=torch.float32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     fwd = lambda: native.attention_fwd(qkv, out, lse, B, T, H, hd, engine=args.engine, status=st)  # noqa: E731
     bwd = lambda: native.attention_bwd(qkv, out, dout, lse, dqkv, B, T, H, hd, ws,  # noqa: E731

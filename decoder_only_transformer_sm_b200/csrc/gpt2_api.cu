@@ -55,6 +55,7 @@ struct DevScalars {
     double sumsq;        // global gradient sum of squares
     int n_valid;         // targets != -1 in the current micro-batch
     unsigned status;     // STATUS_* bits
+    int work;            // work-item counter of the attention backward
 };
 
 struct ProfSite {
@@ -421,7 +422,10 @@ template <>
 void attn_bwd<bf16>(gpt2_handle* h, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
                     bf16* dqkv, int B, int T, float* colsum_part) {
     if (attn_bwd_sums<bf16>(h)) {
-        if (!launch_attention_bwd_tc(h->ctx(), qkv, out, dout, lse, h->dpre, dqkv, B, T, h->H, colsum_part))
+        // the fp32 dQ accumulator (B*T*C floats) lives in du, which is dead between the
+        // c_fc input-gradient GEMM and the next block's mlp.c_proj backward
+        if (!launch_attention_bwd_tc(h->ctx(), qkv, out, dout, lse, h->dpre, (float*)h->du, &h->d_sc->work, dqkv,
+                                     B, T, h->H, colsum_part))
             h->host_error = "tensor-map encoding failed for the attention backward";
     } else if (h->use_tc_attention)
         launch_attention_bwd_mma(h->ctx(), qkv, out, dout, lse, h->dpre, dqkv, B, T, h->H, h->hd);

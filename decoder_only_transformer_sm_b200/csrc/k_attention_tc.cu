@@ -1,5 +1,6 @@
-// Causal flash attention forward on the sm_100a tensor cores (tcgen05), head
-// width 64, bf16 operands, fp32 softmax and accumulation.
+// Causal flash attention forward and backward on the sm_100a tensor cores
+// (tcgen05), head width 64, bf16 operands, fp32 softmax and accumulation. The
+// backward is described above its kernel, further down.
 //
 // Definition ("GPT-2 from Scratch", "CausalSelfAttention"; "Let's reproduce
 // GPT-2 (124M)", "FlashAttention and vocabulary padding"): per (b, h),
@@ -410,42 +411,49 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ============================================================================
-// Backward. D = rowsum(dO * O) comes from the pre-pass kernel. With
-// P = exp(S - lse) recomputed from the saved lse:
+// Backward. With P = exp(S - lse) recomputed from the saved lse and
+// D = rowsum(dO * O) from the pre-pass:
 //   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),
 //   dK = dS^T Q / sqrt(64),  dQ = dS K / sqrt(64).
-// dK/dV kernel: one CTA per (b, h, 128-key tile); it walks the 64-query tiles
-// at or after the key tile. K and V are copied once into TMEM as packed bf16
-// A operands, so the N=64 MMAs read only their B operand from shared memory
-// (with both operands there they are limited by shared-memory bandwidth).
-// S^T = K Q^T and dP^T = V dO^T (M=128 keys, N=64 queries) go to
-// double-buffered TMEM so the tensor core computes tile i+1 while 8 warps turn
-// tile i into P^T and dS^T, written back as packed bf16 over the S^T / dP^T
-// columns they came from; dV += P^T dO and dK += dS^T Q (A from TMEM; dO and Q
-// as N-major shared operands) accumulate in TMEM. dQ kernel: one CTA per (b, h, 128-query tile) over the 64-key tiles at
-// or before it: S = Q K^T, dP = dO V^T, dS, then dQ += dS K in TMEM.
+// One CTA per (b, h, 128-key tile) walks the 128-query tiles at or after its
+// key tile, so each (key tile, query tile) pair computes S and dP once:
+//   S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 128 queries, K = 64) into
+//     TMEM (one buffer each; the element-wise warps copy them to registers
+//     and release them at once, so the next pair's MMAs run during the
+//     element-wise math of this one);
+//   8 element-wise warps (thread = key row) form P^T, written to TMEM as the
+//     packed-bf16 A operand of dV += P^T dO, and dS^T, written to shared memory
+//     (128-byte swizzle, two 64-query atoms): K-major it is the A operand of
+//     dK += dS^T Q, MN-major the A operand of dQ = dS K;
+//   dV and dK accumulate in TMEM over the query tiles; the pair's dQ (M = 128
+//     queries, N = 64) goes to TMEM, and 4 drain warps scale it, stage it in
+//     shared memory and add it into an fp32 (B T, C) accumulator with the TMA
+//     bulk reduce-add (zeroed by the pre-pass; the post-pass rounds it to
+//     bf16 into dqkv).
+// The 5 matrix products of the algorithm are each computed once; no T x T
+// matrix goes to HBM.
 // ============================================================================
-constexpr int BW_EW_WARPS = 8;                     // 2 warps per TMEM lane quarter, 32 columns each
-constexpr int BW_THREADS = 64 + 32 * BW_EW_WARPS;
-constexpr int T64_BYTES = 64 * HD * 2;      // 8 KB: 64 rows x 128 bytes
-constexpr int T128_BYTES = 128 * HD * 2;    // 16 KB
+constexpr int T128_BYTES = 128 * HD * 2;    // 16 KB: 128 rows x 128 bytes
 
-// Write one 64-column bf16 result row (128 bytes) per thread of a 4-warp group
-// through a swizzled 128-row staging tile, then copy whole rows to global
-// memory: dst(row) = base + row * ld (elements), rows >= n_rows skipped.
-// If csum is non-null, the warp also writes the column sums of its 32 rows
-// (rows at or beyond n_rows excluded) of the stored bf16 values as 64 floats
-// at csum; a warp whose rows all lie beyond n_rows writes nothing.
-__device__ __forceinline__ void store_rows_64(uint8_t* stage, int r, const float* v, float scale, bf16* base,
-                                              long long ld, int n_rows, float* csum) {
-    const int lane = threadIdx.x & 31, quarter = (threadIdx.x >> 5) & 3;
+// Rows of a 64-column bf16 result pass through a 128-row staging tile (128
+// bytes per row, 128-byte swizzle): each thread writes 32 columns of its own row
+// at a time (stage_row_32), then its warp copies whole rows of its 32-row group
+// to global memory (flush_rows_64): dst(row) = base + row * ld (elements), rows
+// >= n_rows skipped. If csum is non-null, the warp also writes the column sums
+// of its 32 rows (rows at or beyond n_rows excluded) of the stored bf16 values
+// as 64 floats at csum; a warp whose rows all lie beyond n_rows writes nothing.
+__device__ __forceinline__ void stage_row_32(uint8_t* stage, int r, const float* v, float scale, int half) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < 4; ++c) {
         float t[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) t[e] = v[8 * c + e] * scale;
-        *reinterpret_cast<uint4*>(stage + swz128(r, c)) = pack8_bf16(t);
+        *reinterpret_cast<uint4*>(stage + swz128(r, 4 * half + c)) = pack8_bf16(t);
     }
+}
+__device__ __forceinline__ void flush_rows_64(const uint8_t* stage, bf16* base, long long ld, int n_rows,
+                                              float* csum) {
+    const int lane = threadIdx.x & 31, quarter = (threadIdx.x >> 5) & 3;
     __syncwarp();
     const int lrow = lane >> 3, lseg = lane & 7;
 #pragma unroll
@@ -472,68 +480,109 @@ __device__ __forceinline__ void store_rows_64(uint8_t* stage, int r, const float
     __syncwarp();
 }
 
-constexpr int DKV_STAGES = 6;   // Q/dO ring deep enough to cover a ~1.3 us tile load
-struct CtlDkv {
-    uint64_t kv_full;
-    uint64_t q_full[DKV_STAGES], q_empty[DKV_STAGES];
-    uint64_t st_full[2], st_empty[2];
-    uint64_t ew_done[2];
-    uint64_t kv_tmem;                            // K and V copied into TMEM (A operands)
-    uint64_t acc_done;
+constexpr int BW_EW_WARPS = 8;         // 2 per TMEM lane quarter, 64 query columns each (two chunks of 32)
+constexpr int BW_DR_WARPS = 4;         // dQ drain and dK/dV write-out: one per TMEM lane quarter
+constexpr int BW_THREADS = 64 + 32 * (BW_EW_WARPS + BW_DR_WARPS);
+constexpr int BW_STAGES = 3;           // Q/dO ring
+constexpr int BW_ITEM_READERS = 1 + BW_EW_WARPS + BW_DR_WARPS;   // MMA thread, element-wise and drain warps
+struct CtlBwd {
+    uint64_t item_full[2], item_empty[2];            // work-item ring, filled by the producer warp
+    uint64_t kv_full[2], kv_empty[2];                // K and V of the item in ring slot s
+    uint64_t q_full[BW_STAGES], q_empty[BW_STAGES];  // Q, dO, lse and D of one query tile
+    uint64_t st_full, st_empty;                      // S^T and dP^T in TMEM: computed / copied to registers
+    uint64_t ew_done;                                // P^T (TMEM) and dS^T (shared memory) written
+    uint64_t pt_free;                                // a pair's dV MMAs done: P^T reusable
+    uint64_t ds_free;                                // a pair's dK, dQ MMAs done: dS^T reusable
+    uint64_t dq_full, dq_empty;                      // a pair's dQ in TMEM: computed / copied to registers
+    uint64_t acc_done, dkv_free;                     // an item's dK, dV complete in TMEM / copied out
     uint64_t drain;
     uint32_t tmem_base;
     uint32_t abort;
-    alignas(16) float lse2[2][64];   // negated, log2 units (read as float2 pairs)
-    alignas(16) float dd[2][64];     // negated D
+    int item[2];
 };
-// smem: K | V | (Q | dO) stages | output staging | ctl
-constexpr int DKV_OFF_K = 0;
-constexpr int DKV_OFF_V = DKV_OFF_K + T128_BYTES;
-constexpr int DKV_OFF_Q = DKV_OFF_V + T128_BYTES;
-constexpr int DKV_STAGE_BYTES = 2 * T64_BYTES;                  // Q tile + dO tile
-constexpr int DKV_OFF_STAGE = DKV_OFF_Q + DKV_STAGES * DKV_STAGE_BYTES;   // dK / dV output staging
-constexpr int DKV_OFF_CTL = DKV_OFF_STAGE + T128_BYTES;
-constexpr size_t DKV_SMEM = DKV_OFF_CTL + sizeof(CtlDkv) + 1024;
-// TMEM columns
-// TMEM columns: S^T and dP^T (fp32, double-buffered; after the element-wise step
-// the first 16 columns of each 32-column half hold that half's P^T / dS^T as
-// packed bf16, the A operand of the dV / dK MMAs), the dV and dK accumulators,
-// and K and V as packed bf16 A operands of the S^T and dP^T MMAs.
-constexpr uint32_t DKV_ST = 0, DKV_DPT = 128, DKV_DV = 256, DKV_DK = 320, DKV_KT = 384, DKV_VT = 416;
+// smem: K/V (2 ring slots) | stages x (Q | dO) | dS^T (two 64-query atoms) |
+//       staging (per drain warp 32 rows x 128 bytes) | stages x (-lse log2(e) | -D) | ctl
+constexpr int BW_KV_BYTES = 2 * T128_BYTES;
+constexpr int BW_STAGE_BYTES = 2 * T128_BYTES;
+constexpr int BW_DS_BYTES = 2 * T128_BYTES;
+constexpr int BW_OFF_KV = 0;
+constexpr int BW_OFF_Q = 2 * BW_KV_BYTES;
+constexpr int BW_OFF_DS = BW_OFF_Q + BW_STAGES * BW_STAGE_BYTES;
+constexpr int BW_OFF_STG = BW_OFF_DS + BW_DS_BYTES;
+constexpr int BW_OFF_LSE = BW_OFF_STG + T128_BYTES;  // per stage: 128 floats of -lse log2(e), 128 of -D
+constexpr int BW_OFF_CTL = BW_OFF_LSE + BW_STAGES * 1024;
+constexpr size_t BW_SMEM = BW_OFF_CTL + sizeof(CtlBwd) + 1024;
+// TMEM columns: S^T, dP^T (fp32, 128 queries each), P^T (packed bf16: 128
+// queries in 64 columns), the dV and dK accumulators, the pair's dQ.
+constexpr uint32_t BW_ST = 0, BW_DPT = 128, BW_PT = 256, BW_DV = 320, BW_DK = 384, BW_DQ = 448;
 
+// Work item i (longest first): key tile i / BH of head-sequence i % BH; its
+// query tiles are kt .. n_qt - 1.
+struct BwItem {
+    int bh, kt, n_it;
+};
+__device__ __forceinline__ BwItem bw_item(int i, int BH, int n_qt) {
+    BwItem w;
+    w.kt = i / BH;
+    w.bh = i - w.kt * BH;
+    w.n_it = n_qt - w.kt;
+    return w;
+}
+// Item of ring slot ictr & 1 (waits for the producer, then frees the slot for
+// this reader): the item index, -1 when the work is done, -2 after a failed wait.
+__device__ __forceinline__ int bw_read_item(CtlBwd* ctl, uint32_t ictr, volatile uint32_t* abort, unsigned* status) {
+    const int s = ictr & 1;
+    if (!tc::mbar_wait(&ctl->item_full[s], (ictr >> 1) & 1, abort, status)) return -2;
+    const int item = *reinterpret_cast<volatile int*>(&ctl->item[s]);
+    tc::mbar_arrive(&ctl->item_empty[s]);
+    return item;
+}
+// The same for a warp: lane 0 reads, every lane gets the value.
+__device__ __forceinline__ int bw_read_item_warp(CtlBwd* ctl, uint32_t ictr, volatile uint32_t* abort,
+                                                 unsigned* status) {
+    int item = 0;
+    if ((threadIdx.x & 31) == 0) item = bw_read_item(ctl, ictr, abort, status);
+    return __shfl_sync(0xffffffffu, item, 0);
+}
+
+// Persistent: gridDim.x CTAs (at most one per SM) take work items in order
+// from the counter *work (zeroed by the pre-pass); the producer warp fetches
+// the next item's K, V and first query tiles while the current one runs, and
+// every ring and barrier parity runs on counters over all of the CTA's pairs.
 __global__ void __launch_bounds__(BW_THREADS, 1)
-    flash_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q,
-                            const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ lse,
-                            const float* __restrict__ dpre, bf16* __restrict__ dqkv, int Tn, int H,
-                            float* __restrict__ colsum_part, unsigned* status) {
+    flash_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
+                        const __grid_constant__ CUtensorMap tm_dq, const float* __restrict__ lse,
+                        const float* __restrict__ dpre, bf16* __restrict__ dqkv, int Tn, int H, int BH,
+                        int* __restrict__ work, float* __restrict__ colsum_part, unsigned* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    CtlDkv* ctl = reinterpret_cast<CtlDkv*>(smem + DKV_OFF_CTL);
+    CtlBwd* ctl = reinterpret_cast<CtlBwd*>(smem + BW_OFF_CTL);
     volatile uint32_t* abort = &ctl->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // grid (B H, key tiles): key tile 0 sees the most queries and is dispatched first
-    const int kt = blockIdx.y;
-    const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const int C = H * HD;
-    const int k0 = kt * 128;
-    const int n_q64 = (Tn + 63) / 64;
-    const int it0 = k0 / 64;                            // first 64-query tile that sees these keys
-    const int n_it = n_q64 - it0;
-    const int row_base = b * Tn;
+    const int n_qt = (Tn + 127) / 128;
+    const int n_items = BH * n_qt;
 
     if (threadIdx.x == 0) {
-        tc::mbar_init(&ctl->kv_full, 1);
-        for (int s = 0; s < DKV_STAGES; ++s) {
-            tc::mbar_init(&ctl->q_full[s], 1);
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&ctl->item_full[i], 1);
+            tc::mbar_init(&ctl->item_empty[i], BW_ITEM_READERS);
+            tc::mbar_init(&ctl->kv_full[i], 1);
+            tc::mbar_init(&ctl->kv_empty[i], 1);
+        }
+        for (int s = 0; s < BW_STAGES; ++s) {
+            tc::mbar_init(&ctl->q_full[s], 2);   // the TMA bytes, and the producer's lse / D stores
             tc::mbar_init(&ctl->q_empty[s], 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&ctl->st_full[i], 1);
-            tc::mbar_init(&ctl->st_empty[i], BW_EW_WARPS);
-            tc::mbar_init(&ctl->ew_done[i], BW_EW_WARPS);
-        }
-        tc::mbar_init(&ctl->kv_tmem, BW_EW_WARPS);
+        tc::mbar_init(&ctl->st_full, 1);
+        tc::mbar_init(&ctl->st_empty, BW_EW_WARPS);
+        tc::mbar_init(&ctl->ew_done, BW_EW_WARPS);
+        tc::mbar_init(&ctl->pt_free, 1);
+        tc::mbar_init(&ctl->ds_free, 1);
+        tc::mbar_init(&ctl->dq_full, 1);
+        tc::mbar_init(&ctl->dq_empty, BW_DR_WARPS);
         tc::mbar_init(&ctl->acc_done, 1);
+        tc::mbar_init(&ctl->dkv_free, BW_DR_WARPS);
         tc::mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
         tc::fence_barrier_init();
@@ -548,390 +597,470 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
     const uint32_t tmem = ctl->tmem_base;
 
     if (warp == 0) {
+        // -------------------------------------------------------------- producer
+        // lane 0 takes items and issues the TMA loads; all 32 lanes stage each
+        // query tile's lse (negated, log2 units) and D (negated) next to it.
         if (lane == 0) {
-            tc::tma_prefetch_desc(&tm_kv);
-            tc::tma_prefetch_desc(&tm_q);
+            tc::tma_prefetch_desc(&tm_qkv);
             tc::tma_prefetch_desc(&tm_do);
-            tc::mbar_expect_tx(&ctl->kv_full, 2 * T128_BYTES);
-            tc::tma_load_2d(smem + DKV_OFF_K, &tm_kv, C + h * HD, row_base + k0, &ctl->kv_full);
-            tc::tma_load_2d(smem + DKV_OFF_V, &tm_kv, 2 * C + h * HD, row_base + k0, &ctl->kv_full);
-            for (int it = 0; it < n_it; ++it) {
-                const int s = it % DKV_STAGES;
-                if (!tc::mbar_wait(&ctl->q_empty[s], ((it / DKV_STAGES) & 1) ^ 1, abort, status)) break;
-                const int q0 = (it0 + it) * 64;
-                uint8_t* st = smem + DKV_OFF_Q + s * DKV_STAGE_BYTES;
-                tc::mbar_expect_tx(&ctl->q_full[s], 2 * T64_BYTES);
-                tc::tma_load_2d(st, &tm_q, h * HD, row_base + q0, &ctl->q_full[s]);
-                tc::tma_load_2d(st + T64_BYTES, &tm_do, h * HD, row_base + q0, &ctl->q_full[s]);
+            tc::tma_prefetch_desc(&tm_dq);
+        }
+        uint32_t ictr = 0, g = 0;
+        for (;;) {
+            const int s = ictr & 1;
+            const uint32_t ph = (ictr >> 1) & 1;
+            int item = -2;
+            if (lane == 0 && tc::mbar_wait(&ctl->item_empty[s], ph ^ 1, abort, status)) {
+                const int i = atomicAdd(work, 1);
+                item = i < n_items ? i : -1;
+                ctl->item[s] = item;
+                tc::mbar_arrive(&ctl->item_full[s]);
             }
+            item = __shfl_sync(0xffffffffu, item, 0);
+            if (item < 0) break;
+            const BwItem w = bw_item(item, BH, n_qt);
+            const int b = w.bh / H, h = w.bh % H, row_base = b * Tn;
+            // lse (negated, log2 units) and D (negated) of one query tile, 4 queries per
+            // lane, loaded one tile ahead of their stage so that their latency overlaps
+            // the wait for the stage
+            float nl[4], nd[4];
+            auto fetch = [&](int it) {
+                const int q0 = (w.kt + it) * 128;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int q = q0 + lane + 32 * j;
+                    nl[j] = q < Tn ? lse[(long long)w.bh * Tn + q] : INFINITY;
+                    nd[j] = q < Tn ? dpre[(long long)w.bh * Tn + q] : 0.f;
+                }
+            };
+            fetch(0);
+            uint32_t ok = 0;
+            if (lane == 0 && tc::mbar_wait(&ctl->kv_empty[s], ph ^ 1, abort, status)) {
+                uint8_t* kv = smem + BW_OFF_KV + s * BW_KV_BYTES;
+                tc::mbar_expect_tx(&ctl->kv_full[s], 2 * T128_BYTES);
+                tc::tma_load_2d(kv, &tm_qkv, C + h * HD, row_base + w.kt * 128, &ctl->kv_full[s]);
+                tc::tma_load_2d(kv + T128_BYTES, &tm_qkv, 2 * C + h * HD, row_base + w.kt * 128, &ctl->kv_full[s]);
+                ok = 1;
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);   // every exit of this loop is taken by the whole warp
+            if (!ok) break;
+            ++ictr;
+            for (int it = 0; it < w.n_it; ++it, ++g) {
+                const int st = g % BW_STAGES;
+                const int q0 = (w.kt + it) * 128;
+                uint8_t* stg = smem + BW_OFF_Q + st * BW_STAGE_BYTES;
+                ok = 0;
+                if (lane == 0 && tc::mbar_wait(&ctl->q_empty[st], ((g / BW_STAGES) & 1) ^ 1, abort, status)) {
+                    tc::mbar_expect_tx(&ctl->q_full[st], 2 * T128_BYTES);
+                    tc::tma_load_2d(stg, &tm_qkv, h * HD, row_base + q0, &ctl->q_full[st]);
+                    tc::tma_load_2d(stg + T128_BYTES, &tm_do, h * HD, row_base + q0, &ctl->q_full[st]);
+                    ok = 1;
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                float* sl = reinterpret_cast<float*>(smem + BW_OFF_LSE + st * 1024);
+                float* sd = sl + 128;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    sl[lane + 32 * j] = -nl[j] * LOG2E;   // a query past the sequence: -inf, so P = 0
+                    sd[lane + 32 * j] = -nd[j];
+                }
+                if (it + 1 < w.n_it) fetch(it + 1);
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&ctl->q_full[st]);
+            }
+            if (!ok) break;
+        }
+        // before the CTA exits, every load it issued has landed (bounded; at once normally)
+        if (lane == 0) {
+            volatile uint32_t no_abort = 0;
+            for (uint32_t x = ictr > 2 ? ictr - 2 : 0; x < ictr; ++x)
+                tc::mbar_wait(&ctl->kv_full[x & 1], (x >> 1) & 1, &no_abort, status);
+            for (uint32_t x = g > BW_STAGES ? g - BW_STAGES : 0; x < g; ++x)
+                tc::mbar_wait(&ctl->q_full[x % BW_STAGES], (x / BW_STAGES) & 1, &no_abort, status);
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc_st = tc::idesc_bf16_f32(128, 64, 0, 0);   // K Q^T, V dO^T
+            // ------------------------------------------------------------------- MMA
+            constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128, 0, 0);   // K Q^T, V dO^T
             constexpr uint32_t idesc_acc = tc::idesc_bf16_f32(128, 64, 0, 1);  // P^T dO, dS^T Q
-            bool ok = tc::mbar_wait(&ctl->kv_tmem, 0, abort, status);
-            auto accumulate = [&](int it) -> bool {   // dV += P^T dO, dK += dS^T Q for tile it
-                const int r = it & 1, s = it % DKV_STAGES;
-                if (!tc::mbar_wait(&ctl->ew_done[r], (it >> 1) & 1, abort, status)) return false;
-                tc::fence_after_sync();
-                const uint32_t q_addr = tc::smem_u32(smem + DKV_OFF_Q + s * DKV_STAGE_BYTES);
-                const uint32_t do_addr = q_addr + T64_BYTES;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {   // K = 64 queries: 16 per MMA, 8 packed columns
-                    const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    const uint32_t col = r * 64 + (kk >> 1) * 32 + (kk & 1) * 8;
-                    tc::mma_bf16_ts(tmem + DKV_DV, tmem + DKV_ST + col,
-                                    tc::smem_desc_sw128(do_addr + kk * 2048, T64_BYTES, 1024), idesc_acc, acc);
-                    tc::mma_bf16_ts(tmem + DKV_DK, tmem + DKV_DPT + col,
-                                    tc::smem_desc_sw128(q_addr + kk * 2048, T64_BYTES, 1024), idesc_acc, acc);
-                }
-                tc::mma_commit(&ctl->q_empty[s]);
-                return true;
+            constexpr uint32_t idesc_dq = tc::idesc_bf16_f32(128, 64, 1, 1);   // dS K (dS from the dS^T tile)
+            // Shared-memory descriptors, built once: the start address sits in the low bits
+            // (address >> 4), so stepping inside a tile adds (byte offset >> 4).
+            const uint32_t kv0 = tc::smem_u32(smem + BW_OFF_KV), q_base = tc::smem_u32(smem + BW_OFF_Q);
+            const uint64_t d_ds_k = tc::smem_desc_sw128(tc::smem_u32(smem + BW_OFF_DS), 16, 1024);
+            const uint64_t d_ds_mn = tc::smem_desc_sw128(tc::smem_u32(smem + BW_OFF_DS), T128_BYTES, 1024);
+            auto kdesc_k = [&](int slot) { return tc::smem_desc_sw128(kv0 + slot * BW_KV_BYTES, 16, 1024); };
+            auto kdesc_mn = [&](int slot) {
+                return tc::smem_desc_sw128(kv0 + slot * BW_KV_BYTES, T128_BYTES, 1024);
             };
-            for (int it = 0; it < n_it && ok; ++it) {
-                const int r = it & 1, s = it % DKV_STAGES;
-                if (!tc::mbar_wait(&ctl->q_full[s], (it / DKV_STAGES) & 1, abort, status)) break;
-                if (!tc::mbar_wait(&ctl->st_empty[r], ((it >> 1) & 1) ^ 1, abort, status)) break;
+            auto qdesc_k = [&](int st) { return tc::smem_desc_sw128(q_base + st * BW_STAGE_BYTES, 16, 1024); };
+            auto qdesc_mn = [&](int st) {
+                return tc::smem_desc_sw128(q_base + st * BW_STAGE_BYTES, T128_BYTES, 1024);
+            };
+            constexpr uint64_t TILE16 = T128_BYTES >> 4;   // descriptor step of one 16 KB tile
+            // S^T and dP^T of pair g (query tile stage g % STAGES) against K/V slot `slot`
+            auto issue_sdp = [&](uint32_t g, int slot) -> bool {
+                const int st = g % BW_STAGES;
+                if (!tc::mbar_wait(&ctl->q_full[st], (g / BW_STAGES) & 1, abort, status)) return false;
                 tc::fence_after_sync();
-                const uint32_t q_addr = tc::smem_u32(smem + DKV_OFF_Q + s * DKV_STAGE_BYTES);
-                const uint32_t do_addr = q_addr + T64_BYTES;
+                const uint64_t dk = kdesc_k(slot), dq = qdesc_k(st);
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
-                    tc::mma_bf16_ts(tmem + DKV_ST + r * 64, tmem + DKV_KT + kk * 8,
-                                    tc::smem_desc_sw128(q_addr + kk * 32, 16, 1024), idesc_st, kk > 0 ? 1u : 0u);
-                    tc::mma_bf16_ts(tmem + DKV_DPT + r * 64, tmem + DKV_VT + kk * 8,
-                                    tc::smem_desc_sw128(do_addr + kk * 32, 16, 1024), idesc_st, kk > 0 ? 1u : 0u);
+                    tc::mma_bf16(tmem + BW_ST, dk + 2 * kk, dq + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
+                    tc::mma_bf16(tmem + BW_DPT, dk + TILE16 + 2 * kk, dq + TILE16 + 2 * kk, idesc_s,
+                                 kk > 0 ? 1u : 0u);
                 }
-                tc::mma_commit(&ctl->st_full[r]);
-                if (it > 0 && !accumulate(it - 1)) { ok = false; break; }
+                tc::mma_commit(&ctl->st_full);
+                return true;
+            };
+            uint32_t ictr = 0, g = 0;
+            int item = bw_read_item(ctl, ictr, abort, status);
+            BwItem cur = bw_item(item < 0 ? 0 : item, BH, n_qt);
+            int it = 0;
+            bool ok = item >= 0 && tc::mbar_wait(&ctl->kv_full[0], 0, abort, status) && issue_sdp(0, 0);
+            while (ok) {
+                const int st = g % BW_STAGES, slot = ictr & 1;
+                const uint32_t par = g & 1;
+                // the next pair: the next query tile, or the first of the next item
+                bool has_next = it + 1 < cur.n_it;
+                uint32_t nictr = ictr;
+                BwItem nxt = cur;
+                if (!has_next) {
+                    nictr = ictr + 1;
+                    const int ni = bw_read_item(ctl, nictr, abort, status);
+                    if (ni == -2) break;
+                    has_next = ni >= 0;
+                    if (has_next) nxt = bw_item(ni, BH, n_qt);
+                }
+                if (has_next) {   // its S^T / dP^T once this pair's are in registers
+                    if (!tc::mbar_wait(&ctl->st_empty, par, abort, status)) break;
+                    if (nictr != ictr && !tc::mbar_wait(&ctl->kv_full[nictr & 1], (nictr >> 1) & 1, abort, status))
+                        break;
+                    if (!issue_sdp(g + 1, nictr & 1)) break;
+                }
+                if (!tc::mbar_wait(&ctl->ew_done, par, abort, status)) break;
+                tc::fence_after_sync();
+                const uint64_t dmn = qdesc_mn(st);
+                const uint64_t kmn = kdesc_mn(slot);
+                // dQ = dS K: K = 128 keys in steps of 16; A is the dS^T tile read as an MN-major
+                // (query-contiguous) operand, the next 64 queries one atom (16 KB) further
+                auto issue_dq = [&]() -> bool {
+                    if (!tc::mbar_wait(&ctl->dq_empty, par ^ 1, abort, status)) return false;
+                    tc::fence_after_sync();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_bf16(tmem + BW_DQ, d_ds_mn + 128 * kk, kmn + 128 * kk, idesc_dq, kk > 0 ? 1u : 0u);
+                    tc::mma_commit(&ctl->dq_full);
+                    return true;
+                };
+                // The first pair of an item overwrites dV / dK, so it waits for the last item's
+                // to be copied out; its dQ, which needs neither, goes first.
+                if (it == 0) {
+                    if (!issue_dq()) break;
+                    if (!tc::mbar_wait(&ctl->dkv_free, (ictr & 1) ^ 1, abort, status)) break;
+                    tc::fence_after_sync();
+                }
+                // dV += P^T dO, then dK += dS^T Q: K = 128 queries in steps of 16
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16_ts(tmem + BW_DV, tmem + BW_PT + kk * 8, dmn + TILE16 + 128 * kk, idesc_acc,
+                                    (it > 0 || kk > 0) ? 1u : 0u);
+                tc::mma_commit(&ctl->pt_free);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16(tmem + BW_DK, d_ds_k + (kk >> 2) * TILE16 + 2 * (kk & 3), dmn + 128 * kk, idesc_acc,
+                                 (it > 0 || kk > 0) ? 1u : 0u);
+                tc::mma_commit(&ctl->q_empty[st]);
+                if (it > 0 && !issue_dq()) break;
+                tc::mma_commit(&ctl->ds_free);
+                if (it + 1 == cur.n_it) {
+                    tc::mma_commit(&ctl->kv_empty[slot]);
+                    tc::mma_commit(&ctl->acc_done);
+                }
+                if (!has_next) break;
+                if (nictr != ictr) {
+                    ictr = nictr;
+                    cur = nxt;
+                    it = 0;
+                } else {
+                    ++it;
+                }
+                ++g;
             }
-            if (ok && n_it > 0) ok = accumulate(n_it - 1);
-            tc::mma_commit(&ctl->acc_done);
             volatile uint32_t no_abort = 0;
             tc::mma_commit(&ctl->drain);
             tc::mbar_wait(&ctl->drain, 0, &no_abort, status);
         }
-    } else {
-        // ------------------------------------------- P^T, dS^T (thread = key row)
+    } else if (warp < 2 + BW_EW_WARPS) {
+        // --------------------------------------------- P^T, dS^T (thread = key row)
         const int quarter = warp & 3;
-        const int chalf = (warp - 2) >> 2;              // query columns [32 chalf, 32 chalf + 32)
+        const int chalf = (warp - 2) >> 2;              // query columns [64 chalf, 64 chalf + 64)
         const int r = quarter * 32 + lane;              // key row in the tile = TMEM lane
-        const int key = k0 + r;
-        const int et = threadIdx.x - 64;                // 0..255 within the element-wise warps
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const float sl2 = LOG2E * 0.125f;
-        // per-query lse (log2 units) and D of the next tile, one value per thread
-        // stored negated, the form the packed exponent and dS arithmetic take
-        auto fetch = [&](int it) -> float {
-            const int q = (it0 + it) * 64 + (et & 63);
-            if (et < 64) return q < Tn ? -lse[(long long)bh * Tn + q] * LOG2E : -INFINITY;
-            if (et < 128) return q < Tn ? -dpre[(long long)bh * Tn + q] : 0.f;
-            return 0.f;
-        };
-        // two tiles of lookahead: a global load's latency exceeds one tile's work
-        float nxt = n_it > 0 ? fetch(0) : 0.f;
-        float nxt2 = n_it > 1 ? fetch(1) : 0.f;
-        bool ok = true;
-        {
-            // K and V rows into TMEM as the packed bf16 A operands of the S^T and dP^T MMAs:
-            // this thread's key row, head columns [32 chalf, 32 chalf + 32) = 16 columns
-            uint32_t w = 0;
-            if (lane == 0) w = tc::mbar_wait(&ctl->kv_full, 0, abort, status) ? 1u : 0u;
-            w = __shfl_sync(0xffffffffu, w, 0);
-            if (w) {
-                uint32_t kw[16], vw[16];
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const uint4 kq = *reinterpret_cast<const uint4*>(smem + DKV_OFF_K + swz128(r, chalf * 4 + g));
-                    const uint4 vq = *reinterpret_cast<const uint4*>(smem + DKV_OFF_V + swz128(r, chalf * 4 + g));
-                    kw[4 * g] = kq.x; kw[4 * g + 1] = kq.y; kw[4 * g + 2] = kq.z; kw[4 * g + 3] = kq.w;
-                    vw[4 * g] = vq.x; vw[4 * g + 1] = vq.y; vw[4 * g + 2] = vq.z; vw[4 * g + 3] = vq.w;
-                }
-                tc::tmem_st_32x32b_x16(tmem + DKV_KT + chalf * 16 + lane_off, kw);
-                tc::tmem_st_32x32b_x16(tmem + DKV_VT + chalf * 16 + lane_off, vw);
-                tc::tmem_wait_st();
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&ctl->kv_tmem);
-            } else {
-                ok = false;
-            }
-        }
-        for (int it = 0; it < n_it; ++it) {
-            const int rb = it & 1;
-            const int q0 = (it0 + it) * 64;
-            if (et < 64) ctl->lse2[rb][et] = nxt;
-            else if (et < 128) ctl->dd[rb][et - 64] = nxt;
-            ew_bar();
-            nxt = nxt2;
-            if (it + 2 < n_it) nxt2 = fetch(it + 2);
-            uint32_t w = 0;
-            // st_full also means every earlier MMA is done, among them the dV/dK MMAs that
-            // read this buffer's P^T / dS^T two tiles ago
-            if (lane == 0 && ok) w = tc::mbar_wait(&ctl->st_full[rb], (it >> 1) & 1, abort, status) ? 1u : 0u;
-            w = __shfl_sync(0xffffffffu, w, 0);
-            // after a failed wait keep looping without work, so that every
-            // element-wise warp reaches the named barrier equally often
-            if (!w) { ok = false; continue; }
-            tc::fence_after_sync();
-            const bool diag = (q0 < k0 + 128);          // some queries of the tile precede some keys
-            float sv[32], dp[32];
-            tc::tmem_ld2_32x32b_x32(tmem + DKV_ST + rb * 64 + chalf * 32 + lane_off,
-                                    tmem + DKV_DPT + rb * 64 + chalf * 32 + lane_off, sv, dp);
-            // P^T = 2^(s sl2 - lse2), dS^T = P^T (dP^T - D) on packed pairs of queries
+        const int qa = chalf * 64;
+        // P^T = 2^(s sl2 - lse2), dS^T = P^T (dP^T - D) for the 32 queries from qc, in
+        // place (sv becomes P^T, dp becomes dS^T), packed to bf16 pairs
+        auto ew_chunk = [&](float* sv, float* dp, const float* sl, const float* sd, int qc, bool diag, uint32_t* pw,
+                            uint32_t* dw) {
             const f32x2 SL = pk2(sl2, sl2);
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-                const int qi = chalf * 32 + e;
-                const float2 nl = *reinterpret_cast<const float2*>(&ctl->lse2[rb][qi]);
-                const float2 nd = *reinterpret_cast<const float2*>(&ctl->dd[rb][qi]);
-                float t0, t1;
+            for (int e = 0; e < 32; e += 4) {
+                const float4 nl = *reinterpret_cast<const float4*>(sl + qc + e);
+                const float4 nd = *reinterpret_cast<const float4*>(sd + qc + e);
+                float t0, t1, t2, t3;
                 upk2(fma2(pk2(sv[e], sv[e + 1]), SL, pk2(nl.x, nl.y)), t0, t1);
+                upk2(fma2(pk2(sv[e + 2], sv[e + 3]), SL, pk2(nl.z, nl.w)), t2, t3);
                 sv[e] = ex2(t0);
                 sv[e + 1] = ex2(t1);
-                if (diag) {   // queries before this key
-                    if (key > q0 + qi) sv[e] = 0.f;
-                    if (key > q0 + qi + 1) sv[e + 1] = 0.f;
+                sv[e + 2] = ex2(t2);
+                sv[e + 3] = ex2(t3);
+                if (diag) {   // queries before this key (the diagonal pair: q0 = k0)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (r > qc + e + j) sv[e + j] = 0.f;
                 }
                 upk2(mul2(pk2(sv[e], sv[e + 1]), add2(pk2(dp[e], dp[e + 1]), pk2(nd.x, nd.y))), dp[e], dp[e + 1]);
+                upk2(mul2(pk2(sv[e + 2], sv[e + 3]), add2(pk2(dp[e + 2], dp[e + 3]), pk2(nd.z, nd.w))), dp[e + 2],
+                     dp[e + 3]);
             }
-            // P^T and dS^T as packed bf16 over the first 16 columns of this warp's S^T / dP^T half
-            uint32_t pw[16], dw[16];
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                const uint4 a = pack8_bf16(sv + 8 * g), d = pack8_bf16(dp + 8 * g);
-                pw[4 * g] = a.x; pw[4 * g + 1] = a.y; pw[4 * g + 2] = a.z; pw[4 * g + 3] = a.w;
-                dw[4 * g] = d.x; dw[4 * g + 1] = d.y; dw[4 * g + 2] = d.z; dw[4 * g + 3] = d.w;
+            for (int gq = 0; gq < 4; ++gq) {
+                const uint4 a = pack8_bf16(sv + 8 * gq), d = pack8_bf16(dp + 8 * gq);
+                pw[4 * gq] = a.x; pw[4 * gq + 1] = a.y; pw[4 * gq + 2] = a.z; pw[4 * gq + 3] = a.w;
+                dw[4 * gq] = d.x; dw[4 * gq + 1] = d.y; dw[4 * gq + 2] = d.z; dw[4 * gq + 3] = d.w;
             }
-            tc::tmem_st_32x32b_x16(tmem + DKV_ST + rb * 64 + chalf * 32 + lane_off, pw);
-            tc::tmem_st_32x32b_x16(tmem + DKV_DPT + rb * 64 + chalf * 32 + lane_off, dw);
+        };
+        uint32_t ictr = 0, g = 0;
+        int item = bw_read_item_warp(ctl, ictr, abort, status);
+        BwItem cur = bw_item(item < 0 ? 0 : item, BH, n_qt);
+        int it = 0;
+        while (item >= 0) {
+            const int st = g % BW_STAGES;
+            const uint32_t par = g & 1;
+            uint32_t w = 0;
+            if (lane == 0) w = tc::mbar_wait(&ctl->st_full, par, abort, status) ? 1u : 0u;
+            if (!__shfl_sync(0xffffffffu, w, 0)) break;
+            // the producer's lse / D stores of this stage (complete long before S^T is);
+            // every lane acquires them, and the warp leaves together if one lane's wait fails
+            w = tc::mbar_wait(&ctl->q_full[st], (g / BW_STAGES) & 1, abort, status) ? 1u : 0u;
+            if (!__all_sync(0xffffffffu, w)) break;
+            tc::fence_after_sync();
+            const float* sl = reinterpret_cast<const float*>(smem + BW_OFF_LSE + st * 1024);
+            const float* sd = sl + 128;
+            const bool diag = (it == 0);
+            uint8_t* ds_tile = smem + BW_OFF_DS + chalf * T128_BYTES;
+            bool fail = false;
+            uint32_t dw0[16];   // dS^T of chunk 0, kept until the previous pair's dK / dQ MMAs are done
+#pragma unroll 1
+            for (int c = 0; c < 2; ++c) {
+                float sv[32], dp[32];
+                uint32_t pw[16], dw[16];
+                tc::tmem_ld2_32x32b_x32(tmem + BW_ST + qa + 32 * c + lane_off, tmem + BW_DPT + qa + 32 * c + lane_off,
+                                        sv, dp);
+                if (c == 1) {   // S^T and dP^T are in registers: the next pair's MMAs may overwrite them
+                    tc::fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&ctl->st_empty);
+                }
+                ew_chunk(sv, dp, sl, sd, qa + 32 * c, diag, pw, dw);
+                // P^T's TMEM columns: the previous pair's dV MMAs are done (chunk 0 waits)
+                if (c == 0) {
+                    if (lane == 0) w = tc::mbar_wait(&ctl->pt_free, par ^ 1, abort, status) ? 1u : 0u;
+                    if (!__shfl_sync(0xffffffffu, w, 0)) { fail = true; break; }
+                    tc::fence_after_sync();
+                }
+                tc::tmem_st_32x32b_x16(tmem + BW_PT + chalf * 32 + 16 * c + lane_off, pw);
+                if (c == 0) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) dw0[j] = dw[j];
+                } else {
+                    // dS^T: the previous pair's dK / dQ MMAs are done
+                    if (lane == 0) w = tc::mbar_wait(&ctl->ds_free, par ^ 1, abort, status) ? 1u : 0u;
+                    if (!__shfl_sync(0xffffffffu, w, 0)) { fail = true; break; }
+                    tc::fence_after_sync();
+#pragma unroll
+                    for (int gq = 0; gq < 4; ++gq) {
+                        *reinterpret_cast<uint4*>(ds_tile + swz128(r, gq)) =
+                            make_uint4(dw0[4 * gq], dw0[4 * gq + 1], dw0[4 * gq + 2], dw0[4 * gq + 3]);
+                        *reinterpret_cast<uint4*>(ds_tile + swz128(r, 4 + gq)) =
+                            make_uint4(dw[4 * gq], dw[4 * gq + 1], dw[4 * gq + 2], dw[4 * gq + 3]);
+                    }
+                }
+            }
+            if (fail) break;
             tc::tmem_wait_st();
+            tc::fence_proxy_async_smem();      // dS^T visible to the tensor core
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) {
-                tc::mbar_arrive(&ctl->st_empty[rb]);
-                tc::mbar_arrive(&ctl->ew_done[rb]);
+            if (lane == 0) tc::mbar_arrive(&ctl->ew_done);
+            ++g;
+            if (++it == cur.n_it) {
+                item = bw_read_item_warp(ctl, ++ictr, abort, status);
+                if (item >= 0) cur = bw_item(item, BH, n_qt);
+                it = 0;
             }
         }
-        if (ok && chalf == 0) {
+    } else {
+        // ------------------------------- dQ drain, dK / dV write-out (thread = row)
+        // Each warp moves its own 32 rows through its own 4 KB of staging: dQ as two
+        // fp32 32 x 32 boxes added into the accumulator by this warp's TMA reduce,
+        // then at an item's end dK and dV as bf16 rows. No barrier spans warps.
+        const int quarter = warp & 3;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const int r = quarter * 32 + lane;
+        uint8_t* stage = smem + BW_OFF_STG;                   // 128 rows x 128 bytes
+        uint8_t* mine = stage + quarter * 4096;               // this warp's rows
+        uint32_t ictr = 0, g = 0;
+        int item = bw_read_item_warp(ctl, ictr, abort, status);
+        BwItem cur = bw_item(item < 0 ? 0 : item, BH, n_qt);
+        int it = 0;
+        while (item >= 0) {
+            const int b = cur.bh / H, h = cur.bh % H, row_base = b * Tn, k0 = cur.kt * 128;
+            const int q0 = (cur.kt + it) * 128;
             uint32_t w = 0;
-            if (lane == 0) w = tc::mbar_wait(&ctl->acc_done, 0, abort, status) ? 1u : 0u;
-            w = __shfl_sync(0xffffffffu, w, 0);
-            if (w) {
+            if (lane == 0) w = tc::mbar_wait(&ctl->dq_full, g & 1, abort, status) ? 1u : 0u;
+            if (!__shfl_sync(0xffffffffu, w, 0)) break;
+            tc::fence_after_sync();
+            const bool live = q0 + quarter * 32 < Tn;          // rows past the sequence add nothing
+            // dQ in two 32-column halves: each a fp32 box of 32 rows x 32 columns (128-byte
+            // swizzle) added into the accumulator; dQ = dS K / sqrt(64). The TMEM columns
+            // are free once the second half is in registers.
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float v[32];
+                tc::tmem_ld_32x32b_x32(tmem + BW_DQ + 32 * half + lane_off, v);
+                if (half == 1) {
+                    tc::fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&ctl->dq_empty);
+                }
+                if (lane == 0) tc::bulk_wait_read<0>();       // this warp's last reduce has read the staging
+                __syncwarp();
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc)
+                    *reinterpret_cast<float4*>(mine + swz128(lane, cc)) =
+                        make_float4(v[4 * cc] * 0.125f, v[4 * cc + 1] * 0.125f, v[4 * cc + 2] * 0.125f,
+                                    v[4 * cc + 3] * 0.125f);
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && live) {
+                    tc::tma_reduce_add_2d(&tm_dq, mine, h * HD + 32 * half, row_base + q0 + quarter * 32);
+                    tc::bulk_commit();
+                }
+            }
+            ++g;
+            if (++it == cur.n_it) {
+                // the item's dK, dV: TMEM -> bf16 rows (+ column sums), then TMEM is free
+                if (lane == 0) w = tc::mbar_wait(&ctl->acc_done, ictr & 1, abort, status) ? 1u : 0u;
+                if (!__shfl_sync(0xffffffffu, w, 0)) break;
                 tc::fence_after_sync();
-                float v[64];
-                tc::tmem_ld_32x32b_x64(tmem + DKV_DK + lane_off, v);
+                if (lane == 0) tc::bulk_wait_read<0>();
+                __syncwarp();
                 bf16* kbase = dqkv + ((long long)row_base + k0) * 3 * C + C + h * HD;
-                uint8_t* stage = smem + DKV_OFF_STAGE;
                 // column sums (the c_attn bias gradient) of this warp's 32-row group
-                float* cs = colsum_part ? colsum_part + ((long long)b * ((Tn + 31) / 32) + kt * 4 + quarter) * 3 * C
-                                        : nullptr;
-                store_rows_64(stage, r, v, 0.125f, kbase, 3LL * C, Tn - k0, cs ? cs + C + h * HD : nullptr);
-                tc::tmem_ld_32x32b_x64(tmem + DKV_DV + lane_off, v);
-                store_rows_64(stage, r, v, 1.0f, kbase + C, 3LL * C, Tn - k0, cs ? cs + 2 * C + h * HD : nullptr);
+                float* cs = colsum_part
+                                ? colsum_part + ((long long)b * ((Tn + 31) / 32) + cur.kt * 4 + quarter) * 3 * C
+                                : nullptr;
+#pragma unroll 1
+                for (int m = 0; m < 2; ++m) {   // dK (scaled by 1 / sqrt(64)), then dV
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        float v[32];
+                        tc::tmem_ld_32x32b_x32(tmem + (m ? BW_DV : BW_DK) + 32 * half + lane_off, v);
+                        stage_row_32(stage, r, v, m ? 1.0f : 0.125f, half);
+                    }
+                    flush_rows_64(stage, kbase + m * C, 3LL * C, Tn - k0, cs ? cs + (m + 1) * C + h * HD : nullptr);
+                }
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&ctl->dkv_free);
+                item = bw_read_item_warp(ctl, ++ictr, abort, status);
+                if (item >= 0) cur = bw_item(item, BH, n_qt);
+                it = 0;
             }
         }
+        if (lane == 0) tc::bulk_wait<0>();
     }
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 1) tc::tmem_dealloc(tmem, 512);
 }
 
-constexpr int DQ_STAGES = 6;    // K/V ring, likewise
-struct CtlDq {
-    uint64_t q_full;
-    uint64_t kv_full[DQ_STAGES], kv_empty[DQ_STAGES];
-    uint64_t s_full[2], s_empty[2];
-    uint64_t ds_full[2], ds_free[2];
-    uint64_t acc_done;
-    uint64_t drain;
-    uint32_t tmem_base;
-    uint32_t abort;
-};
-// smem: Q | dO | (K | V) stages | dS[2] | ctl
-constexpr int DQ_OFF_Q = 0;
-constexpr int DQ_OFF_DO = DQ_OFF_Q + T128_BYTES;
-constexpr int DQ_OFF_KV = DQ_OFF_DO + T128_BYTES;
-constexpr int DQ_STAGE_BYTES = 2 * T64_BYTES;
-constexpr int DQ_OFF_DS = DQ_OFF_KV + DQ_STAGES * DQ_STAGE_BYTES;
-constexpr int DQ_OFF_CTL = DQ_OFF_DS + 2 * T128_BYTES;   // 128 queries x 64 keys bf16 = 16 KB each
-constexpr size_t DQ_SMEM = DQ_OFF_CTL + sizeof(CtlDq) + 1024;
-constexpr uint32_t DQ_S = 0, DQ_DP = 128, DQ_DQ = 256;
-
-__global__ void __launch_bounds__(BW_THREADS, 1)
-    flash_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q128, const __grid_constant__ CUtensorMap tm_kv64,
-                           const __grid_constant__ CUtensorMap tm_do128, const float* __restrict__ lse,
-                           const float* __restrict__ dpre, bf16* __restrict__ dqkv, int Tn, int H,
-                           float* __restrict__ colsum_part, unsigned* status) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    CtlDq* ctl = reinterpret_cast<CtlDq*>(smem + DQ_OFF_CTL);
-    volatile uint32_t* abort = &ctl->abort;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // grid (B H, query tiles): the last query tile sees the most keys and is dispatched first
-    const int n_qt = gridDim.y;
-    const int qt = n_qt - 1 - blockIdx.y;
-    const int bh = blockIdx.x, b = bh / H, h = bh % H;
-    const int C = H * HD;
-    const int q0 = qt * 128;
-    const int n_k64 = (min(Tn, q0 + 128) + 63) / 64;    // key tiles that some query of the tile sees
-    const int row_base = b * Tn;
-
-    if (threadIdx.x == 0) {
-        tc::mbar_init(&ctl->q_full, 1);
-        for (int s = 0; s < DQ_STAGES; ++s) {
-            tc::mbar_init(&ctl->kv_full[s], 1);
-            tc::mbar_init(&ctl->kv_empty[s], 1);
+// D = rowsum(dO * O) for every head of one (b, t) row, the fp32 dQ accumulator
+// row set to zero, and the work-item counter reset: one warp per row; 8 lanes
+// per head (16 bytes of O and of dO each), 4 heads per pass.
+__global__ void __launch_bounds__(256) flash_bwd_pre_tc_kernel(const bf16* __restrict__ out,
+                                                               const bf16* __restrict__ dout,
+                                                               float* __restrict__ dpre, float* __restrict__ dq_acc,
+                                                               int* __restrict__ work, int Tn, int H, long long rows) {
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *work = 0;
+    if (row >= rows) return;
+    const int b = (int)(row / Tn), t = (int)(row % Tn);
+    const long long C = (long long)H * HD;
+    for (int h0 = 0; h0 < H; h0 += 4) {
+        const int h = h0 + (lane >> 3);
+        float s = 0.f;
+        if (h < H) {
+            const long long o = row * C + h * HD + (lane & 7) * 8;
+            const uint4 x = *reinterpret_cast<const uint4*>(out + o);
+            const uint4 y = *reinterpret_cast<const uint4*>(dout + o);
+            const __nv_bfloat162* xa = reinterpret_cast<const __nv_bfloat162*>(&x);
+            const __nv_bfloat162* ya = reinterpret_cast<const __nv_bfloat162*>(&y);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 fx = __bfloat1622float2(xa[j]), fy = __bfloat1622float2(ya[j]);
+                s = fmaf(fx.x, fy.x, fmaf(fx.y, fy.y, s));
+            }
         }
-        for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&ctl->s_full[i], 1);
-            tc::mbar_init(&ctl->s_empty[i], BW_EW_WARPS);
-            tc::mbar_init(&ctl->ds_full[i], BW_EW_WARPS);
-            tc::mbar_init(&ctl->ds_free[i], 1);
-        }
-        tc::mbar_init(&ctl->acc_done, 1);
-        tc::mbar_init(&ctl->drain, 1);
-        ctl->abort = 0;
-        tc::fence_barrier_init();
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        s += __shfl_xor_sync(0xffffffffu, s, 4);
+        if (h < H && (lane & 7) == 0) dpre[((long long)b * H + h) * Tn + t] = s;
     }
-    if (warp == 1) {
-        tc::tmem_alloc(&ctl->tmem_base, 512);
-        tc::tmem_relinquish();
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tmem = ctl->tmem_base;
+    float4* z = reinterpret_cast<float4*>(dq_acc + row * C);
+    for (long long i = lane; i < C / 4; i += 32) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
 
-    if (warp == 0) {
-        if (lane == 0) {
-            tc::tma_prefetch_desc(&tm_q128);
-            tc::tma_prefetch_desc(&tm_kv64);
-            tc::tma_prefetch_desc(&tm_do128);
-            tc::mbar_expect_tx(&ctl->q_full, 2 * T128_BYTES);
-            tc::tma_load_2d(smem + DQ_OFF_Q, &tm_q128, h * HD, row_base + q0, &ctl->q_full);
-            tc::tma_load_2d(smem + DQ_OFF_DO, &tm_do128, h * HD, row_base + q0, &ctl->q_full);
-            for (int j = 0; j < n_k64; ++j) {
-                const int s = j % DQ_STAGES;
-                if (!tc::mbar_wait(&ctl->kv_empty[s], ((j / DQ_STAGES) & 1) ^ 1, abort, status)) break;
-                uint8_t* st = smem + DQ_OFF_KV + s * DQ_STAGE_BYTES;
-                tc::mbar_expect_tx(&ctl->kv_full[s], 2 * T64_BYTES);
-                tc::tma_load_2d(st, &tm_kv64, C + h * HD, row_base + j * 64, &ctl->kv_full[s]);
-                tc::tma_load_2d(st + T64_BYTES, &tm_kv64, 2 * C + h * HD, row_base + j * 64, &ctl->kv_full[s]);
-            }
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 64, 0, 0);    // Q K^T, dO V^T
-            constexpr uint32_t idesc_dq = tc::idesc_bf16_f32(128, 64, 0, 1);   // dS K
-            const uint32_t q_addr = tc::smem_u32(smem + DQ_OFF_Q), do_addr = tc::smem_u32(smem + DQ_OFF_DO);
-            bool ok = tc::mbar_wait(&ctl->q_full, 0, abort, status);
-            auto accumulate = [&](int j) -> bool {   // dQ += dS K for key tile j
-                const int r = j & 1, s = j % DQ_STAGES;
-                if (!tc::mbar_wait(&ctl->ds_full[r], (j >> 1) & 1, abort, status)) return false;
-                tc::fence_after_sync();
-                const uint32_t k_addr = tc::smem_u32(smem + DQ_OFF_KV + s * DQ_STAGE_BYTES);
-                const uint32_t ds = tc::smem_u32(smem + DQ_OFF_DS + r * T128_BYTES);
+// dq columns of dqkv = the fp32 accumulator rounded to bf16, and (if
+// colsum_part) the column sums of each 32-row group of the stored values, in
+// row order. Block = one 32-row group of one sequence; thread = 8 columns of
+// each blockDim.x * 8 column stretch.
+__global__ void __launch_bounds__(256) flash_bwd_dq_post_kernel(const float* __restrict__ dq_acc,
+                                                                bf16* __restrict__ dqkv, int Tn, int C,
+                                                                float* __restrict__ colsum_part) {
+    const int G = (Tn + 31) / 32;
+    const int b = blockIdx.x / G, grp = blockIdx.x % G;
+    const int t0 = grp * 32, t1 = min(Tn, t0 + 32);
+    for (int c0 = threadIdx.x * 8; c0 < C; c0 += blockDim.x * 8) {
+    float sum[8];
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)   // K = 64 keys
-                    tc::mma_bf16(tmem + DQ_DQ, tc::smem_desc_sw128(ds + kk * 32, 16, 1024),
-                                 tc::smem_desc_sw128(k_addr + kk * 2048, T64_BYTES, 1024), idesc_dq,
-                                 (j > 0 || kk > 0) ? 1u : 0u);
-                tc::mma_commit(&ctl->ds_free[r]);
-                tc::mma_commit(&ctl->kv_empty[s]);
-                return true;
-            };
-            for (int j = 0; j < n_k64 && ok; ++j) {
-                const int r = j & 1, s = j % DQ_STAGES;
-                if (!tc::mbar_wait(&ctl->kv_full[s], (j / DQ_STAGES) & 1, abort, status)) break;
-                if (!tc::mbar_wait(&ctl->s_empty[r], ((j >> 1) & 1) ^ 1, abort, status)) break;
-                tc::fence_after_sync();
-                const uint32_t k_addr = tc::smem_u32(smem + DQ_OFF_KV + s * DQ_STAGE_BYTES);
-                const uint32_t v_addr = k_addr + T64_BYTES;
+    for (int e = 0; e < 8; ++e) sum[e] = 0.f;
+#pragma unroll 4
+    for (int t = t0; t < t1; ++t) {
+        const long long row = (long long)b * Tn + t;
+        const float4 x0 = *reinterpret_cast<const float4*>(dq_acc + row * C + c0);
+        const float4 x1 = *reinterpret_cast<const float4*>(dq_acc + row * C + c0 + 4);
+        const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        const uint4 q = pack8_bf16(v);
+        *reinterpret_cast<uint4*>(dqkv + row * 3 * C + c0) = q;
+        const __nv_bfloat162* qa = reinterpret_cast<const __nv_bfloat162*>(&q);
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    tc::mma_bf16(tmem + DQ_S + r * 64, tc::smem_desc_sw128(q_addr + kk * 32, 16, 1024),
-                                 tc::smem_desc_sw128(k_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-                    tc::mma_bf16(tmem + DQ_DP + r * 64, tc::smem_desc_sw128(do_addr + kk * 32, 16, 1024),
-                                 tc::smem_desc_sw128(v_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-                }
-                tc::mma_commit(&ctl->s_full[r]);
-                if (j > 0 && !accumulate(j - 1)) { ok = false; break; }
-            }
-            if (ok && n_k64 > 0) ok = accumulate(n_k64 - 1);
-            tc::mma_commit(&ctl->acc_done);
-            volatile uint32_t no_abort = 0;
-            tc::mma_commit(&ctl->drain);
-            tc::mbar_wait(&ctl->drain, 0, &no_abort, status);
-        }
-    } else {
-        // --------------------------------------------------- dS (thread = query row)
-        const int quarter = warp & 3;
-        const int chalf = (warp - 2) >> 2;              // key columns [32 chalf, 32 chalf + 32)
-        const int r = quarter * 32 + lane;
-        const int q = q0 + r;
-        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const float sl2 = LOG2E * 0.125f;
-        const float L2 = q < Tn ? lse[(long long)bh * Tn + q] * LOG2E : INFINITY;
-        const float Dv = q < Tn ? dpre[(long long)bh * Tn + q] : 0.f;
-        bool ok = true;
-        for (int j = 0; j < n_k64; ++j) {
-            const int rb = j & 1;
-            uint32_t w = 0;
-            if (lane == 0) {
-                w = tc::mbar_wait(&ctl->s_full[rb], (j >> 1) & 1, abort, status) ? 1u : 0u;
-                if (w) w = tc::mbar_wait(&ctl->ds_free[rb], ((j >> 1) & 1) ^ 1, abort, status) ? 1u : 0u;
-            }
-            w = __shfl_sync(0xffffffffu, w, 0);
-            if (!w) { ok = false; break; }
-            tc::fence_after_sync();
-            const bool diag = (j * 64 + 64 > q0);
-            uint8_t* ds = smem + DQ_OFF_DS + rb * T128_BYTES;
-            float sv[32], dp[32];
-            tc::tmem_ld2_32x32b_x32(tmem + DQ_S + rb * 64 + chalf * 32 + lane_off,
-                                    tmem + DQ_DP + rb * 64 + chalf * 32 + lane_off, sv, dp);
-            // dS = 2^(s sl2 - lse2) (dP - D) on packed pairs of keys
-            const f32x2 SL = pk2(sl2, sl2), NL = pk2(-L2, -L2), ND = pk2(-Dv, -Dv);
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-                float t0, t1;
-                upk2(fma2(pk2(sv[e], sv[e + 1]), SL, NL), t0, t1);
-                float p0 = ex2(t0), p1 = ex2(t1);
-                if (diag) {   // keys after this query
-                    if (j * 64 + chalf * 32 + e > q) p0 = 0.f;
-                    if (j * 64 + chalf * 32 + e + 1 > q) p1 = 0.f;
-                }
-                upk2(mul2(pk2(p0, p1), add2(pk2(dp[e], dp[e + 1]), ND)), dp[e], dp[e + 1]);
-            }
-#pragma unroll
-            for (int g = 0; g < 4; ++g)
-                *reinterpret_cast<uint4*>(ds + swz128(r, chalf * 4 + g)) = pack8_bf16(dp + 8 * g);
-            tc::fence_proxy_async_smem();
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) {
-                tc::mbar_arrive(&ctl->s_empty[rb]);
-                tc::mbar_arrive(&ctl->ds_full[rb]);
-            }
-        }
-        if (ok && chalf == 0) {
-            uint32_t w = 0;
-            if (lane == 0) w = tc::mbar_wait(&ctl->acc_done, 0, abort, status) ? 1u : 0u;
-            w = __shfl_sync(0xffffffffu, w, 0);
-            if (w) {
-                tc::fence_after_sync();
-                float v[64];
-                tc::tmem_ld_32x32b_x64(tmem + DQ_DQ + lane_off, v);
-                bf16* qbase = dqkv + ((long long)row_base + q0) * 3 * C + h * HD;
-                float* cs = colsum_part ? colsum_part + ((long long)b * ((Tn + 31) / 32) + qt * 4 + quarter) * 3 * C
-                                        : nullptr;
-                store_rows_64(smem + DQ_OFF_DS, r, v, 0.125f, qbase, 3LL * C, Tn - q0, cs ? cs + h * HD : nullptr);
-            }
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(qa[j]);
+            sum[2 * j] += f.x;
+            sum[2 * j + 1] += f.y;
         }
     }
-    tc::fence_before_sync();
-    __syncthreads();
-    if (warp == 1) tc::tmem_dealloc(tmem, 512);
+    if (colsum_part) {
+        float* dst = colsum_part + (long long)blockIdx.x * 3 * C + c0;
+        *reinterpret_cast<float4*>(dst) = make_float4(sum[0], sum[1], sum[2], sum[3]);
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(sum[4], sum[5], sum[6], sum[7]);
+    }
+    }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn_attn() {
@@ -976,36 +1105,41 @@ bool launch_attention_fwd_tc(const Ctx& ctx, const bf16* qkv, bf16* out, float* 
 }
 
 bool launch_attention_bwd_tc(const Ctx& ctx, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
-                             float* dpre, bf16* dqkv, int B, int Tn, int H, float* colsum_part) {
+                             float* dpre, float* dq_acc, int* work, bf16* dqkv, int B, int Tn, int H,
+                             float* colsum_part) {
     auto fn = encode_fn_attn();
     if (!fn) return false;
     const long long C = (long long)H * HD;
-    auto make = [&](CUtensorMap* m, const bf16* base, long long cols, int box_rows) {
+    auto make = [&](CUtensorMap* m, CUtensorMapDataType dt, const void* base, long long cols, int esize,
+                    int box_cols, int box_rows) {
         cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)B * Tn};
-        cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-        cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+        cuuint64_t strides[1] = {(cuuint64_t)cols * esize};
+        cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
         cuuint32_t estr[2] = {1, 1};
-        return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<bf16*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+        return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
     };
-    CUtensorMap qkv128, qkv64, do64, do128;
-    if (!make(&qkv128, qkv, 3 * C, 128) || !make(&qkv64, qkv, 3 * C, 64) || !make(&do64, dout, C, 64) ||
-        !make(&do128, dout, C, 128))
+    CUtensorMap m_qkv, m_do, m_dq;
+    if (!make(&m_qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qkv, 3 * C, 2, 64, 128) ||
+        !make(&m_do, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dout, C, 2, 64, 128) ||
+        !make(&m_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dq_acc, C, 4, 32, 32))
         return false;
     static bool configured = false;
     if (!configured) {
-        cudaFuncSetAttribute(flash_bwd_dkv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DKV_SMEM);
-        cudaFuncSetAttribute(flash_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DQ_SMEM);
+        cudaFuncSetAttribute(flash_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BW_SMEM);
         configured = true;
     }
-    launch_attention_bwd_pre(ctx, out, dout, dpre, B, Tn, H, HD);
-    const dim3 grid(B * H, ceil_div(Tn, 128));
-    flash_bwd_dkv_tc_kernel<<<grid, BW_THREADS, DKV_SMEM, ctx.stream>>>(qkv128, qkv64, do64, lse, dpre, dqkv, Tn, H,
-                                                                         colsum_part, ctx.status);
-    flash_bwd_dq_tc_kernel<<<grid, BW_THREADS, DQ_SMEM, ctx.stream>>>(qkv128, qkv64, do128, lse, dpre, dqkv, Tn, H,
-                                                                       colsum_part, ctx.status);
-    *ctx.launches += 2;
+    const long long rows = (long long)B * Tn;
+    flash_bwd_pre_tc_kernel<<<(unsigned)ceil_div_ll(rows, 8), 256, 0, ctx.stream>>>(out, dout, dpre, dq_acc, work, Tn,
+                                                                                   H, rows);
+    const int n_items = B * H * ceil_div(Tn, 128);
+    const int grid = min(n_items, ctx.num_sms > 0 ? ctx.num_sms : 148);
+    flash_bwd_tc_kernel<<<grid, BW_THREADS, BW_SMEM, ctx.stream>>>(m_qkv, m_do, m_dq, lse, dpre, dqkv, Tn, H, B * H,
+                                                                   work, colsum_part, ctx.status);
+    flash_bwd_dq_post_kernel<<<B * ceil_div(Tn, 32), (unsigned)min(C / 8, 256LL), 0, ctx.stream>>>(
+        dq_acc, dqkv, Tn, (int)C, colsum_part);
+    *ctx.launches += 3;
     return true;
 }
 

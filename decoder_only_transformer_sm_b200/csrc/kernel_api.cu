@@ -105,6 +105,22 @@ extern "C" int gpt2k_attention_fwd(int dtype, const void* qkv, void* out, float*
     return GPT2_OK;
 }
 
+namespace {
+// engine 2 workspace: [D: B*H*T floats, padded to 64][dQ accumulator: B*T*C floats][work counter: 64]
+long long attention_bwd_dq_offset(int B, int T, int H) { return ((long long)B * H * T + 63) / 64 * 64; }
+long long attention_bwd_work_offset(int B, int T, int H, int hd) {
+    return attention_bwd_dq_offset(B, T, H) + ((long long)B * T * H * hd + 63) / 64 * 64;
+}
+}  // namespace
+
+extern "C" int gpt2k_attention_bwd_workspace(int B, int T, int H, int hd, int engine, int64_t* floats) {
+    if (!floats) return set_error(GPT2_ERR_INVALID_ARG, "NULL argument");
+    if (B < 1 || T < 1 || H < 1 || (hd != 32 && hd != 64) || engine < 0 || engine > 2)
+        return set_error(GPT2_ERR_INVALID_ARG, "bad size, head width or engine");
+    *floats = engine == 2 ? attention_bwd_work_offset(B, T, H, hd) + 64 : (long long)B * H * T;
+    return GPT2_OK;
+}
+
 extern "C" int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, const void* dout, const float* lse,
                                    void* dqkv, int B, int T, int H, int hd, float* workspace_dev,
                                    float* colsum_part, int engine, uint32_t* status_dev, void* stream) {
@@ -117,7 +133,9 @@ extern "C" int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, 
     Ctx c = kctx(stream, status_dev, &launches);
     if (engine == 2) {
         if (!launch_attention_bwd_tc(c, (const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, workspace_dev,
-                                     (bf16*)dqkv, B, T, H, colsum_part))
+                                     workspace_dev + attention_bwd_dq_offset(B, T, H),
+                                     (int*)(workspace_dev + attention_bwd_work_offset(B, T, H, hd)), (bf16*)dqkv, B,
+                                     T, H, colsum_part))
             return set_error(GPT2_ERR_CUDA, "tensor-map encoding failed");
     } else if (engine == 1)
         launch_attention_bwd_mma(c, (const bf16*)qkv, (const bf16*)out, (const bf16*)dout, lse, workspace_dev,

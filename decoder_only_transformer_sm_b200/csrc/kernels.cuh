@@ -124,11 +124,16 @@ void launch_attention_bwd_mma(const Ctx& ctx, const bf16* qkv, const bf16* out, 
 // could not be encoded (nothing launched).
 bool attention_tc_supported(int hd);
 bool launch_attention_fwd_tc(const Ctx& ctx, const bf16* qkv, bf16* out, float* lse, int B, int Tn, int H);
-// tcgen05 flash attention backward (head width 64): D pre-pass, dK/dV kernel, dQ kernel.
+// tcgen05 flash attention backward (head width 64): a pre-pass (D = rowsum(dout *
+// out) into dpre (B*H*T floats), dq_acc zeroed, *work zeroed), the fused
+// persistent kernel (dK, dV into dqkv; dQ added into dq_acc, fp32 (B*T, C),
+// 16-byte aligned; *work is its work-item counter) and a post-pass (dq_acc
+// rounded into the dq columns of dqkv).
 // colsum_part (nullable): fp32 [B * ceil(Tn / 32)][3C]; row b * ceil(Tn / 32) + g
 // receives the column sums of dqkv rows 32 g .. 32 g + 31 of sequence b.
 bool launch_attention_bwd_tc(const Ctx& ctx, const bf16* qkv, const bf16* out, const bf16* dout, const float* lse,
-                             float* dpre, bf16* dqkv, int B, int Tn, int H, float* colsum_part);
+                             float* dpre, float* dq_acc, int* work, bf16* dqkv, int B, int Tn, int H,
+                             float* colsum_part);
 // D = rowsum(dout * out) per (b, h, t) (the backward's pre-pass).
 void launch_attention_bwd_pre(const Ctx& ctx, const bf16* out, const bf16* dout, float* dpre, int B, int Tn, int H,
                               int hd);

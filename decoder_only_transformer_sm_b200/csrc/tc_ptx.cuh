@@ -88,6 +88,18 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, int
         : "memory");
 }
 
+// Prefetch of one box of a 2-D tiled tensor into L2 (no shared memory, no
+// completion to wait for): a later tma_load_2d of the box then hits L2.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Shared -> global tiled store and reduce-add (bulk async groups). The
 // coordinates must be >= 0 and x * element size a multiple of 16 bytes; parts
 // of the box outside the tensor are not written.

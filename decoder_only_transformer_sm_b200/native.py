@@ -95,6 +95,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gpt2k_matmul_bf16": (I, [I, P, P, I, I, I, I, P, ctypes.c_int64, P, P, P, P, P, F, I, P, P]),
         "gpt2k_attention_fwd": (I, [I, P, P, P, I, I, I, I, I, P, P]),
         "gpt2k_attention_bwd": (I, [I, P, P, P, P, P, I, I, I, I, P, P, I, P, P]),
+        "gpt2k_attention_bwd_workspace": (I, [I, I, I, I, I, ctypes.POINTER(ctypes.c_int64)]),
         "gpt2k_attention_decode": (I, [I, P, P, I, I, I, I, I, P, P, P]),
         "gpt2k_sample": (I, [I, P, I, I, ctypes.c_int64, F, I, P, P, P, P]),
     }
@@ -354,9 +355,16 @@ def attention_fwd(qkv, out, lse, B: int, T: int, H: int, hd: int, engine: int = 
     return status
 
 
+def attention_bwd_workspace(B: int, T: int, H: int, hd: int, engine: int = 0) -> int:
+    """Float32 elements of the workspace gpt2k_attention_bwd needs (gpt2k_attention_bwd_workspace)."""
+    n = ctypes.c_int64()
+    _check(load_library().gpt2k_attention_bwd_workspace(B, T, H, hd, engine, ctypes.byref(n)))
+    return n.value
+
+
 def attention_bwd(qkv, out, dout, lse, dqkv, B: int, T: int, H: int, hd: int, workspace, engine: int = 0,
                   status=None, stream=None, colsum_part=None):
-    """gpt2k_attention_bwd on torch device tensors (workspace: B*H*T float32)."""
+    """gpt2k_attention_bwd on torch device tensors (workspace: attention_bwd_workspace(...) float32)."""
     status, stream = _stream_and_status(qkv, status, stream)
     _check(load_library().gpt2k_attention_bwd(_dtype_code(qkv), _ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse),
                                               _ptr(dqkv), B, T, H, hd, _ptr(workspace), _ptr(colsum_part), engine,

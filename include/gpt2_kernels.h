@@ -87,13 +87,25 @@ int gpt2k_attention_fwd(int dtype, const void* qkv, void* out, float* lse, int B
 
 /* Backward of gpt2k_attention_fwd: dqkv (B, T, 3C) = [dq | dk | dv] from qkv,
  * out, dout (B, T, C) and lse.
- * workspace_dev: caller-owned scratch of B*H*T floats (D = rowsum(dout * out)).
+ * workspace_dev: caller-owned scratch, 16-byte aligned, of the number of floats
+ *         gpt2k_attention_bwd_workspace gives: B*H*T (D = rowsum(dout * out))
+ *         for engines 0 and 1; for engine 2 also an fp32 (B*T, C) accumulator
+ *         of dQ, which the key tiles' partial products are added into, and
+ *         the persistent kernel's work-item counter. Calls sharing one
+ *         workspace must not overlap on the GPU.
  * colsum_part: engine 2 only, else NULL: fp32 [B * ceil(T / 32), 3C] (stride
  *         3C); row b * ceil(T / 32) + g receives the column sums of the stored
  *         dqkv rows 32 g .. min(32 g + 31, T - 1) of sequence b. Adding its rows
  *         gives the bias gradient of the layer that produced qkv.
  * engine: 0 = SIMT kernel; 1 = mma.sync tensor-core kernels (bf16); 2 = tcgen05
- *         kernels (bf16, hd = 64: TMEM accumulators for dK, dV, dQ). */
+ *         kernels (bf16, hd = 64: one pass per (key tile, query tile) pair
+ *         computes S and dP once; dK, dV accumulate in TMEM, dQ in the fp32
+ *         workspace through bulk reduce-adds, whose order of arrival decides
+ *         the last bits of dq). */
+/* Workspace size of gpt2k_attention_bwd in floats (into *floats). Errors:
+ * INVALID_ARG for sizes < 1, hd not 32 or 64, or an unknown engine. */
+int gpt2k_attention_bwd_workspace(int B, int T, int H, int hd, int engine, int64_t* floats);
+
 int gpt2k_attention_bwd(int dtype, const void* qkv, const void* out, const void* dout, const float* lse,
                         void* dqkv, int B, int T, int H, int hd, float* workspace_dev, float* colsum_part,
                         int engine, uint32_t* status_dev, void* stream);

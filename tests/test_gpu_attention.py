@@ -45,7 +45,7 @@ def test_attention_fwd_bwd_vs_oracle(dtype, engine, case):
     out = torch.empty((B, T, C), dtype=tdt, device="cuda")
     lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
     dqkv = torch.empty_like(qkv)
-    ws = torch.empty((B * H * T,), dtype=torch.float32, device="cuda")
+    ws = torch.empty((native.attention_bwd_workspace(B, T, H, hd, engine),), dtype=torch.float32, device="cuda")
     st = native.attention_fwd(qkv, out, lse, B, T, H, hd, engine=engine)
     native.attention_bwd(qkv, out, dout, lse, dqkv, B, T, H, hd, ws, engine=engine, status=st)
     torch.cuda.synchronize()
@@ -81,7 +81,7 @@ def test_tcgen05_backward_column_sums(case):
     out = torch.empty((B, T, C), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
     dqkv = torch.empty_like(qkv)
-    ws = torch.empty((B * H * T,), dtype=torch.float32, device="cuda")
+    ws = torch.empty((native.attention_bwd_workspace(B, T, H, hd, 2),), dtype=torch.float32, device="cuda")
     G = (T + 31) // 32
     part = torch.full((B * G, 3 * C), float("nan"), device="cuda")
     st = native.attention_fwd(qkv, out, lse, B, T, H, hd, engine=2)
