@@ -4,11 +4,16 @@
 // Warp 0 streams A/B k-blocks with TMA into a 4-stage shared-memory ring that
 // runs continuously across units; warp 1 issues tcgen05.mma (kind::f16, bf16
 // operands, M=128, N=256, K=16) from one thread into one of two fp32
-// accumulators in tensor memory (2 x 256 columns = all 512); warps 2..9 read
-// the other accumulator with tcgen05.ld and run the fused epilogue while the
-// next unit's MMAs proceed, then hand the accumulator back. Each epilogue warp
-// turns its rows around in a private swizzled shared-memory buffer so that
-// results and epilogue inputs move through global memory as whole 128-byte rows.
+// accumulators in tensor memory (2 x 256 columns = all 512); the epilogue
+// warps (from warp 2 on) read the other accumulator with tcgen05.ld and run the
+// fused epilogue while the next unit's MMAs proceed, then hand the accumulator
+// back. Eight epilogue warps (two per TMEM lane quarter, 128 of the 256 columns
+// each) serve the light epilogues; the GELU epilogue, whose arithmetic per
+// element is the longest, gets sixteen (four per lane quarter, 64 columns
+// each), so each scheduler has four of them to hide its latencies. Each
+// epilogue warp turns its rows around in a private swizzled shared-memory
+// buffer so that results and epilogue inputs move through global memory as
+// 128-byte rows (64-byte row segments for the sixteen-warp layout).
 //
 // All three operand layouts of the training step run on the same kernel:
 //   NT (forward, y = x W^T):   A K-major,  B K-major
@@ -33,12 +38,9 @@ constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
 constexpr int B_BYTES = BN * BK * 2;   // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int EPI_WARPS = 8;
-constexpr int THREADS = 64 + 32 * EPI_WARPS;   // 320
 constexpr int MN_BOX_BYTES = 64 * BK * 2;       // one 64-wide MN-major box: 8 KB
 constexpr int TMEM_COLS = 2 * BN;               // two accumulators
-constexpr int EBUF = 4096;                      // per epilogue warp: 32 rows x 128 bytes
-constexpr int EPI_BYTES = EPI_WARPS * EBUF;
+constexpr int EPI_BYTES = 32 * 1024;            // epilogue staging, split evenly among the epilogue warps
 
 struct Ctl {
     uint64_t full[STAGES];
@@ -52,10 +54,14 @@ struct Ctl {
 
 constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + EPI_BYTES + 1024 + sizeof(Ctl);
 
-// Byte offset of 16-byte segment c (0..7) of row r (0..31) in a warp's chunk
-// buffer of 128-byte rows; the XOR keeps both access patterns (a lane per
-// row, and eight lanes per row) free of bank conflicts.
-__device__ __forceinline__ uint32_t swz(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
+// Byte offset of 16-byte segment c of row r (0..31) in a warp's chunk buffer
+// of ROWB-byte rows; the XOR spreads eight consecutive rows over all 32 banks,
+// so both access patterns (a lane per row, and ROWB / 16 lanes per row) take the
+// minimum four wavefronts per 512 bytes.
+template <int ROWB>
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+    return ROWB == 128 ? r * 128 + ((c ^ (r & 7)) << 4) : r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
+}
 
 struct Units {
     int tiles_m, tiles_n, splits, kb_total, kb_per_split;
@@ -80,26 +86,35 @@ struct Units {
 template <int KIND>
 struct EpiTraits {
     static constexpr bool F32 = (KIND == EPI_BIAS_RESID || KIND == EPI_ACCUM_F32);   // fp32 result
-    static constexpr int CW = F32 ? 32 : 64;       // columns per chunk: 128 bytes of results per row
-    static constexpr int EPS = F32 ? 4 : 8;        // elements per 16-byte segment
+    static constexpr bool WIDE = (KIND == EPI_BIAS_GELU);   // sixteen epilogue warps
+    static constexpr int WARPS = WIDE ? 16 : 8;
+    static constexpr int THREADS = 64 + 32 * WARPS;
+    static constexpr int ROWB = WIDE ? 64 : 128;   // staged bytes per row and chunk
+    static constexpr int SEGS = ROWB / 16;         // 16-byte segments per staged row = lanes per row when copying
+    static constexpr int RPS = 32 / SEGS;          // rows per copy step
+    static constexpr int EBUF = 32 * ROWB;         // staging per epilogue warp
     static constexpr int ES = F32 ? 4 : 2;         // element size
+    static constexpr int CW = ROWB / ES;           // columns per chunk
+    static constexpr int EPS = 16 / ES;            // elements per 16-byte segment
+    static constexpr int WCOLS = BN / (WARPS / 4); // columns per warp and tile
     static constexpr bool HAS_IN = (KIND == EPI_BIAS_RESID || KIND == EPI_MUL);
     static constexpr bool HAS_BIAS = (KIND == EPI_BIAS || KIND == EPI_BIAS_GELU || KIND == EPI_BIAS_RESID);
     static constexpr int DEPTH = F32 ? 2 : 1;      // input chunks prefetched ahead (fp32 chunks are narrower)
 };
 
-// Start the coalesced loads of one input chunk (the residual, or the GELU
-// pre-activation) into registers: lane = 8 lanes per row, 4 rows per step.
+// Start the coalesced loads of one input chunk (the residual, or the stored
+// GELU derivative) into registers: SEGS lanes per row, RPS rows per step.
 template <int KIND>
-__device__ __forceinline__ void prefetch_in(const Epilogue& ep, uint4 (&pre)[8], int row0, int col0, int M, int N) {
+__device__ __forceinline__ void prefetch_in(const Epilogue& ep, uint4 (&pre)[EpiTraits<KIND>::SEGS], int row0,
+                                            int col0, int M, int N) {
     using E = EpiTraits<KIND>;
     const int lane = threadIdx.x & 31;
-    const int lrow = lane >> 3, lseg = lane & 7;
+    const int lrow = lane / E::SEGS, lseg = lane % E::SEGS;
     const char* src = KIND == EPI_BIAS_RESID ? reinterpret_cast<const char*>(ep.resid)
                                              : reinterpret_cast<const char*>(ep.aux);
 #pragma unroll
-    for (int st = 0; st < 8; ++st) {
-        const int r = st * 4 + lrow;
+    for (int st = 0; st < E::SEGS; ++st) {
+        const int r = st * E::RPS + lrow;
         const int c = col0 + lseg * E::EPS;
         pre[st] = make_uint4(0, 0, 0, 0);
         if (row0 + r < M && c < N)
@@ -110,23 +125,26 @@ __device__ __forceinline__ void prefetch_in(const Epilogue& ep, uint4 (&pre)[8],
 // One chunk of the epilogue for the calling warp: rows row0 .. row0+31 (lane =
 // row of acc) by CW columns from col0. Results (and the prefetched residual /
 // GELU' inputs, which have the same shape as the result) pass through the
-// warp's shared-memory buffer, so global memory is read and written in whole
-// 128-byte rows, four rows per instruction; each lane updates its row's
-// 16-byte segments in place in the buffer. If next_col0 >= 0, the input chunk
-// at next_col0 is prefetched into `pre` while this chunk is computed.
+// warp's shared-memory buffer, so global memory is read and written in
+// ROWB-byte row segments, RPS rows per instruction; each lane updates its
+// row's 16-byte segments in place in the buffer. If next_col0 >= 0, the input
+// chunk at next_col0 is prefetched into `pre` while this chunk is computed.
 template <int KIND>
 __device__ __forceinline__ void epilogue_chunk(const Epilogue& ep, float* acc, int row0, int col0, int M, int N,
-                                               uint8_t* buf, uint4 (&pre)[8], int next_col0) {
+                                               uint8_t* buf, float4 bq, uint4 (&pre)[EpiTraits<KIND>::SEGS],
+                                               int next_col0) {
     using E = EpiTraits<KIND>;
     constexpr bool F32 = E::F32;
     constexpr int EPS = E::EPS;
     constexpr int ES = E::ES;
     constexpr int kind = KIND;
     const int lane = threadIdx.x & 31;
-    const int lrow = lane >> 3, lseg = lane & 7;   // copy pattern: 8 lanes per row, 4 rows per step
+    constexpr int ROWB = E::ROWB;
+    const int lrow = lane / E::SEGS, lseg = lane % E::SEGS;   // copy pattern: SEGS lanes per row
     if (E::HAS_IN) {
 #pragma unroll
-        for (int st = 0; st < 8; ++st) *reinterpret_cast<uint4*>(buf + swz(st * 4 + lrow, lseg)) = pre[st];
+        for (int st = 0; st < E::SEGS; ++st)
+            *reinterpret_cast<uint4*>(buf + swz<ROWB>(st * E::RPS + lrow, lseg)) = pre[st];
         __syncwarp();
         if (next_col0 >= 0) prefetch_in<KIND>(ep, pre, row0, next_col0, M, N);
     }
@@ -134,23 +152,25 @@ __device__ __forceinline__ void epilogue_chunk(const Epilogue& ep, float* acc, i
 #pragma unroll
     for (int pass = 0; pass < npass; ++pass) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < ROWB / 16; ++c) {
             float* x = acc + c * EPS;
             float in[EPS], b[EPS];
             if (E::HAS_IN) {
                 if (F32) {
-                    const float4 q = *reinterpret_cast<const float4*>(buf + swz(lane, c));
+                    const float4 q = *reinterpret_cast<const float4*>(buf + swz<ROWB>(lane, c));
                     in[0] = q.x; in[1] = q.y; in[2] = q.z; in[3] = q.w;
                 } else {
-                    load8(reinterpret_cast<const bf16*>(buf + swz(lane, c)), in);
+                    load8(reinterpret_cast<const bf16*>(buf + swz<ROWB>(lane, c)), in);
                 }
             }
-            if (E::HAS_BIAS && pass == 0) {
+            if (E::HAS_BIAS && pass == 0) {   // the chunk's bias: column 4 l + i sits in lane l, component i
 #pragma unroll
                 for (int g = 0; g < EPS / 4; ++g) {
-                    float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (col0 + c * EPS + 4 * g < N) q = *reinterpret_cast<const float4*>(ep.bias + col0 + c * EPS + 4 * g);
-                    b[4 * g] = q.x; b[4 * g + 1] = q.y; b[4 * g + 2] = q.z; b[4 * g + 3] = q.w;
+                    const int src = (c * EPS) / 4 + g;
+                    b[4 * g] = __shfl_sync(0xffffffffu, bq.x, src);
+                    b[4 * g + 1] = __shfl_sync(0xffffffffu, bq.y, src);
+                    b[4 * g + 2] = __shfl_sync(0xffffffffu, bq.z, src);
+                    b[4 * g + 3] = __shfl_sync(0xffffffffu, bq.w, src);
                 }
             }
             float v[EPS];
@@ -182,20 +202,20 @@ __device__ __forceinline__ void epilogue_chunk(const Epilogue& ep, float* acc, i
             }
             }
             if (F32) {
-                *reinterpret_cast<float4*>(buf + swz(lane, c)) = make_float4(v[0], v[1], v[2], v[3]);
+                *reinterpret_cast<float4*>(buf + swz<ROWB>(lane, c)) = make_float4(v[0], v[1], v[2], v[3]);
             } else {
-                store8(reinterpret_cast<bf16*>(buf + swz(lane, c)), v);
+                store8(reinterpret_cast<bf16*>(buf + swz<ROWB>(lane, c)), v);
             }
         }
         __syncwarp();
         // whole rows out to global memory
         char* dst = reinterpret_cast<char*>((kind == EPI_BIAS_GELU && pass == 0) ? ep.out2 : ep.out);
 #pragma unroll
-        for (int st = 0; st < 8; ++st) {
-            const int r = st * 4 + lrow;
+        for (int st = 0; st < E::SEGS; ++st) {
+            const int r = st * E::RPS + lrow;
             const int c = col0 + lseg * EPS;
             if (row0 + r < M && c < N) {
-                const uint4 q = *reinterpret_cast<const uint4*>(buf + swz(r, lseg));
+                const uint4 q = *reinterpret_cast<const uint4*>(buf + swz<ROWB>(r, lseg));
                 char* gp = dst + ((long long)(row0 + r) * ep.ldo + c) * ES;
                 if (F32 && kind == EPI_ACCUM_F32) {
                     float4 a = *reinterpret_cast<const float4*>(&q);
@@ -214,27 +234,31 @@ __device__ __forceinline__ void epilogue_chunk(const Epilogue& ep, float* acc, i
             }
         }
         if (kind == EPI_MUL && ep.colsum_part) {
-            // column sums of the warp's 32 rows: lane = columns 2 lane, 2 lane + 1 of the chunk
-            float s0 = 0.f, s1 = 0.f;
-            const int rmax = M - row0;
+            // column sums of the warp's 32 rows: lane l < 16 = columns 2 l, 2 l + 1 of the chunk
+            if (lane < E::CW / 2) {
+                float s0 = 0.f, s1 = 0.f;
+                const int rmax = M - row0;
 #pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                if (r < rmax) {
-                    const uint32_t w2 = *reinterpret_cast<const uint32_t*>(buf + swz(r, lane >> 2) + (lane & 3) * 4);
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w2));
-                    s0 += f.x;
-                    s1 += f.y;
+                for (int r = 0; r < 32; ++r) {
+                    if (r < rmax) {
+                        const uint32_t w2 =
+                            *reinterpret_cast<const uint32_t*>(buf + swz<ROWB>(r, lane >> 2) + (lane & 3) * 4);
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w2));
+                        s0 += f.x;
+                        s1 += f.y;
+                    }
                 }
+                const int c = col0 + 2 * lane;
+                if (c < N)
+                    *reinterpret_cast<float2*>(ep.colsum_part + (long long)(row0 >> 5) * N + c) = make_float2(s0, s1);
             }
-            const int c = col0 + 2 * lane;
-            if (c < N) *reinterpret_cast<float2*>(ep.colsum_part + (long long)(row0 >> 5) * N + c) = make_float2(s0, s1);
         }
         __syncwarp();
     }
 }
 
 template <int A_MN, int B_MN, int KIND>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(EpiTraits<KIND>::THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
                    Units units, Epilogue ep, unsigned* status) {
     extern __shared__ uint8_t smem_raw[];
@@ -252,7 +276,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(&ctl->acc_full[b], 1);
-            tc::mbar_init(&ctl->acc_empty[b], EPI_WARPS);
+            tc::mbar_init(&ctl->acc_empty[b], EpiTraits<KIND>::WARPS);
         }
         tc::mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
@@ -345,21 +369,30 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else {
         // ---------------------------------------------------------- epilogue
-        const int ew = warp - 2;                 // 0..7
-        const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
-        const int col_half = ew >> 2;            // columns [half*BN/2, half*BN/2 + BN/2)
-        uint8_t* buf = epi_smem + ew * EBUF;
         using E = EpiTraits<KIND>;
+        const int ew = warp - 2;                 // 0 .. E::WARPS - 1
+        const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
+        const int col_q = ew >> 2;               // columns [col_q * WCOLS, col_q * WCOLS + WCOLS)
+        uint8_t* buf = epi_smem + ew * E::EBUF;
         constexpr int CW = E::CW;
-        constexpr int NCH = (BN / 2) / CW;       // chunks per warp and tile
-        uint4 pre[E::DEPTH][8];                  // input chunks in flight (ring)
+        constexpr int NCH = E::WCOLS / CW;       // chunks per warp and tile
+        uint4 pre[E::DEPTH][E::SEGS];            // input chunks in flight (ring)
+        // the bias of one chunk: lane l < CW / 4 holds columns 4 l .. 4 l + 3 (zero past N),
+        // loaded one chunk ahead; the chunk's lanes read it with shuffles
+        auto load_bias = [&](int col0) {
+            float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (E::HAS_BIAS && lane < CW / 4 && col0 + 4 * lane < N)
+                q = *reinterpret_cast<const float4*>(ep.bias + col0 + 4 * lane);
+            return q;
+        };
         uint32_t acc_it = 0;
         for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++acc_it) {
             int mb, nb, kb0, kb1;
             units.decode(u, mb, nb, kb0, kb1);
             const uint32_t ab = acc_it & 1, aph = (acc_it >> 1) & 1;
             const int row0 = mb * BM + quarter * 32;
-            const int cbase = col_half * (BN / 2);
+            const int cbase = col_q * E::WCOLS;
+            float4 bq = load_bias(nb * BN + cbase);
             // the first input chunks of this tile are requested before waiting for the accumulator
             if (E::HAS_IN && row0 < M) {
 #pragma unroll
@@ -377,12 +410,20 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int c = ci * CW;
                 const int col0 = nb * BN + cbase + c;
                 if (col0 >= N) break;
+                const float4 bcur = bq;
+                if (E::HAS_BIAS && ci + 1 < NCH) bq = load_bias(col0 + CW);
                 float acc[CW];
-                tc::tmem_ld_32x32b_x32(taddr + (uint32_t)c, acc);
-                if (CW == 64) tc::tmem_ld_32x32b_x32(taddr + (uint32_t)c + 32, acc + 32);
+                if (CW == 64) {
+                    tc::tmem_ld_32x32b_x32(taddr + (uint32_t)c, acc);
+                    tc::tmem_ld_32x32b_x32(taddr + (uint32_t)c + 32, acc + 32);
+                } else if (CW == 32) {
+                    tc::tmem_ld_32x32b_x32(taddr + (uint32_t)c, acc);
+                } else {
+                    tc::tmem_ld_32x32b_x16(taddr + (uint32_t)c, acc);
+                }
                 const int nc = c + E::DEPTH * CW;     // chunk whose input this buffer prefetches next
-                const int next = (nc < BN / 2 && nb * BN + cbase + nc < N) ? nb * BN + cbase + nc : -1;
-                if (row0 < M) epilogue_chunk<KIND>(ep, acc, row0, col0, M, N, buf, pre[ci % E::DEPTH], next);
+                const int next = (nc < E::WCOLS && nb * BN + cbase + nc < N) ? nb * BN + cbase + nc : -1;
+                if (row0 < M) epilogue_chunk<KIND>(ep, acc, row0, col0, M, N, buf, bcur, pre[ci % E::DEPTH], next);
             }
             tc::fence_before_sync();
             __syncwarp();
@@ -439,7 +480,8 @@ void launch_kernel(dim3 grid, cudaStream_t stream, const CUtensorMap& ta, const 
                              (int)SMEM_BYTES);
         configured = true;
     }
-    gemm_tc_kernel<A_MN, B_MN, KIND><<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, M, N, u, ep, status);
+    gemm_tc_kernel<A_MN, B_MN, KIND><<<grid, EpiTraits<KIND>::THREADS, SMEM_BYTES, stream>>>(ta, tb, M, N, u, ep,
+                                                                                             status);
 }
 
 template <int A_MN, int B_MN>
