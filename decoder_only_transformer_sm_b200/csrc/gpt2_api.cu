@@ -144,6 +144,11 @@ struct gpt2_handle {
     int* d_window = nullptr;         // contiguous token window of a prefill inside gpt2_generate (maxBT)
     int kv_B = 0, kv_len = 0;        // rows and positions the cache holds
 
+    // Data-parallel exchange: caller-owned events recorded as each gradient bucket
+    // becomes final in an eager backward (not inside a graph capture).
+    std::vector<cudaEvent_t> grad_events;
+    bool capturing = false;
+
     bool profiling = false;
     std::vector<ProfSite> psites;
     std::unordered_map<std::string, int> pidx;
@@ -506,6 +511,23 @@ void forward_impl(gpt2_handle* h, const int* idx, const int* targets, int B, int
 }
 
 // ----------------------------------------------------------------- backward
+// Gradient buckets in the order the backward finishes them: ln_f, block L-1, ...,
+// block 0, then wte and wpe (the embedding backward adds into the tied wte last).
+void grad_buckets(const gpt2_handle* h, std::vector<std::pair<long long, long long>>& out) {
+    out.clear();
+    out.push_back({h->off_lnfw, h->n_params - h->off_lnfw});
+    for (int l = h->L - 1; l >= 0; --l) {
+        const long long end = l + 1 < h->L ? h->lo[l + 1].ln1w : h->off_lnfw;
+        out.push_back({h->lo[l].ln1w, end - h->lo[l].ln1w});
+    }
+    out.push_back({0, h->lo[0].ln1w});
+}
+
+// Bucket k of grad_buckets is final: record the caller's event k.
+void bucket_done(gpt2_handle* h, int k) {
+    if (!h->grad_events.empty() && !h->capturing) cudaEventRecord(h->grad_events[k], h->stream);
+}
+
 template <typename A>
 void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
     Ctx c = h->ctx();
@@ -525,6 +547,7 @@ void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
          launch_layernorm_bwd<A>(c, (const A*)h->dtmp, h->resid[2 * L], h->ln_mean[2 * L], h->ln_rstd[2 * L],
                                  P + h->off_lnfw, nullptr, h->dres, (A*)h->dres_act, G + h->off_lnfw,
                                  G + h->off_lnfb, G + h->lo[L - 1].bfcp, BT, C, h->red_scratch));
+    bucket_done(h, 0);   // ln_f
     for (int l = L - 1; l >= 0; --l) {
         const LayerOff& o = h->lo[l];
         // mlp.c_proj: dW += dY^T g ; du = (dY W) * gelu'(u)
@@ -587,9 +610,11 @@ void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
              launch_layernorm_bwd<A>(c, (const A*)h->dtmp, h->resid[2 * l], h->ln_mean[2 * l], h->ln_rstd[2 * l],
                                      P + o.ln1w, h->dres, h->dres, (A*)h->dres_act, G + o.ln1w, G + o.ln1b,
                                      l > 0 ? G + h->lo[l - 1].bfcp : nullptr, BT, C, h->red_scratch));
+        bucket_done(h, L - l);   // block l (its mlp.c_proj bias gradient was added by block l+1 or ln_f)
     }
     PROF("embedding bwd", 0, 0, 0, 0.0, (double)BT * C * 12 + (double)T * C * 8,
          launch_embed_bwd(c, idx, h->dres, B, T, C, V, G + h->off_wte, G + h->off_wpe));
+    bucket_done(h, L + 1);   // wte, wpe
 }
 
 // -------------------------------------------------------------- generation
@@ -789,7 +814,9 @@ int grad_pass_impl(gpt2_handle* h, int B, int T) {
     const long long l0 = h->launches;
     CK(cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal));
     h->stream = h->cap_stream;
+    h->capturing = true;
     int rc = eager();
+    h->capturing = false;
     h->stream = user;
     cudaGraph_t g = nullptr;
     cudaError_t e = cudaStreamEndCapture(h->cap_stream, &g);
@@ -1353,6 +1380,36 @@ int gpt2_profile_read(gpt2_handle* h, gpt2_kernel_stat* out, int capacity, int* 
         out[i].flops = h->psites[i].flops;
         out[i].bytes = h->psites[i].bytes;
     }
+    return GPT2_OK;
+}
+
+int gpt2_grad_buckets(const gpt2_handle* h, int64_t* offsets, int64_t* counts, int capacity, int* n) {
+    if (!h || !n) return fail(GPT2_ERR_INVALID_ARG, "NULL argument");
+    std::vector<std::pair<long long, long long>> b;
+    grad_buckets(h, b);
+    *n = (int)b.size();
+    if (!offsets && !counts) return GPT2_OK;
+    if (!offsets || !counts || capacity < *n) return fail(GPT2_ERR_INVALID_ARG, "need offsets, counts and capacity >= n");
+    for (size_t i = 0; i < b.size(); ++i) {
+        offsets[i] = b[i].first;
+        counts[i] = b[i].second;
+    }
+    return GPT2_OK;
+}
+
+int gpt2_set_grad_events(gpt2_handle* h, void* const* events, int n) {
+    if (!h) return fail(GPT2_ERR_INVALID_ARG, "NULL handle");
+    if (!events || n == 0) {
+        h->grad_events.clear();
+        return GPT2_OK;
+    }
+    if (n != h->L + 2) return fail(GPT2_ERR_INVALID_ARG, "n must be the bucket count (n_layer + 2)");
+    std::vector<cudaEvent_t> ev(n);
+    for (int i = 0; i < n; ++i) {
+        if (!events[i]) return fail(GPT2_ERR_INVALID_ARG, "NULL event");
+        ev[i] = (cudaEvent_t)events[i];
+    }
+    h->grad_events = ev;
     return GPT2_OK;
 }
 

@@ -90,6 +90,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gpt2_step": (I, [P, P, P, I, I, F, ctypes.POINTER(F), ctypes.POINTER(F)]),
         "gpt2_step_host": (I, [P, P, P, I, I, F, ctypes.POINTER(F), ctypes.POINTER(F)]),
         "gpt2_last_launch_count": (I, [P, ctypes.POINTER(ctypes.c_int64)]),
+        "gpt2_grad_buckets": (I, [P, P, P, I, ctypes.POINTER(I)]),
+        "gpt2_set_grad_events": (I, [P, P, I]),
         "gpt2_profile": (I, [P, I]),
         "gpt2_profile_read": (I, [P, P, I, ctypes.POINTER(I)]),
         "gpt2k_matmul_bf16": (I, [I, P, P, I, I, I, I, P, ctypes.c_int64, P, P, P, P, P, F, I, P, P]),
@@ -210,6 +212,28 @@ class GPT2:
         ptr, n = ctypes.c_void_p(), ctypes.c_int64()
         _check(self._lib.gpt2_grads_device(self._h, ctypes.byref(ptr), ctypes.byref(n)))
         return torch.as_tensor(_DeviceArray(ptr.value, n.value), device="cuda")
+
+    def grad_buckets(self):
+        """[(offset, count)] ranges of the flat gradient vector in the order the
+        backward finishes them (gpt2_grad_buckets)."""
+        n = ctypes.c_int()
+        _check(self._lib.gpt2_grad_buckets(self._h, None, None, 0, ctypes.byref(n)))
+        off = np.empty(n.value, np.int64)
+        cnt = np.empty(n.value, np.int64)
+        _check(self._lib.gpt2_grad_buckets(self._h, _ptr(off), _ptr(cnt), n.value, ctypes.byref(n)))
+        return [(int(o), int(c)) for o, c in zip(off, cnt)]
+
+    def set_grad_events(self, events):
+        """torch.cuda.Event per bucket, recorded by every eager backward as each bucket
+        becomes final (gpt2_set_grad_events); None stops the recording. The events are
+        kept alive here while set."""
+        if events is None:
+            _check(self._lib.gpt2_set_grad_events(self._h, None, 0))
+            self._grad_events = None
+            return
+        handles = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
+        _check(self._lib.gpt2_set_grad_events(self._h, handles, len(events)))
+        self._grad_events = list(events)
 
     def get_opt_state(self):
         m = np.empty(self.n_params, np.float32)

@@ -317,6 +317,28 @@ int gpt2_step_host(gpt2_handle* h, const int32_t* idx_host, const int32_t* targe
  * Errors: INVALID_ARG (step < 0, warmup < 1, max_steps < warmup, lr_out NULL). */
 int gpt2_lr_at(int64_t step, float max_lr, float min_lr, int64_t warmup, int64_t max_steps, float* lr_out);
 
+/* Gradient buckets for the data-parallel exchange ("Let's reproduce GPT-2
+ * (124M)", "Scaling to 8 GPUs with DistributedDataParallel": every process
+ * averages its gradients with the others' before the update; the pages' DDP
+ * overlaps that exchange with the backward). The flat gradient vector splits
+ * into contiguous ranges that the backward finishes one after another: ln_f,
+ * block n_layer-1, ..., block 0, then wte and wpe (the embedding backward adds
+ * into the tied wte last). offsets and counts (host, capacity entries, in
+ * elements of the flat vector) receive the ranges in that order and *n their
+ * number, n_layer + 2. With offsets and counts NULL only *n is written.
+ * Errors: INVALID_ARG (NULL handle or n, capacity below the count). */
+int gpt2_grad_buckets(const gpt2_handle* h, int64_t* offsets, int64_t* counts, int capacity, int* n);
+
+/* events: n CUDA events (cudaEvent_t, created by the caller on the handle's
+ * device and owned by it) that every eager backward (gpt2_accumulate, and the
+ * first step of a (B, T) in gpt2_step / gpt2_step_host) records on the handle's
+ * stream, event k as soon as bucket k of gpt2_grad_buckets is final; a collective
+ * on bucket k may then start on another stream while the backward continues.
+ * Backwards replayed from the step graph record nothing. n must be the bucket
+ * count; events NULL or n = 0 stops the recording. The events must outlive the
+ * setting. Errors: INVALID_ARG (NULL handle, a wrong n, a NULL event). */
+int gpt2_set_grad_events(gpt2_handle* h, void* const* events, int n);
+
 /* Number of kernel launches the last forward/accumulate/update/step issued. */
 int gpt2_last_launch_count(const gpt2_handle* h, int64_t* n);
 

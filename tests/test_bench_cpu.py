@@ -42,7 +42,7 @@ def test_workload_config_and_metric_names():
     w = bench.WORKLOAD
     c = bench.workload_config(w["B"], w["T"], 1)
     assert c["tokens_per_step_per_gpu"] == w["B"] * w["T"] and c["parallelism"] == "single-gpu"
-    assert bench.workload_config(w["B"], w["T"], 8)["parallelism"] == "replicas"
+    assert bench.workload_config(w["B"], w["T"], 8)["parallelism"].startswith("dp8")
     assert bench.metric_for(w, w["B"], w["T"]) == bench.METRIC
     assert bench.metric_for(bench.MODELS["xl"], 4, 1024) != bench.METRIC
     # 6N + 12 L C T with the tied wte counted once at the padded vocabulary

@@ -45,6 +45,20 @@ class OracleModel:
     def grads_view(self):
         return self.g
 
+    def grad_buckets(self):
+        """The flat layout's ranges in the order a backward finishes them: ln_f,
+        the blocks from the last to the first, then wte and wpe."""
+        offs, o = {}, 0
+        for name, shp in O.layout(self.s):
+            offs[name] = o
+            o += int(np.prod(shp))
+        L = self.s.n_layer
+        start = [offs[f"h.{l}.ln_1.weight"] for l in range(L)] + [offs["ln_f.weight"]]
+        out = [(offs["ln_f.weight"], o - offs["ln_f.weight"])]
+        out += [(start[l], start[l + 1] - start[l]) for l in range(L - 1, -1, -1)]
+        out.append((0, start[0]))
+        return out
+
     def update(self, lr):
         G = O.unflatten(self.s, self.g.numpy())
         self.t += 1
@@ -78,7 +92,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank_main(rank, world, port, out_dir):
+def _rank_main(rank, world, port, out_dir, bucketed):
     import torch.distributed as dist
     from decoder_only_transformer_sm_b200.ddp import DataParallel
     os.environ["MASTER_ADDR"] = "127.0.0.1"
@@ -87,7 +101,8 @@ def _rank_main(rank, world, port, out_dir):
     try:
         # rank 1 starts from other weights: broadcast_params must replace them
         flat = S.random_params(_syn(MICRO), seed=77 + rank).astype(np.float64)
-        dp = DataParallel(OracleModel(MICRO, flat))
+        dp = DataParallel(OracleModel(MICRO, flat), bucketed=bucketed)
+        assert (dp.buckets is not None) == bucketed
         dp.broadcast_params()
         res = [dp.step(_batches(rank), LR) for _ in range(2)]
         np.savez(os.path.join(out_dir, f"r{rank}.npz"), params=dp.model.get_params(),
@@ -96,10 +111,22 @@ def _rank_main(rank, world, port, out_dir):
         dist.destroy_process_group()
 
 
-def test_two_ranks_equal_one_process_over_the_combined_batches(tmp_path):
+def test_oracle_model_buckets_partition_the_gradient():
+    m = OracleModel(MICRO, S.random_params(_syn(MICRO), seed=1).astype(np.float64))
+    b = m.grad_buckets()
+    assert len(b) == MICRO.n_layer + 2
+    assert sum(c for _, c in b) == len(m.g)
+    ends = sorted(b)
+    assert all(ends[i][0] + ends[i][1] == ends[i + 1][0] for i in range(len(ends) - 1))
+    assert b[-1][0] == 0 and b[0][0] + b[0][1] == len(m.g)      # wte/wpe last, ln_f first
+
+
+@pytest.mark.parametrize("bucketed", [True, False])
+def test_two_ranks_equal_one_process_over_the_combined_batches(tmp_path, bucketed):
     import torch.multiprocessing as mp
     world = 2
-    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, start_method="spawn")
+    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path), bucketed), nprocs=world,
+                       start_method="spawn")
     r = [np.load(tmp_path / f"r{k}.npz") for k in range(world)]
     assert np.array_equal(r[0]["params"], r[1]["params"])          # the replicas stay identical
     assert np.array_equal(r[0]["losses"], r[1]["losses"])

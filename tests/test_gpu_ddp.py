@@ -81,3 +81,59 @@ def test_single_rank_nccl_allreduce_then_update_equals_step():
         b.close()
     finally:
         dist.destroy_process_group()
+
+
+def test_grad_buckets_follow_the_backward_order():
+    """gpt2_grad_buckets: ln_f, blocks n_layer-1 .. 0, then wte and wpe; together
+    they cover the flat gradient vector once."""
+    from oracle import gpt2_oracle as O
+    m = _model()
+    b = m.grad_buckets()
+    s = TINY
+    offs, o = {}, 0
+    for name, shp in O.layout(O.Shape(s.n_layer, s.n_head, s.n_embd, s.vocab_size, s.block_size)):
+        offs[name] = o
+        o += int(np.prod(shp))
+    assert o == m.n_params and len(b) == s.n_layer + 2
+    assert b[0] == (offs["ln_f.weight"], m.n_params - offs["ln_f.weight"])
+    for k, l in enumerate(range(s.n_layer - 1, -1, -1), start=1):
+        end = offs[f"h.{l + 1}.ln_1.weight"] if l + 1 < s.n_layer else offs["ln_f.weight"]
+        assert b[k] == (offs[f"h.{l}.ln_1.weight"], end - offs[f"h.{l}.ln_1.weight"])
+    assert b[-1] == (0, offs["h.0.ln_1.weight"])
+    m.close()
+
+
+def test_bucketed_exchange_on_one_nccl_rank_equals_step():
+    """The bucketed exchange on a one-rank NCCL group: the library records one
+    event per bucket in the backward, the communication stream waits for each and
+    all-reduces that bucket (the identity over one rank), the update waits for
+    the communication stream; the result equals a plain step."""
+    import torch.distributed as dist
+    from decoder_only_transformer_sm_b200.ddp import DataParallel
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    try:
+        flat = S.random_params(TINY, seed=64)
+        idx, tgt = S.uniform_tokens(2, 32, TINY.vocab_size, seed=65)
+        a, b = _model("bf16"), _model("bf16")
+        a.set_params(flat)
+        b.set_params(flat)
+        dp = DataParallel(a)
+        assert dp.buckets == a.grad_buckets() and dp.comm is not None and len(dp.events) == len(dp.buckets)
+        for step in range(2):
+            a.zero_grad()
+            a.accumulate(_dev(idx), _dev(tgt), 1.0)
+            dp._exchange(a.grads_view())
+            torch.cuda.current_stream().synchronize()
+            assert all(ev.query() for ev in dp.events)
+            loss_a, norm_a = a.update(6e-4)
+            loss_b, norm_b = b.step(_dev(idx), _dev(tgt), 6e-4)
+            assert loss_a == pytest.approx(loss_b, rel=1e-6)
+            assert norm_a == pytest.approx(norm_b, rel=1e-5)
+        a.set_grad_events(None)
+        a.close()
+        b.close()
+    finally:
+        dist.destroy_process_group()
