@@ -338,15 +338,27 @@ template <typename A>
 void gemm_raw(gpt2_handle* h, GemmLayout layout, const void* a, const void* b, int M, int N, int K,
               const Epilogue& ep);
 
+// A handful of rows (a decode step, last-position logits) on the weight-streaming
+// kernel, which spreads the weight rows over every SM.
+template <typename A>
+bool gemm_few_rows(gpt2_handle* h, GemmLayout layout, const void* a, const void* b, int M, int N, int K,
+                   const Epilogue& ep) {
+    if (layout != GEMM_NT || !gemv_supported(sizeof(A), M, K) || ep.split_atomic) return false;
+    launch_gemv<A>(h->ctx(), (const A*)a, (const A*)b, M, N, K, ep);
+    return true;
+}
+
 template <>
 void gemm_raw<float>(gpt2_handle* h, GemmLayout layout, const void* a, const void* b, int M, int N, int K,
                      const Epilogue& ep) {
+    if (gemm_few_rows<float>(h, layout, a, b, M, N, K, ep)) return;
     launch_gemm_simt<float>(h->ctx(), layout, (const float*)a, (const float*)b, M, N, K, ep);
 }
 
 template <>
 void gemm_raw<bf16>(gpt2_handle* h, GemmLayout layout, const void* a, const void* b, int M, int N, int K,
                     const Epilogue& ep) {
+    if (gemm_few_rows<bf16>(h, layout, a, b, M, N, K, ep)) return;
     if (h->use_tc_gemm && gemm_tc_supported(layout, M, N, K)) {
         if (!launch_gemm_tc(h->ctx(), layout, (const bf16*)a, (const bf16*)b, M, N, K, ep))
             h->host_error = "tensor-map encoding failed for a tensor-core GEMM";

@@ -206,9 +206,18 @@ __global__ void __launch_bounds__(SMP_THREADS)
         for (int shift = 24; shift >= 0; shift -= 8) {
             for (int i = tid; i < 256; i += SMP_THREADS) hist[i] = 0;
             __syncthreads();
-            for (int i = tid; i < V; i += SMP_THREADS) {
-                const unsigned k = order_key(to_f(x[i]));
-                if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+            // Values of one row tend to share their high key bytes, so most keys of a
+            // pass fall into a few bins: the lanes of a warp that hit one bin add once
+            // (warp-aggregated), instead of 32 adds to one address.
+            for (int i0 = 0; i0 < V; i0 += SMP_THREADS) {
+                const int i = i0 + tid;
+                unsigned bin = 256u;   // no bin: out of range, or outside the prefix
+                if (i < V) {
+                    const unsigned k = order_key(to_f(x[i]));
+                    if ((k & mask) == prefix) bin = (k >> shift) & 255u;
+                }
+                const unsigned peers = __match_any_sync(0xffffffffu, bin);
+                if (bin < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (unsigned)__popc(peers));
             }
             __syncthreads();
             if (tid == 0) {

@@ -61,6 +61,14 @@ bool gemm_tc_supported(GemmLayout layout, int M, int N, int K);
 bool launch_gemm_tc(const Ctx& ctx, GemmLayout layout, const bf16* A, const bf16* B, int M, int N, int K,
                     const Epilogue& ep);
 
+// Weight-streaming GEMM for M <= GEMV_MAX_M rows, NT layout only: out(m, n) =
+// sum_k A[m, k] B[n, k] through the epilogue ep (every kind; epilogue_scalar's
+// arithmetic). gemv_supported: the row count and 16-byte rows of A and B.
+constexpr int GEMV_MAX_M = 4;
+bool gemv_supported(size_t elem_size, int M, int K);
+template <typename T>
+void launch_gemv(const Ctx& ctx, const T* A, const T* B, int M, int N, int K, const Epilogue& ep);
+
 // ----------------------------------------------------------------------------
 // Row-wise kernels.
 // ----------------------------------------------------------------------------

@@ -18,7 +18,9 @@ fills a key/value cache with a prefill and then runs one position per draw.
     all three branches of the loop: the first prefill, decode steps, and the
     re-prefill of the cropped window once the sequence outgrows block_size.
   * bf16 generation, whose draws the bf16 logit error can flip, against the same
-    loop composed of the single calls (prefill, decode, sample): equal tokens.
+    loop composed of the single calls (prefill, decode, sample): equal tokens; and
+    for the pages' call at 124M, the logits of every one of its 40 draws,
+    teacher-forced with the generated tokens, against the oracle's forward.
 """
 import numpy as np
 import pytest
@@ -307,3 +309,34 @@ def test_124m_decode_logits_and_generation_loop():
     m.generate(_dev(prompt), 40, 0.8, 40, u, out)
     assert np.array_equal(out.cpu().numpy(), _composed_loop(m, W, prompt, 40, 0.8, 40, u, torch.bfloat16))
     m.close()
+
+
+def test_124m_pages_call_decode_logits_match_oracle_at_every_step():
+    """The pages' sampling call on GPT-2 124M in bf16 (one prompt of 4 tokens, 40
+    new tokens, temperature 0.8, top-k 40) through gpt2_generate; then its tokens,
+    teacher-forced through prefill + decode, give the logits of all 40 draws, each
+    compared with the oracle's forward over the generated sequence at the same
+    position (one causal forward gives every prefix's last position): 3e-2 of max
+    |logit| and cosine > 0.999, the tolerances of the full-size forward check."""
+    OS = _oshape(W)
+    m = _model(W, "bf16", 1, W.block_size, seed=3)
+    flat = S.init_params(W, seed=0)
+    m.set_params(flat)
+    prompt = S.zipf_tokens(1, 4, W.real_vocab, seed=1001)[0]
+    u = torch.from_numpy(S.uniforms(40, 1, seed=1002)).cuda()
+    out = torch.full((1, 44), -1, dtype=torch.int32, device="cuda")
+    m.generate(_dev(prompt), 40, 0.8, 40, u, out)
+    seq = out.cpu().numpy()
+    assert np.array_equal(seq[:, :4], prompt) and seq.min() >= 0 and seq.max() < W.vocab_size
+    lg = torch.empty((1, W.vocab_size), dtype=torch.bfloat16, device="cuda")
+    m.prefill(_dev(seq[:, :4]), lg)
+    got = [lg.float().cpu().numpy()[0]]
+    for i in range(39):
+        m.decode(_dev(seq[:, 4 + i]), 4 + i, lg)
+        got.append(lg.float().cpu().numpy()[0])
+    m.close()
+    _, ref, _ = O.forward(OS, O.unflatten(OS, flat), seq[:, :43])
+    for i, g in enumerate(got):
+        r = ref[0, 3 + i]
+        assert np.max(np.abs(g - r)) / np.max(np.abs(r)) < 3e-2, i
+        assert _cos(g, r) > 0.999, i
