@@ -48,6 +48,16 @@ __device__ __forceinline__ void store4(bf16* p, const float v[4]) {
     *reinterpret_cast<uint2*>(p) = q;
 }
 
+// Programmatic dependent launch (sm_90 and later). A kernel launched with the
+// programmatic stream serialisation attribute may start while its predecessor
+// in the stream still runs: griddep_wait blocks until that predecessor has
+// completed and its writes are visible (a no-op for a kernel launched without
+// the attribute), griddep_launch lets the next such kernel start. Every block
+// of a kernel launched this way calls griddep_wait before it ends, so each
+// kernel of a chain completes after all kernels before it.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ reductions
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

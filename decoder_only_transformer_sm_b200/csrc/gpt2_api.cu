@@ -143,6 +143,18 @@ struct gpt2_handle {
     int* d_next = nullptr;           // last drawn token per row (max_B): the next decode step's input
     int* d_window = nullptr;         // contiguous token window of a prefill inside gpt2_generate (maxBT)
     int kv_B = 0, kv_len = 0;        // rows and positions the cache holds
+    // gpt2_generate's decode steps read their position, draw index and output
+    // slot from d_dec, so one captured step (decode, draw, advance of d_dec)
+    // serves every position: captured on the second step with the same
+    // (B, temperature, top_k) (the first runs the same launches eagerly).
+    DecodeArgs* d_dec = nullptr;
+    cudaGraphExec_t dec_graph = nullptr;
+    bool dec_seen = false;
+    int dec_B = 0, dec_top_k = 0;
+    float dec_temperature = 0.f;
+    long long dec_graph_launches = 0;
+    int* dec_counters = nullptr;     // (max_B * H) tickets of the decode attention, zero between calls
+    bool pdl = false;                // launch_pdl kernels get programmatic dependent launch
 
     // Data-parallel exchange: caller-owned events recorded as each gradient bucket
     // becomes final in an eager backward (not inside a graph capture).
@@ -162,8 +174,18 @@ struct gpt2_handle {
         c.status = &d_sc->status;
         c.launches = &launches;
         c.num_sms = num_sms;
+        c.pdl = pdl && !profiling;
         return c;
     }
+};
+
+// Programmatic dependent launch for the kernels enqueued while it lives (the
+// generation path's chains of short kernels; see launch_pdl).
+struct PdlScope {
+    gpt2_handle* h;
+    bool old;
+    explicit PdlScope(gpt2_handle* hh) : h(hh), old(hh->pdl) { h->pdl = true; }
+    ~PdlScope() { h->pdl = old; }
 };
 
 namespace {
@@ -343,7 +365,13 @@ void gemm_raw(gpt2_handle* h, GemmLayout layout, const void* a, const void* b, i
 template <typename A>
 bool gemm_few_rows(gpt2_handle* h, GemmLayout layout, const void* a, const void* b, int M, int N, int K,
                    const Epilogue& ep) {
-    if (layout != GEMM_NT || !gemv_supported(sizeof(A), M, K) || ep.split_atomic) return false;
+    if (layout != GEMM_NT || !gemv_supported(sizeof(A), M, K) || ep.split_atomic) {
+        if (ep.out_row_dev) {   // a device-picked output row needs this kernel
+            h->host_error = "a GEMM with a device-side output row needs the weight-streaming kernel";
+            return true;
+        }
+        return false;
+    }
     launch_gemv<A>(h->ctx(), (const A*)a, (const A*)b, M, N, K, ep);
     return true;
 }
@@ -639,8 +667,10 @@ int ensure_gen(gpt2_handle* h) {
     const size_t part = align_up((size_t)decode_part_floats(h->cfg.max_B * h->H, (int)Tc, h->hd) * 4);
     const size_t ptrs = align_up(2 * L * sizeof(void*));
     const size_t next = align_up(Bm * 4), win = align_up((size_t)h->maxBT * 4);
+    const size_t dargs = align_up(sizeof(DecodeArgs));
+    const size_t cnt = align_up(Bm * h->H * sizeof(int));
     char* pool = nullptr;
-    if (cudaMalloc((void**)&pool, L * layer + part + ptrs + next + win) != cudaSuccess) {
+    if (cudaMalloc((void**)&pool, L * layer + part + ptrs + next + win + dargs + cnt) != cudaSuccess) {
         cudaGetLastError();
         return fail(GPT2_ERR_OOM, "cudaMalloc of the key/value cache failed");
     }
@@ -654,6 +684,10 @@ int ensure_gen(gpt2_handle* h) {
     int* d_next = (int*)(pool + off);
     off += next;
     int* d_window = (int*)(pool + off);
+    off += win;
+    DecodeArgs* d_dec = (DecodeArgs*)(pool + off);
+    off += dargs;
+    int* dec_counters = (int*)(pool + off);
     std::vector<void*> tab(2 * L);
     for (size_t l = 0; l < L; ++l) {
         tab[l] = h->qkv[l];
@@ -662,6 +696,7 @@ int ensure_gen(gpt2_handle* h) {
     // the handle takes the pool only once the pointer table is on the device
     cudaError_t e = cudaMemcpyAsync(layer_ptrs, tab.data(), tab.size() * sizeof(void*), cudaMemcpyHostToDevice,
                                     h->stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dec_counters, 0, cnt, h->stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(h->stream);
     if (e != cudaSuccess) {
         cudaFree(pool);
@@ -673,6 +708,8 @@ int ensure_gen(gpt2_handle* h) {
     h->d_layer_ptrs = layer_ptrs;
     h->d_next = d_next;
     h->d_window = d_window;
+    h->d_dec = d_dec;
+    h->dec_counters = dec_counters;
     h->kv_B = h->kv_len = 0;
     return GPT2_OK;
 }
@@ -688,59 +725,105 @@ void prefill_impl(gpt2_handle* h, const int* idx, int B, int T, A* logits_out) {
                          h->cfg.block_size, h->C, (int)sizeof(A)));
 }
 
+// A decode GEMM whose operand is LN(ln.x) with (ln.w, ln.b), the LayerNorm
+// computed inside the weight-streaming kernel.
+template <typename A>
+void gemv_ln(gpt2_handle* h, const char* site, long long w_off, int M, int N, int K, const Epilogue& ep,
+             const LnIn& ln) {
+    PROF(site, M, N, K, 2.0 * M * N * K, gemm_bytes(M, N, K, sizeof(A), ep) + (double)M * K * (4.0 - sizeof(A)),
+         launch_gemv<A>(h->ctx(), nullptr, wop<A>(h, w_off), M, N, K, ep, ln));
+}
+
 // One new position `pos` of B sequences whose cache holds rows 0 .. pos-1:
 // the blocks' forward for tok (B) at that position, its q, k, v written to
-// cache row pos, attention over rows 0 .. pos, logits (B, V).
+// cache row pos, attention over rows 0 .. pos, logits (B, V). With pos_dev the
+// position is *pos_dev, read on the device by the embedding, the c_attn GEMM's
+// output row and the attention (the host's pos then only sizes the profile).
+// With at most GEMV_MAX_M rows every GEMM runs on the weight-streaming kernel
+// and the LayerNorms before c_attn (after the first), c_fc and lm_head run
+// inside it; the kernels are chained by programmatic dependent launch.
 template <typename A>
-void decode_impl(gpt2_handle* h, const int* tok, int B, int pos, A* logits_out) {
+void decode_impl(gpt2_handle* h, const int* tok, int B, int pos, A* logits_out, const int* pos_dev = nullptr) {
+    PdlScope pdl(h);
     Ctx c = h->ctx();
     const int C = h->C, V = h->V, L = h->L, H = h->H, hd = h->hd, Tc = h->cfg.block_size;
     const long long ld_kv = 3LL * C * Tc;
     const double es = sizeof(A);
     const double ln_fwd_bytes = (double)B * C * (4 + es) + 8.0 * B;
     const int n = pos + 1;
+    const bool fuse = gemv_supported(sizeof(A), B, C) && gemv_supported(sizeof(A), B, 4 * C);
     float* P = h->params;
     PROF("decode embed+ln_1", 0, 0, 0, 0.0, (double)B * C * (4 + 4 + 4 + es),
-         launch_embed_ln<A>(c, tok, P + h->off_wte, P + h->off_wpe + (long long)pos * C, B, 1, C, V,
-                            P + h->lo[0].ln1w, P + h->lo[0].ln1b, h->resid[0], (A*)h->ln1[0], h->ln_mean[0],
-                            h->ln_rstd[0]));
+         launch_embed_ln<A>(c, tok, P + h->off_wte, P + h->off_wpe + (pos_dev ? 0 : (long long)pos * C), B, 1, C,
+                            V, P + h->lo[0].ln1w, P + h->lo[0].ln1b, h->resid[0], (A*)h->ln1[0], h->ln_mean[0],
+                            h->ln_rstd[0], pos_dev));
     for (int l = 0; l < L; ++l) {
         const LayerOff& o = h->lo[l];
-        Epilogue e = epi(EPI_BIAS, (A*)h->kv[l] + (long long)pos * 3 * C, ld_kv);
+        Epilogue e = epi(EPI_BIAS, (A*)h->kv[l] + (pos_dev ? 0 : (long long)pos * 3 * C), ld_kv);
         e.bias = P + o.bqkv;
-        gemm<A>(h, "decode gemm c_attn", GEMM_NT, h->ln1[l], wop<A>(h, o.wqkv), B, 3 * C, C, e);
+        e.out_row_dev = pos_dev;
+        e.out_row_bytes = 3LL * C * (long long)sizeof(A);
+        if (fuse && l > 0) {
+            LnIn ln;
+            ln.x = h->resid[2 * l];
+            ln.w = P + o.ln1w;
+            ln.b = P + o.ln1b;
+            gemv_ln<A>(h, "decode ln_1+gemm c_attn", o.wqkv, B, 3 * C, C, e, ln);
+        } else {
+            gemm<A>(h, "decode gemm c_attn", GEMM_NT, h->ln1[l], wop<A>(h, o.wqkv), B, 3 * C, C, e);
+        }
         PROF("decode attention", 0, 0, 0, 4.0 * B * H * (double)n * hd, (double)B * n * 2 * C * es,
-             launch_attention_decode<A>(c, (const A*)h->kv[l], (A*)h->att[l], h->dec_part, B, H, hd, Tc, n));
+             launch_attention_decode<A>(c, (const A*)h->kv[l], (A*)h->att[l], h->dec_part, B, H, hd, Tc, n,
+                                        pos_dev, h->dec_counters));
         e = epi(EPI_BIAS_RESID, h->resid[2 * l + 1], C);
         e.bias = P + o.bproj;
         e.resid = h->resid[2 * l];
         gemm<A>(h, "decode gemm attn.c_proj", GEMM_NT, h->att[l], wop<A>(h, o.wproj), B, C, C, e);
-        PROF("decode layernorm", 0, 0, 0, 0.0, ln_fwd_bytes,
-             launch_layernorm_fwd<A>(c, h->resid[2 * l + 1], P + o.ln2w, P + o.ln2b, (A*)h->ln2[l],
-                                     h->ln_mean[2 * l + 1], h->ln_rstd[2 * l + 1], B, C));
         e = epi(EPI_BIAS_GELU, h->fcg[l], 4 * C);
         e.out2 = h->fch[l];
         e.bias = P + o.bfc;
-        gemm<A>(h, "decode gemm c_fc+gelu", GEMM_NT, h->ln2[l], wop<A>(h, o.wfc), B, 4 * C, C, e);
+        if (fuse) {
+            LnIn ln;
+            ln.x = h->resid[2 * l + 1];
+            ln.w = P + o.ln2w;
+            ln.b = P + o.ln2b;
+            gemv_ln<A>(h, "decode ln_2+gemm c_fc+gelu", o.wfc, B, 4 * C, C, e, ln);
+        } else {
+            PROF("decode layernorm", 0, 0, 0, 0.0, ln_fwd_bytes,
+                 launch_layernorm_fwd<A>(c, h->resid[2 * l + 1], P + o.ln2w, P + o.ln2b, (A*)h->ln2[l],
+                                         h->ln_mean[2 * l + 1], h->ln_rstd[2 * l + 1], B, C));
+            gemm<A>(h, "decode gemm c_fc+gelu", GEMM_NT, h->ln2[l], wop<A>(h, o.wfc), B, 4 * C, C, e);
+        }
         e = epi(EPI_BIAS_RESID, h->resid[2 * l + 2], C);
         e.bias = P + o.bfcp;
         e.resid = h->resid[2 * l + 1];
         gemm<A>(h, "decode gemm mlp.c_proj", GEMM_NT, h->fcg[l], wop<A>(h, o.wfcp), B, C, 4 * C, e);
         const bool last = (l + 1 == L);
-        PROF("decode layernorm", 0, 0, 0, 0.0, ln_fwd_bytes,
-             launch_layernorm_fwd<A>(c, h->resid[2 * l + 2], last ? P + h->off_lnfw : P + h->lo[l + 1].ln1w,
-                                     last ? P + h->off_lnfb : P + h->lo[l + 1].ln1b,
-                                     last ? (A*)h->lnf : (A*)h->ln1[l + 1], h->ln_mean[2 * l + 2],
-                                     h->ln_rstd[2 * l + 2], B, C));
+        if (!fuse)
+            PROF("decode layernorm", 0, 0, 0, 0.0, ln_fwd_bytes,
+                 launch_layernorm_fwd<A>(c, h->resid[2 * l + 2], last ? P + h->off_lnfw : P + h->lo[l + 1].ln1w,
+                                         last ? P + h->off_lnfb : P + h->lo[l + 1].ln1b,
+                                         last ? (A*)h->lnf : (A*)h->ln1[l + 1], h->ln_mean[2 * l + 2],
+                                         h->ln_rstd[2 * l + 2], B, C));
     }
-    gemm<A>(h, "decode gemm lm_head", GEMM_NT, h->lnf, wop<A>(h, h->off_wte), B, V, C, epi(EPI_STORE, logits_out, V));
+    if (fuse) {
+        LnIn ln;
+        ln.x = h->resid[2 * L];
+        ln.w = P + h->off_lnfw;
+        ln.b = P + h->off_lnfb;
+        gemv_ln<A>(h, "decode ln_f+gemm lm_head", h->off_wte, B, V, C, epi(EPI_STORE, logits_out, V), ln);
+    } else {
+        gemm<A>(h, "decode gemm lm_head", GEMM_NT, h->lnf, wop<A>(h, h->off_wte), B, V, C,
+                epi(EPI_STORE, logits_out, V));
+    }
 }
 
 template <typename A>
 void sample_impl(gpt2_handle* h, const A* logits, int B, float temperature, int top_k, const float* u, int* next,
-                 int* out, long long out_ld, int out_col) {
+                 int* out, long long out_ld, int out_col, const DecodeArgs* da = nullptr) {
     PROF("sample", 0, 0, 0, 0.0, (double)B * h->V * sizeof(A),
-         launch_sample<A>(h->ctx(), logits, h->V, B, h->V, temperature, top_k, u, next, out, out_ld, out_col));
+         launch_sample<A>(h->ctx(), logits, h->V, B, h->V, temperature, top_k, u, next, out, out_ld, out_col,
+                          da));
 }
 
 int check_sampling(float temperature) {
@@ -873,6 +956,64 @@ int update_impl(gpt2_handle* h, float lr, float* loss_host, float* norm_host) {
     return GPT2_OK;
 }
 
+// One decode step of gpt2_generate on the device arguments h->d_dec: decode at
+// position d_dec->pos, the draw d_dec->step into its output slot, then d_dec
+// advanced to the next position and draw. `pos` is the host's copy of the
+// position (profile sizes only).
+template <typename A>
+void decode_step_dev(gpt2_handle* h, int B, int pos, float temperature, int top_k) {
+    PdlScope pdl(h);
+    A* lg = (A*)h->logits;
+    decode_impl<A>(h, h->d_next, B, pos, lg, &h->d_dec->pos);
+    sample_impl<A>(h, lg, B, temperature, top_k, nullptr, h->d_next, nullptr, 0, 0, h->d_dec);
+    launch_decode_advance(h->ctx(), h->d_dec);
+}
+
+// decode_step_dev through its CUDA graph: eager on the first step with a
+// (B, temperature, top_k), captured on the second, replayed afterwards.
+template <typename A>
+int decode_step_graph(gpt2_handle* h, int B, int pos, float temperature, int top_k) {
+    const bool same = h->dec_B == B && h->dec_temperature == temperature && h->dec_top_k == top_k;
+    if (same && h->dec_graph) {
+        CK(cudaGraphLaunch(h->dec_graph, h->stream));
+        h->launches += h->dec_graph_launches;
+        return GPT2_OK;
+    }
+    if (!same || !h->dec_seen) {
+        if (h->dec_graph) cudaGraphExecDestroy(h->dec_graph);
+        h->dec_graph = nullptr;
+        h->dec_B = B;
+        h->dec_temperature = temperature;
+        h->dec_top_k = top_k;
+        h->dec_seen = true;
+        decode_step_dev<A>(h, B, pos, temperature, top_k);
+        return GPT2_OK;
+    }
+    if (!h->cap_stream) CK(cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking));
+    cudaStream_t user = h->stream;
+    const long long l0 = h->launches;
+    CK(cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal));
+    h->stream = h->cap_stream;
+    h->capturing = true;
+    decode_step_dev<A>(h, B, pos, temperature, top_k);
+    h->capturing = false;
+    h->stream = user;
+    cudaGraph_t g = nullptr;
+    cudaError_t e = cudaStreamEndCapture(h->cap_stream, &g);
+    if (h->host_error.empty() && e == cudaSuccess) e = cudaGraphInstantiate(&h->dec_graph, g, 0);
+    if (g) cudaGraphDestroy(g);
+    if (!h->host_error.empty()) return GPT2_OK;   // reported by the caller
+    if (e != cudaSuccess) {
+        h->dec_graph = nullptr;
+        return fail(GPT2_ERR_CUDA, std::string("decode graph capture failed: ") + cudaGetErrorString(e));
+    }
+    h->dec_graph_launches = h->launches - l0;
+    h->launches = l0;
+    CK(cudaGraphLaunch(h->dec_graph, h->stream));
+    h->launches += h->dec_graph_launches;
+    return GPT2_OK;
+}
+
 template <typename A>
 int generate_impl(gpt2_handle* h, const int* prompt, int B, int T0, int max_new, float temperature, int top_k,
                   const float* u, int* out) {
@@ -880,6 +1021,11 @@ int generate_impl(gpt2_handle* h, const int* prompt, int B, int T0, int max_new,
     Ctx c = h->ctx();
     PROF("token copy", 0, 0, 0, 0.0, 8.0 * B * T0, launch_copy_tokens(c, prompt, T0, out, Ttot, B, T0));
     A* lg = (A*)h->logits;
+    // decode steps on device arguments (and a graph) where every decode GEMM runs
+    // on the weight-streaming kernel, whose output row can be picked on the device
+    const bool dev_args = h->use_graphs && !h->profiling && gemv_supported(sizeof(A), B, h->C) &&
+                          gemv_supported(sizeof(A), B, 4 * h->C);
+    bool args_set = false;
     for (int s = 0; s < max_new; ++s) {
         const int n = T0 + s;   // tokens so far; the draw is token n
         if (s == 0 || n > Tb) {
@@ -889,6 +1035,15 @@ int generate_impl(gpt2_handle* h, const int* prompt, int B, int T0, int max_new,
             prefill_impl<A>(h, h->d_window, B, W, lg);
             h->kv_B = B;
             h->kv_len = W;
+            args_set = false;
+        } else if (dev_args) {
+            if (!args_set) launch_decode_set(c, h->d_dec, n - 1, s, u, out, Ttot, T0);
+            args_set = true;
+            const int rc = decode_step_graph<A>(h, B, n - 1, temperature, top_k);
+            if (rc) return rc;
+            h->kv_len = n;
+            if (!h->host_error.empty()) break;
+            continue;
         } else {
             decode_impl<A>(h, h->d_next, B, n - 1, lg);
             h->kv_len = n;
@@ -1037,6 +1192,7 @@ void gpt2_destroy(gpt2_handle* h) {
     if (!h) return;
     cudaStreamSynchronize(h->stream);
     if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
+    if (h->dec_graph) cudaGraphExecDestroy(h->dec_graph);
     if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
     cudaFree(h->params);
     cudaFree(h->grads);

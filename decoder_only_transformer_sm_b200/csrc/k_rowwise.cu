@@ -31,9 +31,12 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const int* __restrict__ idx
                                                       const float* __restrict__ x_in, const float* __restrict__ w,
                                                       const float* __restrict__ b, float* __restrict__ x_out,
                                                       T* __restrict__ y, float* __restrict__ mean,
-                                                      float* __restrict__ rstd, int rows, int C, unsigned* status) {
+                                                      float* __restrict__ rstd, int rows, int C, unsigned* status,
+                                                      const int* __restrict__ pos_dev) {
     const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
+    griddep_launch();
+    griddep_wait();
     if (row >= rows) return;
     float v[NV][4];
     const float* src;
@@ -45,7 +48,7 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const int* __restrict__ idx
             tok = tok < 0 ? 0 : V - 1;
         }
         src = wte + (long long)tok * C;
-        src2 = wpe + (long long)(row % Tn) * C;
+        src2 = wpe + (long long)((pos_dev ? *pos_dev : 0) + row % Tn) * C;
     } else {
         src = x_in + (long long)row * C;
     }
@@ -633,15 +636,14 @@ __global__ void embed_bwd_wpe_kernel(const float* __restrict__ dx, int B, int Tn
 template <typename T, bool EMBED>
 void ln_fwd_dispatch(const Ctx& ctx, const int* idx, const float* wte, const float* wpe, int Tn, int V,
                      const float* x_in, const float* w, const float* b, float* x_out, T* y, float* mean,
-                     float* rstd, int rows, int C) {
+                     float* rstd, int rows, int C, const int* pos_dev) {
     const int threads = 256;
     const int blocks = ceil_div(rows, threads / 32);
     const int nv = ceil_div(C, 128);
 #define LNF_CASE(N)                                                                                 \
     case N:                                                                                         \
-        ln_fwd_kernel<T, N, EMBED><<<blocks, threads, 0, ctx.stream>>>(idx, wte, wpe, Tn, V, x_in, w, b, \
-                                                                       x_out, y, mean, rstd, rows, C,  \
-                                                                       ctx.status);                  \
+        launch_pdl(ctx, ln_fwd_kernel<T, N, EMBED>, dim3(blocks), dim3(threads), 0, idx, wte, wpe, Tn, V, \
+                   x_in, w, b, x_out, y, mean, rstd, rows, C, ctx.status, pos_dev);                     \
         break;
     switch (nv) {
         LNF_CASE(1) LNF_CASE(2) LNF_CASE(3) LNF_CASE(4) LNF_CASE(5) LNF_CASE(6) LNF_CASE(7)
@@ -657,14 +659,16 @@ void ln_fwd_dispatch(const Ctx& ctx, const int* idx, const float* wte, const flo
 
 template <typename T>
 void launch_embed_ln(const Ctx& ctx, const int* idx, const float* wte, const float* wpe, int rows, int Tn, int C,
-                     int V, const float* w, const float* b, float* x, T* y, float* mean, float* rstd) {
-    ln_fwd_dispatch<T, true>(ctx, idx, wte, wpe, Tn, V, nullptr, w, b, x, y, mean, rstd, rows, C);
+                     int V, const float* w, const float* b, float* x, T* y, float* mean, float* rstd,
+                     const int* pos_dev) {
+    ln_fwd_dispatch<T, true>(ctx, idx, wte, wpe, Tn, V, nullptr, w, b, x, y, mean, rstd, rows, C, pos_dev);
 }
 
 template <typename T>
 void launch_layernorm_fwd(const Ctx& ctx, const float* x, const float* w, const float* b, T* y, float* mean,
                           float* rstd, int rows, int C) {
-    ln_fwd_dispatch<T, false>(ctx, nullptr, nullptr, nullptr, 1, 1, x, w, b, nullptr, y, mean, rstd, rows, C);
+    ln_fwd_dispatch<T, false>(ctx, nullptr, nullptr, nullptr, 1, 1, x, w, b, nullptr, y, mean, rstd, rows, C,
+                              nullptr);
 }
 
 template <typename T>
@@ -785,7 +789,7 @@ void launch_embed_bwd(const Ctx& ctx, const int* idx, const float* dx, int B, in
 
 #define INST(T)                                                                                                 \
     template void launch_embed_ln<T>(const Ctx&, const int*, const float*, const float*, int, int, int, int,   \
-                                     const float*, const float*, float*, T*, float*, float*);                  \
+                                     const float*, const float*, float*, T*, float*, float*, const int*);      \
     template void launch_layernorm_fwd<T>(const Ctx&, const float*, const float*, const float*, T*, float*,    \
                                           float*, int, int);                                                   \
     template void launch_layernorm_bwd<T>(const Ctx&, const T*, const float*, const float*, const float*,      \

@@ -11,7 +11,29 @@ struct Ctx {
     unsigned* status;      // device status word (STATUS_* bits)
     long long* launches;   // host counter of kernel launches
     int num_sms;
+    // launch_pdl adds the programmatic stream serialisation attribute (the
+    // kernels launched through it call griddep_wait in every block)
+    bool pdl = false;
 };
+
+// Launch of a kernel whose blocks all call griddep_wait before they end (and
+// griddep_launch): with ctx.pdl, programmatic dependent launch, so the kernel's
+// blocks start, and run up to griddep_wait, while its predecessor finishes.
+template <typename... KArgs, typename... Args>
+inline void launch_pdl(const Ctx& ctx, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = ctx.stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = ctx.pdl ? 1 : 0;
+    cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 // ----------------------------------------------------------------------------
 // GEMM epilogues. The contraction produces fp32 acc(row, col); the epilogue
@@ -40,6 +62,23 @@ struct Epilogue {
     // column sums of the bf16 results go to colsum_part[g * N + col]
     // (ceil(M / 32) x N floats); launch_colred_finalize adds them up.
     float* colsum_part = nullptr;
+    // weight-streaming kernel only: if set, out moves (*out_row_dev) * out_row_bytes
+    // bytes on before use (a row picked on the device, e.g. a key/value cache row)
+    const int* out_row_dev = nullptr;
+    long long out_row_bytes = 0;
+};
+
+// Device-resident arguments of one decode step of the generation loop, so that a
+// captured step can be replayed for every position: the new token's position
+// (the cache row written, the last key attended), the draw's index within the
+// call, and the call's uniforms and output rows.
+struct DecodeArgs {
+    int pos;
+    int step;
+    const float* u;      // (n_draws, B) uniforms of the call
+    int* out;            // (B, out_ld) token rows of the call
+    long long out_ld;
+    int out_col0;        // column of draw 0
 };
 
 // Operand layouts of C[M,N] = sum_k A(m,k) B(n,k):
@@ -64,18 +103,29 @@ bool launch_gemm_tc(const Ctx& ctx, GemmLayout layout, const bf16* A, const bf16
 // Weight-streaming GEMM for M <= GEMV_MAX_M rows, NT layout only: out(m, n) =
 // sum_k A[m, k] B[n, k] through the epilogue ep (every kind; epilogue_scalar's
 // arithmetic). gemv_supported: the row count and 16-byte rows of A and B.
+// With ln.x set, A is not read: A[m, :] = LN(ln.x[m, :]) with (ln.w, ln.b)
+// (fp32 rows of K, the arithmetic of launch_layernorm_fwd), rounded to T, is
+// computed in the kernel. Launched through launch_pdl.
 constexpr int GEMV_MAX_M = 4;
+struct LnIn {
+    const float* x = nullptr;
+    const float* w = nullptr;
+    const float* b = nullptr;
+};
 bool gemv_supported(size_t elem_size, int M, int K);
 template <typename T>
-void launch_gemv(const Ctx& ctx, const T* A, const T* B, int M, int N, int K, const Epilogue& ep);
+void launch_gemv(const Ctx& ctx, const T* A, const T* B, int M, int N, int K, const Epilogue& ep,
+                 const LnIn& ln = LnIn());
 
 // ----------------------------------------------------------------------------
 // Row-wise kernels.
 // ----------------------------------------------------------------------------
 // x[r] = wte[idx[r]] + wpe[r % T]; then y = LN(x) with (w, b); mean/rstd saved.
+// pos_dev (nullable): the wpe row of row r is *pos_dev + r % Tn.
 template <typename T>
 void launch_embed_ln(const Ctx& ctx, const int* idx, const float* wte, const float* wpe, int rows, int Tn, int C,
-                     int V, const float* w, const float* b, float* x, T* y, float* mean, float* rstd);
+                     int V, const float* w, const float* b, float* x, T* y, float* mean, float* rstd,
+                     const int* pos_dev = nullptr);
 template <typename T>
 void launch_layernorm_fwd(const Ctx& ctx, const float* x, const float* w, const float* b, T* y, float* mean,
                           float* rstd, int rows, int C);
@@ -159,15 +209,28 @@ inline long long decode_part_floats(int BH, int Tc, int hd) {
     return (long long)BH * ceil_div(Tc, DECODE_MIN_KEYS) * (hd + 2);
 }
 void attention_decode_split(int BH, int n, int num_sms, int* splits, int* chunk);
+// pos_dev (nullable): n is *pos_dev + 1, read on the device (n is then ignored; the
+// key range is split for n = Tc, and splits past the last key add nothing).
+// counters (nullable): B*H ints, zero before the call and left zero by it; with
+// them the last block of each (b, h) to finish merges the partials (one kernel),
+// else a second kernel does. Launched through launch_pdl.
 template <typename T>
 void launch_attention_decode(const Ctx& ctx, const T* cache, T* out, float* part, int B, int H, int hd, int Tc,
-                             int n);
+                             int n, const int* pos_dev = nullptr, int* counters = nullptr);
 // One draw per row of logits (row stride ld): temperature, top-k (top_k <= 0
 // or >= V keeps every entry), inverse CDF at u[row] in vocabulary order.
 // next[row] = the drawn index; if out != null also out[row * out_ld + out_col].
+// da (nullable): u, out, out_ld and out_col are taken from *da on the device (the
+// uniforms of draw da->step, column da->out_col0 + da->step).
 template <typename T>
 void launch_sample(const Ctx& ctx, const T* logits, long long ld, int rows, int V, float temperature, int top_k,
-                   const float* u, int* next, int* out, long long out_ld, int out_col);
+                   const float* u, int* next, int* out, long long out_ld, int out_col,
+                   const DecodeArgs* da = nullptr);
+// *da = {pos, step, u, out, out_ld, out_col0} (one thread), and its advance to the
+// next position and draw (pos + 1, step + 1).
+void launch_decode_set(const Ctx& ctx, DecodeArgs* da, int pos, int step, const float* u, int* out,
+                       long long out_ld, int out_col0);
+void launch_decode_advance(const Ctx& ctx, DecodeArgs* da);
 // k, v columns of qkv rows (b * Tn + t) of every layer -> cache rows (b, t).
 // qkv_ptrs, cache_ptrs: device arrays of L pointers.
 void launch_kv_store(const Ctx& ctx, const void* const* qkv_ptrs, void* const* cache_ptrs, int L, int B, int Tn,

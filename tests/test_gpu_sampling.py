@@ -18,7 +18,8 @@ fills a key/value cache with a prefill and then runs one position per draw.
     all three branches of the loop: the first prefill, decode steps, and the
     re-prefill of the cropped window once the sequence outgrows block_size.
   * bf16 generation, whose draws the bf16 logit error can flip, against the same
-    loop composed of the single calls (prefill, decode, sample): equal tokens; and
+    loop composed of the single calls (prefill, decode, sample): equal tokens,
+    also across calls that replay the graphed decode step; and
     for the pages' call at 124M, the logits of every one of its 40 draws,
     teacher-forced with the generated tokens, against the oracle's forward.
 """
@@ -276,6 +277,32 @@ def test_generate_bf16_equals_composed_calls():
     got = out.cpu().numpy()
     assert np.array_equal(got, ref)
     assert got.min() >= 0 and got.max() < s.vocab_size
+    m.close()
+
+
+def test_generate_decode_graph_across_calls():
+    """gpt2_generate's decode steps read position, draw index and output slot from
+    device arguments and run as one CUDA graph per (B, temperature, top_k): the
+    first decode step runs eagerly, the second is captured, later ones replay it,
+    and a later call with another (temperature, top_k) starts over. Every call
+    must equal the loop of single calls, and a repeated call its first run."""
+    s = TINY64
+    B, T0, n_new = 2, 3, 20
+    m = _model(s, "bf16", B, s.block_size, seed=6)
+    prompt, _ = S.uniform_tokens(B, T0, s.vocab_size, seed=752)
+    u = torch.from_numpy(S.uniforms(n_new, B, seed=753)).cuda()
+    runs = []
+    for temperature, top_k in [(0.8, 40), (1.0, 0), (0.8, 40), (0.8, 40)]:
+        out = torch.full((B, T0 + n_new), -1, dtype=torch.int32, device="cuda")
+        m.generate(_dev(prompt), n_new, temperature, top_k, u, out)
+        runs.append(out.cpu().numpy())
+    assert np.array_equal(runs[0], _composed_loop(m, s, prompt, n_new, 0.8, 40, u, torch.bfloat16))
+    assert np.array_equal(runs[1], _composed_loop(m, s, prompt, n_new, 1.0, 0, u, torch.bfloat16))
+    assert np.array_equal(runs[2], runs[0]) and np.array_equal(runs[3], runs[0])
+    # a shorter call after a longer one: the draws stop at its own length
+    out = torch.full((B, T0 + 5), -1, dtype=torch.int32, device="cuda")
+    m.generate(_dev(prompt), 5, 0.8, 40, u, out)
+    assert np.array_equal(out.cpu().numpy(), runs[0][:, :T0 + 5])
     m.close()
 
 
