@@ -154,6 +154,12 @@ struct gpt2_handle {
     float dec_temperature = 0.f;
     long long dec_graph_launches = 0;
     int* dec_counters = nullptr;     // (max_B * H) tickets of the decode attention, zero between calls
+    // bf16 decode steps of at most MEGA_MAX_B rows run as one persistent kernel
+    // (decode_mega_kernel) when the shape fits; its layer offsets and barrier
+    // words live in the generation pool
+    bool use_mega = true;
+    DecodeLayer* d_dec_layers = nullptr;
+    unsigned long long* d_mega_bar = nullptr;
     bool pdl = false;                // launch_pdl kernels get programmatic dependent launch
 
     // Data-parallel exchange: caller-owned events recorded as each gradient bucket
@@ -669,8 +675,9 @@ int ensure_gen(gpt2_handle* h) {
     const size_t next = align_up(Bm * 4), win = align_up((size_t)h->maxBT * 4);
     const size_t dargs = align_up(sizeof(DecodeArgs));
     const size_t cnt = align_up(Bm * h->H * sizeof(int));
+    const size_t dlay = align_up(L * sizeof(DecodeLayer)), mbar = align_up(sizeof(unsigned long long));
     char* pool = nullptr;
-    if (cudaMalloc((void**)&pool, L * layer + part + ptrs + next + win + dargs + cnt) != cudaSuccess) {
+    if (cudaMalloc((void**)&pool, L * layer + part + ptrs + next + win + dargs + cnt + dlay + mbar) != cudaSuccess) {
         cudaGetLastError();
         return fail(GPT2_ERR_OOM, "cudaMalloc of the key/value cache failed");
     }
@@ -688,6 +695,16 @@ int ensure_gen(gpt2_handle* h) {
     DecodeArgs* d_dec = (DecodeArgs*)(pool + off);
     off += dargs;
     int* dec_counters = (int*)(pool + off);
+    off += cnt;
+    DecodeLayer* dec_layers = (DecodeLayer*)(pool + off);
+    off += dlay;
+    unsigned long long* mega_bar = (unsigned long long*)(pool + off);
+    std::vector<DecodeLayer> dl(L);
+    for (size_t l = 0; l < L; ++l) {
+        const LayerOff& o = h->lo[l];
+        dl[l] = DecodeLayer{o.ln1w, o.ln1b, o.wqkv, o.bqkv, o.wproj, o.bproj, o.ln2w, o.ln2b, o.wfc, o.bfc,
+                            o.wfcp, o.bfcp};
+    }
     std::vector<void*> tab(2 * L);
     for (size_t l = 0; l < L; ++l) {
         tab[l] = h->qkv[l];
@@ -697,6 +714,9 @@ int ensure_gen(gpt2_handle* h) {
     cudaError_t e = cudaMemcpyAsync(layer_ptrs, tab.data(), tab.size() * sizeof(void*), cudaMemcpyHostToDevice,
                                     h->stream);
     if (e == cudaSuccess) e = cudaMemsetAsync(dec_counters, 0, cnt, h->stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(mega_bar, 0, mbar, h->stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(dec_layers, dl.data(), L * sizeof(DecodeLayer), cudaMemcpyHostToDevice, h->stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(h->stream);
     if (e != cudaSuccess) {
         cudaFree(pool);
@@ -710,6 +730,8 @@ int ensure_gen(gpt2_handle* h) {
     h->d_window = d_window;
     h->d_dec = d_dec;
     h->dec_counters = dec_counters;
+    h->d_dec_layers = dec_layers;
+    h->d_mega_bar = mega_bar;
     h->kv_B = h->kv_len = 0;
     return GPT2_OK;
 }
@@ -742,8 +764,46 @@ void gemv_ln(gpt2_handle* h, const char* site, long long w_off, int M, int N, in
 // With at most GEMV_MAX_M rows every GEMM runs on the weight-streaming kernel
 // and the LayerNorms before c_attn (after the first), c_fc and lm_head run
 // inside it; the kernels are chained by programmatic dependent launch.
+// The persistent one-kernel decode step; false if the shape or mode does not fit.
+template <typename A>
+bool decode_mega(gpt2_handle* h, const int* tok, int B, int pos, A* logits_out, const int* pos_dev) {
+    if (sizeof(A) != 2 || !h->use_mega || !h->bf16_mode) return false;
+    MegaDecode p = {};
+    p.L = h->L;
+    p.C = h->C;
+    p.H = h->H;
+    p.V = h->V;
+    p.Tc = h->cfg.block_size;
+    p.B = B;
+    p.pos_now = pos;
+    p.pos_dev = pos_dev;
+    if (!decode_mega_plan(p, h->num_sms)) return false;
+    p.P = h->params;
+    p.W = h->shadow;
+    p.layers = h->d_dec_layers;
+    p.off_wte = h->off_wte;
+    p.off_wpe = h->off_wpe;
+    p.off_lnfw = h->off_lnfw;
+    p.off_lnfb = h->off_lnfb;
+    p.kv = h->d_layer_ptrs + h->L;
+    p.resid = h->resid[0];
+    p.att = (bf16*)h->att[0];
+    p.fcg = (bf16*)h->fcg[0];
+    p.logits = (bf16*)logits_out;
+    p.tok = tok;
+    p.bar = h->d_mega_bar;
+    Ctx c = h->ctx();
+    p.status = c.status;
+    const double C = h->C, weights = 2.0 * (h->L * 12.0 * C * C + (double)h->V * C);
+    PROF("decode step (one persistent kernel)", 0, 0, 0, 2.0 * B * weights / 2.0,
+         weights + 2.0 * h->L * B * (pos + 1.0) * 2 * C,
+         if (!launch_decode_mega(c, p)) h->host_error = "the persistent decode kernel could not be launched");
+    return true;
+}
+
 template <typename A>
 void decode_impl(gpt2_handle* h, const int* tok, int B, int pos, A* logits_out, const int* pos_dev = nullptr) {
+    if (decode_mega<A>(h, tok, B, pos, logits_out, pos_dev)) return;
     PdlScope pdl(h);
     Ctx c = h->ctx();
     const int C = h->C, V = h->V, L = h->L, H = h->H, hd = h->hd, Tc = h->cfg.block_size;
@@ -846,7 +906,11 @@ int status_error(gpt2_handle* h) {
     if (!s) return GPT2_OK;
     h->h_sc->status = 0;
     CK(cudaMemsetAsync(&h->d_sc->status, 0, sizeof(unsigned), h->stream));
-    if (s & STATUS_TIMEOUT) return fail(GPT2_ERR_TIMEOUT, "a bounded wait inside a kernel gave up");
+    if (s & STATUS_TIMEOUT) {
+        // a grid barrier left mid-way would hold a stale count
+        if (h->d_mega_bar) CK(cudaMemsetAsync(h->d_mega_bar, 0, sizeof(unsigned long long), h->stream));
+        return fail(GPT2_ERR_TIMEOUT, "a bounded wait inside a kernel gave up");
+    }
     if (s & STATUS_BAD_TOKEN) return fail(GPT2_ERR_BAD_TOKEN, "token id or target out of range");
     return GPT2_OK;
 }
@@ -1089,6 +1153,7 @@ int gpt2_create(const gpt2_config* cfg, void* stream, gpt2_handle** out) {
     h->maxBT = cfg->max_B * cfg->max_T;
     if (const char* e = getenv("GPT2_B200_SIMT_GEMM")) h->use_tc_gemm = (e[0] == '0');
     if (const char* e = getenv("GPT2_B200_NO_GRAPH")) h->use_graphs = (e[0] == '0');
+    if (const char* e = getenv("GPT2_B200_NO_MEGA")) h->use_mega = (e[0] == '0');
     if (const char* e = getenv("GPT2_B200_SIMT_ATTENTION")) h->use_tc_attention = (e[0] == '0');
     if (const char* e = getenv("GPT2_B200_TCGEN05_ATTENTION")) h->use_tcgen05_attention = (e[0] == '1');
     if (const char* e = getenv("GPT2_B200_TCGEN05_ATTENTION_BWD")) h->use_tcgen05_attention_bwd = (e[0] == '1');

@@ -81,6 +81,47 @@ struct DecodeArgs {
     int out_col0;        // column of draw 0
 };
 
+// One decode step as one persistent kernel (bf16, head width 64, B <=
+// MEGA_MAX_B rows): embedding, every block and the tied lm_head, for the
+// position pos (or *pos_dev) of tokens tok (B), the cache rows written and read
+// in place. Offsets are element offsets into P (fp32 parameters: LayerNorm
+// weights, biases, wte and wpe for the embedding) and W (the bf16 weights).
+constexpr int MEGA_MAX_B = 4;
+constexpr int MEGA_MAX_L = 48;
+constexpr int MEGA_SLOTS = 5;
+constexpr int MEGA_SLOT_BYTES = 36 * 1024;
+constexpr int MEGA_X_BYTES = 24 * 1024;   // the operand rows (B x 4C bf16 at most)
+struct DecodeLayer {
+    long long ln1w, ln1b, wqkv, bqkv, wproj, bproj, ln2w, ln2b, wfc, bfc, wfcp, bfcp;
+};
+struct MegaDecode {
+    int L, C, H, V, Tc, B;
+    int pos_now;                 // the position (replaced by *pos_dev if set)
+    const int* pos_dev;
+    const float* P;
+    const bf16* W;
+    const DecodeLayer* layers;   // device, L entries
+    long long off_wte, off_wpe, off_lnfw, off_lnfb;
+    void* const* kv;             // device, L cache pointers ((B, Tc, 3C) rows)
+    float* resid;                // (B, C) fp32 residual stream
+    bf16* att;                   // (B, C)
+    bf16* fcg;                   // (B, 4C)
+    bf16* logits;                // (B, V)
+    const int* tok;              // (B)
+    unsigned long long* bar;     // grid barrier count: zero before the first launch; each launch adds
+                                 // 5 L x grid, so it stays a multiple of that between launches
+    unsigned* status;
+    // decode_mega_plan: per CTA rows of c_attn, attn.c_proj, c_fc, mlp.c_proj; the
+    // lm_head rows per CTA, rows per ring chunk and chunks; the grid
+    int rows[4];
+    int rows_lm, chunk_lm, n_lm, grid;
+};
+// Fills the plan for num_sms CTAs; false if the shape does not fit (then the
+// step runs as separate kernels).
+bool decode_mega_plan(MegaDecode& p, int num_sms);
+// false if the launch was refused (e.g. not all CTAs can be resident).
+bool launch_decode_mega(const Ctx& ctx, const MegaDecode& p);
+
 // Operand layouts of C[M,N] = sum_k A(m,k) B(n,k):
 //   GEMM_NT: A row-major [M,K], B row-major [N,K]   (forward: y = x W^T)
 //   GEMM_NN: A row-major [M,K], B row-major [K,N]   (dgrad:  dx = dy W)

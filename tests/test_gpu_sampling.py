@@ -306,6 +306,45 @@ def test_generate_decode_graph_across_calls():
     m.close()
 
 
+def _profile_sites(m, fn):
+    m.profile(True)
+    fn()
+    sites = {st["name"] for st in m.profile_read()}
+    m.profile(False)
+    return sites
+
+
+@pytest.mark.parametrize("B", [1, 3])
+def test_decode_persistent_kernel_matches_kernel_chain(B, monkeypatch):
+    """A bf16 decode step of at most four rows runs as one persistent kernel (grid
+    barriers between the phases of a layer, weights streamed into shared memory);
+    GPT2_B200_NO_MEGA=1 at creation keeps the chain of separate kernels. Same
+    weights and cache contents: the logits of five teacher-forced decode steps
+    agree to bf16 rounding (1e-2 of max |logit|, cosine > 0.9999), and the profile
+    names the kernel that ran."""
+    s = TINY64
+    seq, _ = S.uniform_tokens(B, 12, s.vocab_size, seed=770 + B)
+    out = {}
+    for mode in ("mega", "chain"):
+        if mode == "chain":
+            monkeypatch.setenv("GPT2_B200_NO_MEGA", "1")
+        m = _model(s, "bf16", B, s.block_size, seed=7)
+        lg = torch.empty((B, s.vocab_size), dtype=torch.bfloat16, device="cuda")
+        m.prefill(_dev(seq[:, :6]), lg)
+        got = []
+        for i in range(5):
+            m.decode(_dev(seq[:, 6 + i]), 6 + i, lg)
+            got.append(lg.float().cpu().numpy())
+        sites = _profile_sites(m, lambda: m.decode(_dev(seq[:, 11]), 11, lg))
+        out[mode] = (np.stack(got), sites)
+        m.close()
+        monkeypatch.delenv("GPT2_B200_NO_MEGA", raising=False)
+    assert any("persistent" in x for x in out["mega"][1]), out["mega"][1]
+    assert not any("persistent" in x for x in out["chain"][1]), out["chain"][1]
+    a, b = out["mega"][0], out["chain"][0]
+    assert _rel(a, b) < 1e-2 and _cos(a, b) > 0.9999
+
+
 # ----------------------------------------------------------------------------
 # GPT-2 124M, bf16: the generation workload of the benchmark (B = 1, a short
 # prompt, 40 new tokens, temperature 0.8, top-k 40).
