@@ -116,6 +116,9 @@ const char* gpt2_last_error(void);
  *   GPT2_B200_TCGEN05_ATTENTION=0     mma.sync attention forward instead of tcgen05
  *   GPT2_B200_TCGEN05_ATTENTION_BWD=0 mma.sync attention backward instead of tcgen05
  *   GPT2_B200_NO_GRAPH=1              no CUDA-graph replay of the step (see gpt2_step)
+ *                                     nor of gpt2_generate's decode steps
+ *   GPT2_B200_NO_MEGA=1               decode steps as a chain of kernels instead of
+ *                                     the one persistent kernel (see gpt2_decode)
  * fp32 mode always uses the SIMT kernels.
  * Errors: INVALID_ARG (sizes), UNSUPPORTED_ARCH, OOM, CUDA. */
 int gpt2_create(const gpt2_config* cfg, void* stream, gpt2_handle** out);
@@ -235,9 +238,16 @@ int gpt2_prefill(gpt2_handle* h, const int32_t* idx_dev, int B, int T, void* log
  * 0 .. pos, and writes the logits (B, vocab_size) (fp32 or bf16 by mode) to
  * logits_dev. Afterwards the cache holds pos + 1 positions of sequences
  * 0 .. B-1 only: later decodes may use at most B rows.
+ * In bf16 mode with B <= 4 and head width 64, when each SM's slice of every
+ * weight matrix fits its 36 KB shared-memory slots (GPT-2 124M; wider models
+ * fall back), the step is one persistent kernel (one CTA per SM, grid
+ * barriers between the phases of a layer, the bias + rounding + residual
+ * arithmetic of the other engines); otherwise a chain of kernels. The two
+ * agree to bf16 rounding.
  * Synchronises once at the end. Errors: INVALID_ARG (no prefill yet, B above
  * the rows of the last prefill or decode, pos < 1, pos above the cached
- * length, or pos >= block_size); BAD_TOKEN for an id outside [0, vocab_size). */
+ * length, or pos >= block_size); BAD_TOKEN for an id outside [0, vocab_size);
+ * TIMEOUT if a grid barrier of the persistent kernel gave up (bounded wait). */
 int gpt2_decode(gpt2_handle* h, const int32_t* tokens_dev, int B, int pos, void* logits_dev);
 
 /* One draw per row of logits_dev (B, vocab_size) (fp32 or bf16 by mode, rows
@@ -261,7 +271,9 @@ int gpt2_sample(gpt2_handle* h, const void* logits_dev, int B, float temperature
  * draw runs gpt2_prefill on the last block_size tokens (the pages' crop, which
  * shifts every position, so the cache cannot be reused). Each draw is
  * gpt2_sample with u = u_dev[s * B + b] (u_dev: (max_new_tokens, B) floats in
- * [0, 1)). Synchronises once at the end.
+ * [0, 1)). Synchronises once at the end. The decode steps read their position
+ * and output slot from device memory and run as one CUDA graph per step
+ * (captured once per B, temperature and top_k) unless graphs are off.
  * Errors: INVALID_ARG (NULL pointer, B outside [1, max_B], T0 < 1,
  * max_new_tokens < 0, a bad temperature, or a prefill window longer than
  * max_T: min(T0, block_size), or block_size when the sequence outgrows it);
