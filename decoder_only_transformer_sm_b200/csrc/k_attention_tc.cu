@@ -75,6 +75,10 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 __device__ __forceinline__ void ew_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// The two softmax warps of one TMEM lane quarter (named barriers 2..5).
+__device__ __forceinline__ void pair_bar(int quarter) {
+    asm volatile("bar.sync %0, 64;" ::"r"(2 + quarter) : "memory");
+}
 
 // max(a, b, c) in one instruction (sm_100 three-input max.f32)
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -307,24 +311,22 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t s_addr = tmem + (sb ? TM_S1 : TM_S0) + chalf * 64 + lane_off;
                 const int kbase = j * BKV + chalf * 64;   // first key of this warp's columns
                 const bool diag = (j * BKV + BKV > q0);
-                // pass 1: partial row max over this warp's 64 keys, exchanged with the pair
+                // pass 1: partial row max over this warp's 64 keys (one TMEM load), exchanged
+                // with the pair
                 float mx = -INFINITY;
                 if (w) {
                     tc::fence_after_sync();
+                    float sv[64];
+                    tc::tmem_ld_32x32b_x64(s_addr, sv);
+                    if (diag) {   // keys after the query do not count
 #pragma unroll
-                    for (int c = 0; c < 64; c += 32) {
-                        float sv[32];
-                        tc::tmem_ld_32x32b_x32(s_addr + c, sv);
-                        if (diag) {   // keys after the query do not count
-#pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                if (kbase + c + e > q) sv[e] = -INFINITY;
-                        }
-                        mx = max32(sv, mx);
+                        for (int e = 0; e < 64; ++e)
+                            if (kbase + e > q) sv[e] = -INFINITY;
                     }
+                    mx = max32(sv + 32, max32(sv, mx));
                 }
                 ctl->mx[sb][chalf][r] = mx;
-                ew_bar();
+                pair_bar(quarter);
                 if (!w) { ok = false; continue; }
                 mx = fmaxf(mx, ctl->mx[sb][chalf ^ 1][r]);
                 const float m_new = fmaxf(m, mx * sl2);
@@ -334,12 +336,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 // the exponent s * sl2 - m_new and the row sum on packed pairs
                 const f32x2 SL = pk2(sl2, sl2), NM = pk2(-m_new, -m_new);
                 f32x2 RS = pk2(0.f, 0.f);
+                {
+                    float sv[64];
+                    tc::tmem_ld_32x32b_x64(s_addr, sv);   // the 64 columns, one TMEM round trip
 #pragma unroll
-                for (int c = 0; c < 64; c += 32) {
-                    float sv[32];
-                    tc::tmem_ld_32x32b_x32(s_addr + c, sv);
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
+                    for (int e = 0; e < 64; e += 2) {
                         float t0, t1;
                         upk2(fma2(pk2(sv[e], sv[e + 1]), SL, NM), t0, t1);
                         sv[e] = ex2(t0);
@@ -347,14 +348,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                     if (diag) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (kbase + c + e > q) sv[e] = 0.f;
+                        for (int e = 0; e < 64; ++e)
+                            if (kbase + e > q) sv[e] = 0.f;
                     }
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) RS = add2(RS, pk2(sv[e], sv[e + 1]));
+                    for (int e = 0; e < 64; e += 2) RS = add2(RS, pk2(sv[e], sv[e + 1]));
 #pragma unroll
-                    for (int gg = 0; gg < 4; ++gg)
-                        *reinterpret_cast<uint4*>(pt + swz128(r, (c >> 3) + gg)) = pack8_bf16(sv + 8 * gg);
+                    for (int gg = 0; gg < 8; ++gg)
+                        *reinterpret_cast<uint4*>(pt + swz128(r, gg)) = pack8_bf16(sv + 8 * gg);
                 }
                 float rs0, rs1;
                 upk2(RS, rs0, rs1);
