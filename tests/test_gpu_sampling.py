@@ -98,6 +98,29 @@ def test_sample_kernel_matches_oracle(dtype, V, temperature, top_k):
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("temperature,top_k", [(1.0, 0), (0.8, 40)])
+def test_sample_kernel_long_rows_single_block(dtype, temperature, top_k):
+    """Rows of 500,000 values: the slices of an 8-CTA cluster no longer fit its
+    shared memory, so the draw runs on one block per row reading the row from
+    memory at every pass. Same oracle check as above."""
+    from decoder_only_transformer_sm_b200 import native
+    rows, V = 3, 500_000
+    rng = np.random.default_rng(720 + top_k)
+    x = rng.normal(0.0, 2.0, (rows, V)).astype(np.float32)
+    tdt = torch.float32 if dtype == "fp32" else torch.bfloat16
+    xd = torch.from_numpy(x).to(tdt).cuda()
+    x64 = xd.float().cpu().numpy().astype(np.float64)
+    u = S.uniforms(1, rows, seed=721)[0]
+    nxt = torch.full((rows,), -1, dtype=torch.int32, device="cuda")
+    st = native.sample(xd, V, temperature, top_k, torch.from_numpy(u).cuda(), nxt)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    got = nxt.cpu().numpy()
+    for r in range(rows):
+        _check_draw(int(got[r]), x64[r], temperature, top_k, float(u[r]))
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
 def test_sample_kernel_ties_row_stride_and_edges(dtype):
     """Integer-valued logits (many ties at the k-th value), a row stride above V,
     an all-equal row, and the u edge cases 0 and just below 1."""
