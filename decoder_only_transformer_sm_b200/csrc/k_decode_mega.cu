@@ -42,9 +42,9 @@
 // is a multiple of 5 L x grid; a CTA reads it at start (no CTA can pass the
 // first barrier before every CTA has arrived, so the value read lies below
 // the next multiple) and barrier i of the launch waits for base + (i+1) x grid.
-// Arrival is a fence and an add; the wait polls the count (bounded by wall
-// time; on timeout the kernel sets STATUS_TIMEOUT and skips the remaining
-// waits, and the host clears the count). Data written before a barrier by
+// Arrival is a release add after the block barrier; the wait polls the count
+// with acquire loads (bounded by wall time; on timeout the kernel sets
+// STATUS_TIMEOUT and skips the remaining waits, and the host clears the count). Data written before a barrier by
 // other CTAs is read after it through L2 (ld.global.cg). The launch is
 // cooperative, so all CTAs are resident together.
 //
@@ -157,8 +157,9 @@ __device__ void grid_sync(const MegaDecode& p, const MegaSmem& s) {
     if (threadIdx.x == 0 && !*s.abort) {
         const unsigned long long target = *s.target + gridDim.x;
         *s.target = target;
-        __threadfence();
-        asm volatile("red.relaxed.gpu.global.add.u64 [%0], 1;" ::"l"(p.bar) : "memory");
+        // release: this CTA's writes (ordered before thread 0 by the block barrier)
+        // become visible before the arrival; the acquiring poll orders the reads after
+        asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(p.bar) : "memory");
         if (ld_acquire_u64(p.bar) < target) {
             unsigned long long t0 = 0;
             for (uint32_t it = 0; ld_acquire_u64(p.bar) < target; ++it) {
@@ -174,7 +175,6 @@ __device__ void grid_sync(const MegaDecode& p, const MegaSmem& s) {
                 }
             }
         }
-        __threadfence();
     }
     __syncthreads();
 }
