@@ -21,8 +21,8 @@
 //      c_attn rows of this CTA: q, k, v of position pos into
 //      the cache row (bias added, rounded to bf16).            -> grid barrier
 //   B  attention of (b, h) = CTA index (B*H CTAs): q against cache rows
-//      0 .. pos, online softmax over 64 key groups of 8 lanes, merged in
-//      shared memory -> att (bf16).                             -> grid barrier
+//      0 .. pos, online softmax over 64 key groups of 8 lanes, merged by
+//      shuffles in each warp, then over the 16 warps -> att (bf16). -> grid barrier
 //   C  att into shared memory; attn.c_proj rows: resid += att W^T + b.
 //                                                               -> grid barrier
 //   D  x = LN_2(resid); c_fc rows: fcg = gelu(bf16(x W^T + b)) (bf16).
@@ -424,19 +424,35 @@ __device__ __forceinline__ void attention(const MegaDecode& p, const MegaSmem& s
             m = mx;
         }
     }
-    if (sub == 0) {
-        sm_m[grp] = m;
-        sm_l[grp] = lsum;
-    }
+    // merge the warp's four groups (lanes l, l + 8, l + 16, l + 24 hold the same dims)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) sm_acc[grp * MG_HD + sub * 8 + i] = acc[i];
+    for (int o = MG_G; o < 32; o <<= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o), l2 = __shfl_xor_sync(0xffffffffu, lsum, o);
+        const float M = fmaxf(m, m2);
+        const float w1 = M == -INFINITY ? 0.f : exp2f(m - M), w2 = M == -INFINITY ? 0.f : exp2f(m2 - M);
+        lsum = fmaf(lsum, w1, l2 * w2);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float a2 = __shfl_xor_sync(0xffffffffu, acc[i], o);
+            acc[i] = fmaf(acc[i], w1, a2 * w2);
+        }
+        m = M;
+    }
+    if (lane < MG_G) {   // the warp's partial: (m, l, acc[64]) of its keys
+        if (sub == 0) {
+            sm_m[warp] = m;
+            sm_l[warp] = lsum;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sm_acc[warp * MG_HD + sub * 8 + i] = acc[i];
+    }
     __syncthreads();
-    if (threadIdx.x < MG_HD) {
+    if (threadIdx.x < MG_HD) {   // the 16 warp partials, in warp order
         const int d = threadIdx.x;
         float M = -INFINITY;
-        for (int g = 0; g < MG_NG; ++g) M = fmaxf(M, sm_m[g]);   // finite: group 0 holds key 0
+        for (int g = 0; g < MG_WARPS; ++g) M = fmaxf(M, sm_m[g]);   // finite: warp 0 holds key 0
         float L = 0.f, A = 0.f;
-        for (int g = 0; g < MG_NG; ++g) {
+        for (int g = 0; g < MG_WARPS; ++g) {
             const float wgt = exp2f(sm_m[g] - M);
             L = fmaf(sm_l[g], wgt, L);
             A = fmaf(sm_acc[g * MG_HD + d], wgt, A);
