@@ -72,6 +72,7 @@ constexpr int MEGA_LN_NV = 8;           // float4 per lane of a LayerNorm row: C
 struct MegaSmem {
     unsigned char* ring;   // MEGA_SLOTS x MEGA_SLOT_BYTES
     bf16* xs;              // B x K operand rows (or the attention merge scratch)
+    float* lnw;            // the next LayerNorm's weight (C floats) then bias (C floats)
     uint64_t* full;        // MEGA_SLOTS mbarriers
     int* issued;           // MEGA_SLOTS: the last job issued into each slot (-1: none)
     volatile uint32_t* abort;
@@ -183,9 +184,12 @@ __device__ void grid_sync(const MegaDecode& p, const MegaSmem& s) {
 // warp per row (launch_layernorm_fwd's arithmetic and order), the row read
 // once into registers.
 template <int MB>
-__device__ __forceinline__ void stage_ln(const MegaDecode& p, const MegaSmem& s, const float* src, const float* w,
-                                         const float* b) {
+__device__ __forceinline__ void stage_ln(const MegaDecode& p, const MegaSmem& s, const float* src) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, C = p.C;
+    asm volatile("cp.async.wait_all;" ::: "memory");   // this thread's part of the staged weights
+    __syncthreads();                                     // everyone's
+    const float* w = s.lnw;
+    const float* b = s.lnw + C;
     if (warp < MB) {
         const float* x = src + (long long)warp * C;
         bf16* y = s.xs + (long long)warp * C;
@@ -271,14 +275,18 @@ __device__ __forceinline__ void preload(const MegaDecode& p, const MegaSmem& s, 
     }
 }
 
-__device__ __forceinline__ void prefetch_l2(const float* a) { asm volatile("prefetch.global.L2 [%0];" ::"l"(a)); }
-
-// The weights of a LayerNorm, into L2 a phase before it runs.
-__device__ __forceinline__ void prefetch_ln(const MegaDecode& p, const float* w, const float* b) {
-    for (int i = threadIdx.x; i < p.C / 32; i += MG_THREADS) {
-        prefetch_l2(w + i * 32);
-        prefetch_l2(b + i * 32);
+// The weight and bias of the next LayerNorm into s.lnw a phase before it runs
+// (cp.async, 16 bytes a thread; stage_ln waits for them). Its previous reader,
+// the LayerNorm before, has finished: each LayerNorm ends with a block barrier.
+__device__ __forceinline__ void stage_ln_weights(const MegaDecode& p, const MegaSmem& s, const float* w,
+                                                 const float* b) {
+    const int n16 = p.C / 4;
+    for (int i = threadIdx.x; i < 2 * n16; i += MG_THREADS) {
+        const float* src = i < n16 ? w + 4 * i : b + 4 * (i - n16);
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(s.lnw + 4 * i)), "l"(src)
+                     : "memory");
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
 // Rows of job j from its ring slot against the MB operand rows in xs, then the
@@ -481,6 +489,7 @@ __global__ void __launch_bounds__(MG_THREADS, 1) decode_mega_kernel(const __grid
     s.ring = mg_smem;
     s.xs = reinterpret_cast<bf16*>(mg_smem + (size_t)MEGA_SLOTS * MEGA_SLOT_BYTES);
     s.full = reinterpret_cast<uint64_t*>(mg_smem + (size_t)MEGA_SLOTS * MEGA_SLOT_BYTES + MEGA_X_BYTES);
+    s.lnw = reinterpret_cast<float*>(mg_smem + (size_t)MEGA_SLOTS * MEGA_SLOT_BYTES + MEGA_X_BYTES + 64);
     s.issued = s_issued;
     s.abort = &s_abort;
     s.layers = s_layers;
@@ -569,11 +578,11 @@ __global__ void __launch_bounds__(MG_THREADS, 1) decode_mega_kernel(const __grid
         int job = -1;
         switch (op) {
         case OP_LN1:
-            if (l > 0) stage_ln<MB>(p, s, p.resid, p.P + o.ln1w, p.P + o.ln1b);
+            if (l > 0) stage_ln<MB>(p, s, p.resid);
             break;
         case OP_QKV:
             job = 4 * l + J_QKV;
-            prefetch_ln(p, p.P + o.ln2w, p.P + o.ln2b);
+            stage_ln_weights(p, s, p.P + o.ln2w, p.P + o.ln2b);
             break;
         case OP_ATTN:
             attention(p, s, l);
@@ -585,12 +594,12 @@ __global__ void __launch_bounds__(MG_THREADS, 1) decode_mega_kernel(const __grid
             job = 4 * l + J_PROJ;
             break;
         case OP_LN2:
-            stage_ln<MB>(p, s, p.resid, p.P + o.ln2w, p.P + o.ln2b);
+            stage_ln<MB>(p, s, p.resid);
             break;
         case OP_FC:
             job = 4 * l + J_FC;
-            if (l + 1 < p.L) prefetch_ln(p, p.P + s_layers[l + 1].ln1w, p.P + s_layers[l + 1].ln1b);
-            else prefetch_ln(p, p.P + p.off_lnfw, p.P + p.off_lnfb);
+            if (l + 1 < p.L) stage_ln_weights(p, s, p.P + s_layers[l + 1].ln1w, p.P + s_layers[l + 1].ln1b);
+            else stage_ln_weights(p, s, p.P + p.off_lnfw, p.P + p.off_lnfb);
             break;
         case OP_STAGE_FCG:
             stage_rows<MB>(s, p.fcg, 4 * C);
@@ -599,7 +608,7 @@ __global__ void __launch_bounds__(MG_THREADS, 1) decode_mega_kernel(const __grid
             job = 4 * l + J_FCP;
             break;
         case -1:
-            stage_ln<MB>(p, s, p.resid, p.P + p.off_lnfw, p.P + p.off_lnfb);
+            stage_ln<MB>(p, s, p.resid);
             break;
         case -2:
             job = 4 * p.L + (t - n_layer_ops - 1);
@@ -627,7 +636,8 @@ __global__ void __launch_bounds__(MG_THREADS, 1) decode_mega_kernel(const __grid
 
 }  // namespace
 
-size_t decode_mega_smem() { return (size_t)MEGA_SLOTS * MEGA_SLOT_BYTES + MEGA_X_BYTES + MEGA_SLOTS * 8; }
+// ring | operand rows | mbarriers (64 bytes) | LayerNorm weight and bias (C <= 1024)
+size_t decode_mega_smem() { return (size_t)MEGA_SLOTS * MEGA_SLOT_BYTES + MEGA_X_BYTES + 64 + 2 * 1024 * 4; }
 
 template <int MB>
 static bool mega_fits_one() {
