@@ -595,17 +595,22 @@ __global__ void __launch_bounds__(SMP_THREADS)
     s_excl[tid] = woff + (lane == 0 ? 0.f : prev);
     if (tid == SMP_THREADS - 1) s_excl[SMP_THREADS] = s_wred[31];
     cluster.sync();   // slice sums and last kept indices visible to the cluster
-    if (tid == 0) {
+    if (warp == 0) {   // lane r < SMP_CS reads slice r's; the sums are added in rank order
+        const float t = lane < SMP_CS ? *cluster.map_shared_rank(&s_total, lane) : 0.f;
+        int glk = lane < SMP_CS ? *cluster.map_shared_rank(&s_last, lane) : -1;
         float tot = 0.f, off = 0.f;
-        int glk = -1;
+#pragma unroll
         for (int r = 0; r < SMP_CS; ++r) {
             if (r == rank) off = tot;
-            tot += *cluster.map_shared_rank(&s_total, r);
-            glk = max(glk, *cluster.map_shared_rank(&s_last, r));
+            tot += __shfl_sync(0xffffffffu, t, r);
         }
-        s_off = off;
-        s_gtot = tot;
-        s_glast = glk;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) glk = max(glk, __shfl_xor_sync(0xffffffffu, glk, o));
+        if (lane == 0) {
+            s_off = off;
+            s_gtot = tot;
+            s_glast = glk;
+        }
     }
     __syncthreads();
 
@@ -631,12 +636,15 @@ __global__ void __launch_bounds__(SMP_THREADS)
         atomicMin(&s_pick, pick);
     }
     cluster.sync();   // every slice's pick
-    if (rank == 0 && tid == 0) {
-        int j = INT_MAX;
-        for (int r = 0; r < SMP_CS; ++r) j = min(j, *cluster.map_shared_rank(&s_pick, r));
-        if (j == INT_MAX) j = s_glast;
-        next[row] = j;
-        if (out) out[(long long)row * out_ld + out_col] = j;
+    if (rank == 0 && warp == 0) {
+        int j = lane < SMP_CS ? *cluster.map_shared_rank(&s_pick, lane) : INT_MAX;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) j = min(j, __shfl_xor_sync(0xffffffffu, j, o));
+        if (lane == 0) {
+            if (j == INT_MAX) j = s_glast;
+            next[row] = j;
+            if (out) out[(long long)row * out_ld + out_col] = j;
+        }
     }
     cluster.sync();   // rank 0's reads of the other slices are done before they exit
 }
