@@ -658,8 +658,12 @@ void backward_impl(gpt2_handle* h, const int* idx, int B, int T) {
                                      l > 0 ? G + h->lo[l - 1].bfcp : nullptr, BT, C, h->red_scratch));
         bucket_done(h, L - l);   // block l (its mlp.c_proj bias gradient was added by block l+1 or ln_f)
     }
-    PROF("embedding bwd", 0, 0, 0, 0.0, (double)BT * C * 12 + (double)T * C * 8,
-         launch_embed_bwd(c, idx, h->dres, B, T, C, V, G + h->off_wte, G + h->off_wpe));
+    // deterministic: the GELU-backward buffer (free by now; BT x 4C elements of at least
+    // 2 bytes, so at least BT x 8C bytes) holds the per-run partial sums and the sort.
+    // Bytes: dx read once, ids, dwpe read and written (the used rows of dwte, a
+    // data-dependent count, are left out)
+    PROF("embedding bwd", 0, 0, 0, 0.0, (double)BT * C * 4 + (double)BT * 4 + (double)T * C * 8,
+         launch_embed_bwd(c, idx, h->dres, B, T, C, V, G + h->off_wte, G + h->off_wpe, (float*)h->du));
     bucket_done(h, L + 1);   // wte, wpe
 }
 

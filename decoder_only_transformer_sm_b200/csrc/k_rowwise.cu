@@ -9,6 +9,8 @@
 // loss when targets are given" (F.cross_entropy with ignore_index=-1);
 // "Weight tying" (the embedding gradient lands in the same wte gradient as the
 // lm_head weight gradient).
+#include <algorithm>
+
 #include "kernels.cuh"
 
 namespace gpt2 {
@@ -625,6 +627,238 @@ __global__ void embed_bwd_wte_kernel(const int* __restrict__ idx, const float* _
     for (int j = 0; j < 4; ++j) atomicAdd(d + j, v[j]);
 }
 
+// Deterministic embedding backward, per tile of at most EMB_TILE rows (tiles in
+// row order). (1) Each block sorts one chunk of EMB_CHUNK packed keys
+// (token << 16 | row in the tile) in shared memory (bitonic; the row breaks ties,
+// so within a token the rows keep their order). (2) A warp per window of EMB_WIN
+// sorted entries sums its rows, one piece per run of one token, in row order,
+// into part[first position of the piece]; chunk ends are window ends. (3) A warp
+// per run (a token's entries in one chunk) adds the run's pieces in position
+// order into the run's first slot; then a warp per token adds its runs' sums in
+// chunk order into dwte[token]. Chunks hold ascending rows, so each token's rows
+// are added in row order, grouped; no atomics, every sum has a fixed order.
+constexpr int EMB_TILE = 16384;
+constexpr int EMB_CHUNK = 2048;
+constexpr int EMB_WIN = 16;
+static_assert(EMB_TILE <= 65536 && EMB_CHUNK % EMB_WIN == 0 && EMB_TILE / EMB_CHUNK <= 32, "emb tiling");
+
+__global__ void __launch_bounds__(EMB_CHUNK / 2) emb_sort_kernel(const int* __restrict__ idx, int rows, int V,
+                                                                 unsigned* __restrict__ sorted) {
+    __shared__ unsigned ekey[EMB_CHUNK];
+    const int base = blockIdx.x * EMB_CHUNK;
+    for (int i = threadIdx.x; i < EMB_CHUNK; i += blockDim.x) {
+        unsigned k = 0xFFFFFFFFu;   // padding sorts last
+        if (base + i < rows) {
+            int tok = idx[base + i];
+            tok = tok < 0 ? 0 : (tok >= V ? V - 1 : tok);
+            k = ((unsigned)tok << 16) | (unsigned)(base + i);
+        }
+        ekey[i] = k;
+    }
+    __syncthreads();
+    const int t = threadIdx.x;   // one compare-exchange pair per thread and stage
+    for (int k = 2; k <= EMB_CHUNK; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const int i = 2 * t - (t & (j - 1));   // bit j of i is clear; the partner is i + j
+            const unsigned a = ekey[i], b = ekey[i + j];
+            if ((a > b) == ((i & k) == 0)) {
+                ekey[i] = b;
+                ekey[i + j] = a;
+            }
+            __syncthreads();
+        }
+    }
+    for (int i = threadIdx.x; i < EMB_CHUNK && base + i < rows; i += blockDim.x) sorted[base + i] = ekey[i];
+}
+
+// Rows loaded together per batch (independent loads in flight), so that the
+// buffer stays within the register file for the wider models.
+template <int NV>
+constexpr int emb_batch() { return NV <= 6 ? 4 : (NV <= 12 ? 2 : 1); }
+
+template <int NV>
+__global__ void __launch_bounds__(256) emb_piece_kernel(const unsigned* __restrict__ sorted, int n,
+                                                        const float* __restrict__ dx, int C, float* __restrict__ part) {
+    constexpr int U = emb_batch<NV>();
+    const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const int e0 = w * EMB_WIN;
+    if (e0 >= n) return;
+    const int cnt = min(EMB_WIN, n - e0);
+    const unsigned mykey = lane < cnt ? sorted[e0 + lane] : 0xFFFFFFFFu;
+    float acc[NV][4];
+    auto clear = [&]() {
+#pragma unroll
+        for (int i = 0; i < NV; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    };
+    auto store = [&](int pos) {
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int c = (lane + 32 * i) * 4;
+            if (c < C) store4(part + (long long)pos * C + c, acc[i]);
+        }
+    };
+    clear();
+    int pstart = e0;
+    unsigned tok_cur = __shfl_sync(0xffffffffu, mykey, 0) >> 16;
+    for (int e = 0; e < cnt; e += U) {
+        float v[U][NV][4];
+        unsigned key[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            key[u] = __shfl_sync(0xffffffffu, mykey, e + u);
+            if (e + u < cnt) {
+                const float* src = dx + (long long)(key[u] & 0xFFFFu) * C;
+#pragma unroll
+                for (int i = 0; i < NV; ++i) {
+                    const int c = (lane + 32 * i) * 4;
+                    if (c < C) load4(src + c, v[u][i]);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (e + u < cnt) {
+                if ((key[u] >> 16) != tok_cur) {   // a new run starts a new piece
+                    store(pstart);
+                    clear();
+                    pstart = e0 + e + u;
+                    tok_cur = key[u] >> 16;
+                }
+#pragma unroll
+                for (int i = 0; i < NV; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] += v[u][i][j];
+            }
+        }
+    }
+    store(pstart);
+}
+
+// (3a) A warp per run (a token's entries inside one chunk) adds the run's pieces in
+// position order and leaves the run's sum in the slot of its first piece.
+template <int NV>
+__global__ void __launch_bounds__(256) emb_run_kernel(const unsigned* __restrict__ sorted, int n,
+                                                      float* __restrict__ part, int C) {
+    constexpr int U = emb_batch<NV>();
+    const int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    if (p >= n) return;
+    const int chunk = p / EMB_CHUNK;
+    const unsigned tok = sorted[p] >> 16;
+    if (p > chunk * EMB_CHUNK && (sorted[p - 1] >> 16) == tok) return;   // not the start of a run
+    const int cend = min(n, (chunk + 1) * EMB_CHUNK);
+    const int b1 = (p / EMB_WIN + 1) * EMB_WIN;   // the run's later pieces start at window boundaries
+    if (b1 >= cend || (sorted[b1] >> 16) != tok) return;   // one piece: already the run's sum
+    float acc[NV][4];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c = (lane + 32 * i) * 4;
+        if (c < C) load4(part + (long long)p * C + c, acc[i]);
+    }
+    for (int q = b1; q < cend && (sorted[q] >> 16) == tok; q += U * EMB_WIN) {
+        float v[U][NV][4];
+        bool ok[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int qu = q + u * EMB_WIN;
+            ok[u] = u == 0 || (ok[u - 1] && qu < cend && (sorted[qu] >> 16) == tok);
+            if (ok[u]) {
+#pragma unroll
+                for (int i = 0; i < NV; ++i) {
+                    const int c = (lane + 32 * i) * 4;
+                    if (c < C) load4(part + (long long)qu * C + c, v[u][i]);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (ok[u]) {
+#pragma unroll
+                for (int i = 0; i < NV; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] += v[u][i][j];
+            }
+        }
+        if (!ok[U - 1]) break;
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c = (lane + 32 * i) * 4;
+        if (c < C) store4(part + (long long)p * C + c, acc[i]);
+    }
+}
+
+// (3b) A warp per run finds, by a binary search per chunk (one lane each), where
+// its token's run starts in every chunk; the warp of the token's first chunk adds
+// the runs' sums in chunk order into dwte[token].
+template <int NV>
+__global__ void __launch_bounds__(256) emb_token_kernel(const unsigned* __restrict__ sorted, int n,
+                                                        const float* __restrict__ part, int C,
+                                                        float* __restrict__ dwte) {
+    const int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    if (p >= n) return;
+    const int chunk = p / EMB_CHUNK;
+    const unsigned tok = sorted[p] >> 16;
+    if (p > chunk * EMB_CHUNK && (sorted[p - 1] >> 16) == tok) return;   // not the start of a run
+    const int nch = (n + EMB_CHUNK - 1) / EMB_CHUNK;
+    int start = -1;   // lane c: where the token's run starts in chunk c (lower bound of tok << 16)
+    if (lane < nch && lane != chunk) {
+        int lo = lane * EMB_CHUNK, hi = min(n, lo + EMB_CHUNK);
+        const int end = hi;
+        const unsigned key = tok << 16;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (sorted[mid] < key) lo = mid + 1;
+            else hi = mid;
+        }
+        if (lo < end && (sorted[lo] >> 16) == tok) start = lo;
+    }
+    if (lane == chunk) start = p;
+    const unsigned present = __ballot_sync(0xffffffffu, start >= 0);
+    if ((int)(__ffs(present) - 1) != chunk) return;   // an earlier chunk's run owns the token
+    float acc[NV][4];
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    float* d = dwte + (long long)tok * C;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c = (lane + 32 * i) * 4;
+        if (c < C) load4(d + c, acc[i]);
+    }
+    for (unsigned m = present; m; m &= m - 1) {
+        const int q = __shfl_sync(0xffffffffu, start, __ffs(m) - 1);
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int c = (lane + 32 * i) * 4;
+            if (c < C) {
+                float v[4];
+                load4(part + (long long)q * C + c, v);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] += v[j];
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c = (lane + 32 * i) * 4;
+        if (c < C) store4(d + c, acc[i]);
+    }
+}
+
+template <int NV>
+void emb_tile(const Ctx& ctx, const int* idx, const float* dx, int rows, int C, int V, float* dwte, float* part,
+              unsigned* sorted) {
+    emb_sort_kernel<<<ceil_div(rows, EMB_CHUNK), EMB_CHUNK / 2, 0, ctx.stream>>>(idx, rows, V, sorted);
+    const int windows = ceil_div(rows, EMB_WIN);
+    emb_piece_kernel<NV><<<ceil_div(windows, 8), 256, 0, ctx.stream>>>(sorted, rows, dx, C, part);
+    emb_run_kernel<NV><<<ceil_div(rows, 8), 256, 0, ctx.stream>>>(sorted, rows, part, C);
+    emb_token_kernel<NV><<<ceil_div(rows, 8), 256, 0, ctx.stream>>>(sorted, rows, part, C, dwte);
+    *ctx.launches += 4;
+}
+
 __global__ void embed_bwd_wpe_kernel(const float* __restrict__ dx, int B, int Tn, int C, float* dwpe) {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (long long)Tn * C) return;
@@ -780,11 +1014,33 @@ void launch_colsum(const Ctx& ctx, const T* in, int rows, int cols, float* out, 
 }
 
 void launch_embed_bwd(const Ctx& ctx, const int* idx, const float* dx, int B, int Tn, int C, int V, float* dwte,
-                      float* dwpe) {
-    const long long n4 = (long long)B * Tn * (C / 4);
-    embed_bwd_wte_kernel<<<(unsigned)ceil_div_ll(n4, 256), 256, 0, ctx.stream>>>(idx, dx, B * Tn, C, V, dwte);
+                      float* dwpe, float* scratch) {
+    const long long rows = (long long)B * Tn;
+    const int nv = ceil_div(C, 128);
+    if (scratch && V <= 65536 && nv <= 16 && C % 4 == 0) {
+        float* part = scratch;
+        unsigned* sorted = reinterpret_cast<unsigned*>(scratch + rows * C);
+        for (long long r0 = 0; r0 < rows; r0 += EMB_TILE) {   // tiles in row order
+            const int n = (int)std::min<long long>(EMB_TILE, rows - r0);
+            const int* ti = idx + r0;
+            const float* td = dx + r0 * C;
+#define EMB_CASE(NV) \
+    case NV: emb_tile<NV>(ctx, ti, td, n, C, V, dwte, part, sorted); break;
+            switch (nv) {
+                EMB_CASE(1) EMB_CASE(2) EMB_CASE(3) EMB_CASE(4) EMB_CASE(5) EMB_CASE(6) EMB_CASE(7) EMB_CASE(8)
+                EMB_CASE(9) EMB_CASE(10) EMB_CASE(11) EMB_CASE(12) EMB_CASE(13) EMB_CASE(14) EMB_CASE(15)
+                EMB_CASE(16)
+                default: break;
+            }
+#undef EMB_CASE
+        }
+    } else {
+        const long long n4 = rows * (C / 4);
+        embed_bwd_wte_kernel<<<(unsigned)ceil_div_ll(n4, 256), 256, 0, ctx.stream>>>(idx, dx, (int)rows, C, V, dwte);
+        ++*ctx.launches;
+    }
     embed_bwd_wpe_kernel<<<(unsigned)ceil_div_ll((long long)Tn * C, 256), 256, 0, ctx.stream>>>(dx, B, Tn, C, dwpe);
-    *ctx.launches += 2;
+    ++*ctx.launches;
 }
 
 #define INST(T)                                                                                                 \

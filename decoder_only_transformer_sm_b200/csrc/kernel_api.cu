@@ -187,3 +187,22 @@ extern "C" int gpt2k_sample(int dtype, const void* logits, int rows, int V, int6
     if (err != cudaSuccess) return set_error(GPT2_ERR_CUDA, cudaGetErrorString(err));
     return GPT2_OK;
 }
+
+extern "C" int gpt2k_embedding_bwd_workspace(int B, int T, int C, int64_t* floats) {
+    if (B < 1 || T < 1 || C < 1 || !floats) return set_error(GPT2_ERR_INVALID_ARG, "need B, T, C >= 1 and floats");
+    *floats = (int64_t)embed_bwd_scratch_floats((long long)B * T, C);
+    return GPT2_OK;
+}
+
+extern "C" int gpt2k_embedding_bwd(const int32_t* idx, const float* dx, int B, int T, int C, int V, float* dwte,
+                                   float* dwpe, float* workspace_dev, uint32_t* status_dev, void* stream) {
+    if (B < 1 || T < 1 || C < 1 || V < 1) return set_error(GPT2_ERR_INVALID_ARG, "need B, T, C, V >= 1");
+    if (C % 4 != 0) return set_error(GPT2_ERR_INVALID_ARG, "C must be a multiple of 4");
+    if (!idx || !dx || !dwte || !dwpe || !status_dev) return set_error(GPT2_ERR_INVALID_ARG, "NULL operand");
+    long long launches = 0;
+    Ctx c = kctx(stream, status_dev, &launches);
+    launch_embed_bwd(c, idx, dx, B, T, C, V, dwte, dwpe, workspace_dev);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return set_error(GPT2_ERR_CUDA, cudaGetErrorString(err));
+    return GPT2_OK;
+}

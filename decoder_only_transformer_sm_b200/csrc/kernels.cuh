@@ -200,9 +200,13 @@ template <typename T>
 void launch_colsum(const Ctx& ctx, const T* in, int rows, int cols, float* out, float* scratch);
 // out[j] += sum_b partial[b * n + j], b < nblk, in a fixed order.
 void launch_colred_finalize(const Ctx& ctx, const float* partial, int nblk, int n, float* out);
-// dwte[idx[r]] += dx[r]; dwpe[t] += sum_b dx[b, t].
+// dwte[idx[r]] += dx[r]; dwpe[t] += sum_b dx[b, t]. With scratch (at least
+// embed_bwd_scratch_floats(B * Tn, C) floats) and V <= 65536, deterministic: the
+// rows of each token are added in row order (a sort by token, then sums of runs);
+// otherwise per-element atomics.
+inline long long embed_bwd_scratch_floats(long long rows, int C) { return rows * (long long)C + rows + 64; }
 void launch_embed_bwd(const Ctx& ctx, const int* idx, const float* dx, int B, int Tn, int C, int V, float* dwte,
-                      float* dwpe);
+                      float* dwpe, float* scratch = nullptr);
 
 // ----------------------------------------------------------------------------
 // Attention (causal, per (b, h); q/k/v are column blocks of the qkv rows).

@@ -100,6 +100,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "gpt2k_attention_bwd_workspace": (I, [I, I, I, I, I, ctypes.POINTER(ctypes.c_int64)]),
         "gpt2k_attention_decode": (I, [I, P, P, I, I, I, I, I, P, P, P]),
         "gpt2k_sample": (I, [I, P, I, I, ctypes.c_int64, F, I, P, P, P, P]),
+        "gpt2k_embedding_bwd": (I, [P, P, I, I, I, I, P, P, P, P, P]),
+        "gpt2k_embedding_bwd_workspace": (I, [I, I, I, ctypes.POINTER(ctypes.c_int64)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -409,6 +411,23 @@ def attention_bwd_noalloc(qkv, out, dout, lse, dqkv, B: int, T: int, H: int, hd:
     status, stream = _stream_and_status(qkv, status, stream)
     _check(fn(_dtype_code(qkv), _ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dqkv), B, T, H, hd, engine,
               _ptr(status), stream))
+    return status
+
+
+def embedding_bwd_workspace(B: int, T: int, C: int) -> int:
+    """Float32 elements of the workspace gpt2k_embedding_bwd needs."""
+    n = ctypes.c_int64()
+    _check(load_library().gpt2k_embedding_bwd_workspace(B, T, C, ctypes.byref(n)))
+    return n.value
+
+
+def embedding_bwd(idx, dx, dwte, dwpe, B: int, T: int, workspace=None, status=None, stream=None):
+    """gpt2k_embedding_bwd: dwte[idx] += dx rows and dwpe[t] += sum over b, on torch
+    device tensors (idx int32 (B*T), dx float32 (B*T, C), dwte (V, C), dwpe (T, C));
+    with a workspace (embedding_bwd_workspace(...) float32) in a fixed order."""
+    status, stream = _stream_and_status(dx, status, stream)
+    _check(load_library().gpt2k_embedding_bwd(_ptr(idx), _ptr(dx), B, T, dx.shape[-1], dwte.shape[0], _ptr(dwte),
+                                              _ptr(dwpe), _ptr(workspace), _ptr(status), stream))
     return status
 
 

@@ -151,6 +151,26 @@ int gpt2k_attention_decode(int dtype, const void* cache, void* out, int B, int H
 int gpt2k_sample(int dtype, const void* logits, int rows, int V, int64_t ld, float temperature, int top_k,
                  const float* u_dev, int32_t* next_dev, uint32_t* status_dev, void* stream);
 
+/* Backward of the embedding sum ("GPT-2 from Scratch", "Embeddings: tokens and
+ * positions", with the token table tied to lm_head as in "Weight tying"):
+ * dwte[idx[r]] += dx[r] for every row r = b * T + t, and dwpe[t] += sum_b dx[b * T + t].
+ * idx (B*T) int32 ids in [0, V) (an id outside is clamped to that range, as in
+ * the step, which rejects such ids before it gets here); dx fp32 [B*T, C];
+ * dwte fp32 [V, C] and dwpe fp32 [T, C] are accumulated into, not overwritten.
+ * workspace_dev: NULL, or at least gpt2k_embedding_bwd_workspace(...) floats.
+ * With a workspace, V <= 65536, C a multiple of 4 and C <= 2048, each token's
+ * rows are added in row order (per tile of 16384 rows, tiles in order), so
+ * identical inputs give bit-identical results; otherwise fp32 atomics, whose
+ * last bits depend on the order of arrival. dwpe's sums are in b order in both.
+ * Errors: INVALID_ARG (B, T, C or V < 1, C not a multiple of 4, a NULL pointer
+ * other than workspace_dev). */
+int gpt2k_embedding_bwd(const int32_t* idx, const float* dx, int B, int T, int C, int V, float* dwte, float* dwpe,
+                        float* workspace_dev, uint32_t* status_dev, void* stream);
+
+/* Workspace size of gpt2k_embedding_bwd in floats (into *floats). Errors:
+ * INVALID_ARG (B, T or C < 1, floats NULL). */
+int gpt2k_embedding_bwd_workspace(int B, int T, int C, int64_t* floats);
+
 #ifdef __cplusplus
 }
 #endif

@@ -289,10 +289,26 @@ def backward(s: Shape, P: dict, cache, loss_scale: float = 1.0) -> dict:
         G[pre + "ln_1.weight"] += dw
         G[pre + "ln_1.bias"] += db
         dx = dx + dln
-    # x0 = wte[idx] + wpe[arange(T)]: scatter-add into the same tied wte gradient
-    np.add.at(G["wte"], idx.reshape(-1), dx.reshape(-1, C))
-    G["wpe"][:T] += dx.sum(axis=0)
+    dwte, dwpe = embedding_backward(idx, dx, s.vocab_size, s.block_size)
+    G["wte"] += dwte
+    G["wpe"] += dwpe
     return G
+
+
+def embedding_backward(idx, dx, V: int, block_size: int):
+    """Gradient of x0 = wte[idx] + wpe[arange(T)] ("GPT-2 from Scratch",
+    "Embeddings: tokens and positions"): every row of dx lands on its token's row
+    of the token table (a token seen n times gets the sum of its n rows; with
+    "Weight tying" this adds to the lm_head term of the same table), and position
+    t gets the sum over the batch of dx[:, t]. Returns (dwte (V, C), dwpe
+    (block_size, C)); rows of dwpe at t >= T are zero."""
+    B, T = idx.shape
+    C = dx.shape[-1]
+    dwte = np.zeros((V, C))
+    np.add.at(dwte, idx.reshape(-1), dx.reshape(-1, C))
+    dwpe = np.zeros((block_size, C))
+    dwpe[:T] = dx.sum(axis=0)
+    return dwte, dwpe
 
 
 # ----------------------------------------------------------------------------

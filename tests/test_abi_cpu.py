@@ -111,3 +111,21 @@ def test_generation_entries_reject_bad_arguments_on_host():
         args = list(okd)
         args[i] = bad
         assert lib.gpt2k_attention_decode(*args) == -1, (i, bad)
+
+
+def test_embedding_bwd_rejects_bad_arguments_on_host():
+    """gpt2k_embedding_bwd validates sizes and pointers before any CUDA call (no GPU
+    needed): sizes below 1, C not a multiple of 4, NULL operands (the workspace
+    alone may be NULL). Its workspace size is rows x C + rows + 64 floats."""
+    lib = native.load_library()
+    dummy = ctypes.c_void_p(16)   # never dereferenced: validation fails first
+    ok = (dummy, dummy, 2, 4, 8, 100, dummy, dummy, None, dummy, None)
+    for i, bad in [(2, 0), (3, 0), (4, 0), (4, 6), (5, 0), (0, None), (1, None), (6, None), (7, None), (9, None)]:
+        args = list(ok)
+        args[i] = bad
+        assert lib.gpt2k_embedding_bwd(*args) == -1, (i, bad)
+    n = ctypes.c_int64()
+    assert lib.gpt2k_embedding_bwd_workspace(2, 4, 8, ctypes.byref(n)) == 0
+    assert n.value == 8 * 8 + 8 + 64
+    assert lib.gpt2k_embedding_bwd_workspace(0, 4, 8, ctypes.byref(n)) == -1
+    assert lib.gpt2k_embedding_bwd_workspace(2, 4, 8, None) == -1

@@ -389,6 +389,63 @@ def test_bf16_accumulation_with_masks_matches_oracle():
     m.close()
 
 
+def test_embedding_gradient_is_deterministic():
+    """The token-embedding gradient adds each token's rows in row order (a sort by
+    token, then sums of each token's run), not with atomics: in fp32 mode, whose
+    other kernels have fixed summation orders too at this shape, two identical
+    gradient passes give a bit-identical wte gradient. The shape keeps the tied
+    lm_head's weight gradient, the other term of that gradient, off split-K (V x C
+    has more 128 x 256 tiles than the GPU has SMs). Zipf tokens repeat many ids
+    (the most frequent one thousands of times, across many windows of the sorted
+    list), and 20480 rows are more than one sort tile (16384). (In bf16 mode the
+    rows reaching the embedding already differ in their last bits from pass to
+    pass: the attention backward adds dQ partials in order of arrival. The
+    kernel-level tests check the embedding backward itself on fixed rows.)"""
+    s = S.ModelShape(1, 2, 128, 50304, 1024)
+    B, T = 20, 1024
+    flat = S.random_params(s, seed=81)
+    idx, tgt = S.zipf_tokens(B, T, 50257, seed=82)
+    m = _model(s, "fp32", B, T)
+    m.set_params(flat)
+    grads = []
+    for _ in range(2):
+        m.zero_grad()
+        m.accumulate(_dev(idx), _dev(tgt), 1.0)
+        grads.append(_split(s, m.get_grads())["wte"])
+    assert np.array_equal(grads[0], grads[1])
+    m.close()
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_embedding_gradient_two_sort_tiles_matches_oracle(precision):
+    """17 x 1024 rows: one full sort tile of 16384 rows and a ragged one of 1024.
+    A vocabulary of 256 Zipf ids makes runs from a few rows up to thousands, so
+    runs cross 16-entry windows and the tile boundary. The wte gradient is
+    compared row by row with the oracle's (each row against its own largest
+    element), so that a dropped or doubled embedding row shows even for a rare
+    token: fp32 to 1e-4 of the row, bf16 by the row's cosine."""
+    s = S.ModelShape(1, 1, 64, 256, 1024)
+    B, T = 17, 1024
+    idx, tgt = S.zipf_tokens(B, T, s.vocab_size, seed=82)
+    flat = S.random_params(s, seed=81)
+    P = O.unflatten(_oshape(s), flat.astype(np.float64))
+    Mo, Vo = O.zeros_like(_oshape(s)), O.zeros_like(_oshape(s))
+    _, _, G = O.train_step(_oshape(s), P, Mo, Vo, 1, idx, tgt, lr=1e-4)
+    m = _model(s, precision, B, T)
+    m.set_params(flat)
+    m.zero_grad()
+    m.accumulate(_dev(idx), _dev(tgt), 1.0)
+    g, r = _split(s, m.get_grads())["wte"].astype(np.float64), G["wte"]
+    counts = np.bincount(idx.ravel(), minlength=s.vocab_size)
+    assert counts.min() >= 1 and counts.max() > 16384 // 16
+    for v in range(s.vocab_size):
+        if precision == "fp32":
+            assert np.max(np.abs(g[v] - r[v])) <= 1e-4 * np.max(np.abs(r[v])), (v, counts[v])
+        else:
+            assert _cos(g[v], r[v]) >= 0.99, (v, counts[v], _cos(g[v], r[v]))
+    m.close()
+
+
 def test_step_graph_replay_matches_eager(monkeypatch):
     """Steps 3+ with one (B, T) replay a captured CUDA graph; a shape change drops
     it. A graph model and an eager model (graphs off) take the same ten steps,

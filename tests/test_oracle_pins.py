@@ -143,6 +143,31 @@ def test_position_zero_indexing():
     assert np.array_equal(la[:, :7], lb[:, :7]) and not np.allclose(la[:, 7], lb[:, 7])
 
 
+def test_embedding_backward_is_the_transposed_jacobian():
+    """x0[b, t] = wte[idx[b, t]] + wpe[t] is linear in both tables, so the gradient
+    of sum(x0 * dx) is the transposed selection matrix applied to dx: one-hot(idx)^T
+    dx for wte (repeated ids add up, unused ids stay zero) and, for wpe, the sum
+    over b at each used position. Also a hand-worked case with a repeated id."""
+    rng = np.random.default_rng(11)
+    B, T, V, C, bs = 3, 5, 7, 4, 8
+    idx = rng.integers(0, V, size=(B, T))
+    idx[0, 0] = idx[2, 4] = 3                       # a repeat across sequences
+    dx = rng.normal(size=(B, T, C))
+    dwte, dwpe = O.embedding_backward(idx, dx, V, bs)
+    onehot = np.zeros((B * T, V))
+    onehot[np.arange(B * T), idx.reshape(-1)] = 1.0
+    np.testing.assert_allclose(dwte, onehot.T @ dx.reshape(-1, C), rtol=0, atol=1e-12)
+    sel = np.zeros((B * T, bs))
+    sel[np.arange(B * T), np.tile(np.arange(T), B)] = 1.0
+    np.testing.assert_allclose(dwpe, sel.T @ dx.reshape(-1, C), rtol=0, atol=1e-12)
+    assert not dwpe[T:].any()
+    small = np.array([[1, 0, 1]])
+    d = np.array([[[1.0, 2.0], [3.0, 4.0], [5.0, 6.0]]])
+    w, p = O.embedding_backward(small, d, 3, 4)
+    assert np.array_equal(w, [[3.0, 4.0], [6.0, 8.0], [0.0, 0.0]])
+    assert np.array_equal(p, [[1.0, 2.0], [3.0, 4.0], [5.0, 6.0], [0.0, 0.0]])
+
+
 # ----------------------------------------------------------------------------
 # GELU ("The MLP and GPT-2's GELU").
 # ----------------------------------------------------------------------------
@@ -500,7 +525,8 @@ def test_overfit_single_batch():
 # ----------------------------------------------------------------------------
 # The pins are sensitive: a planted mistake in the oracle's backward fails them.
 # ----------------------------------------------------------------------------
-@pytest.mark.parametrize("mutation", ["ln_drop_term", "gelu_grad_const", "attn_rowsum", "tie_scatter"])
+@pytest.mark.parametrize("mutation", ["ln_drop_term", "gelu_grad_const", "attn_rowsum", "tie_scatter",
+                                      "scatter_drops_repeats"])
 def test_planted_mistakes_are_caught(monkeypatch, mutation):
     if mutation == "ln_drop_term":
         def bad(dy, saved, w):
@@ -527,14 +553,24 @@ def test_planted_mistakes_are_caught(monkeypatch, mutation):
             G["wte"][cache["idx"].reshape(-1)] *= 0.5      # lose part of the embedding scatter
             return G
         monkeypatch.setattr(O, "backward", bad_backward)
+    elif mutation == "scatter_drops_repeats":
+        def bad(idx, dx, V, block_size):
+            C = dx.shape[-1]
+            dwte = np.zeros((V, C))
+            dwte[idx.reshape(-1)] += dx.reshape(-1, C)   # buffered: a repeated id keeps one row
+            dwpe = np.zeros((block_size, C))
+            dwpe[:idx.shape[1]] = dx.sum(axis=0)
+            return dwte, dwpe
+        monkeypatch.setattr(O, "embedding_backward", bad)
     s = MICRO
     P = _params(s, seed=30, kind="random")
     for k in P:
         if P[k].ndim == 2:
             P[k] *= 10.0
-    idx, tgt = S.uniform_tokens(2, 8, 64, seed=31)
+    idx, tgt = S.uniform_tokens(2, 8, 64, seed=31)   # ids 43 and 11 occur twice
+    coords = None if mutation == "scatter_drops_repeats" else 8   # every coordinate reaches the repeated rows
     with pytest.raises(AssertionError):
-        _fd_check(s, P, idx, tgt, 8, np.random.default_rng(2))
+        _fd_check(s, P, idx, tgt, coords, np.random.default_rng(2))
 
 
 # ----------------------------------------------------------------------------
