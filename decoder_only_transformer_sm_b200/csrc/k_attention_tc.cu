@@ -9,20 +9,27 @@
 // and row sum l, so no T x T matrix is stored; lse = m + log(l) is kept for
 // the backward.
 //
-// Work item = one (b, h) and 128 queries (one query row per TMEM lane). The
-// kernel is persistent: one CTA per SM walks the items, longest causal prefix
-// first. Warp 0 loads each item's Q (double-buffered, so the next item's Q
-// arrives during the current one) and the K/V tiles of its causal prefix
-// through a 3-stage TMA ring; warp 1 issues, from one thread, S_j = Q K_j^T (M=128,
-// N=128, K=64) into one of two TMEM S buffers and PV_j = P_j V_j (M=128, N=64,
-// K=128; V described as an N-major operand) into one of two TMEM PV buffers;
-// warps 2..9 are the softmax warps, two per TMEM lane quarter: each owns 64 of
-// the 128 keys of S_j (one 64-key swizzle atom of P) and 32 of the 64 output
-// columns. They read S_j from TMEM in two passes (partial row max, exchanged
-// with the pair through shared memory; then exp2 / partial row sum / bf16 P
-// into the 128-byte-swizzled K-major shared tile), then fold their half of
-// PV_{j-1} into the register-resident output row:
-// O = O * exp2(m_{j-2} - m_{j-1}) + PV. The pair's row sums meet once at the end.
+// Work item = one (b, h) and a pair of consecutive 128-query tiles (2p, 2p+1),
+// one per softmax warpgroup ("group"); both walk the same key tiles, so each K/V
+// tile is loaded once for the pair. The kernel is persistent: one CTA per SM
+// walks the items, longest causal prefixes first, dealt to the CTAs round by
+// round in alternating direction. Warp 0 loads an item's two Q tiles
+// (double-buffered over items) and its K/V tiles through a 3-stage TMA ring.
+// Warp 1 issues, from one thread, for group g and key tile j: S_g = Q_g K_j^T
+// (M=128, N=128, K=64) into the group's TMEM S columns; once the group's softmax
+// has written P_g, O_g += P_g V_j (M=128, N=64, K=128; P_g read from TMEM as
+// packed bf16, V an N-major shared-memory operand, O_g accumulated in TMEM), and
+// right after it the S of the group's next tile. While one group's softmax runs,
+// the other group's MMAs run.
+// Warps 2..5 (group 0) and 6..9 (group 1) are the softmax warps: thread = query
+// row (TMEM lane) with all 128 keys of S_g in registers. The running row max m
+// is raised only when a tile's max exceeds it by more than FW_RESCALE (log2
+// units); then O (in TMEM) and l are rescaled by 2^(m_old - m_new). Otherwise P
+// = 2^(s - m) stays below 2^FW_RESCALE and O / l is the same in exact
+// arithmetic. P goes to TMEM as bf16 pairs; the row sum l (fp32, of the
+// unrounded exponentials) stays in a register. At an item's end each thread
+// reads its O row from TMEM, divides by l and writes it through a
+// shared-memory staging tile in 128-byte rows.
 // Every wait is bounded (2 s) and reports a timeout in the status word.
 #include <cudaTypedefs.h>
 
@@ -36,33 +43,32 @@ namespace {
 constexpr int HD = 64;
 constexpr int BQ = 128, BKV = 128;
 constexpr int KV_STAGES = 3;
-constexpr int SM_WARPS = 8;                       // softmax warps: 2 per TMEM lane quarter
-constexpr int THREADS = 64 + 32 * SM_WARPS;
+constexpr int FW_THREADS = 64 + 32 * 8;           // TMA warp, MMA warp, two softmax warpgroups
 constexpr int TILE_BYTES = 128 * HD * 2;          // 16 KB: 128 rows x 128 bytes
-constexpr int P_BYTES = BQ * BKV * 2;             // 32 KB: two 64-key swizzle atoms of 16 KB
-constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_PV0 = 256, TM_PV1 = 320;
 constexpr float LOG2E = 1.4426950408889634f;
+constexpr float FW_RESCALE = 8.f;                 // growth of the row max (log2 units) that triggers a rescale
+// TMEM columns of group g, from g * FT_GROUP: S (128 fp32), P (128 keys as bf16
+// pairs), O (64 fp32)
+constexpr uint32_t FT_S = 0, FT_P = 128, FT_O = 192, FT_GROUP = 256;
 
-struct Ctl {
-    uint64_t q_full[2], q_empty[2];
+struct FwCtl {
+    uint64_t q_full[2], q_empty[2];               // Q sets (both groups' tiles of one item)
     uint64_t kv_full[KV_STAGES], kv_empty[KV_STAGES];
-    uint64_t s_full[2], s_empty[2];
-    uint64_t p_full[2];
-    uint64_t pv_full[2], pv_empty[2];
+    uint64_t s_full[2];                           // per group: S of its current tile is in TMEM
+    uint64_t p_full[2];                           // per group: P written to TMEM (its 4 warps arrive)
+    uint64_t pv_done[2];                          // per group: O += P V of its latest tile is done
     uint64_t drain;
     uint32_t tmem_base;
     uint32_t abort;
-    float mx[2][2][BQ];                           // [tile parity][column half][row]: partial row max
-    float lsum[2][BQ];                            // [column half][row]: partial row sum at the end
 };
 
-// smem: Q[2] | K[3] | V[3] | P[2] | ctl
-constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
-constexpr int OFF_V = OFF_K + KV_STAGES * TILE_BYTES;
-constexpr int OFF_P = OFF_V + KV_STAGES * TILE_BYTES;
-constexpr int OFF_CTL = OFF_P + 2 * P_BYTES;
-constexpr size_t SMEM_BYTES = OFF_CTL + sizeof(Ctl) + 1024;
+// smem: Q[2 sets x 2 groups] | K[3] | V[3] | output staging [2 groups] | ctl
+constexpr int FW_OFF_Q = 0;
+constexpr int FW_OFF_K = 4 * TILE_BYTES;
+constexpr int FW_OFF_V = FW_OFF_K + KV_STAGES * TILE_BYTES;
+constexpr int FW_OFF_ST = FW_OFF_V + KV_STAGES * TILE_BYTES;
+constexpr int FW_OFF_CTL = FW_OFF_ST + 2 * TILE_BYTES;
+constexpr size_t FW_SMEM = FW_OFF_CTL + sizeof(FwCtl) + 1024;
 
 __device__ __forceinline__ uint32_t swz128(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 
@@ -74,11 +80,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-__device__ __forceinline__ void ew_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-// The two softmax warps of one TMEM lane quarter (named barriers 2..5).
-__device__ __forceinline__ void pair_bar(int quarter) {
-    asm volatile("bar.sync %0, 64;" ::"r"(2 + quarter) : "memory");
-}
 
 // max(a, b, c) in one instruction (sm_100 three-input max.f32)
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -113,33 +114,55 @@ __device__ __forceinline__ uint4 pack8_bf16(const float* v) {
     return q;
 }
 
-// Work item i of the forward (longest causal prefixes first over the whole
-// grid): query tile n_qt - 1 - i / BH of head-sequence i % BH.
-struct FwdItem {
+// Work item i: head-sequence i % BH and query-tile pair n_pairs - 1 - i / BH
+// (longest causal prefixes first). Group g's tile starts at q0 + 128 g and uses
+// key tiles 0 .. n[g] - 1 (n[1] = 0 when that tile lies past Tn); the item walks
+// n_kv = max(n[0], n[1]) key tiles.
+struct FwItem {
     int bh, q0, n_kv;
+    int n[2];
 };
-__device__ __forceinline__ FwdItem fwd_item(int i, int BH, int n_qt, int Tn) {
-    FwdItem it;
+__device__ __forceinline__ FwItem fw_item(int i, int BH, int n_pairs, int Tn) {
+    FwItem it;
     it.bh = i % BH;
-    it.q0 = (n_qt - 1 - i / BH) * BQ;
-    it.n_kv = (min(Tn, it.q0 + BQ) + BKV - 1) / BKV;   // key tiles 0 .. n_kv-1
+    it.q0 = (n_pairs - 1 - i / BH) * 2 * BQ;
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        const int q = it.q0 + g * BQ;
+        it.n[g] = q < Tn ? (min(Tn, q + BQ) + BKV - 1) / BKV : 0;
+    }
+    it.n_kv = max(it.n[0], it.n[1]);
     return it;
 }
 
-// Persistent: gridDim.x CTAs (at most one per SM) walk the items
-// blockIdx.x, blockIdx.x + gridDim.x, ... Every ring and buffer parity runs on
-// counters over all the CTA's tiles, so the loads and S MMAs of the next item
-// overlap the softmax and output of the current one.
-__global__ void __launch_bounds__(THREADS, 1)
+// The item this CTA takes in round k (rounds of gridDim.x items, dealt in
+// alternating direction so that the longest and shortest even out), or -1.
+__device__ __forceinline__ int fw_round_item(int k, int n_items) {
+    const int G = gridDim.x;
+    const int i = k * G + ((k & 1) ? G - 1 - (int)blockIdx.x : (int)blockIdx.x);
+    return i < n_items ? i : -1;
+}
+
+// Lane 0 waits on the mbarrier phase; the whole warp gets the result.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
+                                          unsigned* status) {
+    uint32_t w = 0;
+    if ((threadIdx.x & 31) == 0) w = tc::mbar_wait(bar, parity, abort, status) ? 1u : 0u;
+    return __shfl_sync(0xffffffffu, w, 0) != 0;
+}
+
+__global__ void __launch_bounds__(FW_THREADS, 1)
     flash_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse,
                         int Tn, int H, int BH, unsigned* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Ctl* ctl = reinterpret_cast<Ctl*>(smem + OFF_CTL);
+    FwCtl* ctl = reinterpret_cast<FwCtl*>(smem + FW_OFF_CTL);
     volatile uint32_t* abort = &ctl->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_qt = (Tn + BQ - 1) / BQ;
-    const int n_items = BH * n_qt;
+    const int n_pairs = (n_qt + 1) / 2;
+    const int n_items = BH * n_pairs;
+    const int n_rounds = (n_items + (int)gridDim.x - 1) / (int)gridDim.x;
     const int C = H * HD;
 
     if (threadIdx.x == 0) {
@@ -147,10 +170,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::mbar_init(&ctl->q_full[i], 1);
             tc::mbar_init(&ctl->q_empty[i], 1);
             tc::mbar_init(&ctl->s_full[i], 1);
-            tc::mbar_init(&ctl->s_empty[i], SM_WARPS);
-            tc::mbar_init(&ctl->p_full[i], SM_WARPS);
-            tc::mbar_init(&ctl->pv_full[i], 1);
-            tc::mbar_init(&ctl->pv_empty[i], SM_WARPS);
+            tc::mbar_init(&ctl->p_full[i], 4);
+            tc::mbar_init(&ctl->pv_done[i], 1);
         }
         for (int s = 0; s < KV_STAGES; ++s) {
             tc::mbar_init(&ctl->kv_full[s], 1);
@@ -173,26 +194,32 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0) {
             // --------------------------------------------------------------- TMA
             tc::tma_prefetch_desc(&tm_qkv);
-            uint32_t g = 0;                           // K/V tile counter over all items
-            uint32_t ord = 0;                         // item counter (Q buffer ring)
+            uint32_t gs = 0;                          // K/V step counter over all items
+            uint32_t ord = 0;                         // item counter (Q set ring)
             bool ok = true;
-            for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, ++ord) {
-                const FwdItem it = fwd_item(i, BH, n_qt, Tn);
+            for (int k = 0; k < n_rounds && ok; ++k) {
+                const int i = fw_round_item(k, n_items);
+                if (i < 0) continue;
+                const FwItem it = fw_item(i, BH, n_pairs, Tn);
                 const int row_base = (it.bh / H) * Tn, h = it.bh % H;
-                const int qb = ord & 1;
-                if (!tc::mbar_wait(&ctl->q_empty[qb], ((ord >> 1) & 1) ^ 1, abort, status)) break;
-                tc::mbar_expect_tx(&ctl->q_full[qb], TILE_BYTES);
-                tc::tma_load_2d(smem + OFF_Q + qb * TILE_BYTES, &tm_qkv, h * HD, row_base + it.q0, &ctl->q_full[qb]);
-                for (int j = 0; j < it.n_kv; ++j, ++g) {
-                    const int s = g % KV_STAGES;
-                    const uint32_t ph = (g / KV_STAGES) & 1;
+                const int qs = ord & 1;
+                if (!tc::mbar_wait(&ctl->q_empty[qs], ((ord >> 1) & 1) ^ 1, abort, status)) break;
+                tc::mbar_expect_tx(&ctl->q_full[qs], 2 * TILE_BYTES);
+                // the second tile may lie past Tn (then unused; rows past the tensor read as zero)
+                for (int g = 0; g < 2; ++g)
+                    tc::tma_load_2d(smem + FW_OFF_Q + (2 * qs + g) * TILE_BYTES, &tm_qkv, h * HD,
+                                    row_base + it.q0 + g * BQ, &ctl->q_full[qs]);
+                for (int j = 0; j < it.n_kv; ++j, ++gs) {
+                    const int s = gs % KV_STAGES;
+                    const uint32_t ph = (gs / KV_STAGES) & 1;
                     if (!tc::mbar_wait(&ctl->kv_empty[s], ph ^ 1, abort, status)) { ok = false; break; }
                     tc::mbar_expect_tx(&ctl->kv_full[s], 2 * TILE_BYTES);
-                    tc::tma_load_2d(smem + OFF_K + s * TILE_BYTES, &tm_qkv, C + h * HD, row_base + j * BKV,
+                    tc::tma_load_2d(smem + FW_OFF_K + s * TILE_BYTES, &tm_qkv, C + h * HD, row_base + j * BKV,
                                     &ctl->kv_full[s]);
-                    tc::tma_load_2d(smem + OFF_V + s * TILE_BYTES, &tm_qkv, 2 * C + h * HD, row_base + j * BKV,
+                    tc::tma_load_2d(smem + FW_OFF_V + s * TILE_BYTES, &tm_qkv, 2 * C + h * HD, row_base + j * BKV,
                                     &ctl->kv_full[s]);
                 }
+                ++ord;
             }
         }
     } else if (warp == 1) {
@@ -200,62 +227,90 @@ __global__ void __launch_bounds__(THREADS, 1)
             // --------------------------------------------------------------- MMA
             constexpr uint32_t idesc_s = tc::idesc_bf16_f32(BQ, BKV, 0, 0);
             constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(BQ, HD, 0, 1);
-            // tile cursor over (item, key tile) in the CTA's order
+            // an item in the CTA's order: round k, item ordinal, global index of its first key step
             struct Cur {
-                int i, j, n_kv;
-                uint32_t ord;
+                int k, i, ord, gs0;
+                FwItem it;
             };
-            auto start = [&](Cur& c, int i, uint32_t ord) {
-                c.i = i;
-                c.j = 0;
-                c.ord = ord;
-                c.n_kv = i < n_items ? fwd_item(i, BH, n_qt, Tn).n_kv : 0;
+            auto settle = [&](Cur c) {   // from round c.k on, the first round that has an item
+                while (c.k < n_rounds && fw_round_item(c.k, n_items) < 0) ++c.k;
+                c.i = c.k < n_rounds ? fw_round_item(c.k, n_items) : -1;
+                if (c.i >= 0) c.it = fw_item(c.i, BH, n_pairs, Tn);
+                return c;
             };
-            auto advance = [&](Cur c) {
+            auto next_item = [&](Cur c) {
                 Cur n = c;
-                if (++n.j == n.n_kv) start(n, c.i + (int)gridDim.x, c.ord + 1);
-                return n;
+                n.ord = c.ord + 1;
+                n.gs0 = c.gs0 + c.it.n_kv;
+                n.k = c.k + 1;
+                return settle(n);
             };
-            // S_g = Q K_g^T for the tile at cursor c (global tile index g)
-            auto issue_s = [&](const Cur& c, uint32_t g) -> bool {
-                const int s = g % KV_STAGES, sb = g & 1, qb = c.ord & 1;
-                if (c.j == 0 && !tc::mbar_wait(&ctl->q_full[qb], (c.ord >> 1) & 1, abort, status)) return false;
-                if (!tc::mbar_wait(&ctl->kv_full[s], (g / KV_STAGES) & 1, abort, status)) return false;
-                if (!tc::mbar_wait(&ctl->s_empty[sb], ((g >> 1) & 1) ^ 1, abort, status)) return false;
+            // next S tile to issue for a group: (item cursor, key tile j)
+            struct Tile {
+                Cur c;
+                int j;
+            };
+            auto group_first = [&](Cur c, int g) {   // group g's first tile at or after item c
+                while (c.i >= 0 && c.it.n[g] == 0) c = next_item(c);
+                return Tile{c, 0};
+            };
+            auto group_next = [&](Tile t, int g) {
+                if (t.j + 1 < t.c.it.n[g]) return Tile{t.c, t.j + 1};
+                return group_first(next_item(t.c), g);
+            };
+            // S_g = Q_g K^T for tile t of group g
+            auto issue_s = [&](const Tile& t, int g) -> bool {
+                const int gs = t.c.gs0 + t.j, s = gs % KV_STAGES, qs = t.c.ord & 1;
+                if (t.j == 0 && !tc::mbar_wait(&ctl->q_full[qs], (t.c.ord >> 1) & 1, abort, status)) return false;
+                if (!tc::mbar_wait(&ctl->kv_full[s], (gs / KV_STAGES) & 1, abort, status)) return false;
                 tc::fence_after_sync();
-                const uint32_t q_addr = tc::smem_u32(smem + OFF_Q + qb * TILE_BYTES);
-                const uint32_t k_addr = tc::smem_u32(smem + OFF_K + s * TILE_BYTES);
+                const uint32_t q_addr = tc::smem_u32(smem + FW_OFF_Q + (2 * qs + g) * TILE_BYTES);
+                const uint32_t k_addr = tc::smem_u32(smem + FW_OFF_K + s * TILE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk)
-                    tc::mma_bf16(tmem + (sb ? TM_S1 : TM_S0), tc::smem_desc_sw128(q_addr + kk * 32, 16, 1024),
+                    tc::mma_bf16(tmem + g * FT_GROUP + FT_S, tc::smem_desc_sw128(q_addr + kk * 32, 16, 1024),
                                  tc::smem_desc_sw128(k_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-                tc::mma_commit(&ctl->s_full[sb]);
-                if (c.j == c.n_kv - 1) tc::mma_commit(&ctl->q_empty[qb]);   // Q done once this S completes
+                tc::mma_commit(&ctl->s_full[g]);
                 return true;
             };
-            Cur cur;
-            start(cur, blockIdx.x, 0);
-            uint32_t g = 0;
-            bool ok = cur.i < n_items ? issue_s(cur, 0) : false;
-            while (ok && cur.i < n_items) {
-                const Cur nxt = advance(cur);
-                if (nxt.i < n_items && !issue_s(nxt, g + 1)) break;
-                const int s = g % KV_STAGES, pb = g & 1;
-                if (!tc::mbar_wait(&ctl->p_full[pb], (g >> 1) & 1, abort, status)) break;
-                if (!tc::mbar_wait(&ctl->pv_empty[pb], ((g >> 1) & 1) ^ 1, abort, status)) break;
-                tc::fence_after_sync();
-                const uint32_t p_addr = tc::smem_u32(smem + OFF_P + pb * P_BYTES);
-                const uint32_t v_addr = tc::smem_u32(smem + OFF_V + s * TILE_BYTES);
+            Cur c = settle(Cur{0, -1, 0, 0, FwItem{}});
+            Tile nt[2] = {group_first(c, 0), group_first(c, 1)};   // each group's next S to issue
+            uint32_t tp[2] = {0, 0};                                // PV MMAs issued per group
+            bool ok = true;
+            while (ok && c.i >= 0) {
+                for (int j = 0; j < c.it.n_kv && ok; ++j) {
+                    const int gs = c.gs0 + j, s = gs % KV_STAGES;
+                    // S of this step for a group whose S was not issued ahead
+                    for (int g = 0; g < 2 && ok; ++g)
+                        if (j < c.it.n[g] && nt[g].c.i >= 0 && nt[g].c.ord == c.ord && nt[g].j == j) {
+                            ok = issue_s(nt[g], g);
+                            nt[g] = group_next(nt[g], g);
+                        }
+                    for (int g = 0; g < 2 && ok; ++g) {
+                        if (j >= c.it.n[g]) continue;
+                        if (!tc::mbar_wait(&ctl->p_full[g], tp[g] & 1, abort, status)) { ok = false; break; }
+                        tc::fence_after_sync();
+                        const uint32_t v_addr = tc::smem_u32(smem + FW_OFF_V + s * TILE_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < BKV / 16; ++kk)
-                    tc::mma_bf16(tmem + (pb ? TM_PV1 : TM_PV0),
-                                 tc::smem_desc_sw128(p_addr + (kk >> 2) * TILE_BYTES + (kk & 3) * 32, 16, 1024),
-                                 tc::smem_desc_sw128(v_addr + kk * 2048, TILE_BYTES, 1024), idesc_pv,
-                                 kk > 0 ? 1u : 0u);
-                tc::mma_commit(&ctl->pv_full[pb]);
-                tc::mma_commit(&ctl->kv_empty[s]);
-                cur = nxt;
-                ++g;
+                        for (int kk = 0; kk < BKV / 16; ++kk)
+                            tc::mma_bf16_ts(tmem + g * FT_GROUP + FT_O, tmem + g * FT_GROUP + FT_P + kk * 8,
+                                            tc::smem_desc_sw128(v_addr + kk * 2048, TILE_BYTES, 1024), idesc_pv,
+                                            (j > 0 || kk > 0) ? 1u : 0u);
+                        tc::mma_commit(&ctl->pv_done[g]);
+                        ++tp[g];
+                        // the group's next S right away, when its K/V and Q are at most two steps
+                        // and one item ahead (so the producer can have them without further frees)
+                        const Tile& t = nt[g];
+                        if (t.c.i >= 0 && t.c.ord <= c.ord + 1 && t.c.gs0 + t.j <= gs + 2) {
+                            ok = issue_s(t, g);
+                            nt[g] = group_next(t, g);
+                        }
+                    }
+                    if (ok) tc::mma_commit(&ctl->kv_empty[s]);   // K and V of this step read by all its MMAs
+                }
+                if (!ok) break;
+                tc::mma_commit(&ctl->q_empty[c.ord & 1]);   // every S of the item issued
+                c = next_item(c);
             }
             volatile uint32_t no_abort = 0;
             tc::mma_commit(&ctl->drain);
@@ -263,147 +318,141 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else {
         // ---------------------------------------------------- softmax / output
-        // Warp pair (chalf 0/1) of a lane quarter shares 32 query rows: each warp
-        // owns 64 of the 128 keys of an S tile (one swizzle atom of P) and 32 of
-        // the 64 output columns. Only the row max is exchanged per tile.
+        const int g = (warp - 2) >> 2;
         const int quarter = warp & 3;
-        const int chalf = (warp - 2) >> 2;
         const int r = quarter * 32 + lane;            // query row within the tile = TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const uint32_t tS = tmem + g * FT_GROUP + FT_S + lane_off;
+        const uint32_t tP = tmem + g * FT_GROUP + FT_P + lane_off;
+        const uint32_t tO = tmem + g * FT_GROUP + FT_O + lane_off;
         const float sl2 = LOG2E * 0.125f;             // log2(e) / sqrt(64)
+        uint8_t* stage = smem + FW_OFF_ST + g * TILE_BYTES;
         bool ok = true;
-        uint32_t g = 0;                               // tile counter over all items
-        float o[32];
-        float corr_prev = 1.f;
-        auto consume_pv = [&](uint32_t gt) -> bool {
-            const int pb = gt & 1;
-            uint32_t w = 0;
-            if (lane == 0) w = tc::mbar_wait(&ctl->pv_full[pb], (gt >> 1) & 1, abort, status) ? 1u : 0u;
-            w = __shfl_sync(0xffffffffu, w, 0);
-            if (!w) return false;
-            tc::fence_after_sync();
-            float pv[32];
-            tc::tmem_ld_32x32b_x32(tmem + (pb ? TM_PV1 : TM_PV0) + chalf * 32 + lane_off, pv);
-            const f32x2 CP = pk2(corr_prev, corr_prev);
-#pragma unroll
-            for (int d = 0; d < 32; d += 2)
-                upk2(fma2(pk2(o[d], o[d + 1]), CP, pk2(pv[d], pv[d + 1])), o[d], o[d + 1]);
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&ctl->pv_empty[pb]);
-            return true;
-        };
-        // Every softmax warp passes the named barrier n_kv + 2 times per item, also
-        // after a failed wait (then without work), so none is left waiting there.
-        for (int i = blockIdx.x; i < n_items; i += gridDim.x) {
-            const FwdItem it = fwd_item(i, BH, n_qt, Tn);
-            const int q0 = it.q0, n_kv = it.n_kv;
+        uint32_t tg = 0;                              // this group's tiles so far
+        for (int k = 0; k < n_rounds && ok; ++k) {
+            const int i = fw_round_item(k, n_items);
+            if (i < 0) continue;
+            const FwItem it = fw_item(i, BH, n_pairs, Tn);
+            const int n = it.n[g];
+            if (n == 0) continue;
+            const int q0 = it.q0 + g * BQ;
             const int q = q0 + r;
-#pragma unroll
-            for (int d = 0; d < 32; ++d) o[d] = 0.f;
-            float m = -INFINITY, l = 0.f;
-            corr_prev = 1.f;
-            for (int j = 0; j < n_kv; ++j, ++g) {
-                const int sb = g & 1;
-                uint32_t w = 0;
-                if (lane == 0 && ok) w = tc::mbar_wait(&ctl->s_full[sb], (g >> 1) & 1, abort, status) ? 1u : 0u;
-                w = __shfl_sync(0xffffffffu, w, 0);
-                const uint32_t s_addr = tmem + (sb ? TM_S1 : TM_S0) + chalf * 64 + lane_off;
-                const int kbase = j * BKV + chalf * 64;   // first key of this warp's columns
-                const bool diag = (j * BKV + BKV > q0);
-                // pass 1: partial row max over this warp's 64 keys (one TMEM load), exchanged
-                // with the pair
+            float m = 0.f, l = 0.f;
+            for (int j = 0; j < n; ++j, ++tg) {
+                if (!warp_wait(&ctl->s_full[g], tg & 1, abort, status)) { ok = false; break; }
+                tc::fence_after_sync();
+                // pass 1: the row max over the tile's 128 keys, 64 columns at a time
+                const int kbase = j * BKV;
+                const bool diag = kbase + BKV > q0;   // keys after the query do not count
                 float mx = -INFINITY;
-                if (w) {
-                    tc::fence_after_sync();
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
                     float sv[64];
-                    tc::tmem_ld_32x32b_x64(s_addr, sv);
-                    if (diag) {   // keys after the query do not count
-#pragma unroll
-                        for (int e = 0; e < 64; ++e)
-                            if (kbase + e > q) sv[e] = -INFINITY;
-                    }
-                    mx = max32(sv + 32, max32(sv, mx));
-                }
-                ctl->mx[sb][chalf][r] = mx;
-                pair_bar(quarter);
-                if (!w) { ok = false; continue; }
-                mx = fmaxf(mx, ctl->mx[sb][chalf ^ 1][r]);
-                const float m_new = fmaxf(m, mx * sl2);
-                const float corr = ex2(m - m_new);   // m = -inf at an item's start: 0
-                // pass 2: P = exp2(s * sl2 - m_new) as bf16 into this warp's 64-key atom of P
-                uint8_t* pt = smem + OFF_P + sb * P_BYTES + chalf * TILE_BYTES;
-                // the exponent s * sl2 - m_new and the row sum on packed pairs
-                const f32x2 SL = pk2(sl2, sl2), NM = pk2(-m_new, -m_new);
-                f32x2 RS = pk2(0.f, 0.f);
-                {
-                    float sv[64];
-                    tc::tmem_ld_32x32b_x64(s_addr, sv);   // the 64 columns, one TMEM round trip
-#pragma unroll
-                    for (int e = 0; e < 64; e += 2) {
-                        float t0, t1;
-                        upk2(fma2(pk2(sv[e], sv[e + 1]), SL, NM), t0, t1);
-                        sv[e] = ex2(t0);
-                        sv[e + 1] = ex2(t1);
-                    }
+                    tc::tmem_ld_32x32b_x64(tS + 64 * hh, sv);
                     if (diag) {
 #pragma unroll
                         for (int e = 0; e < 64; ++e)
-                            if (kbase + e > q) sv[e] = 0.f;
+                            if (kbase + 64 * hh + e > q) sv[e] = -INFINITY;
+                    }
+                    mx = max32(sv + 32, max32(sv, mx));
+                }
+                const float mt = mx * sl2;
+                bool need = false;
+                if (j == 0) m = mt;   // the first tile's PV overwrites O
+                else need = mt > m + FW_RESCALE;
+                // P's TMEM columns and O: the group's previous O += P V must be done
+                if (tg > 0) {
+                    if (!warp_wait(&ctl->pv_done[g], (tg - 1) & 1, abort, status)) { ok = false; break; }
+                    tc::fence_after_sync();
+                }
+                if (__any_sync(0xffffffffu, need)) {
+                    const float cr = need ? ex2(m - mt) : 1.f;
+                    if (need) {
+                        m = mt;
+                        l *= cr;
+                    }
+#pragma unroll 1
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float o[32];
+                        uint32_t ow[16];
+                        tc::tmem_ld_32x32b_x32(tO + 32 * hh, o);
+#pragma unroll
+                        for (int hq = 0; hq < 2; ++hq) {
+#pragma unroll
+                            for (int d = 0; d < 16; ++d) ow[d] = __float_as_uint(o[16 * hq + d] * cr);
+                            tc::tmem_st_32x32b_x16(tO + 32 * hh + 16 * hq, ow);
+                        }
+                    }
+                }
+                // pass 2: P = 2^(s sl2 - m), 64 keys per load: row sum, bf16 pairs into TMEM
+                const f32x2 SL = pk2(sl2, sl2), NM = pk2(-m, -m);
+                f32x2 RS = pk2(0.f, 0.f);
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    float sv[64];
+                    tc::tmem_ld_32x32b_x64(tS + 64 * hh, sv);
+                    if (diag) {
+#pragma unroll
+                        for (int e = 0; e < 64; ++e)
+                            if (kbase + 64 * hh + e > q) sv[e] = -INFINITY;
                     }
 #pragma unroll
-                    for (int e = 0; e < 64; e += 2) RS = add2(RS, pk2(sv[e], sv[e + 1]));
+                    for (int cq = 0; cq < 2; ++cq) {
+                        float* v = sv + 32 * cq;
 #pragma unroll
-                    for (int gg = 0; gg < 8; ++gg)
-                        *reinterpret_cast<uint4*>(pt + swz128(r, gg)) = pack8_bf16(sv + 8 * gg);
+                        for (int e = 0; e < 32; e += 2) {
+                            float t0, t1;
+                            upk2(fma2(pk2(v[e], v[e + 1]), SL, NM), t0, t1);
+                            v[e] = ex2(t0);
+                            v[e + 1] = ex2(t1);
+                            RS = add2(RS, pk2(v[e], v[e + 1]));
+                        }
+                        uint32_t pw[16];
+#pragma unroll
+                        for (int gq = 0; gq < 4; ++gq) {
+                            const uint4 a = pack8_bf16(v + 8 * gq);
+                            pw[4 * gq] = a.x; pw[4 * gq + 1] = a.y; pw[4 * gq + 2] = a.z; pw[4 * gq + 3] = a.w;
+                        }
+                        tc::tmem_st_32x32b_x16(tP + 32 * hh + 16 * cq, pw);
+                    }
                 }
+                tc::tmem_wait_st();
                 float rs0, rs1;
                 upk2(RS, rs0, rs1);
-                const float rs = rs0 + rs1;
-                l = l * corr + rs;
-                m = m_new;
-                tc::fence_proxy_async_smem();      // P visible to the tensor core
+                l += rs0 + rs1;
                 tc::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) {
-                    tc::mbar_arrive(&ctl->p_full[sb]);
-                    tc::mbar_arrive(&ctl->s_empty[sb]);
-                }
-                if (j > 0 && !consume_pv(g - 1)) { ok = false; continue; }
-                corr_prev = corr;
+                if (lane == 0) tc::mbar_arrive(&ctl->p_full[g]);
             }
-            if (ok && n_kv > 0) ok = consume_pv(g - 1);
-            // row sum of both halves
-            ctl->lsum[chalf][r] = l;
-            ew_bar();
-            const float l_tot = l + ctl->lsum[chalf ^ 1][r];
-            // out rows: O / l, staged in the first 64-key atom of P buffer 0 (every PV MMA of
-            // this item has completed; only these warps write P, and only after this store)
-            uint8_t* stage = smem + OFF_P;
-            if (ok) {
-                const float inv = 1.f / l_tot;
+            if (!ok) break;
+            // the item's O is complete once the PV of its last tile is done
+            if (!warp_wait(&ctl->pv_done[g], (tg - 1) & 1, abort, status)) { ok = false; break; }
+            tc::fence_after_sync();
+            {
+                float o[64];
+                tc::tmem_ld_32x32b_x64(tO, o);
+                const float inv = 1.f / l;
 #pragma unroll
-                for (int gg = 0; gg < 4; ++gg) {
+                for (int gg = 0; gg < 8; ++gg) {
                     float t[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) t[e] = o[8 * gg + e] * inv;
-                    *reinterpret_cast<uint4*>(stage + swz128(r, chalf * 4 + gg)) = pack8_bf16(t);
+                    *reinterpret_cast<uint4*>(stage + swz128(r, gg)) = pack8_bf16(t);
                 }
-                if (chalf == 0 && q < Tn) lse[(long long)it.bh * Tn + q] = (m + log2f(l_tot)) / LOG2E;
             }
-            ew_bar();
-            if (ok && chalf == 0) {
-                const int b = it.bh / H, h = it.bh % H;
-                const int lrow = lane >> 3, lseg = lane & 7;
+            if (q < Tn) lse[(long long)it.bh * Tn + q] = (m + log2f(l)) / LOG2E;
+            __syncwarp();
+            // this warp's 32 rows out, 8 lanes per 128-byte row
+            const int b = it.bh / H, h = it.bh % H;
+            const int lrow = lane >> 3, lseg = lane & 7;
 #pragma unroll
-                for (int st = 0; st < 8; ++st) {
-                    const int rr = quarter * 32 + st * 4 + lrow;
-                    if (q0 + rr < Tn)
-                        *reinterpret_cast<uint4*>(out + ((long long)b * Tn + q0 + rr) * C + h * HD + lseg * 8) =
-                            *reinterpret_cast<const uint4*>(stage + swz128(rr, lseg));
-                }
-                __syncwarp();
+            for (int st = 0; st < 8; ++st) {
+                const int rr = quarter * 32 + st * 4 + lrow;
+                if (q0 + rr < Tn)
+                    *reinterpret_cast<uint4*>(out + ((long long)b * Tn + q0 + rr) * C + h * HD + lseg * 8) =
+                        *reinterpret_cast<const uint4*>(stage + swz128(rr, lseg));
             }
+            __syncwarp();
         }
     }
     tc::fence_before_sync();
@@ -426,6 +475,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 //     packed-bf16 A operand of dV += P^T dO, and dS^T, written to shared memory
 //     (128-byte swizzle, two 64-query atoms): K-major it is the A operand of
 //     dK += dS^T Q, MN-major the A operand of dQ = dS K;
+//   two MMA threads: one issues S^T, dP^T and dV += P^T dO, the other
+//     dK += dS^T Q and dQ = dS K, so that the tensor pipe is fed from two
+//     instruction streams (one thread issues at most about one M = 128
+//     instruction per 100 cycles, measured; two reach the shared-memory
+//     operand bandwidth);
 //   dV and dK accumulate in TMEM over the query tiles; the pair's dQ (M = 128
 //     queries, N = 64) goes to TMEM, and 4 drain warps scale it, stage it in
 //     shared memory and add it into an fp32 (B T, C) accumulator with the TMA
@@ -483,9 +537,10 @@ __device__ __forceinline__ void flush_rows_64(const uint8_t* stage, bf16* base, 
 
 constexpr int BW_EW_WARPS = 8;         // 2 per TMEM lane quarter, 64 query columns each (two chunks of 32)
 constexpr int BW_DR_WARPS = 4;         // dQ drain and dK/dV write-out: one per TMEM lane quarter
-constexpr int BW_THREADS = 64 + 32 * (BW_EW_WARPS + BW_DR_WARPS);
+constexpr int BW_MMA2_WARP = 2 + BW_EW_WARPS + BW_DR_WARPS;   // the second MMA thread's warp
+constexpr int BW_THREADS = 32 * (BW_MMA2_WARP + 1);
 constexpr int BW_STAGES = 3;           // Q/dO ring
-constexpr int BW_ITEM_READERS = 1 + BW_EW_WARPS + BW_DR_WARPS;   // MMA thread, element-wise and drain warps
+constexpr int BW_ITEM_READERS = 2 + BW_EW_WARPS + BW_DR_WARPS;   // both MMA threads, element-wise and drain warps
 struct CtlBwd {
     uint64_t item_full[2], item_empty[2];            // work-item ring, filled by the producer warp
     uint64_t kv_full[2], kv_empty[2];                // K and V of the item in ring slot s
@@ -496,7 +551,7 @@ struct CtlBwd {
     uint64_t ds_free;                                // a pair's dK, dQ MMAs done: dS^T reusable
     uint64_t dq_full, dq_empty;                      // a pair's dQ in TMEM: computed / copied to registers
     uint64_t acc_done, dkv_free;                     // an item's dK, dV complete in TMEM / copied out
-    uint64_t drain;
+    uint64_t drain, drain2;
     uint32_t tmem_base;
     uint32_t abort;
     int item[2];
@@ -569,11 +624,11 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             tc::mbar_init(&ctl->item_full[i], 1);
             tc::mbar_init(&ctl->item_empty[i], BW_ITEM_READERS);
             tc::mbar_init(&ctl->kv_full[i], 1);
-            tc::mbar_init(&ctl->kv_empty[i], 1);
+            tc::mbar_init(&ctl->kv_empty[i], 2);   // both MMA threads
         }
         for (int s = 0; s < BW_STAGES; ++s) {
             tc::mbar_init(&ctl->q_full[s], 2);   // the TMA bytes, and the producer's lse / D stores
-            tc::mbar_init(&ctl->q_empty[s], 1);
+            tc::mbar_init(&ctl->q_empty[s], 2);  // both MMA threads
         }
         tc::mbar_init(&ctl->st_full, 1);
         tc::mbar_init(&ctl->st_empty, BW_EW_WARPS);
@@ -582,9 +637,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         tc::mbar_init(&ctl->ds_free, 1);
         tc::mbar_init(&ctl->dq_full, 1);
         tc::mbar_init(&ctl->dq_empty, BW_DR_WARPS);
-        tc::mbar_init(&ctl->acc_done, 1);
+        tc::mbar_init(&ctl->acc_done, 2);   // dV (first MMA thread), dK (second)
         tc::mbar_init(&ctl->dkv_free, BW_DR_WARPS);
         tc::mbar_init(&ctl->drain, 1);
+        tc::mbar_init(&ctl->drain2, 1);
         ctl->abort = 0;
         tc::fence_barrier_init();
     }
@@ -682,19 +738,13 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            // ------------------------------------------------------------------- MMA
+            // --------------------------------------- first MMA thread: S^T, dP^T, dV
             constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128, 0, 0);   // K Q^T, V dO^T
-            constexpr uint32_t idesc_acc = tc::idesc_bf16_f32(128, 64, 0, 1);  // P^T dO, dS^T Q
-            constexpr uint32_t idesc_dq = tc::idesc_bf16_f32(128, 64, 1, 1);   // dS K (dS from the dS^T tile)
+            constexpr uint32_t idesc_acc = tc::idesc_bf16_f32(128, 64, 0, 1);  // P^T dO
             // Shared-memory descriptors, built once: the start address sits in the low bits
             // (address >> 4), so stepping inside a tile adds (byte offset >> 4).
             const uint32_t kv0 = tc::smem_u32(smem + BW_OFF_KV), q_base = tc::smem_u32(smem + BW_OFF_Q);
-            const uint64_t d_ds_k = tc::smem_desc_sw128(tc::smem_u32(smem + BW_OFF_DS), 16, 1024);
-            const uint64_t d_ds_mn = tc::smem_desc_sw128(tc::smem_u32(smem + BW_OFF_DS), T128_BYTES, 1024);
             auto kdesc_k = [&](int slot) { return tc::smem_desc_sw128(kv0 + slot * BW_KV_BYTES, 16, 1024); };
-            auto kdesc_mn = [&](int slot) {
-                return tc::smem_desc_sw128(kv0 + slot * BW_KV_BYTES, T128_BYTES, 1024);
-            };
             auto qdesc_k = [&](int st) { return tc::smem_desc_sw128(q_base + st * BW_STAGE_BYTES, 16, 1024); };
             auto qdesc_mn = [&](int st) {
                 return tc::smem_desc_sw128(q_base + st * BW_STAGE_BYTES, T128_BYTES, 1024);
@@ -743,38 +793,19 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 if (!tc::mbar_wait(&ctl->ew_done, par, abort, status)) break;
                 tc::fence_after_sync();
                 const uint64_t dmn = qdesc_mn(st);
-                const uint64_t kmn = kdesc_mn(slot);
-                // dQ = dS K: K = 128 keys in steps of 16; A is the dS^T tile read as an MN-major
-                // (query-contiguous) operand, the next 64 queries one atom (16 KB) further
-                auto issue_dq = [&]() -> bool {
-                    if (!tc::mbar_wait(&ctl->dq_empty, par ^ 1, abort, status)) return false;
-                    tc::fence_after_sync();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_bf16(tmem + BW_DQ, d_ds_mn + 128 * kk, kmn + 128 * kk, idesc_dq, kk > 0 ? 1u : 0u);
-                    tc::mma_commit(&ctl->dq_full);
-                    return true;
-                };
-                // The first pair of an item overwrites dV / dK, so it waits for the last item's
-                // to be copied out; its dQ, which needs neither, goes first.
+                // The first pair of an item overwrites dV, so it waits for the last item's to be
+                // copied out.
                 if (it == 0) {
-                    if (!issue_dq()) break;
                     if (!tc::mbar_wait(&ctl->dkv_free, (ictr & 1) ^ 1, abort, status)) break;
                     tc::fence_after_sync();
                 }
-                // dV += P^T dO, then dK += dS^T Q: K = 128 queries in steps of 16
+                // dV += P^T dO: K = 128 queries in steps of 16
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_bf16_ts(tmem + BW_DV, tmem + BW_PT + kk * 8, dmn + TILE16 + 128 * kk, idesc_acc,
                                     (it > 0 || kk > 0) ? 1u : 0u);
                 tc::mma_commit(&ctl->pt_free);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_bf16(tmem + BW_DK, d_ds_k + (kk >> 2) * TILE16 + 2 * (kk & 3), dmn + 128 * kk, idesc_acc,
-                                 (it > 0 || kk > 0) ? 1u : 0u);
                 tc::mma_commit(&ctl->q_empty[st]);
-                if (it > 0 && !issue_dq()) break;
-                tc::mma_commit(&ctl->ds_free);
                 if (it + 1 == cur.n_it) {
                     tc::mma_commit(&ctl->kv_empty[slot]);
                     tc::mma_commit(&ctl->acc_done);
@@ -902,6 +933,83 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 if (item >= 0) cur = bw_item(item, BH, n_qt);
                 it = 0;
             }
+        }
+    } else if (warp == BW_MMA2_WARP) {
+        if (lane == 0) {
+            // ------------------------------------------------ second MMA thread: dK, dQ
+            // It follows the same pairs: once the element-wise warps have written dS^T,
+            // dK += dS^T Q and dQ = dS K, while the first MMA thread issues dV and the next
+            // pair's S^T / dP^T. Both feed the tensor pipe, whose single-issuer rate
+            // (about one M = 128 instruction per 100 cycles) would otherwise bound the pair.
+            constexpr uint32_t idesc_acc = tc::idesc_bf16_f32(128, 64, 0, 1);  // dS^T Q
+            constexpr uint32_t idesc_dq = tc::idesc_bf16_f32(128, 64, 1, 1);   // dS K (dS from the dS^T tile)
+            constexpr uint64_t TILE16 = T128_BYTES >> 4;
+            const uint32_t kv0 = tc::smem_u32(smem + BW_OFF_KV), q_base = tc::smem_u32(smem + BW_OFF_Q);
+            const uint64_t d_ds_k = tc::smem_desc_sw128(tc::smem_u32(smem + BW_OFF_DS), 16, 1024);
+            const uint64_t d_ds_mn = tc::smem_desc_sw128(tc::smem_u32(smem + BW_OFF_DS), T128_BYTES, 1024);
+            uint32_t ictr = 0, g = 0;
+            int item = bw_read_item(ctl, ictr, abort, status);
+            bool ok = item >= 0;
+            while (ok) {
+                const BwItem cur = bw_item(item, BH, n_qt);
+                const int slot = ictr & 1;
+                const uint64_t kmn = tc::smem_desc_sw128(kv0 + slot * BW_KV_BYTES, T128_BYTES, 1024);
+                // K of this item (dQ reads it; the first MMA thread waited for it already)
+                if (!tc::mbar_wait(&ctl->kv_full[slot], (ictr >> 1) & 1, abort, status)) break;
+                for (int it = 0; it < cur.n_it && ok; ++it, ++g) {
+                    const int st = g % BW_STAGES;
+                    const uint32_t par = g & 1;
+                    // after the pair's dV: the next pair's P^T waits for dV, its dS^T (written
+                    // later) for dK and dQ, so dV goes through the tensor pipe first
+                    if (!tc::mbar_wait(&ctl->q_full[st], (g / BW_STAGES) & 1, abort, status) ||
+                        !tc::mbar_wait(&ctl->ew_done, par, abort, status) ||
+                        !tc::mbar_wait(&ctl->pt_free, par, abort, status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                    const uint64_t dmn = tc::smem_desc_sw128(q_base + st * BW_STAGE_BYTES, T128_BYTES, 1024);
+                    // dQ = dS K: K = 128 keys in steps of 16; A is the dS^T tile read as an MN-major
+                    // (query-contiguous) operand, the next 64 queries one atom (16 KB) further
+                    auto issue_dq = [&]() -> bool {
+                        if (!tc::mbar_wait(&ctl->dq_empty, par ^ 1, abort, status)) return false;
+                        tc::fence_after_sync();
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            tc::mma_bf16(tmem + BW_DQ, d_ds_mn + 128 * kk, kmn + 128 * kk, idesc_dq,
+                                         kk > 0 ? 1u : 0u);
+                        tc::mma_commit(&ctl->dq_full);
+                        return true;
+                    };
+                    // The first pair of an item overwrites dK, so it waits for the last item's to
+                    // be copied out; its dQ, which needs neither, goes first.
+                    if (it == 0) {
+                        if (!issue_dq() || !tc::mbar_wait(&ctl->dkv_free, (ictr & 1) ^ 1, abort, status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after_sync();
+                    }
+                    // dK += dS^T Q: K = 128 queries in steps of 16
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_bf16(tmem + BW_DK, d_ds_k + (kk >> 2) * TILE16 + 2 * (kk & 3), dmn + 128 * kk,
+                                     idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
+                    tc::mma_commit(&ctl->q_empty[st]);
+                    if (it > 0 && !issue_dq()) { ok = false; break; }
+                    tc::mma_commit(&ctl->ds_free);
+                    if (it + 1 == cur.n_it) {
+                        tc::mma_commit(&ctl->kv_empty[slot]);
+                        tc::mma_commit(&ctl->acc_done);
+                    }
+                }
+                if (!ok) break;
+                item = bw_read_item(ctl, ++ictr, abort, status);
+                ok = item >= 0;
+            }
+            volatile uint32_t no_abort = 0;
+            tc::mma_commit(&ctl->drain2);
+            tc::mbar_wait(&ctl->drain2, 0, &no_abort, status);
         }
     } else {
         // ------------------------------- dQ drain, dK / dV write-out (thread = row)
@@ -1095,12 +1203,12 @@ bool launch_attention_fwd_tc(const Ctx& ctx, const bf16* qkv, bf16* out, float* 
         return false;
     static bool configured = false;
     if (!configured) {
-        cudaFuncSetAttribute(flash_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        cudaFuncSetAttribute(flash_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FW_SMEM);
         configured = true;
     }
-    const int n_items = B * H * ceil_div(Tn, BQ);
+    const int n_items = B * H * ((ceil_div(Tn, BQ) + 1) / 2);   // query-tile pairs
     const int grid = min(n_items, ctx.num_sms > 0 ? ctx.num_sms : 148);
-    flash_fwd_tc_kernel<<<grid, THREADS, SMEM_BYTES, ctx.stream>>>(m, out, lse, Tn, H, B * H, ctx.status);
+    flash_fwd_tc_kernel<<<grid, FW_THREADS, FW_SMEM, ctx.stream>>>(m, out, lse, Tn, H, B * H, ctx.status);
     ++*ctx.launches;
     return true;
 }
