@@ -475,11 +475,6 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
 //     packed-bf16 A operand of dV += P^T dO, and dS^T, written to shared memory
 //     (128-byte swizzle, two 64-query atoms): K-major it is the A operand of
 //     dK += dS^T Q, MN-major the A operand of dQ = dS K;
-//   two MMA threads: one issues S^T, dP^T and dV += P^T dO, the other
-//     dK += dS^T Q and dQ = dS K, so that the tensor pipe is fed from two
-//     instruction streams (one thread issues at most about one M = 128
-//     instruction per 100 cycles, measured; two reach the shared-memory
-//     operand bandwidth);
 //   dV and dK accumulate in TMEM over the query tiles; the pair's dQ (M = 128
 //     queries, N = 64) goes to TMEM, and 4 drain warps scale it, stage it in
 //     shared memory and add it into an fp32 (B T, C) accumulator with the TMA
@@ -537,10 +532,9 @@ __device__ __forceinline__ void flush_rows_64(const uint8_t* stage, bf16* base, 
 
 constexpr int BW_EW_WARPS = 8;         // 2 per TMEM lane quarter, 64 query columns each (two chunks of 32)
 constexpr int BW_DR_WARPS = 4;         // dQ drain and dK/dV write-out: one per TMEM lane quarter
-constexpr int BW_MMA2_WARP = 2 + BW_EW_WARPS + BW_DR_WARPS;   // the second MMA thread's warp
-constexpr int BW_THREADS = 32 * (BW_MMA2_WARP + 1);
+constexpr int BW_THREADS = 64 + 32 * (BW_EW_WARPS + BW_DR_WARPS);
 constexpr int BW_STAGES = 3;           // Q/dO ring
-constexpr int BW_ITEM_READERS = 2 + BW_EW_WARPS + BW_DR_WARPS;   // both MMA threads, element-wise and drain warps
+constexpr int BW_ITEM_READERS = 1 + BW_EW_WARPS + BW_DR_WARPS;   // MMA thread, element-wise and drain warps
 struct CtlBwd {
     uint64_t item_full[2], item_empty[2];            // work-item ring, filled by the producer warp
     uint64_t kv_full[2], kv_empty[2];                // K and V of the item in ring slot s
@@ -551,7 +545,7 @@ struct CtlBwd {
     uint64_t ds_free;                                // a pair's dK, dQ MMAs done: dS^T reusable
     uint64_t dq_full, dq_empty;                      // a pair's dQ in TMEM: computed / copied to registers
     uint64_t acc_done, dkv_free;                     // an item's dK, dV complete in TMEM / copied out
-    uint64_t drain, drain2;
+    uint64_t drain;
     uint32_t tmem_base;
     uint32_t abort;
     int item[2];
@@ -624,11 +618,11 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             tc::mbar_init(&ctl->item_full[i], 1);
             tc::mbar_init(&ctl->item_empty[i], BW_ITEM_READERS);
             tc::mbar_init(&ctl->kv_full[i], 1);
-            tc::mbar_init(&ctl->kv_empty[i], 2);   // both MMA threads
+            tc::mbar_init(&ctl->kv_empty[i], 1);
         }
         for (int s = 0; s < BW_STAGES; ++s) {
             tc::mbar_init(&ctl->q_full[s], 2);   // the TMA bytes, and the producer's lse / D stores
-            tc::mbar_init(&ctl->q_empty[s], 2);  // both MMA threads
+            tc::mbar_init(&ctl->q_empty[s], 1);
         }
         tc::mbar_init(&ctl->st_full, 1);
         tc::mbar_init(&ctl->st_empty, BW_EW_WARPS);
@@ -637,10 +631,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         tc::mbar_init(&ctl->ds_free, 1);
         tc::mbar_init(&ctl->dq_full, 1);
         tc::mbar_init(&ctl->dq_empty, BW_DR_WARPS);
-        tc::mbar_init(&ctl->acc_done, 2);   // dV (first MMA thread), dK (second)
+        tc::mbar_init(&ctl->acc_done, 1);
         tc::mbar_init(&ctl->dkv_free, BW_DR_WARPS);
         tc::mbar_init(&ctl->drain, 1);
-        tc::mbar_init(&ctl->drain2, 1);
         ctl->abort = 0;
         tc::fence_barrier_init();
     }
@@ -738,13 +731,19 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            // --------------------------------------- first MMA thread: S^T, dP^T, dV
+            // ------------------------------------------------------------------- MMA
             constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128, 0, 0);   // K Q^T, V dO^T
-            constexpr uint32_t idesc_acc = tc::idesc_bf16_f32(128, 64, 0, 1);  // P^T dO
+            constexpr uint32_t idesc_acc = tc::idesc_bf16_f32(128, 64, 0, 1);  // P^T dO, dS^T Q
+            constexpr uint32_t idesc_dq = tc::idesc_bf16_f32(128, 64, 1, 1);   // dS K (dS from the dS^T tile)
             // Shared-memory descriptors, built once: the start address sits in the low bits
             // (address >> 4), so stepping inside a tile adds (byte offset >> 4).
             const uint32_t kv0 = tc::smem_u32(smem + BW_OFF_KV), q_base = tc::smem_u32(smem + BW_OFF_Q);
+            const uint64_t d_ds_k = tc::smem_desc_sw128(tc::smem_u32(smem + BW_OFF_DS), 16, 1024);
+            const uint64_t d_ds_mn = tc::smem_desc_sw128(tc::smem_u32(smem + BW_OFF_DS), T128_BYTES, 1024);
             auto kdesc_k = [&](int slot) { return tc::smem_desc_sw128(kv0 + slot * BW_KV_BYTES, 16, 1024); };
+            auto kdesc_mn = [&](int slot) {
+                return tc::smem_desc_sw128(kv0 + slot * BW_KV_BYTES, T128_BYTES, 1024);
+            };
             auto qdesc_k = [&](int st) { return tc::smem_desc_sw128(q_base + st * BW_STAGE_BYTES, 16, 1024); };
             auto qdesc_mn = [&](int st) {
                 return tc::smem_desc_sw128(q_base + st * BW_STAGE_BYTES, T128_BYTES, 1024);
@@ -793,19 +792,38 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 if (!tc::mbar_wait(&ctl->ew_done, par, abort, status)) break;
                 tc::fence_after_sync();
                 const uint64_t dmn = qdesc_mn(st);
-                // The first pair of an item overwrites dV, so it waits for the last item's to be
-                // copied out.
+                const uint64_t kmn = kdesc_mn(slot);
+                // dQ = dS K: K = 128 keys in steps of 16; A is the dS^T tile read as an MN-major
+                // (query-contiguous) operand, the next 64 queries one atom (16 KB) further
+                auto issue_dq = [&]() -> bool {
+                    if (!tc::mbar_wait(&ctl->dq_empty, par ^ 1, abort, status)) return false;
+                    tc::fence_after_sync();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_bf16(tmem + BW_DQ, d_ds_mn + 128 * kk, kmn + 128 * kk, idesc_dq, kk > 0 ? 1u : 0u);
+                    tc::mma_commit(&ctl->dq_full);
+                    return true;
+                };
+                // The first pair of an item overwrites dV / dK, so it waits for the last item's
+                // to be copied out; its dQ, which needs neither, goes first.
                 if (it == 0) {
+                    if (!issue_dq()) break;
                     if (!tc::mbar_wait(&ctl->dkv_free, (ictr & 1) ^ 1, abort, status)) break;
                     tc::fence_after_sync();
                 }
-                // dV += P^T dO: K = 128 queries in steps of 16
+                // dV += P^T dO, then dK += dS^T Q: K = 128 queries in steps of 16
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_bf16_ts(tmem + BW_DV, tmem + BW_PT + kk * 8, dmn + TILE16 + 128 * kk, idesc_acc,
                                     (it > 0 || kk > 0) ? 1u : 0u);
                 tc::mma_commit(&ctl->pt_free);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16(tmem + BW_DK, d_ds_k + (kk >> 2) * TILE16 + 2 * (kk & 3), dmn + 128 * kk, idesc_acc,
+                                 (it > 0 || kk > 0) ? 1u : 0u);
                 tc::mma_commit(&ctl->q_empty[st]);
+                if (it > 0 && !issue_dq()) break;
+                tc::mma_commit(&ctl->ds_free);
                 if (it + 1 == cur.n_it) {
                     tc::mma_commit(&ctl->kv_empty[slot]);
                     tc::mma_commit(&ctl->acc_done);
@@ -933,83 +951,6 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 if (item >= 0) cur = bw_item(item, BH, n_qt);
                 it = 0;
             }
-        }
-    } else if (warp == BW_MMA2_WARP) {
-        if (lane == 0) {
-            // ------------------------------------------------ second MMA thread: dK, dQ
-            // It follows the same pairs: once the element-wise warps have written dS^T,
-            // dK += dS^T Q and dQ = dS K, while the first MMA thread issues dV and the next
-            // pair's S^T / dP^T. Both feed the tensor pipe, whose single-issuer rate
-            // (about one M = 128 instruction per 100 cycles) would otherwise bound the pair.
-            constexpr uint32_t idesc_acc = tc::idesc_bf16_f32(128, 64, 0, 1);  // dS^T Q
-            constexpr uint32_t idesc_dq = tc::idesc_bf16_f32(128, 64, 1, 1);   // dS K (dS from the dS^T tile)
-            constexpr uint64_t TILE16 = T128_BYTES >> 4;
-            const uint32_t kv0 = tc::smem_u32(smem + BW_OFF_KV), q_base = tc::smem_u32(smem + BW_OFF_Q);
-            const uint64_t d_ds_k = tc::smem_desc_sw128(tc::smem_u32(smem + BW_OFF_DS), 16, 1024);
-            const uint64_t d_ds_mn = tc::smem_desc_sw128(tc::smem_u32(smem + BW_OFF_DS), T128_BYTES, 1024);
-            uint32_t ictr = 0, g = 0;
-            int item = bw_read_item(ctl, ictr, abort, status);
-            bool ok = item >= 0;
-            while (ok) {
-                const BwItem cur = bw_item(item, BH, n_qt);
-                const int slot = ictr & 1;
-                const uint64_t kmn = tc::smem_desc_sw128(kv0 + slot * BW_KV_BYTES, T128_BYTES, 1024);
-                // K of this item (dQ reads it; the first MMA thread waited for it already)
-                if (!tc::mbar_wait(&ctl->kv_full[slot], (ictr >> 1) & 1, abort, status)) break;
-                for (int it = 0; it < cur.n_it && ok; ++it, ++g) {
-                    const int st = g % BW_STAGES;
-                    const uint32_t par = g & 1;
-                    // after the pair's dV: the next pair's P^T waits for dV, its dS^T (written
-                    // later) for dK and dQ, so dV goes through the tensor pipe first
-                    if (!tc::mbar_wait(&ctl->q_full[st], (g / BW_STAGES) & 1, abort, status) ||
-                        !tc::mbar_wait(&ctl->ew_done, par, abort, status) ||
-                        !tc::mbar_wait(&ctl->pt_free, par, abort, status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc::fence_after_sync();
-                    const uint64_t dmn = tc::smem_desc_sw128(q_base + st * BW_STAGE_BYTES, T128_BYTES, 1024);
-                    // dQ = dS K: K = 128 keys in steps of 16; A is the dS^T tile read as an MN-major
-                    // (query-contiguous) operand, the next 64 queries one atom (16 KB) further
-                    auto issue_dq = [&]() -> bool {
-                        if (!tc::mbar_wait(&ctl->dq_empty, par ^ 1, abort, status)) return false;
-                        tc::fence_after_sync();
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            tc::mma_bf16(tmem + BW_DQ, d_ds_mn + 128 * kk, kmn + 128 * kk, idesc_dq,
-                                         kk > 0 ? 1u : 0u);
-                        tc::mma_commit(&ctl->dq_full);
-                        return true;
-                    };
-                    // The first pair of an item overwrites dK, so it waits for the last item's to
-                    // be copied out; its dQ, which needs neither, goes first.
-                    if (it == 0) {
-                        if (!issue_dq() || !tc::mbar_wait(&ctl->dkv_free, (ictr & 1) ^ 1, abort, status)) {
-                            ok = false;
-                            break;
-                        }
-                        tc::fence_after_sync();
-                    }
-                    // dK += dS^T Q: K = 128 queries in steps of 16
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_bf16(tmem + BW_DK, d_ds_k + (kk >> 2) * TILE16 + 2 * (kk & 3), dmn + 128 * kk,
-                                     idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
-                    tc::mma_commit(&ctl->q_empty[st]);
-                    if (it > 0 && !issue_dq()) { ok = false; break; }
-                    tc::mma_commit(&ctl->ds_free);
-                    if (it + 1 == cur.n_it) {
-                        tc::mma_commit(&ctl->kv_empty[slot]);
-                        tc::mma_commit(&ctl->acc_done);
-                    }
-                }
-                if (!ok) break;
-                item = bw_read_item(ctl, ++ictr, abort, status);
-                ok = item >= 0;
-            }
-            volatile uint32_t no_abort = 0;
-            tc::mma_commit(&ctl->drain2);
-            tc::mbar_wait(&ctl->drain2, 0, &no_abort, status);
         }
     } else {
         // ------------------------------- dQ drain, dK / dV write-out (thread = row)
