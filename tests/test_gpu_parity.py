@@ -67,7 +67,7 @@ def _check_params_fp32(s, p_gpu, p_ref, g_gpu, g_ref, tol=1e-5):
 
 
 # ----------------------------------------------------------------------------
-# fp32 mode, tiny config: the BASELINE parity case.
+# fp32 mode, tiny config (2 layers, C = 128, V = 1024): the small parity case.
 # ----------------------------------------------------------------------------
 @pytest.mark.parametrize("kind", ["init", "random"])
 def test_tiny_fp32_step_matches_oracle(kind):
