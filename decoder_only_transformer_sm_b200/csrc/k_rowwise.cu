@@ -206,7 +206,10 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 constexpr int LNB_RING_BLOCKS = 148;   // one block per SM of a B200; a fixed count keeps the sum order fixed
-template <typename T, int NV>
+// RING slots per warp (RING - 1 rows in flight ahead of the one processed). The
+// column partial sums stay in registers (each lane owns its columns) and meet in
+// shared memory, reusing the ring, once the block's rows are done.
+template <typename T, int NV, int RING>
 __global__ void __launch_bounds__(32 * LNB_WARPS, 1)
     ln_bwd_ring_kernel(const T* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ mean,
                        const float* __restrict__ rstd, const float* __restrict__ w, const float* dres_in,
@@ -215,16 +218,15 @@ __global__ void __launch_bounds__(32 * LNB_WARPS, 1)
     extern __shared__ float4 smem4[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int C4 = C >> 2;
-    float4* acc4 = smem4;                              // [LNB_WARPS][3][C / 4]
-    float4* mine = acc4 + warp * 3 * C4;
     const size_t row_bytes = (size_t)C * (sizeof(T) + 8);   // dy | x | dres_in
-    uint8_t* ring = reinterpret_cast<uint8_t*>(smem4 + LNB_WARPS * 3 * C4) + (size_t)warp * 2 * row_bytes;
-    for (int i = lane; i < 3 * C4; i += 32) mine[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    float ww[NV][4];
+    uint8_t* ring = reinterpret_cast<uint8_t*>(smem4) + (size_t)warp * RING * row_bytes;
+    float ww[NV][4], aw[NV][4], ab[NV][4], an[NV][4];
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
         const int c4 = lane + 32 * i;
         if (c4 < C4) load4(w + 4 * c4, ww[i]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) aw[i][j] = ab[i][j] = an[i][j] = 0.f;
     }
     auto issue = [&](int row, int slot) {
         uint8_t* b = ring + slot * row_bytes;
@@ -246,13 +248,18 @@ __global__ void __launch_bounds__(32 * LNB_WARPS, 1)
     };
     const int r0 = blockIdx.x * rows_per_block;
     const int r1 = min(rows, r0 + rows_per_block);
-    if (r0 + warp < r1) issue(r0 + warp, 0);
+#pragma unroll
+    for (int k = 0; k < RING - 1; ++k)
+        if (r0 + warp + k * LNB_WARPS < r1) issue(r0 + warp + k * LNB_WARPS, k);
     int slot = 0;
-    for (int row = r0 + warp; row < r1; row += LNB_WARPS, slot ^= 1) {
-        const int nxt = row + LNB_WARPS;
+    for (int row = r0 + warp; row < r1; row += LNB_WARPS, slot = (slot + 1 == RING) ? 0 : slot + 1) {
         const float mu = mean[row], rs = rstd[row];
-        if (nxt < r1) {
-            issue(nxt, slot ^ 1);
+        // the row RING - 1 ahead into the slot processed last; then wait for this row's copies
+        const int ahead = row + (RING - 1) * LNB_WARPS;
+        if (ahead < r1) {
+            issue(ahead, slot == 0 ? RING - 1 : slot - 1);
+            cp_async_wait_group<RING - 1>();
+        } else if (RING == 3 && row + LNB_WARPS < r1) {
             cp_async_wait_group<1>();
         } else {
             cp_async_wait_group<0>();
@@ -270,18 +277,15 @@ __global__ void __launch_bounds__(32 * LNB_WARPS, 1)
                 float g[4], xx[4];
                 load4(sdy + 4 * c4, g);
                 load4(sx + 4 * c4, xx);
-                float4 aw = mine[c4], ab = mine[C4 + c4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     xh[i][j] = (xx[j] - mu) * rs;
                     dxh[i][j] = g[j] * ww[i][j];
                     s1 += dxh[i][j];
                     s2 += dxh[i][j] * xh[i][j];
+                    aw[i][j] += g[j] * xh[i][j];
+                    ab[i][j] += g[j];
                 }
-                aw.x += g[0] * xh[i][0]; aw.y += g[1] * xh[i][1]; aw.z += g[2] * xh[i][2]; aw.w += g[3] * xh[i][3];
-                ab.x += g[0]; ab.y += g[1]; ab.z += g[2]; ab.w += g[3];
-                mine[c4] = aw;
-                mine[C4 + c4] = ab;
             }
         }
         s1 = warp_sum(s1) / C;
@@ -298,11 +302,22 @@ __global__ void __launch_bounds__(32 * LNB_WARPS, 1)
                 store4(dres_out + (long long)row * C + c, o);
                 if (dres_act) store4(dres_act + (long long)row * C + c, o);
                 if (want_dx_sum) {
-                    float4 an = mine[2 * C4 + c4];
-                    an.x += o[0]; an.y += o[1]; an.z += o[2]; an.w += o[3];
-                    mine[2 * C4 + c4] = an;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) an[i][j] += o[j];
                 }
             }
+        }
+    }
+    __syncthreads();   // every warp is past its ring: the shared memory now holds the partial rows
+    float4* acc4 = smem4;   // [LNB_WARPS][3][C / 4]
+    float4* mine = acc4 + warp * 3 * C4;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c4 = lane + 32 * i;
+        if (c4 < C4) {
+            mine[c4] = make_float4(aw[i][0], aw[i][1], aw[i][2], aw[i][3]);
+            mine[C4 + c4] = make_float4(ab[i][0], ab[i][1], ab[i][2], ab[i][3]);
+            mine[2 * C4 + c4] = make_float4(an[i][0], an[i][1], an[i][2], an[i][3]);
         }
     }
     __syncthreads();
@@ -911,7 +926,12 @@ void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const flo
                           float* db, float* dbias_next, int rows, int C, float* scratch) {
     const int nv = ceil_div(C, 128);
     const int want = dbias_next != nullptr;
-    const size_t ring_smem = (size_t)LNB_WARPS * (3 * C * sizeof(float) + 2 * C * (sizeof(T) + 8));
+    // shared memory: the ring (RING rows per warp), reused for the partial rows at the end
+    const size_t row_bytes = (size_t)C * (sizeof(T) + 8), parts = (size_t)LNB_WARPS * 3 * C * sizeof(float);
+    const size_t ring3 = std::max((size_t)LNB_WARPS * 3 * row_bytes, parts);
+    const size_t ring2 = std::max((size_t)LNB_WARPS * 2 * row_bytes, parts);
+    const int ring = ring3 <= 220 * 1024 ? 3 : 2;
+    const size_t ring_smem = ring == 3 ? ring3 : ring2;
     if (ring_smem <= 220 * 1024 && nv <= 8) {
         const int nblk = min(ceil_div(rows, LNB_WARPS), LNB_RING_BLOCKS);
         const int rpb = ceil_div(rows, nblk);
@@ -919,12 +939,18 @@ void launch_layernorm_bwd(const Ctx& ctx, const T* dy, const float* x, const flo
     case N: {                                                                                               \
         static bool configured = false;                                                                     \
         if (!configured) {                                                                                  \
-            cudaFuncSetAttribute(ln_bwd_ring_kernel<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,     \
+            cudaFuncSetAttribute(ln_bwd_ring_kernel<T, N, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                                 220 * 1024);                                                               \
+            cudaFuncSetAttribute(ln_bwd_ring_kernel<T, N, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
                                  220 * 1024);                                                               \
             configured = true;                                                                              \
         }                                                                                                   \
-        ln_bwd_ring_kernel<T, N><<<nblk, 32 * LNB_WARPS, ring_smem, ctx.stream>>>(                          \
-            dy, x, mean, rstd, w, dres_in, dres_out, dres_act, rows, C, rpb, want, scratch);                \
+        if (ring == 3)                                                                                      \
+            ln_bwd_ring_kernel<T, N, 3><<<nblk, 32 * LNB_WARPS, ring_smem, ctx.stream>>>(                   \
+                dy, x, mean, rstd, w, dres_in, dres_out, dres_act, rows, C, rpb, want, scratch);            \
+        else                                                                                                \
+            ln_bwd_ring_kernel<T, N, 2><<<nblk, 32 * LNB_WARPS, ring_smem, ctx.stream>>>(                   \
+                dy, x, mean, rstd, w, dres_in, dres_out, dres_act, rows, C, rpb, want, scratch);            \
         break;                                                                                              \
     }
         switch (nv) {
