@@ -805,7 +805,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     return true;
                 };
                 // The first pair of an item overwrites dV / dK, so it waits for the last item's
-                // to be copied out; its dQ, which needs neither, goes first.
+                // to be copied out; its dQ, which needs neither, goes first. Later pairs issue
+                // dQ right after dV, before dK, so the drain warps can start on it sooner.
                 if (it == 0) {
                     if (!issue_dq()) break;
                     if (!tc::mbar_wait(&ctl->dkv_free, (ictr & 1) ^ 1, abort, status)) break;
@@ -817,12 +818,12 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                     tc::mma_bf16_ts(tmem + BW_DV, tmem + BW_PT + kk * 8, dmn + TILE16 + 128 * kk, idesc_acc,
                                     (it > 0 || kk > 0) ? 1u : 0u);
                 tc::mma_commit(&ctl->pt_free);
+                if (it > 0 && !issue_dq()) break;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_bf16(tmem + BW_DK, d_ds_k + (kk >> 2) * TILE16 + 2 * (kk & 3), dmn + 128 * kk, idesc_acc,
                                  (it > 0 || kk > 0) ? 1u : 0u);
                 tc::mma_commit(&ctl->q_empty[st]);
-                if (it > 0 && !issue_dq()) break;
                 tc::mma_commit(&ctl->ds_free);
                 if (it + 1 == cur.n_it) {
                     tc::mma_commit(&ctl->kv_empty[slot]);
