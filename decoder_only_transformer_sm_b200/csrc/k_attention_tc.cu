@@ -15,13 +15,15 @@
 // walks the items, longest causal prefixes first, dealt to the CTAs round by
 // round in alternating direction. Warp 0 loads an item's two Q tiles
 // (double-buffered over items) and its K/V tiles through a 3-stage TMA ring.
-// Warp 1 issues, from one thread, for group g and key tile j: S_g = Q_g K_j^T
-// (M=128, N=128, K=64) into the group's TMEM S columns; once the group's softmax
-// has written P_g, O_g += P_g V_j (M=128, N=64, K=128; P_g read from TMEM as
-// packed bf16, V an N-major shared-memory operand, O_g accumulated in TMEM), and
-// right after it the S of the group's next tile. While one group's softmax runs,
-// the other group's MMAs run.
-// Warps 2..5 (group 0) and 6..9 (group 1) are the softmax warps: thread = query
+// Warp 1 + g issues group g's MMAs from one thread: for key tile j, S_g = Q_g
+// K_j^T (M=128, N=128, K=64) into the group's TMEM S columns, once the group's
+// softmax has written P_g of tile j - 1; then O_g += P_g V_{j-1} (M=128, N=64,
+// K=128; P_g read from TMEM as packed bf16, V an N-major shared-memory operand,
+// O_g accumulated in TMEM). The tensor pipe runs the two threads' instructions
+// concurrently (one thread's instructions run one after another, about 120
+// cycles each at N <= 128), so each group's S and PV do not queue behind the
+// other group's.
+// Warps 3..6 (group 0) and 7..10 (group 1) are the softmax warps: thread = query
 // row (TMEM lane) with all 128 keys of S_g in registers. The running row max m
 // is raised only when a tile's max exceeds it by more than FW_RESCALE (log2
 // units); then O (in TMEM) and l are rescaled by 2^(m_old - m_new). Otherwise P
@@ -43,7 +45,7 @@ namespace {
 constexpr int HD = 64;
 constexpr int BQ = 128, BKV = 128;
 constexpr int KV_STAGES = 3;
-constexpr int FW_THREADS = 64 + 32 * 8;           // TMA warp, MMA warp, two softmax warpgroups
+constexpr int FW_THREADS = 96 + 32 * 8;           // TMA warp, two MMA warps, two softmax warpgroups
 constexpr int TILE_BYTES = 128 * HD * 2;          // 16 KB: 128 rows x 128 bytes
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float FW_RESCALE = 8.f;                 // growth of the row max (log2 units) that triggers a rescale
@@ -52,12 +54,12 @@ constexpr float FW_RESCALE = 8.f;                 // growth of the row max (log2
 constexpr uint32_t FT_S = 0, FT_P = 128, FT_O = 192, FT_GROUP = 256;
 
 struct FwCtl {
-    uint64_t q_full[2], q_empty[2];               // Q sets (both groups' tiles of one item)
-    uint64_t kv_full[KV_STAGES], kv_empty[KV_STAGES];
+    uint64_t q_full[2], q_empty[2];               // Q sets (both groups' tiles of one item); empty: count 2
+    uint64_t kv_full[KV_STAGES], kv_empty[KV_STAGES];   // empty: one release per MMA thread
     uint64_t s_full[2];                           // per group: S of its current tile is in TMEM
     uint64_t p_full[2];                           // per group: P written to TMEM (its 4 warps arrive)
     uint64_t pv_done[2];                          // per group: O += P V of its latest tile is done
-    uint64_t drain;
+    uint64_t drain[2];
     uint32_t tmem_base;
     uint32_t abort;
 };
@@ -168,16 +170,16 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&ctl->q_full[i], 1);
-            tc::mbar_init(&ctl->q_empty[i], 1);
+            tc::mbar_init(&ctl->q_empty[i], 2);
             tc::mbar_init(&ctl->s_full[i], 1);
             tc::mbar_init(&ctl->p_full[i], 4);
             tc::mbar_init(&ctl->pv_done[i], 1);
+            tc::mbar_init(&ctl->drain[i], 1);
         }
         for (int s = 0; s < KV_STAGES; ++s) {
             tc::mbar_init(&ctl->kv_full[s], 1);
-            tc::mbar_init(&ctl->kv_empty[s], 1);
+            tc::mbar_init(&ctl->kv_empty[s], 2);
         }
-        tc::mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
         tc::fence_barrier_init();
     }
@@ -222,103 +224,87 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
                 ++ord;
             }
         }
-    } else if (warp == 1) {
+    } else if (warp <= 2) {
         if (lane == 0) {
-            // --------------------------------------------------------------- MMA
+            // ------------------------------------------------ MMA, one thread per group
+            // Thread g walks every K/V step of the CTA's items in the producer's order.
+            // A K/V stage and a Q set are free once both threads have released them, so
+            // each thread releases every step and every item, also those its group does
+            // not use, and in step order: it waits for a step's fill before releasing it
+            // and releases its pending tile (S issued, PV not yet) before any later step.
+            const int g = warp - 1;
             constexpr uint32_t idesc_s = tc::idesc_bf16_f32(BQ, BKV, 0, 0);
             constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(BQ, HD, 0, 1);
-            // an item in the CTA's order: round k, item ordinal, global index of its first key step
-            struct Cur {
-                int k, i, ord, gs0;
-                FwItem it;
-            };
-            auto settle = [&](Cur c) {   // from round c.k on, the first round that has an item
-                while (c.k < n_rounds && fw_round_item(c.k, n_items) < 0) ++c.k;
-                c.i = c.k < n_rounds ? fw_round_item(c.k, n_items) : -1;
-                if (c.i >= 0) c.it = fw_item(c.i, BH, n_pairs, Tn);
-                return c;
-            };
-            auto next_item = [&](Cur c) {
-                Cur n = c;
-                n.ord = c.ord + 1;
-                n.gs0 = c.gs0 + c.it.n_kv;
-                n.k = c.k + 1;
-                return settle(n);
-            };
-            // next S tile to issue for a group: (item cursor, key tile j)
-            struct Tile {
-                Cur c;
-                int j;
-            };
-            auto group_first = [&](Cur c, int g) {   // group g's first tile at or after item c
-                while (c.i >= 0 && c.it.n[g] == 0) c = next_item(c);
-                return Tile{c, 0};
-            };
-            auto group_next = [&](Tile t, int g) {
-                if (t.j + 1 < t.c.it.n[g]) return Tile{t.c, t.j + 1};
-                return group_first(next_item(t.c), g);
-            };
-            // S_g = Q_g K^T for tile t of group g
-            auto issue_s = [&](const Tile& t, int g) -> bool {
-                const int gs = t.c.gs0 + t.j, s = gs % KV_STAGES, qs = t.c.ord & 1;
-                if (t.j == 0 && !tc::mbar_wait(&ctl->q_full[qs], (t.c.ord >> 1) & 1, abort, status)) return false;
-                if (!tc::mbar_wait(&ctl->kv_full[s], (gs / KV_STAGES) & 1, abort, status)) return false;
-                tc::fence_after_sync();
-                const uint32_t q_addr = tc::smem_u32(smem + FW_OFF_Q + (2 * qs + g) * TILE_BYTES);
-                const uint32_t k_addr = tc::smem_u32(smem + FW_OFF_K + s * TILE_BYTES);
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
-                    tc::mma_bf16(tmem + g * FT_GROUP + FT_S, tc::smem_desc_sw128(q_addr + kk * 32, 16, 1024),
-                                 tc::smem_desc_sw128(k_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-                tc::mma_commit(&ctl->s_full[g]);
-                return true;
-            };
-            Cur c = settle(Cur{0, -1, 0, 0, FwItem{}});
-            Tile nt[2] = {group_first(c, 0), group_first(c, 1)};   // each group's next S to issue
-            uint32_t tp[2] = {0, 0};                                // PV MMAs issued per group
+            const uint32_t tSg = tmem + g * FT_GROUP + FT_S;
+            const uint32_t tPg = tmem + g * FT_GROUP + FT_P;
+            const uint32_t tOg = tmem + g * FT_GROUP + FT_O;
+            uint32_t gs = 0, ord = 0, tp = 0;    // K/V steps, items, PV MMAs issued
+            int pend = -1;                       // stage of the pending tile (-1: none)
+            bool pend_first = false;             // the pending tile is its item's first: PV overwrites O
             bool ok = true;
-            while (ok && c.i >= 0) {
-                for (int j = 0; j < c.it.n_kv && ok; ++j) {
-                    const int gs = c.gs0 + j, s = gs % KV_STAGES;
-                    // S of this step for a group whose S was not issued ahead
-                    for (int g = 0; g < 2 && ok; ++g)
-                        if (j < c.it.n[g] && nt[g].c.i >= 0 && nt[g].c.ord == c.ord && nt[g].j == j) {
-                            ok = issue_s(nt[g], g);
-                            nt[g] = group_next(nt[g], g);
-                        }
-                    for (int g = 0; g < 2 && ok; ++g) {
-                        if (j >= c.it.n[g]) continue;
-                        if (!tc::mbar_wait(&ctl->p_full[g], tp[g] & 1, abort, status)) { ok = false; break; }
-                        tc::fence_after_sync();
-                        const uint32_t v_addr = tc::smem_u32(smem + FW_OFF_V + s * TILE_BYTES);
+            for (int k = 0; k < n_rounds && ok; ++k) {
+                const int i = fw_round_item(k, n_items);
+                if (i < 0) continue;
+                const FwItem it = fw_item(i, BH, n_pairs, Tn);
+                const int ng = g == 0 ? it.n[0] : it.n[1];   // this group's key tiles
+                const int qs = ord & 1;
+                if (!tc::mbar_wait(&ctl->q_full[qs], (ord >> 1) & 1, abort, status)) { ok = false; break; }
+                for (int j = 0; j < it.n_kv; ++j, ++gs) {
+                    const int s = gs % KV_STAGES;
+                    const bool mine = j < ng;
+                    if (!tc::mbar_wait(&ctl->kv_full[s], (gs / KV_STAGES) & 1, abort, status)) { ok = false; break; }
+                    // the pending tile's P is written (and its S read) before S is overwritten
+                    if (pend >= 0 && !tc::mbar_wait(&ctl->p_full[g], tp & 1, abort, status)) { ok = false; break; }
+                    tc::fence_after_sync();
+                    if (mine) {
+                        const uint32_t q_addr = tc::smem_u32(smem + FW_OFF_Q + (2 * qs + g) * TILE_BYTES);
+                        const uint32_t k_addr = tc::smem_u32(smem + FW_OFF_K + s * TILE_BYTES);
+#pragma unroll
+                        for (int kk = 0; kk < HD / 16; ++kk)
+                            tc::mma_bf16(tSg, tc::smem_desc_sw128(q_addr + kk * 32, 16, 1024),
+                                         tc::smem_desc_sw128(k_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                        tc::mma_commit(&ctl->s_full[g]);
+                        if (j == ng - 1) tc::mma_commit(&ctl->q_empty[qs]);   // the group's last S of the item
+                    }
+                    if (pend >= 0) {
+                        const uint32_t v_addr = tc::smem_u32(smem + FW_OFF_V + pend * TILE_BYTES);
 #pragma unroll
                         for (int kk = 0; kk < BKV / 16; ++kk)
-                            tc::mma_bf16_ts(tmem + g * FT_GROUP + FT_O, tmem + g * FT_GROUP + FT_P + kk * 8,
-                                            tc::smem_desc_sw128(v_addr + kk * 2048, TILE_BYTES, 1024), idesc_pv,
-                                            (j > 0 || kk > 0) ? 1u : 0u);
+                            tc::mma_bf16_ts(tOg, tPg + kk * 8, tc::smem_desc_sw128(v_addr + kk * 2048, TILE_BYTES, 1024),
+                                            idesc_pv, (!pend_first || kk > 0) ? 1u : 0u);
                         tc::mma_commit(&ctl->pv_done[g]);
-                        ++tp[g];
-                        // the group's next S right away, when its K/V and Q are at most two steps
-                        // and one item ahead (so the producer can have them without further frees)
-                        const Tile& t = nt[g];
-                        if (t.c.i >= 0 && t.c.ord <= c.ord + 1 && t.c.gs0 + t.j <= gs + 2) {
-                            ok = issue_s(t, g);
-                            nt[g] = group_next(t, g);
-                        }
+                        tc::mma_commit(&ctl->kv_empty[pend]);
+                        ++tp;
+                        pend = -1;
                     }
-                    if (ok) tc::mma_commit(&ctl->kv_empty[s]);   // K and V of this step read by all its MMAs
+                    if (mine) {
+                        pend = s;
+                        pend_first = j == 0;
+                    } else {
+                        tc::mma_commit(&ctl->kv_empty[s]);   // a step this group does not use
+                    }
                 }
                 if (!ok) break;
-                tc::mma_commit(&ctl->q_empty[c.ord & 1]);   // every S of the item issued
-                c = next_item(c);
+                if (ng == 0) tc::mma_commit(&ctl->q_empty[qs]);
+                ++ord;
+            }
+            if (ok && pend >= 0 && tc::mbar_wait(&ctl->p_full[g], tp & 1, abort, status)) {
+                tc::fence_after_sync();
+                const uint32_t v_addr = tc::smem_u32(smem + FW_OFF_V + pend * TILE_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < BKV / 16; ++kk)
+                    tc::mma_bf16_ts(tOg, tPg + kk * 8, tc::smem_desc_sw128(v_addr + kk * 2048, TILE_BYTES, 1024),
+                                    idesc_pv, (!pend_first || kk > 0) ? 1u : 0u);
+                tc::mma_commit(&ctl->pv_done[g]);
+                tc::mma_commit(&ctl->kv_empty[pend]);
             }
             volatile uint32_t no_abort = 0;
-            tc::mma_commit(&ctl->drain);
-            tc::mbar_wait(&ctl->drain, 0, &no_abort, status);
+            tc::mma_commit(&ctl->drain[g]);
+            tc::mbar_wait(&ctl->drain[g], 0, &no_abort, status);
         }
     } else {
         // ---------------------------------------------------- softmax / output
-        const int g = (warp - 2) >> 2;
+        const int g = (warp - 3) >> 2;
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;            // query row within the tile = TMEM lane
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
