@@ -466,6 +466,9 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
 //     shared memory and add it into an fp32 (B T, C) accumulator with the TMA
 //     bulk reduce-add (zeroed by the pre-pass; the post-pass rounds it to
 //     bf16 into dqkv).
+// Two threads issue the MMAs: warp 1 dV, dQ and dK of each pair, warp 14 the
+// S^T and dP^T of the next, so the tensor pipe runs the two streams side by
+// side instead of one after the other.
 // The 5 matrix products of the algorithm are each computed once; no T x T
 // matrix goes to HBM.
 // ============================================================================
@@ -518,9 +521,10 @@ __device__ __forceinline__ void flush_rows_64(const uint8_t* stage, bf16* base, 
 
 constexpr int BW_EW_WARPS = 8;         // 2 per TMEM lane quarter, 64 query columns each (two chunks of 32)
 constexpr int BW_DR_WARPS = 4;         // dQ drain and dK/dV write-out: one per TMEM lane quarter
-constexpr int BW_THREADS = 64 + 32 * (BW_EW_WARPS + BW_DR_WARPS);
+constexpr int BW_THREADS = 64 + 32 * (BW_EW_WARPS + BW_DR_WARPS) + 32;
+constexpr int BW_SDP_WARP = 2 + BW_EW_WARPS + BW_DR_WARPS;   // the thread that issues S^T and dP^T
 constexpr int BW_STAGES = 3;           // Q/dO ring
-constexpr int BW_ITEM_READERS = 1 + BW_EW_WARPS + BW_DR_WARPS;   // MMA thread, element-wise and drain warps
+constexpr int BW_ITEM_READERS = 2 + BW_EW_WARPS + BW_DR_WARPS;   // two MMA threads, element-wise and drain warps
 struct CtlBwd {
     uint64_t item_full[2], item_empty[2];            // work-item ring, filled by the producer warp
     uint64_t kv_full[2], kv_empty[2];                // K and V of the item in ring slot s
@@ -531,7 +535,7 @@ struct CtlBwd {
     uint64_t ds_free;                                // a pair's dK, dQ MMAs done: dS^T reusable
     uint64_t dq_full, dq_empty;                      // a pair's dQ in TMEM: computed / copied to registers
     uint64_t acc_done, dkv_free;                     // an item's dK, dV complete in TMEM / copied out
-    uint64_t drain;
+    uint64_t drain[2];                               // per MMA thread
     uint32_t tmem_base;
     uint32_t abort;
     int item[2];
@@ -604,11 +608,11 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             tc::mbar_init(&ctl->item_full[i], 1);
             tc::mbar_init(&ctl->item_empty[i], BW_ITEM_READERS);
             tc::mbar_init(&ctl->kv_full[i], 1);
-            tc::mbar_init(&ctl->kv_empty[i], 1);
+            tc::mbar_init(&ctl->kv_empty[i], 2);   // released by both MMA threads
         }
         for (int s = 0; s < BW_STAGES; ++s) {
             tc::mbar_init(&ctl->q_full[s], 2);   // the TMA bytes, and the producer's lse / D stores
-            tc::mbar_init(&ctl->q_empty[s], 1);
+            tc::mbar_init(&ctl->q_empty[s], 2);
         }
         tc::mbar_init(&ctl->st_full, 1);
         tc::mbar_init(&ctl->st_empty, BW_EW_WARPS);
@@ -619,7 +623,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         tc::mbar_init(&ctl->dq_empty, BW_DR_WARPS);
         tc::mbar_init(&ctl->acc_done, 1);
         tc::mbar_init(&ctl->dkv_free, BW_DR_WARPS);
-        tc::mbar_init(&ctl->drain, 1);
+        tc::mbar_init(&ctl->drain[0], 1);
+        tc::mbar_init(&ctl->drain[1], 1);
         ctl->abort = 0;
         tc::fence_barrier_init();
     }
@@ -717,8 +722,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            // ------------------------------------------------------------------- MMA
-            constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128, 0, 0);   // K Q^T, V dO^T
+            // ------------------------------------------ MMA: dV, dQ, dK of each pair
             constexpr uint32_t idesc_acc = tc::idesc_bf16_f32(128, 64, 0, 1);  // P^T dO, dS^T Q
             constexpr uint32_t idesc_dq = tc::idesc_bf16_f32(128, 64, 1, 1);   // dS K (dS from the dS^T tile)
             // Shared-memory descriptors, built once: the start address sits in the low bits
@@ -726,108 +730,84 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             const uint32_t kv0 = tc::smem_u32(smem + BW_OFF_KV), q_base = tc::smem_u32(smem + BW_OFF_Q);
             const uint64_t d_ds_k = tc::smem_desc_sw128(tc::smem_u32(smem + BW_OFF_DS), 16, 1024);
             const uint64_t d_ds_mn = tc::smem_desc_sw128(tc::smem_u32(smem + BW_OFF_DS), T128_BYTES, 1024);
-            auto kdesc_k = [&](int slot) { return tc::smem_desc_sw128(kv0 + slot * BW_KV_BYTES, 16, 1024); };
             auto kdesc_mn = [&](int slot) {
                 return tc::smem_desc_sw128(kv0 + slot * BW_KV_BYTES, T128_BYTES, 1024);
             };
-            auto qdesc_k = [&](int st) { return tc::smem_desc_sw128(q_base + st * BW_STAGE_BYTES, 16, 1024); };
             auto qdesc_mn = [&](int st) {
                 return tc::smem_desc_sw128(q_base + st * BW_STAGE_BYTES, T128_BYTES, 1024);
             };
             constexpr uint64_t TILE16 = T128_BYTES >> 4;   // descriptor step of one 16 KB tile
-            // S^T and dP^T of pair g (query tile stage g % STAGES) against K/V slot `slot`
-            auto issue_sdp = [&](uint32_t g, int slot) -> bool {
-                const int st = g % BW_STAGES;
-                if (!tc::mbar_wait(&ctl->q_full[st], (g / BW_STAGES) & 1, abort, status)) return false;
-                tc::fence_after_sync();
-                const uint64_t dk = kdesc_k(slot), dq = qdesc_k(st);
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    tc::mma_bf16(tmem + BW_ST, dk + 2 * kk, dq + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
-                    tc::mma_bf16(tmem + BW_DPT, dk + TILE16 + 2 * kk, dq + TILE16 + 2 * kk, idesc_s,
-                                 kk > 0 ? 1u : 0u);
-                }
-                tc::mma_commit(&ctl->st_full);
-                return true;
-            };
             uint32_t ictr = 0, g = 0;
             int item = bw_read_item(ctl, ictr, abort, status);
             BwItem cur = bw_item(item < 0 ? 0 : item, BH, n_qt);
-            int it = 0;
-            bool ok = item >= 0 && tc::mbar_wait(&ctl->kv_full[0], 0, abort, status) && issue_sdp(0, 0);
+            bool ok = item >= 0;
             while (ok) {
-                const int st = g % BW_STAGES, slot = ictr & 1;
-                const uint32_t par = g & 1;
-                // the next pair: the next query tile, or the first of the next item
-                bool has_next = it + 1 < cur.n_it;
-                uint32_t nictr = ictr;
-                BwItem nxt = cur;
-                if (!has_next) {
-                    nictr = ictr + 1;
-                    const int ni = bw_read_item(ctl, nictr, abort, status);
-                    if (ni == -2) break;
-                    has_next = ni >= 0;
-                    if (has_next) nxt = bw_item(ni, BH, n_qt);
-                }
-                if (has_next) {   // its S^T / dP^T once this pair's are in registers
-                    if (!tc::mbar_wait(&ctl->st_empty, par, abort, status)) break;
-                    if (nictr != ictr && !tc::mbar_wait(&ctl->kv_full[nictr & 1], (nictr >> 1) & 1, abort, status))
-                        break;
-                    if (!issue_sdp(g + 1, nictr & 1)) break;
-                }
-                if (!tc::mbar_wait(&ctl->ew_done, par, abort, status)) break;
-                tc::fence_after_sync();
-                const uint64_t dmn = qdesc_mn(st);
+                const int slot = ictr & 1;
+                // K, V of the item (read by dQ), as filled for this thread's MMAs
+                if (!tc::mbar_wait(&ctl->kv_full[slot], (ictr >> 1) & 1, abort, status)) break;
                 const uint64_t kmn = kdesc_mn(slot);
-                // dQ = dS K: K = 128 keys in steps of 16; A is the dS^T tile read as an MN-major
-                // (query-contiguous) operand, the next 64 queries one atom (16 KB) further
-                auto issue_dq = [&]() -> bool {
-                    if (!tc::mbar_wait(&ctl->dq_empty, par ^ 1, abort, status)) return false;
+                for (int it = 0; it < cur.n_it && ok; ++it, ++g) {
+                    const int st = g % BW_STAGES;
+                    const uint32_t par = g & 1;
+                    // Q and dO of the pair (read by dK and dV), then its P^T and dS^T
+                    if (!tc::mbar_wait(&ctl->q_full[st], (g / BW_STAGES) & 1, abort, status) ||
+                        !tc::mbar_wait(&ctl->ew_done, par, abort, status)) {
+                        ok = false;
+                        break;
+                    }
                     tc::fence_after_sync();
+                    const uint64_t dmn = qdesc_mn(st);
+                    // dQ = dS K: K = 128 keys in steps of 16; A is the dS^T tile read as an MN-major
+                    // (query-contiguous) operand, the next 64 queries one atom (16 KB) further
+                    auto issue_dq = [&]() -> bool {
+                        if (!tc::mbar_wait(&ctl->dq_empty, par ^ 1, abort, status)) return false;
+                        tc::fence_after_sync();
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            tc::mma_bf16(tmem + BW_DQ, d_ds_mn + 128 * kk, kmn + 128 * kk, idesc_dq,
+                                         kk > 0 ? 1u : 0u);
+                        tc::mma_commit(&ctl->dq_full);
+                        return true;
+                    };
+                    // The first pair of an item overwrites dV / dK, so it waits for the last item's
+                    // to be copied out; its dQ, which needs neither, goes first. Later pairs issue
+                    // dQ right after dV, before dK, so the drain warps can start on it sooner.
+                    if (it == 0) {
+                        if (!issue_dq() || !tc::mbar_wait(&ctl->dkv_free, (ictr & 1) ^ 1, abort, status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after_sync();
+                    }
+                    // dV += P^T dO, then dK += dS^T Q: K = 128 queries in steps of 16
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_bf16(tmem + BW_DQ, d_ds_mn + 128 * kk, kmn + 128 * kk, idesc_dq, kk > 0 ? 1u : 0u);
-                    tc::mma_commit(&ctl->dq_full);
-                    return true;
-                };
-                // The first pair of an item overwrites dV / dK, so it waits for the last item's
-                // to be copied out; its dQ, which needs neither, goes first. Later pairs issue
-                // dQ right after dV, before dK, so the drain warps can start on it sooner.
-                if (it == 0) {
-                    if (!issue_dq()) break;
-                    if (!tc::mbar_wait(&ctl->dkv_free, (ictr & 1) ^ 1, abort, status)) break;
-                    tc::fence_after_sync();
-                }
-                // dV += P^T dO, then dK += dS^T Q: K = 128 queries in steps of 16
+                        tc::mma_bf16_ts(tmem + BW_DV, tmem + BW_PT + kk * 8, dmn + TILE16 + 128 * kk, idesc_acc,
+                                        (it > 0 || kk > 0) ? 1u : 0u);
+                    tc::mma_commit(&ctl->pt_free);
+                    if (it > 0 && !issue_dq()) {
+                        ok = false;
+                        break;
+                    }
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_bf16_ts(tmem + BW_DV, tmem + BW_PT + kk * 8, dmn + TILE16 + 128 * kk, idesc_acc,
-                                    (it > 0 || kk > 0) ? 1u : 0u);
-                tc::mma_commit(&ctl->pt_free);
-                if (it > 0 && !issue_dq()) break;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_bf16(tmem + BW_DK, d_ds_k + (kk >> 2) * TILE16 + 2 * (kk & 3), dmn + 128 * kk, idesc_acc,
-                                 (it > 0 || kk > 0) ? 1u : 0u);
-                tc::mma_commit(&ctl->q_empty[st]);
-                tc::mma_commit(&ctl->ds_free);
-                if (it + 1 == cur.n_it) {
-                    tc::mma_commit(&ctl->kv_empty[slot]);
-                    tc::mma_commit(&ctl->acc_done);
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_bf16(tmem + BW_DK, d_ds_k + (kk >> 2) * TILE16 + 2 * (kk & 3), dmn + 128 * kk,
+                                     idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
+                    tc::mma_commit(&ctl->q_empty[st]);
+                    tc::mma_commit(&ctl->ds_free);
+                    if (it + 1 == cur.n_it) {
+                        tc::mma_commit(&ctl->kv_empty[slot]);
+                        tc::mma_commit(&ctl->acc_done);
+                    }
                 }
-                if (!has_next) break;
-                if (nictr != ictr) {
-                    ictr = nictr;
-                    cur = nxt;
-                    it = 0;
-                } else {
-                    ++it;
-                }
-                ++g;
+                if (!ok) break;
+                item = bw_read_item(ctl, ++ictr, abort, status);
+                if (item < 0) break;
+                cur = bw_item(item, BH, n_qt);
             }
             volatile uint32_t no_abort = 0;
-            tc::mma_commit(&ctl->drain);
-            tc::mbar_wait(&ctl->drain, 0, &no_abort, status);
+            tc::mma_commit(&ctl->drain[0]);
+            tc::mbar_wait(&ctl->drain[0], 0, &no_abort, status);
         }
     } else if (warp < 2 + BW_EW_WARPS) {
         // --------------------------------------------- P^T, dS^T (thread = key row)
@@ -939,7 +919,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
                 it = 0;
             }
         }
-    } else {
+    } else if (warp < BW_SDP_WARP) {
         // ------------------------------- dQ drain, dK / dV write-out (thread = row)
         // Each warp moves its own 32 rows through its own 4 KB of staging: dQ as two
         // fp32 32 x 32 boxes added into the accumulator by this warp's TMA reduce,
@@ -1019,6 +999,50 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             }
         }
         if (lane == 0) tc::bulk_wait<0>();
+    } else if (lane == 0) {
+        // ----------------------------------------------- MMA: S^T and dP^T of each pair
+        // S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 128 queries, K = 64) of pair g,
+        // once the element-wise warps hold pair g - 1's in registers. This thread and the
+        // dV / dQ / dK thread each release the Q/dO stage and the K/V slot they read, and
+        // each waits for the fills itself, so every release lands in its own phase.
+        constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128, 0, 0);
+        constexpr uint64_t TILE16 = T128_BYTES >> 4;
+        const uint32_t kv0 = tc::smem_u32(smem + BW_OFF_KV), q_base = tc::smem_u32(smem + BW_OFF_Q);
+        uint32_t ictr = 0, g = 0;
+        int item = bw_read_item(ctl, ictr, abort, status);
+        BwItem cur = bw_item(item < 0 ? 0 : item, BH, n_qt);
+        bool ok = item >= 0;
+        while (ok) {
+            const int slot = ictr & 1;
+            if (!tc::mbar_wait(&ctl->kv_full[slot], (ictr >> 1) & 1, abort, status)) break;
+            const uint64_t dk = tc::smem_desc_sw128(kv0 + slot * BW_KV_BYTES, 16, 1024);
+            for (int it = 0; it < cur.n_it; ++it, ++g) {
+                const int st = g % BW_STAGES;
+                if ((g > 0 && !tc::mbar_wait(&ctl->st_empty, (g - 1) & 1, abort, status)) ||
+                    !tc::mbar_wait(&ctl->q_full[st], (g / BW_STAGES) & 1, abort, status)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                const uint64_t dq = tc::smem_desc_sw128(q_base + st * BW_STAGE_BYTES, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    tc::mma_bf16(tmem + BW_ST, dk + 2 * kk, dq + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
+                    tc::mma_bf16(tmem + BW_DPT, dk + TILE16 + 2 * kk, dq + TILE16 + 2 * kk, idesc_s,
+                                 kk > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(&ctl->st_full);
+                tc::mma_commit(&ctl->q_empty[st]);
+            }
+            if (!ok) break;
+            tc::mma_commit(&ctl->kv_empty[slot]);
+            item = bw_read_item(ctl, ++ictr, abort, status);
+            if (item < 0) break;
+            cur = bw_item(item, BH, n_qt);
+        }
+        volatile uint32_t no_abort = 0;
+        tc::mma_commit(&ctl->drain[1]);
+        tc::mbar_wait(&ctl->drain[1], 0, &no_abort, status);
     }
     tc::fence_before_sync();
     __syncthreads();
