@@ -61,3 +61,22 @@ def test_exact_causal_flop_count():
     assert bench.exact_step_flops(w, B, T) == pytest.approx(1.32e13, rel=5e-3)
     # the 6N + 12 L C T convention counts more: non-causal attention and the embeddings' 6N share
     assert bench.flops_per_token(w) * B * T > bench.exact_step_flops(w, B, T)
+
+
+def test_roofline_traffic_only_for_the_captured_source(tmp_path, monkeypatch):
+    """`traffic` comes from the committed ncu record only while the kernel source
+    it was captured from is unchanged; any edit of that file turns it into null."""
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    src = tmp_path / "decoder_only_transformer_sm_b200" / "csrc"
+    src.mkdir(parents=True)
+    (src / "k_attention_tc.cu").write_text("// kernel v1\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    sha = bench.kernel_source_sha("k_attention_tc.cu")
+    assert len(sha) == 16
+    (prof / "dram_traffic.json").write_text(
+        '{"attention bwd": {"kernel_source_sha": "%s", "bytes_per_launch": 123.0}}' % sha)
+    assert bench.traffic_for("attention bwd") == 123.0
+    assert bench.traffic_for("attention fwd") is None           # no record for that site
+    (src / "k_attention_tc.cu").write_text("// kernel v2\n")
+    assert bench.traffic_for("attention bwd") is None           # source changed since the capture
